@@ -1,0 +1,345 @@
+"""Throughput of the BPT layer forward (libbpt) on synthetic inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl bpt|reference] [--no-cpu-baseline]
+
+One step = one full layer forward (LN1, QKV projection, every wave of
+attention + W_O + LN2 + FFN) over one batch of the workload, through
+bpt_layer_forward with inputs resident in HBM.  The workload defaults to the
+long-context layer (B=1, N=65536, d=2048, h=16, d_ff=8192, causal, bf16).
+Its per-step traffic (x 256 MiB, QKV 768 MiB, out 512 MiB, scratch 768 MiB)
+is far above the 126 MB L2, so no flush is needed between steps.
+
+Multi-GPU (torchrun): each rank runs its own batch of the workload (the outer
+loop is data parallel across sequences), no collective on the data path;
+value = tokens of all ranks / max-over-ranks time (weak scaling).
+
+Prints one JSON line on rank 0.  `--impl reference` times the fp64 CPU oracle
+instead (a bounded row sample per step, on the host cores).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from blockwise_attn_ffn_b200 import accounting  # noqa: E402
+from blockwise_attn_ffn_b200.inputs import WORKLOADS, make_inputs, sample_rows  # noqa: E402
+
+METRIC = "BPT layer fwd tokens/s, TFLOP/s (% bf16 peak) at N=64K; peak live bytes"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(cfg, world, extra=None):
+    c = {"workload": cfg.name, "global_batch": cfg.B * world, "seq_len": cfg.N, "d": cfg.d,
+         "h": cfg.h, "d_ff": cfg.d_ff, "causal": cfg.causal, "block": cfg.block,
+         "parallelism": f"dp{world}" if world > 1 else "single",
+         "l2": "inputs larger than L2 (per-step traffic > 1.5 GiB), no flush"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+# ------------------------------------------------------------------ clocks --
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"bpt_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------- CPU baseline --
+def cpu_oracle_rate(cfg, n_rows: int):
+    """Times the fp64 oracle (as it stands) on a sample of rows; tokens/s."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        threads = None
+    inp = make_inputs(cfg, B=1)
+    rows = sample_rows(cfg, n_rows, B=1)
+    t0 = time.perf_counter()
+    oracle.layer_rows(inp, cfg.h, cfg.causal, rows)
+    dt = time.perf_counter() - t0
+    cores = len(os.sched_getaffinity(0))
+    return {"value": len(rows) / dt, "unit": UNIT, "cores": threads or cores,
+            "host_cores": cores, "kind": "oracle", "seconds": dt,
+            "sample": f"{len(rows)} seeded rows of {cfg.name} (incl. row N-1, so K/V for all "
+                      f"{cfg.N} keys) through oracle.layer_rows, fp64"}
+
+
+# ------------------------------------------------------------- reference --
+def run_reference(args, cfg, rank, world):
+    if rank != 0:
+        return 0
+    rows = args.ref_rows
+    per = []
+    for _ in range(args.warmup):
+        cpu_oracle_rate(cfg, rows)
+    for _ in range(args.steps):
+        per.append(cpu_oracle_rate(cfg, rows))
+    value = float(np.mean([p["value"] for p in per]))
+    cb = dict(per[-1])
+    cb["value"] = value
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": float(np.mean([p["seconds"] for p in per]) * 1e3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(cfg, 1),
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ main --
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="long_n64k", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="bpt", choices=["bpt", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=32)
+    ap.add_argument("--ref-rows", type=int, default=16)
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        return run_reference(args, cfg, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    import blockwise_attn_ffn_b200 as bpt
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    # Inputs: the workload's weights on every rank; rank r's x is the
+    # workload's draw for r = 0 and a rank-seeded draw otherwise.
+    inp = make_inputs(cfg)
+    if rank > 0:
+        rng = np.random.default_rng([cfg.seed, rank])
+        x32 = rng.standard_normal(size=inp["x"].shape, dtype=np.float32)
+        from blockwise_attn_ffn_b200.inputs import bf16_bits_to_f32, f32_to_bf16_bits
+        if cfg.dtype == "bf16":
+            inp["x_bits"] = f32_to_bf16_bits(x32)
+            inp["x"] = bf16_bits_to_f32(inp["x_bits"])
+        else:
+            inp["x"] = x32
+    torch.cuda.reset_peak_memory_stats(dev)
+    base_mem = torch.cuda.memory_allocated(dev)
+    p = bpt.to_device(inp, cfg.dtype, dev)
+    x_host = None
+    if not args.no_e2e:
+        x_host = bpt.to_device(inp, cfg.dtype, dev, pin_x=True)["x"]
+    del inp
+    x = p["x"]
+    out, ws = bpt.layer_forward(x, p, cfg.h, cfg.causal)
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    st, site = bpt.bpt_read_device_error(ws.data_ptr(), stream.cuda_stream)
+    if st != bpt.BPT_OK:
+        raise SystemExit(f"device error {bpt.status_string(st)} site {site}")
+    peak_fused = torch.cuda.max_memory_allocated(dev) - base_mem
+
+    for _ in range(args.warmup):
+        bpt.layer_forward(x, p, cfg.h, cfg.causal, out=out, workspace=ws)
+    torch.cuda.synchronize(dev)
+
+    flops = accounting.layer_flops(cfg.B, cfg.N, cfg.d, cfg.h, cfg.d_ff, cfg.causal)
+    _, launches_per_step = bpt.bpt_layer_launch_count(cfg.B, cfg.N, cfg.d, cfg.h, cfg.d_ff,
+                                                      cfg.causal, bpt.BPT_BF16 if cfg.dtype == "bf16" else bpt.BPT_F32)
+
+    # -------- timed region (device time, CUDA events on the launching stream)
+    bpt.bpt_profile_read()  # clear
+    bpt.bpt_profile_enable(True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            bpt.layer_forward(x, p, cfg.h, cfg.causal, out=out, workspace=ws)
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+    bpt.bpt_profile_enable(False)
+    ms_total = ev0.elapsed_time(ev1)
+    _, kind_ms, kind_n = bpt.bpt_profile_read()
+    st, site = bpt.bpt_read_device_error(ws.data_ptr(), stream.cuda_stream)
+    if st != bpt.BPT_OK:
+        raise SystemExit(f"device error {bpt.status_string(st)} site {site}")
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    tokens_step = cfg.B * cfg.N * world
+    value = tokens_step / (ms_step / 1e3)
+
+    # -------- end to end: pinned x -> device, forward, out -> pinned host
+    e2e = None
+    if not args.no_e2e:
+        out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        xd = torch.empty_like(x)
+        for _ in range(2):
+            xd.copy_(x_host, non_blocking=True)
+            bpt.layer_forward(xd, p, cfg.h, cfg.causal, out=out, workspace=ws)
+            out_host.copy_(out, non_blocking=True)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            xd.copy_(x_host, non_blocking=True)
+            bpt.layer_forward(xd, p, cfg.h, cfg.causal, out=out, workspace=ws)
+            out_host.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e2e = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        e2e = {"value": tokens_step / (ms_e2e / args.steps / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(x.numel() * x.element_size()),
+               "d2h_bytes_per_step": int(out.numel() * out.element_size()),
+               "ms_per_step": ms_e2e / args.steps}
+
+    peaks, peak_src = load_peaks()
+    n_attn = max(1, kind_n.get("attn", 0))
+    attn_ms_launch = kind_ms["attn"] / n_attn
+    attn_flops_launch = flops["attention"] * args.steps / n_attn
+    achieved = attn_flops_launch / (attn_ms_launch / 1e3) / 1e12
+    peak_sus = peaks["bf16_tflops_sustained"]
+    total_kernel_ms = sum(kind_ms.values())
+    kernels = {k: {"ms_per_step": kind_ms[k] / args.steps, "launches_per_step": kind_n[k] / args.steps,
+                   "share": kind_ms[k] / total_kernel_ms if total_kernel_ms else None}
+               for k in kind_ms}
+    flop_kind = {"qkv": flops["qkv"], "attn": flops["attention"], "wo": flops["wo"],
+                 "w1": flops["ffn"] / 2, "w2": flops["ffn"] / 2}
+    for k, f in flop_kind.items():
+        ms = kind_ms[k] / args.steps
+        kernels[k]["tflops"] = f / (ms / 1e3) / 1e12 if ms > 0 else None
+    tflops = flops["total"] * world / (ms_step / 1e3) / 1e12
+    unfused = accounting.unfused_activation_elems(cfg.N, cfg.d, cfg.h, cfg.d_ff,
+                                                  with_logits=False)
+    esz = 2 if cfg.dtype == "bf16" else 4
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+        "config": workload_config(cfg, world),
+        "tflops": tflops,
+        "pct_bf16_peak": tflops / world / peaks["bf16_tflops"],
+        "pct_bf16_peak_sustained": tflops / world / peak_sus,
+        "peak_src": peak_src,
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_tc_kernel", "achieved": achieved,
+                     "peak": peak_sus, "unit": "TFLOP/s", "frac": achieved / peak_sus,
+                     "peak_kind": f"bf16_tflops_sustained ({peak_src})",
+                     "frac_of_burst": achieved / peaks["bf16_tflops"], "traffic": None},
+        "kernels": kernels,
+        "peak_bytes": {"fused_device_total": int(peak_fused),
+                       "unfused_activations_analytic": int(cfg.B * unfused["total"] * esz),
+                       "unfused_ffn_hidden_analytic": int(cfg.B * unfused["ffn_hidden"] * esz)},
+        "gpu_launches": int(launches_per_step * args.steps),
+        "e2e": e2e,
+    }
+    with_clk = clk.summary()
+    line["clocks"] = with_clk
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_rate(cfg, args.cpu_rows)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,120 @@
+"""ctypes binding of libbpt (argument marshalling only).
+
+The functions named ``bpt_*`` mirror the C ABI of ``include/bpt.h`` one to
+one: pointers are passed as Python ints (device addresses), sizes as ints.
+Every step of the layer runs in the library's CUDA kernels; there is no other
+implementation behind this module, and loading fails loudly when the shared
+library is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libbpt.so")
+
+BPT_OK, BPT_ERR_INVALID_ARG, BPT_ERR_UNSUPPORTED, BPT_ERR_WORKSPACE, BPT_ERR_CUDA, \
+    BPT_ERR_TIMEOUT = range(6)
+BPT_F32, BPT_BF16 = 0, 1
+KINDS = ["ln1", "qkv", "attn", "wo", "ln2", "w1", "w2"]
+BPT_WAVE_BLOCKS = 256
+
+EXPORTED = [
+    "bpt_layer_workspace_size", "bpt_layer_forward", "bpt_read_device_error",
+    "bpt_status_string", "bpt_profile_enable", "bpt_profile_read",
+    "bpt_layer_launch_count",
+]
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+class BptError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status_string(status)}")
+        self.status = status
+
+
+def load() -> ctypes.CDLL:
+    """Load libbpt.so (built in-tree); raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with `python -m blockwise_attn_ffn_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    i64, vp, i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
+    lib.bpt_layer_workspace_size.argtypes = [i64, i64, i64, i64, i64, i32, i32,
+                                             ctypes.POINTER(ctypes.c_size_t)]
+    lib.bpt_layer_workspace_size.restype = i32
+    lib.bpt_layer_forward.argtypes = [vp] * 11 + [i64] * 5 + [i32, i32, vp, vp, ctypes.c_size_t, vp]
+    lib.bpt_layer_forward.restype = i32
+    lib.bpt_read_device_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
+    lib.bpt_read_device_error.restype = i32
+    lib.bpt_status_string.argtypes = [i32]
+    lib.bpt_status_string.restype = ctypes.c_char_p
+    lib.bpt_profile_enable.argtypes = [i32]
+    lib.bpt_profile_enable.restype = i32
+    lib.bpt_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double),
+                                     ctypes.POINTER(ctypes.c_int64), i32]
+    lib.bpt_profile_read.restype = i32
+    lib.bpt_layer_launch_count.argtypes = [i64, i64, i64, i64, i64, i32, i32,
+                                           ctypes.POINTER(ctypes.c_int64)]
+    lib.bpt_layer_launch_count.restype = i32
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().bpt_status_string(int(status)).decode()
+
+
+# ------------------------------------------------------------ C ABI mirror --
+def bpt_layer_workspace_size(B, N, d, h, d_ff, causal, dtype) -> Tuple[int, int]:
+    """Returns (status, bytes)."""
+    out = ctypes.c_size_t(0)
+    st = load().bpt_layer_workspace_size(B, N, d, h, d_ff, int(bool(causal)), dtype,
+                                         ctypes.byref(out))
+    return st, out.value
+
+
+def bpt_layer_forward(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
+                      B, N, d, h, d_ff, causal, dtype, out, workspace, workspace_bytes,
+                      stream) -> int:
+    """Pointer-level call; returns the status code."""
+    return load().bpt_layer_forward(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
+                                    B, N, d, h, d_ff, int(bool(causal)), dtype, out,
+                                    workspace, workspace_bytes, stream)
+
+
+def bpt_read_device_error(workspace, stream) -> Tuple[int, int]:
+    """Returns (status, site)."""
+    site = ctypes.c_uint32(0)
+    st = load().bpt_read_device_error(workspace, stream, ctypes.byref(site))
+    return st, site.value
+
+
+def bpt_status_string(status: int) -> str:
+    return status_string(status)
+
+
+def bpt_profile_enable(enable: bool) -> int:
+    return load().bpt_profile_enable(int(bool(enable)))
+
+
+def bpt_profile_read() -> Tuple[int, dict, dict]:
+    """Returns (status, ms per kind, launches per kind)."""
+    n = len(KINDS)
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_int64 * n)()
+    st = load().bpt_profile_read(ms, cnt, n)
+    return st, {k: ms[i] for i, k in enumerate(KINDS)}, {k: cnt[i] for i, k in enumerate(KINDS)}
+
+
+def bpt_layer_launch_count(B, N, d, h, d_ff, causal, dtype) -> Tuple[int, int]:
+    out = ctypes.c_int64(0)
+    st = load().bpt_layer_launch_count(B, N, d, h, d_ff, int(bool(causal)), dtype,
+                                       ctypes.byref(out))
+    return st, out.value

@@ -1,0 +1,591 @@
+// libbpt host side: argument validation, workspace layout, TMA descriptors and
+// the launch sequence of one BPT layer forward.
+//
+// Schedule ("Blockwise Parallel Transformer — BPT", sections "The fused
+// blockwise algorithm" and "Why parallel is in the name"): the outer loop over
+// query blocks is embarrassingly parallel, and P concurrent blocks cost
+// P x O(b d) of transient memory.  On this GPU one wave holds up to
+// BPT_WAVE_BLOCKS query blocks; per wave the loop body runs as five
+// stream-ordered kernels whose intermediates are wave-shaped:
+//   attention (online softmax over K/V blocks)  -> o      [P b, d]
+//   W_O GEMM, epilogue + x                      -> y      (into out rows)
+//   LN2                                         -> v      [P b, d]
+//   W_1 GEMM, epilogue + b_1, GELU              -> H      [P b, d_ff]
+//   W_2 GEMM, epilogue + b_2 + y                -> Z      (into out rows)
+// Before the waves: LN1 (into out, reused as scratch) and the QKV GEMM.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "bpt.h"
+#include "attn_tc.cuh"
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "rows.cuh"
+#include "simt_f32.cuh"
+
+namespace {
+
+using bpt::RowMap;
+
+constexpr int64_t kMaxWave = BPT_WAVE_BLOCKS;
+constexpr size_t kHeaderBytes = 256;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Wave {
+  int64_t item0, count, seqs;
+};
+
+struct Plan {
+  int64_t B, N, d, h, d_ff, dk;
+  int causal;
+  bpt_dtype dtype;
+  int64_t blk, nb, items;
+  int64_t cps;   // >0: each sequence is split into cps waves
+  int64_t G;     // >0: each wave holds G whole sequences
+  int64_t n_waves, P;
+  size_t esize;
+  size_t off_qkv, off_o, off_v, off_h, total;
+
+  Wave wave(int64_t w) const {
+    Wave r;
+    if (cps > 0) {
+      const int64_t csize = (nb + cps - 1) / cps;
+      const int64_t b = w / cps, c = w % cps;
+      const int64_t i0 = c * csize, i1 = std::min(nb, i0 + csize);
+      r.item0 = b * nb + i0;
+      r.count = i1 - i0;
+      r.seqs = 0;
+    } else {
+      const int64_t b0 = w * G;
+      const int64_t g = std::min(G, B - b0);
+      r.item0 = b0 * nb;
+      r.count = g * nb;
+      r.seqs = g;
+    }
+    return r;
+  }
+};
+
+bpt_status check_shape(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff, int causal,
+                       bpt_dtype dtype) {
+  (void)causal;
+  if (B < 0 || N < 0 || d <= 0 || h <= 0 || d_ff <= 0) return BPT_ERR_INVALID_ARG;
+  if (dtype != BPT_F32 && dtype != BPT_BF16) return BPT_ERR_INVALID_ARG;
+  if (d % h != 0) return BPT_ERR_INVALID_ARG;
+  const int64_t dk = d / h;
+  if (d % 8 != 0) return BPT_ERR_UNSUPPORTED;
+  if (dtype == BPT_BF16) {
+    if (dk != 64 && dk != 128) return BPT_ERR_UNSUPPORTED;
+    if (d % 64 != 0 || d_ff % 64 != 0) return BPT_ERR_UNSUPPORTED;
+  } else {
+    if (dk > bpt::kF32AttnMaxDk || d_ff % 4 != 0) return BPT_ERR_UNSUPPORTED;
+  }
+  if (d > 8192 || d_ff > 65536) return BPT_ERR_UNSUPPORTED;
+  // Rows and TMA coordinates are 32-bit; element offsets are 64-bit.  The
+  // largest buffers are QKV [B*N, 3d] and the wave scratch (bounded by the
+  // wave size), so only B*N is limited.
+  if (B > 0 && N > 0 && B * N > (int64_t(1) << 30)) return BPT_ERR_UNSUPPORTED;
+  return BPT_OK;
+}
+
+Plan make_plan(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff, int causal,
+               bpt_dtype dtype) {
+  Plan p{};
+  p.B = B; p.N = N; p.d = d; p.h = h; p.d_ff = d_ff; p.dk = d / h;
+  p.causal = causal ? 1 : 0;
+  p.dtype = dtype;
+  p.blk = dtype == BPT_BF16 ? 128 : bpt::kF32AttnRows;
+  p.esize = dtype == BPT_BF16 ? 2 : 4;
+  p.nb = (N + p.blk - 1) / p.blk;
+  p.items = B * p.nb;
+  if (p.items == 0) {
+    p.n_waves = 0;
+    p.P = 0;
+  } else if (p.nb > kMaxWave) {
+    p.cps = (p.nb + kMaxWave - 1) / kMaxWave;
+    p.G = 0;
+    p.n_waves = B * p.cps;
+    p.P = (p.nb + p.cps - 1) / p.cps;
+  } else {
+    p.cps = 0;
+    p.G = std::min<int64_t>(B, kMaxWave / p.nb);
+    p.n_waves = (B + p.G - 1) / p.G;
+    p.P = p.G * p.nb;
+  }
+  size_t off = align_up(kHeaderBytes, 1024);
+  p.off_qkv = off;
+  off = align_up(off + size_t(B * N) * size_t(3 * d) * p.esize, 1024);
+  const size_t rows = size_t(p.P * p.blk);
+  p.off_o = off;
+  off = align_up(off + rows * size_t(d) * p.esize, 1024);
+  p.off_v = off;
+  off = align_up(off + rows * size_t(d) * p.esize, 1024);
+  p.off_h = off;
+  off = align_up(off + rows * size_t(d_ff) * p.esize, 1024);
+  p.total = off;
+  return p;
+}
+
+// ------------------------------------------------------------ device info --
+struct DeviceInfo {
+  bool init = false;
+  bool ok = false;
+  int sms = 0;
+};
+std::mutex g_mu;
+DeviceInfo g_dev[64];
+
+bpt_status device_info(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BPT_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.init) {
+    int major = 0, minor = 0, n = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return BPT_ERR_CUDA;
+    di.ok = (major == 10 && minor == 0);
+    di.sms = n;
+    if (di.ok) {
+      if (cudaFuncSetAttribute(bpt::gemm_bf16_tc_kernel,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               bpt::kGemmSmem) != cudaSuccess ||
+          cudaFuncSetAttribute(bpt::attn_fwd_tc_kernel<64>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               bpt::AttnTile<64>::SMEM) != cudaSuccess ||
+          cudaFuncSetAttribute(bpt::attn_fwd_tc_kernel<128>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               bpt::AttnTile<128>::SMEM) != cudaSuccess ||
+          cudaFuncSetAttribute(bpt::attn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (3 * 64 * 128 + 64 * 65) * 4) != cudaSuccess)
+        return BPT_ERR_CUDA;
+    }
+    di.init = true;
+  }
+  if (!di.ok) return BPT_ERR_UNSUPPORTED;
+  *sms = di.sms;
+  return BPT_OK;
+}
+
+// ------------------------------------------------------------ tensor maps --
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+bpt_status get_encoder() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_encode) return BPT_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+          cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fn == nullptr)
+    return BPT_ERR_CUDA;
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return BPT_OK;
+}
+
+// bf16 tiles with the 128-byte swizzle; dims/strides innermost first.
+bool encode_bf16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                 const uint64_t* strides_bytes, const uint32_t* box) {
+  cuuint64_t gd[3], gs[2];
+  cuuint32_t bx[3], es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) gs[i] = strides_bytes[i];
+  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base),
+                              gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// A operand: [rows, K] row-major, 128 x 64 boxes.
+bool map_a(CUtensorMap* m, const void* base, int64_t rows, int64_t K) {
+  const uint64_t dims[2] = {uint64_t(K), uint64_t(rows)};
+  const uint64_t st[1] = {uint64_t(K) * 2};
+  const uint32_t box[2] = {64, 128};
+  return encode_bf16(m, base, 2, dims, st, box);
+}
+// B operand: [K, cols] row-major, 64 x 64 boxes.
+bool map_b(CUtensorMap* m, const void* base, int64_t K, int64_t cols) {
+  const uint64_t dims[2] = {uint64_t(cols), uint64_t(K)};
+  const uint64_t st[1] = {uint64_t(cols) * 2};
+  const uint32_t box[2] = {64, 64};
+  return encode_bf16(m, base, 2, dims, st, box);
+}
+// QKV viewed as [B][N][3d]: boxes of 64 columns x 128 tokens x 1 sequence.
+bool map_qkv(CUtensorMap* m, const void* base, int64_t B, int64_t N, int64_t d) {
+  const uint64_t dims[3] = {uint64_t(3 * d), uint64_t(N), uint64_t(B)};
+  const uint64_t st[2] = {uint64_t(3 * d) * 2, uint64_t(N) * uint64_t(3 * d) * 2};
+  const uint32_t box[3] = {64, 128, 1};
+  return encode_bf16(m, base, 3, dims, st, box);
+}
+
+// -------------------------------------------------------------- profiling --
+struct ProfRec {
+  int kind;
+  cudaEvent_t a, b;
+};
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t pool_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+struct LaunchScope {
+  int kind;
+  cudaStream_t s;
+  cudaEvent_t a = nullptr;
+  LaunchScope(int k, cudaStream_t st) : kind(k), s(st) {
+    if (g_prof_on) {
+      a = pool_event();
+      cudaEventRecord(a, s);
+    }
+  }
+  ~LaunchScope() {
+    if (g_prof_on && a) {
+      cudaEvent_t b = pool_event();
+      cudaEventRecord(b, s);
+      g_prof.push_back({kind, a, b});
+    }
+  }
+};
+
+// ----------------------------------------------------------------- launches --
+template <typename TIn, typename TOut, typename TP>
+cudaError_t launch_ln(const TIn* in, const TP* ln, TOut* out, int64_t rows, int64_t d, RowMap map,
+                      cudaStream_t s) {
+  const int nv = int((d + 255) / 256);
+  const dim3 grid(unsigned((rows + bpt::kLnWarps - 1) / bpt::kLnWarps));
+  const dim3 block(bpt::kLnWarps * 32);
+#define BPT_LN_CASE(NV)                                                                    \
+  if (nv <= NV) {                                                                          \
+    bpt::ln_rows_kernel<NV, TIn, TOut, TP><<<grid, block, 0, s>>>(in, ln, out, rows, int(d), \
+                                                                  map);                    \
+    return cudaGetLastError();                                                             \
+  }
+  BPT_LN_CASE(1)
+  BPT_LN_CASE(2)
+  BPT_LN_CASE(3)
+  BPT_LN_CASE(4)
+  BPT_LN_CASE(6)
+  BPT_LN_CASE(8)
+  BPT_LN_CASE(12)
+  BPT_LN_CASE(16)
+  BPT_LN_CASE(32)
+#undef BPT_LN_CASE
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                        const CUtensorMap& b2, const bpt::GemmParams& gp, int sms,
+                        cudaStream_t s) {
+  const int64_t tiles = int64_t((gp.M + bpt::kGemmBM - 1) / bpt::kGemmBM) *
+                        int64_t((gp.N + bpt::kGemmBN - 1) / bpt::kGemmBN);
+  const unsigned grid = unsigned(std::min<int64_t>(tiles, sms));
+  bpt::gemm_bf16_tc_kernel<<<grid, bpt::kGemmThreads, bpt::kGemmSmem, s>>>(a, b0, b1, b2, gp);
+  return cudaGetLastError();
+}
+
+bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const void* W_Q,
+                        const void* W_K, const void* W_V, const void* W_O, const void* ln2,
+                        const void* W_1, const void* b_1, const void* W_2, const void* b_2,
+                        float* out, uint8_t* ws, cudaStream_t s, int sms) {
+  using bf = __nv_bfloat16;
+  const int64_t M = P.B * P.N, d = P.d, d_ff = P.d_ff;
+  uint32_t* err = reinterpret_cast<uint32_t*>(ws);
+  bf* xn = reinterpret_cast<bf*>(out);  // LN1(x) lives in `out` until the waves start
+  bf* qkv = reinterpret_cast<bf*>(ws + P.off_qkv);
+  bf* so = reinterpret_cast<bf*>(ws + P.off_o);
+  bf* sv = reinterpret_cast<bf*>(ws + P.off_v);
+  bf* sh = reinterpret_cast<bf*>(ws + P.off_h);
+  const int64_t R = P.P * P.blk;  // scratch rows
+
+  CUtensorMap mXn, mWq, mWk, mWv, mQKV, mO, mWo, mV, mW1, mH, mW2;
+  bool ok = map_a(&mXn, xn, M, d) && map_b(&mWq, W_Q, d, d) && map_b(&mWk, W_K, d, d) &&
+            map_b(&mWv, W_V, d, d) && map_qkv(&mQKV, qkv, P.B, P.N, d) && map_a(&mO, so, R, d) &&
+            map_b(&mWo, W_O, d, d) && map_a(&mV, sv, R, d) && map_b(&mW1, W_1, d, d_ff) &&
+            map_a(&mH, sh, R, d_ff) && map_b(&mW2, W_2, d_ff, d);
+  if (!ok) return BPT_ERR_CUDA;
+
+  RowMap ident{0, 1, 1, 1, 1};
+  {
+    LaunchScope ls(BPT_KIND_LN1, s);
+    if (launch_ln<bf, bf, bf>(static_cast<const bf*>(x), static_cast<const bf*>(ln1), xn, M, d,
+                              ident, s) != cudaSuccess)
+      return BPT_ERR_CUDA;
+  }
+  {
+    bpt::GemmParams g{};
+    g.M = int(M); g.N = int(3 * d); g.K = int(d);
+    g.n_sub = int(d); g.n_maps = 3;
+    g.epi = bpt::kEpiStoreBf16;
+    g.out_bf16 = qkv; g.ld_out = 3 * d;
+    g.map = ident;
+    g.err = err;
+    LaunchScope ls(BPT_KIND_QKV, s);
+    if (launch_gemm(mXn, mWq, mWk, mWv, g, sms, s) != cudaSuccess) return BPT_ERR_CUDA;
+  }
+  const float scale_log2 = float(1.4426950408889634 / std::sqrt(double(P.dk)));
+  for (int64_t w = 0; w < P.n_waves; ++w) {
+    const Wave wv = P.wave(w);
+    const int64_t rows = wv.count * P.blk;
+    RowMap map{int(wv.item0), int(P.nb), int(P.N), int(P.blk), 0};
+    {
+      bpt::AttnParams ap{};
+      ap.N = int(P.N); ap.nb = int(P.nb); ap.h = int(P.h); ap.d = int(d);
+      ap.causal = P.causal; ap.item0 = int(wv.item0); ap.count = int(wv.count);
+      ap.seqs = int(wv.seqs); ap.o = so; ap.scale_log2 = scale_log2; ap.err = err;
+      const unsigned grid = unsigned(wv.count * P.h);
+      LaunchScope ls(BPT_KIND_ATTN, s);
+      if (P.dk == 128)
+        bpt::attn_fwd_tc_kernel<128><<<grid, 256, bpt::AttnTile<128>::SMEM, s>>>(mQKV, ap);
+      else
+        bpt::attn_fwd_tc_kernel<64><<<grid, 256, bpt::AttnTile<64>::SMEM, s>>>(mQKV, ap);
+      if (cudaGetLastError() != cudaSuccess) return BPT_ERR_CUDA;
+    }
+    {
+      bpt::GemmParams g{};
+      g.M = int(rows); g.N = int(d); g.K = int(d);
+      g.n_sub = int(d); g.n_maps = 1;
+      g.epi = bpt::kEpiResidX;
+      g.out_f32 = out; g.ld_f32 = d;
+      g.resid = static_cast<const bf*>(x); g.ld_resid = d;
+      g.map = map; g.err = err;
+      LaunchScope ls(BPT_KIND_WO, s);
+      if (launch_gemm(mO, mWo, mWo, mWo, g, sms, s) != cudaSuccess) return BPT_ERR_CUDA;
+    }
+    {
+      LaunchScope ls(BPT_KIND_LN2, s);
+      if (launch_ln<float, bf, bf>(out, static_cast<const bf*>(ln2), sv, rows, d, map, s) !=
+          cudaSuccess)
+        return BPT_ERR_CUDA;
+    }
+    {
+      bpt::GemmParams g{};
+      g.M = int(rows); g.N = int(d_ff); g.K = int(d);
+      g.n_sub = int(d_ff); g.n_maps = 1;
+      g.epi = bpt::kEpiGeluBias;
+      g.out_bf16 = sh; g.ld_out = d_ff;
+      g.bias = static_cast<const bf*>(b_1);
+      g.map = ident; g.err = err;
+      LaunchScope ls(BPT_KIND_W1, s);
+      if (launch_gemm(mV, mW1, mW1, mW1, g, sms, s) != cudaSuccess) return BPT_ERR_CUDA;
+    }
+    {
+      bpt::GemmParams g{};
+      g.M = int(rows); g.N = int(d); g.K = int(d_ff);
+      g.n_sub = int(d); g.n_maps = 1;
+      g.epi = bpt::kEpiBiasAccum;
+      g.out_f32 = out; g.ld_f32 = d;
+      g.bias = static_cast<const bf*>(b_2);
+      g.map = map; g.err = err;
+      LaunchScope ls(BPT_KIND_W2, s);
+      if (launch_gemm(mH, mW2, mW2, mW2, g, sms, s) != cudaSuccess) return BPT_ERR_CUDA;
+    }
+  }
+  return BPT_OK;
+}
+
+bpt_status forward_f32(const Plan& P, const float* x, const float* ln1, const float* W_Q,
+                       const float* W_K, const float* W_V, const float* W_O, const float* ln2,
+                       const float* W_1, const float* b_1, const float* W_2, const float* b_2,
+                       float* out, uint8_t* ws, cudaStream_t s) {
+  const int64_t M = P.B * P.N, d = P.d, d_ff = P.d_ff;
+  float* qkv = reinterpret_cast<float*>(ws + P.off_qkv);
+  float* so = reinterpret_cast<float*>(ws + P.off_o);
+  float* sv = reinterpret_cast<float*>(ws + P.off_v);
+  float* sh = reinterpret_cast<float*>(ws + P.off_h);
+  float* xn = out;  // LN1(x) lives in `out` until the waves start
+  RowMap ident{0, 1, 1, 1, 1};
+  auto gemm = [&](int kind, const float* A, int64_t Mr, int64_t Nc, int64_t K, const float* B0,
+                  const float* B1, const float* B2, int64_t n_sub, int epi, float* o,
+                  int64_t ld_out, const float* resid, const float* bias, RowMap map) -> bool {
+    bpt::GemmF32Params g{};
+    g.M = int(Mr); g.N = int(Nc); g.K = int(K); g.n_sub = int(n_sub);
+    g.A = A; g.B[0] = B0; g.B[1] = B1; g.B[2] = B2;
+    g.epi = epi; g.out = o; g.ld_out = ld_out; g.resid = resid; g.ld_resid = d;
+    g.bias = bias; g.map = map;
+    const dim3 grid(unsigned((Nc + bpt::kF32Tile - 1) / bpt::kF32Tile),
+                    unsigned((Mr + bpt::kF32Tile - 1) / bpt::kF32Tile));
+    LaunchScope ls(kind, s);
+    bpt::gemm_f32_kernel<<<grid, 256, 0, s>>>(g);
+    return cudaGetLastError() == cudaSuccess;
+  };
+  {
+    LaunchScope ls(BPT_KIND_LN1, s);
+    if (launch_ln<float, float, float>(x, ln1, xn, M, d, ident, s) != cudaSuccess)
+      return BPT_ERR_CUDA;
+  }
+  if (!gemm(BPT_KIND_QKV, xn, M, 3 * d, d, W_Q, W_K, W_V, d, bpt::kEpiStoreBf16, qkv, 3 * d,
+            nullptr, nullptr, ident))
+    return BPT_ERR_CUDA;
+  for (int64_t w = 0; w < P.n_waves; ++w) {
+    const Wave wv = P.wave(w);
+    const int64_t rows = wv.count * P.blk;
+    RowMap map{int(wv.item0), int(P.nb), int(P.N), int(P.blk), 0};
+    {
+      bpt::AttnF32Params ap{};
+      ap.qkv = qkv; ap.o = so; ap.N = int(P.N); ap.nb = int(P.nb); ap.h = int(P.h);
+      ap.d = int(d); ap.causal = P.causal; ap.item0 = int(wv.item0); ap.blk = int(P.blk);
+      ap.scale = float(1.0 / std::sqrt(double(P.dk)));
+      const size_t smem = size_t(3 * 64 * P.dk + 64 * 65) * 4;
+      LaunchScope ls(BPT_KIND_ATTN, s);
+      bpt::attn_f32_kernel<<<unsigned(wv.count * P.h), 256, smem, s>>>(ap);
+      if (cudaGetLastError() != cudaSuccess) return BPT_ERR_CUDA;
+    }
+    if (!gemm(BPT_KIND_WO, so, rows, d, d, W_O, W_O, W_O, d, bpt::kEpiResidX, out, d, x, nullptr,
+              map))
+      return BPT_ERR_CUDA;
+    {
+      LaunchScope ls(BPT_KIND_LN2, s);
+      if (launch_ln<float, float, float>(out, ln2, sv, rows, d, map, s) != cudaSuccess)
+        return BPT_ERR_CUDA;
+    }
+    if (!gemm(BPT_KIND_W1, sv, rows, d_ff, d, W_1, W_1, W_1, d_ff, bpt::kEpiGeluBias, sh, d_ff,
+              nullptr, b_1, ident))
+      return BPT_ERR_CUDA;
+    if (!gemm(BPT_KIND_W2, sh, rows, d, d_ff, W_2, W_2, W_2, d, bpt::kEpiBiasAccum, out, d,
+              nullptr, b_2, map))
+      return BPT_ERR_CUDA;
+  }
+  return BPT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+bpt_status bpt_layer_workspace_size(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff,
+                                    int causal, bpt_dtype dtype, size_t* bytes) {
+  if (!bytes) return BPT_ERR_INVALID_ARG;
+  const bpt_status st = check_shape(B, N, d, h, d_ff, causal, dtype);
+  if (st != BPT_OK) return st;
+  *bytes = make_plan(B, N, d, h, d_ff, causal, dtype).total;
+  return BPT_OK;
+}
+
+bpt_status bpt_layer_launch_count(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff,
+                                  int causal, bpt_dtype dtype, int64_t* launches) {
+  if (!launches) return BPT_ERR_INVALID_ARG;
+  const bpt_status st = check_shape(B, N, d, h, d_ff, causal, dtype);
+  if (st != BPT_OK) return st;
+  const Plan P = make_plan(B, N, d, h, d_ff, causal, dtype);
+  *launches = P.items == 0 ? 0 : 2 + 5 * P.n_waves;
+  return BPT_OK;
+}
+
+bpt_status bpt_layer_forward(const void* x, const void* ln1, const void* W_Q, const void* W_K,
+                             const void* W_V, const void* W_O, const void* ln2, const void* W_1,
+                             const void* b_1, const void* W_2, const void* b_2, int64_t B,
+                             int64_t N, int64_t d, int64_t h, int64_t d_ff, int causal,
+                             bpt_dtype dtype, float* out, void* workspace, size_t workspace_bytes,
+                             bpt_stream_t stream) {
+  bpt_status st = check_shape(B, N, d, h, d_ff, causal, dtype);
+  if (st != BPT_OK) return st;
+  if (B == 0 || N == 0) return BPT_OK;
+  const void* ptrs[] = {x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, out, workspace};
+  for (const void* p : ptrs)
+    if (p == nullptr || misaligned(p)) return BPT_ERR_INVALID_ARG;
+  const Plan P = make_plan(B, N, d, h, d_ff, causal, dtype);
+  if (workspace_bytes < P.total) return BPT_ERR_WORKSPACE;
+  // out must not overlap x (it is written before x is last read)
+  const uintptr_t xo = reinterpret_cast<uintptr_t>(x), oo = reinterpret_cast<uintptr_t>(out);
+  const size_t xbytes = size_t(B * N * d) * P.esize, obytes = size_t(B * N * d) * 4;
+  if (xo < oo + obytes && oo < xo + xbytes) return BPT_ERR_INVALID_ARG;
+  const uintptr_t wo = reinterpret_cast<uintptr_t>(workspace);
+  if (wo < oo + obytes && oo < wo + P.total) return BPT_ERR_INVALID_ARG;
+
+  int sms = 0;
+  st = device_info(&sms);
+  if (st != BPT_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (cudaMemsetAsync(ws, 0, kHeaderBytes, s) != cudaSuccess) return BPT_ERR_CUDA;
+  if (dtype == BPT_BF16) {
+    st = get_encoder();
+    if (st != BPT_OK) return st;
+    return forward_bf16(P, x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, out, ws, s, sms);
+  }
+  return forward_f32(P, static_cast<const float*>(x), static_cast<const float*>(ln1),
+                     static_cast<const float*>(W_Q), static_cast<const float*>(W_K),
+                     static_cast<const float*>(W_V), static_cast<const float*>(W_O),
+                     static_cast<const float*>(ln2), static_cast<const float*>(W_1),
+                     static_cast<const float*>(b_1), static_cast<const float*>(W_2),
+                     static_cast<const float*>(b_2), out, ws, s);
+}
+
+bpt_status bpt_read_device_error(void* workspace, bpt_stream_t stream, uint32_t* site) {
+  if (!workspace) return BPT_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BPT_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, workspace, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return BPT_ERR_CUDA;
+  if (word == 0) {
+    if (site) *site = 0;
+    return BPT_OK;
+  }
+  if (cudaMemset(workspace, 0, 4) != cudaSuccess) return BPT_ERR_CUDA;
+  if (site) *site = word >> 8;
+  return static_cast<bpt_status>(word & 0xFFu);
+}
+
+const char* bpt_status_string(bpt_status status) {
+  switch (status) {
+    case BPT_OK: return "BPT_OK";
+    case BPT_ERR_INVALID_ARG: return "BPT_ERR_INVALID_ARG: null or misaligned pointer, or inconsistent sizes";
+    case BPT_ERR_UNSUPPORTED: return "BPT_ERR_UNSUPPORTED: shape or device not handled by the kernels";
+    case BPT_ERR_WORKSPACE: return "BPT_ERR_WORKSPACE: workspace smaller than bpt_layer_workspace_size";
+    case BPT_ERR_CUDA: return "BPT_ERR_CUDA: a CUDA call failed";
+    case BPT_ERR_TIMEOUT: return "BPT_ERR_TIMEOUT: a kernel gave up waiting on a barrier";
+  }
+  return "BPT_UNKNOWN_STATUS";
+}
+
+bpt_status bpt_profile_enable(int enable) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_prof_on = enable != 0;
+  return BPT_OK;
+}
+
+bpt_status bpt_profile_read(double* ms, int64_t* launches, int n) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  bpt_status st = BPT_OK;
+  for (const ProfRec& r : g_prof) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
+      st = BPT_ERR_CUDA;
+    if (r.kind < n) {
+      if (ms) ms[r.kind] += double(t);
+      if (launches) launches[r.kind] += 1;
+    }
+    g_event_pool.push_back(r.a);
+    g_event_pool.push_back(r.b);
+  }
+  g_prof.clear();
+  return st;
+}
+
+}  // extern "C"

@@ -1,0 +1,301 @@
+// Persistent tcgen05 GEMM with fused epilogues: C[M, N] = A[M, K] * B[K, N].
+//
+//   A: bf16 [M, K] row-major (K contiguous), loaded by TMA as 128 x 64 tiles
+//      with the 128-byte swizzle -> K-major UMMA operand.
+//   B: bf16 [K, N] row-major (N contiguous; weights are [d_in, d_out]) loaded
+//      as four 64(N) x 64(K) boxes -> MN-major UMMA operand, no transpose.
+//      B may be the column concatenation of up to three matrices with the
+//      same number of columns each (W_Q | W_K | W_V).
+//   Accumulator: fp32 128 x 256 tile in tensor memory, double buffered, so
+//      the epilogue of one tile overlaps the main loop of the next.
+//
+// Warp roles (256 threads): warp 0 issues TMA loads, warp 1 issues UMMA,
+// warp 2 owns the tensor-memory allocation, warps 4..7 run the epilogue (warp
+// 4+e reads TMEM lanes 32e..32e+31, i.e. accumulator rows 32e..32e+31).
+//
+// Epilogues (all in fp32 before the final rounding):
+//   kEpiStoreBf16   out_bf16[row, col] = acc                     (QKV)
+//   kEpiResidX      out_f32[g, col]    = x[g, col] + acc         (y = x + o W_O)
+//   kEpiGeluBias    out_bf16[row, col] = GELU(acc + bias[col])   (FFN hidden)
+//   kEpiBiasAccum   out_f32[g, col]   += acc + bias[col]         (Z = y + h W_2 + b_2)
+// where g = map(row) is the residual-stream row of a scratch row.
+#pragma once
+
+#include "common.cuh"
+
+namespace bpt {
+
+enum GemmEpi : int { kEpiStoreBf16 = 0, kEpiResidX = 1, kEpiGeluBias = 2, kEpiBiasAccum = 3 };
+
+struct GemmParams {
+  int M, N, K;     // problem size (N, K multiples of 64)
+  int n_sub;       // columns of each concatenated B matrix
+  int n_maps;      // B matrices in use (1..3)
+  int epi;
+  __nv_bfloat16* out_bf16;
+  long long ld_out;
+  float* out_f32;
+  long long ld_f32;
+  const __nv_bfloat16* resid;
+  long long ld_resid;
+  const __nv_bfloat16* bias;
+  RowMap map;
+  uint32_t* err;
+};
+
+constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 64, kGemmStages = 4;
+constexpr int kGemmABytes = kGemmBM * kGemmBK * 2;  // 16 KB
+constexpr int kGemmBBytes = kGemmBK * kGemmBN * 2;  // 32 KB
+constexpr int kGemmStageBytes = kGemmABytes + kGemmBBytes;
+constexpr int kGemmBarrierBytes = 256;
+constexpr int kGemmSmem = kGemmStages * kGemmStageBytes + kGemmBarrierBytes + 1024;
+constexpr int kGemmThreads = 256;
+constexpr int kGemmGroupM = 16;  // row blocks per rasterisation group (L2 reuse)
+constexpr uint32_t kGemmTmemCols = 512;
+
+__device__ __forceinline__ void gemm_tile_coords(int tile, int m_blocks, int n_blocks, int& mb,
+                                                 int& nb) {
+  const int per_group = kGemmGroupM * n_blocks;
+  const int group = tile / per_group;
+  const int first_m = group * kGemmGroupM;
+  const int gm = min(kGemmGroupM, m_blocks - first_m);
+  const int in = tile - group * per_group;
+  mb = first_m + in % gm;
+  nb = in / gm;
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap mapA,
+                        const __grid_constant__ CUtensorMap mapB0,
+                        const __grid_constant__ CUtensorMap mapB1,
+                        const __grid_constant__ CUtensorMap mapB2, const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kGemmStages * kGemmABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kGemmStages * kGemmStageBytes);
+  // barrier slots
+  const uint32_t full0 = smem_u32(bars + 0);
+  const uint32_t empty0 = smem_u32(bars + kGemmStages);
+  const uint32_t accf0 = smem_u32(bars + 2 * kGemmStages);
+  const uint32_t acce0 = smem_u32(bars + 2 * kGemmStages + 2);
+  const uint32_t drain = smem_u32(bars + 2 * kGemmStages + 4);
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m_blocks = (p.M + kGemmBM - 1) / kGemmBM;
+  const int n_blocks = (p.N + kGemmBN - 1) / kGemmBN;
+  const int k_blocks = p.K / kGemmBK;
+  const int tiles = m_blocks * n_blocks;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kGemmStages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accf0 + 8 * b, 1);
+      mbar_init(acce0 + 8 * b, 4);
+    }
+    mbar_init(drain, 1);
+    abort_sh = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(&tmem_base_sh), kGemmTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  volatile int* abort_flag = &abort_sh;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    tma_prefetch_desc(&mapA);
+    tma_prefetch_desc(&mapB0);
+    if (p.n_maps > 1) tma_prefetch_desc(&mapB1);
+    if (p.n_maps > 2) tma_prefetch_desc(&mapB2);
+    int armed[kGemmStages];
+    for (int s = 0; s < kGemmStages; ++s) armed[s] = -1;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+      int mb, nb;
+      gemm_tile_coords(tile, m_blocks, n_blocks, mb, nb);
+      for (int kb = 0; kb < k_blocks; ++kb) {
+        if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.err, kSiteGemmProducer)) {
+          ok = false;
+          break;
+        }
+        const uint32_t fb = full0 + 8 * stage;
+        mbar_arrive_expect_tx(fb, kGemmStageBytes);
+        armed[stage] = static_cast<int>(phase);
+        tma_load_2d(smem_u32(sA + stage * kGemmABytes), &mapA, fb, kb * kGemmBK, mb * kGemmBM);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int c = nb * kGemmBN + q * 64;
+          int which = c / p.n_sub;
+          if (which > p.n_maps - 1) which = p.n_maps - 1;  // past the end: TMA zero-fills
+          const CUtensorMap* mB = which == 0 ? &mapB0 : (which == 1 ? &mapB1 : &mapB2);
+          tma_load_2d(smem_u32(sB + stage * kGemmBBytes + q * 8192), mB, fb, c - which * p.n_sub,
+                      kb * kGemmBK);
+        }
+        if (++stage == kGemmStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    // Drain: every load this thread armed has landed before the CTA exits.
+    for (int s = 0; s < kGemmStages; ++s)
+      if (armed[s] >= 0) mbar_wait_drain(full0 + 8 * s, static_cast<uint32_t>(armed[s]), p.err);
+  } else if (warp == 1 && lane == 0) {
+    // ----------------------------------------------------------- UMMA issue
+    constexpr uint32_t idesc = idesc_bf16_f32(kGemmBM, kGemmBN, false, true);
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+      if (!mbar_wait(acce0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.err, kSiteGemmMma)) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * kGemmBN);
+      for (int kb = 0; kb < k_blocks; ++kb) {
+        if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, p.err, kSiteGemmMma)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(sA + stage * kGemmABytes);
+        const uint32_t b_base = smem_u32(sB + stage * kGemmBBytes);
+#pragma unroll
+        for (int k = 0; k < kGemmBK / 16; ++k) {
+          const uint64_t ad = sdesc_sw128(a_base + k * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(b_base + k * 2048, 8192, 1024);
+          umma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+        }
+        umma_commit(empty0 + 8 * stage);
+        if (++stage == kGemmStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      umma_commit(accf0 + 8 * acc);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+    // Drain: all issued UMMA complete before tensor memory is released.
+    umma_commit(drain);
+    mbar_wait_drain(drain, 0, p.err);
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------- epilogue
+    const int e = warp - 4;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+      int mb, nb;
+      gemm_tile_coords(tile, m_blocks, n_blocks, mb, nb);
+      if (!mbar_wait(accf0 + 8 * acc, acc_phase, abort_flag, p.err, kSiteGemmEpilogue)) break;
+      tc_fence_after();
+      const long long row = static_cast<long long>(mb) * kGemmBM + e * 32 + lane;
+      long long g = -1;
+      bool row_ok;
+      if (p.epi == kEpiStoreBf16 || p.epi == kEpiGeluBias) {
+        row_ok = row < p.M;
+      } else {
+        g = row < p.M ? p.map.map(row) : -1;
+        row_ok = g >= 0;
+      }
+      const uint32_t t_row = tmem + (static_cast<uint32_t>(e * 32) << 16) +
+                             static_cast<uint32_t>(acc * kGemmBN);
+#pragma unroll 1
+      for (int ch = 0; ch < kGemmBN / 32; ++ch) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(t_row + ch * 32, r);
+        tmem_ld_wait();
+        const int col0 = nb * kGemmBN + ch * 32;
+        if (!row_ok || col0 >= p.N) continue;
+        float v[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
+        if (p.epi == kEpiStoreBf16 || p.epi == kEpiGeluBias) {
+          if (p.epi == kEpiGeluBias) {
+            const uint4* bp = reinterpret_cast<const uint4*>(p.bias + col0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 bb = __ldg(bp + q);
+              const __nv_bfloat16* bh = reinterpret_cast<const __nv_bfloat16*>(&bb);
+#pragma unroll
+              for (int k = 0; k < 8; ++k) v[q * 8 + k] = gelu_erf(v[q * 8 + k] + __bfloat162float(bh[k]));
+            }
+          }
+          uint4* dst = reinterpret_cast<uint4*>(p.out_bf16 + row * p.ld_out + col0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 w;
+            w.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+            w.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+            w.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+            w.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+            dst[q] = w;
+          }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(p.out_f32 + g * p.ld_f32 + col0);
+          if (p.epi == kEpiResidX) {
+            const uint4* xp = reinterpret_cast<const uint4*>(p.resid + g * p.ld_resid + col0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 xx = __ldg(xp + q);
+              const __nv_bfloat16* xh = reinterpret_cast<const __nv_bfloat16*>(&xx);
+#pragma unroll
+              for (int k = 0; k < 8; ++k) v[q * 8 + k] += __bfloat162float(xh[k]);
+            }
+          } else {
+            const uint4* bp = reinterpret_cast<const uint4*>(p.bias + col0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 bb = __ldg(bp + q);
+              const __nv_bfloat16* bh = reinterpret_cast<const __nv_bfloat16*>(&bb);
+#pragma unroll
+              for (int k = 0; k < 8; ++k) v[q * 8 + k] += __bfloat162float(bh[k]);
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float4 y = dst[q];
+              v[q * 4 + 0] += y.x;
+              v[q * 4 + 1] += y.y;
+              v[q * 4 + 2] += y.z;
+              v[q * 4 + 3] += y.w;
+            }
+          }
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            dst[q] = make_float4(v[q * 4 + 0], v[q * 4 + 1], v[q * 4 + 2], v[q * 4 + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce0 + 8 * acc);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, kGemmTmemCols);
+}
+
+}  // namespace bpt

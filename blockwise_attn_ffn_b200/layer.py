@@ -1,0 +1,89 @@
+"""torch-tensor front end of ``bpt_layer_forward`` (marshalling only).
+
+PyTorch provides device memory and the stream; the layer itself runs in
+libbpt's kernels.
+"""
+from __future__ import annotations
+
+from typing import Dict, Optional
+
+import numpy as np
+import torch
+
+from . import _lib
+
+# Parameter tensors in C-ABI order, with their shapes in terms of (d, d_ff).
+PARAM_NAMES = ["ln1", "W_Q", "W_K", "W_V", "W_O", "ln2", "W_1", "b_1", "W_2", "b_2"]
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return _lib.BPT_BF16
+    if t.dtype == torch.float32:
+        return _lib.BPT_F32
+    raise TypeError(f"x must be bfloat16 or float32, got {t.dtype}")
+
+
+def to_device(inp: Dict[str, np.ndarray], dtype: str, device="cuda",
+              pin_x: bool = False) -> Dict[str, torch.Tensor]:
+    """Moves generator output (``inputs.make_inputs``) to device tensors.
+
+    bf16 tensors are rebuilt from their exact bit patterns.  LN parameters
+    are packed as [2, d] (gamma; beta).  With ``pin_x`` the input x stays in
+    pinned host memory (for end-to-end timing, which copies it each step).
+    """
+    def conv(name):
+        if dtype == "bf16":
+            a = torch.from_numpy(np.ascontiguousarray(inp[name + "_bits"]).view(np.int16))
+            return a.view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(inp[name], dtype=np.float32))
+
+    out = {}
+    x = conv("x")
+    out["x"] = x.pin_memory() if pin_x else x.to(device)
+    for k in ("W_Q", "W_K", "W_V", "W_O", "W_1", "b_1", "W_2", "b_2"):
+        out[k] = conv(k).to(device)
+    out["ln1"] = torch.stack([conv("gamma1"), conv("beta1")]).to(device)
+    out["ln2"] = torch.stack([conv("gamma2"), conv("beta2")]).to(device)
+    return out
+
+
+def workspace_for(B: int, N: int, d: int, h: int, d_ff: int, causal: bool,
+                  dtype: torch.dtype, device="cuda") -> torch.Tensor:
+    """Allocates (through torch) a workspace of the size the library asks for."""
+    code = _lib.BPT_BF16 if dtype == torch.bfloat16 else _lib.BPT_F32
+    st, nbytes = _lib.bpt_layer_workspace_size(B, N, d, h, d_ff, causal, code)
+    if st != _lib.BPT_OK:
+        raise _lib.BptError(st, "bpt_layer_workspace_size")
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def layer_forward(x: torch.Tensor, p: Dict[str, torch.Tensor], h: int, causal: bool,
+                  out: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None,
+                  stream: Optional[torch.cuda.Stream] = None):
+    """Z = BPT layer(x) via ``bpt_layer_forward``; returns (out, workspace).
+
+    x: [B, N, d] bf16 or fp32 on the GPU; p: ``PARAM_NAMES`` tensors of the
+    same dtype (ln1/ln2 as [2, d]); out: [B, N, d] fp32.
+    """
+    if x.dim() != 3:
+        raise ValueError("x must be [B, N, d]")
+    B, N, d = x.shape
+    d_ff = p["W_1"].shape[1]
+    code = _dtype_code(x)
+    tensors = [x] + [p[k] for k in PARAM_NAMES]
+    for t in tensors:
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != x.dtype:
+            raise ValueError("inputs must be contiguous CUDA tensors of one dtype")
+    if out is None:
+        out = torch.empty((B, N, d), dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = workspace_for(B, N, d, h, d_ff, causal, x.dtype, x.device)
+    s = stream if stream is not None else torch.cuda.current_stream(x.device)
+    st = _lib.bpt_layer_forward(*[t.data_ptr() for t in tensors], B, N, d, h, d_ff, causal,
+                                code, out.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                s.cuda_stream)
+    if st != _lib.BPT_OK:
+        raise _lib.BptError(st, "bpt_layer_forward")
+    return out, workspace

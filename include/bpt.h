@@ -1,0 +1,154 @@
+/*
+ * bpt.h -- C ABI of libbpt: the forward pass of one pre-LN Blockwise Parallel
+ * Transformer (BPT) layer on an NVIDIA B200 (sm_100a).
+ *
+ * What the layer computes ("Blockwise Parallel Transformer — BPT",
+ * aicassindra.com, sections "The bottleneck that survives FlashAttention" and
+ * "The fused blockwise algorithm"), per batch element and token row:
+ *
+ *   U = LN1(x);  Q = U W_Q;  K = U W_K;  V = U W_V
+ *   per head t (columns t*d_k .. (t+1)*d_k, d_k = d / h):
+ *       o_t = softmax(Q_t K_t^T / sqrt(d_k) [causal: keys j <= i]) V_t
+ *   y = x + o W_O
+ *   Z = y + GELU(LN2(y) W_1 + b_1) W_2 + b_2
+ *
+ * LN(v) = gamma * (v - mean) / sqrt(var + 1e-5) + beta over the d features of
+ * a token (biased variance); GELU(z) = z/2 (1 + erf(z / sqrt 2)).  Q, K, V and
+ * W_O carry no bias.
+ *
+ * How it is computed: blockwise, as the pages' two-level loop.  The outer loop
+ * over query blocks of b rows (b = 128 for bf16, 64 for fp32) runs in waves of
+ * at most BPT_WAVE_BLOCKS concurrent blocks; for each wave the kernels run
+ * exact blockwise attention with an online softmax (causal blocks j > i are
+ * skipped), then W_O + residual, LN2, W_1 + b_1 + GELU and W_2 + b_2 +
+ * residual for the wave's rows only.  Neither the [N, N] scores nor the
+ * [N, d_ff] FFN hidden state ever exists; the only sequence-shaped buffers are
+ * x, out and the Q/K/V projection in the workspace.
+ *
+ * Conventions shared by every entry point:
+ *   - All pointers except `bytes` and the profile arrays are DEVICE pointers
+ *     on the current CUDA device, 16-byte aligned.  The caller owns every
+ *     buffer; the library never allocates or frees device memory.
+ *   - Weights are row-major [d_in, d_out] (the layer computes x W).
+ *   - Work is enqueued on `stream` and the call returns before it finishes.
+ *   - Argument errors are reported by the return value BEFORE anything is
+ *     enqueued.  A wait inside a kernel that runs out of time (a lost
+ *     signal; never expected) makes the kernel exit early and sets an error
+ *     word in the workspace header, read by bpt_read_device_error.
+ */
+#ifndef BPT_H_
+#define BPT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BPT_OK = 0,
+  BPT_ERR_INVALID_ARG = 1, /* null or misaligned pointer, inconsistent sizes */
+  BPT_ERR_UNSUPPORTED = 2, /* valid layer the kernels do not handle (see below) */
+  BPT_ERR_WORKSPACE = 3,   /* workspace smaller than bpt_layer_workspace_size */
+  BPT_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed */
+  BPT_ERR_TIMEOUT = 5      /* a kernel gave up waiting (device error word) */
+} bpt_status;
+
+typedef enum {
+  BPT_F32 = 0,  /* x, weights, params fp32; fp32 arithmetic on CUDA cores */
+  BPT_BF16 = 1  /* x, weights, params bf16; tensor cores, fp32 accumulate */
+} bpt_dtype;
+
+/* Same object as cudaStream_t; 0 is the legacy default stream. */
+typedef struct CUstream_st* bpt_stream_t;
+
+/* Maximum query blocks processed concurrently (one wave of the outer loop). */
+#define BPT_WAVE_BLOCKS 256
+
+/*
+ * bpt_layer_workspace_size -- device workspace bytes bpt_layer_forward needs.
+ *
+ * Pure host arithmetic.  Layout (each region 1024-byte aligned):
+ *   [0, 256)       header; uint32 at offset 0 = device error word
+ *   QKV            [B*N, 3d] of dtype (Q | K | V per row)
+ *   block scratch  P*b rows of o [d], LN2(y) [d] and FFN hidden [d_ff], dtype,
+ *                  P = blocks in the largest wave (<= BPT_WAVE_BLOCKS)
+ * The scratch term does not grow with N once B*ceil(N/b) >= BPT_WAVE_BLOCKS.
+ * Returns BPT_ERR_INVALID_ARG for bytes == NULL or negative / inconsistent
+ * sizes, BPT_ERR_UNSUPPORTED for shapes bpt_layer_forward rejects.
+ */
+bpt_status bpt_layer_workspace_size(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff,
+                                    int causal, bpt_dtype dtype, size_t* bytes);
+
+/*
+ * bpt_layer_forward -- Z = layer(x), written to `out`.
+ *
+ *   x     [B, N, d]  dtype     layer input (residual stream)
+ *   ln1   [2, d]     dtype     LN1 gamma (row 0) and beta (row 1)
+ *   W_Q, W_K, W_V, W_O [d, d]  dtype
+ *   ln2   [2, d]     dtype     LN2 gamma, beta
+ *   W_1   [d, d_ff]  dtype;  b_1 [d_ff] dtype
+ *   W_2   [d_ff, d]  dtype;  b_2 [d]    dtype
+ *   causal  nonzero: token i attends to tokens j <= i; zero: to all tokens
+ *   out   [B, N, d]  fp32      layer output; also used as scratch for LN1(x)
+ *                              before it is written, so it must not alias any
+ *                              input
+ *   workspace / workspace_bytes   device buffer of >= the size above
+ *
+ * Supported shapes: d = h * d_k; d % 8 == 0.
+ *   BPT_BF16: d_k in {64, 128}; d % 64 == 0; d_ff % 64 == 0; any N >= 1
+ *             (a ragged last block is masked).
+ *   BPT_F32:  d_k <= 128; d_ff % 4 == 0; any N >= 1.
+ *   B * N <= 2^30 tokens.
+ * B == 0 or N == 0: nothing to do, returns BPT_OK without touching memory.
+ * Results are deterministic: the same inputs give bitwise the same `out`.
+ */
+bpt_status bpt_layer_forward(const void* x, const void* ln1, const void* W_Q, const void* W_K,
+                             const void* W_V, const void* W_O, const void* ln2, const void* W_1,
+                             const void* b_1, const void* W_2, const void* b_2, int64_t B,
+                             int64_t N, int64_t d, int64_t h, int64_t d_ff, int causal,
+                             bpt_dtype dtype, float* out, void* workspace, size_t workspace_bytes,
+                             bpt_stream_t stream);
+
+/*
+ * bpt_read_device_error -- synchronises `stream`, reads and clears the error
+ * word in the workspace header.  Returns BPT_OK if no kernel gave up,
+ * BPT_ERR_TIMEOUT if one did (*site, if non-NULL, receives the code of the
+ * wait that ran out), BPT_ERR_CUDA if synchronisation failed.
+ */
+bpt_status bpt_read_device_error(void* workspace, bpt_stream_t stream, uint32_t* site);
+
+/* Human-readable name of a status code (static string). */
+const char* bpt_status_string(bpt_status status);
+
+/*
+ * Optional per-kernel timing, for measurement only.  While enabled, every
+ * launch made by bpt_layer_forward is bracketed by CUDA events recorded on the
+ * launching stream (host-side event objects, no device memory).
+ * bpt_profile_read synchronises the recorded events, adds the elapsed time
+ * and launch count per kernel kind into ms[k] / launches[k] for
+ * k < min(n, BPT_KIND_COUNT), and clears the record.
+ */
+enum {
+  BPT_KIND_LN1 = 0,
+  BPT_KIND_QKV = 1,
+  BPT_KIND_ATTN = 2,
+  BPT_KIND_WO = 3,
+  BPT_KIND_LN2 = 4,
+  BPT_KIND_W1 = 5,
+  BPT_KIND_W2 = 6,
+  BPT_KIND_COUNT = 7
+};
+bpt_status bpt_profile_enable(int enable);
+bpt_status bpt_profile_read(double* ms, int64_t* launches, int n);
+
+/* Kernel launches one bpt_layer_forward call makes for these sizes. */
+bpt_status bpt_layer_launch_count(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff,
+                                  int causal, bpt_dtype dtype, int64_t* launches);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BPT_H_ */

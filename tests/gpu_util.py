@@ -1,0 +1,51 @@
+"""Helpers shared by the GPU parity tests: run the CUDA path through the C ABI
+and compare with the fp64 oracle."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import blockwise_attn_ffn_b200 as bpt
+from blockwise_attn_ffn_b200.inputs import LayerShape, make_inputs
+
+# Tolerances (max abs, mean abs) against the fp64 oracle.
+TOL_F32 = (1e-4, None)
+TOL_BF16 = (2e-2, 2e-3)
+
+
+def tol_for(cfg: LayerShape):
+    return TOL_F32 if cfg.dtype == "f32" else TOL_BF16
+
+
+def run_cuda(cfg: LayerShape, inp=None, B=None):
+    """One forward through bpt_layer_forward; returns (Z float32 numpy, dev, ws)."""
+    if inp is None:
+        inp = make_inputs(cfg, B=B)
+    dev = bpt.to_device(inp, cfg.dtype)
+    x = dev["x"]
+    out, ws = bpt.layer_forward(x, dev, cfg.h, cfg.causal)
+    st, site = bpt.bpt_read_device_error(ws.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    assert st == bpt.BPT_OK, f"device error {bpt.status_string(st)} at site {site}"
+    return out.float().cpu().numpy(), dev, ws
+
+
+def compare(got: np.ndarray, want: np.ndarray, tol):
+    err = np.abs(got.astype(np.float64) - want)
+    assert np.all(np.isfinite(got)), "non-finite values in the CUDA result"
+    mx, mean = float(err.max()), float(err.mean())
+    msg = f"max abs {mx:.3e} (tol {tol[0]}), mean abs {mean:.3e} (tol {tol[1]})"
+    assert mx <= tol[0], msg
+    if tol[1] is not None:
+        assert mean <= tol[1], msg
+    return mx, mean
+
+
+def workspace_qkv(ws: torch.Tensor, cfg: LayerShape, B: int) -> np.ndarray:
+    """The QKV projection the library leaves in its workspace ([B*N, 3d])."""
+    off = 1024
+    n = B * cfg.N * 3 * cfg.d
+    if cfg.dtype == "bf16":
+        t = ws[off:off + 2 * n].view(torch.bfloat16)
+    else:
+        t = ws[off:off + 4 * n].view(torch.float32)
+    return t.float().cpu().numpy().reshape(B, cfg.N, 3 * cfg.d)

@@ -1,0 +1,151 @@
+"""The C-ABI boundary on the host (no GPU needed).
+
+The library loads, exports every function include/bpt.h declares, and rejects
+bad arguments with the documented status before it touches the GPU.  The
+workspace query is pure arithmetic, so its block-shaped growth is checked
+here too.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import blockwise_attn_ffn_b200 as bpt
+from blockwise_attn_ffn_b200 import build as bbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib():
+    bbuild.build()
+    return bpt.load()
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "bpt.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(bpt_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_every_declared_function_is_exported(lib):
+    names = header_functions()
+    assert "bpt_layer_forward" in names and "bpt_layer_workspace_size" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(bpt.EXPORTED) == names
+
+
+def test_status_strings():
+    for s in range(6):
+        assert bpt.status_string(s).startswith("BPT_")
+    assert "UNKNOWN" in bpt.status_string(99)
+
+
+BF, F32 = bpt.BPT_BF16, bpt.BPT_F32
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((1, 256, 64, 1, 256, 0, F32), bpt.BPT_OK),
+    ((8, 2048, 768, 12, 3072, 1, BF), bpt.BPT_OK),
+    ((1, 300, 256, 4, 512, 1, BF), bpt.BPT_OK),            # ragged N
+    ((1, 256, 100, 3, 256, 1, BF), bpt.BPT_ERR_INVALID_ARG),  # d % h
+    ((1, 256, 96, 3, 256, 1, BF), bpt.BPT_ERR_UNSUPPORTED),   # d_k = 32
+    ((1, 256, 256, 1, 512, 1, BF), bpt.BPT_ERR_UNSUPPORTED),  # d_k = 256
+    ((1, 256, 256, 2, 500, 1, BF), bpt.BPT_ERR_UNSUPPORTED),  # d_ff % 64
+    ((1, 256, 64, 1, 256, 0, 7), bpt.BPT_ERR_INVALID_ARG),    # dtype
+    ((-1, 256, 64, 1, 256, 0, F32), bpt.BPT_ERR_INVALID_ARG),
+    ((1, 256, 0, 1, 256, 0, F32), bpt.BPT_ERR_INVALID_ARG),
+    ((1, 256, 1024, 4, 256, 0, F32), bpt.BPT_ERR_UNSUPPORTED),  # fp32 d_k = 256
+])
+def test_workspace_size_validation(args, expect):
+    st, nbytes = bpt.bpt_layer_workspace_size(*args)
+    assert st == expect
+    if st == bpt.BPT_OK:
+        assert nbytes > 0
+
+
+def test_workspace_null_out_pointer(lib):
+    assert lib.bpt_layer_workspace_size(1, 256, 64, 1, 256, 0, F32, None) == bpt.BPT_ERR_INVALID_ARG
+
+
+def test_workspace_is_block_shaped():
+    """Beyond the QKV projection (3 B N d elements) the workspace does not grow
+    with N once a wave is full, and never exceeds that bound."""
+    d, h, d_ff = 2048, 16, 8192
+    extra = []
+    for N in (8192, 16384, 32768, 65536, 131072):
+        st, nbytes = bpt.bpt_layer_workspace_size(1, N, d, h, d_ff, 1, BF)
+        assert st == bpt.BPT_OK
+        extra.append(nbytes - 3 * N * d * 2)
+    full = extra[2:]
+    assert max(full) - min(full) <= 2048           # alignment slack only
+    assert all(e <= max(full) for e in extra)
+    bound = bpt.BPT_WAVE_BLOCKS * 128 * (2 * d + d_ff) * 2
+    assert max(full) <= bound + 8192
+
+
+def test_launch_count():
+    st, n = bpt.bpt_layer_launch_count(1, 65536, 2048, 16, 8192, 1, BF)
+    assert st == bpt.BPT_OK and n == 2 + 5 * 2   # two waves of 256 blocks
+    st, n = bpt.bpt_layer_launch_count(8, 2048, 768, 12, 3072, 1, BF)
+    assert st == bpt.BPT_OK and n == 2 + 5      # one wave of 8 sequences
+    st, n = bpt.bpt_layer_launch_count(0, 2048, 768, 12, 3072, 1, BF)
+    assert st == bpt.BPT_OK and n == 0
+
+
+def fwd(ptrs, B=1, N=256, d=256, h=2, d_ff=512, causal=1, dtype=BF, ws_bytes=1 << 30):
+    return bpt.bpt_layer_forward(*ptrs[:11], B, N, d, h, d_ff, causal, dtype, ptrs[11],
+                                 ptrs[12], ws_bytes, None)
+
+
+# Fake, never-dereferenced addresses: validation must fail before any use.
+GOOD = [0x10000000 + i * 0x1000000 for i in range(13)]
+
+
+def test_forward_rejects_null_pointers():
+    for i in range(13):
+        p = list(GOOD)
+        p[i] = None
+        assert fwd(p) == bpt.BPT_ERR_INVALID_ARG, i
+
+
+def test_forward_rejects_misaligned_pointers():
+    for i in range(13):
+        p = list(GOOD)
+        p[i] += 8
+        assert fwd(p) == bpt.BPT_ERR_INVALID_ARG, i
+
+
+def test_forward_rejects_small_workspace():
+    st, need = bpt.bpt_layer_workspace_size(1, 256, 256, 2, 512, 1, BF)
+    assert fwd(GOOD, ws_bytes=need - 1) == bpt.BPT_ERR_WORKSPACE
+
+
+def test_forward_rejects_aliasing_out_and_x():
+    p = list(GOOD)
+    p[11] = p[0]
+    assert fwd(p) == bpt.BPT_ERR_INVALID_ARG
+
+
+def test_forward_rejects_unsupported_shapes():
+    assert fwd(GOOD, d=96, h=3) == bpt.BPT_ERR_UNSUPPORTED
+    assert fwd(GOOD, d=100, h=3) == bpt.BPT_ERR_INVALID_ARG
+
+
+def test_forward_empty_is_a_no_op():
+    assert fwd([None] * 13, B=0) == bpt.BPT_OK
+    assert fwd([None] * 13, N=0) == bpt.BPT_OK
+
+
+def test_read_error_rejects_null():
+    st, _ = bpt.bpt_read_device_error(None, None)
+    assert st == bpt.BPT_ERR_INVALID_ARG
+
+
+def test_library_has_no_host_fallback_symbols(lib):
+    """The library exports only the C ABI: no second implementation."""
+    out = os.popen(f"nm -D --defined-only {bpt.LIB_PATH}").read()
+    exported = sorted(set(re.findall(r" T (bpt_\w+)", out)))
+    assert exported == header_functions()
