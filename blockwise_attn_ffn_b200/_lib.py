@@ -20,11 +20,12 @@ BPT_OK, BPT_ERR_INVALID_ARG, BPT_ERR_UNSUPPORTED, BPT_ERR_WORKSPACE, BPT_ERR_CUD
 BPT_F32, BPT_BF16 = 0, 1
 KINDS = ["ln1", "qkv", "attn", "wo", "ln2", "w1", "w2"]
 BPT_WAVE_BLOCKS = 256
+BPT_STATIC_WORKSPACE_BYTES = 64 * 1024 * 1024
 
 EXPORTED = [
     "bpt_layer_workspace_size", "bpt_layer_forward", "bpt_read_device_error",
     "bpt_status_string", "bpt_profile_enable", "bpt_profile_read",
-    "bpt_layer_launch_count",
+    "bpt_layer_launch_count", "bpt_layer_forward_static",
 ]
 
 _lib: Optional[ctypes.CDLL] = None
@@ -63,6 +64,8 @@ def load() -> ctypes.CDLL:
     lib.bpt_layer_launch_count.argtypes = [i64, i64, i64, i64, i64, i32, i32,
                                            ctypes.POINTER(ctypes.c_int64)]
     lib.bpt_layer_launch_count.restype = i32
+    lib.bpt_layer_forward_static.argtypes = [vp] * 11 + [i64] * 5 + [i32, i32, vp, vp]
+    lib.bpt_layer_forward_static.restype = i32
     _lib = lib
     return lib
 
@@ -111,6 +114,18 @@ def bpt_profile_read() -> Tuple[int, dict, dict]:
     cnt = (ctypes.c_int64 * n)()
     st = load().bpt_profile_read(ms, cnt, n)
     return st, {k: ms[i] for i, k in enumerate(KINDS)}, {k: cnt[i] for i, k in enumerate(KINDS)}
+
+
+def bpt_layer_forward_static(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
+                             B, N, d, h, d_ff, causal, dtype, out, stream) -> int:
+    """Pointer-level call of the allocation-free variant; returns the status.
+
+    For callers that may not allocate device memory: the library uses its own
+    fixed device array (BPT_STATIC_WORKSPACE_BYTES) as the workspace.
+    """
+    return load().bpt_layer_forward_static(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
+                                           B, N, d, h, d_ff, int(bool(causal)), dtype, out,
+                                           stream)
 
 
 def bpt_layer_launch_count(B, N, d, h, d_ff, causal, dtype) -> Tuple[int, int]:

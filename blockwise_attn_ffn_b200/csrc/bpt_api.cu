@@ -589,3 +589,54 @@ bpt_status bpt_profile_read(double* ms, int64_t* launches, int n) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------ allocation-free variant --
+// Workspace of bpt_layer_forward_static: a file-scope device array, so that
+// callers that may not allocate still get the full layer.  In host code the
+// symbol is only a stand-in; its device address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+static __device__ __align__(256) uint8_t g_bpt_static_ws[BPT_STATIC_WORKSPACE_BYTES];
+
+namespace {
+void* g_static_ws_ptr[64] = {};
+
+bpt_status static_ws_address(void** ptr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BPT_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_static_ws_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_bpt_static_ws) != cudaSuccess || p == nullptr)
+      return BPT_ERR_CUDA;
+    g_static_ws_ptr[dev] = p;
+  }
+  *ptr = g_static_ws_ptr[dev];
+  return BPT_OK;
+}
+}  // namespace
+
+extern "C" bpt_status bpt_layer_forward_static(const void* x, const void* ln1, const void* W_Q,
+                                               const void* W_K, const void* W_V, const void* W_O,
+                                               const void* ln2, const void* W_1, const void* b_1,
+                                               const void* W_2, const void* b_2, int64_t B,
+                                               int64_t N, int64_t d, int64_t h, int64_t d_ff,
+                                               int causal, bpt_dtype dtype, float* out,
+                                               bpt_stream_t stream) {
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_prof_on) return BPT_ERR_INVALID_ARG;
+  }
+  bpt_status st = check_shape(B, N, d, h, d_ff, causal, dtype);
+  if (st != BPT_OK) return st;
+  if (B == 0 || N == 0) return BPT_OK;
+  const void* ptrs[] = {x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, out};
+  for (const void* p : ptrs)
+    if (p == nullptr || misaligned(p)) return BPT_ERR_INVALID_ARG;
+  if (make_plan(B, N, d, h, d_ff, causal, dtype).total > size_t(BPT_STATIC_WORKSPACE_BYTES))
+    return BPT_ERR_WORKSPACE;
+  void* ws = nullptr;
+  st = static_ws_address(&ws);
+  if (st != BPT_OK) return st;
+  return bpt_layer_forward(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, B, N, d, h, d_ff,
+                           causal, dtype, out, ws, size_t(BPT_STATIC_WORKSPACE_BYTES), stream);
+}

@@ -147,6 +147,48 @@ bpt_status bpt_profile_read(double* ms, int64_t* launches, int n);
 bpt_status bpt_layer_launch_count(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff,
                                   int causal, bpt_dtype dtype, int64_t* launches);
 
+/*
+ * bpt_layer_forward_static -- bpt_layer_forward for callers that cannot
+ * allocate device memory.  The paper has no counterpart: this is a deployment
+ * convenience of this library, not part of the method.
+ *
+ * Some callers are not allowed to allocate: code that runs while its stream is
+ * being captured into a CUDA graph (an allocation may synchronise the device
+ * and break the capture), plug-ins whose host framework owns all device memory,
+ * and latency-critical loops that cannot pay for an allocation.  This entry
+ * point takes the same arguments as bpt_layer_forward minus the workspace and
+ * uses instead a workspace of BPT_STATIC_WORKSPACE_BYTES that lives in a
+ * file-scope __device__ array of the library.  The caller still provides x,
+ * the parameters and out.  It calls no cudaMalloc, cudaFree or other
+ * allocating routine.
+ *
+ *   - Size limit: layers whose bpt_layer_workspace_size exceeds
+ *     BPT_STATIC_WORKSPACE_BYTES are rejected with BPT_ERR_WORKSPACE before
+ *     anything is enqueued (for example B=1, N=2048, d=768, d_ff=3072 fits;
+ *     the larger long-context layers do not and need bpt_layer_forward).
+ *   - Memory: every GPU that loads the library holds the array until the
+ *     process exits, whether or not this entry point is used.
+ *   - First call on a device: it looks up the array's device address (once
+ *     per device, with that device current).  Make that first call before any
+ *     stream capture begins.
+ *   - Sharing: all calls on a device use the same array, and it keeps the
+ *     last call's contents (each call clears the header it needs).  Calls
+ *     whose work overlaps on the GPU (different streams, no ordering) race on
+ *     the array and give undefined results: order them on one stream or with
+ *     events.
+ *   - Profiling: returns BPT_ERR_INVALID_ARG while bpt_profile_enable is on
+ *     (profiling creates event objects).
+ *   - A kernel that gives up waiting records it in the array's header, which
+ *     the caller cannot read; as with any timeout, `out` is then undefined.
+ */
+#define BPT_STATIC_WORKSPACE_BYTES (64u * 1024u * 1024u)
+bpt_status bpt_layer_forward_static(const void* x, const void* ln1, const void* W_Q,
+                                    const void* W_K, const void* W_V, const void* W_O,
+                                    const void* ln2, const void* W_1, const void* b_1,
+                                    const void* W_2, const void* b_2, int64_t B, int64_t N,
+                                    int64_t d, int64_t h, int64_t d_ff, int causal,
+                                    bpt_dtype dtype, float* out, bpt_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
