@@ -168,6 +168,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=32)
     ap.add_argument("--ref-rows", type=int, default=16)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="override the workload's N (profiling runs on a smaller case)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -176,6 +178,8 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     cfg = WORKLOADS[args.workload]
+    if args.seq_len:
+        cfg = cfg.with_(N=args.seq_len, name=f"{cfg.name}@N={args.seq_len}")
 
     if args.impl == "reference":
         return run_reference(args, cfg, rank, world)
