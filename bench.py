@@ -321,7 +321,7 @@ def main():
         "pct_bf16_peak": tflops / world / peaks["bf16_tflops"],
         "pct_bf16_peak_sustained": tflops / world / peak_sus,
         "peak_src": peak_src,
-        "roofline": {"bound": "tensor", "kernel": "attn_fwd_tc_kernel", "achieved": achieved,
+        "roofline": {"bound": "tensor", "kernel": "attn_pair_tc_kernel", "achieved": achieved,
                      "peak": peak_sus, "unit": "TFLOP/s", "frac": achieved / peak_sus,
                      "peak_kind": f"bf16_tflops_sustained ({peak_src})",
                      "frac_of_burst": achieved / peaks["bf16_tflops"], "traffic": None},

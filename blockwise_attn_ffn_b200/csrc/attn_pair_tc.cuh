@@ -1,0 +1,458 @@
+// Blockwise attention, two query blocks per CTA (the BPT inner loop on the
+// tcgen05 tensor cores).
+//
+// A CTA owns one head t and two consecutive query blocks of one sequence, tile
+// A = block iA and tile B = block iA + 1 (B may be absent at the end of a
+// sequence or of a wave).  Both tiles walk the same key/value blocks, so each
+// K_j / V_j tile is loaded once into shared memory and used by both.  Per key
+// block j and tile X the CTA keeps the online-softmax state of every query row
+// (reference max m, running sum l, accumulator o):
+//
+//   S_X = Q_X K_j^T                        UMMA, fp32 in tensor memory
+//   P_X = exp2(S_X * log2(e)/sqrt(d_k) - m), l = alpha l + rowsum(P_X)
+//                                           softmax warpgroup X, P_X in bf16
+//                                           written back over S_X in TMEM
+//   O_X = alpha O_X + P_X V_j               UMMA with A = P_X from TMEM
+//
+// Causal: tile X visits blocks j <= iX only (blocks above the diagonal are
+// never loaded or scored) and masks keys after the query on its diagonal
+// block.  Non-causal: a ragged last key block masks keys >= N.
+// The reference max moves only when a row's maximum grows by more than 2^8 in
+// exp2 units; then O_X is rescaled by alpha = exp2(m_old - m_new).  Smaller
+// growth keeps the old reference (exact: o / l does not depend on it; P stays
+// <= 2^8).
+//
+// Ping-pong: the UMMA warp issues PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), ...
+// so the tensor core works on one tile while the other tile's softmax runs.
+// tcgen05.mma issued by one thread executes in order, so S_X(j+1) overwriting
+// the TMEM that P_X(j) occupies is ordered after PV_X(j) has read it.
+//
+// exp2: most elements use the MUFU ex2 instruction; on blocks with no masked
+// key, EMU_CHUNKS of the four 32-column chunks of each row use a polynomial
+// on the FMA pipe instead (Cody-Waite range reduction 2^x = 2^floor(x) *
+// 2^frac, and a cubic fit of 2^f on [0, 1), relative error < 1e-4, below
+// bf16 resolution), so MUFU and FMA share the work.
+//
+// Shared memory: Q_A, Q_B and a ring of NSLOT K/V tiles (loaded K_0, V_0,
+// K_1, V_1, ...), all 128 rows x d_k bf16 in 64-column chunks with the
+// 128-byte swizzle.  Tensor memory: S_A 0..127, S_B 128..255, O_A 256..,
+// O_B 256+d_k...
+//
+// Warp roles (384 threads): 0 TMA, 1 UMMA issue, 2 TMEM owner, 3 idle,
+// 4..7 softmax of tile A, 8..11 softmax of tile B (thread = query row).
+#pragma once
+
+#include "common.cuh"
+
+namespace bpt {
+
+struct AttnPairParams {
+  int N;       // tokens per sequence
+  int nb;      // query blocks per sequence
+  int h;       // heads
+  int d;       // model width (row stride of Q, K and V is 3d)
+  int causal;
+  int item0;   // first flattened block item (batch * nb + block) of the wave
+  int count;   // block items in the wave
+  int seqs;    // >0: the wave is `seqs` whole sequences; 0: part of one sequence
+  __nv_bfloat16* o;  // [count * 128, d] block scratch
+  float scale_log2;  // log2(e) / sqrt(d_k)
+  uint32_t* err;
+};
+
+// Coefficients of 2^f ~ c0 + c1 f + c2 f^2 + c3 f^3 on [0, 1): relative-error
+// fit at Chebyshev nodes refined towards equal ripple (printed by
+// csrc/fit_exp2_poly.py), max relative error 7.5e-5.
+constexpr float kExp2C0 = 0.9999252f;
+constexpr float kExp2C1 = 0.69583344f;
+constexpr float kExp2C2 = 0.22606751f;
+constexpr float kExp2C3 = 0.07802427f;
+
+template <int D, int EMU_CHUNKS>
+struct AttnPairCfg {
+  static constexpr int BQ = 128;
+  static constexpr int BKV = 128;
+  static constexpr int TILE = 128 * D * 2;   // one Q, K or V tile
+  static constexpr int CHUNK = 128 * 128;    // one 64-column swizzled chunk (16 KB)
+  static constexpr int NSLOT = (D == 128) ? 5 : 10;
+  static constexpr int OFF_QA = 0;
+  static constexpr int OFF_QB = TILE;
+  static constexpr int OFF_RING = 2 * TILE;
+  static constexpr int OFF_BAR = OFF_RING + NSLOT * TILE;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t TM_S_B = 128;
+  static constexpr uint32_t TM_O_A = 256;
+  static constexpr uint32_t TM_O_B = 256 + D;
+  static constexpr int THREADS = 384;
+};
+
+// Pair rank -> first block item of the pair and whether its second block
+// exists.  Causal work is handed out longest first (descending query block).
+__device__ __forceinline__ void attn_pair_decode(const AttnPairParams& p, int rank, int& itemA,
+                                                 bool& has_b) {
+  if (p.seqs == 0) {
+    const int npairs = (p.count + 1) >> 1;
+    const int q = p.causal ? (npairs - 1 - rank) : rank;
+    itemA = p.item0 + 2 * q;
+    has_b = 2 * q + 1 < p.count;
+  } else {
+    const int pp = (p.nb + 1) >> 1;  // pairs per sequence
+    int s, q;
+    if (p.causal) {
+      q = pp - 1 - rank / p.seqs;
+      s = rank % p.seqs;
+    } else {
+      s = rank / pp;
+      q = rank % pp;
+    }
+    itemA = p.item0 + s * p.nb + 2 * q;
+    has_b = 2 * q + 1 < p.nb;
+  }
+}
+
+// x is clamped at -125 so that the cubic (>= c0, just under 1, exponent field
+// 126) plus floor(x) keeps a positive exponent field: results stay normal
+// floats down to 2^-125, which bf16 P treats as zero anyway.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.0f);
+  const float xi = floorf(x);
+  const float f = x - xi;
+  float q = fmaf(kExp2C3, f, kExp2C2);
+  q = fmaf(q, f, kExp2C1);
+  q = fmaf(q, f, kExp2C0);
+  return __int_as_float(__float_as_int(q) + (static_cast<int>(xi) << 23));
+}
+
+// Two lanes at once on the packed fp32x2 FMA pipe.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 xi = make_float2(floorf(x.x), floorf(x.y));
+  const float2 f = __fadd2_rn(x, make_float2(-xi.x, -xi.y));
+  float2 q = __ffma2_rn(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
+  q = __ffma2_rn(q, f, make_float2(kExp2C1, kExp2C1));
+  q = __ffma2_rn(q, f, make_float2(kExp2C0, kExp2C0));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (static_cast<int>(xi.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (static_cast<int>(xi.y) << 23)));
+}
+
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc], bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+template <int D, int EMU_CHUNKS>
+__global__ void __launch_bounds__(384, 1)
+    attn_pair_tc_kernel(const __grid_constant__ CUtensorMap mapQKV, const AttnPairParams p) {
+  using C = AttnPairCfg<D, EMU_CHUNKS>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  const uint32_t q_full = smem_u32(bars + 0);
+  const uint32_t ring_full0 = smem_u32(bars + 1);
+  const uint32_t ring_empty0 = smem_u32(bars + 1 + C::NSLOT);
+  const uint32_t s_full0 = smem_u32(bars + 1 + 2 * C::NSLOT);   // [A, B]
+  const uint32_t p_full0 = smem_u32(bars + 3 + 2 * C::NSLOT);   // [A, B]
+  const uint32_t o_done0 = smem_u32(bars + 5 + 2 * C::NSLOT);   // [A, B]
+  const uint32_t drain = smem_u32(bars + 7 + 2 * C::NSLOT);
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rank = blockIdx.x / p.h;
+  const int head = blockIdx.x - rank * p.h;
+  int itemA;
+  bool has_b;
+  attn_pair_decode(p, rank, itemA, has_b);
+  const int bidx = itemA / p.nb;
+  const int iA = itemA - bidx * p.nb;
+  const int iB = iA + 1;
+  const int nA = p.causal ? iA + 1 : p.nb;
+  const int nB = has_b ? (p.causal ? iB + 1 : p.nb) : 0;
+  const int n_kv = nA > nB ? nA : nB;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < C::NSLOT; ++s) {
+      mbar_init(ring_full0 + 8 * s, 1);
+      mbar_init(ring_empty0 + 8 * s, 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(s_full0 + 8 * x, 1);
+      mbar_init(p_full0 + 8 * x, 4);
+      mbar_init(o_done0 + 8 * x, 1);
+    }
+    mbar_init(drain, 1);
+    abort_sh = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(&tmem_base_sh), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  volatile int* abort_flag = &abort_sh;
+  const int colQ = head * D, colK = p.d + head * D, colV = 2 * p.d + head * D;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    tma_prefetch_desc(&mapQKV);
+    int armed[C::NSLOT];
+    for (int s = 0; s < C::NSLOT; ++s) armed[s] = -1;
+    mbar_arrive_expect_tx(q_full, C::TILE * (has_b ? 2 : 1));
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      tma_load_3d(smem_u32(smem + C::OFF_QA + c * C::CHUNK), &mapQKV, q_full, colQ + 64 * c,
+                  iA * C::BQ, bidx);
+      if (has_b)
+        tma_load_3d(smem_u32(smem + C::OFF_QB + c * C::CHUNK), &mapQKV, q_full, colQ + 64 * c,
+                    iB * C::BQ, bidx);
+    }
+    int slot = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int j = 0; j < n_kv && ok; ++j) {
+      for (int w = 0; w < 2; ++w) {
+        if (!mbar_wait(ring_empty0 + 8 * slot, phase ^ 1u, abort_flag, p.err, kSiteAttnProducer)) {
+          ok = false;
+          break;
+        }
+        const uint32_t fb = ring_full0 + 8 * slot;
+        mbar_arrive_expect_tx(fb, C::TILE);
+        armed[slot] = static_cast<int>(phase);
+        const int col = w == 0 ? colK : colV;
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(smem_u32(smem + C::OFF_RING + slot * C::TILE + c * C::CHUNK), &mapQKV, fb,
+                      col + 64 * c, j * C::BKV, bidx);
+        if (++slot == C::NSLOT) {
+          slot = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    mbar_wait_drain(q_full, 0, p.err);
+    for (int s = 0; s < C::NSLOT; ++s)
+      if (armed[s] >= 0) mbar_wait_drain(ring_full0 + 8 * s, static_cast<uint32_t>(armed[s]), p.err);
+  } else if (warp == 1 && lane == 0) {
+    // ----------------------------------------------------------- UMMA issue
+    constexpr uint32_t idesc_s = idesc_bf16_f32(C::BQ, C::BKV, false, false);
+    constexpr uint32_t idesc_o = idesc_bf16_f32(C::BQ, D, false, true);
+    const uint32_t sQA = smem_u32(smem + C::OFF_QA);
+    const uint32_t sQB = smem_u32(smem + C::OFF_QB);
+    const uint32_t ring = smem_u32(smem + C::OFF_RING);
+    auto slot_of = [&](int t) { return t % C::NSLOT; };
+    auto phase_of = [&](int t) { return static_cast<uint32_t>((t / C::NSLOT) & 1); };
+    auto issue_s = [&](uint32_t sQ, uint32_t sK, uint32_t d_tmem) {
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t off = (k >> 2) * C::CHUNK + (k & 3) * 32;
+        umma_bf16(d_tmem, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024),
+                  idesc_s, k > 0 ? 1u : 0u);
+      }
+    };
+    auto issue_pv = [&](uint32_t tP, uint32_t sV, uint32_t d_tmem, bool first) {
+#pragma unroll
+      for (int k = 0; k < C::BKV / 16; ++k)
+        umma_bf16_ts(d_tmem, tP + 8 * k, sdesc_sw128(sV + k * 2048, C::CHUNK, 1024), idesc_o,
+                     (!first || k > 0) ? 1u : 0u);
+    };
+    uint32_t pph[2] = {0, 0};
+    bool ok = mbar_wait(q_full, 0, abort_flag, p.err, kSiteAttnMma);
+    if (ok) ok = mbar_wait(ring_full0 + 8 * slot_of(0), phase_of(0), abort_flag, p.err, kSiteAttnMma);
+    if (ok) {
+      tc_fence_after();
+      const uint32_t sK0 = ring + slot_of(0) * C::TILE;
+      if (nA > 0) {
+        issue_s(sQA, sK0, tmem);
+        umma_commit(s_full0);
+      }
+      if (nB > 0) {
+        issue_s(sQB, sK0, tmem + C::TM_S_B);
+        umma_commit(s_full0 + 8);
+      }
+      umma_commit(ring_empty0 + 8 * slot_of(0));
+    }
+    for (int j = 0; j < n_kv && ok; ++j) {
+      const int tk = 2 * (j + 1), tv = 2 * j + 1;
+      bool k_ready = false;
+      if (!mbar_wait(ring_full0 + 8 * slot_of(tv), phase_of(tv), abort_flag, p.err, kSiteAttnMma)) break;
+      const uint32_t sV = ring + slot_of(tv) * C::TILE;
+      const uint32_t sK = ring + slot_of(tk) * C::TILE;
+      for (int x = 0; x < 2 && ok; ++x) {
+        const int nX = x == 0 ? nA : nB;
+        if (j >= nX) continue;
+        if (!mbar_wait(p_full0 + 8 * x, pph[x], abort_flag, p.err, kSiteAttnMma)) {
+          ok = false;
+          break;
+        }
+        pph[x] ^= 1u;
+        tc_fence_after();
+        const uint32_t tS = tmem + (x == 0 ? 0u : C::TM_S_B);
+        issue_pv(tS, sV, tmem + (x == 0 ? C::TM_O_A : C::TM_O_B), j == 0);
+        if (j + 1 < nX) {
+          if (!k_ready) {
+            if (!mbar_wait(ring_full0 + 8 * slot_of(tk), phase_of(tk), abort_flag, p.err,
+                           kSiteAttnMma)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            k_ready = true;
+          }
+          issue_s(x == 0 ? sQA : sQB, sK, tS);
+          umma_commit(s_full0 + 8 * x);
+        } else {
+          umma_commit(o_done0 + 8 * x);
+        }
+      }
+      if (!ok) break;
+      umma_commit(ring_empty0 + 8 * slot_of(tv));
+      if (k_ready) umma_commit(ring_empty0 + 8 * slot_of(tk));
+    }
+    umma_commit(drain);
+    mbar_wait_drain(drain, 0, p.err);
+  } else if (warp >= 4) {
+    // -------------------------------------------------------------- softmax
+    const int x = (warp - 4) >> 2;  // 0: tile A, 1: tile B
+    const int e = warp & 3;         // TMEM lane quarter
+    const int r = e * 32 + lane;    // query row within the tile
+    const int nX = x == 0 ? nA : nB;
+    const int iX = x == 0 ? iA : iB;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(e * 32) << 16);
+    const uint32_t tS = t_lane + (x == 0 ? 0u : C::TM_S_B);
+    const uint32_t tO = t_lane + (x == 0 ? C::TM_O_A : C::TM_O_B);
+    const uint32_t s_full = s_full0 + 8 * x, p_full = p_full0 + 8 * x, o_done = o_done0 + 8 * x;
+    const float c = p.scale_log2;
+    const bool ragged = (p.N % C::BKV) != 0;
+    float m_run = -INFINITY;
+    float l = 0.f;
+    bool ok = nX > 0;
+    for (int j = 0; j < nX && ok; ++j) {
+      if (!mbar_wait(s_full, j & 1, abort_flag, p.err, kSiteAttnSoftmax)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[C::BKV];
+#pragma unroll
+      for (int cc = 0; cc < C::BKV / 32; ++cc)
+        tmem_ld_32x32b_x32(tS + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[cc * 32]));
+      tmem_ld_wait();
+      const bool masked = p.causal ? (j == iX) : (ragged && j == p.nb - 1);
+      if (masked) {
+        const int lim = p.causal ? r + 1 : p.N - j * C::BKV;
+#pragma unroll
+        for (int k = 0; k < C::BKV; ++k)
+          if (k >= lim) sr[k] = __float_as_uint(-INFINITY);
+      }
+      float mx0 = __uint_as_float(sr[0]), mx1 = __uint_as_float(sr[1]);
+#pragma unroll
+      for (int k = 2; k < C::BKV; k += 2) {
+        mx0 = fmaxf(mx0, __uint_as_float(sr[k]));
+        mx1 = fmaxf(mx1, __uint_as_float(sr[k + 1]));
+      }
+      const float mx = fmaxf(mx0, mx1);
+      float m_new = m_run;
+      bool need = false;
+      if (mx > m_run) {
+        need = (m_run == -INFINITY) || ((mx - m_run) * c > 8.0f);
+        if (need) m_new = mx;
+      }
+      const bool warp_need = __any_sync(0xffffffffu, need) && j > 0;
+      const float alpha =
+          need ? (m_run == -INFINITY ? 0.f : ex2_approx((m_run - m_new) * c)) : 1.f;
+      const float2 cc2 = make_float2(c, c);
+      const float2 mref2 = make_float2(-m_new * c, -m_new * c);
+      float2 sum2 = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int cc = 0; cc < C::BKV / 32; ++cc) {
+        uint32_t pk[16];
+        const bool emu = !masked && cc >= 4 - EMU_CHUNKS;
+#pragma unroll
+        for (int k = 0; k < 32; k += 2) {
+          float2 a = __ffma2_rn(
+              make_float2(__uint_as_float(sr[cc * 32 + k]), __uint_as_float(sr[cc * 32 + k + 1])),
+              cc2, mref2);
+          float2 e2;
+          if (emu) {
+            e2 = exp2_poly2(a);
+          } else {
+            e2.x = ex2_approx(a.x);
+            e2.y = ex2_approx(a.y);
+          }
+          sum2 = __fadd2_rn(sum2, e2);
+          pk[k >> 1] = pack_bf16x2(e2.x, e2.y);
+        }
+        tmem_st_32x32b_x16(tS + cc * 16, pk);
+      }
+      l = alpha * l + (sum2.x + sum2.y);
+      m_run = m_new;
+      if (warp_need) {
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tO + cc * 32, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * alpha);
+          tmem_st_32x32b_x32(tO + cc * 32, v);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    if (ok && mbar_wait(o_done, 0, abort_flag, p.err, kSiteAttnSoftmax)) {
+      tc_fence_after();
+      const float inv_l = 1.0f / l;
+      const long long srow = static_cast<long long>(itemA + x - p.item0) * C::BQ + r;
+      __nv_bfloat16* dst = p.o + srow * p.d + head * D;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tO + cc * 32, v);
+        tmem_ld_wait();
+        uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(v[q * 8 + 0]) * inv_l, __uint_as_float(v[q * 8 + 1]) * inv_l);
+          w.y = pack_bf16x2(__uint_as_float(v[q * 8 + 2]) * inv_l, __uint_as_float(v[q * 8 + 3]) * inv_l);
+          w.z = pack_bf16x2(__uint_as_float(v[q * 8 + 4]) * inv_l, __uint_as_float(v[q * 8 + 5]) * inv_l);
+          w.w = pack_bf16x2(__uint_as_float(v[q * 8 + 6]) * inv_l, __uint_as_float(v[q * 8 + 7]) * inv_l);
+          d4[q] = w;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+}  // namespace bpt

@@ -24,7 +24,7 @@
 #include <vector>
 
 #include "bpt.h"
-#include "attn_tc.cuh"
+#include "attn_pair_tc.cuh"
 #include "common.cuh"
 #include "gemm_tc.cuh"
 #include "rows.cuh"
@@ -35,6 +35,9 @@ namespace {
 using bpt::RowMap;
 
 constexpr int64_t kMaxWave = BPT_WAVE_BLOCKS;
+// 32-column chunks (of four per 128-key row) whose exp2 runs on the FMA pipe.
+constexpr int kEmu128 = 1;
+constexpr int kEmu64 = 2;
 constexpr size_t kHeaderBytes = 256;
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -160,12 +163,12 @@ bpt_status device_info(int* sms) {
       if (cudaFuncSetAttribute(bpt::gemm_bf16_tc_kernel,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                bpt::kGemmSmem) != cudaSuccess ||
-          cudaFuncSetAttribute(bpt::attn_fwd_tc_kernel<64>,
+          cudaFuncSetAttribute(bpt::attn_pair_tc_kernel<64, kEmu64>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               bpt::AttnTile<64>::SMEM) != cudaSuccess ||
-          cudaFuncSetAttribute(bpt::attn_fwd_tc_kernel<128>,
+                               bpt::AttnPairCfg<64, kEmu64>::SMEM) != cudaSuccess ||
+          cudaFuncSetAttribute(bpt::attn_pair_tc_kernel<128, kEmu128>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               bpt::AttnTile<128>::SMEM) != cudaSuccess ||
+                               bpt::AttnPairCfg<128, kEmu128>::SMEM) != cudaSuccess ||
           cudaFuncSetAttribute(bpt::attn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (3 * 64 * 128 + 64 * 65) * 4) != cudaSuccess)
         return BPT_ERR_CUDA;
@@ -354,16 +357,19 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
     const int64_t rows = wv.count * P.blk;
     RowMap map{int(wv.item0), int(P.nb), int(P.N), int(P.blk), 0};
     {
-      bpt::AttnParams ap{};
+      bpt::AttnPairParams ap{};
       ap.N = int(P.N); ap.nb = int(P.nb); ap.h = int(P.h); ap.d = int(d);
       ap.causal = P.causal; ap.item0 = int(wv.item0); ap.count = int(wv.count);
       ap.seqs = int(wv.seqs); ap.o = so; ap.scale_log2 = scale_log2; ap.err = err;
-      const unsigned grid = unsigned(wv.count * P.h);
+      const int64_t pairs = wv.seqs == 0 ? (wv.count + 1) / 2 : wv.seqs * ((P.nb + 1) / 2);
+      const unsigned grid = unsigned(pairs * P.h);
       LaunchScope ls(BPT_KIND_ATTN, s);
       if (P.dk == 128)
-        bpt::attn_fwd_tc_kernel<128><<<grid, 256, bpt::AttnTile<128>::SMEM, s>>>(mQKV, ap);
+        bpt::attn_pair_tc_kernel<128, kEmu128>
+            <<<grid, 384, bpt::AttnPairCfg<128, kEmu128>::SMEM, s>>>(mQKV, ap);
       else
-        bpt::attn_fwd_tc_kernel<64><<<grid, 256, bpt::AttnTile<64>::SMEM, s>>>(mQKV, ap);
+        bpt::attn_pair_tc_kernel<64, kEmu64>
+            <<<grid, 384, bpt::AttnPairCfg<64, kEmu64>::SMEM, s>>>(mQKV, ap);
       if (cudaGetLastError() != cudaSuccess) return BPT_ERR_CUDA;
     }
     {
