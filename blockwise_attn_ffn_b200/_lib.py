@@ -16,9 +16,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libbpt.so")
 
 BPT_OK, BPT_ERR_INVALID_ARG, BPT_ERR_UNSUPPORTED, BPT_ERR_WORKSPACE, BPT_ERR_CUDA, \
-    BPT_ERR_TIMEOUT = range(6)
+    BPT_ERR_TIMEOUT, BPT_ERR_RANGE = range(7)
 BPT_F32, BPT_BF16 = 0, 1
-KINDS = ["ln1", "qkv", "attn", "wo", "ln2", "w1", "w2"]
+KINDS = ["ln1", "qkv", "attn", "wo", "ln2", "w1", "w2", "cvt"]
 BPT_WAVE_BLOCKS = 256
 BPT_STATIC_WORKSPACE_BYTES = 64 * 1024 * 1024
 

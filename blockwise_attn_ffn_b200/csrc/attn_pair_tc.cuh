@@ -10,7 +10,7 @@
 //
 //   S_X = Q_X K_j^T                        UMMA, fp32 in tensor memory
 //   P_X = exp2(S_X * log2(e)/sqrt(d_k) - m), l = alpha l + rowsum(P_X)
-//                                           softmax warpgroup X, P_X in bf16
+//                                           softmax warpgroup X, P_X in fp16
 //                                           written back over S_X in TMEM
 //   O_X = alpha O_X + P_X V_j               UMMA with A = P_X from TMEM
 //
@@ -30,11 +30,11 @@
 // exp2: most elements use the MUFU ex2 instruction; on blocks with no masked
 // key, EMU_CHUNKS of the four 32-column chunks of each row use a polynomial
 // on the FMA pipe instead (Cody-Waite range reduction 2^x = 2^floor(x) *
-// 2^frac, and a cubic fit of 2^f on [0, 1), relative error < 1e-4, below
-// bf16 resolution), so MUFU and FMA share the work.
+// 2^frac, and a cubic fit of 2^f on [0, 1), relative error < 1e-4, near
+// the fp16 resolution of P), so MUFU and FMA share the work.
 //
 // Shared memory: Q_A, Q_B and a ring of NSLOT K/V tiles (loaded K_0, V_0,
-// K_1, V_1, ...), all 128 rows x d_k bf16 in 64-column chunks with the
+// K_1, V_1, ...), all 128 rows x d_k fp16 in 64-column chunks with the
 // 128-byte swizzle.  Tensor memory: S_A 0..127, S_B 128..255, O_A 256..,
 // O_B 256+d_k...
 //
@@ -55,7 +55,7 @@ struct AttnPairParams {
   int item0;   // first flattened block item (batch * nb + block) of the wave
   int count;   // block items in the wave
   int seqs;    // >0: the wave is `seqs` whole sequences; 0: part of one sequence
-  __nv_bfloat16* o;  // [count * 128, d] block scratch
+  __half* o;         // [count * 128, d] block scratch (fp16)
   float scale_log2;  // log2(e) / sqrt(d_k)
   uint32_t* err;
 };
@@ -113,7 +113,7 @@ __device__ __forceinline__ void attn_pair_decode(const AttnPairParams& p, int ra
 
 // x is clamped at -125 so that the cubic (>= c0, just under 1, exponent field
 // 126) plus floor(x) keeps a positive exponent field: results stay normal
-// floats down to 2^-125, which bf16 P treats as zero anyway.
+// floats down to 2^-125, which fp16 P (smallest subnormal 2^-24) rounds to zero.
 __device__ __forceinline__ float exp2_poly(float x) {
   x = fmaxf(x, -125.0f);
   const float xi = floorf(x);
@@ -147,8 +147,8 @@ __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_
       : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem desc], bf16 inputs, fp32 accumulate.
-__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+// D[tmem] (+)= A[tmem] * B[smem desc], fp16 inputs, fp32 accumulate.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                              uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -257,8 +257,8 @@ __global__ void __launch_bounds__(384, 1)
       if (armed[s] >= 0) mbar_wait_drain(ring_full0 + 8 * s, static_cast<uint32_t>(armed[s]), p.err);
   } else if (warp == 1 && lane == 0) {
     // ----------------------------------------------------------- UMMA issue
-    constexpr uint32_t idesc_s = idesc_bf16_f32(C::BQ, C::BKV, false, false);
-    constexpr uint32_t idesc_o = idesc_bf16_f32(C::BQ, D, false, true);
+    constexpr uint32_t idesc_s = idesc_f16_f32(C::BQ, C::BKV, false, false);
+    constexpr uint32_t idesc_o = idesc_f16_f32(C::BQ, D, false, true);
     const uint32_t sQA = smem_u32(smem + C::OFF_QA);
     const uint32_t sQB = smem_u32(smem + C::OFF_QB);
     const uint32_t ring = smem_u32(smem + C::OFF_RING);
@@ -268,14 +268,14 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t off = (k >> 2) * C::CHUNK + (k & 3) * 32;
-        umma_bf16(d_tmem, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024),
+        umma_f16(d_tmem, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024),
                   idesc_s, k > 0 ? 1u : 0u);
       }
     };
     auto issue_pv = [&](uint32_t tP, uint32_t sV, uint32_t d_tmem, bool first) {
 #pragma unroll
       for (int k = 0; k < C::BKV / 16; ++k)
-        umma_bf16_ts(d_tmem, tP + 8 * k, sdesc_sw128(sV + k * 2048, C::CHUNK, 1024), idesc_o,
+        umma_f16_ts(d_tmem, tP + 8 * k, sdesc_sw128(sV + k * 2048, C::CHUNK, 1024), idesc_o,
                      (!first || k > 0) ? 1u : 0u);
     };
     uint32_t pph[2] = {0, 0};
@@ -367,13 +367,15 @@ __global__ void __launch_bounds__(384, 1)
         for (int k = 0; k < C::BKV; ++k)
           if (k >= lim) sr[k] = __float_as_uint(-INFINITY);
       }
-      float mx0 = __uint_as_float(sr[0]), mx1 = __uint_as_float(sr[1]);
+      // Row max as eight independent partial maxima (short dependency chains).
+      float mxp[8];
 #pragma unroll
-      for (int k = 2; k < C::BKV; k += 2) {
-        mx0 = fmaxf(mx0, __uint_as_float(sr[k]));
-        mx1 = fmaxf(mx1, __uint_as_float(sr[k + 1]));
-      }
-      const float mx = fmaxf(mx0, mx1);
+      for (int k = 0; k < 8; ++k) mxp[k] = __uint_as_float(sr[k]);
+#pragma unroll
+      for (int k = 8; k < C::BKV; ++k) mxp[k & 7] = fmaxf(mxp[k & 7], __uint_as_float(sr[k]));
+#pragma unroll
+      for (int k = 0; k < 4; ++k) mxp[k] = fmaxf(mxp[k], mxp[k + 4]);
+      const float mx = fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3]));
       float m_new = m_run;
       bool need = false;
       if (mx > m_run) {
@@ -385,7 +387,8 @@ __global__ void __launch_bounds__(384, 1)
           need ? (m_run == -INFINITY ? 0.f : ex2_approx((m_run - m_new) * c)) : 1.f;
       const float2 cc2 = make_float2(c, c);
       const float2 mref2 = make_float2(-m_new * c, -m_new * c);
-      float2 sum2 = make_float2(0.f, 0.f);
+      float2 sum2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
 #pragma unroll
       for (int cc = 0; cc < C::BKV / 32; ++cc) {
         uint32_t pk[16];
@@ -402,12 +405,13 @@ __global__ void __launch_bounds__(384, 1)
             e2.x = ex2_approx(a.x);
             e2.y = ex2_approx(a.y);
           }
-          sum2 = __fadd2_rn(sum2, e2);
-          pk[k >> 1] = pack_bf16x2(e2.x, e2.y);
+          sum2[(k >> 1) & 3] = __fadd2_rn(sum2[(k >> 1) & 3], e2);
+          pk[k >> 1] = pack_f16x2(e2.x, e2.y);
         }
         tmem_st_32x32b_x16(tS + cc * 16, pk);
       }
-      l = alpha * l + (sum2.x + sum2.y);
+      sum2[0] = __fadd2_rn(__fadd2_rn(sum2[0], sum2[1]), __fadd2_rn(sum2[2], sum2[3]));
+      l = alpha * l + (sum2[0].x + sum2[0].y);
       m_run = m_new;
       if (warp_need) {
 #pragma unroll 1
@@ -429,7 +433,7 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       const float inv_l = 1.0f / l;
       const long long srow = static_cast<long long>(itemA + x - p.item0) * C::BQ + r;
-      __nv_bfloat16* dst = p.o + srow * p.d + head * D;
+      __half* dst = p.o + srow * p.d + head * D;
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t v[32];
@@ -439,10 +443,10 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(v[q * 8 + 0]) * inv_l, __uint_as_float(v[q * 8 + 1]) * inv_l);
-          w.y = pack_bf16x2(__uint_as_float(v[q * 8 + 2]) * inv_l, __uint_as_float(v[q * 8 + 3]) * inv_l);
-          w.z = pack_bf16x2(__uint_as_float(v[q * 8 + 4]) * inv_l, __uint_as_float(v[q * 8 + 5]) * inv_l);
-          w.w = pack_bf16x2(__uint_as_float(v[q * 8 + 6]) * inv_l, __uint_as_float(v[q * 8 + 7]) * inv_l);
+          w.x = pack_f16x2(__uint_as_float(v[q * 8 + 0]) * inv_l, __uint_as_float(v[q * 8 + 1]) * inv_l);
+          w.y = pack_f16x2(__uint_as_float(v[q * 8 + 2]) * inv_l, __uint_as_float(v[q * 8 + 3]) * inv_l);
+          w.z = pack_f16x2(__uint_as_float(v[q * 8 + 4]) * inv_l, __uint_as_float(v[q * 8 + 5]) * inv_l);
+          w.w = pack_f16x2(__uint_as_float(v[q * 8 + 6]) * inv_l, __uint_as_float(v[q * 8 + 7]) * inv_l);
           d4[q] = w;
         }
       }

@@ -35,9 +35,16 @@ namespace {
 using bpt::RowMap;
 
 constexpr int64_t kMaxWave = BPT_WAVE_BLOCKS;
-// 32-column chunks (of four per 128-key row) whose exp2 runs on the FMA pipe.
-constexpr int kEmu128 = 1;
-constexpr int kEmu64 = 2;
+// 32-column chunks (of four per 128-key row) whose exp2 runs on the FMA pipe
+// (compile-time tuning knobs).
+#ifndef BPT_EMU_CHUNKS_DK128
+#define BPT_EMU_CHUNKS_DK128 0
+#endif
+#ifndef BPT_EMU_CHUNKS_DK64
+#define BPT_EMU_CHUNKS_DK64 0
+#endif
+constexpr int kEmu128 = BPT_EMU_CHUNKS_DK128;
+constexpr int kEmu64 = BPT_EMU_CHUNKS_DK64;
 constexpr size_t kHeaderBytes = 256;
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -55,7 +62,7 @@ struct Plan {
   int64_t G;     // >0: each wave holds G whole sequences
   int64_t n_waves, P;
   size_t esize;
-  size_t off_qkv, off_o, off_v, off_h, total;
+  size_t off_w16, off_qkv, off_o, off_v, off_h, total;
 
   Wave wave(int64_t w) const {
     Wave r;
@@ -124,6 +131,9 @@ Plan make_plan(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff, int cau
     p.P = p.G * p.nb;
   }
   size_t off = align_up(kHeaderBytes, 1024);
+  p.off_w16 = off;
+  if (dtype == BPT_BF16)  // fp16 copies of W_Q, W_K, W_V, W_O, W_1, W_2
+    off = align_up(off + (size_t(4 * d * d) + size_t(2 * d * d_ff)) * 2, 1024);
   p.off_qkv = off;
   off = align_up(off + size_t(B * N) * size_t(3 * d) * p.esize, 1024);
   const size_t rows = size_t(p.P * p.blk);
@@ -160,7 +170,7 @@ bpt_status device_info(int* sms) {
     di.ok = (major == 10 && minor == 0);
     di.sms = n;
     if (di.ok) {
-      if (cudaFuncSetAttribute(bpt::gemm_bf16_tc_kernel,
+      if (cudaFuncSetAttribute(bpt::gemm_f16_tc_kernel,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                bpt::kGemmSmem) != cudaSuccess ||
           cudaFuncSetAttribute(bpt::attn_pair_tc_kernel<64, kEmu64>,
@@ -196,9 +206,9 @@ bpt_status get_encoder() {
   return BPT_OK;
 }
 
-// bf16 tiles with the 128-byte swizzle; dims/strides innermost first.
-bool encode_bf16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
-                 const uint64_t* strides_bytes, const uint32_t* box) {
+// fp16 tiles with the 128-byte swizzle; dims/strides innermost first.
+bool encode_f16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                const uint64_t* strides_bytes, const uint32_t* box) {
   cuuint64_t gd[3], gs[2];
   cuuint32_t bx[3], es[3] = {1, 1, 1};
   for (int i = 0; i < rank; ++i) {
@@ -206,7 +216,7 @@ bool encode_bf16(CUtensorMap* m, const void* base, int rank, const uint64_t* dim
     bx[i] = box[i];
   }
   for (int i = 0; i + 1 < rank; ++i) gs[i] = strides_bytes[i];
-  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base),
+  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, rank, const_cast<void*>(base),
                               gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -218,21 +228,21 @@ bool map_a(CUtensorMap* m, const void* base, int64_t rows, int64_t K) {
   const uint64_t dims[2] = {uint64_t(K), uint64_t(rows)};
   const uint64_t st[1] = {uint64_t(K) * 2};
   const uint32_t box[2] = {64, 128};
-  return encode_bf16(m, base, 2, dims, st, box);
+  return encode_f16(m, base, 2, dims, st, box);
 }
 // B operand: [K, cols] row-major, 64 x 64 boxes.
 bool map_b(CUtensorMap* m, const void* base, int64_t K, int64_t cols) {
   const uint64_t dims[2] = {uint64_t(cols), uint64_t(K)};
   const uint64_t st[1] = {uint64_t(cols) * 2};
   const uint32_t box[2] = {64, 64};
-  return encode_bf16(m, base, 2, dims, st, box);
+  return encode_f16(m, base, 2, dims, st, box);
 }
 // QKV viewed as [B][N][3d]: boxes of 64 columns x 128 tokens x 1 sequence.
 bool map_qkv(CUtensorMap* m, const void* base, int64_t B, int64_t N, int64_t d) {
   const uint64_t dims[3] = {uint64_t(3 * d), uint64_t(N), uint64_t(B)};
   const uint64_t st[2] = {uint64_t(3 * d) * 2, uint64_t(N) * uint64_t(3 * d) * 2};
   const uint32_t box[3] = {64, 128, 1};
-  return encode_bf16(m, base, 3, dims, st, box);
+  return encode_f16(m, base, 3, dims, st, box);
 }
 
 // -------------------------------------------------------------- profiling --
@@ -277,14 +287,14 @@ struct LaunchScope {
 // ----------------------------------------------------------------- launches --
 template <typename TIn, typename TOut, typename TP>
 cudaError_t launch_ln(const TIn* in, const TP* ln, TOut* out, int64_t rows, int64_t d, RowMap map,
-                      cudaStream_t s) {
+                      uint32_t* err, cudaStream_t s) {
   const int nv = int((d + 255) / 256);
   const dim3 grid(unsigned((rows + bpt::kLnWarps - 1) / bpt::kLnWarps));
   const dim3 block(bpt::kLnWarps * 32);
 #define BPT_LN_CASE(NV)                                                                    \
   if (nv <= NV) {                                                                          \
     bpt::ln_rows_kernel<NV, TIn, TOut, TP><<<grid, block, 0, s>>>(in, ln, out, rows, int(d), \
-                                                                  map);                    \
+                                                                  map, err);               \
     return cudaGetLastError();                                                             \
   }
   BPT_LN_CASE(1)
@@ -306,7 +316,7 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUten
   const int64_t tiles = int64_t((gp.M + bpt::kGemmBM - 1) / bpt::kGemmBM) *
                         int64_t((gp.N + bpt::kGemmBN - 1) / bpt::kGemmBN);
   const unsigned grid = unsigned(std::min<int64_t>(tiles, sms));
-  bpt::gemm_bf16_tc_kernel<<<grid, bpt::kGemmThreads, bpt::kGemmSmem, s>>>(a, b0, b1, b2, gp);
+  bpt::gemm_f16_tc_kernel<<<grid, bpt::kGemmThreads, bpt::kGemmSmem, s>>>(a, b0, b1, b2, gp);
   return cudaGetLastError();
 }
 
@@ -317,35 +327,63 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
                         const void* W_1, const void* b_1, const void* W_2, const void* b_2,
                         float* out, uint8_t* ws, cudaStream_t s, int sms) {
   using bf = __nv_bfloat16;
+  using hf = __half;
   const int64_t M = P.B * P.N, d = P.d, d_ff = P.d_ff;
   uint32_t* err = reinterpret_cast<uint32_t*>(ws);
-  bf* xn = reinterpret_cast<bf*>(out);  // LN1(x) lives in `out` until the waves start
-  bf* qkv = reinterpret_cast<bf*>(ws + P.off_qkv);
-  bf* so = reinterpret_cast<bf*>(ws + P.off_o);
-  bf* sv = reinterpret_cast<bf*>(ws + P.off_v);
-  bf* sh = reinterpret_cast<bf*>(ws + P.off_h);
+  // Tensor-core operands are fp16: the bf16 weights are copied to fp16 once
+  // per call (exact in the fp16 normal range), activations are stored fp16.
+  hf* w16 = reinterpret_cast<hf*>(ws + P.off_w16);
+  hf* wq = w16;
+  hf* wk = wq + d * d;
+  hf* wv = wk + d * d;
+  hf* wo = wv + d * d;
+  hf* w1 = wo + d * d;
+  hf* w2 = w1 + d * d_ff;
+  hf* xn = reinterpret_cast<hf*>(out);  // LN1(x) lives in `out` until the waves start
+  hf* qkv = reinterpret_cast<hf*>(ws + P.off_qkv);
+  hf* so = reinterpret_cast<hf*>(ws + P.off_o);
+  hf* sv = reinterpret_cast<hf*>(ws + P.off_v);
+  hf* sh = reinterpret_cast<hf*>(ws + P.off_h);
   const int64_t R = P.P * P.blk;  // scratch rows
 
   CUtensorMap mXn, mWq, mWk, mWv, mQKV, mO, mWo, mV, mW1, mH, mW2;
-  bool ok = map_a(&mXn, xn, M, d) && map_b(&mWq, W_Q, d, d) && map_b(&mWk, W_K, d, d) &&
-            map_b(&mWv, W_V, d, d) && map_qkv(&mQKV, qkv, P.B, P.N, d) && map_a(&mO, so, R, d) &&
-            map_b(&mWo, W_O, d, d) && map_a(&mV, sv, R, d) && map_b(&mW1, W_1, d, d_ff) &&
-            map_a(&mH, sh, R, d_ff) && map_b(&mW2, W_2, d_ff, d);
+  bool ok = map_a(&mXn, xn, M, d) && map_b(&mWq, wq, d, d) && map_b(&mWk, wk, d, d) &&
+            map_b(&mWv, wv, d, d) && map_qkv(&mQKV, qkv, P.B, P.N, d) && map_a(&mO, so, R, d) &&
+            map_b(&mWo, wo, d, d) && map_a(&mV, sv, R, d) && map_b(&mW1, w1, d, d_ff) &&
+            map_a(&mH, sh, R, d_ff) && map_b(&mW2, w2, d_ff, d);
   if (!ok) return BPT_ERR_CUDA;
 
+  {
+    bpt::CvtSegments cs{};
+    const void* src[6] = {W_Q, W_K, W_V, W_O, W_1, W_2};
+    hf* dst[6] = {wq, wk, wv, wo, w1, w2};
+    const int64_t n[6] = {d * d, d * d, d * d, d * d, d * d_ff, d_ff * d};
+    long long acc = 0;
+    for (int k = 0; k < 6; ++k) {
+      cs.src[k] = static_cast<const bf*>(src[k]);
+      cs.dst[k] = dst[k];
+      acc += n[k] / 8;
+      cs.n8_end[k] = acc;
+    }
+    cs.count = 6;
+    const unsigned grid = unsigned(std::min<long long>((acc + 255) / 256, int64_t(sms) * 8));
+    LaunchScope ls(BPT_KIND_CVT, s);
+    bpt::cvt_bf16_to_f16_kernel<<<grid, 256, 0, s>>>(cs, err);
+    if (cudaGetLastError() != cudaSuccess) return BPT_ERR_CUDA;
+  }
   RowMap ident{0, 1, 1, 1, 1};
   {
     LaunchScope ls(BPT_KIND_LN1, s);
-    if (launch_ln<bf, bf, bf>(static_cast<const bf*>(x), static_cast<const bf*>(ln1), xn, M, d,
-                              ident, s) != cudaSuccess)
+    if (launch_ln<bf, hf, bf>(static_cast<const bf*>(x), static_cast<const bf*>(ln1), xn, M, d,
+                              ident, err, s) != cudaSuccess)
       return BPT_ERR_CUDA;
   }
   {
     bpt::GemmParams g{};
     g.M = int(M); g.N = int(3 * d); g.K = int(d);
     g.n_sub = int(d); g.n_maps = 3;
-    g.epi = bpt::kEpiStoreBf16;
-    g.out_bf16 = qkv; g.ld_out = 3 * d;
+    g.epi = bpt::kEpiStoreF16;
+    g.out_h = qkv; g.ld_out = 3 * d;
     g.map = ident;
     g.err = err;
     LaunchScope ls(BPT_KIND_QKV, s);
@@ -353,15 +391,15 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
   }
   const float scale_log2 = float(1.4426950408889634 / std::sqrt(double(P.dk)));
   for (int64_t w = 0; w < P.n_waves; ++w) {
-    const Wave wv = P.wave(w);
-    const int64_t rows = wv.count * P.blk;
-    RowMap map{int(wv.item0), int(P.nb), int(P.N), int(P.blk), 0};
+    const Wave wv_ = P.wave(w);
+    const int64_t rows = wv_.count * P.blk;
+    RowMap map{int(wv_.item0), int(P.nb), int(P.N), int(P.blk), 0};
     {
       bpt::AttnPairParams ap{};
       ap.N = int(P.N); ap.nb = int(P.nb); ap.h = int(P.h); ap.d = int(d);
-      ap.causal = P.causal; ap.item0 = int(wv.item0); ap.count = int(wv.count);
-      ap.seqs = int(wv.seqs); ap.o = so; ap.scale_log2 = scale_log2; ap.err = err;
-      const int64_t pairs = wv.seqs == 0 ? (wv.count + 1) / 2 : wv.seqs * ((P.nb + 1) / 2);
+      ap.causal = P.causal; ap.item0 = int(wv_.item0); ap.count = int(wv_.count);
+      ap.seqs = int(wv_.seqs); ap.o = so; ap.scale_log2 = scale_log2; ap.err = err;
+      const int64_t pairs = wv_.seqs == 0 ? (wv_.count + 1) / 2 : wv_.seqs * ((P.nb + 1) / 2);
       const unsigned grid = unsigned(pairs * P.h);
       LaunchScope ls(BPT_KIND_ATTN, s);
       if (P.dk == 128)
@@ -385,7 +423,7 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
     }
     {
       LaunchScope ls(BPT_KIND_LN2, s);
-      if (launch_ln<float, bf, bf>(out, static_cast<const bf*>(ln2), sv, rows, d, map, s) !=
+      if (launch_ln<float, hf, bf>(out, static_cast<const bf*>(ln2), sv, rows, d, map, err, s) !=
           cudaSuccess)
         return BPT_ERR_CUDA;
     }
@@ -394,7 +432,7 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
       g.M = int(rows); g.N = int(d_ff); g.K = int(d);
       g.n_sub = int(d_ff); g.n_maps = 1;
       g.epi = bpt::kEpiGeluBias;
-      g.out_bf16 = sh; g.ld_out = d_ff;
+      g.out_h = sh; g.ld_out = d_ff;
       g.bias = static_cast<const bf*>(b_1);
       g.map = ident; g.err = err;
       LaunchScope ls(BPT_KIND_W1, s);
@@ -425,6 +463,7 @@ bpt_status forward_f32(const Plan& P, const float* x, const float* ln1, const fl
   float* sv = reinterpret_cast<float*>(ws + P.off_v);
   float* sh = reinterpret_cast<float*>(ws + P.off_h);
   float* xn = out;  // LN1(x) lives in `out` until the waves start
+  uint32_t* err = reinterpret_cast<uint32_t*>(ws);
   RowMap ident{0, 1, 1, 1, 1};
   auto gemm = [&](int kind, const float* A, int64_t Mr, int64_t Nc, int64_t K, const float* B0,
                   const float* B1, const float* B2, int64_t n_sub, int epi, float* o,
@@ -442,10 +481,10 @@ bpt_status forward_f32(const Plan& P, const float* x, const float* ln1, const fl
   };
   {
     LaunchScope ls(BPT_KIND_LN1, s);
-    if (launch_ln<float, float, float>(x, ln1, xn, M, d, ident, s) != cudaSuccess)
+    if (launch_ln<float, float, float>(x, ln1, xn, M, d, ident, err, s) != cudaSuccess)
       return BPT_ERR_CUDA;
   }
-  if (!gemm(BPT_KIND_QKV, xn, M, 3 * d, d, W_Q, W_K, W_V, d, bpt::kEpiStoreBf16, qkv, 3 * d,
+  if (!gemm(BPT_KIND_QKV, xn, M, 3 * d, d, W_Q, W_K, W_V, d, bpt::kEpiStoreF16, qkv, 3 * d,
             nullptr, nullptr, ident))
     return BPT_ERR_CUDA;
   for (int64_t w = 0; w < P.n_waves; ++w) {
@@ -467,7 +506,7 @@ bpt_status forward_f32(const Plan& P, const float* x, const float* ln1, const fl
       return BPT_ERR_CUDA;
     {
       LaunchScope ls(BPT_KIND_LN2, s);
-      if (launch_ln<float, float, float>(out, ln2, sv, rows, d, map, s) != cudaSuccess)
+      if (launch_ln<float, float, float>(out, ln2, sv, rows, d, map, err, s) != cudaSuccess)
         return BPT_ERR_CUDA;
     }
     if (!gemm(BPT_KIND_W1, sv, rows, d_ff, d, W_1, W_1, W_1, d_ff, bpt::kEpiGeluBias, sh, d_ff,
@@ -499,7 +538,7 @@ bpt_status bpt_layer_launch_count(int64_t B, int64_t N, int64_t d, int64_t h, in
   const bpt_status st = check_shape(B, N, d, h, d_ff, causal, dtype);
   if (st != BPT_OK) return st;
   const Plan P = make_plan(B, N, d, h, d_ff, causal, dtype);
-  *launches = P.items == 0 ? 0 : 2 + 5 * P.n_waves;
+  *launches = P.items == 0 ? 0 : (dtype == BPT_BF16 ? 3 : 2) + 5 * P.n_waves;
   return BPT_OK;
 }
 
@@ -566,6 +605,7 @@ const char* bpt_status_string(bpt_status status) {
     case BPT_ERR_WORKSPACE: return "BPT_ERR_WORKSPACE: workspace smaller than bpt_layer_workspace_size";
     case BPT_ERR_CUDA: return "BPT_ERR_CUDA: a CUDA call failed";
     case BPT_ERR_TIMEOUT: return "BPT_ERR_TIMEOUT: a kernel gave up waiting on a barrier";
+    case BPT_ERR_RANGE: return "BPT_ERR_RANGE: a tensor-core operand exceeded the fp16 range";
   }
   return "BPT_UNKNOWN_STATUS";
 }

@@ -9,6 +9,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -18,12 +19,17 @@ namespace bpt {
 // Device error word layout: low byte = bpt_status code, next byte = site.
 enum : uint32_t {
   kErrTimeout = 5u,
+  kErrRange = 6u,  // a value outside the fp16 range of the tensor-core operands
 };
 enum : uint32_t {
   kSiteGemmProducer = 1, kSiteGemmMma = 2, kSiteGemmEpilogue = 3,
   kSiteAttnProducer = 4, kSiteAttnMma = 5, kSiteAttnSoftmax = 6,
   kSiteDrain = 7,
+  kSiteRangeWeights = 8, kSiteRangeQKV = 9, kSiteRangeHidden = 10, kSiteRangeLN = 11,
 };
+
+// Largest finite fp16 value; operands beyond it (or NaN) are reported.
+constexpr float kF16Max = 65504.0f;
 
 // Wall-time bound of one wait.  Kernels here finish in milliseconds; a wait
 // this long means a lost arrive, so the kernel gives up instead of spinning.
@@ -150,8 +156,8 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem desc] * B[smem desc], bf16 inputs, fp32 accumulate.
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+// D[tmem] (+)= A[smem desc] * B[smem desc], 16-bit inputs, fp32 accumulate.
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                           uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -169,11 +175,12 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
                : "memory");
 }
 
-// Instruction descriptor, kind::f16: D fp32, A and B bf16.  a_mn / b_mn select
-// MN-major operands.  Field positions: D format [4,6), A format [7,10),
-// B format [10,13), A major 15, B major 16, N>>3 [17,23), M>>4 [24,29).
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, bool b_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) |
+// Instruction descriptor, kind::f16 with D fp32 and A, B both fp16 (format
+// code 0; bf16 would be 1 -- one instruction never mixes the two).  a_mn /
+// b_mn select MN-major operands.  Field positions: D format [4,6), A format
+// [7,10), B format [10,13), A major 15, B major 16, N>>3 [17,23), M>>4 [24,29).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4) | (0u << 7) | (0u << 10) | ((a_mn ? 1u : 0u) << 15) |
          ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
@@ -235,6 +242,17 @@ __device__ __forceinline__ float ex2_approx(float x) {
 }
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+// Two floats -> fp16x2 (round to nearest even); `bad` is raised when either is
+// outside the finite fp16 range or NaN.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi, bool& bad) {
+  bad |= !(fabsf(lo) <= kF16Max) || !(fabsf(hi) <= kF16Max);
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
 __device__ __forceinline__ float gelu_erf(float z) {

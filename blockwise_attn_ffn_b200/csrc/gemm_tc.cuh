@@ -1,8 +1,8 @@
 // Persistent tcgen05 GEMM with fused epilogues: C[M, N] = A[M, K] * B[K, N].
 //
-//   A: bf16 [M, K] row-major (K contiguous), loaded by TMA as 128 x 64 tiles
+//   A: fp16 [M, K] row-major (K contiguous), loaded by TMA as 128 x 64 tiles
 //      with the 128-byte swizzle -> K-major UMMA operand.
-//   B: bf16 [K, N] row-major (N contiguous; weights are [d_in, d_out]) loaded
+//   B: fp16 [K, N] row-major (N contiguous; weights are [d_in, d_out]) loaded
 //      as four 64(N) x 64(K) boxes -> MN-major UMMA operand, no transpose.
 //      B may be the column concatenation of up to three matrices with the
 //      same number of columns each (W_Q | W_K | W_V).
@@ -14,25 +14,27 @@
 // 4+e reads TMEM lanes 32e..32e+31, i.e. accumulator rows 32e..32e+31).
 //
 // Epilogues (all in fp32 before the final rounding):
-//   kEpiStoreBf16   out_bf16[row, col] = acc                     (QKV)
-//   kEpiResidX      out_f32[g, col]    = x[g, col] + acc         (y = x + o W_O)
-//   kEpiGeluBias    out_bf16[row, col] = GELU(acc + bias[col])   (FFN hidden)
-//   kEpiBiasAccum   out_f32[g, col]   += acc + bias[col]         (Z = y + h W_2 + b_2)
-// where g = map(row) is the residual-stream row of a scratch row.
+//   kEpiStoreF16    out_h[row, col]  = acc                       (QKV, fp16)
+//   kEpiResidX      out_f32[g, col]  = x[g, col] + acc           (y = x + o W_O)
+//   kEpiGeluBias    out_h[row, col]  = GELU(acc + bias[col])     (FFN hidden, fp16)
+//   kEpiBiasAccum   out_f32[g, col] += acc + bias[col]           (Z = y + h W_2 + b_2)
+// where g = map(row) is the residual-stream row of a scratch row; x and the
+// biases are the caller's bf16 tensors.  An fp16 store of a value beyond the
+// fp16 range (or NaN) is reported in the device error word.
 #pragma once
 
 #include "common.cuh"
 
 namespace bpt {
 
-enum GemmEpi : int { kEpiStoreBf16 = 0, kEpiResidX = 1, kEpiGeluBias = 2, kEpiBiasAccum = 3 };
+enum GemmEpi : int { kEpiStoreF16 = 0, kEpiResidX = 1, kEpiGeluBias = 2, kEpiBiasAccum = 3 };
 
 struct GemmParams {
   int M, N, K;     // problem size (N, K multiples of 64)
   int n_sub;       // columns of each concatenated B matrix
   int n_maps;      // B matrices in use (1..3)
   int epi;
-  __nv_bfloat16* out_bf16;
+  __half* out_h;
   long long ld_out;
   float* out_f32;
   long long ld_f32;
@@ -65,7 +67,7 @@ __device__ __forceinline__ void gemm_tile_coords(int tile, int m_blocks, int n_b
 }
 
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap mapA,
+    gemm_f16_tc_kernel(const __grid_constant__ CUtensorMap mapA,
                         const __grid_constant__ CUtensorMap mapB0,
                         const __grid_constant__ CUtensorMap mapB1,
                         const __grid_constant__ CUtensorMap mapB2, const GemmParams p) {
@@ -156,7 +158,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (armed[s] >= 0) mbar_wait_drain(full0 + 8 * s, static_cast<uint32_t>(armed[s]), p.err);
   } else if (warp == 1 && lane == 0) {
     // ----------------------------------------------------------- UMMA issue
-    constexpr uint32_t idesc = idesc_bf16_f32(kGemmBM, kGemmBN, false, true);
+    constexpr uint32_t idesc = idesc_f16_f32(kGemmBM, kGemmBN, false, true);
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
@@ -178,7 +180,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int k = 0; k < kGemmBK / 16; ++k) {
           const uint64_t ad = sdesc_sw128(a_base + k * 32, 16, 1024);
           const uint64_t bd = sdesc_sw128(b_base + k * 2048, 8192, 1024);
-          umma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+          umma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
         }
         umma_commit(empty0 + 8 * stage);
         if (++stage == kGemmStages) {
@@ -209,7 +211,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const long long row = static_cast<long long>(mb) * kGemmBM + e * 32 + lane;
       long long g = -1;
       bool row_ok;
-      if (p.epi == kEpiStoreBf16 || p.epi == kEpiGeluBias) {
+      if (p.epi == kEpiStoreF16 || p.epi == kEpiGeluBias) {
         row_ok = row < p.M;
       } else {
         g = row < p.M ? p.map.map(row) : -1;
@@ -227,7 +229,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         float v[32];
 #pragma unroll
         for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
-        if (p.epi == kEpiStoreBf16 || p.epi == kEpiGeluBias) {
+        if (p.epi == kEpiStoreF16 || p.epi == kEpiGeluBias) {
           if (p.epi == kEpiGeluBias) {
             const uint4* bp = reinterpret_cast<const uint4*>(p.bias + col0);
 #pragma unroll
@@ -238,16 +240,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               for (int k = 0; k < 8; ++k) v[q * 8 + k] = gelu_erf(v[q * 8 + k] + __bfloat162float(bh[k]));
             }
           }
-          uint4* dst = reinterpret_cast<uint4*>(p.out_bf16 + row * p.ld_out + col0);
+          uint4* dst = reinterpret_cast<uint4*>(p.out_h + row * p.ld_out + col0);
+          bool bad = false;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             uint4 w;
-            w.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
-            w.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
-            w.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
-            w.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+            w.x = pack_f16x2(v[q * 8 + 0], v[q * 8 + 1], bad);
+            w.y = pack_f16x2(v[q * 8 + 2], v[q * 8 + 3], bad);
+            w.z = pack_f16x2(v[q * 8 + 4], v[q * 8 + 5], bad);
+            w.w = pack_f16x2(v[q * 8 + 6], v[q * 8 + 7], bad);
             dst[q] = w;
           }
+          if (bad)
+            record_error(p.err, kErrRange,
+                         p.epi == kEpiGeluBias ? kSiteRangeHidden : kSiteRangeQKV);
         } else {
           float4* dst = reinterpret_cast<float4*>(p.out_f32 + g * p.ld_f32 + col0);
           if (p.epi == kEpiResidX) {

@@ -4,10 +4,13 @@
 // deviations (two passes over registers), eps = 1e-5 inside the square root,
 // then gamma * (x - mean) / sqrt(var + eps) + beta.
 //
-//   ln_rows_bf16:  bf16 rows -> bf16 rows                       (LN1)
-//   ln_rows_f32to_bf16: fp32 residual rows (via a row map) -> bf16 scratch
-//                  rows; scratch rows with no residual row get zeros  (LN2)
-//   ln_rows_f32:   fp32 rows (via a row map) -> fp32 rows        (fp32 path)
+// One template serves every case: input rows are read through a row map
+// (scratch rows with no residual row get zeros) and written densely.
+//   bf16 x rows            -> fp16 rows    (LN1, tensor-core path)
+//   fp32 residual rows y   -> fp16 rows    (LN2, tensor-core path)
+//   fp32 rows              -> fp32 rows    (LN1 / LN2, fp32 path)
+// An fp16 output beyond the fp16 range (or NaN) is reported in the device
+// error word.
 #pragma once
 
 #include "common.cuh"
@@ -49,6 +52,24 @@ __device__ __forceinline__ void store8(__nv_bfloat16* p, const float* v) {
   w.w = pack_bf16x2(v[6], v[7]);
   *reinterpret_cast<uint4*>(p) = w;
 }
+__device__ __forceinline__ void load8(const __half* p, float* v) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const __half* h = reinterpret_cast<const __half*>(&u);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) v[k] = __half2float(h[k]);
+}
+__device__ __forceinline__ void store8(__half* p, const float* v, bool& bad) {
+  uint4 w;
+  w.x = pack_f16x2(v[0], v[1], bad);
+  w.y = pack_f16x2(v[2], v[3], bad);
+  w.z = pack_f16x2(v[4], v[5], bad);
+  w.w = pack_f16x2(v[6], v[7], bad);
+  *reinterpret_cast<uint4*>(p) = w;
+}
+__device__ __forceinline__ void store8(float* p, const float* v, bool&) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  *reinterpret_cast<float4*>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
 __device__ __forceinline__ void store8(float* p, const float* v) {
   *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
   *reinterpret_cast<float4*>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
@@ -59,18 +80,19 @@ __device__ __forceinline__ void store8(float* p, const float* v) {
 template <int NV, typename TIn, typename TOut, typename TP>
 __global__ void __launch_bounds__(kLnWarps * 32)
     ln_rows_kernel(const TIn* __restrict__ in, const TP* __restrict__ ln, TOut* __restrict__ out,
-                   long long rows, int d, RowMap in_map) {
+                   long long rows, int d, RowMap in_map, uint32_t* err) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long s = static_cast<long long>(blockIdx.x) * kLnWarps + warp;
   if (s >= rows) return;
   const long long g = in_map.map(s);
   TOut* orow = out + s * d;
+  bool bad = false;
   if (g < 0) {
     float z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
     for (int q = 0; q < NV; ++q) {
       const int c = (lane + 32 * q) * 8;
-      if (c < d) store8(orow + c, z);
+      if (c < d) store8(orow + c, z, bad);
     }
     return;
   }
@@ -110,9 +132,37 @@ __global__ void __launch_bounds__(kLnWarps * 32)
       load8(ln + d + c, bt);
 #pragma unroll
       for (int k = 0; k < 8; ++k) o[k] = (v[q][k] - mean) * rstd * gm[k] + bt[k];
-      store8(orow + c, o);
+      store8(orow + c, o, bad);
     }
   }
+  if (bad) record_error(err, kErrRange, kSiteRangeLN);
+}
+
+// bf16 -> fp16 copies of the weight matrices, eight elements per thread and
+// step (each segment's length is a multiple of 8).  Values within the fp16
+// normal range convert exactly; magnitudes below 2^-14 become fp16 subnormals
+// (absolute error <= 2^-25); anything beyond the fp16 range is reported.
+struct CvtSegments {
+  const __nv_bfloat16* src[6];
+  __half* dst[6];
+  long long n8_end[6];  // cumulative count of 8-element groups
+  int count;
+};
+
+__global__ void __launch_bounds__(256) cvt_bf16_to_f16_kernel(const CvtSegments seg,
+                                                             uint32_t* err) {
+  const long long total = seg.n8_end[seg.count - 1];
+  bool bad = false;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    int k = 0;
+    while (i >= seg.n8_end[k]) ++k;
+    const long long j = i - (k ? seg.n8_end[k - 1] : 0);
+    float v[8];
+    load8(seg.src[k] + 8 * j, v);
+    store8(seg.dst[k] + 8 * j, v, bad);
+  }
+  if (bad) record_error(err, kErrRange, kSiteRangeWeights);
 }
 
 }  // namespace bpt

@@ -17,7 +17,7 @@ struct GemmF32Params {
   const float* A;     // [M, K]
   const float* B[3];  // [K, n_sub] each
   int epi;            // GemmEpi
-  float* out;         // kEpiStoreBf16 / kEpiGeluBias (fp32 here): [M, ld_out]; else residual rows
+  float* out;         // kEpiStoreF16 / kEpiGeluBias (fp32 here): [M, ld_out]; else residual rows
   long long ld_out;
   const float* resid;  // kEpiResidX: x
   long long ld_resid;
@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const GemmF32Params p) {
       const int col = n0 + tx * 4 + j;
       if (col >= p.N) continue;
       const float v = acc[i][j];
-      if (p.epi == kEpiStoreBf16) {
+      if (p.epi == kEpiStoreF16) {
         p.out[row * p.ld_out + col] = v;
       } else if (p.epi == kEpiGeluBias) {
         const float z = v + p.bias[col];

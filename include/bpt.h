@@ -52,12 +52,14 @@ typedef enum {
   BPT_ERR_UNSUPPORTED = 2, /* valid layer the kernels do not handle (see below) */
   BPT_ERR_WORKSPACE = 3,   /* workspace smaller than bpt_layer_workspace_size */
   BPT_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed */
-  BPT_ERR_TIMEOUT = 5      /* a kernel gave up waiting (device error word) */
+  BPT_ERR_TIMEOUT = 5,     /* a kernel gave up waiting (device error word) */
+  BPT_ERR_RANGE = 6        /* an fp16 tensor-core operand overflowed (device error word) */
 } bpt_status;
 
 typedef enum {
   BPT_F32 = 0,  /* x, weights, params fp32; fp32 arithmetic on CUDA cores */
-  BPT_BF16 = 1  /* x, weights, params bf16; tensor cores, fp32 accumulate */
+  BPT_BF16 = 1  /* x, weights, params bf16; tensor cores with fp16 operands
+                   (see below), fp32 accumulation */
 } bpt_dtype;
 
 /* Same object as cudaStream_t; 0 is the legacy default stream. */
@@ -71,9 +73,13 @@ typedef struct CUstream_st* bpt_stream_t;
  *
  * Pure host arithmetic.  Layout (each region 1024-byte aligned):
  *   [0, 256)       header; uint32 at offset 0 = device error word
- *   QKV            [B*N, 3d] of dtype (Q | K | V per row)
- *   block scratch  P*b rows of o [d], LN2(y) [d] and FFN hidden [d_ff], dtype,
- *                  P = blocks in the largest wave (<= BPT_WAVE_BLOCKS)
+ *   weights        BPT_BF16 only: fp16 copies of W_Q, W_K, W_V, W_O ([d, d]
+ *                  each), W_1 [d, d_ff], W_2 [d_ff, d], in that order
+ *   QKV            [B*N, 3d] (Q | K | V per row); fp16 for BPT_BF16, fp32
+ *                  for BPT_F32 (the "operand type" below)
+ *   block scratch  P*b rows of o [d], LN2(y) [d] and FFN hidden [d_ff], in
+ *                  the operand type, P = blocks in the largest wave
+ *                  (<= BPT_WAVE_BLOCKS)
  * The scratch term does not grow with N once B*ceil(N/b) >= BPT_WAVE_BLOCKS.
  * Returns BPT_ERR_INVALID_ARG for bytes == NULL or negative / inconsistent
  * sizes, BPT_ERR_UNSUPPORTED for shapes bpt_layer_forward rejects.
@@ -103,6 +109,15 @@ bpt_status bpt_layer_workspace_size(int64_t B, int64_t N, int64_t d, int64_t h, 
  *   B * N <= 2^30 tokens.
  * B == 0 or N == 0: nothing to do, returns BPT_OK without touching memory.
  * Results are deterministic: the same inputs give bitwise the same `out`.
+ *
+ * Precision of BPT_BF16: the tensor cores take fp16 operands (same rate as
+ * bf16, 3 more mantissa bits).  Each call first copies the six bf16 weight
+ * matrices to fp16 in the workspace; the copy is exact for magnitudes in
+ * [2^-14, 65504] and has absolute error <= 2^-25 below.  LN outputs, Q/K/V,
+ * the softmax weights P, the attention output and the FFN hidden state are
+ * rounded to fp16; every product is accumulated in fp32; the residual stream
+ * y and the output Z stay fp32.  A weight or an fp16 intermediate beyond
+ * +-65504 (or NaN) sets BPT_ERR_RANGE in the device error word.
  */
 bpt_status bpt_layer_forward(const void* x, const void* ln1, const void* W_Q, const void* W_K,
                              const void* W_V, const void* W_O, const void* ln2, const void* W_1,
@@ -113,9 +128,11 @@ bpt_status bpt_layer_forward(const void* x, const void* ln1, const void* W_Q, co
 
 /*
  * bpt_read_device_error -- synchronises `stream`, reads and clears the error
- * word in the workspace header.  Returns BPT_OK if no kernel gave up,
- * BPT_ERR_TIMEOUT if one did (*site, if non-NULL, receives the code of the
- * wait that ran out), BPT_ERR_CUDA if synchronisation failed.
+ * word in the workspace header (written by the latest bpt_layer_forward on
+ * this workspace).  Returns BPT_OK if nothing was recorded, BPT_ERR_TIMEOUT if
+ * a kernel gave up waiting, BPT_ERR_RANGE if an fp16 operand overflowed
+ * (*site, if non-NULL, receives the code of the place that recorded it), or
+ * BPT_ERR_CUDA if synchronisation failed.
  */
 bpt_status bpt_read_device_error(void* workspace, bpt_stream_t stream, uint32_t* site);
 
@@ -138,7 +155,8 @@ enum {
   BPT_KIND_LN2 = 4,
   BPT_KIND_W1 = 5,
   BPT_KIND_W2 = 6,
-  BPT_KIND_COUNT = 7
+  BPT_KIND_CVT = 7, /* bf16 -> fp16 weight copy */
+  BPT_KIND_COUNT = 8
 };
 bpt_status bpt_profile_enable(int enable);
 bpt_status bpt_profile_read(double* ms, int64_t* launches, int n);

@@ -2,6 +2,9 @@
 and compare with the fp64 oracle."""
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -34,6 +37,12 @@ def compare(got: np.ndarray, want: np.ndarray, tol):
     assert np.all(np.isfinite(got)), "non-finite values in the CUDA result"
     mx, mean = float(err.max()), float(err.mean())
     msg = f"max abs {mx:.3e} (tol {tol[0]}), mean abs {mean:.3e} (tol {tol[1]})"
+    log = os.environ.get("BPT_PARITY_LOG")
+    if log:
+        with open(log, "a") as f:
+            f.write(json.dumps({"test": os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0],
+                                "n": int(err.size), "max_abs": mx, "mean_abs": mean,
+                                "tol": list(tol)}) + "\n")
     assert mx <= tol[0], msg
     if tol[1] is not None:
         assert mean <= tol[1], msg
@@ -41,11 +50,17 @@ def compare(got: np.ndarray, want: np.ndarray, tol):
 
 
 def workspace_qkv(ws: torch.Tensor, cfg: LayerShape, B: int) -> np.ndarray:
-    """The QKV projection the library leaves in its workspace ([B*N, 3d])."""
+    """The QKV projection the library leaves in its workspace ([B*N, 3d]).
+
+    Layout (include/bpt.h): 1024-byte header region, then for bf16 layers the
+    fp16 weight copies, then QKV in the operand type (fp16 / fp32).
+    """
     off = 1024
     n = B * cfg.N * 3 * cfg.d
     if cfg.dtype == "bf16":
-        t = ws[off:off + 2 * n].view(torch.bfloat16)
+        w16 = (4 * cfg.d * cfg.d + 2 * cfg.d * cfg.d_ff) * 2
+        off += (w16 + 1023) // 1024 * 1024
+        t = ws[off:off + 2 * n].view(torch.float16)
     else:
         t = ws[off:off + 4 * n].view(torch.float32)
     return t.float().cpu().numpy().reshape(B, cfg.N, 3 * cfg.d)

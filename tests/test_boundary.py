@@ -38,7 +38,7 @@ def test_every_declared_function_is_exported(lib):
 
 
 def test_status_strings():
-    for s in range(6):
+    for s in range(7):
         assert bpt.status_string(s).startswith("BPT_")
     assert "UNKNOWN" in bpt.status_string(99)
 
@@ -74,11 +74,12 @@ def test_workspace_is_block_shaped():
     """Beyond the QKV projection (3 B N d elements) the workspace does not grow
     with N once a wave is full, and never exceeds that bound."""
     d, h, d_ff = 2048, 16, 8192
+    weights = (4 * d * d + 2 * d * d_ff) * 2
     extra = []
     for N in (8192, 16384, 32768, 65536, 131072):
         st, nbytes = bpt.bpt_layer_workspace_size(1, N, d, h, d_ff, 1, BF)
         assert st == bpt.BPT_OK
-        extra.append(nbytes - 3 * N * d * 2)
+        extra.append(nbytes - 3 * N * d * 2 - weights)
     full = extra[2:]
     assert max(full) - min(full) <= 2048           # alignment slack only
     assert all(e <= max(full) for e in extra)
@@ -88,9 +89,11 @@ def test_workspace_is_block_shaped():
 
 def test_launch_count():
     st, n = bpt.bpt_layer_launch_count(1, 65536, 2048, 16, 8192, 1, BF)
-    assert st == bpt.BPT_OK and n == 2 + 5 * 2   # two waves of 256 blocks
+    assert st == bpt.BPT_OK and n == 3 + 5 * 2   # weight copy, LN1, QKV; two waves
     st, n = bpt.bpt_layer_launch_count(8, 2048, 768, 12, 3072, 1, BF)
-    assert st == bpt.BPT_OK and n == 2 + 5      # one wave of 8 sequences
+    assert st == bpt.BPT_OK and n == 3 + 5      # one wave of 8 sequences
+    st, n = bpt.bpt_layer_launch_count(1, 256, 64, 1, 256, 0, F32)
+    assert st == bpt.BPT_OK and n == 2 + 5      # fp32: no weight copy
     st, n = bpt.bpt_layer_launch_count(0, 2048, 768, 12, 3072, 1, BF)
     assert st == bpt.BPT_OK and n == 0
 
