@@ -174,9 +174,8 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    from blockwise_attn_ffn_b200 import dist as bdist
+    rank, local_rank, world = bdist.env_rank()
     cfg = WORKLOADS[args.workload]
     if args.seq_len:
         cfg = cfg.with_(N=args.seq_len, name=f"{cfg.name}@N={args.seq_len}")
@@ -193,22 +192,10 @@ def main():
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+        bdist.init_process_group("nccl", device=dev)
 
-    # Inputs: the workload's weights on every rank; rank r's x is the
-    # workload's draw for r = 0 and a rank-seeded draw otherwise.
-    inp = make_inputs(cfg)
-    if rank > 0:
-        rng = np.random.default_rng([cfg.seed, rank])
-        x32 = rng.standard_normal(size=inp["x"].shape, dtype=np.float32)
-        from blockwise_attn_ffn_b200.inputs import bf16_bits_to_f32, f32_to_bf16_bits
-        if cfg.dtype == "bf16":
-            inp["x_bits"] = f32_to_bf16_bits(x32)
-            inp["x"] = bf16_bits_to_f32(inp["x_bits"])
-        else:
-            inp["x"] = x32
+    # Inputs: the workload's weights on every rank, a rank-seeded x each.
+    inp = bdist.rank_inputs(cfg, rank)
     torch.cuda.reset_peak_memory_stats(dev)
     base_mem = torch.cuda.memory_allocated(dev)
     p = bpt.to_device(inp, cfg.dtype, dev)
@@ -254,13 +241,10 @@ def main():
     st, site = bpt.bpt_read_device_error(ws.data_ptr(), stream.cuda_stream)
     if st != bpt.BPT_OK:
         raise SystemExit(f"device error {bpt.status_string(st)} site {site}")
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = bdist.max_over_ranks(ms_total, dist, dev)
     ms_step = ms_total / args.steps
     tokens_step = cfg.B * cfg.N * world
-    value = tokens_step / (ms_step / 1e3)
+    value = bdist.weak_scaling_tokens_per_s(cfg, world, ms_step)
 
     # -------- end to end: pinned x -> device, forward, out -> pinned host
     e2e = None
@@ -282,11 +266,7 @@ def main():
             out_host.copy_(out, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        ms_e2e = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
+        ms_e2e = bdist.max_over_ranks(e0.elapsed_time(e1), dist, dev)
         e2e = {"value": tokens_step / (ms_e2e / args.steps / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": int(x.numel() * x.element_size()),
                "d2h_bytes_per_step": int(out.numel() * out.element_size()),

@@ -25,7 +25,7 @@ BPT_STATIC_WORKSPACE_BYTES = 64 * 1024 * 1024
 EXPORTED = [
     "bpt_layer_workspace_size", "bpt_layer_forward", "bpt_read_device_error",
     "bpt_status_string", "bpt_profile_enable", "bpt_profile_read",
-    "bpt_layer_launch_count", "bpt_layer_forward_static",
+    "bpt_layer_launch_count", "bpt_layer_forward_static", "bpt_debug_inject_fault",
 ]
 
 _lib: Optional[ctypes.CDLL] = None
@@ -66,6 +66,8 @@ def load() -> ctypes.CDLL:
     lib.bpt_layer_launch_count.restype = i32
     lib.bpt_layer_forward_static.argtypes = [vp] * 11 + [i64] * 5 + [i32, i32, vp, vp]
     lib.bpt_layer_forward_static.restype = i32
+    lib.bpt_debug_inject_fault.argtypes = [i32]
+    lib.bpt_debug_inject_fault.restype = i32
     _lib = lib
     return lib
 
@@ -126,6 +128,12 @@ def bpt_layer_forward_static(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2
     return load().bpt_layer_forward_static(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
                                            B, N, d, h, d_ff, int(bool(causal)), dtype, out,
                                            stream)
+
+
+def bpt_debug_inject_fault(code: int) -> int:
+    """Test hook: the next bf16 forward loses one TMA load (1: QKV GEMM,
+    2: attention) so a bounded wait runs out and reports BPT_ERR_TIMEOUT."""
+    return load().bpt_debug_inject_fault(int(code))
 
 
 def bpt_layer_launch_count(B, N, d, h, d_ff, causal, dtype) -> Tuple[int, int]:

@@ -58,6 +58,7 @@ struct AttnPairParams {
   __half* o;         // [count * 128, d] block scratch (fp16)
   float scale_log2;  // log2(e) / sqrt(d_k)
   uint32_t* err;
+  int fault;         // test hook: 2 = CTA 0 never loads V_0 (a lost arrive)
 };
 
 // Coefficients of 2^f ~ c0 + c1 f + c2 f^2 + c3 f^3 on [0, 1): relative-error
@@ -239,13 +240,16 @@ __global__ void __launch_bounds__(384, 1)
           break;
         }
         const uint32_t fb = ring_full0 + 8 * slot;
-        mbar_arrive_expect_tx(fb, C::TILE);
-        armed[slot] = static_cast<int>(phase);
-        const int col = w == 0 ? colK : colV;
+        const bool lost = p.fault == 2 && blockIdx.x == 0 && j == 0 && w == 1;
+        if (!lost) {
+          mbar_arrive_expect_tx(fb, C::TILE);
+          armed[slot] = static_cast<int>(phase);
+          const int col = w == 0 ? colK : colV;
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem_u32(smem + C::OFF_RING + slot * C::TILE + c * C::CHUNK), &mapQKV, fb,
-                      col + 64 * c, j * C::BKV, bidx);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(smem_u32(smem + C::OFF_RING + slot * C::TILE + c * C::CHUNK), &mapQKV, fb,
+                        col + 64 * c, j * C::BKV, bidx);
+        }
         if (++slot == C::NSLOT) {
           slot = 0;
           phase ^= 1u;

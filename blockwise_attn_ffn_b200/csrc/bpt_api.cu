@@ -251,6 +251,7 @@ struct ProfRec {
   cudaEvent_t a, b;
 };
 bool g_prof_on = false;
+int g_fault = 0;  // test hook, consumed by the next bf16 forward
 std::vector<ProfRec> g_prof;
 std::vector<cudaEvent_t> g_event_pool;
 
@@ -329,6 +330,12 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
   using bf = __nv_bfloat16;
   using hf = __half;
   const int64_t M = P.B * P.N, d = P.d, d_ff = P.d_ff;
+  int fault = 0;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    fault = g_fault;
+    g_fault = 0;
+  }
   uint32_t* err = reinterpret_cast<uint32_t*>(ws);
   // Tensor-core operands are fp16: the bf16 weights are copied to fp16 once
   // per call (exact in the fp16 normal range), activations are stored fp16.
@@ -386,6 +393,7 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
     g.out_h = qkv; g.ld_out = 3 * d;
     g.map = ident;
     g.err = err;
+    g.fault = fault == 1 ? 1 : 0;
     LaunchScope ls(BPT_KIND_QKV, s);
     if (launch_gemm(mXn, mWq, mWk, mWv, g, sms, s) != cudaSuccess) return BPT_ERR_CUDA;
   }
@@ -399,6 +407,7 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
       ap.N = int(P.N); ap.nb = int(P.nb); ap.h = int(P.h); ap.d = int(d);
       ap.causal = P.causal; ap.item0 = int(wv_.item0); ap.count = int(wv_.count);
       ap.seqs = int(wv_.seqs); ap.o = so; ap.scale_log2 = scale_log2; ap.err = err;
+      ap.fault = (fault == 2 && w == 0) ? 2 : 0;
       const int64_t pairs = wv_.seqs == 0 ? (wv_.count + 1) / 2 : wv_.seqs * ((P.nb + 1) / 2);
       const unsigned grid = unsigned(pairs * P.h);
       LaunchScope ls(BPT_KIND_ATTN, s);
@@ -608,6 +617,13 @@ const char* bpt_status_string(bpt_status status) {
     case BPT_ERR_RANGE: return "BPT_ERR_RANGE: a tensor-core operand exceeded the fp16 range";
   }
   return "BPT_UNKNOWN_STATUS";
+}
+
+bpt_status bpt_debug_inject_fault(int code) {
+  if (code < 0 || code > 2) return BPT_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_fault = code;
+  return BPT_OK;
 }
 
 bpt_status bpt_profile_enable(int enable) {

@@ -43,6 +43,7 @@ struct GemmParams {
   const __nv_bfloat16* bias;
   RowMap map;
   uint32_t* err;
+  int fault;  // test hook: 1 = CTA 0 never loads its first stage (a lost arrive)
 };
 
 constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 64, kGemmStages = 4;
@@ -135,17 +136,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           break;
         }
         const uint32_t fb = full0 + 8 * stage;
-        mbar_arrive_expect_tx(fb, kGemmStageBytes);
-        armed[stage] = static_cast<int>(phase);
-        tma_load_2d(smem_u32(sA + stage * kGemmABytes), &mapA, fb, kb * kGemmBK, mb * kGemmBM);
+        const bool lost = p.fault == 1 && blockIdx.x == 0 && tile == blockIdx.x && kb == 0;
+        if (!lost) {
+          mbar_arrive_expect_tx(fb, kGemmStageBytes);
+          armed[stage] = static_cast<int>(phase);
+          tma_load_2d(smem_u32(sA + stage * kGemmABytes), &mapA, fb, kb * kGemmBK, mb * kGemmBM);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int c = nb * kGemmBN + q * 64;
-          int which = c / p.n_sub;
-          if (which > p.n_maps - 1) which = p.n_maps - 1;  // past the end: TMA zero-fills
-          const CUtensorMap* mB = which == 0 ? &mapB0 : (which == 1 ? &mapB1 : &mapB2);
-          tma_load_2d(smem_u32(sB + stage * kGemmBBytes + q * 8192), mB, fb, c - which * p.n_sub,
-                      kb * kGemmBK);
+          for (int q = 0; q < 4; ++q) {
+            const int c = nb * kGemmBN + q * 64;
+            int which = c / p.n_sub;
+            if (which > p.n_maps - 1) which = p.n_maps - 1;  // past the end: TMA zero-fills
+            const CUtensorMap* mB = which == 0 ? &mapB0 : (which == 1 ? &mapB1 : &mapB2);
+            tma_load_2d(smem_u32(sB + stage * kGemmBBytes + q * 8192), mB, fb, c - which * p.n_sub,
+                        kb * kGemmBK);
+          }
         }
         if (++stage == kGemmStages) {
           stage = 0;

@@ -161,6 +161,20 @@ enum {
 bpt_status bpt_profile_enable(int enable);
 bpt_status bpt_profile_read(double* ms, int64_t* launches, int n);
 
+/*
+ * bpt_debug_inject_fault -- TEST HOOK for the failure-detection path.  The
+ * next BPT_BF16 bpt_layer_forward makes one CTA skip one TMA load, so that
+ * the wait for it runs out (after about 2 s) instead of completing:
+ *   code 1: the QKV GEMM's CTA 0 never loads its first stage;
+ *   code 2: the first attention wave's CTA 0 never loads V_0.
+ * The kernel then records BPT_ERR_TIMEOUT in the device error word, drains
+ * the loads and tensor-core work it did issue, frees its tensor memory and
+ * exits; the layer's output is garbage for that call and the context stays
+ * usable.  code 0 cancels.  The hook is consumed by one forward call.
+ * Returns BPT_ERR_INVALID_ARG for other codes.
+ */
+bpt_status bpt_debug_inject_fault(int code);
+
 /* Kernel launches one bpt_layer_forward call makes for these sizes. */
 bpt_status bpt_layer_launch_count(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff,
                                   int causal, bpt_dtype dtype, int64_t* launches);
