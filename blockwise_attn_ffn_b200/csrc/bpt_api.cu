@@ -148,15 +148,22 @@ Plan make_plan(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff, int cau
 }
 
 // ------------------------------------------------------------ device info --
+// GEMM kernel: CTA pairs (cta_group::2, 256x256 tiles) unless built with
+// -DBPT_GEMM_PAIR=0 (one CTA per 128x256 tile).
+#ifndef BPT_GEMM_PAIR
+#define BPT_GEMM_PAIR 1
+#endif
+
 struct DeviceInfo {
   bool init = false;
   bool ok = false;
   int sms = 0;
+  int pair_clusters = 0;  // co-resident CTA pairs of the pair GEMM
 };
 std::mutex g_mu;
 DeviceInfo g_dev[64];
 
-bpt_status device_info(int* sms) {
+bpt_status device_info(int* sms, int* pair_clusters = nullptr) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BPT_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_mu);
@@ -179,14 +186,31 @@ bpt_status device_info(int* sms) {
           cudaFuncSetAttribute(bpt::attn_pair_tc_kernel<128, kEmu128>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                bpt::AttnPairCfg<128, kEmu128>::SMEM) != cudaSuccess ||
+          cudaFuncSetAttribute(bpt::gemm_f16_pair_kernel,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               bpt::kPairSmem) != cudaSuccess ||
           cudaFuncSetAttribute(bpt::attn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (3 * 64 * 128 + 64 * 65) * 4) != cudaSuccess)
         return BPT_ERR_CUDA;
+      // How many CTA pairs of the pair GEMM fit on the device at once.
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(unsigned(2 * (n / 2)));
+      cfg.blockDim = dim3(bpt::kGemmThreads);
+      cfg.dynamicSmemBytes = bpt::kPairSmem;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, bpt::gemm_f16_pair_kernel, &cfg) !=
+              cudaSuccess ||
+          clusters <= 0) {
+        cudaGetLastError();
+        clusters = n / 2;
+      }
+      di.pair_clusters = clusters;
     }
     di.init = true;
   }
   if (!di.ok) return BPT_ERR_UNSUPPORTED;
   *sms = di.sms;
+  if (pair_clusters) *pair_clusters = di.pair_clusters;
   return BPT_OK;
 }
 
@@ -314,10 +338,20 @@ cudaError_t launch_ln(const TIn* in, const TP* ln, TOut* out, int64_t rows, int6
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                         const CUtensorMap& b2, const bpt::GemmParams& gp, int sms,
                         cudaStream_t s) {
+#if BPT_GEMM_PAIR
+  int dummy = 0, pairs_max = 0;
+  if (device_info(&dummy, &pairs_max) != BPT_OK) return cudaErrorInvalidDevice;
+  const int64_t tiles = int64_t((gp.M + bpt::kPairBM - 1) / bpt::kPairBM) *
+                        int64_t((gp.N + bpt::kGemmBN - 1) / bpt::kGemmBN);
+  const unsigned pairs = unsigned(std::max<int64_t>(1, std::min<int64_t>(tiles, pairs_max)));
+  bpt::gemm_f16_pair_kernel<<<2 * pairs, bpt::kGemmThreads, bpt::kPairSmem, s>>>(a, b0, b1, b2,
+                                                                                 gp);
+#else
   const int64_t tiles = int64_t((gp.M + bpt::kGemmBM - 1) / bpt::kGemmBM) *
                         int64_t((gp.N + bpt::kGemmBN - 1) / bpt::kGemmBN);
   const unsigned grid = unsigned(std::min<int64_t>(tiles, sms));
   bpt::gemm_f16_tc_kernel<<<grid, bpt::kGemmThreads, bpt::kGemmSmem, s>>>(a, b0, b1, b2, gp);
+#endif
   return cudaGetLastError();
 }
 

@@ -67,6 +67,89 @@ __device__ __forceinline__ void gemm_tile_coords(int tile, int m_blocks, int n_b
   nb = in / gm;
 }
 
+// Epilogue of one accumulator row (this thread's TMEM lane): 256 columns
+// starting at global column col_base, read in 32-column chunks.  Every lane of
+// the warp must call it (tcgen05.ld is warp-collective).
+__device__ __forceinline__ void gemm_epilogue_row(const GemmParams& p, uint32_t t_row,
+                                                  long long row, int col_base) {
+  long long g = -1;
+  bool row_ok;
+  if (p.epi == kEpiStoreF16 || p.epi == kEpiGeluBias) {
+    row_ok = row < p.M;
+  } else {
+    g = row < p.M ? p.map.map(row) : -1;
+    row_ok = g >= 0;
+  }
+  bool bad = false;
+#pragma unroll 1
+  for (int ch = 0; ch < kGemmBN / 32; ++ch) {
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(t_row + ch * 32, r);
+    tmem_ld_wait();
+    const int col0 = col_base + ch * 32;
+    if (!row_ok || col0 >= p.N) continue;
+    float v[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
+    if (p.epi == kEpiStoreF16 || p.epi == kEpiGeluBias) {
+      if (p.epi == kEpiGeluBias) {
+        const uint4* bp = reinterpret_cast<const uint4*>(p.bias + col0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 bb = __ldg(bp + q);
+          const __nv_bfloat16* bh = reinterpret_cast<const __nv_bfloat16*>(&bb);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) v[q * 8 + k] = gelu_erf(v[q * 8 + k] + __bfloat162float(bh[k]));
+        }
+      }
+      uint4* dst = reinterpret_cast<uint4*>(p.out_h + row * p.ld_out + col0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 w;
+        w.x = pack_f16x2(v[q * 8 + 0], v[q * 8 + 1], bad);
+        w.y = pack_f16x2(v[q * 8 + 2], v[q * 8 + 3], bad);
+        w.z = pack_f16x2(v[q * 8 + 4], v[q * 8 + 5], bad);
+        w.w = pack_f16x2(v[q * 8 + 6], v[q * 8 + 7], bad);
+        dst[q] = w;
+      }
+    } else {
+      float4* dst = reinterpret_cast<float4*>(p.out_f32 + g * p.ld_f32 + col0);
+      if (p.epi == kEpiResidX) {
+        const uint4* xp = reinterpret_cast<const uint4*>(p.resid + g * p.ld_resid + col0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 xx = __ldg(xp + q);
+          const __nv_bfloat16* xh = reinterpret_cast<const __nv_bfloat16*>(&xx);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) v[q * 8 + k] += __bfloat162float(xh[k]);
+        }
+      } else {
+        const uint4* bp = reinterpret_cast<const uint4*>(p.bias + col0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 bb = __ldg(bp + q);
+          const __nv_bfloat16* bh = reinterpret_cast<const __nv_bfloat16*>(&bb);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) v[q * 8 + k] += __bfloat162float(bh[k]);
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 y = dst[q];
+          v[q * 4 + 0] += y.x;
+          v[q * 4 + 1] += y.y;
+          v[q * 4 + 2] += y.z;
+          v[q * 4 + 3] += y.w;
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        dst[q] = make_float4(v[q * 4 + 0], v[q * 4 + 1], v[q * 4 + 2], v[q * 4 + 3]);
+    }
+  }
+  if (bad)
+    record_error(p.err, kErrRange, p.epi == kEpiGeluBias ? kSiteRangeHidden : kSiteRangeQKV);
+}
+
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_f16_tc_kernel(const __grid_constant__ CUtensorMap mapA,
                         const __grid_constant__ CUtensorMap mapB0,
@@ -213,85 +296,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!mbar_wait(accf0 + 8 * acc, acc_phase, abort_flag, p.err, kSiteGemmEpilogue)) break;
       tc_fence_after();
       const long long row = static_cast<long long>(mb) * kGemmBM + e * 32 + lane;
-      long long g = -1;
-      bool row_ok;
-      if (p.epi == kEpiStoreF16 || p.epi == kEpiGeluBias) {
-        row_ok = row < p.M;
-      } else {
-        g = row < p.M ? p.map.map(row) : -1;
-        row_ok = g >= 0;
-      }
       const uint32_t t_row = tmem + (static_cast<uint32_t>(e * 32) << 16) +
                              static_cast<uint32_t>(acc * kGemmBN);
-#pragma unroll 1
-      for (int ch = 0; ch < kGemmBN / 32; ++ch) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(t_row + ch * 32, r);
-        tmem_ld_wait();
-        const int col0 = nb * kGemmBN + ch * 32;
-        if (!row_ok || col0 >= p.N) continue;
-        float v[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
-        if (p.epi == kEpiStoreF16 || p.epi == kEpiGeluBias) {
-          if (p.epi == kEpiGeluBias) {
-            const uint4* bp = reinterpret_cast<const uint4*>(p.bias + col0);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 bb = __ldg(bp + q);
-              const __nv_bfloat16* bh = reinterpret_cast<const __nv_bfloat16*>(&bb);
-#pragma unroll
-              for (int k = 0; k < 8; ++k) v[q * 8 + k] = gelu_erf(v[q * 8 + k] + __bfloat162float(bh[k]));
-            }
-          }
-          uint4* dst = reinterpret_cast<uint4*>(p.out_h + row * p.ld_out + col0);
-          bool bad = false;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint4 w;
-            w.x = pack_f16x2(v[q * 8 + 0], v[q * 8 + 1], bad);
-            w.y = pack_f16x2(v[q * 8 + 2], v[q * 8 + 3], bad);
-            w.z = pack_f16x2(v[q * 8 + 4], v[q * 8 + 5], bad);
-            w.w = pack_f16x2(v[q * 8 + 6], v[q * 8 + 7], bad);
-            dst[q] = w;
-          }
-          if (bad)
-            record_error(p.err, kErrRange,
-                         p.epi == kEpiGeluBias ? kSiteRangeHidden : kSiteRangeQKV);
-        } else {
-          float4* dst = reinterpret_cast<float4*>(p.out_f32 + g * p.ld_f32 + col0);
-          if (p.epi == kEpiResidX) {
-            const uint4* xp = reinterpret_cast<const uint4*>(p.resid + g * p.ld_resid + col0);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 xx = __ldg(xp + q);
-              const __nv_bfloat16* xh = reinterpret_cast<const __nv_bfloat16*>(&xx);
-#pragma unroll
-              for (int k = 0; k < 8; ++k) v[q * 8 + k] += __bfloat162float(xh[k]);
-            }
-          } else {
-            const uint4* bp = reinterpret_cast<const uint4*>(p.bias + col0);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 bb = __ldg(bp + q);
-              const __nv_bfloat16* bh = reinterpret_cast<const __nv_bfloat16*>(&bb);
-#pragma unroll
-              for (int k = 0; k < 8; ++k) v[q * 8 + k] += __bfloat162float(bh[k]);
-            }
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const float4 y = dst[q];
-              v[q * 4 + 0] += y.x;
-              v[q * 4 + 1] += y.y;
-              v[q * 4 + 2] += y.z;
-              v[q * 4 + 3] += y.w;
-            }
-          }
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            dst[q] = make_float4(v[q * 4 + 0], v[q * 4 + 1], v[q * 4 + 2], v[q * 4 + 3]);
-        }
-      }
+      gemm_epilogue_row(p, t_row, row, nb * kGemmBN);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acce0 + 8 * acc);
@@ -306,6 +313,222 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 2) tmem_dealloc(tmem, kGemmTmemCols);
+}
+
+// ---------------------------------------------------------------------------
+// CTA-pair variant: a cluster of two CTAs on two SMs computes one 256 x 256
+// output tile with tcgen05.mma.cta_group::2 (M = 256).  Each CTA loads its own
+// 128 rows of A and its half (128 columns) of the 256-column B slab, so per SM
+// a 64-deep k-block is 32 KB of shared memory instead of 48 KB: six stages
+// fit, and B traffic per SM halves.  Each CTA's tensor memory holds its own
+// 128 accumulator rows (two 256-column buffers), read by its own epilogue.
+//
+// Protocol (CTA rank 0 = leader, rank 1 = peer):
+//   full[s]   leader only; the leader's producer arms it with the bytes of
+//             both CTAs; both CTAs' TMA loads complete on it.
+//   empty[s]  both CTAs; the leader's UMMA commit arrives on both (multicast).
+//   accf[b]   both CTAs; the leader's UMMA commit arrives on both (multicast).
+//   acce[b]   leader only, 8 arrivals: the four epilogue warps of each CTA.
+// No TMA load uses cluster multicast.  The pair starts and ends with a
+// cluster barrier, so neither CTA frees memory the other may still signal.
+constexpr int kPairStages = 6;
+constexpr int kPairABytes = 128 * kGemmBK * 2;  // 16 KB: this CTA's 128 rows
+constexpr int kPairBBytes = kGemmBK * 128 * 2;  // 16 KB: this CTA's 128 columns
+constexpr int kPairStageBytes = kPairABytes + kPairBBytes;
+constexpr int kPairSmem = kPairStages * kPairStageBytes + kGemmBarrierBytes + 1024;
+constexpr int kPairBM = 256;
+constexpr int kPairGroupM = 8;  // 256-row blocks per rasterisation group
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm_f16_pair_kernel(const __grid_constant__ CUtensorMap mapA,
+                         const __grid_constant__ CUtensorMap mapB0,
+                         const __grid_constant__ CUtensorMap mapB1,
+                         const __grid_constant__ CUtensorMap mapB2, const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kPairStages * kPairABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kPairStages * kPairStageBytes);
+  const uint32_t full0 = smem_u32(bars + 0);
+  const uint32_t empty0 = smem_u32(bars + kPairStages);
+  const uint32_t accf0 = smem_u32(bars + 2 * kPairStages);
+  const uint32_t acce0 = smem_u32(bars + 2 * kPairStages + 2);
+  const uint32_t drain = smem_u32(bars + 2 * kPairStages + 4);
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = static_cast<int>(cluster_id_x());
+  const int npairs = static_cast<int>(nclusters_x());
+  const int m_blocks = (p.M + kPairBM - 1) / kPairBM;
+  const int n_blocks = (p.N + kGemmBN - 1) / kGemmBN;
+  const int k_blocks = p.K / kGemmBK;
+  const int tiles = m_blocks * n_blocks;
+
+  if (threadIdx.x == 0) {
+    for (int s2 = 0; s2 < kPairStages; ++s2) {
+      mbar_init(full0 + 8 * s2, 1);
+      mbar_init(empty0 + 8 * s2, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accf0 + 8 * b, 1);
+      mbar_init(acce0 + 8 * b, 8);
+    }
+    mbar_init(drain, 1);
+    abort_sh = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc_pair(smem_u32(&tmem_base_sh), kGemmTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  volatile int* abort_flag = &abort_sh;
+  bool aborted = false;
+
+  auto coords = [&](int tile, int& mb, int& nb) {
+    const int per_group = kPairGroupM * n_blocks;
+    const int group = tile / per_group;
+    const int first_m = group * kPairGroupM;
+    const int gm = min(kPairGroupM, m_blocks - first_m);
+    const int in = tile - group * per_group;
+    mb = first_m + in % gm;
+    nb = in / gm;
+  };
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    tma_prefetch_desc(&mapA);
+    tma_prefetch_desc(&mapB0);
+    if (p.n_maps > 1) tma_prefetch_desc(&mapB1);
+    if (p.n_maps > 2) tma_prefetch_desc(&mapB2);
+    int armed[kPairStages];
+    for (int s2 = 0; s2 < kPairStages; ++s2) armed[s2] = -1;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = pair; tile < tiles && ok; tile += npairs) {
+      int mb, nb;
+      coords(tile, mb, nb);
+      for (int kb = 0; kb < k_blocks; ++kb) {
+        if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.err, kSiteGemmProducer)) {
+          ok = false;
+          break;
+        }
+        const uint32_t fb_leader = map_to_rank(full0 + 8 * stage, 0);
+        const bool lost = p.fault == 1 && pair == 0 && rank == 0 && tile == pair && kb == 0;
+        if (!lost) {
+          if (rank == 0) {
+            mbar_arrive_expect_tx(full0 + 8 * stage, 2 * kPairStageBytes);
+            armed[stage] = static_cast<int>(phase);
+          }
+          tma_load_2d_pair(smem_u32(sA + stage * kPairABytes), &mapA, fb_leader, kb * kGemmBK,
+                           mb * kPairBM + static_cast<int>(rank) * 128);
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const int c = nb * kGemmBN + static_cast<int>(rank) * 128 + q * 64;
+            int which = c / p.n_sub;
+            if (which > p.n_maps - 1) which = p.n_maps - 1;  // past the end: TMA zero-fills
+            const CUtensorMap* mB = which == 0 ? &mapB0 : (which == 1 ? &mapB1 : &mapB2);
+            tma_load_2d_pair(smem_u32(sB + stage * kPairBBytes + q * 8192), mB, fb_leader,
+                             c - which * p.n_sub, kb * kGemmBK);
+          }
+        }
+        if (++stage == kPairStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    aborted = !ok;
+    // Drain.  The leader waits for every phase it armed (they count the
+    // peer's bytes too).  The peer cannot observe its own loads; after a
+    // normal run the leader consumed them all, after an abort it waits a
+    // bounded 200 us for any still in flight before the final cluster barrier.
+    if (rank == 0) {
+      for (int s2 = 0; s2 < kPairStages; ++s2)
+        if (armed[s2] >= 0)
+          mbar_wait_drain(full0 + 8 * s2, static_cast<uint32_t>(armed[s2]), p.err);
+    } else if (aborted || *abort_flag) {
+      const uint64_t t0 = global_ns();
+      while (global_ns() - t0 < 200000ull) {
+      }
+    }
+  } else if (warp == 1 && lane == 0 && rank == 0) {
+    // ------------------------------------------------ UMMA issue (leader)
+    constexpr uint32_t idesc = idesc_f16_f32(kPairBM, kGemmBN, false, true);
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int tile = pair; tile < tiles && ok; tile += npairs) {
+      if (!mbar_wait(acce0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.err, kSiteGemmMma)) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * kGemmBN);
+      for (int kb = 0; kb < k_blocks; ++kb) {
+        if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, p.err, kSiteGemmMma)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(sA + stage * kPairABytes);
+        const uint32_t b_base = smem_u32(sB + stage * kPairBBytes);
+#pragma unroll
+        for (int k = 0; k < kGemmBK / 16; ++k) {
+          const uint64_t ad = sdesc_sw128(a_base + k * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(b_base + k * 2048, 8192, 1024);
+          umma_f16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+        }
+        umma_commit_pair_mc(empty0 + 8 * stage, 0x3);
+        if (++stage == kPairStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      umma_commit_pair_mc(accf0 + 8 * acc, 0x3);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+    umma_commit_pair(drain);
+    mbar_wait_drain(drain, 0, p.err);
+  } else if (warp >= 4) {
+    // ------------------------------------------- epilogue (both CTAs)
+    const int e = warp - 4;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = pair; tile < tiles; tile += npairs) {
+      int mb, nb;
+      coords(tile, mb, nb);
+      if (!mbar_wait(accf0 + 8 * acc, acc_phase, abort_flag, p.err, kSiteGemmEpilogue)) break;
+      tc_fence_after();
+      const long long row =
+          static_cast<long long>(mb) * kPairBM + static_cast<long long>(rank) * 128 + e * 32 + lane;
+      const uint32_t t_row = tmem + (static_cast<uint32_t>(e * 32) << 16) +
+                             static_cast<uint32_t>(acc * kGemmBN);
+      gemm_epilogue_row(p, t_row, row, nb * kGemmBN);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(map_to_rank(acce0 + 8 * acc, 0));
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc_pair(tmem, kGemmTmemCols);
 }
 
 }  // namespace bpt
