@@ -28,11 +28,12 @@
 // the TMEM that P_X(j) occupies is ordered after PV_X(j) has read it.
 //
 // exp2: most elements use the MUFU ex2 instruction; on blocks with no masked
-// key, EMU_CHUNKS of the four 32-column chunks of each row use a polynomial
-// on the FMA pipe instead (Cody-Waite range reduction 2^x = 2^floor(x) *
-// 2^frac, and a cubic fit of 2^f on [0, 1), relative error < 1e-4, near
-// the fp16 resolution of P), so MUFU and FMA share the work.
-//
+// key, EMU of the eight 16-column groups of each row use a cubic on the FMA
+// pipe instead, so MUFU and FMA share the work: 2^x = 2^n * 2^f with
+// n = round(x) (the 1.5 * 2^23 addition trick, no conversion instruction),
+// f = x - n in [-1/2, 1/2], 2^f from a fitted cubic (relative error 7.5e-5,
+// below the fp16 resolution of P), and n added to the exponent field.
+
 // Shared memory: Q_A, Q_B and a ring of NSLOT K/V tiles (loaded K_0, V_0,
 // K_1, V_1, ...), all 128 rows x d_k fp16 in 64-column chunks with the
 // 128-byte swizzle.  Tensor memory: S_A 0..127, S_B 128..255, O_A 256..,
@@ -61,15 +62,15 @@ struct AttnPairParams {
   int fault;         // test hook: 2 = CTA 0 never loads V_0 (a lost arrive)
 };
 
-// Coefficients of 2^f ~ c0 + c1 f + c2 f^2 + c3 f^3 on [0, 1): relative-error
-// fit at Chebyshev nodes refined towards equal ripple (printed by
-// csrc/fit_exp2_poly.py), max relative error 7.5e-5.
-constexpr float kExp2C0 = 0.9999252f;
-constexpr float kExp2C1 = 0.69583344f;
-constexpr float kExp2C2 = 0.22606751f;
-constexpr float kExp2C3 = 0.07802427f;
+// Coefficients of 2^f ~ c0 + c1 f + c2 f^2 + c3 f^3 on [-1/2, 1/2]:
+// relative-error fit at Chebyshev nodes refined towards equal ripple (printed
+// by csrc/fit_exp2_poly.py), max relative error 7.5e-5.
+constexpr float kExp2C0 = 0.99992806f;
+constexpr float kExp2C1 = 0.693261f;
+constexpr float kExp2C2 = 0.24261111f;
+constexpr float kExp2C3 = 0.05517149f;
 
-template <int D, int EMU_CHUNKS>
+template <int D, int EMU>
 struct AttnPairCfg {
   static constexpr int BQ = 128;
   static constexpr int BKV = 128;
@@ -112,30 +113,34 @@ __device__ __forceinline__ void attn_pair_decode(const AttnPairParams& p, int ra
   }
 }
 
-// x is clamped at -125 so that the cubic (>= c0, just under 1, exponent field
-// 126) plus floor(x) keeps a positive exponent field: results stay normal
-// floats down to 2^-125, which fp16 P (smallest subnormal 2^-24) rounds to zero.
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.0f);
-  const float xi = floorf(x);
-  const float f = x - xi;
-  float q = fmaf(kExp2C3, f, kExp2C2);
-  q = fmaf(q, f, kExp2C1);
-  q = fmaf(q, f, kExp2C0);
-  return __int_as_float(__float_as_int(q) + (static_cast<int>(xi) << 23));
-}
-
-// Two lanes at once on the packed fp32x2 FMA pipe.
+// 2^x for two lanes on the FMA / ALU pipes.  x is clamped at -125 so that
+// n + (exponent field of 2^f >= 126) stays >= 1: results stay normal floats
+// down to 2^-125, which fp16 P rounds to zero anyway.
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  const float2 magic = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
   x.x = fmaxf(x.x, -125.0f);
   x.y = fmaxf(x.y, -125.0f);
-  const float2 xi = make_float2(floorf(x.x), floorf(x.y));
-  const float2 f = __fadd2_rn(x, make_float2(-xi.x, -xi.y));
+  const float2 j = __fadd2_rn(x, magic);                          // n in the low mantissa bits
+  const float2 n = __fadd2_rn(j, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));
   float2 q = __ffma2_rn(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
   q = __ffma2_rn(q, f, make_float2(kExp2C1, kExp2C1));
   q = __ffma2_rn(q, f, make_float2(kExp2C0, kExp2C0));
-  return make_float2(__int_as_float(__float_as_int(q.x) + (static_cast<int>(xi.x) << 23)),
-                     __int_as_float(__float_as_int(q.y) + (static_cast<int>(xi.y) << 23)));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(j.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(j.y) << 23)));
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 16-column groups (of eight per 128-key row) whose exp2 runs on the FMA
+// pipe, as a bit mask, spread over the row.
+__host__ __device__ constexpr uint32_t emu_group_mask(int emu) {
+  return emu <= 0 ? 0x00u : emu == 1 ? 0x80u : emu == 2 ? 0x88u : emu == 3 ? 0xA8u
+       : emu == 4 ? 0xAAu : emu == 5 ? 0xBAu : emu == 6 ? 0xEEu : emu == 7 ? 0xFEu : 0xFFu;
 }
 
 __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t* r) {
@@ -159,10 +164,10 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
-template <int D, int EMU_CHUNKS>
+template <int D, int EMU>
 __global__ void __launch_bounds__(384, 1)
     attn_pair_tc_kernel(const __grid_constant__ CUtensorMap mapQKV, const AttnPairParams p) {
-  using C = AttnPairCfg<D, EMU_CHUNKS>;
+  using C = AttnPairCfg<D, EMU>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -371,12 +376,16 @@ __global__ void __launch_bounds__(384, 1)
         for (int k = 0; k < C::BKV; ++k)
           if (k >= lim) sr[k] = __float_as_uint(-INFINITY);
       }
-      // Row max as eight independent partial maxima (short dependency chains).
+      // Row max as eight independent partial maxima (short dependency chains),
+      // three-input max.
       float mxp[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) mxp[k] = __uint_as_float(sr[k]);
 #pragma unroll
-      for (int k = 8; k < C::BKV; ++k) mxp[k & 7] = fmaxf(mxp[k & 7], __uint_as_float(sr[k]));
+      for (int k = 8; k < C::BKV; k += 16)
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          mxp[q] = max3f(mxp[q], __uint_as_float(sr[k + q]), __uint_as_float(sr[k + 8 + q]));
 #pragma unroll
       for (int k = 0; k < 4; ++k) mxp[k] = fmaxf(mxp[k], mxp[k + 4]);
       const float mx = fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3]));
@@ -396,14 +405,13 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int cc = 0; cc < C::BKV / 32; ++cc) {
         uint32_t pk[16];
-        const bool emu = !masked && cc >= 4 - EMU_CHUNKS;
 #pragma unroll
         for (int k = 0; k < 32; k += 2) {
+          const int col = cc * 32 + k;
           float2 a = __ffma2_rn(
-              make_float2(__uint_as_float(sr[cc * 32 + k]), __uint_as_float(sr[cc * 32 + k + 1])),
-              cc2, mref2);
+              make_float2(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])), cc2, mref2);
           float2 e2;
-          if (emu) {
+          if (!masked && ((emu_group_mask(EMU) >> (col >> 4)) & 1u)) {
             e2 = exp2_poly2(a);
           } else {
             e2.x = ex2_approx(a.x);

@@ -35,16 +35,16 @@ namespace {
 using bpt::RowMap;
 
 constexpr int64_t kMaxWave = BPT_WAVE_BLOCKS;
-// 32-column chunks (of four per 128-key row) whose exp2 runs on the FMA pipe
-// (compile-time tuning knobs).
-#ifndef BPT_EMU_CHUNKS_DK128
-#define BPT_EMU_CHUNKS_DK128 0
+// 16-column groups (of eight per 128-key row) whose exp2 runs on the FMA
+// pipe instead of MUFU (compile-time tuning knobs; MUFU-only measured fastest).
+#ifndef BPT_EMU_DK128
+#define BPT_EMU_DK128 0
 #endif
-#ifndef BPT_EMU_CHUNKS_DK64
-#define BPT_EMU_CHUNKS_DK64 0
+#ifndef BPT_EMU_DK64
+#define BPT_EMU_DK64 0
 #endif
-constexpr int kEmu128 = BPT_EMU_CHUNKS_DK128;
-constexpr int kEmu64 = BPT_EMU_CHUNKS_DK64;
+constexpr int kEmu128 = BPT_EMU_DK128;
+constexpr int kEmu64 = BPT_EMU_DK64;
 constexpr size_t kHeaderBytes = 256;
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }

@@ -1,11 +1,12 @@
 """The FMA-pipe exp2 of the attention kernel: constants and error bound.
 
-The kernel computes 2^x as 2^floor(x) * p(x - floor(x)) with a cubic p.  Here
-the constants compiled into the kernel are read from its source, checked
-against the fitting script, and the full float32 evaluation (range reduction,
-Horner steps with fused multiply-adds emulated in float64 then rounded, the
-exponent-field add) is compared with the exact 2^x over the range the kernel
-feeds it.
+The kernel computes 2^x as 2^n * p(x - n), n = round(x) obtained by adding and
+subtracting 1.5 * 2^23, with a cubic p on [-1/2, 1/2].  Here the constants
+compiled into the kernel are read from its source, checked against the fitting
+script, and the full float32 evaluation (clamp, rounding trick, Horner steps
+with fused multiply-adds emulated in float64 then rounded, the exponent-field
+add of the rounded float's low bits shifted by 23) is compared with the exact
+2^x over the range the kernel feeds it.
 """
 import importlib.util
 import os
@@ -37,14 +38,17 @@ def fma32(a, b, c):
 
 def exp2_kernel(x):
     c0, c1, c2, c3 = kernel_coeffs()
+    magic = np.float32(12582912.0)
     x = np.maximum(np.float32(x), np.float32(-125.0)).astype(np.float32)
-    xi = np.floor(x).astype(np.float32)
-    f = (x - xi).astype(np.float32)
+    j = (x + magic).astype(np.float32)
+    n = (j - magic).astype(np.float32)
+    f = (x - n).astype(np.float32)
     q = fma32(c3, f, c2)
     q = fma32(q, f, c1)
     q = fma32(q, f, c0)
-    bits = q.astype(np.float32).view(np.int32) + (xi.astype(np.int32) << 23)
-    return bits.view(np.float32)
+    bits = (q.astype(np.float32).view(np.int32).astype(np.int64)
+            + (j.view(np.int32).astype(np.int64) << 23)) & 0xFFFFFFFF
+    return bits.astype(np.uint32).view(np.float32)
 
 
 def test_relative_error_bound():
