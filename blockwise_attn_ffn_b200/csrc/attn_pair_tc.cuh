@@ -273,32 +273,35 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t ring = smem_u32(smem + C::OFF_RING);
     auto slot_of = [&](int t) { return t % C::NSLOT; };
     auto phase_of = [&](int t) { return static_cast<uint32_t>((t / C::NSLOT) & 1); };
-    auto issue_s = [&](uint32_t sQ, uint32_t sK, uint32_t d_tmem) {
+    // Descriptor words: Q_A, Q_B fixed; K/V per ring slot.  A k-step adds a
+    // constant to the low word (start address >> 4).
+    constexpr uint32_t hi = sdesc_hi(1024);
+    const uint32_t qa_lo = sdesc_lo(sQA, 16), qb_lo = sdesc_lo(sQB, 16);
+    auto issue_s = [&](uint32_t q_lo, uint32_t k_lo, uint32_t d_tmem) {
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
-        const uint32_t off = (k >> 2) * C::CHUNK + (k & 3) * 32;
-        umma_f16(d_tmem, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024),
-                  idesc_s, k > 0 ? 1u : 0u);
+        const uint32_t off = ((k >> 2) * C::CHUNK + (k & 3) * 32) >> 4;
+        umma_ss(d_tmem, q_lo + off, hi, k_lo + off, hi, idesc_s, k > 0 ? 1u : 0u);
       }
     };
-    auto issue_pv = [&](uint32_t tP, uint32_t sV, uint32_t d_tmem, bool first) {
+    auto issue_pv = [&](uint32_t tP, uint32_t v_lo, uint32_t d_tmem, bool first) {
 #pragma unroll
       for (int k = 0; k < C::BKV / 16; ++k)
-        umma_f16_ts(d_tmem, tP + 8 * k, sdesc_sw128(sV + k * 2048, C::CHUNK, 1024), idesc_o,
-                     (!first || k > 0) ? 1u : 0u);
+        umma_ts(d_tmem, tP + 8 * k, v_lo + ((k * 2048) >> 4), hi, idesc_o,
+                (!first || k > 0) ? 1u : 0u);
     };
     uint32_t pph[2] = {0, 0};
     bool ok = mbar_wait(q_full, 0, abort_flag, p.err, kSiteAttnMma);
     if (ok) ok = mbar_wait(ring_full0 + 8 * slot_of(0), phase_of(0), abort_flag, p.err, kSiteAttnMma);
     if (ok) {
       tc_fence_after();
-      const uint32_t sK0 = ring + slot_of(0) * C::TILE;
+      const uint32_t k0_lo = sdesc_lo(ring + slot_of(0) * C::TILE, 16);
       if (nA > 0) {
-        issue_s(sQA, sK0, tmem);
+        issue_s(qa_lo, k0_lo, tmem);
         umma_commit(s_full0);
       }
       if (nB > 0) {
-        issue_s(sQB, sK0, tmem + C::TM_S_B);
+        issue_s(qb_lo, k0_lo, tmem + C::TM_S_B);
         umma_commit(s_full0 + 8);
       }
       umma_commit(ring_empty0 + 8 * slot_of(0));
@@ -307,8 +310,8 @@ __global__ void __launch_bounds__(384, 1)
       const int tk = 2 * (j + 1), tv = 2 * j + 1;
       bool k_ready = false;
       if (!mbar_wait(ring_full0 + 8 * slot_of(tv), phase_of(tv), abort_flag, p.err, kSiteAttnMma)) break;
-      const uint32_t sV = ring + slot_of(tv) * C::TILE;
-      const uint32_t sK = ring + slot_of(tk) * C::TILE;
+      const uint32_t v_lo = sdesc_lo(ring + slot_of(tv) * C::TILE, C::CHUNK);
+      const uint32_t k_lo = sdesc_lo(ring + slot_of(tk) * C::TILE, 16);
       for (int x = 0; x < 2 && ok; ++x) {
         const int nX = x == 0 ? nA : nB;
         if (j >= nX) continue;
@@ -319,7 +322,7 @@ __global__ void __launch_bounds__(384, 1)
         pph[x] ^= 1u;
         tc_fence_after();
         const uint32_t tS = tmem + (x == 0 ? 0u : C::TM_S_B);
-        issue_pv(tS, sV, tmem + (x == 0 ? C::TM_O_A : C::TM_O_B), j == 0);
+        issue_pv(tS, v_lo, tmem + (x == 0 ? C::TM_O_A : C::TM_O_B), j == 0);
         if (j + 1 < nX) {
           if (!k_ready) {
             if (!mbar_wait(ring_full0 + 8 * slot_of(tk), phase_of(tk), abort_flag, p.err,
@@ -330,7 +333,7 @@ __global__ void __launch_bounds__(384, 1)
             tc_fence_after();
             k_ready = true;
           }
-          issue_s(x == 0 ? sQA : sQB, sK, tS);
+          issue_s(x == 0 ? qa_lo : qb_lo, k_lo, tS);
           umma_commit(s_full0 + 8 * x);
         } else {
           umma_commit(o_done0 + 8 * x);

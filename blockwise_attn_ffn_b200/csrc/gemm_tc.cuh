@@ -261,14 +261,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t a_base = smem_u32(sA + stage * kGemmABytes);
-        const uint32_t b_base = smem_u32(sB + stage * kGemmBBytes);
+        const uint32_t a_lo = sdesc_lo(smem_u32(sA + stage * kGemmABytes), 16);
+        const uint32_t b_lo = sdesc_lo(smem_u32(sB + stage * kGemmBBytes), 8192);
+        constexpr uint32_t hi = sdesc_hi(1024);
 #pragma unroll
-        for (int k = 0; k < kGemmBK / 16; ++k) {
-          const uint64_t ad = sdesc_sw128(a_base + k * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(b_base + k * 2048, 8192, 1024);
-          umma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
-        }
+        for (int k = 0; k < kGemmBK / 16; ++k)
+          umma_ss(d_tmem, a_lo + 2 * k, hi, b_lo + 128 * k, hi, idesc, (kb | k) != 0 ? 1u : 0u);
         umma_commit(empty0 + 8 * stage);
         if (++stage == kGemmStages) {
           stage = 0;
@@ -477,14 +475,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t a_base = smem_u32(sA + stage * kPairABytes);
-        const uint32_t b_base = smem_u32(sB + stage * kPairBBytes);
+        const uint32_t a_lo = sdesc_lo(smem_u32(sA + stage * kPairABytes), 16);
+        const uint32_t b_lo = sdesc_lo(smem_u32(sB + stage * kPairBBytes), 8192);
+        constexpr uint32_t hi = sdesc_hi(1024);
 #pragma unroll
-        for (int k = 0; k < kGemmBK / 16; ++k) {
-          const uint64_t ad = sdesc_sw128(a_base + k * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(b_base + k * 2048, 8192, 1024);
-          umma_f16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
-        }
+        for (int k = 0; k < kGemmBK / 16; ++k)
+          umma_ss_pair(d_tmem, a_lo + 2 * k, hi, b_lo + 128 * k, hi, idesc,
+                       (kb | k) != 0 ? 1u : 0u);
         umma_commit_pair_mc(empty0 + 8 * stage, 0x3);
         if (++stage == kPairStages) {
           stage = 0;
