@@ -240,7 +240,7 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;
     for (int j = 0; j < n_kv && ok; ++j) {
       for (int w = 0; w < 2; ++w) {
-        if (!mbar_wait(ring_empty0 + 8 * slot, phase ^ 1u, abort_flag, p.err, kSiteAttnProducer)) {
+        if (!mbar_wait_fast(ring_empty0 + 8 * slot, phase ^ 1u, abort_flag, p.err, kSiteAttnProducer)) {
           ok = false;
           break;
         }
@@ -291,8 +291,8 @@ __global__ void __launch_bounds__(384, 1)
                 (!first || k > 0) ? 1u : 0u);
     };
     uint32_t pph[2] = {0, 0};
-    bool ok = mbar_wait(q_full, 0, abort_flag, p.err, kSiteAttnMma);
-    if (ok) ok = mbar_wait(ring_full0 + 8 * slot_of(0), phase_of(0), abort_flag, p.err, kSiteAttnMma);
+    bool ok = mbar_wait_fast(q_full, 0, abort_flag, p.err, kSiteAttnMma);
+    if (ok) ok = mbar_wait_fast(ring_full0 + 8 * slot_of(0), phase_of(0), abort_flag, p.err, kSiteAttnMma);
     if (ok) {
       tc_fence_after();
       const uint32_t k0_lo = sdesc_lo(ring + slot_of(0) * C::TILE, 16);
@@ -309,13 +309,15 @@ __global__ void __launch_bounds__(384, 1)
     for (int j = 0; j < n_kv && ok; ++j) {
       const int tk = 2 * (j + 1), tv = 2 * j + 1;
       bool k_ready = false;
-      if (!mbar_wait(ring_full0 + 8 * slot_of(tv), phase_of(tv), abort_flag, p.err, kSiteAttnMma)) break;
+      if (!mbar_wait_fast(ring_full0 + 8 * slot_of(tv), phase_of(tv), abort_flag, p.err,
+                          kSiteAttnMma))
+        break;
       const uint32_t v_lo = sdesc_lo(ring + slot_of(tv) * C::TILE, C::CHUNK);
       const uint32_t k_lo = sdesc_lo(ring + slot_of(tk) * C::TILE, 16);
       for (int x = 0; x < 2 && ok; ++x) {
         const int nX = x == 0 ? nA : nB;
         if (j >= nX) continue;
-        if (!mbar_wait(p_full0 + 8 * x, pph[x], abort_flag, p.err, kSiteAttnMma)) {
+        if (!mbar_wait_fast(p_full0 + 8 * x, pph[x], abort_flag, p.err, kSiteAttnMma)) {
           ok = false;
           break;
         }
@@ -325,12 +327,12 @@ __global__ void __launch_bounds__(384, 1)
         issue_pv(tS, v_lo, tmem + (x == 0 ? C::TM_O_A : C::TM_O_B), j == 0);
         if (j + 1 < nX) {
           if (!k_ready) {
-            if (!mbar_wait(ring_full0 + 8 * slot_of(tk), phase_of(tk), abort_flag, p.err,
+            if (!mbar_wait_fast(ring_full0 + 8 * slot_of(tk), phase_of(tk), abort_flag, p.err,
                            kSiteAttnMma)) {
               ok = false;
               break;
             }
-            tc_fence_after();
+            // (TMA data: ordered by the mbarrier wait itself)
             k_ready = true;
           }
           issue_s(x == 0 ? qa_lo : qb_lo, k_lo, tS);
@@ -362,7 +364,7 @@ __global__ void __launch_bounds__(384, 1)
     float l = 0.f;
     bool ok = nX > 0;
     for (int j = 0; j < nX && ok; ++j) {
-      if (!mbar_wait(s_full, j & 1, abort_flag, p.err, kSiteAttnSoftmax)) {
+      if (!mbar_wait_fast(s_full, j & 1, abort_flag, p.err, kSiteAttnSoftmax)) {
         ok = false;
         break;
       }
@@ -444,7 +446,7 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
-    if (ok && mbar_wait(o_done, 0, abort_flag, p.err, kSiteAttnSoftmax)) {
+    if (ok && mbar_wait_fast(o_done, 0, abort_flag, p.err, kSiteAttnSoftmax)) {
       tc_fence_after();
       const float inv_l = 1.0f / l;
       const long long srow = static_cast<long long>(itemA + x - p.item0) * C::BQ + r;

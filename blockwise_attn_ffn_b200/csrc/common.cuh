@@ -97,6 +97,13 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile i
   }
 }
 
+// Same as mbar_wait, with the already-complete case inlined (no call).
+__device__ __forceinline__ bool mbar_wait_fast(uint32_t bar, uint32_t parity,
+                                               volatile int* abort_flag, uint32_t* err,
+                                               uint32_t site) {
+  return mbar_try_wait(bar, parity) || mbar_wait(bar, parity, abort_flag, err, site);
+}
+
 // Bounded wait used while draining after an abort: ignores the abort flag.
 __device__ __noinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint32_t* err) {
   const uint64_t t0 = global_ns();

@@ -214,7 +214,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int mb, nb;
       gemm_tile_coords(tile, m_blocks, n_blocks, mb, nb);
       for (int kb = 0; kb < k_blocks; ++kb) {
-        if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.err, kSiteGemmProducer)) {
+        if (!mbar_wait_fast(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.err, kSiteGemmProducer)) {
           ok = false;
           break;
         }
@@ -252,11 +252,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t acc_phase = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-      if (!mbar_wait(acce0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.err, kSiteGemmMma)) break;
+      if (!mbar_wait_fast(acce0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.err, kSiteGemmMma)) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * kGemmBN);
       for (int kb = 0; kb < k_blocks; ++kb) {
-        if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, p.err, kSiteGemmMma)) {
+        if (!mbar_wait_fast(full0 + 8 * stage, phase, abort_flag, p.err, kSiteGemmMma)) {
           ok = false;
           break;
         }
@@ -291,7 +291,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
       int mb, nb;
       gemm_tile_coords(tile, m_blocks, n_blocks, mb, nb);
-      if (!mbar_wait(accf0 + 8 * acc, acc_phase, abort_flag, p.err, kSiteGemmEpilogue)) break;
+      if (!mbar_wait_fast(accf0 + 8 * acc, acc_phase, abort_flag, p.err, kSiteGemmEpilogue)) break;
       tc_fence_after();
       const long long row = static_cast<long long>(mb) * kGemmBM + e * 32 + lane;
       const uint32_t t_row = tmem + (static_cast<uint32_t>(e * 32) << 16) +
@@ -414,7 +414,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int mb, nb;
       coords(tile, mb, nb);
       for (int kb = 0; kb < k_blocks; ++kb) {
-        if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.err, kSiteGemmProducer)) {
+        if (!mbar_wait_fast(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.err, kSiteGemmProducer)) {
           ok = false;
           break;
         }
@@ -466,15 +466,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     uint32_t acc_phase = 0;
     bool ok = true;
     for (int tile = pair; tile < tiles && ok; tile += npairs) {
-      if (!mbar_wait(acce0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.err, kSiteGemmMma)) break;
+      if (!mbar_wait_fast(acce0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.err, kSiteGemmMma)) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * kGemmBN);
       for (int kb = 0; kb < k_blocks; ++kb) {
-        if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, p.err, kSiteGemmMma)) {
+        if (!mbar_wait_fast(full0 + 8 * stage, phase, abort_flag, p.err, kSiteGemmMma)) {
           ok = false;
           break;
         }
-        tc_fence_after();
         const uint32_t a_lo = sdesc_lo(smem_u32(sA + stage * kPairABytes), 16);
         const uint32_t b_lo = sdesc_lo(smem_u32(sB + stage * kPairBBytes), 8192);
         constexpr uint32_t hi = sdesc_hi(1024);
@@ -505,7 +504,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     for (int tile = pair; tile < tiles; tile += npairs) {
       int mb, nb;
       coords(tile, mb, nb);
-      if (!mbar_wait(accf0 + 8 * acc, acc_phase, abort_flag, p.err, kSiteGemmEpilogue)) break;
+      if (!mbar_wait_fast(accf0 + 8 * acc, acc_phase, abort_flag, p.err, kSiteGemmEpilogue)) break;
       tc_fence_after();
       const long long row =
           static_cast<long long>(mb) * kPairBM + static_cast<long long>(rank) * 128 + e * 32 + lane;
