@@ -43,6 +43,8 @@
 // 4..7 softmax of tile A, 8..11 softmax of tile B (thread = query row).
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace bpt {
@@ -407,26 +409,35 @@ __global__ void __launch_bounds__(384, 1)
       const float2 mref2 = make_float2(-m_new * c, -m_new * c);
       float2 sum2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                         make_float2(0.f, 0.f)};
+      // One unrolled loop per tile kind, so the MUFU / FMA choice of each
+      // 16-column group is fixed at compile time (no per-element branch).
+      auto exp_row = [&](auto emu_mask) {
+        constexpr uint32_t kMask = decltype(emu_mask)::value;
 #pragma unroll
-      for (int cc = 0; cc < C::BKV / 32; ++cc) {
-        uint32_t pk[16];
+        for (int cc = 0; cc < C::BKV / 32; ++cc) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int k = 0; k < 32; k += 2) {
-          const int col = cc * 32 + k;
-          float2 a = __ffma2_rn(
-              make_float2(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])), cc2, mref2);
-          float2 e2;
-          if (!masked && ((emu_group_mask(EMU) >> (col >> 4)) & 1u)) {
-            e2 = exp2_poly2(a);
-          } else {
-            e2.x = ex2_approx(a.x);
-            e2.y = ex2_approx(a.y);
+          for (int k = 0; k < 32; k += 2) {
+            const int col = cc * 32 + k;
+            float2 a = __ffma2_rn(
+                make_float2(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])), cc2, mref2);
+            float2 e2;
+            if ((kMask >> (col >> 4)) & 1u) {
+              e2 = exp2_poly2(a);
+            } else {
+              e2.x = ex2_approx(a.x);
+              e2.y = ex2_approx(a.y);
+            }
+            sum2[(k >> 1) & 3] = __fadd2_rn(sum2[(k >> 1) & 3], e2);
+            pk[k >> 1] = pack_f16x2(e2.x, e2.y);
           }
-          sum2[(k >> 1) & 3] = __fadd2_rn(sum2[(k >> 1) & 3], e2);
-          pk[k >> 1] = pack_f16x2(e2.x, e2.y);
+          tmem_st_32x32b_x16(tS + cc * 16, pk);
         }
-        tmem_st_32x32b_x16(tS + cc * 16, pk);
-      }
+      };
+      if (masked || emu_group_mask(EMU) == 0u)
+        exp_row(std::integral_constant<uint32_t, 0u>{});
+      else
+        exp_row(std::integral_constant<uint32_t, emu_group_mask(EMU)>{});
       sum2[0] = __fadd2_rn(__fadd2_rn(sum2[0], sum2[1]), __fadd2_rn(sum2[2], sum2[3]));
       l = alpha * l + (sum2[0].x + sum2[0].y);
       m_run = m_new;

@@ -36,12 +36,12 @@ using bpt::RowMap;
 
 constexpr int64_t kMaxWave = BPT_WAVE_BLOCKS;
 // 16-column groups (of eight per 128-key row) whose exp2 runs on the FMA
-// pipe instead of MUFU (compile-time tuning knobs; MUFU-only measured fastest).
+// pipe instead of MUFU (compile-time tuning knobs; 2 of 8 measured fastest).
 #ifndef BPT_EMU_DK128
-#define BPT_EMU_DK128 0
+#define BPT_EMU_DK128 2
 #endif
 #ifndef BPT_EMU_DK64
-#define BPT_EMU_DK64 0
+#define BPT_EMU_DK64 2
 #endif
 constexpr int kEmu128 = BPT_EMU_DK128;
 constexpr int kEmu64 = BPT_EMU_DK64;
