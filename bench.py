@@ -39,6 +39,36 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per attention
+# launch, the mean over one step's launches, from one ncu capture of the
+# default bench command.  Valid only for the sources it was taken on: the
+# digest covers the attention kernel, the shared device helpers and the host
+# launch code; after any change the bench reports null until it is retaken.
+ATTN_TRAFFIC = {
+    # 12 launches (6 forwards x 2 waves): waves of 405 + 113 and 1277 + 127 MB
+    "long_n64k": {"digest": "9e67c1468bf71264", "bytes_per_launch": 961234453},
+}
+TRAFFIC_SOURCES = ("blockwise_attn_ffn_b200/csrc/attn_pair_tc.cuh",
+                   "blockwise_attn_ffn_b200/csrc/common.cuh",
+                   "blockwise_attn_ffn_b200/csrc/bpt_api.cu")
+
+
+def sources_digest() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def attn_traffic(workload: str):
+    entry = ATTN_TRAFFIC.get(workload)
+    if entry is None or entry["digest"] != sources_digest():
+        return None
+    return entry["bytes_per_launch"]
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -277,6 +307,7 @@ def main():
     attn_ms_launch = kind_ms["attn"] / n_attn
     attn_flops_launch = flops["attention"] * args.steps / n_attn
     achieved = attn_flops_launch / (attn_ms_launch / 1e3) / 1e12
+    attn_bytes_launch = accounting.attention_bytes(cfg.B, cfg.N, cfg.d, cfg.h) * args.steps / n_attn
     peak_sus = peaks["bf16_tflops_sustained"]
     total_kernel_ms = sum(kind_ms.values())
     kernels = {k: {"ms_per_step": kind_ms[k] / args.steps, "launches_per_step": kind_n[k] / args.steps,
@@ -309,7 +340,10 @@ def main():
         "roofline": {"bound": "tensor", "kernel": "attn_pair_tc_kernel", "achieved": achieved,
                      "peak": peak_sus, "unit": "TFLOP/s", "frac": achieved / peak_sus,
                      "peak_kind": f"bf16_tflops_sustained ({peak_src})",
-                     "frac_of_burst": achieved / peaks["bf16_tflops"], "traffic": None},
+                     "frac_of_burst": achieved / peaks["bf16_tflops"],
+                     "traffic": attn_traffic(cfg.name),
+                     "traffic_unit": "bytes per launch (ncu dram read + write)",
+                     "algorithmic_bytes_per_launch": attn_bytes_launch},
         "kernels": kernels,
         "peak_bytes": {"fused_device_total": int(peak_fused),
                        "unfused_activations_analytic": int(cfg.B * unfused["total"] * esz),

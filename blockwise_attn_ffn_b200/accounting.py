@@ -36,6 +36,13 @@ def layer_flops(B: int, N: int, d: int, h: int, d_ff: int, causal: bool) -> Dict
     return f
 
 
+def attention_bytes(B: int, N: int, d: int, h: int, elem_bytes: int = 2) -> int:
+    """Least HBM bytes of the attention step of one layer forward: Q, K and V
+    read once and the per-head outputs o written once, 16-bit elements."""
+    del h
+    return 4 * B * N * d * elem_bytes
+
+
 def unfused_activation_elems(N: int, d: int, h: int, d_ff: int,
                              with_logits: bool = True) -> Dict[str, int]:
     """Per-layer activation audit of the unfused layer (elements).

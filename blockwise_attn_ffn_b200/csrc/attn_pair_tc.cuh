@@ -58,6 +58,8 @@ struct AttnPairParams {
   int item0;   // first flattened block item (batch * nb + block) of the wave
   int count;   // block items in the wave
   int seqs;    // >0: the wave is `seqs` whole sequences; 0: part of one sequence
+  int hg;      // heads per group (divides h): CTAs run group by group, so the
+               // K/V that concurrent CTAs sweep is that of hg heads only
   __half* o;         // [count * 128, d] block scratch (fp16)
   float scale_log2;  // log2(e) / sqrt(d_k)
   uint32_t* err;
@@ -185,8 +187,13 @@ __global__ void __launch_bounds__(384, 1)
   __shared__ int abort_sh;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rank = blockIdx.x / p.h;
-  const int head = blockIdx.x - rank * p.h;
+  // blockIdx -> (head group, work rank, head): within a group, consecutive
+  // CTAs take the group's heads for one rank, longest ranks first.
+  const int per_group = int(gridDim.x / p.h) * p.hg;
+  const int grp = blockIdx.x / per_group;
+  const int in_grp = blockIdx.x - grp * per_group;
+  const int rank = in_grp / p.hg;
+  const int head = grp * p.hg + (in_grp - rank * p.hg);
   int itemA;
   bool has_b;
   attn_pair_decode(p, rank, itemA, has_b);

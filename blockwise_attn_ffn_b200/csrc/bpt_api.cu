@@ -43,6 +43,12 @@ constexpr int64_t kMaxWave = BPT_WAVE_BLOCKS;
 #ifndef BPT_EMU_DK64
 #define BPT_EMU_DK64 2
 #endif
+// Attention CTAs run head group by head group; a group is the largest
+// divisor of h whose K/V (all keys of the wave) fits this many bytes, half of
+// the 126 MB L2, so concurrent CTAs re-read K/V from L2 rather than HBM.
+#ifndef BPT_ATTN_KV_BUDGET_MB
+#define BPT_ATTN_KV_BUDGET_MB 64
+#endif
 constexpr int kEmu128 = BPT_EMU_DK128;
 constexpr int kEmu64 = BPT_EMU_DK64;
 constexpr size_t kHeaderBytes = 256;
@@ -441,6 +447,13 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
       ap.N = int(P.N); ap.nb = int(P.nb); ap.h = int(P.h); ap.d = int(d);
       ap.causal = P.causal; ap.item0 = int(wv_.item0); ap.count = int(wv_.count);
       ap.seqs = int(wv_.seqs); ap.o = so; ap.scale_log2 = scale_log2; ap.err = err;
+      const int64_t kv_head = (wv_.seqs > 0 ? wv_.seqs : 1) * P.N * P.dk * 2 * 2;
+      ap.hg = 1;
+      for (int g = int(P.h); g > 1; --g)
+        if (P.h % g == 0 && g * kv_head <= (int64_t(BPT_ATTN_KV_BUDGET_MB) << 20)) {
+          ap.hg = g;
+          break;
+        }
       ap.fault = (fault == 2 && w == 0) ? 2 : 0;
       const int64_t pairs = wv_.seqs == 0 ? (wv_.count + 1) / 2 : wv_.seqs * ((P.nb + 1) / 2);
       const unsigned grid = unsigned(pairs * P.h);

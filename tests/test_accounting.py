@@ -55,3 +55,9 @@ def test_causal_pairs_and_long_workload_total():
     assert acc.attention_pairs(4, True) == 10
     f = acc.layer_flops(1, 65536, 2048, 16, 8192, True)
     assert abs(f["total"] / 1e12 - 24.19) < 0.01
+
+
+def test_attention_bytes_counts_q_k_v_and_o_once():
+    # long-context layer: 65536 x 2048 16-bit values each for Q, K, V and o
+    assert acc.attention_bytes(1, 65536, 2048, 16) == 4 * 65536 * 2048 * 2
+    assert acc.attention_bytes(8, 2048, 768, 12) == 8 * acc.attention_bytes(1, 2048, 768, 12)
