@@ -230,39 +230,47 @@ __global__ void __launch_bounds__(384, 1)
   volatile int* abort_flag = &abort_sh;
   const int colQ = head * D, colK = p.d + head * D, colV = 2 * p.d + head * D;
 
-  if (warp == 0 && lane == 0) {
+  if (warp == 0) {
     // ------------------------------------------------------------ producer
-    tma_prefetch_desc(&mapQKV);
+    // The whole warp runs the role (warp-uniform coordinates); the elected
+    // lane issues the TMA loads.
+    const bool leader = elect_one();
+    if (leader) tma_prefetch_desc(&mapQKV);
     int armed[C::NSLOT];
     for (int s = 0; s < C::NSLOT; ++s) armed[s] = -1;
-    mbar_arrive_expect_tx(q_full, C::TILE * (has_b ? 2 : 1));
+    if (leader) {
+      mbar_arrive_expect_tx(q_full, C::TILE * (has_b ? 2 : 1));
 #pragma unroll
-    for (int c = 0; c < D / 64; ++c) {
-      tma_load_3d(smem_u32(smem + C::OFF_QA + c * C::CHUNK), &mapQKV, q_full, colQ + 64 * c,
-                  iA * C::BQ, bidx);
-      if (has_b)
-        tma_load_3d(smem_u32(smem + C::OFF_QB + c * C::CHUNK), &mapQKV, q_full, colQ + 64 * c,
-                    iB * C::BQ, bidx);
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_3d(smem_u32(smem + C::OFF_QA + c * C::CHUNK), &mapQKV, q_full, colQ + 64 * c,
+                    iA * C::BQ, bidx);
+        if (has_b)
+          tma_load_3d(smem_u32(smem + C::OFF_QB + c * C::CHUNK), &mapQKV, q_full,
+                      colQ + 64 * c, iB * C::BQ, bidx);
+      }
     }
     int slot = 0;
     uint32_t phase = 0;
     bool ok = true;
     for (int j = 0; j < n_kv && ok; ++j) {
       for (int w = 0; w < 2; ++w) {
-        if (!mbar_wait_fast(ring_empty0 + 8 * slot, phase ^ 1u, abort_flag, p.err, kSiteAttnProducer)) {
+        if (!mbar_wait_warp(ring_empty0 + 8 * slot, phase ^ 1u, abort_flag, p.err,
+                            kSiteAttnProducer)) {
           ok = false;
           break;
         }
         const uint32_t fb = ring_full0 + 8 * slot;
         const bool lost = p.fault == 2 && blockIdx.x == 0 && j == 0 && w == 1;
         if (!lost) {
-          mbar_arrive_expect_tx(fb, C::TILE);
           armed[slot] = static_cast<int>(phase);
           const int col = w == 0 ? colK : colV;
+          if (leader) {
+            mbar_arrive_expect_tx(fb, C::TILE);
 #pragma unroll
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(smem_u32(smem + C::OFF_RING + slot * C::TILE + c * C::CHUNK), &mapQKV, fb,
-                        col + 64 * c, j * C::BKV, bidx);
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(smem_u32(smem + C::OFF_RING + slot * C::TILE + c * C::CHUNK), &mapQKV,
+                          fb, col + 64 * c, j * C::BKV, bidx);
+          }
         }
         if (++slot == C::NSLOT) {
           slot = 0;
@@ -273,8 +281,13 @@ __global__ void __launch_bounds__(384, 1)
     mbar_wait_drain(q_full, 0, p.err);
     for (int s = 0; s < C::NSLOT; ++s)
       if (armed[s] >= 0) mbar_wait_drain(ring_full0 + 8 * s, static_cast<uint32_t>(armed[s]), p.err);
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1) {
     // ----------------------------------------------------------- UMMA issue
+    // The whole warp runs the role so that descriptors stay warp-uniform; the
+    // elected lane issues each MMA and commit (issuing from one lane with
+    // per-lane descriptors cost ~100 clocks per MMA, above the 64 of an
+    // M128 N128 K16 MMA).
+    const bool leader = elect_one();
     constexpr uint32_t idesc_s = idesc_f16_f32(C::BQ, C::BKV, false, false);
     constexpr uint32_t idesc_o = idesc_f16_f32(C::BQ, D, false, true);
     const uint32_t sQA = smem_u32(smem + C::OFF_QA);
@@ -287,38 +300,50 @@ __global__ void __launch_bounds__(384, 1)
     constexpr uint32_t hi = sdesc_hi(1024);
     const uint32_t qa_lo = sdesc_lo(sQA, 16), qb_lo = sdesc_lo(sQB, 16);
     auto issue_s = [&](uint32_t q_lo, uint32_t k_lo, uint32_t d_tmem) {
+      if (leader) {
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
-        const uint32_t off = ((k >> 2) * C::CHUNK + (k & 3) * 32) >> 4;
-        umma_ss(d_tmem, q_lo + off, hi, k_lo + off, hi, idesc_s, k > 0 ? 1u : 0u);
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = ((k >> 2) * C::CHUNK + (k & 3) * 32) >> 4;
+          umma_ss(d_tmem, q_lo + off, hi, k_lo + off, hi, idesc_s, k > 0 ? 1u : 0u);
+        }
       }
+      __syncwarp();
     };
     auto issue_pv = [&](uint32_t tP, uint32_t v_lo, uint32_t d_tmem, bool first) {
+      if (leader) {
 #pragma unroll
-      for (int k = 0; k < C::BKV / 16; ++k)
-        umma_ts(d_tmem, tP + 8 * k, v_lo + ((k * 2048) >> 4), hi, idesc_o,
-                (!first || k > 0) ? 1u : 0u);
+        for (int k = 0; k < C::BKV / 16; ++k)
+          umma_ts(d_tmem, tP + 8 * k, v_lo + ((k * 2048) >> 4), hi, idesc_o,
+                  (!first || k > 0) ? 1u : 0u);
+      }
+      __syncwarp();
+    };
+    auto commit = [&](uint32_t bar) {
+      if (leader) umma_commit(bar);
+      __syncwarp();
     };
     uint32_t pph[2] = {0, 0};
-    bool ok = mbar_wait_fast(q_full, 0, abort_flag, p.err, kSiteAttnMma);
-    if (ok) ok = mbar_wait_fast(ring_full0 + 8 * slot_of(0), phase_of(0), abort_flag, p.err, kSiteAttnMma);
+    bool ok = mbar_wait_warp(q_full, 0, abort_flag, p.err, kSiteAttnMma);
+    if (ok)
+      ok = mbar_wait_warp(ring_full0 + 8 * slot_of(0), phase_of(0), abort_flag, p.err,
+                          kSiteAttnMma);
     if (ok) {
       tc_fence_after();
       const uint32_t k0_lo = sdesc_lo(ring + slot_of(0) * C::TILE, 16);
       if (nA > 0) {
         issue_s(qa_lo, k0_lo, tmem);
-        umma_commit(s_full0);
+        commit(s_full0);
       }
       if (nB > 0) {
         issue_s(qb_lo, k0_lo, tmem + C::TM_S_B);
-        umma_commit(s_full0 + 8);
+        commit(s_full0 + 8);
       }
-      umma_commit(ring_empty0 + 8 * slot_of(0));
+      commit(ring_empty0 + 8 * slot_of(0));
     }
     for (int j = 0; j < n_kv && ok; ++j) {
       const int tk = 2 * (j + 1), tv = 2 * j + 1;
       bool k_ready = false;
-      if (!mbar_wait_fast(ring_full0 + 8 * slot_of(tv), phase_of(tv), abort_flag, p.err,
+      if (!mbar_wait_warp(ring_full0 + 8 * slot_of(tv), phase_of(tv), abort_flag, p.err,
                           kSiteAttnMma))
         break;
       const uint32_t v_lo = sdesc_lo(ring + slot_of(tv) * C::TILE, C::CHUNK);
@@ -326,7 +351,7 @@ __global__ void __launch_bounds__(384, 1)
       for (int x = 0; x < 2 && ok; ++x) {
         const int nX = x == 0 ? nA : nB;
         if (j >= nX) continue;
-        if (!mbar_wait_fast(p_full0 + 8 * x, pph[x], abort_flag, p.err, kSiteAttnMma)) {
+        if (!mbar_wait_warp(p_full0 + 8 * x, pph[x], abort_flag, p.err, kSiteAttnMma)) {
           ok = false;
           break;
         }
@@ -336,8 +361,8 @@ __global__ void __launch_bounds__(384, 1)
         issue_pv(tS, v_lo, tmem + (x == 0 ? C::TM_O_A : C::TM_O_B), j == 0);
         if (j + 1 < nX) {
           if (!k_ready) {
-            if (!mbar_wait_fast(ring_full0 + 8 * slot_of(tk), phase_of(tk), abort_flag, p.err,
-                           kSiteAttnMma)) {
+            if (!mbar_wait_warp(ring_full0 + 8 * slot_of(tk), phase_of(tk), abort_flag, p.err,
+                                kSiteAttnMma)) {
               ok = false;
               break;
             }
@@ -345,16 +370,16 @@ __global__ void __launch_bounds__(384, 1)
             k_ready = true;
           }
           issue_s(x == 0 ? qa_lo : qb_lo, k_lo, tS);
-          umma_commit(s_full0 + 8 * x);
+          commit(s_full0 + 8 * x);
         } else {
-          umma_commit(o_done0 + 8 * x);
+          commit(o_done0 + 8 * x);
         }
       }
       if (!ok) break;
-      umma_commit(ring_empty0 + 8 * slot_of(tv));
-      if (k_ready) umma_commit(ring_empty0 + 8 * slot_of(tk));
+      commit(ring_empty0 + 8 * slot_of(tv));
+      if (k_ready) commit(ring_empty0 + 8 * slot_of(tk));
     }
-    umma_commit(drain);
+    commit(drain);
     mbar_wait_drain(drain, 0, p.err);
   } else if (warp >= 4) {
     // -------------------------------------------------------------- softmax

@@ -104,6 +104,27 @@ __device__ __forceinline__ bool mbar_wait_fast(uint32_t bar, uint32_t parity,
   return mbar_try_wait(bar, parity) || mbar_wait(bar, parity, abort_flag, err, site);
 }
 
+// A role run by a whole converged warp keeps its operands (descriptors,
+// coordinates, barrier addresses) warp-uniform; one lane, picked by
+// elect.sync, then issues each single-thread instruction (tcgen05.mma,
+// tcgen05.commit, TMA).  Every lane waits on barriers itself; the vote makes
+// the outcome of a bounded wait the same for the whole warp.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
+                                               volatile int* abort_flag, uint32_t* err,
+                                               uint32_t site) {
+  const bool ok = mbar_wait_fast(bar, parity, abort_flag, err, site);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // Bounded wait used while draining after an abort: ignores the abort flag.
 __device__ __noinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint32_t* err) {
   const uint64_t t0 = global_ns();
