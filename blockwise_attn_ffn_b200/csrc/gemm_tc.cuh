@@ -399,12 +399,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     nb = in / gm;
   };
 
-  if (warp == 0 && lane == 0) {
+  if (warp == 0) {
     // ------------------------------------------------------------ producer
-    tma_prefetch_desc(&mapA);
-    tma_prefetch_desc(&mapB0);
-    if (p.n_maps > 1) tma_prefetch_desc(&mapB1);
-    if (p.n_maps > 2) tma_prefetch_desc(&mapB2);
+    // Whole warp (warp-uniform coordinates); the elected lane issues.
+    const bool leader = elect_one();
+    if (leader) {
+      tma_prefetch_desc(&mapA);
+      tma_prefetch_desc(&mapB0);
+      if (p.n_maps > 1) tma_prefetch_desc(&mapB1);
+      if (p.n_maps > 2) tma_prefetch_desc(&mapB2);
+    }
     int armed[kPairStages];
     for (int s2 = 0; s2 < kPairStages; ++s2) armed[s2] = -1;
     int stage = 0;
@@ -413,28 +417,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     for (int tile = pair; tile < tiles && ok; tile += npairs) {
       int mb, nb;
       coords(tile, mb, nb);
+      // This CTA's two 64-column B boxes: which weight map, and the column in it.
+      const CUtensorMap* bmap[2];
+      int bcol[2];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int c = nb * kGemmBN + static_cast<int>(rank) * 128 + q * 64;
+        int which = c / p.n_sub;
+        if (which > p.n_maps - 1) which = p.n_maps - 1;  // past the end: TMA zero-fills
+        bmap[q] = which == 0 ? &mapB0 : (which == 1 ? &mapB1 : &mapB2);
+        bcol[q] = c - which * p.n_sub;
+      }
       for (int kb = 0; kb < k_blocks; ++kb) {
-        if (!mbar_wait_fast(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.err, kSiteGemmProducer)) {
+        if (!mbar_wait_warp(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.err, kSiteGemmProducer)) {
           ok = false;
           break;
         }
         const uint32_t fb_leader = map_to_rank(full0 + 8 * stage, 0);
         const bool lost = p.fault == 1 && pair == 0 && rank == 0 && tile == pair && kb == 0;
         if (!lost) {
-          if (rank == 0) {
-            mbar_arrive_expect_tx(full0 + 8 * stage, 2 * kPairStageBytes);
-            armed[stage] = static_cast<int>(phase);
-          }
-          tma_load_2d_pair(smem_u32(sA + stage * kPairABytes), &mapA, fb_leader, kb * kGemmBK,
-                           mb * kPairBM + static_cast<int>(rank) * 128);
+          if (rank == 0) armed[stage] = static_cast<int>(phase);
+          if (leader) {
+            if (rank == 0) mbar_arrive_expect_tx(full0 + 8 * stage, 2 * kPairStageBytes);
+            tma_load_2d_pair(smem_u32(sA + stage * kPairABytes), &mapA, fb_leader, kb * kGemmBK,
+                             mb * kPairBM + static_cast<int>(rank) * 128);
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const int c = nb * kGemmBN + static_cast<int>(rank) * 128 + q * 64;
-            int which = c / p.n_sub;
-            if (which > p.n_maps - 1) which = p.n_maps - 1;  // past the end: TMA zero-fills
-            const CUtensorMap* mB = which == 0 ? &mapB0 : (which == 1 ? &mapB1 : &mapB2);
-            tma_load_2d_pair(smem_u32(sB + stage * kPairBBytes + q * 8192), mB, fb_leader,
-                             c - which * p.n_sub, kb * kGemmBK);
+            for (int q = 0; q < 2; ++q)
+              tma_load_2d_pair(smem_u32(sB + stage * kPairBBytes + q * 8192), bmap[q], fb_leader,
+                               bcol[q], kb * kGemmBK);
           }
         }
         if (++stage == kPairStages) {
@@ -457,8 +467,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       while (global_ns() - t0 < 200000ull) {
       }
     }
-  } else if (warp == 1 && lane == 0 && rank == 0) {
+  } else if (warp == 1 && rank == 0) {
     // ------------------------------------------------ UMMA issue (leader)
+    // Whole warp (warp-uniform descriptors); the elected lane issues.
+    const bool leader = elect_one();
     constexpr uint32_t idesc = idesc_f16_f32(kPairBM, kGemmBN, false, true);
     int stage = 0;
     uint32_t phase = 0;
@@ -466,35 +478,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     uint32_t acc_phase = 0;
     bool ok = true;
     for (int tile = pair; tile < tiles && ok; tile += npairs) {
-      if (!mbar_wait_fast(acce0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.err, kSiteGemmMma)) break;
+      if (!mbar_wait_warp(acce0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.err, kSiteGemmMma)) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * kGemmBN);
       for (int kb = 0; kb < k_blocks; ++kb) {
-        if (!mbar_wait_fast(full0 + 8 * stage, phase, abort_flag, p.err, kSiteGemmMma)) {
+        if (!mbar_wait_warp(full0 + 8 * stage, phase, abort_flag, p.err, kSiteGemmMma)) {
           ok = false;
           break;
         }
         const uint32_t a_lo = sdesc_lo(smem_u32(sA + stage * kPairABytes), 16);
         const uint32_t b_lo = sdesc_lo(smem_u32(sB + stage * kPairBBytes), 8192);
         constexpr uint32_t hi = sdesc_hi(1024);
+        if (leader) {
 #pragma unroll
-        for (int k = 0; k < kGemmBK / 16; ++k)
-          umma_ss_pair(d_tmem, a_lo + 2 * k, hi, b_lo + 128 * k, hi, idesc,
-                       (kb | k) != 0 ? 1u : 0u);
-        umma_commit_pair_mc(empty0 + 8 * stage, 0x3);
+          for (int k = 0; k < kGemmBK / 16; ++k)
+            umma_ss_pair(d_tmem, a_lo + 2 * k, hi, b_lo + 128 * k, hi, idesc,
+                         (kb | k) != 0 ? 1u : 0u);
+          umma_commit_pair_mc(empty0 + 8 * stage, 0x3);
+        }
+        __syncwarp();
         if (++stage == kPairStages) {
           stage = 0;
           phase ^= 1u;
         }
       }
       if (!ok) break;
-      umma_commit_pair_mc(accf0 + 8 * acc, 0x3);
+      if (leader) umma_commit_pair_mc(accf0 + 8 * acc, 0x3);
+      __syncwarp();
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1u;
       }
     }
-    umma_commit_pair(drain);
+    if (leader) umma_commit_pair(drain);
+    __syncwarp();
     mbar_wait_drain(drain, 0, p.err);
   } else if (warp >= 4) {
     // ------------------------------------------- epilogue (both CTAs)
