@@ -153,13 +153,8 @@ Plan make_plan(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff, int cau
   return p;
 }
 
-// ------------------------------------------------------------ device info --
-// GEMM kernel: CTA pairs (cta_group::2, 256x256 tiles) unless built with
-// -DBPT_GEMM_PAIR=0 (one CTA per 128x256 tile).
-#ifndef BPT_GEMM_PAIR
-#define BPT_GEMM_PAIR 1
-#endif
 
+// ------------------------------------------------------------ device info --
 struct DeviceInfo {
   bool init = false;
   bool ok = false;
@@ -183,10 +178,7 @@ bpt_status device_info(int* sms, int* pair_clusters = nullptr) {
     di.ok = (major == 10 && minor == 0);
     di.sms = n;
     if (di.ok) {
-      if (cudaFuncSetAttribute(bpt::gemm_f16_tc_kernel,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               bpt::kGemmSmem) != cudaSuccess ||
-          cudaFuncSetAttribute(bpt::attn_pair_tc_kernel<64, kEmu64>,
+      if (cudaFuncSetAttribute(bpt::attn_pair_tc_kernel<64, kEmu64>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                bpt::AttnPairCfg<64, kEmu64>::SMEM) != cudaSuccess ||
           cudaFuncSetAttribute(bpt::attn_pair_tc_kernel<128, kEmu128>,
@@ -253,19 +245,21 @@ bool encode_f16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims
   return r == CUDA_SUCCESS;
 }
 
-// A operand: [rows, K] row-major, 128 x 64 boxes.
+// GEMM A operand: [rows, K] row-major, viewed as [K/64][rows][64]; a box is
+// 128 rows x two 64-column chunks (32 KB, chunk-major in shared memory).
 bool map_a(CUtensorMap* m, const void* base, int64_t rows, int64_t K) {
-  const uint64_t dims[2] = {uint64_t(K), uint64_t(rows)};
-  const uint64_t st[1] = {uint64_t(K) * 2};
-  const uint32_t box[2] = {64, 128};
-  return encode_f16(m, base, 2, dims, st, box);
+  const uint64_t dims[3] = {64, uint64_t(rows), uint64_t(K / 64)};
+  const uint64_t st[2] = {uint64_t(K) * 2, 128};
+  const uint32_t box[3] = {64, 128, 2};
+  return encode_f16(m, base, 3, dims, st, box);
 }
-// B operand: [K, cols] row-major, 64 x 64 boxes.
-bool map_b(CUtensorMap* m, const void* base, int64_t K, int64_t cols) {
-  const uint64_t dims[2] = {uint64_t(cols), uint64_t(K)};
-  const uint64_t st[1] = {uint64_t(cols) * 2};
-  const uint32_t box[2] = {64, 64};
-  return encode_f16(m, base, 2, dims, st, box);
+// GEMM B operand: [K, cols] row-major, viewed as [cols/64][K][64]; a box is
+// 128 K rows x `chunks` 64-column chunks (chunk-major in shared memory).
+bool map_b(CUtensorMap* m, const void* base, int64_t K, int64_t cols, int chunks) {
+  const uint64_t dims[3] = {64, uint64_t(K), uint64_t(cols / 64)};
+  const uint64_t st[2] = {uint64_t(cols) * 2, 128};
+  const uint32_t box[3] = {64, 128, uint32_t(chunks)};
+  return encode_f16(m, base, 3, dims, st, box);
 }
 // QKV viewed as [B][N][3d]: boxes of 64 columns x 128 tokens x 1 sequence.
 bool map_qkv(CUtensorMap* m, const void* base, int64_t B, int64_t N, int64_t d) {
@@ -344,7 +338,6 @@ cudaError_t launch_ln(const TIn* in, const TP* ln, TOut* out, int64_t rows, int6
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                         const CUtensorMap& b2, const bpt::GemmParams& gp, int sms,
                         cudaStream_t s) {
-#if BPT_GEMM_PAIR
   int dummy = 0, pairs_max = 0;
   if (device_info(&dummy, &pairs_max) != BPT_OK) return cudaErrorInvalidDevice;
   const int64_t tiles = int64_t((gp.M + bpt::kPairBM - 1) / bpt::kPairBM) *
@@ -352,12 +345,6 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUten
   const unsigned pairs = unsigned(std::max<int64_t>(1, std::min<int64_t>(tiles, pairs_max)));
   bpt::gemm_f16_pair_kernel<<<2 * pairs, bpt::kGemmThreads, bpt::kPairSmem, s>>>(a, b0, b1, b2,
                                                                                  gp);
-#else
-  const int64_t tiles = int64_t((gp.M + bpt::kGemmBM - 1) / bpt::kGemmBM) *
-                        int64_t((gp.N + bpt::kGemmBN - 1) / bpt::kGemmBN);
-  const unsigned grid = unsigned(std::min<int64_t>(tiles, sms));
-  bpt::gemm_f16_tc_kernel<<<grid, bpt::kGemmThreads, bpt::kGemmSmem, s>>>(a, b0, b1, b2, gp);
-#endif
   return cudaGetLastError();
 }
 
@@ -394,10 +381,14 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
   const int64_t R = P.P * P.blk;  // scratch rows
 
   CUtensorMap mXn, mWq, mWk, mWv, mQKV, mO, mWo, mV, mW1, mH, mW2;
-  bool ok = map_a(&mXn, xn, M, d) && map_b(&mWq, wq, d, d) && map_b(&mWk, wk, d, d) &&
-            map_b(&mWv, wv, d, d) && map_qkv(&mQKV, qkv, P.B, P.N, d) && map_a(&mO, so, R, d) &&
-            map_b(&mWo, wo, d, d) && map_a(&mV, sv, R, d) && map_b(&mW1, w1, d, d_ff) &&
-            map_a(&mH, sh, R, d_ff) && map_b(&mW2, w2, d_ff, d);
+  // A CTA's 128 B columns stay inside one of W_Q | W_K | W_V when d is a
+  // multiple of 128 (one two-chunk box); otherwise it loads one chunk per box.
+  const int qkv_chunks = (d % 128 == 0) ? 2 : 1;
+  bool ok = map_a(&mXn, xn, M, d) && map_b(&mWq, wq, d, d, qkv_chunks) &&
+            map_b(&mWk, wk, d, d, qkv_chunks) && map_b(&mWv, wv, d, d, qkv_chunks) &&
+            map_qkv(&mQKV, qkv, P.B, P.N, d) && map_a(&mO, so, R, d) &&
+            map_b(&mWo, wo, d, d, 2) && map_a(&mV, sv, R, d) && map_b(&mW1, w1, d, d_ff, 2) &&
+            map_a(&mH, sh, R, d_ff) && map_b(&mW2, w2, d_ff, d, 2);
   if (!ok) return BPT_ERR_CUDA;
 
   {
@@ -428,7 +419,7 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
   {
     bpt::GemmParams g{};
     g.M = int(M); g.N = int(3 * d); g.K = int(d);
-    g.n_sub = int(d); g.n_maps = 3;
+    g.n_sub = int(d); g.n_maps = 3; g.b_chunks = qkv_chunks;
     g.epi = bpt::kEpiStoreF16;
     g.out_h = qkv; g.ld_out = 3 * d;
     g.map = ident;
@@ -469,7 +460,7 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
     {
       bpt::GemmParams g{};
       g.M = int(rows); g.N = int(d); g.K = int(d);
-      g.n_sub = int(d); g.n_maps = 1;
+      g.n_sub = int(d); g.n_maps = 1; g.b_chunks = 2;
       g.epi = bpt::kEpiResidX;
       g.out_f32 = out; g.ld_f32 = d;
       g.resid = static_cast<const bf*>(x); g.ld_resid = d;
@@ -486,7 +477,7 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
     {
       bpt::GemmParams g{};
       g.M = int(rows); g.N = int(d_ff); g.K = int(d);
-      g.n_sub = int(d_ff); g.n_maps = 1;
+      g.n_sub = int(d_ff); g.n_maps = 1; g.b_chunks = 2;
       g.epi = bpt::kEpiGeluBias;
       g.out_h = sh; g.ld_out = d_ff;
       g.bias = static_cast<const bf*>(b_1);
@@ -497,7 +488,7 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
     {
       bpt::GemmParams g{};
       g.M = int(rows); g.N = int(d); g.K = int(d_ff);
-      g.n_sub = int(d); g.n_maps = 1;
+      g.n_sub = int(d); g.n_maps = 1; g.b_chunks = 2;
       g.epi = bpt::kEpiBiasAccum;
       g.out_f32 = out; g.ld_f32 = d;
       g.bias = static_cast<const bf*>(b_2);

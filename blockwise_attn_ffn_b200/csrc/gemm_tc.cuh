@@ -1,17 +1,26 @@
-// Persistent tcgen05 GEMM with fused epilogues: C[M, N] = A[M, K] * B[K, N].
+// Persistent tcgen05 GEMM with fused epilogues: C[M, N] = A[M, K] * B[K, N],
+// on CTA pairs (tcgen05.mma.cta_group::2, 256 x 256 output tiles).
 //
-//   A: fp16 [M, K] row-major (K contiguous), loaded by TMA as 128 x 64 tiles
-//      with the 128-byte swizzle -> K-major UMMA operand.
-//   B: fp16 [K, N] row-major (N contiguous; weights are [d_in, d_out]) loaded
-//      as four 64(N) x 64(K) boxes -> MN-major UMMA operand, no transpose.
-//      B may be the column concatenation of up to three matrices with the
-//      same number of columns each (W_Q | W_K | W_V).
-//   Accumulator: fp32 128 x 256 tile in tensor memory, double buffered, so
-//      the epilogue of one tile overlaps the main loop of the next.
+//   A: fp16 [M, K] row-major (K contiguous) -> K-major UMMA operand, 128-byte
+//      swizzle.  Viewed by its tensor map as [K/64][M][64] so that one TMA
+//      box brings 128 rows x 128 K (two 64-column chunks, 32 KB).
+//   B: fp16 [K, N] row-major (N contiguous; weights are [d_in, d_out]) ->
+//      MN-major UMMA operand, no transpose.  Viewed as [N/64][K][64]: one box
+//      brings 128 K rows x 128 N (two 64-column chunks, 32 KB).  B may be the
+//      column concatenation of up to three matrices with the same number of
+//      columns each (W_Q | W_K | W_V); when that number is not a multiple of
+//      128 a CTA's 128 columns can straddle two of them, and it loads one
+//      chunk per box instead.
+//   One TMA box costs a CTA ~400 clocks whatever its size (measured), so
+//   boxes are 32 KB: 16 KB boxes delivered ~40 B/clk per SM, 32 KB ~75.
+//   Accumulator: fp32 256 x 256 tile (128 rows per CTA) in tensor memory,
+//      double buffered, so the epilogue of one tile overlaps the main loop of
+//      the next.
 //
-// Warp roles (256 threads): warp 0 issues TMA loads, warp 1 issues UMMA,
-// warp 2 owns the tensor-memory allocation, warps 4..7 run the epilogue (warp
-// 4+e reads TMEM lanes 32e..32e+31, i.e. accumulator rows 32e..32e+31).
+// Warp roles (256 threads per CTA): warp 0 issues TMA loads, warp 1 issues
+// UMMA (leader CTA), warp 2 owns the tensor-memory allocation, warps 4..7 run
+// the epilogue (warp 4+e reads TMEM lanes 32e..32e+31, i.e. accumulator rows
+// 32e..32e+31 of this CTA's 128).
 //
 // Epilogues (all in fp32 before the final rounding):
 //   kEpiStoreF16    out_h[row, col]  = acc                       (QKV, fp16)
@@ -33,6 +42,7 @@ struct GemmParams {
   int M, N, K;     // problem size (N, K multiples of 64)
   int n_sub;       // columns of each concatenated B matrix
   int n_maps;      // B matrices in use (1..3)
+  int b_chunks;    // 64-column chunks per B box: 2, or 1 if n_sub % 128 != 0
   int epi;
   __half* out_h;
   long long ld_out;
@@ -46,26 +56,11 @@ struct GemmParams {
   int fault;  // test hook: 1 = CTA 0 never loads its first stage (a lost arrive)
 };
 
-constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 64, kGemmStages = 4;
-constexpr int kGemmABytes = kGemmBM * kGemmBK * 2;  // 16 KB
-constexpr int kGemmBBytes = kGemmBK * kGemmBN * 2;  // 32 KB
-constexpr int kGemmStageBytes = kGemmABytes + kGemmBBytes;
+constexpr int kGemmBN = 256;  // output columns per tile
+constexpr int kGemmBK = 128;  // K depth of one pipeline stage
 constexpr int kGemmBarrierBytes = 256;
-constexpr int kGemmSmem = kGemmStages * kGemmStageBytes + kGemmBarrierBytes + 1024;
 constexpr int kGemmThreads = 256;
-constexpr int kGemmGroupM = 16;  // row blocks per rasterisation group (L2 reuse)
 constexpr uint32_t kGemmTmemCols = 512;
-
-__device__ __forceinline__ void gemm_tile_coords(int tile, int m_blocks, int n_blocks, int& mb,
-                                                 int& nb) {
-  const int per_group = kGemmGroupM * n_blocks;
-  const int group = tile / per_group;
-  const int first_m = group * kGemmGroupM;
-  const int gm = min(kGemmGroupM, m_blocks - first_m);
-  const int in = tile - group * per_group;
-  mb = first_m + in % gm;
-  nb = in / gm;
-}
 
 // Epilogue of one accumulator row (this thread's TMEM lane): 256 columns
 // starting at global column col_base, read in 32-column chunks.  Every lane of
@@ -150,176 +145,13 @@ __device__ __forceinline__ void gemm_epilogue_row(const GemmParams& p, uint32_t 
     record_error(p.err, kErrRange, p.epi == kEpiGeluBias ? kSiteRangeHidden : kSiteRangeQKV);
 }
 
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_f16_tc_kernel(const __grid_constant__ CUtensorMap mapA,
-                        const __grid_constant__ CUtensorMap mapB0,
-                        const __grid_constant__ CUtensorMap mapB1,
-                        const __grid_constant__ CUtensorMap mapB2, const GemmParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + kGemmStages * kGemmABytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kGemmStages * kGemmStageBytes);
-  // barrier slots
-  const uint32_t full0 = smem_u32(bars + 0);
-  const uint32_t empty0 = smem_u32(bars + kGemmStages);
-  const uint32_t accf0 = smem_u32(bars + 2 * kGemmStages);
-  const uint32_t acce0 = smem_u32(bars + 2 * kGemmStages + 2);
-  const uint32_t drain = smem_u32(bars + 2 * kGemmStages + 4);
-  __shared__ uint32_t tmem_base_sh;
-  __shared__ int abort_sh;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m_blocks = (p.M + kGemmBM - 1) / kGemmBM;
-  const int n_blocks = (p.N + kGemmBN - 1) / kGemmBN;
-  const int k_blocks = p.K / kGemmBK;
-  const int tiles = m_blocks * n_blocks;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kGemmStages; ++s) {
-      mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(accf0 + 8 * b, 1);
-      mbar_init(acce0 + 8 * b, 4);
-    }
-    mbar_init(drain, 1);
-    abort_sh = 0;
-    fence_mbar_init();
-  }
-  if (warp == 2) {
-    tmem_alloc(smem_u32(&tmem_base_sh), kGemmTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = tmem_base_sh;
-  volatile int* abort_flag = &abort_sh;
-
-  if (warp == 0 && lane == 0) {
-    // ------------------------------------------------------------ producer
-    tma_prefetch_desc(&mapA);
-    tma_prefetch_desc(&mapB0);
-    if (p.n_maps > 1) tma_prefetch_desc(&mapB1);
-    if (p.n_maps > 2) tma_prefetch_desc(&mapB2);
-    int armed[kGemmStages];
-    for (int s = 0; s < kGemmStages; ++s) armed[s] = -1;
-    int stage = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-      int mb, nb;
-      gemm_tile_coords(tile, m_blocks, n_blocks, mb, nb);
-      for (int kb = 0; kb < k_blocks; ++kb) {
-        if (!mbar_wait_fast(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.err, kSiteGemmProducer)) {
-          ok = false;
-          break;
-        }
-        const uint32_t fb = full0 + 8 * stage;
-        const bool lost = p.fault == 1 && blockIdx.x == 0 && tile == blockIdx.x && kb == 0;
-        if (!lost) {
-          mbar_arrive_expect_tx(fb, kGemmStageBytes);
-          armed[stage] = static_cast<int>(phase);
-          tma_load_2d(smem_u32(sA + stage * kGemmABytes), &mapA, fb, kb * kGemmBK, mb * kGemmBM);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int c = nb * kGemmBN + q * 64;
-            int which = c / p.n_sub;
-            if (which > p.n_maps - 1) which = p.n_maps - 1;  // past the end: TMA zero-fills
-            const CUtensorMap* mB = which == 0 ? &mapB0 : (which == 1 ? &mapB1 : &mapB2);
-            tma_load_2d(smem_u32(sB + stage * kGemmBBytes + q * 8192), mB, fb, c - which * p.n_sub,
-                        kb * kGemmBK);
-          }
-        }
-        if (++stage == kGemmStages) {
-          stage = 0;
-          phase ^= 1u;
-        }
-      }
-    }
-    // Drain: every load this thread armed has landed before the CTA exits.
-    for (int s = 0; s < kGemmStages; ++s)
-      if (armed[s] >= 0) mbar_wait_drain(full0 + 8 * s, static_cast<uint32_t>(armed[s]), p.err);
-  } else if (warp == 1 && lane == 0) {
-    // ----------------------------------------------------------- UMMA issue
-    constexpr uint32_t idesc = idesc_f16_f32(kGemmBM, kGemmBN, false, true);
-    int stage = 0;
-    uint32_t phase = 0;
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-      if (!mbar_wait_fast(acce0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.err, kSiteGemmMma)) break;
-      tc_fence_after();
-      const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * kGemmBN);
-      for (int kb = 0; kb < k_blocks; ++kb) {
-        if (!mbar_wait_fast(full0 + 8 * stage, phase, abort_flag, p.err, kSiteGemmMma)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t a_lo = sdesc_lo(smem_u32(sA + stage * kGemmABytes), 16);
-        const uint32_t b_lo = sdesc_lo(smem_u32(sB + stage * kGemmBBytes), 8192);
-        constexpr uint32_t hi = sdesc_hi(1024);
-#pragma unroll
-        for (int k = 0; k < kGemmBK / 16; ++k)
-          umma_ss(d_tmem, a_lo + 2 * k, hi, b_lo + 128 * k, hi, idesc, (kb | k) != 0 ? 1u : 0u);
-        umma_commit(empty0 + 8 * stage);
-        if (++stage == kGemmStages) {
-          stage = 0;
-          phase ^= 1u;
-        }
-      }
-      if (!ok) break;
-      umma_commit(accf0 + 8 * acc);
-      if (++acc == 2) {
-        acc = 0;
-        acc_phase ^= 1u;
-      }
-    }
-    // Drain: all issued UMMA complete before tensor memory is released.
-    umma_commit(drain);
-    mbar_wait_drain(drain, 0, p.err);
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------- epilogue
-    const int e = warp - 4;
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
-      int mb, nb;
-      gemm_tile_coords(tile, m_blocks, n_blocks, mb, nb);
-      if (!mbar_wait_fast(accf0 + 8 * acc, acc_phase, abort_flag, p.err, kSiteGemmEpilogue)) break;
-      tc_fence_after();
-      const long long row = static_cast<long long>(mb) * kGemmBM + e * 32 + lane;
-      const uint32_t t_row = tmem + (static_cast<uint32_t>(e * 32) << 16) +
-                             static_cast<uint32_t>(acc * kGemmBN);
-      gemm_epilogue_row(p, t_row, row, nb * kGemmBN);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acce0 + 8 * acc);
-      if (++acc == 2) {
-        acc = 0;
-        acc_phase ^= 1u;
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 2) tmem_dealloc(tmem, kGemmTmemCols);
-}
-
 // ---------------------------------------------------------------------------
-// CTA-pair variant: a cluster of two CTAs on two SMs computes one 256 x 256
-// output tile with tcgen05.mma.cta_group::2 (M = 256).  Each CTA loads its own
-// 128 rows of A and its half (128 columns) of the 256-column B slab, so per SM
-// a 64-deep k-block is 32 KB of shared memory instead of 48 KB: six stages
-// fit, and B traffic per SM halves.  Each CTA's tensor memory holds its own
-// 128 accumulator rows (two 256-column buffers), read by its own epilogue.
+// A cluster of two CTAs on two SMs computes one 256 x 256 output tile with
+// tcgen05.mma.cta_group::2 (M = 256).  Each CTA loads its own 128 rows of A
+// and its half (128 columns) of the 256-column B slab: a 128-deep stage is
+// 64 KB per CTA (one 32 KB box of A, one of B), three stages.  Each CTA's
+// tensor memory holds its own 128 accumulator rows (two 256-column buffers),
+// read by its own epilogue.
 //
 // Protocol (CTA rank 0 = leader, rank 1 = peer):
 //   full[s]   leader only; the leader's producer arms it with the bytes of
@@ -329,9 +161,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 //   acce[b]   leader only, 8 arrivals: the four epilogue warps of each CTA.
 // No TMA load uses cluster multicast.  The pair starts and ends with a
 // cluster barrier, so neither CTA frees memory the other may still signal.
-constexpr int kPairStages = 6;
-constexpr int kPairABytes = 128 * kGemmBK * 2;  // 16 KB: this CTA's 128 rows
-constexpr int kPairBBytes = kGemmBK * 128 * 2;  // 16 KB: this CTA's 128 columns
+constexpr int kPairStages = 3;
+constexpr int kPairABytes = 128 * kGemmBK * 2;  // 32 KB: this CTA's 128 rows, [2][128][64]
+constexpr int kPairBBytes = kGemmBK * 128 * 2;  // 32 KB: this CTA's 128 columns, [2][128][64]
 constexpr int kPairStageBytes = kPairABytes + kPairBBytes;
 constexpr int kPairSmem = kPairStages * kPairStageBytes + kGemmBarrierBytes + 1024;
 constexpr int kPairBM = 256;
@@ -362,7 +194,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const int npairs = static_cast<int>(nclusters_x());
   const int m_blocks = (p.M + kPairBM - 1) / kPairBM;
   const int n_blocks = (p.N + kGemmBN - 1) / kGemmBN;
-  const int k_blocks = p.K / kGemmBK;
+  const int k_blocks = (p.K + kGemmBK - 1) / kGemmBK;  // a half-empty last stage reads zeros
   const int tiles = m_blocks * n_blocks;
 
   if (threadIdx.x == 0) {
@@ -417,16 +249,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     for (int tile = pair; tile < tiles && ok; tile += npairs) {
       int mb, nb;
       coords(tile, mb, nb);
-      // This CTA's two 64-column B boxes: which weight map, and the column in it.
+      // This CTA's two 64-column B chunks: which weight map, and the chunk in it.
       const CUtensorMap* bmap[2];
-      int bcol[2];
+      int bchunk[2];
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
         const int c = nb * kGemmBN + static_cast<int>(rank) * 128 + q * 64;
         int which = c / p.n_sub;
         if (which > p.n_maps - 1) which = p.n_maps - 1;  // past the end: TMA zero-fills
         bmap[q] = which == 0 ? &mapB0 : (which == 1 ? &mapB1 : &mapB2);
-        bcol[q] = c - which * p.n_sub;
+        bchunk[q] = (c - which * p.n_sub) >> 6;
       }
       for (int kb = 0; kb < k_blocks; ++kb) {
         if (!mbar_wait_warp(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.err, kSiteGemmProducer)) {
@@ -439,12 +271,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           if (rank == 0) armed[stage] = static_cast<int>(phase);
           if (leader) {
             if (rank == 0) mbar_arrive_expect_tx(full0 + 8 * stage, 2 * kPairStageBytes);
-            tma_load_2d_pair(smem_u32(sA + stage * kPairABytes), &mapA, fb_leader, kb * kGemmBK,
-                             mb * kPairBM + static_cast<int>(rank) * 128);
+            tma_load_3d_pair(smem_u32(sA + stage * kPairABytes), &mapA, fb_leader, 0,
+                             mb * kPairBM + static_cast<int>(rank) * 128, kb * 2);
+            if (p.b_chunks == 2) {
+              tma_load_3d_pair(smem_u32(sB + stage * kPairBBytes), bmap[0], fb_leader, 0,
+                               kb * kGemmBK, bchunk[0]);
+            } else {
 #pragma unroll
-            for (int q = 0; q < 2; ++q)
-              tma_load_2d_pair(smem_u32(sB + stage * kPairBBytes + q * 8192), bmap[q], fb_leader,
-                               bcol[q], kb * kGemmBK);
+              for (int q = 0; q < 2; ++q)
+                tma_load_3d_pair(smem_u32(sB + stage * kPairBBytes + q * (kPairBBytes / 2)),
+                                 bmap[q], fb_leader, 0, kb * kGemmBK, bchunk[q]);
+            }
           }
         }
         if (++stage == kPairStages) {
@@ -486,14 +323,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           ok = false;
           break;
         }
+        // A: K-major, two 64-K chunks 16 KB apart; B: MN-major, LBO = the
+        // 16 KB between its two 64-column chunks; a 16-deep k-step moves 32 B
+        // in A and 16 rows (2 KB) in B.
         const uint32_t a_lo = sdesc_lo(smem_u32(sA + stage * kPairABytes), 16);
-        const uint32_t b_lo = sdesc_lo(smem_u32(sB + stage * kPairBBytes), 8192);
+        const uint32_t b_lo = sdesc_lo(smem_u32(sB + stage * kPairBBytes), kPairBBytes / 2);
         constexpr uint32_t hi = sdesc_hi(1024);
         if (leader) {
 #pragma unroll
           for (int k = 0; k < kGemmBK / 16; ++k)
-            umma_ss_pair(d_tmem, a_lo + 2 * k, hi, b_lo + 128 * k, hi, idesc,
-                         (kb | k) != 0 ? 1u : 0u);
+            umma_ss_pair(d_tmem, a_lo + (k >> 2) * ((kPairABytes / 2) >> 4) + 2 * (k & 3), hi,
+                         b_lo + 128 * k, hi, idesc, (kb | k) != 0 ? 1u : 0u);
           umma_commit_pair_mc(empty0 + 8 * stage, 0x3);
         }
         __syncwarp();

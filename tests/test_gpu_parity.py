@@ -32,6 +32,10 @@ SMALL = [
     small("dk128_bias_ragged", 1, 520, 384, 3, 768, True, bias=0.5),
     small("one_block", 1, 128, 128, 1, 256, True),
     small("single_token", 1, 1, 128, 2, 256, True),
+    # d and d_ff = 64 (mod 128): a GEMM CTA's 128 B columns straddle W_Q | W_K
+    # | W_V, every K leaves the last 128-deep stage half empty, and W_1's last
+    # column span is half past the end.
+    small("d192_straddle", 1, 260, 192, 3, 448, True, seed=13),
     small("f32_causal_ragged", 2, 150, 64, 2, 192, True, dtype="f32"),
     small("f32_noncausal_bias", 1, 100, 96, 3, 160, False, dtype="f32", bias=0.5),
 ]
@@ -52,7 +56,7 @@ def test_tiny_f32_workload():
     compare(got, oracle.layer_unfused(inp, cfg.h, cfg.causal), tol_for(cfg))
 
 
-@pytest.mark.parametrize("cfg", [SMALL[0], SMALL[2], SMALL[7]], ids=lambda c: c.name)
+@pytest.mark.parametrize("cfg", [SMALL[0], SMALL[2], SMALL[7], SMALL[8]], ids=lambda c: c.name)
 def test_qkv_projection_in_workspace(cfg):
     """Step a2 alone: the Q/K/V rows the prologue GEMM wrote."""
     inp = make_inputs(cfg)
