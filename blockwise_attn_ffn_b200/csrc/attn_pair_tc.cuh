@@ -240,14 +240,9 @@ __global__ void __launch_bounds__(384, 1)
     for (int s = 0; s < C::NSLOT; ++s) armed[s] = -1;
     if (leader) {
       mbar_arrive_expect_tx(q_full, C::TILE * (has_b ? 2 : 1));
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        tma_load_3d(smem_u32(smem + C::OFF_QA + c * C::CHUNK), &mapQKV, q_full, colQ + 64 * c,
-                    iA * C::BQ, bidx);
-        if (has_b)
-          tma_load_3d(smem_u32(smem + C::OFF_QB + c * C::CHUNK), &mapQKV, q_full,
-                      colQ + 64 * c, iB * C::BQ, bidx);
-      }
+      tma_load_4d(smem_u32(smem + C::OFF_QA), &mapQKV, q_full, 0, iA * C::BQ, colQ / 64, bidx);
+      if (has_b)
+        tma_load_4d(smem_u32(smem + C::OFF_QB), &mapQKV, q_full, 0, iB * C::BQ, colQ / 64, bidx);
     }
     int slot = 0;
     uint32_t phase = 0;
@@ -266,10 +261,8 @@ __global__ void __launch_bounds__(384, 1)
           const int col = w == 0 ? colK : colV;
           if (leader) {
             mbar_arrive_expect_tx(fb, C::TILE);
-#pragma unroll
-            for (int c = 0; c < D / 64; ++c)
-              tma_load_3d(smem_u32(smem + C::OFF_RING + slot * C::TILE + c * C::CHUNK), &mapQKV,
-                          fb, col + 64 * c, j * C::BKV, bidx);
+            tma_load_4d(smem_u32(smem + C::OFF_RING + slot * C::TILE), &mapQKV, fb, 0,
+                        j * C::BKV, col / 64, bidx);
           }
         }
         if (++slot == C::NSLOT) {

@@ -231,8 +231,8 @@ bpt_status get_encoder() {
 // fp16 tiles with the 128-byte swizzle; dims/strides innermost first.
 bool encode_f16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
                 const uint64_t* strides_bytes, const uint32_t* box) {
-  cuuint64_t gd[3], gs[2];
-  cuuint32_t bx[3], es[3] = {1, 1, 1};
+  cuuint64_t gd[4], gs[3];
+  cuuint32_t bx[4], es[4] = {1, 1, 1, 1};
   for (int i = 0; i < rank; ++i) {
     gd[i] = dims[i];
     bx[i] = box[i];
@@ -261,12 +261,14 @@ bool map_b(CUtensorMap* m, const void* base, int64_t K, int64_t cols, int chunks
   const uint32_t box[3] = {64, 128, uint32_t(chunks)};
   return encode_f16(m, base, 3, dims, st, box);
 }
-// QKV viewed as [B][N][3d]: boxes of 64 columns x 128 tokens x 1 sequence.
-bool map_qkv(CUtensorMap* m, const void* base, int64_t B, int64_t N, int64_t d) {
-  const uint64_t dims[3] = {uint64_t(3 * d), uint64_t(N), uint64_t(B)};
-  const uint64_t st[2] = {uint64_t(3 * d) * 2, uint64_t(N) * uint64_t(3 * d) * 2};
-  const uint32_t box[3] = {64, 128, 1};
-  return encode_f16(m, base, 3, dims, st, box);
+// QKV [B][N][3d] viewed as [B][3d/64][N][64]: a box is 128 tokens x the
+// d_k/64 chunks of one head's Q, K or V (32 KB at d_k = 128), chunk-major in
+// shared memory.
+bool map_qkv(CUtensorMap* m, const void* base, int64_t B, int64_t N, int64_t d, int64_t dk) {
+  const uint64_t dims[4] = {64, uint64_t(N), uint64_t(3 * d / 64), uint64_t(B)};
+  const uint64_t st[3] = {uint64_t(3 * d) * 2, 128, uint64_t(N) * uint64_t(3 * d) * 2};
+  const uint32_t box[4] = {64, 128, uint32_t(dk / 64), 1};
+  return encode_f16(m, base, 4, dims, st, box);
 }
 
 // -------------------------------------------------------------- profiling --
@@ -386,7 +388,7 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
   const int qkv_chunks = (d % 128 == 0) ? 2 : 1;
   bool ok = map_a(&mXn, xn, M, d) && map_b(&mWq, wq, d, d, qkv_chunks) &&
             map_b(&mWk, wk, d, d, qkv_chunks) && map_b(&mWv, wv, d, d, qkv_chunks) &&
-            map_qkv(&mQKV, qkv, P.B, P.N, d) && map_a(&mO, so, R, d) &&
+            map_qkv(&mQKV, qkv, P.B, P.N, d, P.dk) && map_a(&mO, so, R, d) &&
             map_b(&mWo, wo, d, d, 2) && map_a(&mV, sv, R, d) && map_b(&mW1, w1, d, d_ff, 2) &&
             map_a(&mH, sh, R, d_ff) && map_b(&mW2, w2, d_ff, d, 2);
   if (!ok) return BPT_ERR_CUDA;
