@@ -45,8 +45,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # digest covers the attention kernel, the shared device helpers and the host
 # launch code; after any change the bench reports null until it is retaken.
 ATTN_TRAFFIC = {
-    # 12 launches (6 forwards x 2 waves): waves of 405 + 113 and 1277 + 127 MB
-    "long_n64k": {"digest": "9e67c1468bf71264", "bytes_per_launch": 961234453},
+    # 12 launches (6 forwards x 2 waves): waves of 406 + 115 and 1281 + 130 MB
+    "long_n64k": {"digest": "ea4e1983acde9257", "bytes_per_launch": 967160533},
 }
 TRAFFIC_SOURCES = ("blockwise_attn_ffn_b200/csrc/attn_pair_tc.cuh",
                    "blockwise_attn_ffn_b200/csrc/common.cuh",
@@ -152,14 +152,56 @@ def cpu_oracle_rate(cfg, n_rows: int):
         threads = None
     inp = make_inputs(cfg, B=1)
     rows = sample_rows(cfg, n_rows, B=1)
+    cores = len(os.sched_getaffinity(0))
+    try:  # BLAS threads pinned to the cores this process may use
+        from threadpoolctl import threadpool_limits
+        limit = threadpool_limits(limits=cores)
+        threads = cores
+    except Exception:  # pragma: no cover
+        limit = None
     t0 = time.perf_counter()
     oracle.layer_rows(inp, cfg.h, cfg.causal, rows)
     dt = time.perf_counter() - t0
-    cores = len(os.sched_getaffinity(0))
+    if limit is not None:
+        limit.unregister()
     return {"value": len(rows) / dt, "unit": UNIT, "cores": threads or cores,
             "host_cores": cores, "kind": "oracle", "seconds": dt,
             "sample": f"{len(rows)} seeded rows of {cfg.name} (incl. row N-1, so K/V for all "
                       f"{cfg.N} keys) through oracle.layer_rows, fp64"}
+
+
+# ------------------------------------------------- unfused peak bytes --
+def unfused_torch_peak_bytes(cfg, p, dev):
+    """Peak device bytes of the plain unfused schedule, measured once outside
+    the timed region: LN, Q/K/V matmuls, PyTorch SDPA, W_O matmul + residual,
+    LN, W_1 matmul + GELU, W_2 matmul + residual, all materialised in bf16.
+    A bench-only measurement of the memory the pages' unfused schedule keeps
+    alive; nothing of the library runs here."""
+    import torch.nn.functional as F
+    B, N, d, h = cfg.B, cfg.N, cfg.d, cfg.h
+    torch.cuda.synchronize(dev)
+    base = torch.cuda.memory_allocated(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+    with torch.no_grad():
+        x = p["x"].view(B, N, d)
+        g1, b1n = p["ln1"][0], p["ln1"][1]
+        xn = F.layer_norm(x, (d,), g1, b1n, 1e-5)
+        q, k, v = xn @ p["W_Q"], xn @ p["W_K"], xn @ p["W_V"]
+        del xn
+        def heads(t):
+            return t.view(B, N, h, d // h).transpose(1, 2)
+        o = F.scaled_dot_product_attention(heads(q), heads(k), heads(v), is_causal=cfg.causal)
+        del q, k, v
+        o = o.transpose(1, 2).reshape(B, N, d)
+        y = x + o @ p["W_O"]
+        del o
+        yn = F.layer_norm(y, (d,), p["ln2"][0], p["ln2"][1], 1e-5)
+        hid = F.gelu(yn @ p["W_1"] + p["b_1"])
+        del yn
+        z = y + hid @ p["W_2"] + p["b_2"]
+        del hid, y, z
+    torch.cuda.synchronize(dev)
+    return int(torch.cuda.max_memory_allocated(dev) - base)
 
 
 # ------------------------------------------------------------- reference --
@@ -190,7 +232,7 @@ def run_reference(args, cfg, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="long_n64k", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="bpt", choices=["bpt", "reference"])
@@ -198,6 +240,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=1024)
     ap.add_argument("--ref-rows", type=int, default=16)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-unfused-peak", action="store_true",
+                    help="skip the bench-only unfused-schedule peak-bytes measurement")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="override the workload's N (profiling runs on a smaller case)")
     args = ap.parse_args()
@@ -258,15 +302,20 @@ def main():
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(dev)
+        step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps - 1)]
         ev0.record(stream)
-        for _ in range(args.steps):
+        for i in range(args.steps):
             bpt.layer_forward(x, p, cfg.h, cfg.causal, out=out, workspace=ws)
+            if i + 1 < args.steps:
+                step_ev[i].record(stream)
         ev1.record(stream)
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
     bpt.bpt_profile_enable(False)
     ms_total = ev0.elapsed_time(ev1)
+    marks = [ev0] + step_ev + [ev1]
+    per_step = [marks[i].elapsed_time(marks[i + 1]) for i in range(args.steps)]
     _, kind_ms, kind_n = bpt.bpt_profile_read()
     st, site = bpt.bpt_read_device_error(ws.data_ptr(), stream.cuda_stream)
     if st != bpt.BPT_OK:
@@ -319,6 +368,10 @@ def main():
         ms = kind_ms[k] / args.steps
         kernels[k]["tflops"] = f / (ms / 1e3) / 1e12 if ms > 0 else None
     tflops = flops["total"] * world / (ms_step / 1e3) / 1e12
+    # Step a1+a2 (LN1 + QKV projection): x, W_Q|W_K|W_V and QKV touched once.
+    esz_in = 2 if cfg.dtype == "bf16" else 4
+    kb1_bytes = cfg.B * cfg.N * cfg.d * esz_in + 3 * cfg.d * cfg.d * 2 + cfg.B * cfg.N * 3 * cfg.d * 2
+    kb1_ms = (kind_ms.get("ln1", 0.0) + kind_ms.get("qkv", 0.0)) / args.steps
     unfused = accounting.unfused_activation_elems(cfg.N, cfg.d, cfg.h, cfg.d_ff,
                                                   with_logits=False)
     esz = 2 if cfg.dtype == "bf16" else 4
@@ -336,6 +389,13 @@ def main():
         "tflops": tflops,
         "pct_bf16_peak": tflops / world / peaks["bf16_tflops"],
         "pct_bf16_peak_sustained": tflops / world / peak_sus,
+        "pct_nominal_2250": tflops / world / 2250.0,
+        "ms_per_step_median": float(np.median(per_step)),
+        "ms_per_step_min": float(np.min(per_step)),
+        "kb1_hbm": {"algorithmic_bytes": int(kb1_bytes),
+                    "achieved_gbs": kb1_bytes / (kb1_ms / 1e3) / 1e9 if kb1_ms > 0 else None,
+                    "peak_gbs": peaks["hbm_gbs"],
+                    "note": "LN1 + QKV projection kernels: x + W_QKV + QKV once / their time"},
         "peak_src": peak_src,
         "roofline": {"bound": "tensor", "kernel": "attn_pair_tc_kernel", "achieved": achieved,
                      "peak": peak_sus, "unit": "TFLOP/s", "frac": achieved / peak_sus,
@@ -353,6 +413,8 @@ def main():
     }
     with_clk = clk.summary()
     line["clocks"] = with_clk
+    if not args.no_unfused_peak and cfg.dtype == "bf16":
+        line["peak_bytes"]["unfused_torch_measured"] = unfused_torch_peak_bytes(cfg, p, dev)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_rate(cfg, args.cpu_rows)
