@@ -177,6 +177,7 @@ def unfused_torch_peak_bytes(cfg, p, dev):
     LN, W_1 matmul + GELU, W_2 matmul + residual, all materialised in bf16.
     A bench-only measurement of the memory the pages' unfused schedule keeps
     alive; nothing of the library runs here."""
+    import torch
     import torch.nn.functional as F
     B, N, d, h = cfg.B, cfg.N, cfg.d, cfg.h
     torch.cuda.synchronize(dev)
