@@ -184,19 +184,23 @@ bpt_status device_info(int* sms, int* pair_clusters = nullptr) {
           cudaFuncSetAttribute(bpt::attn_pair_tc_kernel<128, kEmu128>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                bpt::AttnPairCfg<128, kEmu128>::SMEM) != cudaSuccess ||
-          cudaFuncSetAttribute(bpt::gemm_f16_pair_kernel,
+          cudaFuncSetAttribute(bpt::gemm_f16_pair_kernel<4>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               bpt::kPairSmem) != cudaSuccess ||
+          cudaFuncSetAttribute(bpt::gemm_f16_pair_kernel<8>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                bpt::kPairSmem) != cudaSuccess ||
           cudaFuncSetAttribute(bpt::attn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (3 * 64 * 128 + 64 * 65) * 4) != cudaSuccess)
         return BPT_ERR_CUDA;
-      // How many CTA pairs of the pair GEMM fit on the device at once.
+      // How many CTA pairs of the pair GEMM fit on the device at once (the
+      // shared memory, not the thread count, limits it to one CTA per SM).
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(unsigned(2 * (n / 2)));
-      cfg.blockDim = dim3(bpt::kGemmThreads);
+      cfg.blockDim = dim3(bpt::gemm_threads<8>());
       cfg.dynamicSmemBytes = bpt::kPairSmem;
       int clusters = 0;
-      if (cudaOccupancyMaxActiveClusters(&clusters, bpt::gemm_f16_pair_kernel, &cfg) !=
+      if (cudaOccupancyMaxActiveClusters(&clusters, bpt::gemm_f16_pair_kernel<8>, &cfg) !=
               cudaSuccess ||
           clusters <= 0) {
         cudaGetLastError();
@@ -345,8 +349,12 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUten
   const int64_t tiles = int64_t((gp.M + bpt::kPairBM - 1) / bpt::kPairBM) *
                         int64_t((gp.N + bpt::kGemmBN - 1) / bpt::kGemmBN);
   const unsigned pairs = unsigned(std::max<int64_t>(1, std::min<int64_t>(tiles, pairs_max)));
-  bpt::gemm_f16_pair_kernel<<<2 * pairs, bpt::kGemmThreads, bpt::kPairSmem, s>>>(a, b0, b1, b2,
-                                                                                 gp);
+  if (gp.epi == bpt::kEpiGeluBias || gp.epi == bpt::kEpiResidX)
+    bpt::gemm_f16_pair_kernel<8>
+        <<<2 * pairs, bpt::gemm_threads<8>(), bpt::kPairSmem, s>>>(a, b0, b1, b2, gp);
+  else
+    bpt::gemm_f16_pair_kernel<4>
+        <<<2 * pairs, bpt::gemm_threads<4>(), bpt::kPairSmem, s>>>(a, b0, b1, b2, gp);
   return cudaGetLastError();
 }
 

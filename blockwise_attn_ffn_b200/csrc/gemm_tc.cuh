@@ -17,10 +17,14 @@
 //      double buffered, so the epilogue of one tile overlaps the main loop of
 //      the next.
 //
-// Warp roles (256 threads per CTA): warp 0 issues TMA loads, warp 1 issues
-// UMMA (leader CTA), warp 2 owns the tensor-memory allocation, warps 4..7 run
-// the epilogue (warp 4+e reads TMEM lanes 32e..32e+31, i.e. accumulator rows
-// 32e..32e+31 of this CTA's 128).
+// Warp roles (32 x (4 + EPI) threads per CTA): warp 0 issues TMA loads,
+// warp 1 issues UMMA (leader CTA), warp 2 owns the tensor-memory allocation,
+// warps 4.. run the epilogue.  With EPI = 4 warp w reads TMEM lanes
+// 32(w%4)..+31 (accumulator rows of this CTA's 128) and all 256 columns; with
+// EPI = 8 two warps share each lane quarter, 128 columns each.  The GELU and
+// residual epilogues (W_1, W_O) use 8: their per-element work would otherwise
+// outlast the next tile's main loop; the light ones use 4, whose fewer warps
+// leave the TMA and UMMA warps more issue slots.
 //
 // Epilogues (all in fp32 before the final rounding):
 //   kEpiStoreF16    out_h[row, col]  = acc                       (QKV, fp16)
@@ -59,14 +63,17 @@ struct GemmParams {
 constexpr int kGemmBN = 256;  // output columns per tile
 constexpr int kGemmBK = 128;  // K depth of one pipeline stage
 constexpr int kGemmBarrierBytes = 256;
-constexpr int kGemmThreads = 256;
+template <int EPI>
+constexpr int gemm_threads() {
+  return 32 * (4 + EPI);
+}
 constexpr uint32_t kGemmTmemCols = 512;
 
-// Epilogue of one accumulator row (this thread's TMEM lane): 256 columns
+// Epilogue of one accumulator row (this thread's TMEM lane): ncols columns
 // starting at global column col_base, read in 32-column chunks.  Every lane of
 // the warp must call it (tcgen05.ld is warp-collective).
 __device__ __forceinline__ void gemm_epilogue_row(const GemmParams& p, uint32_t t_row,
-                                                  long long row, int col_base) {
+                                                  long long row, int col_base, int ncols) {
   long long g = -1;
   bool row_ok;
   if (p.epi == kEpiStoreF16 || p.epi == kEpiGeluBias) {
@@ -77,7 +84,7 @@ __device__ __forceinline__ void gemm_epilogue_row(const GemmParams& p, uint32_t 
   }
   bool bad = false;
 #pragma unroll 1
-  for (int ch = 0; ch < kGemmBN / 32; ++ch) {
+  for (int ch = 0; ch < ncols / 32; ++ch) {
     uint32_t r[32];
     tmem_ld_32x32b_x32(t_row + ch * 32, r);
     tmem_ld_wait();
@@ -158,7 +165,7 @@ __device__ __forceinline__ void gemm_epilogue_row(const GemmParams& p, uint32_t 
 //             both CTAs; both CTAs' TMA loads complete on it.
 //   empty[s]  both CTAs; the leader's UMMA commit arrives on both (multicast).
 //   accf[b]   both CTAs; the leader's UMMA commit arrives on both (multicast).
-//   acce[b]   leader only, 8 arrivals: the four epilogue warps of each CTA.
+//   acce[b]   leader only, 2 x EPI arrivals: the epilogue warps of both CTAs.
 // No TMA load uses cluster multicast.  The pair starts and ends with a
 // cluster barrier, so neither CTA frees memory the other may still signal.
 constexpr int kPairStages = 3;
@@ -169,7 +176,8 @@ constexpr int kPairSmem = kPairStages * kPairStageBytes + kGemmBarrierBytes + 10
 constexpr int kPairBM = 256;
 constexpr int kPairGroupM = 8;  // 256-row blocks per rasterisation group
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(), 1)
     gemm_f16_pair_kernel(const __grid_constant__ CUtensorMap mapA,
                          const __grid_constant__ CUtensorMap mapB0,
                          const __grid_constant__ CUtensorMap mapB1,
@@ -204,7 +212,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(accf0 + 8 * b, 1);
-      mbar_init(acce0 + 8 * b, 8);
+      mbar_init(acce0 + 8 * b, 2 * EPI);
     }
     mbar_init(drain, 1);
     abort_sh = 0;
@@ -355,7 +363,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     mbar_wait_drain(drain, 0, p.err);
   } else if (warp >= 4) {
     // ------------------------------------------- epilogue (both CTAs)
-    const int e = warp - 4;
+    const int e = warp & 3;                        // TMEM lane quarter
+    constexpr int kCols = kGemmBN * 4 / EPI;       // columns per epilogue warp
+    const int part = (warp - 4) >> 2;              // which kCols-column part
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = pair; tile < tiles; tile += npairs) {
@@ -366,8 +376,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const long long row =
           static_cast<long long>(mb) * kPairBM + static_cast<long long>(rank) * 128 + e * 32 + lane;
       const uint32_t t_row = tmem + (static_cast<uint32_t>(e * 32) << 16) +
-                             static_cast<uint32_t>(acc * kGemmBN);
-      gemm_epilogue_row(p, t_row, row, nb * kGemmBN);
+                             static_cast<uint32_t>(acc * kGemmBN + part * kCols);
+      gemm_epilogue_row(p, t_row, row, nb * kGemmBN + part * kCols, kCols);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(map_to_rank(acce0 + 8 * acc, 0));
