@@ -26,6 +26,7 @@ EXPORTED = [
     "bpt_layer_workspace_size", "bpt_layer_forward", "bpt_read_device_error",
     "bpt_status_string", "bpt_profile_enable", "bpt_profile_read",
     "bpt_layer_launch_count", "bpt_layer_forward_static", "bpt_debug_inject_fault",
+    "bpt_layer_forward_train",
 ]
 
 _lib: Optional[ctypes.CDLL] = None
@@ -52,6 +53,9 @@ def load() -> ctypes.CDLL:
     lib.bpt_layer_workspace_size.restype = i32
     lib.bpt_layer_forward.argtypes = [vp] * 11 + [i64] * 5 + [i32, i32, vp, vp, ctypes.c_size_t, vp]
     lib.bpt_layer_forward.restype = i32
+    lib.bpt_layer_forward_train.argtypes = ([vp] * 11 + [i64] * 5 +
+                                            [i32, i32, vp, vp, vp, ctypes.c_size_t, vp])
+    lib.bpt_layer_forward_train.restype = i32
     lib.bpt_read_device_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     lib.bpt_read_device_error.restype = i32
     lib.bpt_status_string.argtypes = [i32]
@@ -92,6 +96,15 @@ def bpt_layer_forward(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
     return load().bpt_layer_forward(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
                                     B, N, d, h, d_ff, int(bool(causal)), dtype, out,
                                     workspace, workspace_bytes, stream)
+
+
+def bpt_layer_forward_train(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
+                            B, N, d, h, d_ff, causal, dtype, out, stats, workspace,
+                            workspace_bytes, stream) -> int:
+    """Pointer-level call; returns the status code."""
+    return load().bpt_layer_forward_train(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
+                                          B, N, d, h, d_ff, int(bool(causal)), dtype, out,
+                                          stats, workspace, workspace_bytes, stream)
 
 
 def bpt_read_device_error(workspace, stream) -> Tuple[int, int]:

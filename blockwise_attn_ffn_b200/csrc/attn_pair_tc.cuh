@@ -62,6 +62,7 @@ struct AttnPairParams {
                // K/V that concurrent CTAs sweep is that of hg heads only
   __half* o;         // [count * 128, d] block scratch (fp16)
   float scale_log2;  // log2(e) / sqrt(d_k)
+  float2* stats;     // nullable: per-row softmax statistics [B][h][N] (m, l)
   uint32_t* err;
   int fault;         // test hook: 2 = CTA 0 never loads V_0 (a lost arrive)
 };
@@ -387,7 +388,8 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t s_full = s_full0 + 8 * x, p_full = p_full0 + 8 * x, o_done = o_done0 + 8 * x;
     const float c = p.scale_log2;
     const bool ragged = (p.N % C::BKV) != 0;
-    float m_run = -INFINITY;
+    float m_run = -INFINITY;  // reference maximum (moves only by > 2^8 in exp2 units)
+    float m_true = -INFINITY;  // exact running row maximum, for the statistics
     float l = 0.f;
     bool ok = nX > 0;
     for (int j = 0; j < nX && ok; ++j) {
@@ -421,6 +423,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int k = 0; k < 4; ++k) mxp[k] = fmaxf(mxp[k], mxp[k + 4]);
       const float mx = fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3]));
+      m_true = fmaxf(m_true, mx);
       float m_new = m_run;
       bool need = false;
       if (mx > m_run) {
@@ -485,6 +488,17 @@ __global__ void __launch_bounds__(384, 1)
     if (ok && mbar_wait_fast(o_done, 0, abort_flag, p.err, kSiteAttnSoftmax)) {
       tc_fence_after();
       const float inv_l = 1.0f / l;
+      if (p.stats != nullptr) {
+        // (m, l) of the row in the units of s = q.k / sqrt(d_k): m the exact
+        // maximum over its allowed keys, l = sum exp(s - m) (l was kept
+        // relative to the reference maximum m_run <= m_true).
+        const int pos = iX * C::BQ + r;
+        if (pos < p.N) {
+          const float m_s = m_true * p.scale_log2 * 0.69314718055994531f;
+          const float l_s = l * ex2_approx((m_run - m_true) * p.scale_log2);
+          p.stats[(static_cast<long long>(bidx) * p.h + head) * p.N + pos] = make_float2(m_s, l_s);
+        }
+      }
       const long long srow = static_cast<long long>(itemA + x - p.item0) * C::BQ + r;
       __half* dst = p.o + srow * p.d + head * D;
 #pragma unroll 1

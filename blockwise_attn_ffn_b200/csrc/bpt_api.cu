@@ -363,7 +363,7 @@ bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) !
 bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const void* W_Q,
                         const void* W_K, const void* W_V, const void* W_O, const void* ln2,
                         const void* W_1, const void* b_1, const void* W_2, const void* b_2,
-                        float* out, uint8_t* ws, cudaStream_t s, int sms) {
+                        float* out, float* stats, uint8_t* ws, cudaStream_t s, int sms) {
   using bf = __nv_bfloat16;
   using hf = __half;
   const int64_t M = P.B * P.N, d = P.d, d_ff = P.d_ff;
@@ -448,6 +448,7 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
       ap.N = int(P.N); ap.nb = int(P.nb); ap.h = int(P.h); ap.d = int(d);
       ap.causal = P.causal; ap.item0 = int(wv_.item0); ap.count = int(wv_.count);
       ap.seqs = int(wv_.seqs); ap.o = so; ap.scale_log2 = scale_log2; ap.err = err;
+      ap.stats = reinterpret_cast<float2*>(stats);
       const int64_t kv_head = (wv_.seqs > 0 ? wv_.seqs : 1) * P.N * P.dk * 2 * 2;
       ap.hg = 1;
       for (int g = int(P.h); g > 1; --g)
@@ -513,7 +514,7 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
 bpt_status forward_f32(const Plan& P, const float* x, const float* ln1, const float* W_Q,
                        const float* W_K, const float* W_V, const float* W_O, const float* ln2,
                        const float* W_1, const float* b_1, const float* W_2, const float* b_2,
-                       float* out, uint8_t* ws, cudaStream_t s) {
+                       float* out, float* stats, uint8_t* ws, cudaStream_t s) {
   const int64_t M = P.B * P.N, d = P.d, d_ff = P.d_ff;
   float* qkv = reinterpret_cast<float*>(ws + P.off_qkv);
   float* so = reinterpret_cast<float*>(ws + P.off_o);
@@ -553,6 +554,7 @@ bpt_status forward_f32(const Plan& P, const float* x, const float* ln1, const fl
       ap.qkv = qkv; ap.o = so; ap.N = int(P.N); ap.nb = int(P.nb); ap.h = int(P.h);
       ap.d = int(d); ap.causal = P.causal; ap.item0 = int(wv.item0); ap.blk = int(P.blk);
       ap.scale = float(1.0 / std::sqrt(double(P.dk)));
+      ap.stats = stats;
       const size_t smem = size_t(3 * 64 * P.dk + 64 * 65) * 4;
       LaunchScope ls(BPT_KIND_ATTN, s);
       bpt::attn_f32_kernel<<<unsigned(wv.count * P.h), 256, smem, s>>>(ap);
@@ -577,6 +579,58 @@ bpt_status forward_f32(const Plan& P, const float* x, const float* ln1, const fl
 }
 
 }  // namespace
+
+// Shared body of bpt_layer_forward and bpt_layer_forward_train (stats may be
+// null: no statistics are written).
+bpt_status layer_forward_impl(const void* x, const void* ln1, const void* W_Q, const void* W_K,
+                              const void* W_V, const void* W_O, const void* ln2, const void* W_1,
+                              const void* b_1, const void* W_2, const void* b_2, int64_t B,
+                              int64_t N, int64_t d, int64_t h, int64_t d_ff, int causal,
+                              bpt_dtype dtype, float* out, float* stats, void* workspace,
+                              size_t workspace_bytes, bpt_stream_t stream) {
+  bpt_status st = check_shape(B, N, d, h, d_ff, causal, dtype);
+  if (st != BPT_OK) return st;
+  if (B == 0 || N == 0) return BPT_OK;
+  const void* ptrs[] = {x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, out, workspace};
+  for (const void* p : ptrs)
+    if (p == nullptr || misaligned(p)) return BPT_ERR_INVALID_ARG;
+  const Plan P = make_plan(B, N, d, h, d_ff, causal, dtype);
+  if (workspace_bytes < P.total) return BPT_ERR_WORKSPACE;
+  // out must not overlap x (it is written before x is last read)
+  const uintptr_t xo = reinterpret_cast<uintptr_t>(x), oo = reinterpret_cast<uintptr_t>(out);
+  const size_t xbytes = size_t(B * N * d) * P.esize, obytes = size_t(B * N * d) * 4;
+  if (xo < oo + obytes && oo < xo + xbytes) return BPT_ERR_INVALID_ARG;
+  const uintptr_t wo = reinterpret_cast<uintptr_t>(workspace);
+  if (wo < oo + obytes && oo < wo + P.total) return BPT_ERR_INVALID_ARG;
+  if (stats != nullptr) {
+    // stats must not overlap out, x or the workspace (all written or read here)
+    const uintptr_t so = reinterpret_cast<uintptr_t>(stats);
+    const size_t sbytes = size_t(B * h * N) * 2 * sizeof(float);
+    if (misaligned(stats) || (so < oo + obytes && oo < so + sbytes) ||
+        (so < xo + xbytes && xo < so + sbytes) || (so < wo + P.total && wo < so + sbytes))
+      return BPT_ERR_INVALID_ARG;
+  }
+
+  int sms = 0;
+  st = device_info(&sms);
+  if (st != BPT_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (cudaMemsetAsync(ws, 0, kHeaderBytes, s) != cudaSuccess) return BPT_ERR_CUDA;
+  if (dtype == BPT_BF16) {
+    st = get_encoder();
+    if (st != BPT_OK) return st;
+    return forward_bf16(P, x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, out, stats, ws, s,
+                        sms);
+  }
+  return forward_f32(P, static_cast<const float*>(x), static_cast<const float*>(ln1),
+                     static_cast<const float*>(W_Q), static_cast<const float*>(W_K),
+                     static_cast<const float*>(W_V), static_cast<const float*>(W_O),
+                     static_cast<const float*>(ln2), static_cast<const float*>(W_1),
+                     static_cast<const float*>(b_1), static_cast<const float*>(W_2),
+                     static_cast<const float*>(b_2), out, stats, ws, s);
+}
+
 
 extern "C" {
 
@@ -605,39 +659,22 @@ bpt_status bpt_layer_forward(const void* x, const void* ln1, const void* W_Q, co
                              int64_t N, int64_t d, int64_t h, int64_t d_ff, int causal,
                              bpt_dtype dtype, float* out, void* workspace, size_t workspace_bytes,
                              bpt_stream_t stream) {
-  bpt_status st = check_shape(B, N, d, h, d_ff, causal, dtype);
-  if (st != BPT_OK) return st;
-  if (B == 0 || N == 0) return BPT_OK;
-  const void* ptrs[] = {x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, out, workspace};
-  for (const void* p : ptrs)
-    if (p == nullptr || misaligned(p)) return BPT_ERR_INVALID_ARG;
-  const Plan P = make_plan(B, N, d, h, d_ff, causal, dtype);
-  if (workspace_bytes < P.total) return BPT_ERR_WORKSPACE;
-  // out must not overlap x (it is written before x is last read)
-  const uintptr_t xo = reinterpret_cast<uintptr_t>(x), oo = reinterpret_cast<uintptr_t>(out);
-  const size_t xbytes = size_t(B * N * d) * P.esize, obytes = size_t(B * N * d) * 4;
-  if (xo < oo + obytes && oo < xo + xbytes) return BPT_ERR_INVALID_ARG;
-  const uintptr_t wo = reinterpret_cast<uintptr_t>(workspace);
-  if (wo < oo + obytes && oo < wo + P.total) return BPT_ERR_INVALID_ARG;
-
-  int sms = 0;
-  st = device_info(&sms);
-  if (st != BPT_OK) return st;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  if (cudaMemsetAsync(ws, 0, kHeaderBytes, s) != cudaSuccess) return BPT_ERR_CUDA;
-  if (dtype == BPT_BF16) {
-    st = get_encoder();
-    if (st != BPT_OK) return st;
-    return forward_bf16(P, x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, out, ws, s, sms);
-  }
-  return forward_f32(P, static_cast<const float*>(x), static_cast<const float*>(ln1),
-                     static_cast<const float*>(W_Q), static_cast<const float*>(W_K),
-                     static_cast<const float*>(W_V), static_cast<const float*>(W_O),
-                     static_cast<const float*>(ln2), static_cast<const float*>(W_1),
-                     static_cast<const float*>(b_1), static_cast<const float*>(W_2),
-                     static_cast<const float*>(b_2), out, ws, s);
+  return layer_forward_impl(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, B, N, d, h, d_ff,
+                            causal, dtype, out, nullptr, workspace, workspace_bytes, stream);
 }
+
+bpt_status bpt_layer_forward_train(const void* x, const void* ln1, const void* W_Q,
+                                   const void* W_K, const void* W_V, const void* W_O,
+                                   const void* ln2, const void* W_1, const void* b_1,
+                                   const void* W_2, const void* b_2, int64_t B, int64_t N,
+                                   int64_t d, int64_t h, int64_t d_ff, int causal,
+                                   bpt_dtype dtype, float* out, float* stats, void* workspace,
+                                   size_t workspace_bytes, bpt_stream_t stream) {
+  if (stats == nullptr) return BPT_ERR_INVALID_ARG;
+  return layer_forward_impl(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, B, N, d, h, d_ff,
+                            causal, dtype, out, stats, workspace, workspace_bytes, stream);
+}
+
 
 bpt_status bpt_read_device_error(void* workspace, bpt_stream_t stream, uint32_t* site) {
   if (!workspace) return BPT_ERR_INVALID_ARG;

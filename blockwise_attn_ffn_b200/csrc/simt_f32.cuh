@@ -96,6 +96,7 @@ struct AttnF32Params {
   float* o;          // [count * blk, d]
   int N, nb, h, d, causal, item0, blk;
   float scale;       // 1 / sqrt(d_k)
+  float* stats;      // nullable: per-row softmax statistics [B][h][N][2] (m, l)
 };
 
 constexpr int kF32AttnRows = 64;     // query / key-value block
@@ -179,6 +180,11 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(const AttnF32Params p) {
   float* dst = p.o + srow * p.d + head * dk;
   const float inv = l > 0.f ? 1.0f / l : 0.f;
   for (int t = 0; t < dk / 4; ++t) dst[sub + 4 * t] = o[t] * inv;
+  if (p.stats != nullptr && sub == 0 && qpos < p.N) {
+    float* st = p.stats + ((static_cast<long long>(bidx) * p.h + head) * p.N + qpos) * 2;
+    st[0] = m;
+    st[1] = l;
+  }
 }
 
 }  // namespace bpt

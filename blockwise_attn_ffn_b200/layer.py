@@ -87,3 +87,35 @@ def layer_forward(x: torch.Tensor, p: Dict[str, torch.Tensor], h: int, causal: b
     if st != _lib.BPT_OK:
         raise _lib.BptError(st, "bpt_layer_forward")
     return out, workspace
+
+
+def layer_forward_train(x: torch.Tensor, p: Dict[str, torch.Tensor], h: int, causal: bool,
+                        out: Optional[torch.Tensor] = None,
+                        stats: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None,
+                        stream: Optional[torch.cuda.Stream] = None):
+    """``layer_forward`` that also returns the per-row softmax statistics via
+    ``bpt_layer_forward_train``: (out, stats, workspace), stats [B, h, N, 2]
+    fp32 holding (m, l) per (batch, head, query row)."""
+    if x.dim() != 3:
+        raise ValueError("x must be [B, N, d]")
+    B, N, d = x.shape
+    d_ff = p["W_1"].shape[1]
+    code = _dtype_code(x)
+    tensors = [x] + [p[k] for k in PARAM_NAMES]
+    for t in tensors:
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != x.dtype:
+            raise ValueError("inputs must be contiguous CUDA tensors of one dtype")
+    if out is None:
+        out = torch.empty((B, N, d), dtype=torch.float32, device=x.device)
+    if stats is None:
+        stats = torch.empty((B, h, N, 2), dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = workspace_for(B, N, d, h, d_ff, causal, x.dtype, x.device)
+    s = stream if stream is not None else torch.cuda.current_stream(x.device)
+    st = _lib.bpt_layer_forward_train(*[t.data_ptr() for t in tensors], B, N, d, h, d_ff, causal,
+                                      code, out.data_ptr(), stats.data_ptr(),
+                                      workspace.data_ptr(), workspace.numel(), s.cuda_stream)
+    if st != _lib.BPT_OK:
+        raise _lib.BptError(st, "bpt_layer_forward_train")
+    return out, stats, workspace

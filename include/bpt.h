@@ -127,6 +127,33 @@ bpt_status bpt_layer_forward(const void* x, const void* ln1, const void* W_Q, co
                              bpt_stream_t stream);
 
 /*
+ * bpt_layer_forward_train -- bpt_layer_forward that also writes the per-row
+ * softmax statistics the backward pass recomputes from ("Blockwise Parallel
+ * Transformer — BPT", section "The backward pass": the forward keeps the
+ * layer input, the layer output and, per row, the softmax statistics (m, l),
+ * so that each block's attention can be recomputed exactly in one pass).
+ *
+ *   stats [B, h, N, 2] fp32, device, caller-owned, 8-byte aligned; must not
+ *         overlap x, out or the workspace.  For batch b, head t and query
+ *         row i, with s_j = q_i . k_j / sqrt(d_k) over the keys row i may
+ *         attend to (j <= i when causal):
+ *           stats[b, t, i, 0] = m = max_j s_j
+ *           stats[b, t, i, 1] = l = sum_j exp(s_j - m)
+ *         computed from the same scores the forward uses (fp16 Q, K for
+ *         BPT_BF16), so log(l) + m is that row's log-sum-exp.
+ * Every other argument, the supported shapes, the results in `out` and the
+ * workspace are those of bpt_layer_forward.  Returns BPT_ERR_INVALID_ARG for
+ * stats == NULL, misaligned or overlapping; otherwise as bpt_layer_forward.
+ */
+bpt_status bpt_layer_forward_train(const void* x, const void* ln1, const void* W_Q,
+                                   const void* W_K, const void* W_V, const void* W_O,
+                                   const void* ln2, const void* W_1, const void* b_1,
+                                   const void* W_2, const void* b_2, int64_t B, int64_t N,
+                                   int64_t d, int64_t h, int64_t d_ff, int causal,
+                                   bpt_dtype dtype, float* out, float* stats, void* workspace,
+                                   size_t workspace_bytes, bpt_stream_t stream);
+
+/*
  * bpt_read_device_error -- synchronises `stream`, reads and clears the error
  * word in the workspace header (written by the latest bpt_layer_forward on
  * this workspace).  Returns BPT_OK if nothing was recorded, BPT_ERR_TIMEOUT if

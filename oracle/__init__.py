@@ -4,7 +4,7 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  The CUDA path never does.
 """
 from .bpt_oracle import (  # noqa: F401
-    LN_EPS, attention_rows, ffn_residual, gelu, layer_blockwise,
+    LN_EPS, attention_rows, attention_stats_rows, ffn_residual, gelu, layer_blockwise,
     layer_intermediates,
     layer_norm, layer_rows, layer_unfused, online_softmax_init,
     online_softmax_update, softmax_rows,

@@ -16,6 +16,9 @@ Sources (web pages, cited by title and section):
   blocks j > i are skipped).
 * "transformer-cost" (raminaeye.github.io), FlashAttention section: the
   max-subtracted softmax and the running-max / running-sum rescaling.
+* "Blockwise Parallel Transformer — BPT", section "The backward pass": the
+  forward keeps, per row, the softmax statistics (m, l) that the backward's
+  block recomputation reads.
 
 What the layer computes, for every batch element independently (the unfused
 reading, which is the plain definition; the fused schedule reaches the same
@@ -249,6 +252,48 @@ def layer_rows(inp: Dict[str, np.ndarray], h: int, causal: bool,
         Y = X[b, pos] + O @ W_O
         out[sel] = ffn_residual(Y, inp)
     return out
+
+
+def attention_stats_rows(inp: Dict[str, np.ndarray], h: int, causal: bool,
+                         rows: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """Per-row softmax statistics (m, l) at sampled (batch, row) pairs.
+
+    BPT page, "The backward pass": the forward keeps, for every row, the
+    softmax statistics it needs to recompute the row's attention exactly.
+    For head t of row i, with s_j = q_i . k_j / sqrt(d_k) over the keys the
+    row may attend to (j <= i under the causal mask):
+        m = max_j s_j,   l = sum_j exp(s_j - m).
+    Returns float64 arrays m, l of shape [len(rows), h].  Q and K are those
+    of steps 1-2 (LN1, then the projections); K is formed in row chunks as in
+    ``layer_rows``.
+    """
+    X = _as64(inp, "x")
+    Bx, N, d = X.shape
+    d_k = d // h
+    scale = 1.0 / math.sqrt(d_k)
+    rows = np.asarray(rows, dtype=np.int64).reshape(-1, 2)
+    m_out = np.empty((rows.shape[0], h))
+    l_out = np.empty((rows.shape[0], h))
+    W_Q, W_K = _as64(inp, "W_Q"), _as64(inp, "W_K")
+    g1, be1 = _as64(inp, "gamma1"), _as64(inp, "beta1")
+    for b in np.unique(rows[:, 0]):
+        sel = np.nonzero(rows[:, 0] == b)[0]
+        pos = rows[sel, 1]
+        n_keys = int(pos.max()) + 1 if causal else N
+        K = np.empty((n_keys, d))
+        for r0 in range(0, n_keys, ROW_CHUNK):
+            r1 = min(n_keys, r0 + ROW_CHUNK)
+            K[r0:r1] = layer_norm(X[b, r0:r1], g1, be1) @ W_K
+        Qr = layer_norm(X[b, pos], g1, be1) @ W_Q
+        for t in range(h):
+            c = slice(t * d_k, (t + 1) * d_k)
+            S = (Qr[:, c] @ K[:, c].T) * scale
+            if causal:
+                S = np.where(np.arange(n_keys)[None, :] > pos[:, None], -np.inf, S)
+            m = S.max(axis=1)
+            m_out[sel, t] = m
+            l_out[sel, t] = np.exp(S - m[:, None]).sum(axis=1)
+    return m_out, l_out
 
 
 # --------------------------------------------------------------------------
