@@ -9,3 +9,7 @@ from .bpt_oracle import (  # noqa: F401
     layer_norm, layer_rows, layer_unfused, online_softmax_init,
     online_softmax_update, softmax_rows,
 )
+from .bpt_backward import (  # noqa: F401
+    GRAD_NAMES, attention_backward, gelu_grad, layer_backward, layer_backward_blockwise,
+    layer_norm_backward,
+)
