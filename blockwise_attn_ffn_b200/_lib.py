@@ -26,7 +26,8 @@ EXPORTED = [
     "bpt_layer_workspace_size", "bpt_layer_forward", "bpt_read_device_error",
     "bpt_status_string", "bpt_profile_enable", "bpt_profile_read",
     "bpt_layer_launch_count", "bpt_layer_forward_static", "bpt_debug_inject_fault",
-    "bpt_layer_forward_train",
+    "bpt_layer_forward_train", "bpt_layer_backward_workspace_size", "bpt_layer_backward",
+    "bpt_debug_set_max_wave",
 ]
 
 _lib: Optional[ctypes.CDLL] = None
@@ -56,6 +57,14 @@ def load() -> ctypes.CDLL:
     lib.bpt_layer_forward_train.argtypes = ([vp] * 11 + [i64] * 5 +
                                             [i32, i32, vp, vp, vp, ctypes.c_size_t, vp])
     lib.bpt_layer_forward_train.restype = i32
+    lib.bpt_layer_backward_workspace_size.argtypes = [i64, i64, i64, i64, i64, i32, i32,
+                                                      ctypes.POINTER(ctypes.c_size_t)]
+    lib.bpt_layer_backward_workspace_size.restype = i32
+    lib.bpt_layer_backward.argtypes = ([vp] * 13 + [i64] * 5 + [i32, i32] + [vp] * 12 +
+                                       [ctypes.c_size_t, vp])
+    lib.bpt_layer_backward.restype = i32
+    lib.bpt_debug_set_max_wave.argtypes = [i64]
+    lib.bpt_debug_set_max_wave.restype = i32
     lib.bpt_read_device_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     lib.bpt_read_device_error.restype = i32
     lib.bpt_status_string.argtypes = [i32]
@@ -105,6 +114,28 @@ def bpt_layer_forward_train(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
     return load().bpt_layer_forward_train(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
                                           B, N, d, h, d_ff, int(bool(causal)), dtype, out,
                                           stats, workspace, workspace_bytes, stream)
+
+
+def bpt_layer_backward_workspace_size(B, N, d, h, d_ff, causal, dtype) -> Tuple[int, int]:
+    """Returns (status, bytes)."""
+    out = ctypes.c_size_t(0)
+    st = load().bpt_layer_backward_workspace_size(B, N, d, h, d_ff, int(bool(causal)), dtype,
+                                                  ctypes.byref(out))
+    return st, out.value
+
+
+def bpt_layer_backward(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, stats, dZ,
+                       B, N, d, h, d_ff, causal, dtype, dx, d_ln1, dW_Q, dW_K, dW_V, dW_O,
+                       d_ln2, dW_1, db_1, dW_2, db_2, workspace, workspace_bytes, stream) -> int:
+    """Pointer-level call; returns the status code."""
+    return load().bpt_layer_backward(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, stats,
+                                     dZ, B, N, d, h, d_ff, int(bool(causal)), dtype, dx, d_ln1,
+                                     dW_Q, dW_K, dW_V, dW_O, d_ln2, dW_1, db_1, dW_2, db_2,
+                                     workspace, workspace_bytes, stream)
+
+
+def bpt_debug_set_max_wave(blocks: int) -> int:
+    return load().bpt_debug_set_max_wave(blocks)
 
 
 def bpt_read_device_error(workspace, stream) -> Tuple[int, int]:

@@ -18,6 +18,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -25,6 +26,7 @@
 
 #include "bpt.h"
 #include "attn_pair_tc.cuh"
+#include "backward.cuh"
 #include "common.cuh"
 #include "gemm_tc.cuh"
 #include "rows.cuh"
@@ -35,6 +37,8 @@ namespace {
 using bpt::RowMap;
 
 constexpr int64_t kMaxWave = BPT_WAVE_BLOCKS;
+// Query blocks per wave (test hook bpt_debug_set_max_wave lowers it).
+std::atomic<int64_t> g_max_wave{kMaxWave};
 // 16-column groups (of eight per 128-key row) whose exp2 runs on the FMA
 // pipe instead of MUFU (compile-time tuning knobs; 2 of 8 measured fastest).
 #ifndef BPT_EMU_DK128
@@ -125,14 +129,15 @@ Plan make_plan(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff, int cau
   if (p.items == 0) {
     p.n_waves = 0;
     p.P = 0;
-  } else if (p.nb > kMaxWave) {
-    p.cps = (p.nb + kMaxWave - 1) / kMaxWave;
+  } else if (p.nb > g_max_wave.load()) {
+    const int64_t mw = g_max_wave.load();
+    p.cps = (p.nb + mw - 1) / mw;
     p.G = 0;
     p.n_waves = B * p.cps;
     p.P = (p.nb + p.cps - 1) / p.cps;
   } else {
     p.cps = 0;
-    p.G = std::min<int64_t>(B, kMaxWave / p.nb);
+    p.G = std::max<int64_t>(1, std::min<int64_t>(B, g_max_wave.load() / p.nb));
     p.n_waves = (B + p.G - 1) / p.G;
     p.P = p.G * p.nb;
   }
@@ -155,6 +160,13 @@ Plan make_plan(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff, int cau
 
 
 // ------------------------------------------------------------ device info --
+// True on failure (so that calls chain with ||).
+template <typename K>
+bool set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+         cudaSuccess;
+}
+
 struct DeviceInfo {
   bool init = false;
   bool ok = false;
@@ -184,12 +196,15 @@ bpt_status device_info(int* sms, int* pair_clusters = nullptr) {
           cudaFuncSetAttribute(bpt::attn_pair_tc_kernel<128, kEmu128>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                bpt::AttnPairCfg<128, kEmu128>::SMEM) != cudaSuccess ||
-          cudaFuncSetAttribute(bpt::gemm_f16_pair_kernel<4>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               bpt::kPairSmem) != cudaSuccess ||
-          cudaFuncSetAttribute(bpt::gemm_f16_pair_kernel<8>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               bpt::kPairSmem) != cudaSuccess ||
+          set_smem(bpt::gemm_f16_pair_kernel<4, bpt::kLayAkBn>, bpt::kPairSmem) ||
+          set_smem(bpt::gemm_f16_pair_kernel<8, bpt::kLayAkBn>, bpt::kPairSmem) ||
+          set_smem(bpt::gemm_f16_pair_kernel<4, bpt::kLayAnBn>, bpt::kPairSmem) ||
+          set_smem(bpt::gemm_f16_pair_kernel<4, bpt::kLayAkBk>, bpt::kPairSmem) ||
+          set_smem(bpt::gemm_f16_pair_kernel<8, bpt::kLayAkBk>, bpt::kPairSmem) ||
+          set_smem(bpt::attn_bwd_dq_kernel<128>, bpt::AttnBwdSmem<128>::DQ_BYTES) ||
+          set_smem(bpt::attn_bwd_dkv_kernel<128>, bpt::AttnBwdSmem<128>::DKV_BYTES) ||
+          set_smem(bpt::attn_bwd_dq_kernel<64>, bpt::AttnBwdSmem<64>::DQ_BYTES) ||
+          set_smem(bpt::attn_bwd_dkv_kernel<64>, bpt::AttnBwdSmem<64>::DKV_BYTES) ||
           cudaFuncSetAttribute(bpt::attn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (3 * 64 * 128 + 64 * 65) * 4) != cudaSuccess)
         return BPT_ERR_CUDA;
@@ -200,7 +215,8 @@ bpt_status device_info(int* sms, int* pair_clusters = nullptr) {
       cfg.blockDim = dim3(bpt::gemm_threads<8>());
       cfg.dynamicSmemBytes = bpt::kPairSmem;
       int clusters = 0;
-      if (cudaOccupancyMaxActiveClusters(&clusters, bpt::gemm_f16_pair_kernel<8>, &cfg) !=
+      if (cudaOccupancyMaxActiveClusters(&clusters, bpt::gemm_f16_pair_kernel<8, bpt::kLayAkBn>,
+                                         &cfg) !=
               cudaSuccess ||
           clusters <= 0) {
         cudaGetLastError();
@@ -249,19 +265,24 @@ bool encode_f16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims
   return r == CUDA_SUCCESS;
 }
 
-// GEMM A operand: [rows, K] row-major, viewed as [K/64][rows][64]; a box is
-// 128 rows x two 64-column chunks (32 KB, chunk-major in shared memory).
-bool map_a(CUtensorMap* m, const void* base, int64_t rows, int64_t K) {
+// GEMM operand, K-contiguous: [rows, K] with row stride ld (elements), viewed
+// as [K/64][rows][64]; a box is 128 rows x two 64-column chunks (32 KB,
+// chunk-major in shared memory).  The A operand of the forward, and the B
+// operand [N, K] of the data-gradient GEMMs.
+bool map_a(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int64_t ld = 0) {
   const uint64_t dims[3] = {64, uint64_t(rows), uint64_t(K / 64)};
-  const uint64_t st[2] = {uint64_t(K) * 2, 128};
+  const uint64_t st[2] = {uint64_t(ld > 0 ? ld : K) * 2, 128};
   const uint32_t box[3] = {64, 128, 2};
   return encode_f16(m, base, 3, dims, st, box);
 }
-// GEMM B operand: [K, cols] row-major, viewed as [cols/64][K][64]; a box is
-// 128 K rows x `chunks` 64-column chunks (chunk-major in shared memory).
-bool map_b(CUtensorMap* m, const void* base, int64_t K, int64_t cols, int chunks) {
+// GEMM operand, row-contiguous along the output axis: [K, cols] with row
+// stride ld, viewed as [cols/64][K][64]; a box is 128 K rows x `chunks`
+// 64-column chunks.  The B operand of the forward (weights), and the A
+// operand [K, M] of the weight-gradient GEMMs.
+bool map_b(CUtensorMap* m, const void* base, int64_t K, int64_t cols, int chunks,
+           int64_t ld = 0) {
   const uint64_t dims[3] = {64, uint64_t(K), uint64_t(cols / 64)};
-  const uint64_t st[2] = {uint64_t(cols) * 2, 128};
+  const uint64_t st[2] = {uint64_t(ld > 0 ? ld : cols) * 2, 128};
   const uint32_t box[3] = {64, 128, uint32_t(chunks)};
   return encode_f16(m, base, 3, dims, st, box);
 }
@@ -341,24 +362,67 @@ cudaError_t launch_ln(const TIn* in, const TP* ln, TOut* out, int64_t rows, int6
   return cudaErrorInvalidValue;
 }
 
+// layout: bpt::kLayAkBn (forward), kLayAnBn (X^T dY), kLayAkBk (dY W^T).
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                         const CUtensorMap& b2, const bpt::GemmParams& gp, int sms,
-                        cudaStream_t s) {
+                        cudaStream_t s, int layout = bpt::kLayAkBn) {
   int dummy = 0, pairs_max = 0;
   if (device_info(&dummy, &pairs_max) != BPT_OK) return cudaErrorInvalidDevice;
   const int64_t tiles = int64_t((gp.M + bpt::kPairBM - 1) / bpt::kPairBM) *
                         int64_t((gp.N + bpt::kGemmBN - 1) / bpt::kGemmBN);
   const unsigned pairs = unsigned(std::max<int64_t>(1, std::min<int64_t>(tiles, pairs_max)));
-  if (gp.epi == bpt::kEpiGeluBias || gp.epi == bpt::kEpiResidX)
-    bpt::gemm_f16_pair_kernel<8>
-        <<<2 * pairs, bpt::gemm_threads<8>(), bpt::kPairSmem, s>>>(a, b0, b1, b2, gp);
+  // Eight epilogue warps for the per-element-heavy epilogues, four otherwise.
+  const bool heavy = gp.epi == bpt::kEpiGeluBias || gp.epi == bpt::kEpiResidX ||
+                     gp.epi == bpt::kEpiGeluBiasKeep || gp.epi == bpt::kEpiGeluGrad;
+  const unsigned grid = 2 * pairs;
+  if (layout == bpt::kLayAnBn)
+    bpt::gemm_f16_pair_kernel<4, bpt::kLayAnBn>
+        <<<grid, bpt::gemm_threads<4>(), bpt::kPairSmem, s>>>(a, b0, b1, b2, gp);
+  else if (layout == bpt::kLayAkBk && heavy)
+    bpt::gemm_f16_pair_kernel<8, bpt::kLayAkBk>
+        <<<grid, bpt::gemm_threads<8>(), bpt::kPairSmem, s>>>(a, b0, b1, b2, gp);
+  else if (layout == bpt::kLayAkBk)
+    bpt::gemm_f16_pair_kernel<4, bpt::kLayAkBk>
+        <<<grid, bpt::gemm_threads<4>(), bpt::kPairSmem, s>>>(a, b0, b1, b2, gp);
+  else if (heavy)
+    bpt::gemm_f16_pair_kernel<8, bpt::kLayAkBn>
+        <<<grid, bpt::gemm_threads<8>(), bpt::kPairSmem, s>>>(a, b0, b1, b2, gp);
   else
-    bpt::gemm_f16_pair_kernel<4>
-        <<<2 * pairs, bpt::gemm_threads<4>(), bpt::kPairSmem, s>>>(a, b0, b1, b2, gp);
+    bpt::gemm_f16_pair_kernel<4, bpt::kLayAkBn>
+        <<<grid, bpt::gemm_threads<4>(), bpt::kPairSmem, s>>>(a, b0, b1, b2, gp);
   return cudaGetLastError();
 }
 
 bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+// One wave of the tensor-core attention: o (fp16 block rows) and, if stats is
+// non-null, the per-row (m, l).
+cudaError_t launch_attn(const Plan& P, const Wave& wv_, const CUtensorMap& mQKV, __half* so,
+                        float* stats, uint32_t* err, int fault, cudaStream_t s) {
+  bpt::AttnPairParams ap{};
+  ap.N = int(P.N); ap.nb = int(P.nb); ap.h = int(P.h); ap.d = int(P.d);
+  ap.causal = P.causal; ap.item0 = int(wv_.item0); ap.count = int(wv_.count);
+  ap.seqs = int(wv_.seqs); ap.o = so; ap.err = err;
+  ap.scale_log2 = float(1.4426950408889634 / std::sqrt(double(P.dk)));
+  ap.stats = reinterpret_cast<float2*>(stats);
+  const int64_t kv_head = (wv_.seqs > 0 ? wv_.seqs : 1) * P.N * P.dk * 2 * 2;
+  ap.hg = 1;
+  for (int g = int(P.h); g > 1; --g)
+    if (P.h % g == 0 && g * kv_head <= (int64_t(BPT_ATTN_KV_BUDGET_MB) << 20)) {
+      ap.hg = g;
+      break;
+    }
+  ap.fault = fault;
+  const int64_t pairs = wv_.seqs == 0 ? (wv_.count + 1) / 2 : wv_.seqs * ((P.nb + 1) / 2);
+  const unsigned grid = unsigned(pairs * P.h);
+  if (P.dk == 128)
+    bpt::attn_pair_tc_kernel<128, kEmu128>
+        <<<grid, 384, bpt::AttnPairCfg<128, kEmu128>::SMEM, s>>>(mQKV, ap);
+  else
+    bpt::attn_pair_tc_kernel<64, kEmu64>
+        <<<grid, 384, bpt::AttnPairCfg<64, kEmu64>::SMEM, s>>>(mQKV, ap);
+  return cudaGetLastError();
+}
 
 bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const void* W_Q,
                         const void* W_K, const void* W_V, const void* W_O, const void* ln2,
@@ -438,35 +502,15 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
     LaunchScope ls(BPT_KIND_QKV, s);
     if (launch_gemm(mXn, mWq, mWk, mWv, g, sms, s) != cudaSuccess) return BPT_ERR_CUDA;
   }
-  const float scale_log2 = float(1.4426950408889634 / std::sqrt(double(P.dk)));
   for (int64_t w = 0; w < P.n_waves; ++w) {
     const Wave wv_ = P.wave(w);
     const int64_t rows = wv_.count * P.blk;
     RowMap map{int(wv_.item0), int(P.nb), int(P.N), int(P.blk), 0};
     {
-      bpt::AttnPairParams ap{};
-      ap.N = int(P.N); ap.nb = int(P.nb); ap.h = int(P.h); ap.d = int(d);
-      ap.causal = P.causal; ap.item0 = int(wv_.item0); ap.count = int(wv_.count);
-      ap.seqs = int(wv_.seqs); ap.o = so; ap.scale_log2 = scale_log2; ap.err = err;
-      ap.stats = reinterpret_cast<float2*>(stats);
-      const int64_t kv_head = (wv_.seqs > 0 ? wv_.seqs : 1) * P.N * P.dk * 2 * 2;
-      ap.hg = 1;
-      for (int g = int(P.h); g > 1; --g)
-        if (P.h % g == 0 && g * kv_head <= (int64_t(BPT_ATTN_KV_BUDGET_MB) << 20)) {
-          ap.hg = g;
-          break;
-        }
-      ap.fault = (fault == 2 && w == 0) ? 2 : 0;
-      const int64_t pairs = wv_.seqs == 0 ? (wv_.count + 1) / 2 : wv_.seqs * ((P.nb + 1) / 2);
-      const unsigned grid = unsigned(pairs * P.h);
       LaunchScope ls(BPT_KIND_ATTN, s);
-      if (P.dk == 128)
-        bpt::attn_pair_tc_kernel<128, kEmu128>
-            <<<grid, 384, bpt::AttnPairCfg<128, kEmu128>::SMEM, s>>>(mQKV, ap);
-      else
-        bpt::attn_pair_tc_kernel<64, kEmu64>
-            <<<grid, 384, bpt::AttnPairCfg<64, kEmu64>::SMEM, s>>>(mQKV, ap);
-      if (cudaGetLastError() != cudaSuccess) return BPT_ERR_CUDA;
+      if (launch_attn(P, wv_, mQKV, so, stats, err, (fault == 2 && w == 0) ? 2 : 0, s) !=
+          cudaSuccess)
+        return BPT_ERR_CUDA;
     }
     {
       bpt::GemmParams g{};
@@ -580,6 +624,273 @@ bpt_status forward_f32(const Plan& P, const float* x, const float* ln1, const fl
 
 }  // namespace
 
+// ----------------------------------------------------------- backward --
+// Workspace of bpt_layer_backward: the forward's layout (header, fp16
+// weights, QKV, wave scratch o / LN2(y) / H), then the backward's buffers.
+constexpr int kColChunks = 256;  // row chunks of the deterministic column sums
+
+struct BwdLayout {
+  size_t off_hpre, off_dz16, off_dvn, off_dy16, off_do16, off_D, off_rowstat, off_y, off_u16,
+      off_dq, off_dk, off_dv, off_dqkv16, off_du, off_part, total;
+  int64_t part_cols;
+};
+
+BwdLayout make_bwd_layout(const Plan& P) {
+  BwdLayout L{};
+  const size_t R = size_t(P.P * P.blk), M = size_t(P.B * P.N), d = size_t(P.d),
+               dff = size_t(P.d_ff), h = size_t(P.h);
+  size_t off = align_up(P.total, 1024);
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 1024);
+    return o;
+  };
+  L.off_hpre = take(R * dff * 2);
+  L.off_dz16 = take(R * d * 2);
+  L.off_dvn = take(R * d * 4);
+  L.off_dy16 = take(R * d * 2);
+  L.off_do16 = take(R * d * 2);
+  L.off_D = take(R * h * 4);
+  L.off_rowstat = take(std::max(R, M) * 8);
+  L.off_y = take(M * d * 4);
+  L.off_u16 = take(M * d * 2);
+  L.off_dq = take(M * d * 4);
+  L.off_dk = take(M * d * 4);
+  L.off_dv = take(M * d * 4);
+  L.off_dqkv16 = take(M * 3 * d * 2);
+  L.off_du = take(M * d * 4);
+  L.part_cols = int64_t(std::max(d, dff));
+  L.off_part = take(2 * size_t(kColChunks) * size_t(L.part_cols) * 4);
+  L.total = off;
+  return L;
+}
+
+// out[c] (+)= column sums of A (and of A * xh if X) over `rows` rows.
+template <typename TA, typename TX>
+cudaError_t launch_colsum(const TA* A, int a_global, const TX* X, const float2* rowstat,
+                          int64_t rows, int64_t d, RowMap map, float* part_a, float* part_b,
+                          float* out_a, float* out_b, cudaStream_t s) {
+  const int rpc = int((rows + kColChunks - 1) / kColChunks);
+  const int chunks = int((rows + rpc - 1) / rpc);
+  bpt::colsum_partial_kernel<TA, TX><<<dim3(unsigned((d + 255) / 256), unsigned(chunks)), 256, 0,
+                                        s>>>(A, a_global, X, rowstat, part_a, part_b, rows, int(d),
+                                             rpc, map);
+  bpt::colsum_reduce_kernel<<<unsigned((d + 255) / 256), 256, 0, s>>>(part_a, chunks, int(d),
+                                                                     out_a);
+  if (X) bpt::colsum_reduce_kernel<<<unsigned((d + 255) / 256), 256, 0, s>>>(part_b, chunks,
+                                                                            int(d), out_b);
+  return cudaGetLastError();
+}
+
+bpt_status backward_bf16(const Plan& P, const BwdLayout& L, const void* x, const void* ln1,
+                         const void* W_Q, const void* W_K, const void* W_V, const void* W_O,
+                         const void* ln2, const void* W_1, const void* b_1, const void* W_2,
+                         const float* stats, const float* dZ, float* dx, float* d_ln1,
+                         float* dW_Q, float* dW_K, float* dW_V, float* dW_O, float* d_ln2,
+                         float* dW_1, float* db_1, float* dW_2, float* db_2, uint8_t* ws,
+                         cudaStream_t s, int sms) {
+  using bf = __nv_bfloat16;
+  using hf = __half;
+  const int64_t M = P.B * P.N, d = P.d, d_ff = P.d_ff, h = P.h;
+  const int64_t R = P.P * P.blk;
+  uint32_t* err = reinterpret_cast<uint32_t*>(ws);
+  hf* w16 = reinterpret_cast<hf*>(ws + P.off_w16);
+  hf* wq = w16;
+  hf* wk = wq + d * d;
+  hf* wv = wk + d * d;
+  hf* wo = wv + d * d;
+  hf* w1 = wo + d * d;
+  hf* w2 = w1 + d * d_ff;
+  hf* qkv = reinterpret_cast<hf*>(ws + P.off_qkv);
+  hf* so = reinterpret_cast<hf*>(ws + P.off_o);
+  hf* sv = reinterpret_cast<hf*>(ws + P.off_v);
+  hf* sh = reinterpret_cast<hf*>(ws + P.off_h);
+  hf* hpre = reinterpret_cast<hf*>(ws + L.off_hpre);
+  hf* dz16 = reinterpret_cast<hf*>(ws + L.off_dz16);
+  float* dvn = reinterpret_cast<float*>(ws + L.off_dvn);
+  hf* dy16 = reinterpret_cast<hf*>(ws + L.off_dy16);
+  hf* do16 = reinterpret_cast<hf*>(ws + L.off_do16);
+  float* Drow = reinterpret_cast<float*>(ws + L.off_D);
+  float2* rowstat = reinterpret_cast<float2*>(ws + L.off_rowstat);
+  float* y = reinterpret_cast<float*>(ws + L.off_y);
+  hf* u16 = reinterpret_cast<hf*>(ws + L.off_u16);
+  float* dq = reinterpret_cast<float*>(ws + L.off_dq);
+  float* dk = reinterpret_cast<float*>(ws + L.off_dk);
+  float* dv = reinterpret_cast<float*>(ws + L.off_dv);
+  hf* dqkv16 = reinterpret_cast<hf*>(ws + L.off_dqkv16);
+  float* du = reinterpret_cast<float*>(ws + L.off_du);
+  float* part_a = reinterpret_cast<float*>(ws + L.off_part);
+  float* part_b = part_a + size_t(kColChunks) * size_t(L.part_cols);
+  const bf* gamma1 = static_cast<const bf*>(ln1);
+  const bf* gamma2 = static_cast<const bf*>(ln2);
+
+  // Tensor maps (see map_a / map_b): forward recomputation, then the
+  // backward's weight-gradient (A = X^T) and data-gradient (B = W^T) GEMMs.
+  const int qkv_chunks = (d % 128 == 0) ? 2 : 1;
+  CUtensorMap mU, mWq, mWk, mWv, mQKV, mO, mWo, mV, mW1;
+  CUtensorMap mHt, mDzB, mDzA, mW2k, mVnt, mHpB, mHpA, mW1k, mOt, mDyB, mDyA, mWok, mUt;
+  CUtensorMap mDqB[3], mDqA[3], mWk3[3];
+  bool ok = map_a(&mU, u16, M, d) && map_b(&mWq, wq, d, d, qkv_chunks) &&
+            map_b(&mWk, wk, d, d, qkv_chunks) && map_b(&mWv, wv, d, d, qkv_chunks) &&
+            map_qkv(&mQKV, qkv, P.B, P.N, d, P.dk) && map_a(&mO, so, R, d) &&
+            map_b(&mWo, wo, d, d, 2) && map_a(&mV, sv, R, d) && map_b(&mW1, w1, d, d_ff, 2) &&
+            map_b(&mHt, sh, R, d_ff, 2) && map_b(&mDzB, dz16, R, d, 2) &&
+            map_a(&mDzA, dz16, R, d) && map_a(&mW2k, w2, d_ff, d) &&
+            map_b(&mVnt, sv, R, d, 2) && map_b(&mHpB, hpre, R, d_ff, 2) &&
+            map_a(&mHpA, hpre, R, d_ff) && map_a(&mW1k, w1, d, d_ff) &&
+            map_b(&mOt, so, R, d, 2) && map_b(&mDyB, dy16, R, d, 2) &&
+            map_a(&mDyA, dy16, R, d) && map_a(&mWok, wo, d, d) && map_b(&mUt, u16, M, d, 2);
+  const hf* wqkv[3] = {wq, wk, wv};
+  for (int i = 0; i < 3 && ok; ++i)
+    ok = map_b(&mDqB[i], dqkv16 + i * d, M, d, 2, 3 * d) &&
+         map_a(&mDqA[i], dqkv16 + i * d, M, d, 3 * d) && map_a(&mWk3[i], wqkv[i], d, d);
+  if (!ok) return BPT_ERR_CUDA;
+
+  // Zero what is accumulated.
+  const std::pair<float*, size_t> zero[] = {
+      {dW_Q, size_t(d * d)}, {dW_K, size_t(d * d)}, {dW_V, size_t(d * d)}, {dW_O, size_t(d * d)},
+      {dW_1, size_t(d * d_ff)}, {db_1, size_t(d_ff)}, {dW_2, size_t(d_ff * d)}, {db_2, size_t(d)},
+      {d_ln1, size_t(2 * d)}, {d_ln2, size_t(2 * d)}, {dk, size_t(M * d)}, {dv, size_t(M * d)}};
+  for (const auto& z : zero)
+    if (cudaMemsetAsync(z.first, 0, z.second * sizeof(float), s) != cudaSuccess)
+      return BPT_ERR_CUDA;
+  {
+    bpt::CvtSegments cs{};
+    const void* src[6] = {W_Q, W_K, W_V, W_O, W_1, W_2};
+    hf* dst[6] = {wq, wk, wv, wo, w1, w2};
+    const int64_t n[6] = {d * d, d * d, d * d, d * d, d * d_ff, d_ff * d};
+    long long acc = 0;
+    for (int k = 0; k < 6; ++k) {
+      cs.src[k] = static_cast<const bf*>(src[k]);
+      cs.dst[k] = dst[k];
+      acc += n[k] / 8;
+      cs.n8_end[k] = acc;
+    }
+    cs.count = 6;
+    const unsigned grid = unsigned(std::min<long long>((acc + 255) / 256, int64_t(sms) * 8));
+    bpt::cvt_bf16_to_f16_kernel<<<grid, 256, 0, s>>>(cs, err);
+    if (cudaGetLastError() != cudaSuccess) return BPT_ERR_CUDA;
+  }
+  RowMap ident{0, 1, 1, 1, 1};
+  if (launch_ln<bf, hf, bf>(static_cast<const bf*>(x), gamma1, u16, M, d, ident, err, s) !=
+      cudaSuccess)
+    return BPT_ERR_CUDA;
+  auto gemm = [&](const CUtensorMap& a, const CUtensorMap& b, int64_t m, int64_t n, int64_t k,
+                  int epi, int layout, const RowMap& map, auto&& set) {
+    bpt::GemmParams g{};
+    g.M = int(m); g.N = int(n); g.K = int(k);
+    g.n_sub = int(n); g.n_maps = 1; g.b_chunks = 2;
+    g.epi = epi; g.map = map; g.err = err;
+    set(g);
+    return launch_gemm(a, b, b, b, g, sms, s, layout) == cudaSuccess;
+  };
+  {
+    bpt::GemmParams g{};
+    g.M = int(M); g.N = int(3 * d); g.K = int(d);
+    g.n_sub = int(d); g.n_maps = 3; g.b_chunks = qkv_chunks;
+    g.epi = bpt::kEpiStoreF16; g.out_h = qkv; g.ld_out = 3 * d; g.map = ident; g.err = err;
+    if (launch_gemm(mU, mWq, mWk, mWv, g, sms, s) != cudaSuccess) return BPT_ERR_CUDA;
+  }
+  const float scale = float(1.0 / std::sqrt(double(P.dk)));
+  for (int64_t w = 0; w < P.n_waves; ++w) {
+    const Wave wv_ = P.wave(w);
+    const int64_t rows = wv_.count * P.blk;
+    RowMap map{int(wv_.item0), int(P.nb), int(P.N), int(P.blk), 0};
+    // forward recomputation of this wave: o, y, LN2(y), FFN pre-activation and hidden
+    if (launch_attn(P, wv_, mQKV, so, nullptr, err, 0, s) != cudaSuccess) return BPT_ERR_CUDA;
+    if (!gemm(mO, mWo, rows, d, d, bpt::kEpiResidX, bpt::kLayAkBn, map, [&](bpt::GemmParams& g) {
+          g.out_f32 = y; g.ld_f32 = d; g.resid = static_cast<const bf*>(x); g.ld_resid = d;
+        }))
+      return BPT_ERR_CUDA;
+    if (launch_ln<float, hf, bf>(y, gamma2, sv, rows, d, map, err, s) != cudaSuccess)
+      return BPT_ERR_CUDA;
+    if (!gemm(mV, mW1, rows, d_ff, d, bpt::kEpiGeluBiasKeep, bpt::kLayAkBn, ident,
+              [&](bpt::GemmParams& g) {
+                g.out_h = sh; g.out_h2 = hpre; g.ld_out = d_ff;
+                g.bias = static_cast<const bf*>(b_1);
+              }))
+      return BPT_ERR_CUDA;
+    // FFN backward
+    bpt::rows_f32_to_f16_kernel<<<unsigned(std::min<int64_t>((rows * d / 8 + 255) / 256,
+                                                            int64_t(sms) * 16)),
+                                  256, 0, s>>>(dZ, dz16, rows, int(d), map);
+    if (!gemm(mHt, mDzB, d_ff, d, rows, bpt::kEpiAccumF32, bpt::kLayAnBn, ident,
+              [&](bpt::GemmParams& g) { g.out_f32 = dW_2; g.ld_f32 = d; }))
+      return BPT_ERR_CUDA;
+    if (!gemm(mDzA, mW2k, rows, d_ff, d, bpt::kEpiGeluGrad, bpt::kLayAkBk, ident,
+              [&](bpt::GemmParams& g) { g.out_h = hpre; g.ld_out = d_ff; }))
+      return BPT_ERR_CUDA;
+    if (!gemm(mVnt, mHpB, d, d_ff, rows, bpt::kEpiAccumF32, bpt::kLayAnBn, ident,
+              [&](bpt::GemmParams& g) { g.out_f32 = dW_1; g.ld_f32 = d_ff; }))
+      return BPT_ERR_CUDA;
+    if (launch_colsum<hf, float>(hpre, 0, nullptr, nullptr, rows, d_ff, map, part_a, part_b,
+                                 db_1, nullptr, s) != cudaSuccess ||
+        launch_colsum<float, float>(dZ, 1, nullptr, nullptr, rows, d, map, part_a, part_b, db_2,
+                                    nullptr, s) != cudaSuccess)
+      return BPT_ERR_CUDA;
+    if (!gemm(mHpA, mW1k, rows, d, d_ff, bpt::kEpiStoreF32, bpt::kLayAkBk, ident,
+              [&](bpt::GemmParams& g) { g.out_f32 = dvn; g.ld_f32 = d; }))
+      return BPT_ERR_CUDA;
+    // LN2 backward: dY = dZ + LN2'(dVn) -> dx (global rows) and dy16 (block rows)
+    bpt::ln_backward_kernel<float><<<unsigned((rows * 32 + 255) / 256), 256, 0, s>>>(
+        y, gamma2, dvn, dZ, dx, dy16, rowstat, rows, int(d), map, 0);
+    if (launch_colsum<float, float>(dvn, 0, y, rowstat, rows, d, map, part_a, part_b, d_ln2 + d,
+                                    d_ln2, s) != cudaSuccess)
+      return BPT_ERR_CUDA;
+    // W_O backward
+    if (!gemm(mOt, mDyB, d, d, rows, bpt::kEpiAccumF32, bpt::kLayAnBn, ident,
+              [&](bpt::GemmParams& g) { g.out_f32 = dW_O; g.ld_f32 = d; }))
+      return BPT_ERR_CUDA;
+    if (!gemm(mDyA, mWok, rows, d, d, bpt::kEpiStoreF16, bpt::kLayAkBk, ident,
+              [&](bpt::GemmParams& g) { g.out_h = do16; g.ld_out = d; }))
+      return BPT_ERR_CUDA;
+    // attention backward of this wave's query rows
+    bpt::attn_row_dot_kernel<<<unsigned((rows * 32 + 255) / 256), 256, 0, s>>>(do16, so, Drow,
+                                                                               rows, int(d),
+                                                                               int(h));
+    bpt::AttnBwdParams ab{};
+    ab.qkv = qkv; ab.o = so; ab.dO = do16; ab.D = Drow;
+    ab.stats = reinterpret_cast<const float2*>(stats);
+    ab.dq = dq; ab.dk = dk; ab.dv = dv;
+    ab.N = int(P.N); ab.nb = int(P.nb); ab.h = int(h); ab.d = int(d); ab.causal = P.causal;
+    ab.item0 = int(wv_.item0); ab.count = int(wv_.count); ab.seqs = int(wv_.seqs);
+    ab.scale = scale;
+    int64_t key_end = P.N;
+    if (wv_.seqs == 0 && P.causal)
+      key_end = std::min<int64_t>(P.N, (wv_.item0 % P.nb + wv_.count) * P.blk);
+    const dim3 gq(unsigned(2 * wv_.count), unsigned(h));
+    const dim3 gkv(unsigned((key_end + bpt::kBwdRows - 1) / bpt::kBwdRows), unsigned(h),
+                   unsigned(wv_.seqs > 0 ? wv_.seqs : 1));
+    if (P.dk == 128) {
+      bpt::attn_bwd_dq_kernel<128><<<gq, 256, bpt::AttnBwdSmem<128>::DQ_BYTES, s>>>(ab);
+      bpt::attn_bwd_dkv_kernel<128><<<gkv, 256, bpt::AttnBwdSmem<128>::DKV_BYTES, s>>>(ab);
+    } else {
+      bpt::attn_bwd_dq_kernel<64><<<gq, 256, bpt::AttnBwdSmem<64>::DQ_BYTES, s>>>(ab);
+      bpt::attn_bwd_dkv_kernel<64><<<gkv, 256, bpt::AttnBwdSmem<64>::DKV_BYTES, s>>>(ab);
+    }
+    if (cudaGetLastError() != cudaSuccess) return BPT_ERR_CUDA;
+  }
+  // QKV projection and LN1 backward over all rows
+  bpt::pack3_f32_to_f16_kernel<<<unsigned(std::min<int64_t>((M * 3 * d / 8 + 255) / 256,
+                                                           int64_t(sms) * 16)),
+                                 256, 0, s>>>(dq, dk, dv, dqkv16, M, int(d));
+  float* dWqkv[3] = {dW_Q, dW_K, dW_V};
+  for (int i = 0; i < 3; ++i) {
+    if (!gemm(mUt, mDqB[i], d, d, M, bpt::kEpiAccumF32, bpt::kLayAnBn, ident,
+              [&](bpt::GemmParams& g) { g.out_f32 = dWqkv[i]; g.ld_f32 = d; }))
+      return BPT_ERR_CUDA;
+    if (!gemm(mDqA[i], mWk3[i], M, d, d, i == 0 ? bpt::kEpiStoreF32 : bpt::kEpiAccumF32,
+              bpt::kLayAkBk, ident, [&](bpt::GemmParams& g) { g.out_f32 = du; g.ld_f32 = d; }))
+      return BPT_ERR_CUDA;
+  }
+  bpt::ln_backward_kernel<bf><<<unsigned((M * 32 + 255) / 256), 256, 0, s>>>(
+      static_cast<const bf*>(x), gamma1, du, nullptr, dx, nullptr, rowstat, M, int(d), ident, 1);
+  if (launch_colsum<float, bf>(du, 0, static_cast<const bf*>(x), rowstat, M, d, ident, part_a,
+                               part_b, d_ln1 + d, d_ln1, s) != cudaSuccess)
+    return BPT_ERR_CUDA;
+  return BPT_OK;
+}
+
 // Shared body of bpt_layer_forward and bpt_layer_forward_train (stats may be
 // null: no statistics are written).
 bpt_status layer_forward_impl(const void* x, const void* ln1, const void* W_Q, const void* W_K,
@@ -676,6 +987,73 @@ bpt_status bpt_layer_forward_train(const void* x, const void* ln1, const void* W
 }
 
 
+bpt_status bpt_layer_backward_workspace_size(int64_t B, int64_t N, int64_t d, int64_t h,
+                                             int64_t d_ff, int causal, bpt_dtype dtype,
+                                             size_t* bytes) {
+  if (bytes == nullptr) return BPT_ERR_INVALID_ARG;
+  const bpt_status st = check_shape(B, N, d, h, d_ff, causal, dtype);
+  if (st != BPT_OK) return st;
+  if (dtype != BPT_BF16) return BPT_ERR_UNSUPPORTED;
+  const Plan P = make_plan(B, N, d, h, d_ff, causal, dtype);
+  *bytes = make_bwd_layout(P).total;
+  return BPT_OK;
+}
+
+bpt_status bpt_layer_backward(const void* x, const void* ln1, const void* W_Q, const void* W_K,
+                              const void* W_V, const void* W_O, const void* ln2, const void* W_1,
+                              const void* b_1, const void* W_2, const void* b_2,
+                              const float* stats, const float* dZ, int64_t B, int64_t N,
+                              int64_t d, int64_t h, int64_t d_ff, int causal, bpt_dtype dtype,
+                              float* dx, float* d_ln1, float* dW_Q, float* dW_K, float* dW_V,
+                              float* dW_O, float* d_ln2, float* dW_1, float* db_1, float* dW_2,
+                              float* db_2, void* workspace, size_t workspace_bytes,
+                              bpt_stream_t stream) {
+  (void)b_2;  // the output's bias does not enter any gradient but its own
+  bpt_status st = check_shape(B, N, d, h, d_ff, causal, dtype);
+  if (st != BPT_OK) return st;
+  if (dtype != BPT_BF16) return BPT_ERR_UNSUPPORTED;
+  if (B == 0 || N == 0) return BPT_OK;
+  const void* ins[] = {x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, stats, dZ, workspace};
+  for (const void* p : ins)
+    if (p == nullptr || misaligned(p)) return BPT_ERR_INVALID_ARG;
+  float* outs[] = {dx, d_ln1, dW_Q, dW_K, dW_V, dW_O, d_ln2, dW_1, db_1, dW_2, db_2};
+  const size_t out_bytes[] = {size_t(B * N * d) * 4, size_t(2 * d) * 4, size_t(d * d) * 4,
+                              size_t(d * d) * 4, size_t(d * d) * 4, size_t(d * d) * 4,
+                              size_t(2 * d) * 4, size_t(d * d_ff) * 4, size_t(d_ff) * 4,
+                              size_t(d_ff * d) * 4, size_t(d) * 4};
+  const Plan P = make_plan(B, N, d, h, d_ff, causal, dtype);
+  const BwdLayout L = make_bwd_layout(P);
+  if (workspace_bytes < L.total) return BPT_ERR_WORKSPACE;
+  // Outputs must be aligned and must not overlap each other, the workspace,
+  // or the inputs they are written after being read from (x, stats, dZ).
+  const uintptr_t wsb = reinterpret_cast<uintptr_t>(workspace);
+  const std::pair<uintptr_t, size_t> reads[] = {
+      {reinterpret_cast<uintptr_t>(x), size_t(B * N * d) * 2},
+      {reinterpret_cast<uintptr_t>(stats), size_t(B * h * N) * 8},
+      {reinterpret_cast<uintptr_t>(dZ), size_t(B * N * d) * 4},
+      {wsb, L.total}};
+  for (int i = 0; i < 11; ++i) {
+    if (outs[i] == nullptr || misaligned(outs[i])) return BPT_ERR_INVALID_ARG;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(outs[i]);
+    for (const auto& r : reads)
+      if (a < r.first + r.second && r.first < a + out_bytes[i]) return BPT_ERR_INVALID_ARG;
+    for (int j = 0; j < i; ++j) {
+      const uintptr_t b = reinterpret_cast<uintptr_t>(outs[j]);
+      if (a < b + out_bytes[j] && b < a + out_bytes[i]) return BPT_ERR_INVALID_ARG;
+    }
+  }
+  int sms = 0;
+  st = device_info(&sms);
+  if (st != BPT_OK) return st;
+  st = get_encoder();
+  if (st != BPT_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (cudaMemsetAsync(ws, 0, kHeaderBytes, s) != cudaSuccess) return BPT_ERR_CUDA;
+  return backward_bf16(P, L, x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, stats, dZ, dx, d_ln1,
+                       dW_Q, dW_K, dW_V, dW_O, d_ln2, dW_1, db_1, dW_2, db_2, ws, s, sms);
+}
+
 bpt_status bpt_read_device_error(void* workspace, bpt_stream_t stream, uint32_t* site) {
   if (!workspace) return BPT_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -702,6 +1080,12 @@ const char* bpt_status_string(bpt_status status) {
     case BPT_ERR_RANGE: return "BPT_ERR_RANGE: a tensor-core operand exceeded the fp16 range";
   }
   return "BPT_UNKNOWN_STATUS";
+}
+
+bpt_status bpt_debug_set_max_wave(int64_t blocks) {
+  if (blocks < 0 || blocks > kMaxWave) return BPT_ERR_INVALID_ARG;
+  g_max_wave.store(blocks == 0 ? kMaxWave : blocks);
+  return BPT_OK;
 }
 
 bpt_status bpt_debug_inject_fault(int code) {

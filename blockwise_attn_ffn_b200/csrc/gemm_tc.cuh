@@ -40,7 +40,22 @@
 
 namespace bpt {
 
-enum GemmEpi : int { kEpiStoreF16 = 0, kEpiResidX = 1, kEpiGeluBias = 2, kEpiBiasAccum = 3 };
+enum GemmEpi : int {
+  kEpiStoreF16 = 0,
+  kEpiResidX = 1,
+  kEpiGeluBias = 2,
+  kEpiBiasAccum = 3,
+  kEpiAccumF32 = 4,      // out_f32[row, col] += acc                      (weight gradients)
+  kEpiStoreF32 = 5,      // out_f32[row, col]  = acc                      (data gradients)
+  kEpiGeluGrad = 6,      // out_h[row, col]    = acc * GELU'(out_h[row, col])  (in place)
+  kEpiGeluBiasKeep = 7,  // out_h2 = acc + bias[col]; out_h = GELU(out_h2)  (fp16 both)
+};
+
+// Operand layouts (K = the reduction axis):
+//   kLayAkBn  A [M, K] K-contiguous, B [K, N] N-contiguous   (forward: X W)
+//   kLayAnBn  A [K, M] M-contiguous, B [K, N] N-contiguous   (X^T dY: weight gradients)
+//   kLayAkBk  A [M, K] K-contiguous, B [N, K] K-contiguous   (dY W^T: data gradients)
+enum GemmLayout : int { kLayAkBn = 0, kLayAnBn = 1, kLayAkBk = 2 };
 
 struct GemmParams {
   int M, N, K;     // problem size (N, K multiples of 64)
@@ -49,6 +64,7 @@ struct GemmParams {
   int b_chunks;    // 64-column chunks per B box: 2, or 1 if n_sub % 128 != 0
   int epi;
   __half* out_h;
+  __half* out_h2;  // kEpiGeluBiasKeep: pre-activation copy (same ld as out_h)
   long long ld_out;
   float* out_f32;
   long long ld_f32;
@@ -76,7 +92,7 @@ __device__ __forceinline__ void gemm_epilogue_row(const GemmParams& p, uint32_t 
                                                   long long row, int col_base, int ncols) {
   long long g = -1;
   bool row_ok;
-  if (p.epi == kEpiStoreF16 || p.epi == kEpiGeluBias) {
+  if (p.epi != kEpiResidX && p.epi != kEpiBiasAccum) {
     row_ok = row < p.M;
   } else {
     g = row < p.M ? p.map.map(row) : -1;
@@ -93,15 +109,59 @@ __device__ __forceinline__ void gemm_epilogue_row(const GemmParams& p, uint32_t 
     float v[32];
 #pragma unroll
     for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
-    if (p.epi == kEpiStoreF16 || p.epi == kEpiGeluBias) {
-      if (p.epi == kEpiGeluBias) {
+    if (p.epi == kEpiAccumF32 || p.epi == kEpiStoreF32) {
+      float4* dst = reinterpret_cast<float4*>(p.out_f32 + row * p.ld_f32 + col0);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        float4 w = make_float4(v[q * 4 + 0], v[q * 4 + 1], v[q * 4 + 2], v[q * 4 + 3]);
+        if (p.epi == kEpiAccumF32) {
+          const float4 o = dst[q];
+          w.x += o.x;
+          w.y += o.y;
+          w.z += o.z;
+          w.w += o.w;
+        }
+        dst[q] = w;
+      }
+      continue;
+    }
+    if (p.epi == kEpiGeluGrad) {
+      uint4* io = reinterpret_cast<uint4*>(p.out_h + row * p.ld_out + col0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 zz = io[q];
+        const __half* zh = reinterpret_cast<const __half*>(&zz);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[q * 8 + k] *= gelu_erf_grad(__half2float(zh[k]));
+        uint4 w;
+        w.x = pack_f16x2(v[q * 8 + 0], v[q * 8 + 1], bad);
+        w.y = pack_f16x2(v[q * 8 + 2], v[q * 8 + 3], bad);
+        w.z = pack_f16x2(v[q * 8 + 4], v[q * 8 + 5], bad);
+        w.w = pack_f16x2(v[q * 8 + 6], v[q * 8 + 7], bad);
+        io[q] = w;
+      }
+      continue;
+    }
+    if (p.epi == kEpiStoreF16 || p.epi == kEpiGeluBias || p.epi == kEpiGeluBiasKeep) {
+      if (p.epi == kEpiGeluBias || p.epi == kEpiGeluBiasKeep) {
         const uint4* bp = reinterpret_cast<const uint4*>(p.bias + col0);
+        uint4* keep = reinterpret_cast<uint4*>(p.out_h2 + row * p.ld_out + col0);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const uint4 bb = __ldg(bp + q);
           const __nv_bfloat16* bh = reinterpret_cast<const __nv_bfloat16*>(&bb);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) v[q * 8 + k] = gelu_erf(v[q * 8 + k] + __bfloat162float(bh[k]));
+          for (int k = 0; k < 8; ++k) v[q * 8 + k] += __bfloat162float(bh[k]);
+          if (p.epi == kEpiGeluBiasKeep) {
+            uint4 w;
+            w.x = pack_f16x2(v[q * 8 + 0], v[q * 8 + 1], bad);
+            w.y = pack_f16x2(v[q * 8 + 2], v[q * 8 + 3], bad);
+            w.z = pack_f16x2(v[q * 8 + 4], v[q * 8 + 5], bad);
+            w.w = pack_f16x2(v[q * 8 + 6], v[q * 8 + 7], bad);
+            keep[q] = w;
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) v[q * 8 + k] = gelu_erf(v[q * 8 + k]);
         }
       }
       uint4* dst = reinterpret_cast<uint4*>(p.out_h + row * p.ld_out + col0);
@@ -149,7 +209,10 @@ __device__ __forceinline__ void gemm_epilogue_row(const GemmParams& p, uint32_t 
     }
   }
   if (bad)
-    record_error(p.err, kErrRange, p.epi == kEpiGeluBias ? kSiteRangeHidden : kSiteRangeQKV);
+    record_error(p.err, kErrRange,
+                 (p.epi == kEpiGeluBias || p.epi == kEpiGeluBiasKeep || p.epi == kEpiGeluGrad)
+                     ? kSiteRangeHidden
+                     : kSiteRangeQKV);
 }
 
 // ---------------------------------------------------------------------------
@@ -176,7 +239,7 @@ constexpr int kPairSmem = kPairStages * kPairStageBytes + kGemmBarrierBytes + 10
 constexpr int kPairBM = 256;
 constexpr int kPairGroupM = 8;  // 256-row blocks per rasterisation group
 
-template <int EPI>
+template <int EPI, int LAYOUT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(), 1)
     gemm_f16_pair_kernel(const __grid_constant__ CUtensorMap mapA,
                          const __grid_constant__ CUtensorMap mapB0,
@@ -279,9 +342,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
           if (rank == 0) armed[stage] = static_cast<int>(phase);
           if (leader) {
             if (rank == 0) mbar_arrive_expect_tx(full0 + 8 * stage, 2 * kPairStageBytes);
-            tma_load_3d_pair(smem_u32(sA + stage * kPairABytes), &mapA, fb_leader, 0,
-                             mb * kPairBM + static_cast<int>(rank) * 128, kb * 2);
-            if (p.b_chunks == 2) {
+            const int m0 = mb * kPairBM + static_cast<int>(rank) * 128;
+            if (LAYOUT == kLayAnBn)  // A viewed [M/64][K][64]: 128 K rows x two M chunks
+              tma_load_3d_pair(smem_u32(sA + stage * kPairABytes), &mapA, fb_leader, 0,
+                               kb * kGemmBK, m0 >> 6);
+            else                     // A viewed [K/64][M][64]: 128 M rows x two K chunks
+              tma_load_3d_pair(smem_u32(sA + stage * kPairABytes), &mapA, fb_leader, 0, m0,
+                               kb * 2);
+            if (LAYOUT == kLayAkBk) {  // B viewed [K/64][N][64]: 128 N rows x two K chunks
+              tma_load_3d_pair(smem_u32(sB + stage * kPairBBytes), &mapB0, fb_leader, 0,
+                               nb * kGemmBN + static_cast<int>(rank) * 128, kb * 2);
+            } else if (p.b_chunks == 2) {
               tma_load_3d_pair(smem_u32(sB + stage * kPairBBytes), bmap[0], fb_leader, 0,
                                kb * kGemmBK, bchunk[0]);
             } else {
@@ -316,7 +387,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
     // ------------------------------------------------ UMMA issue (leader)
     // Whole warp (warp-uniform descriptors); the elected lane issues.
     const bool leader = elect_one();
-    constexpr uint32_t idesc = idesc_f16_f32(kPairBM, kGemmBN, false, true);
+    constexpr bool a_mn = LAYOUT == kLayAnBn, b_mn = LAYOUT != kLayAkBk;
+    constexpr uint32_t idesc = idesc_f16_f32(kPairBM, kGemmBN, a_mn, b_mn);
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
@@ -331,17 +403,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
           ok = false;
           break;
         }
-        // A: K-major, two 64-K chunks 16 KB apart; B: MN-major, LBO = the
-        // 16 KB between its two 64-column chunks; a 16-deep k-step moves 32 B
-        // in A and 16 rows (2 KB) in B.
-        const uint32_t a_lo = sdesc_lo(smem_u32(sA + stage * kPairABytes), 16);
-        const uint32_t b_lo = sdesc_lo(smem_u32(sB + stage * kPairBBytes), kPairBBytes / 2);
+        // K-major operand: two 64-K chunks 16 KB apart, a 16-deep k-step
+        // moves 32 B (and the next chunk after four).  MN-major operand:
+        // LBO = the 16 KB between its two 64-element chunks, a k-step moves
+        // 16 rows (2 KB).
+        const uint32_t a_lo =
+            sdesc_lo(smem_u32(sA + stage * kPairABytes), a_mn ? kPairABytes / 2 : 16);
+        const uint32_t b_lo =
+            sdesc_lo(smem_u32(sB + stage * kPairBBytes), b_mn ? kPairBBytes / 2 : 16);
         constexpr uint32_t hi = sdesc_hi(1024);
+        auto kstep = [](bool mn, int k) -> uint32_t {
+          return mn ? 128u * k : (k >> 2) * ((kPairABytes / 2) >> 4) + 2u * (k & 3);
+        };
         if (leader) {
 #pragma unroll
           for (int k = 0; k < kGemmBK / 16; ++k)
-            umma_ss_pair(d_tmem, a_lo + (k >> 2) * ((kPairABytes / 2) >> 4) + 2 * (k & 3), hi,
-                         b_lo + 128 * k, hi, idesc, (kb | k) != 0 ? 1u : 0u);
+            umma_ss_pair(d_tmem, a_lo + kstep(a_mn, k), hi, b_lo + kstep(b_mn, k), hi, idesc,
+                         (kb | k) != 0 ? 1u : 0u);
           umma_commit_pair_mc(empty0 + 8 * stage, 0x3);
         }
         __syncwarp();

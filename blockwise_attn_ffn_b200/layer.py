@@ -119,3 +119,43 @@ def layer_forward_train(x: torch.Tensor, p: Dict[str, torch.Tensor], h: int, cau
     if st != _lib.BPT_OK:
         raise _lib.BptError(st, "bpt_layer_forward_train")
     return out, stats, workspace
+
+
+GRAD_SHAPES = ["x", "ln1", "W_Q", "W_K", "W_V", "W_O", "ln2", "W_1", "b_1", "W_2", "b_2"]
+
+
+def layer_backward(x: torch.Tensor, p: Dict[str, torch.Tensor], h: int, causal: bool,
+                   stats: torch.Tensor, dZ: torch.Tensor,
+                   workspace: Optional[torch.Tensor] = None,
+                   stream: Optional[torch.cuda.Stream] = None):
+    """Gradients via ``bpt_layer_backward``; returns (grads, workspace) with
+    grads[name] fp32 for name in GRAD_SHAPES (ln1 / ln2 as [2, d]: d gamma;
+    d beta).  x and p as for ``layer_forward`` (bf16); stats from
+    ``layer_forward_train``; dZ [B, N, d] fp32."""
+    if x.dim() != 3:
+        raise ValueError("x must be [B, N, d]")
+    B, N, d = x.shape
+    d_ff = p["W_1"].shape[1]
+    code = _dtype_code(x)
+    tensors = [x] + [p[k] for k in PARAM_NAMES]
+    for t in tensors:
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != x.dtype:
+            raise ValueError("inputs must be contiguous CUDA tensors of one dtype")
+    if stats.dtype != torch.float32 or dZ.dtype != torch.float32 or not dZ.is_contiguous():
+        raise ValueError("stats and dZ must be contiguous fp32 CUDA tensors")
+    if workspace is None:
+        st, nbytes = _lib.bpt_layer_backward_workspace_size(B, N, d, h, d_ff, causal, code)
+        if st != _lib.BPT_OK:
+            raise _lib.BptError(st, "bpt_layer_backward_workspace_size")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
+    grads = {k: torch.empty(p[k].shape if k != "x" else x.shape, dtype=torch.float32,
+                            device=x.device) for k in GRAD_SHAPES}
+    s = stream if stream is not None else torch.cuda.current_stream(x.device)
+    order = ["x", "ln1", "W_Q", "W_K", "W_V", "W_O", "ln2", "W_1", "b_1", "W_2", "b_2"]
+    st = _lib.bpt_layer_backward(*[t.data_ptr() for t in tensors], stats.data_ptr(),
+                                 dZ.data_ptr(), B, N, d, h, d_ff, causal, code,
+                                 *[grads[k].data_ptr() for k in order],
+                                 workspace.data_ptr(), workspace.numel(), s.cuda_stream)
+    if st != _lib.BPT_OK:
+        raise _lib.BptError(st, "bpt_layer_backward")
+    return grads, workspace

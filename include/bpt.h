@@ -154,6 +154,58 @@ bpt_status bpt_layer_forward_train(const void* x, const void* ln1, const void* W
                                    size_t workspace_bytes, bpt_stream_t stream);
 
 /*
+ * bpt_layer_backward_workspace_size -- device workspace bytes
+ * bpt_layer_backward needs (pure host arithmetic).  BPT_BF16 layers only
+ * (BPT_ERR_UNSUPPORTED for BPT_F32); otherwise the shape rules of
+ * bpt_layer_workspace_size.
+ */
+bpt_status bpt_layer_backward_workspace_size(int64_t B, int64_t N, int64_t d, int64_t h,
+                                             int64_t d_ff, int causal, bpt_dtype dtype,
+                                             size_t* bytes);
+
+/*
+ * bpt_layer_backward -- gradients of sum(Z * dZ) with respect to x and every
+ * parameter, by the block recomputation of "Blockwise Parallel Transformer —
+ * BPT", section "The backward pass": from the layer input and the per-row
+ * softmax statistics of bpt_layer_forward_train, each block's scores,
+ * attention output and FFN hidden are recomputed and consumed at once; no
+ * [N, N] or [N, d_ff] tensor is formed (the FFN hidden exists for one wave of
+ * query blocks at a time, as in the forward).
+ *
+ *   x, ln1, W_Q .. b_2   the forward's inputs (bf16, as bpt_layer_forward)
+ *   stats [B, h, N, 2] fp32   the (m, l) bpt_layer_forward_train wrote
+ *   dZ    [B, N, d] fp32      upstream gradient of the layer output
+ * Outputs, fp32, overwritten (not accumulated):
+ *   dx [B, N, d]; d_ln1 [2, d] (d gamma1; d beta1); dW_Q, dW_K, dW_V, dW_O
+ *   [d, d]; d_ln2 [2, d]; dW_1 [d, d_ff]; db_1 [d_ff]; dW_2 [d_ff, d];
+ *   db_2 [d].
+ * All pointers are device pointers, 16-byte aligned; outputs must not
+ * overlap each other, the workspace, x, stats or dZ.  Workspace: >=
+ * bpt_layer_backward_workspace_size bytes, caller-owned.
+ *
+ * Arithmetic: the GEMMs run on the tensor cores with fp16 operands (the
+ * activations, upstream gradient and intermediate gradients rounded to fp16
+ * as in the forward) and fp32 accumulation; weight gradients accumulate in
+ * fp32 across waves; LayerNorm, GELU' and the bias / gamma / beta sums are
+ * fp32 (the sums in a fixed order: results are deterministic).  The
+ * attention gradients recompute P = exp(s - m) / l and run on the CUDA cores
+ * in fp32 from fp16 Q, K, V, o and dO.
+ * Returns BPT_ERR_UNSUPPORTED for BPT_F32; BPT_ERR_INVALID_ARG for a null,
+ * misaligned or overlapping pointer; BPT_ERR_WORKSPACE if the workspace is
+ * too small; otherwise as bpt_layer_forward (device errors via
+ * bpt_read_device_error).
+ */
+bpt_status bpt_layer_backward(const void* x, const void* ln1, const void* W_Q, const void* W_K,
+                              const void* W_V, const void* W_O, const void* ln2, const void* W_1,
+                              const void* b_1, const void* W_2, const void* b_2,
+                              const float* stats, const float* dZ, int64_t B, int64_t N,
+                              int64_t d, int64_t h, int64_t d_ff, int causal, bpt_dtype dtype,
+                              float* dx, float* d_ln1, float* dW_Q, float* dW_K, float* dW_V,
+                              float* dW_O, float* d_ln2, float* dW_1, float* db_1, float* dW_2,
+                              float* db_2, void* workspace, size_t workspace_bytes,
+                              bpt_stream_t stream);
+
+/*
  * bpt_read_device_error -- synchronises `stream`, reads and clears the error
  * word in the workspace header (written by the latest bpt_layer_forward on
  * this workspace).  Returns BPT_OK if nothing was recorded, BPT_ERR_TIMEOUT if
@@ -187,6 +239,16 @@ enum {
 };
 bpt_status bpt_profile_enable(int enable);
 bpt_status bpt_profile_read(double* ms, int64_t* launches, int n);
+
+/*
+ * bpt_debug_set_max_wave -- TEST HOOK: caps the query blocks of a wave at
+ * `blocks` (1..BPT_WAVE_BLOCKS; 0 restores BPT_WAVE_BLOCKS) for the calls
+ * that follow, so that small layers exercise the multi-wave paths (a
+ * sequence split over several waves, or one sequence per wave).  Results
+ * are the same up to the order of fp32 sums; workspace sizes must be queried
+ * after the call.  Returns BPT_ERR_INVALID_ARG outside that range.
+ */
+bpt_status bpt_debug_set_max_wave(int64_t blocks);
 
 /*
  * bpt_debug_inject_fault -- TEST HOOK for the failure-detection path.  The

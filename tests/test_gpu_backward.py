@@ -1,0 +1,110 @@
+"""bpt_layer_backward against the fp64 backward oracle.
+
+BPT page, section "The backward pass".  The CUDA path recomputes each wave
+of query blocks from x and the saved (m, l) (bpt_layer_forward_train) and
+accumulates the gradients; the oracle is the chain rule through the unfused
+layer (``oracle.layer_backward``, pinned against torch autograd).
+
+Tolerance.  Every GEMM operand on the backward path is rounded to fp16
+(relative 2^-11 ~ 4.9e-4) and the longest chain (dZ -> dH -> dHpre -> dVn ->
+dY -> dO -> dS -> dQ, dK, dV -> dU -> dx) passes about ten such roundings,
+each product accumulated in fp32: per-element relative error of order 5e-3.
+Each gradient tensor is held to a relative L2 error of 1e-2 and a largest
+elementwise error of 5 % of the tensor's largest magnitude.
+"""
+import numpy as np
+import pytest
+import torch
+
+import blockwise_attn_ffn_b200 as bpt
+import oracle
+from blockwise_attn_ffn_b200.inputs import LayerShape, make_inputs
+from test_gpu_parity import small
+
+pytestmark = pytest.mark.gpu
+
+NAMES = {"x": "x", "W_Q": "W_Q", "W_K": "W_K", "W_V": "W_V", "W_O": "W_O", "W_1": "W_1",
+         "b_1": "b_1", "W_2": "W_2", "b_2": "b_2"}
+
+CASES = [
+    small("bwd_dk128_causal", 2, 384, 256, 2, 512, True, seed=21),
+    small("bwd_dk64_noncausal_ragged", 1, 200, 256, 4, 512, False, seed=22),
+    small("bwd_dk128_ragged_bias", 1, 300, 384, 3, 768, True, seed=23, bias=0.5),
+    small("bwd_d192_straddle", 1, 260, 192, 3, 448, True, seed=24),
+]
+
+
+def upstream(cfg, seed=77):
+    return np.random.default_rng(seed).standard_normal((cfg.B, cfg.N, cfg.d)).astype(np.float32)
+
+
+def run_backward(cfg, inp, dZ):
+    dev = bpt.to_device(inp, cfg.dtype)
+    x = dev["x"]
+    _, stats, ws = bpt.layer_forward_train(x, dev, cfg.h, cfg.causal)
+    grads, bws = bpt.layer_backward(x, dev, cfg.h, cfg.causal, stats,
+                                    torch.from_numpy(dZ).cuda())
+    for w in (ws, bws):
+        st, site = bpt.bpt_read_device_error(w.data_ptr(), torch.cuda.current_stream().cuda_stream)
+        assert st == bpt.BPT_OK, f"device error {bpt.status_string(st)} at site {site}"
+    return {k: v.cpu().numpy().astype(np.float64) for k, v in grads.items()}
+
+
+def check(name, got, want):
+    assert np.all(np.isfinite(got)), f"{name}: non-finite gradient"
+    scale = np.abs(want).max()
+    rel_l2 = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
+    mx = np.abs(got - want).max()
+    print(f"  {name:12s} rel L2 {rel_l2:.2e}  max {mx / max(scale, 1e-30):.2e} of scale")
+    assert rel_l2 <= 1e-2, f"{name}: relative L2 error {rel_l2:.3e}"
+    assert mx <= 5e-2 * scale, f"{name}: max abs error {mx:.3e} vs scale {scale:.3e}"
+    return rel_l2
+
+
+@pytest.mark.parametrize("cfg", CASES, ids=lambda c: c.name)
+def test_backward_matches_oracle(cfg):
+    inp = make_inputs(cfg)
+    dZ = upstream(cfg)
+    got = run_backward(cfg, inp, dZ)
+    want = oracle.layer_backward(inp, cfg.h, cfg.causal, dZ.astype(np.float64))
+    for k in NAMES:
+        check(k, got[k], want[k])
+    for k, (g, b) in {"ln1": ("gamma1", "beta1"), "ln2": ("gamma2", "beta2")}.items():
+        check(k + ".gamma", got[k][0], want[g])
+        check(k + ".beta", got[k][1], want[b])
+
+
+# Multi-wave schedules on small layers (bpt_debug_set_max_wave): a sequence
+# split over three waves, and one whole sequence per wave.
+WAVE_CASES = [
+    (small("bwd_split_sequence", 1, 700, 256, 2, 512, True, seed=25), 2),
+    (small("bwd_split_sequence_dk64", 1, 650, 256, 4, 512, True, seed=26), 2),
+    (small("bwd_one_sequence_per_wave", 3, 256, 256, 4, 512, False, seed=27), 2),
+]
+
+
+@pytest.mark.parametrize("cfg,blocks", WAVE_CASES, ids=lambda c: getattr(c, "name", str(c)))
+def test_backward_multi_wave(cfg, blocks):
+    assert bpt.bpt_debug_set_max_wave(blocks) == bpt.BPT_OK
+    try:
+        inp = make_inputs(cfg)
+        dZ = upstream(cfg)
+        got = run_backward(cfg, inp, dZ)
+    finally:
+        bpt.bpt_debug_set_max_wave(0)
+    want = oracle.layer_backward(inp, cfg.h, cfg.causal, dZ.astype(np.float64))
+    for k in NAMES:
+        check(k, got[k], want[k])
+    for k, (g, b) in {"ln1": ("gamma1", "beta1"), "ln2": ("gamma2", "beta2")}.items():
+        check(k + ".gamma", got[k][0], want[g])
+        check(k + ".beta", got[k][1], want[b])
+
+
+def test_backward_is_deterministic():
+    cfg = CASES[0]
+    inp = make_inputs(cfg)
+    dZ = upstream(cfg)
+    a = run_backward(cfg, inp, dZ)
+    b = run_backward(cfg, inp, dZ)
+    for k in a:
+        np.testing.assert_array_equal(a[k], b[k], err_msg=k)
