@@ -1,0 +1,531 @@
+// Attention backward on the tcgen05 tensor cores ("Blockwise Parallel
+// Transformer — BPT", section "The backward pass": each block recomputes its
+// scores from the saved per-row statistics (m, l) and consumes them at once).
+//
+// Per head, with s = q.k / sqrt(d_k), P = exp(s - m) / l, D = rowsum(dO * O):
+//   dP = dO V^T,  dS = P * (dP - D),
+//   dV = P^T dO,  dK = dS^T Q / sqrt(d_k),  dQ = dS K / sqrt(d_k).
+// Two kernels, both deterministic (no atomics):
+//   attn_bwd_dkv_tc_kernel  one CTA per (128-key block, head, sequence of
+//       the wave): K, V stay in shared memory; the wave's query blocks that
+//       see the key block stream through a two-slot ring (Q, dO and the
+//       rows' (m, l, D)).  Per query block:
+//         S^T = K Q^T, dP^T = V dO^T     UMMA (SS), fp32 in TMEM
+//         P^T, dS^T                       elementwise warps, fp16 back in TMEM
+//         dV += P^T dO, dK += dS^T Q     UMMA with A from TMEM
+//       At the end dK, dV are added into the fp32 gradients (waves run in
+//       stream order, so each key row is updated by one CTA at a time).
+//   attn_bwd_dq_tc_kernel  one CTA per (128-query block, head): Q, dO stay
+//       in shared memory, K, V stream through the ring.  Per key block:
+//         S = Q K^T, dP = dO V^T          UMMA (SS)
+//         dS                              elementwise warps, fp16 in TMEM
+//         dQ += dS K                      UMMA with A from TMEM
+// A 128-row tile of Q, K, V or dO in shared memory ([d_k/64 chunks][128
+// rows][64], 128-byte swizzle) is a K-major operand in one product and an
+// MN-major one in another (same bytes, different descriptor).
+// Warp roles (256 threads): 0 TMA, 1 UMMA issue, 2 TMEM owner, 3 idle, 4..7
+// elementwise (thread = a row of the 128 the tile's TMEM lanes hold).  Every
+// wait is bounded; on expiry the kernel records a site code, drains and
+// frees its tensor memory.
+#pragma once
+
+#include "common.cuh"
+
+namespace bpt {
+
+struct AttnBwdTcParams {
+  int N, nb, h, d, causal, item0, count, seqs;
+  const float2* stats;  // [B][h][N] (m, l) from the forward
+  const float* D;       // [count * 128, h] rowsum(dO * O), this wave's block rows
+  float* dq;            // [B*N, d] written (this wave's query rows)
+  float* dk;            // [B*N, d] accumulated (+=)
+  float* dv;            // [B*N, d] accumulated (+=)
+  float scale;          // 1 / sqrt(d_k)
+  uint32_t* err;
+};
+
+template <int D>
+struct AttnBwdCfg {
+  static constexpr int TILE = 128 * D * 2;  // one 128-row fp16 tile
+  static constexpr int CHUNK = 128 * 128;   // one 64-column swizzled chunk
+  static constexpr int NSLOT = 2;
+  static constexpr int STATS = 3 * 128 * 4;  // per query row: -m log2 e, 1/l, D
+  // dK/dV kernel: K, V resident, ring of (Q, dO, stats)
+  static constexpr int KV_SLOT = (2 * TILE + STATS + 1023) / 1024 * 1024;
+  static constexpr int KV_OFF_RING = 2 * TILE;
+  static constexpr int KV_OFF_BAR = KV_OFF_RING + NSLOT * KV_SLOT;
+  static constexpr int KV_SMEM = KV_OFF_BAR + 256 + 1024;
+  // dQ kernel: Q, dO resident, ring of (K, V)
+  static constexpr int Q_SLOT = 2 * TILE;
+  static constexpr int Q_OFF_RING = 2 * TILE;
+  static constexpr int Q_OFF_BAR = Q_OFF_RING + NSLOT * Q_SLOT;
+  static constexpr int Q_SMEM = Q_OFF_BAR + 256 + 1024;
+  static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_A0 = 256, TM_A1 = 256 + D;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(KV_SMEM <= 232448 && Q_SMEM <= 232448, "shared memory budget");
+};
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Issue a 128 x 128 x d_k SS product: D[tmem] = A[a_lo] B[b_lo]^T, both
+// K-major tiles (the k-step walks 32 B inside a 64-column chunk, then the
+// next chunk).
+template <int D>
+__device__ __forceinline__ void bwd_issue_ss(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
+                                             uint32_t idesc) {
+  constexpr uint32_t hi = sdesc_hi(1024);
+#pragma unroll
+  for (int k = 0; k < D / 16; ++k) {
+    const uint32_t off = ((k >> 2) * AttnBwdCfg<D>::CHUNK + (k & 3) * 32) >> 4;
+    umma_ss(d_tmem, a_lo + off, hi, b_lo + off, hi, idesc, k > 0 ? 1u : 0u);
+  }
+}
+
+// Issue a 128 x d_k x 128 TS product: D[tmem] (+)= A[tmem, fp16 pairs] B,
+// with B an MN-major 128-row tile (k-step = 16 rows = 2 KB).
+template <int D>
+__device__ __forceinline__ void bwd_issue_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                             uint32_t idesc, bool first) {
+  constexpr uint32_t hi = sdesc_hi(1024);
+#pragma unroll
+  for (int k = 0; k < 128 / 16; ++k)
+    umma_ts(d_tmem, a_tmem + 8 * k, b_lo + ((k * 2048) >> 4), hi, idesc,
+            (!first || k > 0) ? 1u : 0u);
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
+// ----------------------------------------------------------------- dK, dV --
+template <int D>
+__global__ void __launch_bounds__(256, 1)
+    attn_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap mapQKV,
+                           const __grid_constant__ CUtensorMap mapDO, const AttnBwdTcParams p) {
+  using C = AttnBwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int jb = blockIdx.x, head = blockIdx.y;
+  const int bidx = p.seqs > 0 ? p.item0 / p.nb + static_cast<int>(blockIdx.z) : p.item0 / p.nb;
+  // this wave's query blocks of sequence bidx, and those that see key block jb
+  int ib_lo, ib_hi;
+  if (p.seqs > 0) {
+    ib_lo = 0;
+    ib_hi = p.nb;
+  } else {
+    ib_lo = p.item0 - bidx * p.nb;
+    ib_hi = ib_lo + p.count;
+  }
+  const int ib0 = p.causal ? max(ib_lo, jb) : ib_lo;
+  const int n_q = ib_hi - ib0;
+  if (n_q <= 0 || jb * 128 >= p.N) return;  // no query of this wave sees the block
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::KV_OFF_BAR);
+  const uint32_t kv_full = smem_u32(bars + 0);
+  const uint32_t ring_full0 = smem_u32(bars + 1);
+  const uint32_t ring_empty0 = smem_u32(bars + 1 + C::NSLOT);
+  const uint32_t s_full = smem_u32(bars + 1 + 2 * C::NSLOT);
+  const uint32_t p_full = smem_u32(bars + 2 + 2 * C::NSLOT);
+  const uint32_t acc_done = smem_u32(bars + 3 + 2 * C::NSLOT);
+  const uint32_t drain = smem_u32(bars + 4 + 2 * C::NSLOT);
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < C::NSLOT; ++s) {
+      mbar_init(ring_full0 + 8 * s, 1);
+      mbar_init(ring_empty0 + 8 * s, 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 4);
+    mbar_init(acc_done, 1);
+    mbar_init(drain, 1);
+    abort_sh = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(&tmem_base_sh), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  volatile int* abort_flag = &abort_sh;
+  const int chQ = head * D / 64, chK = (p.d + head * D) / 64, chV = (2 * p.d + head * D) / 64;
+  const long long lbase = static_cast<long long>(bidx * p.nb - p.item0) * 128;  // wave row of pos 0
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    const bool leader = lane == 0;
+    int armed[C::NSLOT];
+    for (int s = 0; s < C::NSLOT; ++s) armed[s] = -1;
+    if (leader) {
+      mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
+      tma_load_4d(smem_u32(smem), &mapQKV, kv_full, 0, jb * 128, chK, bidx);
+      tma_load_4d(smem_u32(smem + C::TILE), &mapQKV, kv_full, 0, jb * 128, chV, bidx);
+    }
+    bool ok = true;
+    for (int t = 0; t < n_q && ok; ++t) {
+      const int slot = t % C::NSLOT;
+      const uint32_t phase = static_cast<uint32_t>((t / C::NSLOT) & 1);
+      if (!mbar_wait_warp(ring_empty0 + 8 * slot, phase ^ 1u, abort_flag, p.err,
+                          kSiteAttnProducer)) {
+        ok = false;
+        break;
+      }
+      const int ib = ib0 + t;
+      uint8_t* sl = smem + C::KV_OFF_RING + slot * C::KV_SLOT;
+      float* st = reinterpret_cast<float*>(sl + 2 * C::TILE);
+      for (int q = lane; q < 128; q += 32) {
+        const int qp = ib * 128 + q;
+        float a = -INFINITY, il = 0.f, dd = 0.f;
+        if (qp < p.N) {
+          const float2 ml = p.stats[(static_cast<long long>(bidx) * p.h + head) * p.N + qp];
+          a = -ml.x * kLog2e;
+          il = 1.0f / ml.y;
+          dd = p.D[(lbase + qp) * p.h + head];
+        }
+        st[q] = a;
+        st[128 + q] = il;
+        st[256 + q] = dd;
+      }
+      __syncwarp();
+      if (leader) {
+        armed[slot] = static_cast<int>(phase);
+        mbar_arrive_expect_tx(ring_full0 + 8 * slot, 2 * C::TILE);
+        tma_load_4d(smem_u32(sl), &mapQKV, ring_full0 + 8 * slot, 0, ib * 128, chQ, bidx);
+        tma_load_3d(smem_u32(sl + C::TILE), &mapDO, ring_full0 + 8 * slot, 0,
+                    static_cast<int>(lbase + ib * 128), head * D / 64);
+      }
+      __syncwarp();
+    }
+    mbar_wait_drain(kv_full, 0, p.err);
+    for (int s = 0; s < C::NSLOT; ++s)
+      if (armed[s] >= 0) mbar_wait_drain(ring_full0 + 8 * s, static_cast<uint32_t>(armed[s]), p.err);
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- UMMA issue
+    const bool leader = lane == 0;
+    constexpr uint32_t idesc_s = idesc_f16_f32(128, 128, false, false);
+    constexpr uint32_t idesc_o = idesc_f16_f32(128, D, false, true);
+    const uint32_t k_lo = sdesc_lo(smem_u32(smem), 16);
+    const uint32_t v_lo = sdesc_lo(smem_u32(smem + C::TILE), 16);
+    auto commit = [&](uint32_t bar) {
+      if (leader) umma_commit(bar);
+      __syncwarp();
+    };
+    bool ok = mbar_wait_warp(kv_full, 0, abort_flag, p.err, kSiteAttnMma);
+    for (int t = 0; t < n_q && ok; ++t) {
+      const int slot = t % C::NSLOT;
+      const uint32_t phase = static_cast<uint32_t>((t / C::NSLOT) & 1);
+      if (!mbar_wait_warp(ring_full0 + 8 * slot, phase, abort_flag, p.err, kSiteAttnMma)) break;
+      tc_fence_after();
+      const uint32_t sl = smem_u32(smem + C::KV_OFF_RING + slot * C::KV_SLOT);
+      if (leader) {
+        bwd_issue_ss<D>(tmem + C::TM_S, k_lo, sdesc_lo(sl, 16), idesc_s);               // S^T
+        bwd_issue_ss<D>(tmem + C::TM_DP, v_lo, sdesc_lo(sl + C::TILE, 16), idesc_s);    // dP^T
+      }
+      __syncwarp();
+      commit(s_full);
+      if (!mbar_wait_warp(p_full, static_cast<uint32_t>(t & 1), abort_flag, p.err,
+                          kSiteAttnMma))
+        break;
+      tc_fence_after();
+      if (leader) {
+        bwd_issue_ts<D>(tmem + C::TM_A0, tmem + C::TM_S, sdesc_lo(sl + C::TILE, C::CHUNK),
+                        idesc_o, t == 0);                                               // dV
+        bwd_issue_ts<D>(tmem + C::TM_A1, tmem + C::TM_DP, sdesc_lo(sl, C::CHUNK), idesc_o,
+                        t == 0);                                                        // dK
+      }
+      __syncwarp();
+      commit(ring_empty0 + 8 * slot);
+    }
+    commit(acc_done);
+    commit(drain);
+    mbar_wait_drain(drain, 0, p.err);
+  } else if (warp >= 4) {
+    // --------------------------------------------------------- elementwise
+    const int e = warp & 3;
+    const int kr = e * 32 + lane;  // key row of the block
+    const int kp = jb * 128 + kr;
+    const bool key_ok = kp < p.N;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(e * 32) << 16);
+    const float c = p.scale * kLog2e;
+    bool ok = true;
+    for (int t = 0; t < n_q && ok; ++t) {
+      if (!mbar_wait_warp(s_full, static_cast<uint32_t>(t & 1), abort_flag, p.err,
+                          kSiteAttnSoftmax)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int slot = t % C::NSLOT;
+      // The producer warp wrote this slot's statistics with ordinary stores
+      // before arriving on its full barrier: acquire that barrier here too
+      // (its phase for block t has completed; the slot is released only
+      // after this warp's p_full arrival below).
+      if (!mbar_wait_warp(ring_full0 + 8 * slot, static_cast<uint32_t>((t / C::NSLOT) & 1),
+                          abort_flag, p.err, kSiteAttnSoftmax)) {
+        ok = false;
+        break;
+      }
+      const float* st =
+          reinterpret_cast<const float*>(smem + C::KV_OFF_RING + slot * C::KV_SLOT + 2 * C::TILE);
+      const int ib = ib0 + t;
+      const bool diag = p.causal && ib == jb;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t sr[32], dr[32];
+        tmem_ld_32x32b_x32(t_lane + C::TM_S + cc * 32, sr);
+        tmem_ld_32x32b_x32(t_lane + C::TM_DP + cc * 32, dr);
+        tmem_ld_wait();
+        uint32_t pk[16], dk16[16];
+#pragma unroll
+        for (int k = 0; k < 32; k += 2) {
+          float pv[2], dv2[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int q = cc * 32 + k + u;
+            float pr = ex2_approx(fmaf(__uint_as_float(sr[k + u]), c, st[q])) * st[128 + q];
+            if (!key_ok || (diag && kr > q)) pr = 0.f;
+            pv[u] = pr;
+            dv2[u] = pr * (__uint_as_float(dr[k + u]) - st[256 + q]);
+          }
+          pk[k >> 1] = pack_f16x2(pv[0], pv[1]);
+          dk16[k >> 1] = pack_f16x2(dv2[0], dv2[1]);
+        }
+        tmem_st16(t_lane + C::TM_S + cc * 16, pk);
+        tmem_st16(t_lane + C::TM_DP + cc * 16, dk16);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    if (ok && mbar_wait_warp(acc_done, 0, abort_flag, p.err, kSiteAttnSoftmax)) {
+      tc_fence_after();
+      const long long g = static_cast<long long>(bidx) * p.N + kp;
+      float* dvr = p.dv + g * p.d + head * D;
+      float* dkr = p.dk + g * p.d + head * D;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t a[32], b[32];  // warp-collective loads: every lane takes them
+        tmem_ld_32x32b_x32(t_lane + C::TM_A0 + cc * 32, a);
+        tmem_ld_32x32b_x32(t_lane + C::TM_A1 + cc * 32, b);
+        tmem_ld_wait();
+        if (key_ok) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            dvr[cc * 32 + k] += __uint_as_float(a[k]);
+            dkr[cc * 32 + k] += __uint_as_float(b[k]) * p.scale;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// ---------------------------------------------------------------------- dQ --
+template <int D>
+__global__ void __launch_bounds__(256, 1)
+    attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap mapQKV,
+                          const __grid_constant__ CUtensorMap mapDO, const AttnBwdTcParams p) {
+  using C = AttnBwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int qb = blockIdx.x, head = blockIdx.y;
+  const int item = p.item0 + qb;
+  const int bidx = item / p.nb, ib = item - (item / p.nb) * p.nb;
+  const int n_kv = p.causal ? ib + 1 : p.nb;
+  const long long lrow = static_cast<long long>(qb) * 128;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::Q_OFF_BAR);
+  const uint32_t q_full = smem_u32(bars + 0);
+  const uint32_t ring_full0 = smem_u32(bars + 1);
+  const uint32_t ring_empty0 = smem_u32(bars + 1 + C::NSLOT);
+  const uint32_t s_full = smem_u32(bars + 1 + 2 * C::NSLOT);
+  const uint32_t p_full = smem_u32(bars + 2 + 2 * C::NSLOT);
+  const uint32_t acc_done = smem_u32(bars + 3 + 2 * C::NSLOT);
+  const uint32_t drain = smem_u32(bars + 4 + 2 * C::NSLOT);
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < C::NSLOT; ++s) {
+      mbar_init(ring_full0 + 8 * s, 1);
+      mbar_init(ring_empty0 + 8 * s, 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 4);
+    mbar_init(acc_done, 1);
+    mbar_init(drain, 1);
+    abort_sh = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(&tmem_base_sh), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  volatile int* abort_flag = &abort_sh;
+  const int chQ = head * D / 64, chK = (p.d + head * D) / 64, chV = (2 * p.d + head * D) / 64;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    const bool leader = lane == 0;
+    int armed[C::NSLOT];
+    for (int s = 0; s < C::NSLOT; ++s) armed[s] = -1;
+    if (leader) {
+      mbar_arrive_expect_tx(q_full, 2 * C::TILE);
+      tma_load_4d(smem_u32(smem), &mapQKV, q_full, 0, ib * 128, chQ, bidx);
+      tma_load_3d(smem_u32(smem + C::TILE), &mapDO, q_full, 0, static_cast<int>(lrow),
+                  head * D / 64);
+    }
+    bool ok = true;
+    for (int j = 0; j < n_kv && ok; ++j) {
+      const int slot = j % C::NSLOT;
+      const uint32_t phase = static_cast<uint32_t>((j / C::NSLOT) & 1);
+      if (!mbar_wait_warp(ring_empty0 + 8 * slot, phase ^ 1u, abort_flag, p.err,
+                          kSiteAttnProducer)) {
+        ok = false;
+        break;
+      }
+      if (leader) {
+        armed[slot] = static_cast<int>(phase);
+        const uint32_t sl = smem_u32(smem + C::Q_OFF_RING + slot * C::Q_SLOT);
+        mbar_arrive_expect_tx(ring_full0 + 8 * slot, 2 * C::TILE);
+        tma_load_4d(sl, &mapQKV, ring_full0 + 8 * slot, 0, j * 128, chK, bidx);
+        tma_load_4d(sl + C::TILE, &mapQKV, ring_full0 + 8 * slot, 0, j * 128, chV, bidx);
+      }
+      __syncwarp();
+    }
+    mbar_wait_drain(q_full, 0, p.err);
+    for (int s = 0; s < C::NSLOT; ++s)
+      if (armed[s] >= 0) mbar_wait_drain(ring_full0 + 8 * s, static_cast<uint32_t>(armed[s]), p.err);
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- UMMA issue
+    const bool leader = lane == 0;
+    constexpr uint32_t idesc_s = idesc_f16_f32(128, 128, false, false);
+    constexpr uint32_t idesc_o = idesc_f16_f32(128, D, false, true);
+    const uint32_t q_lo = sdesc_lo(smem_u32(smem), 16);
+    const uint32_t do_lo = sdesc_lo(smem_u32(smem + C::TILE), 16);
+    auto commit = [&](uint32_t bar) {
+      if (leader) umma_commit(bar);
+      __syncwarp();
+    };
+    bool ok = mbar_wait_warp(q_full, 0, abort_flag, p.err, kSiteAttnMma);
+    for (int j = 0; j < n_kv && ok; ++j) {
+      const int slot = j % C::NSLOT;
+      const uint32_t phase = static_cast<uint32_t>((j / C::NSLOT) & 1);
+      if (!mbar_wait_warp(ring_full0 + 8 * slot, phase, abort_flag, p.err, kSiteAttnMma)) break;
+      tc_fence_after();
+      const uint32_t sl = smem_u32(smem + C::Q_OFF_RING + slot * C::Q_SLOT);
+      if (leader) {
+        bwd_issue_ss<D>(tmem + C::TM_S, q_lo, sdesc_lo(sl, 16), idesc_s);               // S
+        bwd_issue_ss<D>(tmem + C::TM_DP, do_lo, sdesc_lo(sl + C::TILE, 16), idesc_s);   // dP
+      }
+      __syncwarp();
+      commit(s_full);
+      if (!mbar_wait_warp(p_full, static_cast<uint32_t>(j & 1), abort_flag, p.err,
+                          kSiteAttnMma))
+        break;
+      tc_fence_after();
+      if (leader)
+        bwd_issue_ts<D>(tmem + C::TM_A0, tmem + C::TM_S, sdesc_lo(sl, C::CHUNK), idesc_o,
+                        j == 0);                                                        // dQ
+      __syncwarp();
+      commit(ring_empty0 + 8 * slot);
+    }
+    commit(acc_done);
+    commit(drain);
+    mbar_wait_drain(drain, 0, p.err);
+  } else if (warp >= 4) {
+    // --------------------------------------------------------- elementwise
+    const int e = warp & 3;
+    const int qr = e * 32 + lane;  // query row of the block
+    const int qp = ib * 128 + qr;
+    const bool q_ok = qp < p.N;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(e * 32) << 16);
+    const float c = p.scale * kLog2e;
+    float a = -INFINITY, il = 0.f, dd = 0.f;
+    if (q_ok) {
+      const float2 ml = p.stats[(static_cast<long long>(bidx) * p.h + head) * p.N + qp];
+      a = -ml.x * kLog2e;
+      il = 1.0f / ml.y;
+      dd = p.D[(lrow + qr) * p.h + head];
+    }
+    bool ok = true;
+    for (int j = 0; j < n_kv && ok; ++j) {
+      if (!mbar_wait_warp(s_full, static_cast<uint32_t>(j & 1), abort_flag, p.err,
+                          kSiteAttnSoftmax)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const bool diag = p.causal && j == ib;
+      const int klim = p.N - j * 128;  // keys >= klim are past the sequence
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t sr[32], dr[32];
+        tmem_ld_32x32b_x32(t_lane + C::TM_S + cc * 32, sr);
+        tmem_ld_32x32b_x32(t_lane + C::TM_DP + cc * 32, dr);
+        tmem_ld_wait();
+        uint32_t ds16[16];
+#pragma unroll
+        for (int k = 0; k < 32; k += 2) {
+          float dsv[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int kc = cc * 32 + k + u;
+            float pr = ex2_approx(fmaf(__uint_as_float(sr[k + u]), c, a)) * il;
+            if (kc >= klim || (diag && kc > qr)) pr = 0.f;
+            dsv[u] = pr * (__uint_as_float(dr[k + u]) - dd);
+          }
+          ds16[k >> 1] = pack_f16x2(dsv[0], dsv[1]);
+        }
+        tmem_st16(t_lane + C::TM_S + cc * 16, ds16);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    if (ok && mbar_wait_warp(acc_done, 0, abort_flag, p.err, kSiteAttnSoftmax)) {
+      tc_fence_after();
+      float* dst = p.dq + (static_cast<long long>(bidx) * p.N + qp) * p.d + head * D;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(t_lane + C::TM_A0 + cc * 32, v);
+        tmem_ld_wait();
+        if (q_ok) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) dst[cc * 32 + k] = __uint_as_float(v[k]) * p.scale;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+}  // namespace bpt

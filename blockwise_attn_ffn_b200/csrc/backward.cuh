@@ -8,14 +8,11 @@
 //   * row copies fp32 -> fp16 (GEMM operands),
 //   * LayerNorm backward (one warp per row) and the deterministic column
 //     sums of the bias, gamma and beta gradients,
-//   * the attention backward: the row terms D = rowsum(dO * O) per head and
-//     the dQ and dK/dV kernels, which recompute P = exp(s - m) / l from the
-//     saved statistics.  These run on CUDA cores in fp32 arithmetic on fp16
-//     operands (64-row tiles).
-// Formulas (standard calculus), per head with s = q.k / sqrt(d_k):
-//   P = exp(s - m) / l,  dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),
-//   dQ = dS K / sqrt(d_k),  dK = dS^T Q / sqrt(d_k);
-//   LayerNorm y = g * xh + b: dx = rstd * (dxh - mean(dxh) - xh * mean(dxh * xh)),
+//   * the attention backward's row terms D = rowsum(dO * O) per head (the
+//     attention gradients themselves run on the tensor cores,
+//     attn_bwd_tc.cuh).
+// LayerNorm y = g * xh + b (standard calculus):
+//   dx = rstd * (dxh - mean(dxh) - xh * mean(dxh * xh)),
 //   dxh = dy * g,  dg = sum_rows dy * xh,  db = sum_rows dy.
 #pragma once
 
@@ -177,224 +174,6 @@ __global__ void attn_row_dot_kernel(const __half* __restrict__ dO, const __half*
       s += __half2float(dO[r * d + t * dk + c]) * __half2float(O[r * d + t * dk + c]);
     s = warp_sum(s);
     if (lane == 0) D[r * h + t] = s;
-  }
-}
-
-// ------------------------------------------------- attention gradients --
-struct AttnBwdParams {
-  const __half* qkv;     // [B*N, 3d] fp16: Q | K | V per token (global rows)
-  const __half* o;       // [count * 128, d] fp16, this wave's block rows
-  const __half* dO;      // [count * 128, d] fp16, this wave's block rows
-  const float* D;        // [count * 128, h] rowsum(dO * O) per head
-  const float2* stats;   // [B][h][N] (m, l) from the forward
-  float* dq;             // [B*N, d] written for this wave's rows
-  float* dk;             // [B*N, d] accumulated (+=)
-  float* dv;             // [B*N, d] accumulated (+=)
-  int N, nb, h, d, causal, item0, count, seqs;
-  float scale;           // 1 / sqrt(d_k)
-};
-
-constexpr int kBwdRows = 64;  // query / key tile of the SIMT attention backward
-
-template <int DK>
-struct AttnBwdSmem {
-  static constexpr int TILE = kBwdRows * DK;              // floats
-  static constexpr int PT = kBwdRows * (kBwdRows + 1);    // floats, padded
-  static constexpr int DQ_BYTES = (4 * TILE + PT + 3 * kBwdRows) * 4;
-  static constexpr int DKV_BYTES = (4 * TILE + 2 * PT + 3 * kBwdRows) * 4;
-};
-
-__device__ __forceinline__ void load_tile_f16(float* dst, const __half* src, long long ld,
-                                              int col0, int dk, long long row0, int nrows_valid) {
-  // dst[r][c] = src[(row0 + r) * ld + col0 + c] for r < nrows_valid, else 0
-  for (int t = threadIdx.x; t < kBwdRows * dk; t += blockDim.x) {
-    const int r = t / dk, c = t - (t / dk) * dk;
-    dst[t] = r < nrows_valid ? __half2float(src[(row0 + r) * ld + col0 + c]) : 0.f;
-  }
-}
-
-// dQ for one 64-row query tile of the wave and one head.  256 threads: row
-// r = tid / 4 of the tile, sub = tid % 4 takes key columns sub, sub + 4, ...
-template <int DK>
-__global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const AttnBwdParams p) {
-  extern __shared__ float smf[];
-  using S = AttnBwdSmem<DK>;
-  float* sQ = smf;
-  float* sdO = sQ + S::TILE;
-  float* sK = sdO + S::TILE;
-  float* sV = sK + S::TILE;
-  float* sS = sV + S::TILE;          // dS [64][65]
-  float* sM = sS + S::PT;            // m, l, D per row
-  float* sL = sM + kBwdRows;
-  float* sD = sL + kBwdRows;
-  const int head = blockIdx.y;
-  const int q = blockIdx.x;                       // 64-row tile of the wave
-  const int item = p.item0 + q / 2;
-  const int bidx = item / p.nb, iblk = item - (item / p.nb) * p.nb;
-  const int pos0 = iblk * 128 + (q & 1) * kBwdRows;
-  const long long lrow0 = static_cast<long long>(q / 2) * 128 + (q & 1) * kBwdRows;
-  const int nvalid = max(0, min(kBwdRows, p.N - pos0));
-  const long long g0 = static_cast<long long>(bidx) * p.N + pos0;
-  const long long ld3 = 3LL * p.d;
-  const int r = threadIdx.x >> 2, sub = threadIdx.x & 3;
-  if (nvalid == 0) return;
-  load_tile_f16(sQ, p.qkv, ld3, head * DK, DK, g0, nvalid);
-  load_tile_f16(sdO, p.dO, p.d, head * DK, DK, lrow0, nvalid);
-  if (threadIdx.x < kBwdRows) {
-    const int rr = threadIdx.x;
-    const bool ok = rr < nvalid;
-    const float2 st = ok ? p.stats[(static_cast<long long>(bidx) * p.h + head) * p.N + pos0 + rr]
-                         : make_float2(0.f, 1.f);
-    sM[rr] = st.x;
-    sL[rr] = st.y;
-    sD[rr] = ok ? p.D[(lrow0 + rr) * p.h + head] : 0.f;
-  }
-  float acc[DK / 4];
-#pragma unroll
-  for (int t = 0; t < DK / 4; ++t) acc[t] = 0.f;
-  const int pos = pos0 + r;
-  const int kend = p.causal ? min(p.N, pos0 + kBwdRows) : p.N;
-  for (int k0 = 0; k0 < kend; k0 += kBwdRows) {
-    __syncthreads();
-    const int kvalid = min(kBwdRows, p.N - k0);
-    const long long gk = static_cast<long long>(bidx) * p.N + k0;
-    load_tile_f16(sK, p.qkv, ld3, p.d + head * DK, DK, gk, kvalid);
-    load_tile_f16(sV, p.qkv, ld3, 2 * p.d + head * DK, DK, gk, kvalid);
-    __syncthreads();
-    const float m = sM[r], linv = 1.0f / sL[r], Dr = sD[r];
-#pragma unroll 4
-    for (int t = 0; t < kBwdRows / 4; ++t) {
-      const int kk = sub + 4 * t;
-      const int kp = k0 + kk;
-      float ds = 0.f;
-      if (r < nvalid && kk < kvalid && (!p.causal || kp <= pos)) {
-        float sc = 0.f, dp = 0.f;
-        for (int c = 0; c < DK; ++c) {
-          sc = fmaf(sQ[r * DK + c], sK[kk * DK + c], sc);
-          dp = fmaf(sdO[r * DK + c], sV[kk * DK + c], dp);
-        }
-        const float pr = expf(sc * p.scale - m) * linv;
-        ds = pr * (dp - Dr);
-      }
-      sS[r * (kBwdRows + 1) + kk] = ds;
-    }
-    __syncwarp();
-#pragma unroll
-    for (int t = 0; t < DK / 4; ++t) {
-      const int c = sub + 4 * t;
-      float a = 0.f;
-      for (int kk = 0; kk < kBwdRows; ++kk) a = fmaf(sS[r * (kBwdRows + 1) + kk], sK[kk * DK + c], a);
-      acc[t] += a;
-    }
-  }
-  if (r < nvalid) {
-    float* dst = p.dq + (g0 + r) * p.d + head * DK;
-#pragma unroll
-    for (int t = 0; t < DK / 4; ++t) dst[sub + 4 * t] = acc[t] * p.scale;
-  }
-}
-
-// dK, dV contributions of this wave's query rows to one 64-key tile of one
-// head and sequence (grid: key tiles x heads x sequences of the wave).
-// 256 threads: key row k = tid / 4, sub = tid % 4 takes query columns sub,
-// sub + 4, ... of each query tile, and head columns sub, sub + 4, ... of the
-// accumulators.
-template <int DK>
-__global__ void __launch_bounds__(256) attn_bwd_dkv_kernel(const AttnBwdParams p) {
-  extern __shared__ float smf[];
-  using S = AttnBwdSmem<DK>;
-  float* sQ = smf;
-  float* sdO = sQ + S::TILE;
-  float* sK = sdO + S::TILE;
-  float* sV = sK + S::TILE;
-  float* sP = sV + S::TILE;          // P^T [64 keys][65]
-  float* sS = sP + S::PT;            // dS^T [64 keys][65]
-  float* sM = sS + S::PT;
-  float* sL = sM + kBwdRows;
-  float* sD = sL + kBwdRows;
-  const int head = blockIdx.y;
-  const int bidx = (p.seqs > 0 ? p.item0 / p.nb + static_cast<int>(blockIdx.z) : p.item0 / p.nb);
-  const int k0 = blockIdx.x * kBwdRows;
-  if (k0 >= p.N) return;
-  // this wave's query positions in sequence bidx: [qlo, qhi)
-  int qlo, qhi;
-  long long lbase;  // wave scratch row of position 0 of this sequence
-  if (p.seqs > 0) {
-    qlo = 0;
-    qhi = p.N;
-    lbase = static_cast<long long>(bidx * p.nb - p.item0) * 128;
-  } else {
-    const int i0 = p.item0 - bidx * p.nb;
-    qlo = i0 * 128;
-    qhi = min(p.N, (i0 + p.count) * 128);
-    lbase = -static_cast<long long>(qlo);
-  }
-  const int qstart = p.causal ? max(qlo, k0 - (k0 % kBwdRows)) : qlo;
-  if (qstart >= qhi) return;
-  const int kvalid = min(kBwdRows, p.N - k0);
-  const long long ld3 = 3LL * p.d;
-  const long long gk = static_cast<long long>(bidx) * p.N + k0;
-  const int k = threadIdx.x >> 2, sub = threadIdx.x & 3;
-  load_tile_f16(sK, p.qkv, ld3, p.d + head * DK, DK, gk, kvalid);
-  load_tile_f16(sV, p.qkv, ld3, 2 * p.d + head * DK, DK, gk, kvalid);
-  float ak[DK / 4], av[DK / 4];
-#pragma unroll
-  for (int t = 0; t < DK / 4; ++t) ak[t] = av[t] = 0.f;
-  const int kp = k0 + k;
-  for (int q0 = qstart; q0 < qhi; q0 += kBwdRows) {
-    __syncthreads();
-    const int qvalid = min(kBwdRows, qhi - q0);
-    const long long gq = static_cast<long long>(bidx) * p.N + q0;
-    load_tile_f16(sQ, p.qkv, ld3, head * DK, DK, gq, qvalid);
-    load_tile_f16(sdO, p.dO, p.d, head * DK, DK, lbase + q0, qvalid);
-    if (threadIdx.x < kBwdRows) {
-      const int rr = threadIdx.x;
-      const bool ok = rr < qvalid;
-      const float2 st = ok ? p.stats[(static_cast<long long>(bidx) * p.h + head) * p.N + q0 + rr]
-                           : make_float2(0.f, 1.f);
-      sM[rr] = st.x;
-      sL[rr] = st.y;
-      sD[rr] = ok ? p.D[(lbase + q0 + rr) * p.h + head] : 0.f;
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int t = 0; t < kBwdRows / 4; ++t) {
-      const int rr = sub + 4 * t;
-      const int qp = q0 + rr;
-      float pr = 0.f, ds = 0.f;
-      if (k < kvalid && rr < qvalid && (!p.causal || kp <= qp)) {
-        float sc = 0.f, dp = 0.f;
-        for (int c = 0; c < DK; ++c) {
-          sc = fmaf(sQ[rr * DK + c], sK[k * DK + c], sc);
-          dp = fmaf(sdO[rr * DK + c], sV[k * DK + c], dp);
-        }
-        pr = expf(sc * p.scale - sM[rr]) / sL[rr];
-        ds = pr * (dp - sD[rr]);
-      }
-      sP[k * (kBwdRows + 1) + rr] = pr;
-      sS[k * (kBwdRows + 1) + rr] = ds;
-    }
-    __syncwarp();
-#pragma unroll
-    for (int t = 0; t < DK / 4; ++t) {
-      const int c = sub + 4 * t;
-      float a = 0.f, b = 0.f;
-      for (int rr = 0; rr < kBwdRows; ++rr) {
-        a = fmaf(sP[k * (kBwdRows + 1) + rr], sdO[rr * DK + c], a);
-        b = fmaf(sS[k * (kBwdRows + 1) + rr], sQ[rr * DK + c], b);
-      }
-      av[t] += a;
-      ak[t] += b;
-    }
-  }
-  if (k < kvalid) {
-    float* dkr = p.dk + (gk + k) * p.d + head * DK;
-    float* dvr = p.dv + (gk + k) * p.d + head * DK;
-#pragma unroll
-    for (int t = 0; t < DK / 4; ++t) {
-      dkr[sub + 4 * t] += ak[t] * p.scale;
-      dvr[sub + 4 * t] += av[t];
-    }
   }
 }
 

@@ -25,6 +25,7 @@
 #include <vector>
 
 #include "bpt.h"
+#include "attn_bwd_tc.cuh"
 #include "attn_pair_tc.cuh"
 #include "backward.cuh"
 #include "common.cuh"
@@ -201,10 +202,10 @@ bpt_status device_info(int* sms, int* pair_clusters = nullptr) {
           set_smem(bpt::gemm_f16_pair_kernel<4, bpt::kLayAnBn>, bpt::kPairSmem) ||
           set_smem(bpt::gemm_f16_pair_kernel<4, bpt::kLayAkBk>, bpt::kPairSmem) ||
           set_smem(bpt::gemm_f16_pair_kernel<8, bpt::kLayAkBk>, bpt::kPairSmem) ||
-          set_smem(bpt::attn_bwd_dq_kernel<128>, bpt::AttnBwdSmem<128>::DQ_BYTES) ||
-          set_smem(bpt::attn_bwd_dkv_kernel<128>, bpt::AttnBwdSmem<128>::DKV_BYTES) ||
-          set_smem(bpt::attn_bwd_dq_kernel<64>, bpt::AttnBwdSmem<64>::DQ_BYTES) ||
-          set_smem(bpt::attn_bwd_dkv_kernel<64>, bpt::AttnBwdSmem<64>::DKV_BYTES) ||
+          set_smem(bpt::attn_bwd_dq_tc_kernel<128>, bpt::AttnBwdCfg<128>::Q_SMEM) ||
+          set_smem(bpt::attn_bwd_dkv_tc_kernel<128>, bpt::AttnBwdCfg<128>::KV_SMEM) ||
+          set_smem(bpt::attn_bwd_dq_tc_kernel<64>, bpt::AttnBwdCfg<64>::Q_SMEM) ||
+          set_smem(bpt::attn_bwd_dkv_tc_kernel<64>, bpt::AttnBwdCfg<64>::KV_SMEM) ||
           cudaFuncSetAttribute(bpt::attn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (3 * 64 * 128 + 64 * 65) * 4) != cudaSuccess)
         return BPT_ERR_CUDA;
@@ -269,10 +270,11 @@ bool encode_f16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims
 // as [K/64][rows][64]; a box is 128 rows x two 64-column chunks (32 KB,
 // chunk-major in shared memory).  The A operand of the forward, and the B
 // operand [N, K] of the data-gradient GEMMs.
-bool map_a(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int64_t ld = 0) {
+bool map_a(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int64_t ld = 0,
+           int chunks = 2) {
   const uint64_t dims[3] = {64, uint64_t(rows), uint64_t(K / 64)};
   const uint64_t st[2] = {uint64_t(ld > 0 ? ld : K) * 2, 128};
-  const uint32_t box[3] = {64, 128, 2};
+  const uint32_t box[3] = {64, 128, uint32_t(chunks)};
   return encode_f16(m, base, 3, dims, st, box);
 }
 // GEMM operand, row-contiguous along the output axis: [K, cols] with row
@@ -729,7 +731,7 @@ bpt_status backward_bf16(const Plan& P, const BwdLayout& L, const void* x, const
   const int qkv_chunks = (d % 128 == 0) ? 2 : 1;
   CUtensorMap mU, mWq, mWk, mWv, mQKV, mO, mWo, mV, mW1;
   CUtensorMap mHt, mDzB, mDzA, mW2k, mVnt, mHpB, mHpA, mW1k, mOt, mDyB, mDyA, mWok, mUt;
-  CUtensorMap mDqB[3], mDqA[3], mWk3[3];
+  CUtensorMap mDqB[3], mDqA[3], mWk3[3], mDO;
   bool ok = map_a(&mU, u16, M, d) && map_b(&mWq, wq, d, d, qkv_chunks) &&
             map_b(&mWk, wk, d, d, qkv_chunks) && map_b(&mWv, wv, d, d, qkv_chunks) &&
             map_qkv(&mQKV, qkv, P.B, P.N, d, P.dk) && map_a(&mO, so, R, d) &&
@@ -739,7 +741,8 @@ bpt_status backward_bf16(const Plan& P, const BwdLayout& L, const void* x, const
             map_b(&mVnt, sv, R, d, 2) && map_b(&mHpB, hpre, R, d_ff, 2) &&
             map_a(&mHpA, hpre, R, d_ff) && map_a(&mW1k, w1, d, d_ff) &&
             map_b(&mOt, so, R, d, 2) && map_b(&mDyB, dy16, R, d, 2) &&
-            map_a(&mDyA, dy16, R, d) && map_a(&mWok, wo, d, d) && map_b(&mUt, u16, M, d, 2);
+            map_a(&mDyA, dy16, R, d) && map_a(&mWok, wo, d, d) && map_b(&mUt, u16, M, d, 2) &&
+            map_a(&mDO, do16, R, d, 0, int(P.dk / 64));
   const hf* wqkv[3] = {wq, wk, wv};
   for (int i = 0; i < 3 && ok; ++i)
     ok = map_b(&mDqB[i], dqkv16 + i * d, M, d, 2, 3 * d) &&
@@ -848,25 +851,26 @@ bpt_status backward_bf16(const Plan& P, const BwdLayout& L, const void* x, const
     bpt::attn_row_dot_kernel<<<unsigned((rows * 32 + 255) / 256), 256, 0, s>>>(do16, so, Drow,
                                                                                rows, int(d),
                                                                                int(h));
-    bpt::AttnBwdParams ab{};
-    ab.qkv = qkv; ab.o = so; ab.dO = do16; ab.D = Drow;
-    ab.stats = reinterpret_cast<const float2*>(stats);
-    ab.dq = dq; ab.dk = dk; ab.dv = dv;
+    bpt::AttnBwdTcParams ab{};
     ab.N = int(P.N); ab.nb = int(P.nb); ab.h = int(h); ab.d = int(d); ab.causal = P.causal;
     ab.item0 = int(wv_.item0); ab.count = int(wv_.count); ab.seqs = int(wv_.seqs);
-    ab.scale = scale;
+    ab.stats = reinterpret_cast<const float2*>(stats); ab.D = Drow;
+    ab.dq = dq; ab.dk = dk; ab.dv = dv; ab.scale = scale; ab.err = err;
     int64_t key_end = P.N;
     if (wv_.seqs == 0 && P.causal)
       key_end = std::min<int64_t>(P.N, (wv_.item0 % P.nb + wv_.count) * P.blk);
-    const dim3 gq(unsigned(2 * wv_.count), unsigned(h));
-    const dim3 gkv(unsigned((key_end + bpt::kBwdRows - 1) / bpt::kBwdRows), unsigned(h),
+    const dim3 gq(unsigned(wv_.count), unsigned(h));
+    const dim3 gkv(unsigned((key_end + 127) / 128), unsigned(h),
                    unsigned(wv_.seqs > 0 ? wv_.seqs : 1));
     if (P.dk == 128) {
-      bpt::attn_bwd_dq_kernel<128><<<gq, 256, bpt::AttnBwdSmem<128>::DQ_BYTES, s>>>(ab);
-      bpt::attn_bwd_dkv_kernel<128><<<gkv, 256, bpt::AttnBwdSmem<128>::DKV_BYTES, s>>>(ab);
+      bpt::attn_bwd_dq_tc_kernel<128>
+          <<<gq, 256, bpt::AttnBwdCfg<128>::Q_SMEM, s>>>(mQKV, mDO, ab);
+      bpt::attn_bwd_dkv_tc_kernel<128>
+          <<<gkv, 256, bpt::AttnBwdCfg<128>::KV_SMEM, s>>>(mQKV, mDO, ab);
     } else {
-      bpt::attn_bwd_dq_kernel<64><<<gq, 256, bpt::AttnBwdSmem<64>::DQ_BYTES, s>>>(ab);
-      bpt::attn_bwd_dkv_kernel<64><<<gkv, 256, bpt::AttnBwdSmem<64>::DKV_BYTES, s>>>(ab);
+      bpt::attn_bwd_dq_tc_kernel<64><<<gq, 256, bpt::AttnBwdCfg<64>::Q_SMEM, s>>>(mQKV, mDO, ab);
+      bpt::attn_bwd_dkv_tc_kernel<64>
+          <<<gkv, 256, bpt::AttnBwdCfg<64>::KV_SMEM, s>>>(mQKV, mDO, ab);
     }
     if (cudaGetLastError() != cudaSuccess) return BPT_ERR_CUDA;
   }

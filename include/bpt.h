@@ -188,8 +188,9 @@ bpt_status bpt_layer_backward_workspace_size(int64_t B, int64_t N, int64_t d, in
  * as in the forward) and fp32 accumulation; weight gradients accumulate in
  * fp32 across waves; LayerNorm, GELU' and the bias / gamma / beta sums are
  * fp32 (the sums in a fixed order: results are deterministic).  The
- * attention gradients recompute P = exp(s - m) / l and run on the CUDA cores
- * in fp32 from fp16 Q, K, V, o and dO.
+ * attention gradients recompute P = exp(s - m) / l on the tensor cores (fp16
+ * Q, K, V, dO, P and dS, fp32 accumulation), dK and dV by key block and dQ
+ * by query block, without atomics.
  * Returns BPT_ERR_UNSUPPORTED for BPT_F32; BPT_ERR_INVALID_ARG for a null,
  * misaligned or overlapping pointer; BPT_ERR_WORKSPACE if the workspace is
  * too small; otherwise as bpt_layer_forward (device errors via
