@@ -170,6 +170,53 @@ def cpu_oracle_rate(cfg, n_rows: int):
                       f"{cfg.N} keys) through oracle.layer_rows, fp64"}
 
 
+# ------------------------------------------------------ training step --
+def measure_backward(bpt, cfg, x, p, stream, dev, args, flops, world, peaks, dist):
+    """Times bpt_layer_backward (gradients of every parameter and of x from
+    the saved (m, l)) and the whole training step (bpt_layer_forward_train +
+    bpt_layer_backward), CUDA events on the launching stream, max over ranks.
+    Gradient FLOPs are counted as twice the forward's algorithmic FLOPs (the
+    usual convention: one product for the data gradient and one for the
+    weight gradient of every forward product); the block recomputation adds
+    about one forward on top, as the pages state."""
+    import torch
+    from blockwise_attn_ffn_b200 import dist as bdist
+    out, stats, ws = bpt.layer_forward_train(x, p, cfg.h, cfg.causal)
+    gen = torch.Generator(device=dev).manual_seed(cfg.seed + 77)
+    dZ = torch.randn(x.shape, generator=gen, device=dev, dtype=torch.float32)
+    grads, bws = bpt.layer_backward(x, p, cfg.h, cfg.causal, stats, dZ)
+    for _ in range(2):
+        bpt.layer_backward(x, p, cfg.h, cfg.causal, stats, dZ, workspace=bws)
+    torch.cuda.synchronize(dev)
+    k = args.backward_steps
+    e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(k):
+        bpt.layer_backward(x, p, cfg.h, cfg.causal, stats, dZ, workspace=bws)
+    e1.record(stream)
+    for _ in range(k):
+        bpt.layer_forward_train(x, p, cfg.h, cfg.causal, out=out, stats=stats, workspace=ws)
+        bpt.layer_backward(x, p, cfg.h, cfg.causal, stats, dZ, workspace=bws)
+    e2.record(stream)
+    torch.cuda.synchronize(dev)
+    st, site = bpt.bpt_read_device_error(bws.data_ptr(), stream.cuda_stream)
+    if st != bpt.BPT_OK:
+        raise SystemExit(f"device error in backward {bpt.status_string(st)} site {site}")
+    bwd_ms = bdist.max_over_ranks(e0.elapsed_time(e1), dist, dev) / k
+    step_ms = bdist.max_over_ranks(e1.elapsed_time(e2), dist, dev) / k
+    grad_tf = 2 * flops["total"] * world / (bwd_ms / 1e3) / 1e12
+    tokens = cfg.B * cfg.N * world
+    return {"ms_per_step": bwd_ms, "tokens_per_s": tokens / (bwd_ms / 1e3),
+            "grad_tflops": grad_tf, "pct_bf16_peak": grad_tf / world / peaks["bf16_tflops"],
+            "train_step_ms": step_ms, "train_step_tokens_per_s": tokens / (step_ms / 1e3),
+            "train_step_tflops": 3 * flops["total"] * world / (step_ms / 1e3) / 1e12,
+            "steps": k, "workspace_bytes": int(bws.numel()),
+            "note": "grad FLOPs = 2 x forward algorithmic FLOPs; train step = forward_train + "
+                    "backward (3 x forward FLOPs counted; recomputation not counted)"}
+
+
 # ------------------------------------------------- unfused peak bytes --
 def unfused_torch_peak_bytes(cfg, p, dev):
     """Peak device bytes of the plain unfused schedule, measured once outside
@@ -241,6 +288,9 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=1024)
     ap.add_argument("--ref-rows", type=int, default=16)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the training-step (forward_train + backward) measurement")
+    ap.add_argument("--backward-steps", type=int, default=10)
     ap.add_argument("--no-unfused-peak", action="store_true",
                     help="skip the bench-only unfused-schedule peak-bytes measurement")
     ap.add_argument("--seq-len", type=int, default=None,
@@ -414,6 +464,9 @@ def main():
     }
     with_clk = clk.summary()
     line["clocks"] = with_clk
+    if not args.no_backward and cfg.dtype == "bf16":
+        line["backward"] = measure_backward(bpt, cfg, x, p, stream, dev, args, flops, world,
+                                            peaks, dist)
     if not args.no_unfused_peak and cfg.dtype == "bf16":
         line["peak_bytes"]["unfused_torch_measured"] = unfused_torch_peak_bytes(cfg, p, dev)
 
