@@ -23,11 +23,15 @@
 // A 128-row tile of Q, K, V or dO in shared memory ([d_k/64 chunks][128
 // rows][64], 128-byte swizzle) is a K-major operand in one product and an
 // MN-major one in another (same bytes, different descriptor).
-// Warp roles (256 threads): 0 TMA, 1 UMMA issue, 2 TMEM owner, 3 idle, 4..7
-// elementwise (thread = a row of the 128 the tile's TMEM lanes hold).  Every
-// wait is bounded; on expiry the kernel records a site code, drains and
-// frees its tensor memory.
+// Warp roles: 0 TMA, 1 UMMA issue, 2 TMEM owner, 3 idle, 4.. elementwise:
+// warp w takes TMEM lanes 32(w%4).. (a row of the 128 per thread) and, of
+// the four 32-column chunks, those of its group g = (w-4)/4 (no value
+// crosses a row's warps, the statistics being given).  Every wait is
+// bounded; on expiry the kernel records a site code, drains and frees its
+// tensor memory.
 #pragma once
+
+#include <type_traits>
 
 #include "common.cuh"
 
@@ -35,8 +39,8 @@ namespace bpt {
 
 struct AttnBwdTcParams {
   int N, nb, h, d, causal, item0, count, seqs;
-  const float2* stats;  // [B][h][N] (m, l) from the forward
-  const float* D;       // [count * 128, h] rowsum(dO * O), this wave's block rows
+  const float2* qs;     // [h][count * 128] per query row (-(m + ln l) log2 e, D),
+                        // this wave's block rows (attn_row_terms_kernel)
   float* dq;            // [B*N, d] written (this wave's query rows)
   float* dk;            // [B*N, d] accumulated (+=)
   float* dv;            // [B*N, d] accumulated (+=)
@@ -49,7 +53,7 @@ struct AttnBwdCfg {
   static constexpr int TILE = 128 * D * 2;  // one 128-row fp16 tile
   static constexpr int CHUNK = 128 * 128;   // one 64-column swizzled chunk
   static constexpr int NSLOT = 2;
-  static constexpr int STATS = 3 * 128 * 4;  // per query row: -m log2 e, 1/l, D
+  static constexpr int STATS = 128 * 8;  // per query row: float2 (-(m + ln l) log2 e, D)
   // dK/dV kernel: K, V resident, ring of (Q, dO, stats)
   static constexpr int KV_SLOT = (2 * TILE + STATS + 1023) / 1024 * 1024;
   static constexpr int KV_OFF_RING = 2 * TILE;
@@ -66,6 +70,14 @@ struct AttnBwdCfg {
 };
 
 constexpr float kLog2e = 1.4426950408889634f;
+#ifndef BPT_BWD_EW_GROUPS
+#define BPT_BWD_EW_GROUPS 1
+#endif
+// Elementwise warps per TMEM lane quarter; each takes 4 / G of the four
+// 32-column chunks of a 128 x 128 score tile.
+constexpr int kBwdEwGroups = BPT_BWD_EW_GROUPS;
+static_assert(kBwdEwGroups == 1 || kBwdEwGroups == 2, "1 or 2 elementwise warps per quarter");
+constexpr int kBwdThreads = 128 + 128 * kBwdEwGroups;
 
 // Issue a 128 x 128 x d_k SS product: D[tmem] = A[a_lo] B[b_lo]^T, both
 // K-major tiles (the k-step walks 32 B inside a 64-column chunk, then the
@@ -81,16 +93,25 @@ __device__ __forceinline__ void bwd_issue_ss(uint32_t d_tmem, uint32_t a_lo, uin
   }
 }
 
-// Issue a 128 x d_k x 128 TS product: D[tmem] (+)= A[tmem, fp16 pairs] B,
-// with B an MN-major 128-row tile (k-step = 16 rows = 2 KB).
+// TMEM column (of the 128 that held the fp32 scores) where the fp16 pairs of
+// 32-column chunk cc go: the front of the chunk's own 64-column half, so a
+// warp overwrites only scores it has itself already loaded (with two warps
+// per lane quarter, one owns chunks {0, 1} and the other {2, 3}).
+__device__ __forceinline__ constexpr int packed_col(int cc) { return (cc >> 1) * 64 + (cc & 1) * 16; }
+
+// The two 16-deep k-steps of a TS product that cover 32 rows of B (one chunk
+// of the A columns the elementwise warps hand over at a time).
 template <int D>
-__device__ __forceinline__ void bwd_issue_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
-                                             uint32_t idesc, bool first) {
+__device__ __forceinline__ void bwd_issue_ts_chunk(uint32_t d_tmem, uint32_t a_tmem,
+                                                   uint32_t b_lo, uint32_t idesc, int cc,
+                                                   bool first) {
   constexpr uint32_t hi = sdesc_hi(1024);
 #pragma unroll
-  for (int k = 0; k < 128 / 16; ++k)
-    umma_ts(d_tmem, a_tmem + 8 * k, b_lo + ((k * 2048) >> 4), hi, idesc,
+  for (int kk = 0; kk < 2; ++kk) {
+    const int k = 2 * cc + kk;
+    umma_ts(d_tmem, a_tmem + packed_col(cc) + 8 * kk, b_lo + ((k * 2048) >> 4), hi, idesc,
             (!first || k > 0) ? 1u : 0u);
+  }
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
@@ -105,7 +126,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
 
 // ----------------------------------------------------------------- dK, dV --
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap mapQKV,
                            const __grid_constant__ CUtensorMap mapDO, const AttnBwdTcParams p) {
   using C = AttnBwdCfg<D>;
@@ -132,9 +153,9 @@ __global__ void __launch_bounds__(256, 1)
   const uint32_t ring_full0 = smem_u32(bars + 1);
   const uint32_t ring_empty0 = smem_u32(bars + 1 + C::NSLOT);
   const uint32_t s_full = smem_u32(bars + 1 + 2 * C::NSLOT);
-  const uint32_t p_full = smem_u32(bars + 2 + 2 * C::NSLOT);
-  const uint32_t acc_done = smem_u32(bars + 3 + 2 * C::NSLOT);
-  const uint32_t drain = smem_u32(bars + 4 + 2 * C::NSLOT);
+  const uint32_t p_chunk0 = smem_u32(bars + 2 + 2 * C::NSLOT);  // [4]: P / dS columns 32c..
+  const uint32_t acc_done = smem_u32(bars + 6 + 2 * C::NSLOT);
+  const uint32_t drain = smem_u32(bars + 7 + 2 * C::NSLOT);
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -145,7 +166,7 @@ __global__ void __launch_bounds__(256, 1)
       mbar_init(ring_empty0 + 8 * s, 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 4);
+    for (int c = 0; c < 4; ++c) mbar_init(p_chunk0 + 8 * c, 4);
     mbar_init(acc_done, 1);
     mbar_init(drain, 1);
     abort_sh = 0;
@@ -162,6 +183,7 @@ __global__ void __launch_bounds__(256, 1)
   volatile int* abort_flag = &abort_sh;
   const int chQ = head * D / 64, chK = (p.d + head * D) / 64, chV = (2 * p.d + head * D) / 64;
   const long long lbase = static_cast<long long>(bidx * p.nb - p.item0) * 128;  // wave row of pos 0
+  const long long qs_head = static_cast<long long>(head) * p.count * 128;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -184,24 +206,11 @@ __global__ void __launch_bounds__(256, 1)
       }
       const int ib = ib0 + t;
       uint8_t* sl = smem + C::KV_OFF_RING + slot * C::KV_SLOT;
-      float* st = reinterpret_cast<float*>(sl + 2 * C::TILE);
-      for (int q = lane; q < 128; q += 32) {
-        const int qp = ib * 128 + q;
-        float a = -INFINITY, il = 0.f, dd = 0.f;
-        if (qp < p.N) {
-          const float2 ml = p.stats[(static_cast<long long>(bidx) * p.h + head) * p.N + qp];
-          a = -ml.x * kLog2e;
-          il = 1.0f / ml.y;
-          dd = p.D[(lbase + qp) * p.h + head];
-        }
-        st[q] = a;
-        st[128 + q] = il;
-        st[256 + q] = dd;
-      }
-      __syncwarp();
       if (leader) {
         armed[slot] = static_cast<int>(phase);
-        mbar_arrive_expect_tx(ring_full0 + 8 * slot, 2 * C::TILE);
+        mbar_arrive_expect_tx(ring_full0 + 8 * slot, 2 * C::TILE + C::STATS);
+        bulk_load(smem_u32(sl + 2 * C::TILE), p.qs + qs_head + lbase + ib * 128, C::STATS,
+                  ring_full0 + 8 * slot);
         tma_load_4d(smem_u32(sl), &mapQKV, ring_full0 + 8 * slot, 0, ib * 128, chQ, bidx);
         tma_load_3d(smem_u32(sl + C::TILE), &mapDO, ring_full0 + 8 * slot, 0,
                     static_cast<int>(lbase + ib * 128), head * D / 64);
@@ -235,17 +244,24 @@ __global__ void __launch_bounds__(256, 1)
       }
       __syncwarp();
       commit(s_full);
-      if (!mbar_wait_warp(p_full, static_cast<uint32_t>(t & 1), abort_flag, p.err,
-                          kSiteAttnMma))
-        break;
-      tc_fence_after();
-      if (leader) {
-        bwd_issue_ts<D>(tmem + C::TM_A0, tmem + C::TM_S, sdesc_lo(sl + C::TILE, C::CHUNK),
-                        idesc_o, t == 0);                                               // dV
-        bwd_issue_ts<D>(tmem + C::TM_A1, tmem + C::TM_DP, sdesc_lo(sl, C::CHUNK), idesc_o,
-                        t == 0);                                                        // dK
+      // dV += P^T dO and dK += dS^T Q, 32 query columns at a time as the
+      // elementwise warps hand them over.
+      for (int cc = 0; cc < 4 && ok; ++cc) {
+        if (!mbar_wait_warp(p_chunk0 + 8 * cc, static_cast<uint32_t>(t & 1), abort_flag, p.err,
+                            kSiteAttnMma)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (leader) {
+          bwd_issue_ts_chunk<D>(tmem + C::TM_A0, tmem + C::TM_S,
+                                sdesc_lo(sl + C::TILE, C::CHUNK), idesc_o, cc, t == 0);  // dV
+          bwd_issue_ts_chunk<D>(tmem + C::TM_A1, tmem + C::TM_DP, sdesc_lo(sl, C::CHUNK),
+                                idesc_o, cc, t == 0);                                    // dK
+        }
+        __syncwarp();
       }
-      __syncwarp();
+      if (!ok) break;
       commit(ring_empty0 + 8 * slot);
     }
     commit(acc_done);
@@ -254,9 +270,11 @@ __global__ void __launch_bounds__(256, 1)
   } else if (warp >= 4) {
     // --------------------------------------------------------- elementwise
     const int e = warp & 3;
-    const int kr = e * 32 + lane;  // key row of the block
+    const int grp = (warp - 4) >> 2;  // chunks [grp, grp + 1) * 4 / G
+    const int kr = e * 32 + lane;      // key row of the block
     const int kp = jb * 128 + kr;
     const bool key_ok = kp < p.N;
+    const bool key_blk_full = jb * 128 + 128 <= p.N;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(e * 32) << 16);
     const float c = p.scale * kLog2e;
     bool ok = true;
@@ -268,47 +286,57 @@ __global__ void __launch_bounds__(256, 1)
       }
       tc_fence_after();
       const int slot = t % C::NSLOT;
-      // The producer warp wrote this slot's statistics with ordinary stores
-      // before arriving on its full barrier: acquire that barrier here too
-      // (its phase for block t has completed; the slot is released only
-      // after this warp's p_full arrival below).
+      // The slot's row terms arrive by bulk copy on its full barrier: acquire
+      // that barrier here too (its phase for block t has completed; the slot
+      // is released only after this warp's last p_chunk arrival below).
       if (!mbar_wait_warp(ring_full0 + 8 * slot, static_cast<uint32_t>((t / C::NSLOT) & 1),
                           abort_flag, p.err, kSiteAttnSoftmax)) {
         ok = false;
         break;
       }
-      const float* st =
-          reinterpret_cast<const float*>(smem + C::KV_OFF_RING + slot * C::KV_SLOT + 2 * C::TILE);
+      const float2* st = reinterpret_cast<const float2*>(smem + C::KV_OFF_RING +
+                                                         slot * C::KV_SLOT + 2 * C::TILE);
       const int ib = ib0 + t;
-      const bool diag = p.causal && ib == jb;
+      // masking only on the diagonal block and a ragged last key block
+      const bool masked = (p.causal && ib == jb) || !key_blk_full;
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = grp * (4 / kBwdEwGroups); cc < (grp + 1) * (4 / kBwdEwGroups); ++cc) {
         uint32_t sr[32], dr[32];
         tmem_ld_32x32b_x32(t_lane + C::TM_S + cc * 32, sr);
         tmem_ld_32x32b_x32(t_lane + C::TM_DP + cc * 32, dr);
         tmem_ld_wait();
         uint32_t pk[16], dk16[16];
+        // P = 2^(S c - (m + ln l) log2 e), dS = P (dP - D), per query column
+        auto tile = [&](auto mask) {
 #pragma unroll
-        for (int k = 0; k < 32; k += 2) {
-          float pv[2], dv2[2];
+          for (int k = 0; k < 32; k += 2) {
+            float pv[2], dv2[2];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int q = cc * 32 + k + u;
-            float pr = ex2_approx(fmaf(__uint_as_float(sr[k + u]), c, st[q])) * st[128 + q];
-            if (!key_ok || (diag && kr > q)) pr = 0.f;
-            pv[u] = pr;
-            dv2[u] = pr * (__uint_as_float(dr[k + u]) - st[256 + q]);
+            for (int u = 0; u < 2; ++u) {
+              const int q = cc * 32 + k + u;
+              const float2 sq = st[q];  // one broadcast load
+              float pr = ex2_approx(fmaf(__uint_as_float(sr[k + u]), c, sq.x));
+              if constexpr (decltype(mask)::value) {
+                if (!key_ok || (p.causal && ib == jb && kr > q)) pr = 0.f;
+              }
+              pv[u] = pr;
+              dv2[u] = pr * (__uint_as_float(dr[k + u]) - sq.y);
+            }
+            pk[k >> 1] = pack_f16x2(pv[0], pv[1]);
+            dk16[k >> 1] = pack_f16x2(dv2[0], dv2[1]);
           }
-          pk[k >> 1] = pack_f16x2(pv[0], pv[1]);
-          dk16[k >> 1] = pack_f16x2(dv2[0], dv2[1]);
-        }
-        tmem_st16(t_lane + C::TM_S + cc * 16, pk);
-        tmem_st16(t_lane + C::TM_DP + cc * 16, dk16);
+        };
+        if (masked)
+          tile(std::true_type{});
+        else
+          tile(std::false_type{});
+        tmem_st16(t_lane + C::TM_S + packed_col(cc), pk);
+        tmem_st16(t_lane + C::TM_DP + packed_col(cc), dk16);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_chunk0 + 8 * cc);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
     }
     if (ok && mbar_wait_warp(acc_done, 0, abort_flag, p.err, kSiteAttnSoftmax)) {
       tc_fence_after();
@@ -316,7 +344,8 @@ __global__ void __launch_bounds__(256, 1)
       float* dvr = p.dv + g * p.d + head * D;
       float* dkr = p.dk + g * p.d + head * D;
 #pragma unroll 1
-      for (int cc = 0; cc < D / 32; ++cc) {
+      for (int cc = grp * (D / 32 / kBwdEwGroups); cc < (grp + 1) * (D / 32 / kBwdEwGroups);
+           ++cc) {
         uint32_t a[32], b[32];  // warp-collective loads: every lane takes them
         tmem_ld_32x32b_x32(t_lane + C::TM_A0 + cc * 32, a);
         tmem_ld_32x32b_x32(t_lane + C::TM_A1 + cc * 32, b);
@@ -339,7 +368,7 @@ __global__ void __launch_bounds__(256, 1)
 
 // ---------------------------------------------------------------------- dQ --
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap mapQKV,
                           const __grid_constant__ CUtensorMap mapDO, const AttnBwdTcParams p) {
   using C = AttnBwdCfg<D>;
@@ -357,9 +386,9 @@ __global__ void __launch_bounds__(256, 1)
   const uint32_t ring_full0 = smem_u32(bars + 1);
   const uint32_t ring_empty0 = smem_u32(bars + 1 + C::NSLOT);
   const uint32_t s_full = smem_u32(bars + 1 + 2 * C::NSLOT);
-  const uint32_t p_full = smem_u32(bars + 2 + 2 * C::NSLOT);
-  const uint32_t acc_done = smem_u32(bars + 3 + 2 * C::NSLOT);
-  const uint32_t drain = smem_u32(bars + 4 + 2 * C::NSLOT);
+  const uint32_t p_chunk0 = smem_u32(bars + 2 + 2 * C::NSLOT);  // [4]: P / dS columns 32c..
+  const uint32_t acc_done = smem_u32(bars + 6 + 2 * C::NSLOT);
+  const uint32_t drain = smem_u32(bars + 7 + 2 * C::NSLOT);
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -370,7 +399,7 @@ __global__ void __launch_bounds__(256, 1)
       mbar_init(ring_empty0 + 8 * s, 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 4);
+    for (int c = 0; c < 4; ++c) mbar_init(p_chunk0 + 8 * c, 4);
     mbar_init(acc_done, 1);
     mbar_init(drain, 1);
     abort_sh = 0;
@@ -443,14 +472,20 @@ __global__ void __launch_bounds__(256, 1)
       }
       __syncwarp();
       commit(s_full);
-      if (!mbar_wait_warp(p_full, static_cast<uint32_t>(j & 1), abort_flag, p.err,
-                          kSiteAttnMma))
-        break;
-      tc_fence_after();
-      if (leader)
-        bwd_issue_ts<D>(tmem + C::TM_A0, tmem + C::TM_S, sdesc_lo(sl, C::CHUNK), idesc_o,
-                        j == 0);                                                        // dQ
-      __syncwarp();
+      // dQ += dS K, 32 key columns at a time as the elementwise warps hand them over
+      for (int cc = 0; cc < 4 && ok; ++cc) {
+        if (!mbar_wait_warp(p_chunk0 + 8 * cc, static_cast<uint32_t>(j & 1), abort_flag, p.err,
+                            kSiteAttnMma)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (leader)
+          bwd_issue_ts_chunk<D>(tmem + C::TM_A0, tmem + C::TM_S, sdesc_lo(sl, C::CHUNK),
+                                idesc_o, cc, j == 0);                                    // dQ
+        __syncwarp();
+      }
+      if (!ok) break;
       commit(ring_empty0 + 8 * slot);
     }
     commit(acc_done);
@@ -459,18 +494,14 @@ __global__ void __launch_bounds__(256, 1)
   } else if (warp >= 4) {
     // --------------------------------------------------------- elementwise
     const int e = warp & 3;
-    const int qr = e * 32 + lane;  // query row of the block
+    const int grp = (warp - 4) >> 2;  // chunks [grp, grp + 1) * 4 / G
+    const int qr = e * 32 + lane;      // query row of the block
     const int qp = ib * 128 + qr;
     const bool q_ok = qp < p.N;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(e * 32) << 16);
     const float c = p.scale * kLog2e;
-    float a = -INFINITY, il = 0.f, dd = 0.f;
-    if (q_ok) {
-      const float2 ml = p.stats[(static_cast<long long>(bidx) * p.h + head) * p.N + qp];
-      a = -ml.x * kLog2e;
-      il = 1.0f / ml.y;
-      dd = p.D[(lrow + qr) * p.h + head];
-    }
+    const float2 rt = p.qs[static_cast<long long>(head) * p.count * 128 + lrow + qr];
+    const float a = rt.x, dd = rt.y;  // -inf, 0 past the sequence
     bool ok = true;
     for (int j = 0; j < n_kv && ok; ++j) {
       if (!mbar_wait_warp(s_full, static_cast<uint32_t>(j & 1), abort_flag, p.err,
@@ -481,37 +512,48 @@ __global__ void __launch_bounds__(256, 1)
       tc_fence_after();
       const bool diag = p.causal && j == ib;
       const int klim = p.N - j * 128;  // keys >= klim are past the sequence
+      const bool masked = diag || klim < 128;
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = grp * (4 / kBwdEwGroups); cc < (grp + 1) * (4 / kBwdEwGroups); ++cc) {
         uint32_t sr[32], dr[32];
         tmem_ld_32x32b_x32(t_lane + C::TM_S + cc * 32, sr);
         tmem_ld_32x32b_x32(t_lane + C::TM_DP + cc * 32, dr);
         tmem_ld_wait();
         uint32_t ds16[16];
+        // dS = P (dP - D), P = 2^(S c - (m + ln l) log2 e)
+        auto tile = [&](auto mask) {
 #pragma unroll
-        for (int k = 0; k < 32; k += 2) {
-          float dsv[2];
+          for (int k = 0; k < 32; k += 2) {
+            float dsv[2];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int kc = cc * 32 + k + u;
-            float pr = ex2_approx(fmaf(__uint_as_float(sr[k + u]), c, a)) * il;
-            if (kc >= klim || (diag && kc > qr)) pr = 0.f;
-            dsv[u] = pr * (__uint_as_float(dr[k + u]) - dd);
+            for (int u = 0; u < 2; ++u) {
+              const int kc = cc * 32 + k + u;
+              float pr = ex2_approx(fmaf(__uint_as_float(sr[k + u]), c, a));
+              if constexpr (decltype(mask)::value) {
+                if (kc >= klim || (diag && kc > qr)) pr = 0.f;
+              }
+              dsv[u] = pr * (__uint_as_float(dr[k + u]) - dd);
+            }
+            ds16[k >> 1] = pack_f16x2(dsv[0], dsv[1]);
           }
-          ds16[k >> 1] = pack_f16x2(dsv[0], dsv[1]);
-        }
-        tmem_st16(t_lane + C::TM_S + cc * 16, ds16);
+        };
+        if (masked)
+          tile(std::true_type{});
+        else
+          tile(std::false_type{});
+        tmem_st16(t_lane + C::TM_S + packed_col(cc), ds16);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_chunk0 + 8 * cc);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
     }
     if (ok && mbar_wait_warp(acc_done, 0, abort_flag, p.err, kSiteAttnSoftmax)) {
       tc_fence_after();
       float* dst = p.dq + (static_cast<long long>(bidx) * p.N + qp) * p.d + head * D;
 #pragma unroll 1
-      for (int cc = 0; cc < D / 32; ++cc) {
+      for (int cc = grp * (D / 32 / kBwdEwGroups); cc < (grp + 1) * (D / 32 / kBwdEwGroups);
+           ++cc) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(t_lane + C::TM_A0 + cc * 32, v);
         tmem_ld_wait();

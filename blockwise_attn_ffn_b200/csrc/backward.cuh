@@ -8,9 +8,9 @@
 //   * row copies fp32 -> fp16 (GEMM operands),
 //   * LayerNorm backward (one warp per row) and the deterministic column
 //     sums of the bias, gamma and beta gradients,
-//   * the attention backward's row terms D = rowsum(dO * O) per head (the
-//     attention gradients themselves run on the tensor cores,
-//     attn_bwd_tc.cuh).
+//   * the attention backward's per-row terms (D = rowsum(dO * O) per head,
+//     with the row's softmax statistics; the attention gradients themselves
+//     run on the tensor cores, attn_bwd_tc.cuh).
 // LayerNorm y = g * xh + b (standard calculus):
 //   dx = rstd * (dxh - mean(dxh) - xh * mean(dxh * xh)),
 //   dxh = dy * g,  dg = sum_rows dy * xh,  db = sum_rows dy.
@@ -161,19 +161,37 @@ __global__ void colsum_reduce_kernel(const float* __restrict__ part, int chunks,
   out[c] += s;
 }
 
-// D[r, t] = sum over head t's columns of dO[r, c] * O[r, c]; one warp per row.
-__global__ void attn_row_dot_kernel(const __half* __restrict__ dO, const __half* __restrict__ O,
-                                    float* __restrict__ D, long long rows, int d, int h) {
+// Per (head t, local row r) the two numbers the attention backward needs for
+// query row r, packed as one 8-byte record (head-major, so a block's 128
+// records are one contiguous 1 KB run a bulk copy can fetch):
+//   qs[t * rows + r] = (-(m + ln l) log2 e, D),  D = sum over head t's
+//   columns of dO[r, c] * O[r, c],
+// with (m, l) the forward's softmax statistics of the row's global position
+// (stats [B][h][N]); P = 2^(S scale log2 e + qs.x) is then the row's
+// probability.  Rows past the sequence get (-inf, 0), which makes their
+// probabilities 0.  One warp per row.
+__global__ void attn_row_terms_kernel(const __half* __restrict__ dO, const __half* __restrict__ O,
+                                      const float2* __restrict__ stats, float2* __restrict__ qs,
+                                      long long rows, int d, int h, RowMap map) {
   const int lane = threadIdx.x & 31;
   const long long r = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) >> 5;
   if (r >= rows) return;
+  const long long g = map.map(r);
   const int dk = d / h;
+  const long long b = g >= 0 ? g / map.N : 0, pos = g >= 0 ? g - b * map.N : 0;
   for (int t = 0; t < h; ++t) {
     float s = 0.f;
     for (int c = lane; c < dk; c += 32)
       s += __half2float(dO[r * d + t * dk + c]) * __half2float(O[r * d + t * dk + c]);
     s = warp_sum(s);
-    if (lane == 0) D[r * h + t] = s;
+    if (lane == 0) {
+      float2 v = make_float2(-INFINITY, 0.f);
+      if (g >= 0) {
+        const float2 ml = stats[(b * h + t) * map.N + pos];
+        v = make_float2(-(ml.x * 1.4426950408889634f + log2f(ml.y)), s);
+      }
+      qs[t * rows + r] = v;
+    }
   }
 }
 

@@ -652,7 +652,7 @@ BwdLayout make_bwd_layout(const Plan& P) {
   L.off_dvn = take(R * d * 4);
   L.off_dy16 = take(R * d * 2);
   L.off_do16 = take(R * d * 2);
-  L.off_D = take(R * h * 4);
+  L.off_D = take(R * h * 8);
   L.off_rowstat = take(std::max(R, M) * 8);
   L.off_y = take(M * d * 4);
   L.off_u16 = take(M * d * 2);
@@ -712,7 +712,7 @@ bpt_status backward_bf16(const Plan& P, const BwdLayout& L, const void* x, const
   float* dvn = reinterpret_cast<float*>(ws + L.off_dvn);
   hf* dy16 = reinterpret_cast<hf*>(ws + L.off_dy16);
   hf* do16 = reinterpret_cast<hf*>(ws + L.off_do16);
-  float* Drow = reinterpret_cast<float*>(ws + L.off_D);
+  float2* qs = reinterpret_cast<float2*>(ws + L.off_D);
   float2* rowstat = reinterpret_cast<float2*>(ws + L.off_rowstat);
   float* y = reinterpret_cast<float*>(ws + L.off_y);
   hf* u16 = reinterpret_cast<hf*>(ws + L.off_u16);
@@ -848,13 +848,12 @@ bpt_status backward_bf16(const Plan& P, const BwdLayout& L, const void* x, const
               [&](bpt::GemmParams& g) { g.out_h = do16; g.ld_out = d; }))
       return BPT_ERR_CUDA;
     // attention backward of this wave's query rows
-    bpt::attn_row_dot_kernel<<<unsigned((rows * 32 + 255) / 256), 256, 0, s>>>(do16, so, Drow,
-                                                                               rows, int(d),
-                                                                               int(h));
+    bpt::attn_row_terms_kernel<<<unsigned((rows * 32 + 255) / 256), 256, 0, s>>>(
+        do16, so, reinterpret_cast<const float2*>(stats), qs, rows, int(d), int(h), map);
     bpt::AttnBwdTcParams ab{};
     ab.N = int(P.N); ab.nb = int(P.nb); ab.h = int(h); ab.d = int(d); ab.causal = P.causal;
     ab.item0 = int(wv_.item0); ab.count = int(wv_.count); ab.seqs = int(wv_.seqs);
-    ab.stats = reinterpret_cast<const float2*>(stats); ab.D = Drow;
+    ab.qs = qs;
     ab.dq = dq; ab.dk = dk; ab.dv = dv; ab.scale = scale; ab.err = err;
     int64_t key_end = P.N;
     if (wv_.seqs == 0 && P.causal)
@@ -864,13 +863,13 @@ bpt_status backward_bf16(const Plan& P, const BwdLayout& L, const void* x, const
                    unsigned(wv_.seqs > 0 ? wv_.seqs : 1));
     if (P.dk == 128) {
       bpt::attn_bwd_dq_tc_kernel<128>
-          <<<gq, 256, bpt::AttnBwdCfg<128>::Q_SMEM, s>>>(mQKV, mDO, ab);
+          <<<gq, bpt::kBwdThreads, bpt::AttnBwdCfg<128>::Q_SMEM, s>>>(mQKV, mDO, ab);
       bpt::attn_bwd_dkv_tc_kernel<128>
-          <<<gkv, 256, bpt::AttnBwdCfg<128>::KV_SMEM, s>>>(mQKV, mDO, ab);
+          <<<gkv, bpt::kBwdThreads, bpt::AttnBwdCfg<128>::KV_SMEM, s>>>(mQKV, mDO, ab);
     } else {
-      bpt::attn_bwd_dq_tc_kernel<64><<<gq, 256, bpt::AttnBwdCfg<64>::Q_SMEM, s>>>(mQKV, mDO, ab);
+      bpt::attn_bwd_dq_tc_kernel<64><<<gq, bpt::kBwdThreads, bpt::AttnBwdCfg<64>::Q_SMEM, s>>>(mQKV, mDO, ab);
       bpt::attn_bwd_dkv_tc_kernel<64>
-          <<<gkv, 256, bpt::AttnBwdCfg<64>::KV_SMEM, s>>>(mQKV, mDO, ab);
+          <<<gkv, bpt::kBwdThreads, bpt::AttnBwdCfg<64>::KV_SMEM, s>>>(mQKV, mDO, ab);
     }
     if (cudaGetLastError() != cudaSuccess) return BPT_ERR_CUDA;
   }
