@@ -9,12 +9,19 @@
 //   attn_bwd_dkv_tc_kernel  one CTA per (128-key block, head, sequence of
 //       the wave): K, V stay in shared memory; the wave's query blocks that
 //       see the key block stream through a two-slot ring (Q, dO and the
-//       rows' (m, l, D)).  Per query block:
+//       rows' terms a' = -(m + ln l) log2 e and -D).  Per query block:
 //         S^T = K Q^T, dP^T = V dO^T     UMMA (SS), fp32 in TMEM
 //         P^T, dS^T                       elementwise warps, fp16 back in TMEM
 //         dV += P^T dO, dK += dS^T Q     UMMA with A from TMEM
-//       At the end dK, dV are added into the fp32 gradients (waves run in
-//       stream order, so each key row is updated by one CTA at a time).
+//       The elementwise pass runs in two phases so the tensor core is never
+//       left waiting for all of it: P^T (from S^T alone) while dP^T is still
+//       being computed, then dS^T once dP^T is done; P^T stays in registers
+//       (fp16 pairs) in between.  The UMMA warp issues
+//         S_0, dP_0, then per block t: dV_t, S_t+1, dK_t, dP_t+1,
+//       each gradient product 32 query columns at a time as they are handed
+//       over, and S_t+1 as soon as S_t has been read.  At the end dK, dV are
+//       added into the fp32 gradients (waves run in stream order, so each
+//       key row is updated by one CTA at a time).
 //   attn_bwd_dq_tc_kernel  one CTA per (128-query block, head): Q, dO stay
 //       in shared memory, K, V stream through the ring.  Per key block:
 //         S = Q K^T, dP = dO V^T          UMMA (SS)
@@ -23,12 +30,10 @@
 // A 128-row tile of Q, K, V or dO in shared memory ([d_k/64 chunks][128
 // rows][64], 128-byte swizzle) is a K-major operand in one product and an
 // MN-major one in another (same bytes, different descriptor).
-// Warp roles: 0 TMA, 1 UMMA issue, 2 TMEM owner, 3 idle, 4.. elementwise:
-// warp w takes TMEM lanes 32(w%4).. (a row of the 128 per thread) and, of
-// the four 32-column chunks, those of its group g = (w-4)/4 (no value
-// crosses a row's warps, the statistics being given).  Every wait is
-// bounded; on expiry the kernel records a site code, drains and frees its
-// tensor memory.
+// Warp roles (256 threads): 0 TMA, 1 UMMA issue, 2 TMEM owner, 3 idle,
+// 4..7 elementwise (warp w takes TMEM lanes 32(w%4)..: a row of the 128 per
+// thread).  Every wait is bounded; on expiry the kernel records a site code,
+// drains and frees its tensor memory.
 #pragma once
 
 #include <type_traits>
@@ -39,8 +44,9 @@ namespace bpt {
 
 struct AttnBwdTcParams {
   int N, nb, h, d, causal, item0, count, seqs;
-  const float2* qs;     // [h][count * 128] per query row (-(m + ln l) log2 e, D),
-                        // this wave's block rows (attn_row_terms_kernel)
+  const float* qs;      // [h][count][2][128]: per query block of the wave, the
+                        // rows' a' = -(m + ln l) log2 e, then their -D
+                        // (attn_row_terms_kernel)
   float* dq;            // [B*N, d] written (this wave's query rows)
   float* dk;            // [B*N, d] accumulated (+=)
   float* dv;            // [B*N, d] accumulated (+=)
@@ -53,7 +59,7 @@ struct AttnBwdCfg {
   static constexpr int TILE = 128 * D * 2;  // one 128-row fp16 tile
   static constexpr int CHUNK = 128 * 128;   // one 64-column swizzled chunk
   static constexpr int NSLOT = 2;
-  static constexpr int STATS = 128 * 8;  // per query row: float2 (-(m + ln l) log2 e, D)
+  static constexpr int STATS = 2 * 128 * 4;  // a' of the 128 rows, then their -D
   // dK/dV kernel: K, V resident, ring of (Q, dO, stats)
   static constexpr int KV_SLOT = (2 * TILE + STATS + 1023) / 1024 * 1024;
   static constexpr int KV_OFF_RING = 2 * TILE;
@@ -70,14 +76,7 @@ struct AttnBwdCfg {
 };
 
 constexpr float kLog2e = 1.4426950408889634f;
-#ifndef BPT_BWD_EW_GROUPS
-#define BPT_BWD_EW_GROUPS 1
-#endif
-// Elementwise warps per TMEM lane quarter; each takes 4 / G of the four
-// 32-column chunks of a 128 x 128 score tile.
-constexpr int kBwdEwGroups = BPT_BWD_EW_GROUPS;
-static_assert(kBwdEwGroups == 1 || kBwdEwGroups == 2, "1 or 2 elementwise warps per quarter");
-constexpr int kBwdThreads = 128 + 128 * kBwdEwGroups;
+constexpr int kBwdThreads = 256;
 
 // Issue a 128 x 128 x d_k SS product: D[tmem] = A[a_lo] B[b_lo]^T, both
 // K-major tiles (the k-step walks 32 B inside a 64-column chunk, then the
@@ -94,9 +93,9 @@ __device__ __forceinline__ void bwd_issue_ss(uint32_t d_tmem, uint32_t a_lo, uin
 }
 
 // TMEM column (of the 128 that held the fp32 scores) where the fp16 pairs of
-// 32-column chunk cc go: the front of the chunk's own 64-column half, so a
-// warp overwrites only scores it has itself already loaded (with two warps
-// per lane quarter, one owns chunks {0, 1} and the other {2, 3}).
+// 32-column chunk cc go: the front of the chunk's own 64-column half.  The
+// chunks are handled in order, so only scores already loaded are
+// overwritten.
 __device__ __forceinline__ constexpr int packed_col(int cc) { return (cc >> 1) * 64 + (cc & 1) * 16; }
 
 // The two 16-deep k-steps of a TS product that cover 32 rows of B (one chunk
@@ -153,9 +152,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t ring_full0 = smem_u32(bars + 1);
   const uint32_t ring_empty0 = smem_u32(bars + 1 + C::NSLOT);
   const uint32_t s_full = smem_u32(bars + 1 + 2 * C::NSLOT);
-  const uint32_t p_chunk0 = smem_u32(bars + 2 + 2 * C::NSLOT);  // [4]: P / dS columns 32c..
-  const uint32_t acc_done = smem_u32(bars + 6 + 2 * C::NSLOT);
-  const uint32_t drain = smem_u32(bars + 7 + 2 * C::NSLOT);
+  const uint32_t dp_full = smem_u32(bars + 2 + 2 * C::NSLOT);
+  const uint32_t p_chunk0 = smem_u32(bars + 3 + 2 * C::NSLOT);   // [4]: P^T columns 32c..
+  const uint32_t ds_chunk0 = smem_u32(bars + 7 + 2 * C::NSLOT);  // [4]: dS^T columns 32c..
+  const uint32_t acc_done = smem_u32(bars + 11 + 2 * C::NSLOT);
+  const uint32_t drain = smem_u32(bars + 12 + 2 * C::NSLOT);
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -166,7 +167,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(ring_empty0 + 8 * s, 1);
     }
     mbar_init(s_full, 1);
-    for (int c = 0; c < 4; ++c) mbar_init(p_chunk0 + 8 * c, 4);
+    mbar_init(dp_full, 1);
+    for (int c = 0; c < 4; ++c) {
+      mbar_init(p_chunk0 + 8 * c, 4);
+      mbar_init(ds_chunk0 + 8 * c, 4);
+    }
     mbar_init(acc_done, 1);
     mbar_init(drain, 1);
     abort_sh = 0;
@@ -183,7 +188,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   volatile int* abort_flag = &abort_sh;
   const int chQ = head * D / 64, chK = (p.d + head * D) / 64, chV = (2 * p.d + head * D) / 64;
   const long long lbase = static_cast<long long>(bidx * p.nb - p.item0) * 128;  // wave row of pos 0
-  const long long qs_head = static_cast<long long>(head) * p.count * 128;
+  // row terms of this head: [count][2][128] floats from here, by wave block
+  const float* qs_head = p.qs + static_cast<long long>(head) * p.count * 256;
+  const int lblk0 = bidx * p.nb - p.item0;  // wave block of this sequence's block 0
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -195,21 +202,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tma_load_4d(smem_u32(smem), &mapQKV, kv_full, 0, jb * 128, chK, bidx);
       tma_load_4d(smem_u32(smem + C::TILE), &mapQKV, kv_full, 0, jb * 128, chV, bidx);
     }
-    bool ok = true;
-    for (int t = 0; t < n_q && ok; ++t) {
+    for (int t = 0; t < n_q; ++t) {
       const int slot = t % C::NSLOT;
       const uint32_t phase = static_cast<uint32_t>((t / C::NSLOT) & 1);
       if (!mbar_wait_warp(ring_empty0 + 8 * slot, phase ^ 1u, abort_flag, p.err,
-                          kSiteAttnProducer)) {
-        ok = false;
+                          kSiteAttnProducer))
         break;
-      }
       const int ib = ib0 + t;
       uint8_t* sl = smem + C::KV_OFF_RING + slot * C::KV_SLOT;
       if (leader) {
         armed[slot] = static_cast<int>(phase);
         mbar_arrive_expect_tx(ring_full0 + 8 * slot, 2 * C::TILE + C::STATS);
-        bulk_load(smem_u32(sl + 2 * C::TILE), p.qs + qs_head + lbase + ib * 128, C::STATS,
+        bulk_load(smem_u32(sl + 2 * C::TILE), qs_head + (lblk0 + ib) * 256LL, C::STATS,
                   ring_full0 + 8 * slot);
         tma_load_4d(smem_u32(sl), &mapQKV, ring_full0 + 8 * slot, 0, ib * 128, chQ, bidx);
         tma_load_3d(smem_u32(sl + C::TILE), &mapDO, ring_full0 + 8 * slot, 0,
@@ -231,38 +235,57 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (leader) umma_commit(bar);
       __syncwarp();
     };
-    bool ok = mbar_wait_warp(kv_full, 0, abort_flag, p.err, kSiteAttnMma);
-    for (int t = 0; t < n_q && ok; ++t) {
-      const int slot = t % C::NSLOT;
-      const uint32_t phase = static_cast<uint32_t>((t / C::NSLOT) & 1);
-      if (!mbar_wait_warp(ring_full0 + 8 * slot, phase, abort_flag, p.err, kSiteAttnMma)) break;
+    auto slot_of = [&](int t) {
+      return smem_u32(smem + C::KV_OFF_RING + (t % C::NSLOT) * C::KV_SLOT);
+    };
+    // S^T_t = K Q_t^T once Q_t has landed
+    auto issue_s = [&](int t) -> bool {
+      if (!mbar_wait_warp(ring_full0 + 8 * (t % C::NSLOT),
+                          static_cast<uint32_t>((t / C::NSLOT) & 1), abort_flag, p.err,
+                          kSiteAttnMma))
+        return false;
       tc_fence_after();
-      const uint32_t sl = smem_u32(smem + C::KV_OFF_RING + slot * C::KV_SLOT);
-      if (leader) {
-        bwd_issue_ss<D>(tmem + C::TM_S, k_lo, sdesc_lo(sl, 16), idesc_s);               // S^T
-        bwd_issue_ss<D>(tmem + C::TM_DP, v_lo, sdesc_lo(sl + C::TILE, 16), idesc_s);    // dP^T
-      }
+      if (leader) bwd_issue_ss<D>(tmem + C::TM_S, k_lo, sdesc_lo(slot_of(t), 16), idesc_s);
       __syncwarp();
       commit(s_full);
-      // dV += P^T dO and dK += dS^T Q, 32 query columns at a time as the
-      // elementwise warps hand them over.
-      for (int cc = 0; cc < 4 && ok; ++cc) {
-        if (!mbar_wait_warp(p_chunk0 + 8 * cc, static_cast<uint32_t>(t & 1), abort_flag, p.err,
-                            kSiteAttnMma)) {
-          ok = false;
-          break;
-        }
+      return true;
+    };
+    // dP^T_t = V dO_t^T (slot already waited by issue_s)
+    auto issue_dp = [&](int t) {
+      if (leader)
+        bwd_issue_ss<D>(tmem + C::TM_DP, v_lo, sdesc_lo(slot_of(t) + C::TILE, 16), idesc_s);
+      __syncwarp();
+      commit(dp_full);
+    };
+    // one gradient product, 32 query columns at a time as the elementwise
+    // warps hand them over on chunk barriers cb[0..3]
+    auto issue_grad = [&](int t, uint32_t cb, uint32_t acc, uint32_t a_tm, uint32_t b_lo) {
+      for (int cc = 0; cc < 4; ++cc) {
+        if (!mbar_wait_warp(cb + 8 * cc, static_cast<uint32_t>(t & 1), abort_flag, p.err,
+                            kSiteAttnMma))
+          return false;
         tc_fence_after();
-        if (leader) {
-          bwd_issue_ts_chunk<D>(tmem + C::TM_A0, tmem + C::TM_S,
-                                sdesc_lo(sl + C::TILE, C::CHUNK), idesc_o, cc, t == 0);  // dV
-          bwd_issue_ts_chunk<D>(tmem + C::TM_A1, tmem + C::TM_DP, sdesc_lo(sl, C::CHUNK),
-                                idesc_o, cc, t == 0);                                    // dK
-        }
+        if (leader) bwd_issue_ts_chunk<D>(acc, a_tm, b_lo, idesc_o, cc, t == 0);
         __syncwarp();
       }
-      if (!ok) break;
-      commit(ring_empty0 + 8 * slot);
+      return true;
+    };
+    bool ok = mbar_wait_warp(kv_full, 0, abort_flag, p.err, kSiteAttnMma) && issue_s(0);
+    if (ok) issue_dp(0);
+    for (int t = 0; t < n_q && ok; ++t) {
+      const uint32_t sl = slot_of(t);
+      // dV += P^T dO_t
+      if (!(ok = issue_grad(t, p_chunk0, tmem + C::TM_A0, tmem + C::TM_S,
+                            sdesc_lo(sl + C::TILE, C::CHUNK))))
+        break;
+      // S^T_t has been read in full: the next block's scores can go there
+      if (t + 1 < n_q && !(ok = issue_s(t + 1))) break;
+      // dK += dS^T Q_t
+      if (!(ok = issue_grad(t, ds_chunk0, tmem + C::TM_A1, tmem + C::TM_DP,
+                            sdesc_lo(sl, C::CHUNK))))
+        break;
+      commit(ring_empty0 + 8 * (t % C::NSLOT));
+      if (t + 1 < n_q) issue_dp(t + 1);
     }
     commit(acc_done);
     commit(drain);
@@ -270,72 +293,89 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp >= 4) {
     // --------------------------------------------------------- elementwise
     const int e = warp & 3;
-    const int grp = (warp - 4) >> 2;  // chunks [grp, grp + 1) * 4 / G
-    const int kr = e * 32 + lane;      // key row of the block
+    const int kr = e * 32 + lane;  // key row of the block
     const int kp = jb * 128 + kr;
     const bool key_ok = kp < p.N;
     const bool key_blk_full = jb * 128 + 128 <= p.N;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(e * 32) << 16);
-    const float c = p.scale * kLog2e;
+    const float2 c2 = make_float2(p.scale * kLog2e, p.scale * kLog2e);
     bool ok = true;
     for (int t = 0; t < n_q && ok; ++t) {
-      if (!mbar_wait_warp(s_full, static_cast<uint32_t>(t & 1), abort_flag, p.err,
+      const int slot = t % C::NSLOT;
+      // The slot's row terms arrive by bulk copy on its full barrier: acquire
+      // it (long complete by now; the slot is released only after this
+      // warp's last dS^T hand-over of block t).
+      if (!mbar_wait_warp(ring_full0 + 8 * slot, static_cast<uint32_t>((t / C::NSLOT) & 1),
+                          abort_flag, p.err, kSiteAttnSoftmax) ||
+          !mbar_wait_warp(s_full, static_cast<uint32_t>(t & 1), abort_flag, p.err,
                           kSiteAttnSoftmax)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int slot = t % C::NSLOT;
-      // The slot's row terms arrive by bulk copy on its full barrier: acquire
-      // that barrier here too (its phase for block t has completed; the slot
-      // is released only after this warp's last p_chunk arrival below).
-      if (!mbar_wait_warp(ring_full0 + 8 * slot, static_cast<uint32_t>((t / C::NSLOT) & 1),
-                          abort_flag, p.err, kSiteAttnSoftmax)) {
-        ok = false;
-        break;
-      }
-      const float2* st = reinterpret_cast<const float2*>(smem + C::KV_OFF_RING +
-                                                         slot * C::KV_SLOT + 2 * C::TILE);
+      const float* st = reinterpret_cast<const float*>(smem + C::KV_OFF_RING + slot * C::KV_SLOT +
+                                                       2 * C::TILE);
       const int ib = ib0 + t;
       // masking only on the diagonal block and a ragged last key block
-      const bool masked = (p.causal && ib == jb) || !key_blk_full;
-#pragma unroll 1
-      for (int cc = grp * (4 / kBwdEwGroups); cc < (grp + 1) * (4 / kBwdEwGroups); ++cc) {
-        uint32_t sr[32], dr[32];
+      const bool diag = p.causal && ib == jb;
+      const bool masked = diag || !key_blk_full;
+      uint32_t pp[64];  // P^T of this key row, fp16 pairs, kept for the dS^T phase
+      // ---- phase 1: P^T = 2^(S^T c + a'), per query column
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t sr[32];
         tmem_ld_32x32b_x32(t_lane + C::TM_S + cc * 32, sr);
-        tmem_ld_32x32b_x32(t_lane + C::TM_DP + cc * 32, dr);
         tmem_ld_wait();
-        uint32_t pk[16], dk16[16];
-        // P = 2^(S c - (m + ln l) log2 e), dS = P (dP - D), per query column
         auto tile = [&](auto mask) {
 #pragma unroll
           for (int k = 0; k < 32; k += 2) {
-            float pv[2], dv2[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int q = cc * 32 + k + u;
-              const float2 sq = st[q];  // one broadcast load
-              float pr = ex2_approx(fmaf(__uint_as_float(sr[k + u]), c, sq.x));
-              if constexpr (decltype(mask)::value) {
-                if (!key_ok || (p.causal && ib == jb && kr > q)) pr = 0.f;
-              }
-              pv[u] = pr;
-              dv2[u] = pr * (__uint_as_float(dr[k + u]) - sq.y);
+            const int q = cc * 32 + k;
+            const float2 a = *reinterpret_cast<const float2*>(st + q);  // broadcast
+            const float2 x = __ffma2_rn(
+                make_float2(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])), c2, a);
+            float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            if constexpr (decltype(mask)::value) {
+              if (!key_ok || (diag && kr > q)) pr.x = 0.f;
+              if (!key_ok || (diag && kr > q + 1)) pr.y = 0.f;
             }
-            pk[k >> 1] = pack_f16x2(pv[0], pv[1]);
-            dk16[k >> 1] = pack_f16x2(dv2[0], dv2[1]);
+            pp[cc * 16 + (k >> 1)] = pack_f16x2(pr.x, pr.y);
           }
         };
         if (masked)
           tile(std::true_type{});
         else
           tile(std::false_type{});
-        tmem_st16(t_lane + C::TM_S + packed_col(cc), pk);
-        tmem_st16(t_lane + C::TM_DP + packed_col(cc), dk16);
+        tmem_st16(t_lane + C::TM_S + packed_col(cc), pp + cc * 16);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(p_chunk0 + 8 * cc);
+      }
+      // ---- phase 2: dS^T = P^T (dP^T - D)
+      if (!mbar_wait_warp(dp_full, static_cast<uint32_t>(t & 1), abort_flag, p.err,
+                          kSiteAttnSoftmax)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t dr[32], ds[16];
+        tmem_ld_32x32b_x32(t_lane + C::TM_DP + cc * 32, dr);
+        tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < 32; k += 2) {
+          const float2 nd = *reinterpret_cast<const float2*>(st + 128 + cc * 32 + k);
+          const float2 pr = __half22float2(*reinterpret_cast<const __half2*>(&pp[cc * 16 + (k >> 1)]));
+          const float2 v = __fmul2_rn(
+              pr, __fadd2_rn(make_float2(__uint_as_float(dr[k]), __uint_as_float(dr[k + 1])), nd));
+          ds[k >> 1] = pack_f16x2(v.x, v.y);
+        }
+        tmem_st16(t_lane + C::TM_DP + packed_col(cc), ds);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ds_chunk0 + 8 * cc);
       }
     }
     if (ok && mbar_wait_warp(acc_done, 0, abort_flag, p.err, kSiteAttnSoftmax)) {
@@ -344,8 +384,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       float* dvr = p.dv + g * p.d + head * D;
       float* dkr = p.dk + g * p.d + head * D;
 #pragma unroll 1
-      for (int cc = grp * (D / 32 / kBwdEwGroups); cc < (grp + 1) * (D / 32 / kBwdEwGroups);
-           ++cc) {
+      for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t a[32], b[32];  // warp-collective loads: every lane takes them
         tmem_ld_32x32b_x32(t_lane + C::TM_A0 + cc * 32, a);
         tmem_ld_32x32b_x32(t_lane + C::TM_A1 + cc * 32, b);
@@ -494,14 +533,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp >= 4) {
     // --------------------------------------------------------- elementwise
     const int e = warp & 3;
-    const int grp = (warp - 4) >> 2;  // chunks [grp, grp + 1) * 4 / G
-    const int qr = e * 32 + lane;      // query row of the block
+    const int qr = e * 32 + lane;  // query row of the block
     const int qp = ib * 128 + qr;
     const bool q_ok = qp < p.N;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(e * 32) << 16);
-    const float c = p.scale * kLog2e;
-    const float2 rt = p.qs[static_cast<long long>(head) * p.count * 128 + lrow + qr];
-    const float a = rt.x, dd = rt.y;  // -inf, 0 past the sequence
+    const float2 c2 = make_float2(p.scale * kLog2e, p.scale * kLog2e);
+    const float* rt = p.qs + (static_cast<long long>(head) * p.count + qb) * 256;
+    const float2 a2 = make_float2(rt[qr], rt[qr]);               // a': -inf past the sequence
+    const float2 nd2 = make_float2(rt[128 + qr], rt[128 + qr]);  // -D
     bool ok = true;
     for (int j = 0; j < n_kv && ok; ++j) {
       if (!mbar_wait_warp(s_full, static_cast<uint32_t>(j & 1), abort_flag, p.err,
@@ -514,27 +553,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int klim = p.N - j * 128;  // keys >= klim are past the sequence
       const bool masked = diag || klim < 128;
 #pragma unroll 1
-      for (int cc = grp * (4 / kBwdEwGroups); cc < (grp + 1) * (4 / kBwdEwGroups); ++cc) {
+      for (int cc = 0; cc < 4; ++cc) {
         uint32_t sr[32], dr[32];
         tmem_ld_32x32b_x32(t_lane + C::TM_S + cc * 32, sr);
         tmem_ld_32x32b_x32(t_lane + C::TM_DP + cc * 32, dr);
         tmem_ld_wait();
         uint32_t ds16[16];
-        // dS = P (dP - D), P = 2^(S c - (m + ln l) log2 e)
+        // dS = P (dP - D), P = 2^(S c - (m + ln l) log2 e), two keys at a time
         auto tile = [&](auto mask) {
 #pragma unroll
           for (int k = 0; k < 32; k += 2) {
-            float dsv[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int kc = cc * 32 + k + u;
-              float pr = ex2_approx(fmaf(__uint_as_float(sr[k + u]), c, a));
-              if constexpr (decltype(mask)::value) {
-                if (kc >= klim || (diag && kc > qr)) pr = 0.f;
-              }
-              dsv[u] = pr * (__uint_as_float(dr[k + u]) - dd);
+            const int kc = cc * 32 + k;
+            const float2 x = __ffma2_rn(
+                make_float2(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])), c2, a2);
+            float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            if constexpr (decltype(mask)::value) {
+              if (kc >= klim || (diag && kc > qr)) pr.x = 0.f;
+              if (kc + 1 >= klim || (diag && kc + 1 > qr)) pr.y = 0.f;
             }
-            ds16[k >> 1] = pack_f16x2(dsv[0], dsv[1]);
+            const float2 ds = __fmul2_rn(
+                pr, __fadd2_rn(make_float2(__uint_as_float(dr[k]), __uint_as_float(dr[k + 1])),
+                               nd2));
+            ds16[k >> 1] = pack_f16x2(ds.x, ds.y);
           }
         };
         if (masked)
@@ -552,8 +592,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       float* dst = p.dq + (static_cast<long long>(bidx) * p.N + qp) * p.d + head * D;
 #pragma unroll 1
-      for (int cc = grp * (D / 32 / kBwdEwGroups); cc < (grp + 1) * (D / 32 / kBwdEwGroups);
-           ++cc) {
+      for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(t_lane + C::TM_A0 + cc * 32, v);
         tmem_ld_wait();

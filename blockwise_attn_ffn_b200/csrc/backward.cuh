@@ -162,16 +162,17 @@ __global__ void colsum_reduce_kernel(const float* __restrict__ part, int chunks,
 }
 
 // Per (head t, local row r) the two numbers the attention backward needs for
-// query row r, packed as one 8-byte record (head-major, so a block's 128
-// records are one contiguous 1 KB run a bulk copy can fetch):
-//   qs[t * rows + r] = (-(m + ln l) log2 e, D),  D = sum over head t's
-//   columns of dO[r, c] * O[r, c],
-// with (m, l) the forward's softmax statistics of the row's global position
-// (stats [B][h][N]); P = 2^(S scale log2 e + qs.x) is then the row's
-// probability.  Rows past the sequence get (-inf, 0), which makes their
-// probabilities 0.  One warp per row.
+// query row r, stored per 128-row block as 128 a' then 128 -D (1 KB runs a
+// bulk copy can fetch):
+//   qs[((t * blocks + r / 128) * 2 + 0) * 128 + r % 128] = -(m + ln l) log2 e
+//   qs[((t * blocks + r / 128) * 2 + 1) * 128 + r % 128] = -D,
+// D = sum over head t's columns of dO[r, c] * O[r, c], (m, l) the forward's
+// softmax statistics of the row's global position (stats [B][h][N]);
+// P = 2^(S scale log2 e + a') is then the row's probability.  Rows past the
+// sequence get a' = -inf, D = 0, which makes their probabilities 0.  One
+// warp per row; rows is a multiple of 128.
 __global__ void attn_row_terms_kernel(const __half* __restrict__ dO, const __half* __restrict__ O,
-                                      const float2* __restrict__ stats, float2* __restrict__ qs,
+                                      const float2* __restrict__ stats, float* __restrict__ qs,
                                       long long rows, int d, int h, RowMap map) {
   const int lane = threadIdx.x & 31;
   const long long r = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) >> 5;
@@ -179,18 +180,22 @@ __global__ void attn_row_terms_kernel(const __half* __restrict__ dO, const __hal
   const long long g = map.map(r);
   const int dk = d / h;
   const long long b = g >= 0 ? g / map.N : 0, pos = g >= 0 ? g - b * map.N : 0;
+  const long long blocks = rows / 128;
   for (int t = 0; t < h; ++t) {
     float s = 0.f;
     for (int c = lane; c < dk; c += 32)
       s += __half2float(dO[r * d + t * dk + c]) * __half2float(O[r * d + t * dk + c]);
     s = warp_sum(s);
     if (lane == 0) {
-      float2 v = make_float2(-INFINITY, 0.f);
+      float a = -INFINITY, nd = 0.f;
       if (g >= 0) {
         const float2 ml = stats[(b * h + t) * map.N + pos];
-        v = make_float2(-(ml.x * 1.4426950408889634f + log2f(ml.y)), s);
+        a = -(ml.x * 1.4426950408889634f + log2f(ml.y));
+        nd = -s;
       }
-      qs[t * rows + r] = v;
+      float* blk = qs + (t * blocks + r / 128) * 256;
+      blk[r % 128] = a;
+      blk[128 + r % 128] = nd;
     }
   }
 }

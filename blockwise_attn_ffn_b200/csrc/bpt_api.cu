@@ -712,7 +712,7 @@ bpt_status backward_bf16(const Plan& P, const BwdLayout& L, const void* x, const
   float* dvn = reinterpret_cast<float*>(ws + L.off_dvn);
   hf* dy16 = reinterpret_cast<hf*>(ws + L.off_dy16);
   hf* do16 = reinterpret_cast<hf*>(ws + L.off_do16);
-  float2* qs = reinterpret_cast<float2*>(ws + L.off_D);
+  float* qs = reinterpret_cast<float*>(ws + L.off_D);
   float2* rowstat = reinterpret_cast<float2*>(ws + L.off_rowstat);
   float* y = reinterpret_cast<float*>(ws + L.off_y);
   hf* u16 = reinterpret_cast<hf*>(ws + L.off_u16);

@@ -419,6 +419,31 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// Coefficients of 2^f ~ c0 + c1 f + c2 f^2 + c3 f^3 on [-1/2, 1/2]:
+// relative-error fit at Chebyshev nodes refined towards equal ripple (printed
+// by csrc/fit_exp2_poly.py), max relative error 7.5e-5.
+constexpr float kExp2C0 = 0.99992806f;
+constexpr float kExp2C1 = 0.693261f;
+constexpr float kExp2C2 = 0.24261111f;
+constexpr float kExp2C3 = 0.05517149f;
+
+// 2^x for two lanes on the FMA / ALU pipes.  x is clamped at -125 so that
+// n + (exponent field of 2^f >= 126) stays >= 1: results stay normal floats
+// down to 2^-125, which fp16 P rounds to zero anyway.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  const float2 magic = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 j = __fadd2_rn(x, magic);                          // n in the low mantissa bits
+  const float2 n = __fadd2_rn(j, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));
+  float2 q = __ffma2_rn(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
+  q = __ffma2_rn(q, f, make_float2(kExp2C1, kExp2C1));
+  q = __ffma2_rn(q, f, make_float2(kExp2C0, kExp2C0));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(j.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(j.y) << 23)));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

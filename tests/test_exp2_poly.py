@@ -15,7 +15,7 @@ import re
 import numpy as np
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-SRC = os.path.join(ROOT, "blockwise_attn_ffn_b200", "csrc", "attn_pair_tc.cuh")
+SRC = os.path.join(ROOT, "blockwise_attn_ffn_b200", "csrc", "common.cuh")
 FIT = os.path.join(ROOT, "blockwise_attn_ffn_b200", "csrc", "fit_exp2_poly.py")
 
 
