@@ -295,6 +295,9 @@ def main():
                     help="skip the bench-only unfused-schedule peak-bytes measurement")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="override the workload's N (profiling runs on a smaller case)")
+    ap.add_argument("--attn-qpc", type=int, default=2, choices=[1, 2],
+                    help="query blocks per attention CTA (2: paired, 256 query rows per "
+                         "K/V tile; 1: one 128-row block)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -329,6 +332,8 @@ def main():
         x_host = bpt.to_device(inp, cfg.dtype, dev, pin_x=True)["x"]
     del inp
     x = p["x"]
+    if bpt.bpt_debug_set_attn_qpc(args.attn_qpc) != bpt.BPT_OK:
+        raise SystemExit("bpt_debug_set_attn_qpc failed")
     out, ws = bpt.layer_forward(x, p, cfg.h, cfg.causal)
     torch.cuda.synchronize(dev)
     stream = torch.cuda.current_stream(dev)
@@ -436,7 +441,7 @@ def main():
                        "exactly each call), fp32 accumulation, fp32 residual stream and output")
         if cfg.dtype == "bf16" else "fp32 throughout (CUDA cores)",
         "data": "synthetic: seeded N(0,1) x, N(0,1/fan_in) weights, LN gamma~1+0.1N, beta~0.1N",
-        "config": workload_config(cfg, world),
+        "config": dict(workload_config(cfg, world), attn_query_blocks_per_cta=args.attn_qpc),
         "tflops": tflops,
         "pct_bf16_peak": tflops / world / peaks["bf16_tflops"],
         "pct_bf16_peak_sustained": tflops / world / peak_sus,

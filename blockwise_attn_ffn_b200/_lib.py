@@ -28,6 +28,7 @@ EXPORTED = [
     "bpt_layer_launch_count", "bpt_layer_forward_static", "bpt_debug_inject_fault",
     "bpt_layer_forward_train", "bpt_layer_backward_workspace_size", "bpt_layer_backward",
     "bpt_debug_set_max_wave",
+    "bpt_debug_set_attn_qpc",
 ]
 
 _lib: Optional[ctypes.CDLL] = None
@@ -65,6 +66,8 @@ def load() -> ctypes.CDLL:
     lib.bpt_layer_backward.restype = i32
     lib.bpt_debug_set_max_wave.argtypes = [i64]
     lib.bpt_debug_set_max_wave.restype = i32
+    lib.bpt_debug_set_attn_qpc.argtypes = [i32]
+    lib.bpt_debug_set_attn_qpc.restype = i32
     lib.bpt_read_device_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     lib.bpt_read_device_error.restype = i32
     lib.bpt_status_string.argtypes = [i32]
@@ -136,6 +139,10 @@ def bpt_layer_backward(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, stat
 
 def bpt_debug_set_max_wave(blocks: int) -> int:
     return load().bpt_debug_set_max_wave(blocks)
+
+
+def bpt_debug_set_attn_qpc(qpc: int) -> int:
+    return load().bpt_debug_set_attn_qpc(qpc)
 
 
 def bpt_read_device_error(workspace, stream) -> Tuple[int, int]:

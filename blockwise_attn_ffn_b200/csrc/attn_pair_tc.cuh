@@ -65,6 +65,8 @@ struct AttnPairParams {
   float2* stats;     // nullable: per-row softmax statistics [B][h][N] (m, l)
   uint32_t* err;
   int fault;         // test hook: 2 = CTA 0 never loads V_0 (a lost arrive)
+  int qpc;           // query blocks per CTA: 2 (a pair, 256 query rows sharing
+                     // each K/V tile) or 1 (one 128-row block)
 };
 
 
@@ -87,17 +89,19 @@ struct AttnPairCfg {
   static constexpr int THREADS = 384;
 };
 
-// Pair rank -> first block item of the pair and whether its second block
-// exists.  Causal work is handed out longest first (descending query block).
+// Work rank -> first block item of the CTA's query blocks (qpc of them) and
+// whether its second block exists.  Causal work is handed out longest first
+// (descending query block).
 __device__ __forceinline__ void attn_pair_decode(const AttnPairParams& p, int rank, int& itemA,
                                                  bool& has_b) {
+  const int w = p.qpc;
   if (p.seqs == 0) {
-    const int npairs = (p.count + 1) >> 1;
-    const int q = p.causal ? (npairs - 1 - rank) : rank;
-    itemA = p.item0 + 2 * q;
-    has_b = 2 * q + 1 < p.count;
+    const int nunits = (p.count + w - 1) / w;
+    const int q = p.causal ? (nunits - 1 - rank) : rank;
+    itemA = p.item0 + w * q;
+    has_b = w == 2 && 2 * q + 1 < p.count;
   } else {
-    const int pp = (p.nb + 1) >> 1;  // pairs per sequence
+    const int pp = (p.nb + w - 1) / w;  // units per sequence
     int s, q;
     if (p.causal) {
       q = pp - 1 - rank / p.seqs;
@@ -106,8 +110,8 @@ __device__ __forceinline__ void attn_pair_decode(const AttnPairParams& p, int ra
       s = rank / pp;
       q = rank % pp;
     }
-    itemA = p.item0 + s * p.nb + 2 * q;
-    has_b = 2 * q + 1 < p.nb;
+    itemA = p.item0 + s * p.nb + w * q;
+    has_b = w == 2 && 2 * q + 1 < p.nb;
   }
 }
 

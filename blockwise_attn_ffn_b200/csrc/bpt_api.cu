@@ -40,6 +40,8 @@ using bpt::RowMap;
 constexpr int64_t kMaxWave = BPT_WAVE_BLOCKS;
 // Query blocks per wave (test hook bpt_debug_set_max_wave lowers it).
 std::atomic<int64_t> g_max_wave{kMaxWave};
+// Query blocks per attention CTA: 2 (paired) unless bpt_debug_set_attn_qpc.
+std::atomic<int> g_attn_qpc{2};
 // 16-column groups (of eight per 128-key row) whose exp2 runs on the FMA
 // pipe instead of MUFU (compile-time tuning knobs; 2 of 8 measured fastest).
 #ifndef BPT_EMU_DK128
@@ -415,8 +417,10 @@ cudaError_t launch_attn(const Plan& P, const Wave& wv_, const CUtensorMap& mQKV,
       break;
     }
   ap.fault = fault;
-  const int64_t pairs = wv_.seqs == 0 ? (wv_.count + 1) / 2 : wv_.seqs * ((P.nb + 1) / 2);
-  const unsigned grid = unsigned(pairs * P.h);
+  ap.qpc = g_attn_qpc.load();
+  const int64_t units = wv_.seqs == 0 ? (wv_.count + ap.qpc - 1) / ap.qpc
+                                      : wv_.seqs * ((P.nb + ap.qpc - 1) / ap.qpc);
+  const unsigned grid = unsigned(units * P.h);
   if (P.dk == 128)
     bpt::attn_pair_tc_kernel<128, kEmu128>
         <<<grid, 384, bpt::AttnPairCfg<128, kEmu128>::SMEM, s>>>(mQKV, ap);
@@ -1088,6 +1092,12 @@ const char* bpt_status_string(bpt_status status) {
 bpt_status bpt_debug_set_max_wave(int64_t blocks) {
   if (blocks < 0 || blocks > kMaxWave) return BPT_ERR_INVALID_ARG;
   g_max_wave.store(blocks == 0 ? kMaxWave : blocks);
+  return BPT_OK;
+}
+
+bpt_status bpt_debug_set_attn_qpc(int qpc) {
+  if (qpc != 1 && qpc != 2) return BPT_ERR_INVALID_ARG;
+  g_attn_qpc.store(qpc);
   return BPT_OK;
 }
 

@@ -252,6 +252,21 @@ bpt_status bpt_profile_read(double* ms, int64_t* launches, int n);
 bpt_status bpt_debug_set_max_wave(int64_t blocks);
 
 /*
+ * bpt_debug_set_attn_qpc -- TUNING HOOK: query blocks per attention CTA for
+ * the calls that follow.  2 (the default) pairs two 128-row query blocks in
+ * one CTA, so each K/V tile brought in from L2 serves 256 query rows; 1
+ * gives every query block its own CTA.  ("Blockwise Parallel Transformer —
+ * BPT", section "Choosing the block size: arithmetic intensity": the FLOPs
+ * done per byte re-read equal the rows a block shares them over; the pages
+ * state it for the FFN weights, and the same ratio holds for the K/V tiles
+ * each query block re-reads, 4 b d_k FLOPs per 4 d_k bytes of K and V per
+ * key.)  Outputs are bitwise the same either way: a query block's
+ * arithmetic does not depend on its partner.  Returns BPT_ERR_INVALID_ARG
+ * for any other value.
+ */
+bpt_status bpt_debug_set_attn_qpc(int qpc);
+
+/*
  * bpt_debug_inject_fault -- TEST HOOK for the failure-detection path.  The
  * next BPT_BF16 bpt_layer_forward makes one CTA skip one TMA load, so that
  * the wait for it runs out (after about 2 s) instead of completing:

@@ -1,0 +1,57 @@
+"""Query blocks per attention CTA: paired (256 query rows share each K/V tile,
+the default) against one block per CTA (bpt_debug_set_attn_qpc).
+
+"Blockwise Parallel Transformer — BPT", section "Choosing the block size:
+arithmetic intensity": the work done per byte re-read grows with the rows
+that share it.  Pairing changes only which CTA computes a query block, not
+its arithmetic, so the two settings must give bitwise equal layer outputs and
+softmax statistics; the paired output is itself held to the oracle by the
+parity tests.  Cases cover odd block counts (a pair without its second
+block), ragged tails, both wave layouts (part of one sequence, whole
+sequences) and both head widths.
+"""
+import numpy as np
+import pytest
+import torch
+
+import blockwise_attn_ffn_b200 as bpt
+from blockwise_attn_ffn_b200.inputs import make_inputs
+from test_gpu_parity import small
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    (small("qpc_dk128_causal_odd", 1, 640, 256, 2, 512, True, seed=41), 0),
+    (small("qpc_dk64_noncausal_ragged", 2, 300, 256, 4, 512, False, seed=42), 0),
+    (small("qpc_dk128_split_sequence", 1, 900, 256, 2, 512, True, seed=43), 3),
+    (small("qpc_dk64_whole_sequences", 3, 256, 256, 4, 512, True, seed=44), 2),
+]
+
+
+def forward_train(cfg, dev):
+    out, stats, ws = bpt.layer_forward_train(dev["x"], dev, cfg.h, cfg.causal)
+    st, site = bpt.bpt_read_device_error(ws.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    assert st == bpt.BPT_OK, f"device error {bpt.status_string(st)} at site {site}"
+    return out.cpu().numpy(), stats.cpu().numpy()
+
+
+@pytest.mark.parametrize("cfg,wave", CASES, ids=lambda c: getattr(c, "name", str(c)))
+def test_single_block_ctas_match_pairs_bitwise(cfg, wave):
+    dev = bpt.to_device(make_inputs(cfg), cfg.dtype)
+    assert bpt.bpt_debug_set_max_wave(wave) == bpt.BPT_OK
+    try:
+        assert bpt.bpt_debug_set_attn_qpc(2) == bpt.BPT_OK
+        out2, st2 = forward_train(cfg, dev)
+        assert bpt.bpt_debug_set_attn_qpc(1) == bpt.BPT_OK
+        out1, st1 = forward_train(cfg, dev)
+    finally:
+        bpt.bpt_debug_set_attn_qpc(2)
+        bpt.bpt_debug_set_max_wave(0)
+    assert np.all(np.isfinite(out2))
+    np.testing.assert_array_equal(out1, out2)
+    np.testing.assert_array_equal(st1, st2)
+
+
+def test_qpc_rejects_other_values():
+    for bad in (0, 3, -1):
+        assert bpt.bpt_debug_set_attn_qpc(bad) == bpt.BPT_ERR_INVALID_ARG
