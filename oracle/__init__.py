@@ -13,3 +13,7 @@ from .bpt_backward import (  # noqa: F401
     GRAD_NAMES, attention_backward, gelu_grad, layer_backward, layer_backward_blockwise,
     layer_norm_backward,
 )
+from .bsfa import (  # noqa: F401
+    attention_gated, block_max, calibrate_thresholds, head_scores, keep_mask, layer_block_max,
+    layer_gated,
+)
