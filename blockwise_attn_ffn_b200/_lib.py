@@ -26,7 +26,8 @@ EXPORTED = [
     "bpt_layer_workspace_size", "bpt_layer_forward", "bpt_read_device_error",
     "bpt_status_string", "bpt_profile_enable", "bpt_profile_read",
     "bpt_layer_launch_count", "bpt_layer_forward_static", "bpt_debug_inject_fault",
-    "bpt_layer_forward_train", "bpt_layer_backward_workspace_size", "bpt_layer_backward",
+    "bpt_layer_forward_train", "bpt_layer_forward_bsfa", "bpt_layer_backward_workspace_size",
+    "bpt_layer_backward",
     "bpt_debug_set_max_wave",
     "bpt_debug_set_attn_qpc",
 ]
@@ -58,6 +59,9 @@ def load() -> ctypes.CDLL:
     lib.bpt_layer_forward_train.argtypes = ([vp] * 11 + [i64] * 5 +
                                             [i32, i32, vp, vp, vp, ctypes.c_size_t, vp])
     lib.bpt_layer_forward_train.restype = i32
+    lib.bpt_layer_forward_bsfa.argtypes = ([vp] * 11 + [i64] * 5 +
+                                           [i32, i32, vp, vp, vp, vp, vp, ctypes.c_size_t, vp])
+    lib.bpt_layer_forward_bsfa.restype = i32
     lib.bpt_layer_backward_workspace_size.argtypes = [i64, i64, i64, i64, i64, i32, i32,
                                                       ctypes.POINTER(ctypes.c_size_t)]
     lib.bpt_layer_backward_workspace_size.restype = i32
@@ -108,6 +112,15 @@ def bpt_layer_forward(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
     return load().bpt_layer_forward(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
                                     B, N, d, h, d_ff, int(bool(causal)), dtype, out,
                                     workspace, workspace_bytes, stream)
+
+
+def bpt_layer_forward_bsfa(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
+                           B, N, d, h, d_ff, causal, dtype, thresholds, block_max, kept, out,
+                           workspace, workspace_bytes, stream) -> int:
+    """Pointer-level call (block_max, kept may be None); returns the status code."""
+    return load().bpt_layer_forward_bsfa(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
+                                         B, N, d, h, d_ff, int(bool(causal)), dtype, thresholds,
+                                         block_max, kept, out, workspace, workspace_bytes, stream)
 
 
 def bpt_layer_forward_train(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,

@@ -67,6 +67,10 @@ struct AttnPairParams {
   int fault;         // test hook: 2 = CTA 0 never loads V_0 (a lost arrive)
   int qpc;           // query blocks per CTA: 2 (a pair, 256 query rows sharing
                      // each K/V tile) or 1 (one 128-row block)
+  // Block gating (kernel instantiated with GATE only):
+  const float* gate_t;  // [h][nb] thresholds T in units of s = q.k / sqrt(d_k)
+  float* gate_bmax;     // nullable [B][h][nb][nb]: s_max of each visited pair
+  uint8_t* gate_kept;   // nullable [B][h][nb][nb]: 1 processed, 0 pruned
 };
 
 
@@ -149,7 +153,15 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
-template <int D, int EMU>
+// GATE: block-sparse gating ("Block Sparse Flash Attention", sections
+// "Methodology and Mechanism" and "Gating Mechanism and Threshold
+// Calibration").  After S_X(j) the tile's four softmax warps reduce their
+// row maxima (valid query rows only) to the block maximum s_max; an
+// off-diagonal block with s_max < T[head, i] is pruned: no exponentials, no
+// change to (m, l), no PV product (the UMMA warp reads the tile's decision
+// after the P hand-over).  The K/V ring still loads V_j: it is fetched
+// before S_j exists, and with head-grouped CTAs it comes from L2.
+template <int D, int EMU, bool GATE = false>
 __global__ void __launch_bounds__(384, 1)
     attn_pair_tc_kernel(const __grid_constant__ CUtensorMap mapQKV, const AttnPairParams p) {
   using C = AttnPairCfg<D, EMU>;
@@ -166,6 +178,10 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t drain = smem_u32(bars + 7 + 2 * C::NSLOT);
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
+  // per tile, per softmax warp: {max of its rows (float bits), block count}
+  // in one 64-bit word, so a reader sees a value together with its block
+  __shared__ unsigned long long gate_slot[2][4];
+  __shared__ int gate_keep[2];      // per tile: the current block's decision
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // blockIdx -> (head group, work rank, head): within a group, consecutive
@@ -197,6 +213,8 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(o_done0 + 8 * x, 1);
     }
     mbar_init(drain, 1);
+    if constexpr (GATE)
+      for (int i = 0; i < 8; ++i) (&gate_slot[0][0])[i] = 0ull;
     abort_sh = 0;
     fence_mbar_init();
   }
@@ -297,6 +315,7 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
     };
     uint32_t pph[2] = {0, 0};
+    bool o_started[2] = {false, false};  // first PV of a tile overwrites O
     bool ok = mbar_wait_warp(q_full, 0, abort_flag, p.err, kSiteAttnMma);
     if (ok)
       ok = mbar_wait_warp(ring_full0 + 8 * slot_of(0), phase_of(0), abort_flag, p.err,
@@ -332,7 +351,12 @@ __global__ void __launch_bounds__(384, 1)
         pph[x] ^= 1u;
         tc_fence_after();
         const uint32_t tS = tmem + (x == 0 ? 0u : C::TM_S_B);
-        issue_pv(tS, v_lo, tmem + (x == 0 ? C::TM_O_A : C::TM_O_B), j == 0);
+        // (the tile's decision was written before its P hand-over)
+        const bool kept = !GATE || *reinterpret_cast<volatile int*>(&gate_keep[x]) != 0;
+        if (kept) {
+          issue_pv(tS, v_lo, tmem + (x == 0 ? C::TM_O_A : C::TM_O_B), !o_started[x]);
+          o_started[x] = true;
+        }
         if (j + 1 < nX) {
           if (!k_ready) {
             if (!mbar_wait_warp(ring_full0 + 8 * slot_of(tk), phase_of(tk), abort_flag, p.err,
@@ -371,6 +395,11 @@ __global__ void __launch_bounds__(384, 1)
     float m_run = -INFINITY;  // reference maximum (moves only by > 2^8 in exp2 units)
     float m_true = -INFINITY;  // exact running row maximum, for the statistics
     float l = 0.f;
+    bool o_live = false;       // O holds a PV product (a block has been kept)
+    // the tile's threshold (loaded once: the loop below stores to global
+    // memory, so the compiler would not hoist it)
+    float t_thr = 0.f;
+    if constexpr (GATE) t_thr = nX > 0 ? p.gate_t[head * p.nb + iX] : 0.f;
     bool ok = nX > 0;
     for (int j = 0; j < nX && ok; ++j) {
       if (!mbar_wait_fast(s_full, j & 1, abort_flag, p.err, kSiteAttnSoftmax)) {
@@ -403,63 +432,117 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int k = 0; k < 4; ++k) mxp[k] = fmaxf(mxp[k], mxp[k + 4]);
       const float mx = fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3]));
-      m_true = fmaxf(m_true, mx);
-      float m_new = m_run;
-      bool need = false;
-      if (mx > m_run) {
-        need = (m_run == -INFINITY) || ((mx - m_run) * c > 8.0f);
-        if (need) m_new = mx;
-      }
-      const bool warp_need = __any_sync(0xffffffffu, need) && j > 0;
-      const float alpha =
-          need ? (m_run == -INFINITY ? 0.f : ex2_approx((m_run - m_new) * c)) : 1.f;
-      const float2 cc2 = make_float2(c, c);
-      const float2 mref2 = make_float2(-m_new * c, -m_new * c);
-      float2 sum2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                        make_float2(0.f, 0.f)};
-      // One unrolled loop per tile kind, so the MUFU / FMA choice of each
-      // 16-column group is fixed at compile time (no per-element branch).
-      auto exp_row = [&](auto emu_mask) {
-        constexpr uint32_t kMask = decltype(emu_mask)::value;
+      bool keep_blk = true;
+      if constexpr (GATE) {
+        // block maximum over the tile's valid query rows, in units of s
+        float wm = (iX * C::BQ + r < p.N) ? mx : -INFINITY;
 #pragma unroll
-        for (int cc = 0; cc < C::BKV / 32; ++cc) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int k = 0; k < 32; k += 2) {
-            const int col = cc * 32 + k;
-            float2 a = __ffma2_rn(
-                make_float2(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])), cc2, mref2);
-            float2 e2;
-            if ((kMask >> (col >> 4)) & 1u) {
-              e2 = exp2_poly2(a);
-            } else {
-              e2.x = ex2_approx(a.x);
-              e2.y = ex2_approx(a.y);
-            }
-            sum2[(k >> 1) & 3] = __fadd2_rn(sum2[(k >> 1) & 3], e2);
-            pk[k >> 1] = pack_f16x2(e2.x, e2.y);
+        for (int o = 16; o > 0; o >>= 1) wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, o));
+        // exchange through shared memory: write {max, j + 1}, then poll the
+        // tile's four slots until each carries block j (a warp cannot reach
+        // block j + 1 before all four have read block j: S_j+1 waits for
+        // their P hand-over).  The poll is bounded like every other wait.
+        const uint32_t tag = static_cast<uint32_t>(j + 1);
+        if (lane == 0)
+          *reinterpret_cast<volatile unsigned long long*>(&gate_slot[x][e]) =
+              (static_cast<unsigned long long>(tag) << 32) | __float_as_uint(wm);
+        float bmax = -INFINITY;
+        bool seen = false;
+        const uint64_t g0 = global_ns();
+        for (uint32_t it = 0;; ++it) {
+          const volatile unsigned long long* sl = &gate_slot[x][0];
+          const unsigned long long v0 = sl[0], v1 = sl[1], v2 = sl[2], v3 = sl[3];
+          if (static_cast<uint32_t>(v0 >> 32) == tag && static_cast<uint32_t>(v1 >> 32) == tag &&
+              static_cast<uint32_t>(v2 >> 32) == tag && static_cast<uint32_t>(v3 >> 32) == tag) {
+            bmax = fmaxf(fmaxf(__uint_as_float(static_cast<uint32_t>(v0)),
+                               __uint_as_float(static_cast<uint32_t>(v1))),
+                         fmaxf(__uint_as_float(static_cast<uint32_t>(v2)),
+                               __uint_as_float(static_cast<uint32_t>(v3))));
+            seen = true;
+            break;
           }
-          tmem_st_32x32b_x16(tS + cc * 16, pk);
+          if ((it & 63u) == 63u) {
+            if (*abort_flag) break;
+            if (global_ns() - g0 > BPT_WAIT_LIMIT_NS) {
+              record_error(p.err, kErrTimeout, kSiteAttnSoftmax);
+              *abort_flag = 1;
+              break;
+            }
+          }
         }
-      };
-      if (masked || emu_group_mask(EMU) == 0u)
-        exp_row(std::integral_constant<uint32_t, 0u>{});
-      else
-        exp_row(std::integral_constant<uint32_t, emu_group_mask(EMU)>{});
-      sum2[0] = __fadd2_rn(__fadd2_rn(sum2[0], sum2[1]), __fadd2_rn(sum2[2], sum2[3]));
-      l = alpha * l + (sum2[0].x + sum2[0].y);
-      m_run = m_new;
-      if (warp_need) {
-#pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(tO + cc * 32, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * alpha);
-          tmem_st_32x32b_x32(tO + cc * 32, v);
+        if (!__all_sync(0xffffffffu, seen)) {
+          ok = false;
+          break;
+        }
+        const float smax = bmax * (p.scale_log2 * 0.69314718055994531f);
+        keep_blk = (j == iX) || (smax >= t_thr);
+        if (e == 0 && lane == 0) {
+          gate_keep[x] = keep_blk ? 1 : 0;
+          const long long o = ((static_cast<long long>(bidx) * p.h + head) * p.nb + iX) * p.nb + j;
+          if (p.gate_bmax != nullptr) p.gate_bmax[o] = smax;
+          if (p.gate_kept != nullptr) p.gate_kept[o] = keep_blk ? 1 : 0;
         }
       }
+      if (keep_blk) {
+        m_true = fmaxf(m_true, mx);
+        float m_new = m_run;
+        bool need = false;
+        if (mx > m_run) {
+          need = (m_run == -INFINITY) || ((mx - m_run) * c > 8.0f);
+          if (need) m_new = mx;
+        }
+        const bool warp_need = __any_sync(0xffffffffu, need) && o_live;
+        const float alpha =
+            need ? (m_run == -INFINITY ? 0.f : ex2_approx((m_run - m_new) * c)) : 1.f;
+        const float2 cc2 = make_float2(c, c);
+        const float2 mref2 = make_float2(-m_new * c, -m_new * c);
+        float2 sum2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                          make_float2(0.f, 0.f)};
+        // One unrolled loop per tile kind, so the MUFU / FMA choice of each
+        // 16-column group is fixed at compile time (no per-element branch).
+        auto exp_row = [&](auto emu_mask) {
+          constexpr uint32_t kMask = decltype(emu_mask)::value;
+#pragma unroll
+          for (int cc = 0; cc < C::BKV / 32; ++cc) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int k = 0; k < 32; k += 2) {
+              const int col = cc * 32 + k;
+              float2 a = __ffma2_rn(
+                  make_float2(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])), cc2, mref2);
+              float2 e2;
+              if ((kMask >> (col >> 4)) & 1u) {
+                e2 = exp2_poly2(a);
+              } else {
+                e2.x = ex2_approx(a.x);
+                e2.y = ex2_approx(a.y);
+              }
+              sum2[(k >> 1) & 3] = __fadd2_rn(sum2[(k >> 1) & 3], e2);
+              pk[k >> 1] = pack_f16x2(e2.x, e2.y);
+            }
+            tmem_st_32x32b_x16(tS + cc * 16, pk);
+          }
+        };
+        if (masked || emu_group_mask(EMU) == 0u)
+          exp_row(std::integral_constant<uint32_t, 0u>{});
+        else
+          exp_row(std::integral_constant<uint32_t, emu_group_mask(EMU)>{});
+        sum2[0] = __fadd2_rn(__fadd2_rn(sum2[0], sum2[1]), __fadd2_rn(sum2[2], sum2[3]));
+        l = alpha * l + (sum2[0].x + sum2[0].y);
+        m_run = m_new;
+        if (warp_need) {
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(tO + cc * 32, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * alpha);
+            tmem_st_32x32b_x32(tO + cc * 32, v);
+          }
+        }
+        o_live = true;
+      }  // keep_blk
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();

@@ -22,6 +22,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "bpt.h"
@@ -199,6 +200,9 @@ bpt_status device_info(int* sms, int* pair_clusters = nullptr) {
           cudaFuncSetAttribute(bpt::attn_pair_tc_kernel<128, kEmu128>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                bpt::AttnPairCfg<128, kEmu128>::SMEM) != cudaSuccess ||
+          set_smem(bpt::attn_pair_tc_kernel<64, kEmu64, true>, bpt::AttnPairCfg<64, kEmu64>::SMEM) ||
+          set_smem(bpt::attn_pair_tc_kernel<128, kEmu128, true>,
+                   bpt::AttnPairCfg<128, kEmu128>::SMEM) ||
           set_smem(bpt::gemm_f16_pair_kernel<4, bpt::kLayAkBn>, bpt::kPairSmem) ||
           set_smem(bpt::gemm_f16_pair_kernel<8, bpt::kLayAkBn>, bpt::kPairSmem) ||
           set_smem(bpt::gemm_f16_pair_kernel<4, bpt::kLayAnBn>, bpt::kPairSmem) ||
@@ -399,10 +403,18 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUten
 
 bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
 
+// Block gating of the attention (bpt_layer_forward_bsfa).
+struct AttnGate {
+  const float* t;   // [h][nb] thresholds
+  float* bmax;      // nullable [B][h][nb][nb]
+  uint8_t* kept;    // nullable [B][h][nb][nb]
+};
+
 // One wave of the tensor-core attention: o (fp16 block rows) and, if stats is
-// non-null, the per-row (m, l).
+// non-null, the per-row (m, l); gated when gate is non-null.
 cudaError_t launch_attn(const Plan& P, const Wave& wv_, const CUtensorMap& mQKV, __half* so,
-                        float* stats, uint32_t* err, int fault, cudaStream_t s) {
+                        float* stats, uint32_t* err, int fault, cudaStream_t s,
+                        const AttnGate* gate = nullptr) {
   bpt::AttnPairParams ap{};
   ap.N = int(P.N); ap.nb = int(P.nb); ap.h = int(P.h); ap.d = int(P.d);
   ap.causal = P.causal; ap.item0 = int(wv_.item0); ap.count = int(wv_.count);
@@ -421,19 +433,31 @@ cudaError_t launch_attn(const Plan& P, const Wave& wv_, const CUtensorMap& mQKV,
   const int64_t units = wv_.seqs == 0 ? (wv_.count + ap.qpc - 1) / ap.qpc
                                       : wv_.seqs * ((P.nb + ap.qpc - 1) / ap.qpc);
   const unsigned grid = unsigned(units * P.h);
-  if (P.dk == 128)
+  if (gate != nullptr) {
+    ap.gate_t = gate->t;
+    ap.gate_bmax = gate->bmax;
+    ap.gate_kept = gate->kept;
+    if (P.dk == 128)
+      bpt::attn_pair_tc_kernel<128, kEmu128, true>
+          <<<grid, 384, bpt::AttnPairCfg<128, kEmu128>::SMEM, s>>>(mQKV, ap);
+    else
+      bpt::attn_pair_tc_kernel<64, kEmu64, true>
+          <<<grid, 384, bpt::AttnPairCfg<64, kEmu64>::SMEM, s>>>(mQKV, ap);
+  } else if (P.dk == 128) {
     bpt::attn_pair_tc_kernel<128, kEmu128>
         <<<grid, 384, bpt::AttnPairCfg<128, kEmu128>::SMEM, s>>>(mQKV, ap);
-  else
+  } else {
     bpt::attn_pair_tc_kernel<64, kEmu64>
         <<<grid, 384, bpt::AttnPairCfg<64, kEmu64>::SMEM, s>>>(mQKV, ap);
+  }
   return cudaGetLastError();
 }
 
 bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const void* W_Q,
                         const void* W_K, const void* W_V, const void* W_O, const void* ln2,
                         const void* W_1, const void* b_1, const void* W_2, const void* b_2,
-                        float* out, float* stats, uint8_t* ws, cudaStream_t s, int sms) {
+                        float* out, float* stats, uint8_t* ws, cudaStream_t s, int sms,
+                        const AttnGate* gate) {
   using bf = __nv_bfloat16;
   using hf = __half;
   const int64_t M = P.B * P.N, d = P.d, d_ff = P.d_ff;
@@ -514,7 +538,7 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
     RowMap map{int(wv_.item0), int(P.nb), int(P.N), int(P.blk), 0};
     {
       LaunchScope ls(BPT_KIND_ATTN, s);
-      if (launch_attn(P, wv_, mQKV, so, stats, err, (fault == 2 && w == 0) ? 2 : 0, s) !=
+      if (launch_attn(P, wv_, mQKV, so, stats, err, (fault == 2 && w == 0) ? 2 : 0, s, gate) !=
           cudaSuccess)
         return BPT_ERR_CUDA;
     }
@@ -905,9 +929,11 @@ bpt_status layer_forward_impl(const void* x, const void* ln1, const void* W_Q, c
                               const void* b_1, const void* W_2, const void* b_2, int64_t B,
                               int64_t N, int64_t d, int64_t h, int64_t d_ff, int causal,
                               bpt_dtype dtype, float* out, float* stats, void* workspace,
-                              size_t workspace_bytes, bpt_stream_t stream) {
+                              size_t workspace_bytes, bpt_stream_t stream,
+                              const AttnGate* gate = nullptr) {
   bpt_status st = check_shape(B, N, d, h, d_ff, causal, dtype);
   if (st != BPT_OK) return st;
+  if (gate != nullptr && dtype != BPT_BF16) return BPT_ERR_UNSUPPORTED;
   if (B == 0 || N == 0) return BPT_OK;
   const void* ptrs[] = {x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, out, workspace};
   for (const void* p : ptrs)
@@ -939,7 +965,7 @@ bpt_status layer_forward_impl(const void* x, const void* ln1, const void* W_Q, c
     st = get_encoder();
     if (st != BPT_OK) return st;
     return forward_bf16(P, x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, out, stats, ws, s,
-                        sms);
+                        sms, gate);
   }
   return forward_f32(P, static_cast<const float*>(x), static_cast<const float*>(ln1),
                      static_cast<const float*>(W_Q), static_cast<const float*>(W_K),
@@ -993,6 +1019,49 @@ bpt_status bpt_layer_forward_train(const void* x, const void* ln1, const void* W
                             causal, dtype, out, stats, workspace, workspace_bytes, stream);
 }
 
+
+bpt_status bpt_layer_forward_bsfa(const void* x, const void* ln1, const void* W_Q,
+                                  const void* W_K, const void* W_V, const void* W_O,
+                                  const void* ln2, const void* W_1, const void* b_1,
+                                  const void* W_2, const void* b_2, int64_t B, int64_t N,
+                                  int64_t d, int64_t h, int64_t d_ff, int causal,
+                                  bpt_dtype dtype, const float* thresholds, float* block_max,
+                                  uint8_t* kept, float* out, void* workspace,
+                                  size_t workspace_bytes, bpt_stream_t stream) {
+  bpt_status st = check_shape(B, N, d, h, d_ff, causal, dtype);
+  if (st != BPT_OK) return st;
+  if (dtype != BPT_BF16) return BPT_ERR_UNSUPPORTED;
+  if (thresholds == nullptr) return BPT_ERR_INVALID_ARG;
+  if (B == 0 || N == 0) return BPT_OK;
+  const size_t nb = size_t((N + 127) / 128);
+  const size_t tbytes = size_t(h) * nb * 4, pairs = size_t(B) * size_t(h) * nb * nb;
+  auto span = [](const void* p, size_t n) {
+    return std::make_pair(reinterpret_cast<uintptr_t>(p), reinterpret_cast<uintptr_t>(p) + n);
+  };
+  auto overlap = [](std::pair<uintptr_t, uintptr_t> a, std::pair<uintptr_t, uintptr_t> b) {
+    return a.first < b.second && b.first < a.second;
+  };
+  const auto o = span(out, size_t(B * N * d) * 4), w = span(workspace, workspace_bytes),
+             t = span(thresholds, tbytes), xs = span(x, size_t(B * N * d) * 2);
+  if ((reinterpret_cast<uintptr_t>(thresholds) & 3u) || overlap(t, o) || overlap(t, w))
+    return BPT_ERR_INVALID_ARG;
+  if (block_max != nullptr) {
+    const auto m = span(block_max, pairs * 4);
+    if ((reinterpret_cast<uintptr_t>(block_max) & 3u) || overlap(m, o) || overlap(m, w) ||
+        overlap(m, t) || overlap(m, xs))
+      return BPT_ERR_INVALID_ARG;
+  }
+  if (kept != nullptr) {
+    const auto k = span(kept, pairs);
+    if (overlap(k, o) || overlap(k, w) || overlap(k, t) || overlap(k, xs) ||
+        (block_max != nullptr && overlap(k, span(block_max, pairs * 4))))
+      return BPT_ERR_INVALID_ARG;
+  }
+  const AttnGate gate{thresholds, block_max, kept};
+  return layer_forward_impl(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, B, N, d, h, d_ff,
+                            causal, dtype, out, nullptr, workspace, workspace_bytes, stream,
+                            &gate);
+}
 
 bpt_status bpt_layer_backward_workspace_size(int64_t B, int64_t N, int64_t d, int64_t h,
                                              int64_t d_ff, int causal, bpt_dtype dtype,

@@ -121,6 +121,49 @@ def layer_forward_train(x: torch.Tensor, p: Dict[str, torch.Tensor], h: int, cau
     return out, stats, workspace
 
 
+def layer_forward_bsfa(x: torch.Tensor, p: Dict[str, torch.Tensor], h: int, causal: bool,
+                       thresholds: torch.Tensor, block_max: bool = False, kept: bool = False,
+                       out: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None,
+                       stream: Optional[torch.cuda.Stream] = None):
+    """``layer_forward`` with block-gated attention via ``bpt_layer_forward_bsfa``.
+
+    thresholds: fp32 CUDA tensor [h, nb], nb = ceil(N / 128).  Returns
+    (out, block_max or None, kept or None, workspace); block_max [B, h, nb, nb]
+    fp32 and kept [B, h, nb, nb] uint8 are allocated when requested and hold
+    -inf / 0 where a causal mask visits no pair."""
+    if x.dim() != 3:
+        raise ValueError("x must be [B, N, d]")
+    B, N, d = x.shape
+    d_ff = p["W_1"].shape[1]
+    nb = (N + 127) // 128
+    code = _dtype_code(x)
+    tensors = [x] + [p[k] for k in PARAM_NAMES]
+    for t in tensors:
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != x.dtype:
+            raise ValueError("inputs must be contiguous CUDA tensors of one dtype")
+    if (not thresholds.is_cuda or thresholds.dtype != torch.float32
+            or tuple(thresholds.shape) != (h, nb) or not thresholds.is_contiguous()):
+        raise ValueError(f"thresholds must be a contiguous fp32 CUDA tensor [{h}, {nb}]")
+    bm = (torch.full((B, h, nb, nb), float("-inf"), dtype=torch.float32, device=x.device)
+          if block_max else None)
+    kp = torch.zeros((B, h, nb, nb), dtype=torch.uint8, device=x.device) if kept else None
+    if out is None:
+        out = torch.empty((B, N, d), dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = workspace_for(B, N, d, h, d_ff, causal, x.dtype, x.device)
+    s = stream if stream is not None else torch.cuda.current_stream(x.device)
+    st = _lib.bpt_layer_forward_bsfa(*[t.data_ptr() for t in tensors], B, N, d, h, d_ff, causal,
+                                     code, thresholds.data_ptr(),
+                                     bm.data_ptr() if bm is not None else None,
+                                     kp.data_ptr() if kp is not None else None,
+                                     out.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                     s.cuda_stream)
+    if st != _lib.BPT_OK:
+        raise _lib.BptError(st, "bpt_layer_forward_bsfa")
+    return out, bm, kp, workspace
+
+
 GRAD_SHAPES = ["x", "ln1", "W_Q", "W_K", "W_V", "W_O", "ln2", "W_1", "b_1", "W_2", "b_2"]
 
 

@@ -154,6 +154,49 @@ bpt_status bpt_layer_forward_train(const void* x, const void* ln1, const void* W
                                    size_t workspace_bytes, bpt_stream_t stream);
 
 /*
+ * bpt_layer_forward_bsfa -- bpt_layer_forward with block-sparse gating of the
+ * attention ("Block Sparse Flash Attention", sections "Methodology and
+ * Mechanism" and "Gating Mechanism and Threshold Calibration": exact scores
+ * first, then the block's maximum score against a threshold per head and
+ * query-block position decides whether the value block is processed).
+ *
+ * Blocks are the kernel's 128-row query and key blocks; nb = ceil(N / 128).
+ * For batch b, head t, query block i and a key block j the attention visits
+ * (j <= i when causal, every j otherwise):
+ *   s_max = max of s = q.k / sqrt(d_k) over the block pair's valid query rows
+ *           (position < N) and allowed keys (position < N; j' <= i' causal),
+ *           from the same fp16 Q, K and fp32 accumulation as the scores;
+ *   kept  = (j == i) || s_max >= thresholds[t * nb + i].
+ * A pruned block contributes nothing: not to the row maxima and sums of the
+ * softmax, not to the output (no P V product, no exponentials).  The
+ * diagonal block is always kept, so every row has keys.  A NaN threshold
+ * prunes every off-diagonal block of its query block.
+ *
+ *   thresholds [h, nb] fp32, device, 4-byte aligned: T in units of s, shared
+ *              by the batch; must not overlap out or the workspace.  -inf
+ *              keeps every block (the output is then bitwise that of
+ *              bpt_layer_forward); +inf keeps only the diagonal.
+ *   block_max  [B, h, nb, nb] fp32 or NULL: s_max of every visited pair
+ *              (calibration input); entries of unvisited pairs untouched.
+ *   kept       [B, h, nb, nb] uint8 or NULL: 1 where the pair was processed,
+ *              0 where pruned; unvisited pairs untouched.
+ * block_max and kept must not overlap x, out, the workspace, thresholds or
+ * each other.  Every other argument, the supported shapes and the workspace
+ * are those of bpt_layer_forward.  V tiles are still loaded for pruned
+ * blocks (the K/V ring fetches them before the scores exist).
+ * Returns BPT_ERR_UNSUPPORTED for dtype BPT_F32, BPT_ERR_INVALID_ARG for a
+ * NULL, misaligned or overlapping buffer; otherwise as bpt_layer_forward.
+ */
+bpt_status bpt_layer_forward_bsfa(const void* x, const void* ln1, const void* W_Q,
+                                  const void* W_K, const void* W_V, const void* W_O,
+                                  const void* ln2, const void* W_1, const void* b_1,
+                                  const void* W_2, const void* b_2, int64_t B, int64_t N,
+                                  int64_t d, int64_t h, int64_t d_ff, int causal,
+                                  bpt_dtype dtype, const float* thresholds, float* block_max,
+                                  uint8_t* kept, float* out, void* workspace,
+                                  size_t workspace_bytes, bpt_stream_t stream);
+
+/*
  * bpt_layer_backward_workspace_size -- device workspace bytes
  * bpt_layer_backward needs (pure host arithmetic).  BPT_BF16 layers only
  * (BPT_ERR_UNSUPPORTED for BPT_F32); otherwise the shape rules of

@@ -152,3 +152,29 @@ def test_library_has_no_host_fallback_symbols(lib):
     out = os.popen(f"nm -D --defined-only {bpt.LIB_PATH}").read()
     exported = sorted(set(re.findall(r" T (bpt_\w+)", out)))
     assert exported == header_functions()
+
+
+def fwd_bsfa(ptrs, thr=0x70000000, bmax=0x71000000, kept=0x72000000, B=1, N=256, d=256, h=2,
+             d_ff=512, causal=1, dtype=BF, ws_bytes=1 << 30):
+    return bpt.bpt_layer_forward_bsfa(*ptrs[:11], B, N, d, h, d_ff, causal, dtype, thr, bmax,
+                                      kept, ptrs[11], ptrs[12], ws_bytes, None)
+
+
+def test_bsfa_rejects_bad_gate_buffers():
+    assert fwd_bsfa(GOOD, thr=None) == bpt.BPT_ERR_INVALID_ARG
+    assert fwd_bsfa(GOOD, thr=0x70000002) == bpt.BPT_ERR_INVALID_ARG      # misaligned
+    assert fwd_bsfa(GOOD, bmax=0x71000002) == bpt.BPT_ERR_INVALID_ARG     # misaligned
+    assert fwd_bsfa(GOOD, thr=GOOD[11]) == bpt.BPT_ERR_INVALID_ARG        # overlaps out
+    assert fwd_bsfa(GOOD, thr=GOOD[12] + 64) == bpt.BPT_ERR_INVALID_ARG   # in the workspace
+    assert fwd_bsfa(GOOD, bmax=GOOD[0]) == bpt.BPT_ERR_INVALID_ARG        # overlaps x
+    assert fwd_bsfa(GOOD, kept=0x71000001) == bpt.BPT_ERR_INVALID_ARG     # inside block_max
+    assert fwd_bsfa(GOOD, dtype=F32) == bpt.BPT_ERR_UNSUPPORTED
+    assert fwd_bsfa(GOOD, d=96, h=3) == bpt.BPT_ERR_UNSUPPORTED
+    p = list(GOOD)
+    p[3] = None
+    assert fwd_bsfa(p) == bpt.BPT_ERR_INVALID_ARG                          # a null weight
+
+
+def test_bsfa_empty_is_a_no_op():
+    assert fwd_bsfa([None] * 13, B=0) == bpt.BPT_OK
+    assert fwd_bsfa([None] * 13, N=0) == bpt.BPT_OK
