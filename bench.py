@@ -45,8 +45,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # digest covers the attention kernel, the shared device helpers and the host
 # launch code; after any change the bench reports null until it is retaken.
 ATTN_TRAFFIC = {
-    # 12 launches (6 forwards x 2 waves): waves of 406 + 115 and 1281 + 130 MB
-    "long_n64k": {"digest": "ea4e1983acde9257", "bytes_per_launch": 967160533},
+    # 12 launches (6 forwards x 2 waves): waves of 406 + 116 and 1292 + 135 MB
+    "long_n64k": {"digest": "6733337549f20bef", "bytes_per_launch": 974527595},
 }
 TRAFFIC_SOURCES = ("blockwise_attn_ffn_b200/csrc/attn_pair_tc.cuh",
                    "blockwise_attn_ffn_b200/csrc/common.cuh",
@@ -217,6 +217,62 @@ def measure_backward(bpt, cfg, x, p, stream, dev, args, flops, world, peaks, dis
                     "backward (3 x forward FLOPs counted; recomputation not counted)"}
 
 
+# ---------------------------------------------- gated attention (BSFA) --
+def measure_bsfa(bpt, cfg, x, p, out_dense, ms_dense, stream, dev, args, world, dist):
+    """Times bpt_layer_forward_bsfa ("Block Sparse Flash Attention": exact
+    block maxima, a per-(head, query block) threshold, pruned blocks skip
+    their exponentials and PV products).  Thresholds keep the top k
+    off-diagonal key blocks per query block, calibrated (package
+    ``bsfa.calibrate``) on the block maxima of one other seeded synthetic x
+    through the same weights; the timed x is the bench's.  Reports the kept
+    fraction, the time per forward (CUDA events, max over ranks), the speed-up
+    over the dense forward and the largest output deviation from it."""
+    import numpy as np
+    import torch
+    from blockwise_attn_ffn_b200 import bsfa as bbsfa
+    from blockwise_attn_ffn_b200 import dist as bdist
+    from blockwise_attn_ffn_b200.inputs import make_inputs
+    nb = (cfg.N + 127) // 128
+    cal = make_inputs(cfg.with_(seed=cfg.seed + 7919))
+    xc = bpt.to_device(cal, cfg.dtype, dev)["x"]  # its weights are dropped: p's are used
+    del cal
+    none = torch.full((cfg.h, nb), float("-inf"), dtype=torch.float32, device=dev)
+    o2 = torch.empty_like(out_dense)
+    _, bm, _, ws = bpt.layer_forward_bsfa(xc, p, cfg.h, cfg.causal, none, block_max=True, out=o2)
+    del xc
+    T = torch.from_numpy(bbsfa.calibrate(bm.cpu().numpy(), args.bsfa_k, cfg.causal)).to(dev)
+    _, _, kept, _ = bpt.layer_forward_bsfa(x, p, cfg.h, cfg.causal, T, kept=True, out=o2,
+                                           workspace=ws)
+    vis = np.tril(np.ones((nb, nb), bool)) if cfg.causal else np.ones((nb, nb), bool)
+    off = vis & ~np.eye(nb, dtype=bool)
+    kept_frac = float(kept.cpu().numpy()[:, :, off].mean()) if off.any() else 1.0
+    for _ in range(args.warmup):
+        bpt.layer_forward_bsfa(x, p, cfg.h, cfg.causal, T, out=o2, workspace=ws)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        bpt.layer_forward_bsfa(x, p, cfg.h, cfg.causal, T, out=o2, workspace=ws)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    st, site = bpt.bpt_read_device_error(ws.data_ptr(), stream.cuda_stream)
+    if st != bpt.BPT_OK:
+        raise SystemExit(f"device error in bsfa {bpt.status_string(st)} site {site}")
+    ms = bdist.max_over_ranks(e0.elapsed_time(e1), dist, dev) / args.steps
+    dev_max = float((o2 - out_dense).abs().max())
+    return {"k": args.bsfa_k, "kept_offdiag_frac": kept_frac, "ms_per_step": ms,
+            "tokens_per_s": cfg.B * cfg.N * world / (ms / 1e3),
+            "speedup_vs_dense": ms_dense / ms, "max_abs_dev_vs_dense": dev_max,
+            "max_abs_dense": float(out_dense.abs().max()), "steps": args.steps,
+            "calibration": "top-k off-diagonal blocks per query block from the block maxima "
+                           "of one other seeded synthetic x (same weights)",
+            "note": "approximate attention (the pages' method): synthetic inputs have no "
+                    "learned attention sparsity, so the deviation says nothing about model "
+                    "quality; V tiles of pruned blocks are still loaded"}
+
+
 # ------------------------------------------------- unfused peak bytes --
 def unfused_torch_peak_bytes(cfg, p, dev):
     """Peak device bytes of the plain unfused schedule, measured once outside
@@ -295,6 +351,10 @@ def main():
                     help="skip the bench-only unfused-schedule peak-bytes measurement")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="override the workload's N (profiling runs on a smaller case)")
+    ap.add_argument("--no-bsfa", action="store_true",
+                    help="skip the gated-attention (BSFA) forward measurement")
+    ap.add_argument("--bsfa-k", type=int, default=32,
+                    help="off-diagonal key blocks kept per query block by the BSFA thresholds")
     ap.add_argument("--attn-qpc", type=int, default=2, choices=[1, 2],
                     help="query blocks per attention CTA (2: paired, 256 query rows per "
                          "K/V tile; 1: one 128-row block)")
@@ -472,6 +532,8 @@ def main():
     if not args.no_backward and cfg.dtype == "bf16":
         line["backward"] = measure_backward(bpt, cfg, x, p, stream, dev, args, flops, world,
                                             peaks, dist)
+    if not args.no_bsfa and cfg.dtype == "bf16":
+        line["bsfa"] = measure_bsfa(bpt, cfg, x, p, out, ms_step, stream, dev, args, world, dist)
     if not args.no_unfused_peak and cfg.dtype == "bf16":
         line["peak_bytes"]["unfused_torch_measured"] = unfused_torch_peak_bytes(cfg, p, dev)
 
