@@ -85,7 +85,7 @@ struct AttnPairCfg {
   static constexpr int OFF_QB = TILE;
   static constexpr int OFF_RING = 2 * TILE;
   static constexpr int OFF_BAR = OFF_RING + NSLOT * TILE;
-  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  static constexpr int SMEM = OFF_BAR + 512 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t TM_S_B = 128;
   static constexpr uint32_t TM_O_A = 256;
@@ -142,6 +142,22 @@ __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_
       : "memory");
 }
 
+// 32 lanes x 8 columns (the O rescale: few registers, since the scores are
+// still live when it runs).
+__device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
+                   taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+               "r"(r[7])
+               : "memory");
+}
+
 // D[tmem] (+)= A[tmem] * B[smem desc], fp16 inputs, fp32 accumulate.
 __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                              uint32_t idesc, uint32_t accumulate) {
@@ -173,9 +189,10 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t ring_full0 = smem_u32(bars + 1);
   const uint32_t ring_empty0 = smem_u32(bars + 1 + C::NSLOT);
   const uint32_t s_full0 = smem_u32(bars + 1 + 2 * C::NSLOT);   // [A, B]
-  const uint32_t p_full0 = smem_u32(bars + 3 + 2 * C::NSLOT);   // [A, B]
-  const uint32_t o_done0 = smem_u32(bars + 5 + 2 * C::NSLOT);   // [A, B]
-  const uint32_t drain = smem_u32(bars + 7 + 2 * C::NSLOT);
+  // [A: chunks 0..3, B: chunks 0..3]: P columns 32c.. of the tile handed over
+  const uint32_t p_chunk0 = smem_u32(bars + 3 + 2 * C::NSLOT);
+  const uint32_t o_done0 = smem_u32(bars + 11 + 2 * C::NSLOT);  // [A, B]
+  const uint32_t drain = smem_u32(bars + 13 + 2 * C::NSLOT);
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   // per tile, per softmax warp: {max of its rows (float bits), block count}
@@ -209,7 +226,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(s_full0 + 8 * x, 1);
-      mbar_init(p_full0 + 8 * x, 4);
+      for (int c = 0; c < 4; ++c) mbar_init(p_chunk0 + 8 * (4 * x + c), 4);
       mbar_init(o_done0 + 8 * x, 1);
     }
     mbar_init(drain, 1);
@@ -301,12 +318,16 @@ __global__ void __launch_bounds__(384, 1)
       }
       __syncwarp();
     };
-    auto issue_pv = [&](uint32_t tP, uint32_t v_lo, uint32_t d_tmem, bool first) {
+    // the two 16-key k-steps of PV for keys 32c..32c+31 (P packed: 16
+    // columns per 32 keys); `first` = O not yet written by this tile
+    auto issue_pv_chunk = [&](uint32_t tP, uint32_t v_lo, uint32_t d_tmem, int c, bool first) {
       if (leader) {
 #pragma unroll
-        for (int k = 0; k < C::BKV / 16; ++k)
+        for (int kk = 0; kk < 2; ++kk) {
+          const int k = 2 * c + kk;
           umma_ts(d_tmem, tP + 8 * k, v_lo + ((k * 2048) >> 4), hi, idesc_o,
                   (!first || k > 0) ? 1u : 0u);
+        }
       }
       __syncwarp();
     };
@@ -344,19 +365,24 @@ __global__ void __launch_bounds__(384, 1)
       for (int x = 0; x < 2 && ok; ++x) {
         const int nX = x == 0 ? nA : nB;
         if (j >= nX) continue;
-        if (!mbar_wait_warp(p_full0 + 8 * x, pph[x], abort_flag, p.err, kSiteAttnMma)) {
-          ok = false;
-          break;
-        }
-        pph[x] ^= 1u;
-        tc_fence_after();
         const uint32_t tS = tmem + (x == 0 ? 0u : C::TM_S_B);
-        // (the tile's decision was written before its P hand-over)
-        const bool kept = !GATE || *reinterpret_cast<volatile int*>(&gate_keep[x]) != 0;
-        if (kept) {
-          issue_pv(tS, v_lo, tmem + (x == 0 ? C::TM_O_A : C::TM_O_B), !o_started[x]);
-          o_started[x] = true;
+        const uint32_t tO = tmem + (x == 0 ? C::TM_O_A : C::TM_O_B);
+        // PV_X(j) 32 keys at a time, each chunk as soon as its P is stored
+        bool kept = true;
+        for (int c = 0; c < 4; ++c) {
+          if (!mbar_wait_warp(p_chunk0 + 8 * (4 * x + c), pph[x], abort_flag, p.err,
+                              kSiteAttnMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          // (the tile's decision was written before its first P hand-over)
+          if (c == 0) kept = !GATE || *reinterpret_cast<volatile int*>(&gate_keep[x]) != 0;
+          if (kept) issue_pv_chunk(tS, v_lo, tO, c, !o_started[x]);
         }
+        if (!ok) break;
+        pph[x] ^= 1u;
+        if (kept) o_started[x] = true;
         if (j + 1 < nX) {
           if (!k_ready) {
             if (!mbar_wait_warp(ring_full0 + 8 * slot_of(tk), phase_of(tk), abort_flag, p.err,
@@ -389,7 +415,8 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(e * 32) << 16);
     const uint32_t tS = t_lane + (x == 0 ? 0u : C::TM_S_B);
     const uint32_t tO = t_lane + (x == 0 ? C::TM_O_A : C::TM_O_B);
-    const uint32_t s_full = s_full0 + 8 * x, p_full = p_full0 + 8 * x, o_done = o_done0 + 8 * x;
+    const uint32_t s_full = s_full0 + 8 * x, o_done = o_done0 + 8 * x;
+    const uint32_t p_chunk = p_chunk0 + 8 * (4 * x);  // [4]
     const float c = p.scale_log2;
     const bool ragged = (p.N % C::BKV) != 0;
     float m_run = -INFINITY;  // reference maximum (moves only by > 2^8 in exp2 units)
@@ -494,12 +521,26 @@ __global__ void __launch_bounds__(384, 1)
         const bool warp_need = __any_sync(0xffffffffu, need) && o_live;
         const float alpha =
             need ? (m_run == -INFINITY ? 0.f : ex2_approx((m_run - m_new) * c)) : 1.f;
+        // Rescale O first: the PV of this block starts with its first P
+        // chunk (PV_X(j-1) is complete: S_X(j), issued after it, has landed).
+        if (warp_need) {
+#pragma unroll 1
+          for (int cc = 0; cc < D / 8; ++cc) {
+            uint32_t v[8];
+            tmem_ld_32x32b_x8(tO + cc * 8, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * alpha);
+            tmem_st_32x32b_x8(tO + cc * 8, v);
+          }
+        }
         const float2 cc2 = make_float2(c, c);
         const float2 mref2 = make_float2(-m_new * c, -m_new * c);
         float2 sum2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                           make_float2(0.f, 0.f)};
         // One unrolled loop per tile kind, so the MUFU / FMA choice of each
         // 16-column group is fixed at compile time (no per-element branch).
+        // Each 32-key chunk of P is handed over as soon as it is stored.
         auto exp_row = [&](auto emu_mask) {
           constexpr uint32_t kMask = decltype(emu_mask)::value;
 #pragma unroll
@@ -521,6 +562,10 @@ __global__ void __launch_bounds__(384, 1)
               pk[k >> 1] = pack_f16x2(e2.x, e2.y);
             }
             tmem_st_32x32b_x16(tS + cc * 16, pk);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_chunk + 8 * cc);
           }
         };
         if (masked || emu_group_mask(EMU) == 0u)
@@ -530,23 +575,15 @@ __global__ void __launch_bounds__(384, 1)
         sum2[0] = __fadd2_rn(__fadd2_rn(sum2[0], sum2[1]), __fadd2_rn(sum2[2], sum2[3]));
         l = alpha * l + (sum2[0].x + sum2[0].y);
         m_run = m_new;
-        if (warp_need) {
-#pragma unroll 1
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t v[32];
-            tmem_ld_32x32b_x32(tO + cc * 32, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * alpha);
-            tmem_st_32x32b_x32(tO + cc * 32, v);
-          }
-        }
         o_live = true;
+      } else {
+        // pruned: no P; the hand-overs still tell the UMMA warp that S_X(j)
+        // has been read and carry the decision
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0)
+          for (int cc = 0; cc < 4; ++cc) mbar_arrive(p_chunk + 8 * cc);
       }  // keep_blk
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
     }
     if (ok && mbar_wait_fast(o_done, 0, abort_flag, p.err, kSiteAttnSoftmax)) {
       tc_fence_after();
