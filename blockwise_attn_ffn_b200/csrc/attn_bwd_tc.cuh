@@ -23,10 +23,15 @@
 //       added into the fp32 gradients (waves run in stream order, so each
 //       key row is updated by one CTA at a time).
 //   attn_bwd_dq_tc_kernel  one CTA per (128-query block, head): Q, dO stay
-//       in shared memory, K, V stream through the ring.  Per key block:
+//       in shared memory, K and V stream through rings.  Per key block:
 //         S = Q K^T, dP = dO V^T          UMMA (SS)
 //         dS                              elementwise warps, fp16 in TMEM
 //         dQ += dS K                      UMMA with A from TMEM
+//       The scores are double-buffered in TMEM (S, S, dP, dQ fill the 512
+//       columns at d_k = 128), so S_j+2 is computed while block j is being
+//       finished; the elementwise pass keeps P in registers from S alone and
+//       forms dS once dP lands.  Issue order S_0, dP_0, S_1, then per block
+//       j: dQ_j, dP_j+1, S_j+2.
 // A 128-row tile of Q, K, V or dO in shared memory ([d_k/64 chunks][128
 // rows][64], 128-byte swizzle) is a K-major operand in one product and an
 // MN-major one in another (same bytes, different descriptor).
@@ -65,12 +70,16 @@ struct AttnBwdCfg {
   static constexpr int KV_OFF_RING = 2 * TILE;
   static constexpr int KV_OFF_BAR = KV_OFF_RING + NSLOT * KV_SLOT;
   static constexpr int KV_SMEM = KV_OFF_BAR + 256 + 1024;
-  // dQ kernel: Q, dO resident, ring of (K, V)
-  static constexpr int Q_SLOT = 2 * TILE;
-  static constexpr int Q_OFF_RING = 2 * TILE;
-  static constexpr int Q_OFF_BAR = Q_OFF_RING + NSLOT * Q_SLOT;
-  static constexpr int Q_SMEM = Q_OFF_BAR + 256 + 1024;
+  // dQ kernel: Q, dO resident; K in a three-slot ring (held until dQ_j),
+  // V in a two-slot ring (held until dP_j)
+  static constexpr int QK_SLOTS = 3, QV_SLOTS = 2;
+  static constexpr int Q_OFF_K = 2 * TILE;
+  static constexpr int Q_OFF_V = Q_OFF_K + QK_SLOTS * TILE;
+  static constexpr int Q_OFF_BAR = Q_OFF_V + QV_SLOTS * TILE;
+  static constexpr int Q_SMEM = Q_OFF_BAR + 512 + 1024;
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_A0 = 256, TM_A1 = 256 + D;
+  // dQ kernel: scores double-buffered (S_j in TQ_S + 128 (j % 2)), dQ at TQ_A
+  static constexpr uint32_t TQ_S = 0, TQ_DP = 256, TQ_A = 384;
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(KV_SMEM <= 232448 && Q_SMEM <= 232448, "shared memory budget");
 };
@@ -422,23 +431,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::Q_OFF_BAR);
   const uint32_t q_full = smem_u32(bars + 0);
-  const uint32_t ring_full0 = smem_u32(bars + 1);
-  const uint32_t ring_empty0 = smem_u32(bars + 1 + C::NSLOT);
-  const uint32_t s_full = smem_u32(bars + 1 + 2 * C::NSLOT);
-  const uint32_t p_chunk0 = smem_u32(bars + 2 + 2 * C::NSLOT);  // [4]: P / dS columns 32c..
-  const uint32_t acc_done = smem_u32(bars + 6 + 2 * C::NSLOT);
-  const uint32_t drain = smem_u32(bars + 7 + 2 * C::NSLOT);
+  const uint32_t k_full0 = smem_u32(bars + 1);   // [3]
+  const uint32_t k_empty0 = smem_u32(bars + 4);  // [3]
+  const uint32_t v_full0 = smem_u32(bars + 7);   // [2]
+  const uint32_t v_empty0 = smem_u32(bars + 9);  // [2]
+  const uint32_t s_full0 = smem_u32(bars + 11);  // [2]: S_j landed in buffer j % 2
+  const uint32_t s_free0 = smem_u32(bars + 13);  // [2]: buffer j % 2 read by every warp
+  const uint32_t dp_full = smem_u32(bars + 15);
+  const uint32_t ds_chunk0 = smem_u32(bars + 16);  // [4]: dS columns 32c.. handed over
+  const uint32_t acc_done = smem_u32(bars + 20);
+  const uint32_t drain = smem_u32(bars + 21);
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < C::NSLOT; ++s) {
-      mbar_init(ring_full0 + 8 * s, 1);
-      mbar_init(ring_empty0 + 8 * s, 1);
+    for (int s = 0; s < C::QK_SLOTS; ++s) {
+      mbar_init(k_full0 + 8 * s, 1);
+      mbar_init(k_empty0 + 8 * s, 1);
     }
-    mbar_init(s_full, 1);
-    for (int c = 0; c < 4; ++c) mbar_init(p_chunk0 + 8 * c, 4);
+    for (int s = 0; s < C::QV_SLOTS; ++s) {
+      mbar_init(v_full0 + 8 * s, 1);
+      mbar_init(v_empty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(s_full0 + 8 * b, 1);
+      mbar_init(s_free0 + 8 * b, 4);
+    }
+    mbar_init(dp_full, 1);
+    for (int c = 0; c < 4; ++c) mbar_init(ds_chunk0 + 8 * c, 4);
     mbar_init(acc_done, 1);
     mbar_init(drain, 1);
     abort_sh = 0;
@@ -458,35 +479,43 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     const bool leader = lane == 0;
-    int armed[C::NSLOT];
-    for (int s = 0; s < C::NSLOT; ++s) armed[s] = -1;
+    int k_armed[C::QK_SLOTS], v_armed[C::QV_SLOTS];
+    for (int s = 0; s < C::QK_SLOTS; ++s) k_armed[s] = -1;
+    for (int s = 0; s < C::QV_SLOTS; ++s) v_armed[s] = -1;
     if (leader) {
       mbar_arrive_expect_tx(q_full, 2 * C::TILE);
       tma_load_4d(smem_u32(smem), &mapQKV, q_full, 0, ib * 128, chQ, bidx);
       tma_load_3d(smem_u32(smem + C::TILE), &mapDO, q_full, 0, static_cast<int>(lrow),
                   head * D / 64);
     }
-    bool ok = true;
-    for (int j = 0; j < n_kv && ok; ++j) {
-      const int slot = j % C::NSLOT;
-      const uint32_t phase = static_cast<uint32_t>((j / C::NSLOT) & 1);
-      if (!mbar_wait_warp(ring_empty0 + 8 * slot, phase ^ 1u, abort_flag, p.err,
-                          kSiteAttnProducer)) {
-        ok = false;
+    for (int j = 0; j < n_kv; ++j) {
+      const int ks = j % C::QK_SLOTS, vs = j % C::QV_SLOTS;
+      const uint32_t kph = static_cast<uint32_t>((j / C::QK_SLOTS) & 1);
+      const uint32_t vph = static_cast<uint32_t>((j / C::QV_SLOTS) & 1);
+      if (!mbar_wait_warp(k_empty0 + 8 * ks, kph ^ 1u, abort_flag, p.err, kSiteAttnProducer))
         break;
-      }
       if (leader) {
-        armed[slot] = static_cast<int>(phase);
-        const uint32_t sl = smem_u32(smem + C::Q_OFF_RING + slot * C::Q_SLOT);
-        mbar_arrive_expect_tx(ring_full0 + 8 * slot, 2 * C::TILE);
-        tma_load_4d(sl, &mapQKV, ring_full0 + 8 * slot, 0, j * 128, chK, bidx);
-        tma_load_4d(sl + C::TILE, &mapQKV, ring_full0 + 8 * slot, 0, j * 128, chV, bidx);
+        k_armed[ks] = static_cast<int>(kph);
+        mbar_arrive_expect_tx(k_full0 + 8 * ks, C::TILE);
+        tma_load_4d(smem_u32(smem + C::Q_OFF_K + ks * C::TILE), &mapQKV, k_full0 + 8 * ks, 0,
+                    j * 128, chK, bidx);
+      }
+      __syncwarp();
+      if (!mbar_wait_warp(v_empty0 + 8 * vs, vph ^ 1u, abort_flag, p.err, kSiteAttnProducer))
+        break;
+      if (leader) {
+        v_armed[vs] = static_cast<int>(vph);
+        mbar_arrive_expect_tx(v_full0 + 8 * vs, C::TILE);
+        tma_load_4d(smem_u32(smem + C::Q_OFF_V + vs * C::TILE), &mapQKV, v_full0 + 8 * vs, 0,
+                    j * 128, chV, bidx);
       }
       __syncwarp();
     }
     mbar_wait_drain(q_full, 0, p.err);
-    for (int s = 0; s < C::NSLOT; ++s)
-      if (armed[s] >= 0) mbar_wait_drain(ring_full0 + 8 * s, static_cast<uint32_t>(armed[s]), p.err);
+    for (int s = 0; s < C::QK_SLOTS; ++s)
+      if (k_armed[s] >= 0) mbar_wait_drain(k_full0 + 8 * s, static_cast<uint32_t>(k_armed[s]), p.err);
+    for (int s = 0; s < C::QV_SLOTS; ++s)
+      if (v_armed[s] >= 0) mbar_wait_drain(v_full0 + 8 * s, static_cast<uint32_t>(v_armed[s]), p.err);
   } else if (warp == 1) {
     // ---------------------------------------------------------- UMMA issue
     const bool leader = lane == 0;
@@ -498,34 +527,65 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (leader) umma_commit(bar);
       __syncwarp();
     };
-    bool ok = mbar_wait_warp(q_full, 0, abort_flag, p.err, kSiteAttnMma);
-    for (int j = 0; j < n_kv && ok; ++j) {
-      const int slot = j % C::NSLOT;
-      const uint32_t phase = static_cast<uint32_t>((j / C::NSLOT) & 1);
-      if (!mbar_wait_warp(ring_full0 + 8 * slot, phase, abort_flag, p.err, kSiteAttnMma)) break;
+    auto k_slot = [&](int j) { return smem_u32(smem + C::Q_OFF_K + (j % C::QK_SLOTS) * C::TILE); };
+    auto v_slot = [&](int j) { return smem_u32(smem + C::Q_OFF_V + (j % C::QV_SLOTS) * C::TILE); };
+    // S_j = Q K_j^T into buffer j % 2, once K_j has landed
+    auto issue_s = [&](int j) -> bool {
+      if (!mbar_wait_warp(k_full0 + 8 * (j % C::QK_SLOTS),
+                          static_cast<uint32_t>((j / C::QK_SLOTS) & 1), abort_flag, p.err,
+                          kSiteAttnMma))
+        return false;
       tc_fence_after();
-      const uint32_t sl = smem_u32(smem + C::Q_OFF_RING + slot * C::Q_SLOT);
-      if (leader) {
-        bwd_issue_ss<D>(tmem + C::TM_S, q_lo, sdesc_lo(sl, 16), idesc_s);               // S
-        bwd_issue_ss<D>(tmem + C::TM_DP, do_lo, sdesc_lo(sl + C::TILE, 16), idesc_s);   // dP
-      }
+      if (leader)
+        bwd_issue_ss<D>(tmem + C::TQ_S + 128u * static_cast<uint32_t>(j & 1), q_lo,
+                        sdesc_lo(k_slot(j), 16), idesc_s);
       __syncwarp();
-      commit(s_full);
-      // dQ += dS K, 32 key columns at a time as the elementwise warps hand them over
-      for (int cc = 0; cc < 4 && ok; ++cc) {
-        if (!mbar_wait_warp(p_chunk0 + 8 * cc, static_cast<uint32_t>(j & 1), abort_flag, p.err,
+      commit(s_full0 + 8 * (j & 1));
+      return true;
+    };
+    // dP_j = dO V_j^T, once V_j has landed; V_j's slot is free once it is done
+    auto issue_dp = [&](int j) -> bool {
+      if (!mbar_wait_warp(v_full0 + 8 * (j % C::QV_SLOTS),
+                          static_cast<uint32_t>((j / C::QV_SLOTS) & 1), abort_flag, p.err,
+                          kSiteAttnMma))
+        return false;
+      tc_fence_after();
+      if (leader) bwd_issue_ss<D>(tmem + C::TQ_DP, do_lo, sdesc_lo(v_slot(j), 16), idesc_s);
+      __syncwarp();
+      commit(dp_full);
+      commit(v_empty0 + 8 * (j % C::QV_SLOTS));
+      return true;
+    };
+    bool ok = mbar_wait_warp(q_full, 0, abort_flag, p.err, kSiteAttnMma) && issue_s(0) &&
+              issue_dp(0) && (n_kv < 2 || issue_s(1));
+    for (int j = 0; j < n_kv && ok; ++j) {
+      // dQ += dS_j K_j, 32 key columns at a time as they are handed over
+      for (int cc = 0; cc < 4; ++cc) {
+        if (!mbar_wait_warp(ds_chunk0 + 8 * cc, static_cast<uint32_t>(j & 1), abort_flag, p.err,
                             kSiteAttnMma)) {
           ok = false;
           break;
         }
         tc_fence_after();
         if (leader)
-          bwd_issue_ts_chunk<D>(tmem + C::TM_A0, tmem + C::TM_S, sdesc_lo(sl, C::CHUNK),
-                                idesc_o, cc, j == 0);                                    // dQ
+          bwd_issue_ts_chunk<D>(tmem + C::TQ_A, tmem + C::TQ_DP, sdesc_lo(k_slot(j), C::CHUNK),
+                                idesc_o, cc, j == 0);
         __syncwarp();
       }
       if (!ok) break;
-      commit(ring_empty0 + 8 * slot);
+      commit(k_empty0 + 8 * (j % C::QK_SLOTS));
+      // dP_j+1 overwrites dP_j / dS_j: after dQ_j (in order) and after every
+      // warp's last dS hand-over (all of dP_j has been read)
+      if (j + 1 < n_kv && !(ok = issue_dp(j + 1))) break;
+      // S_j+2 reuses S_j's buffer once every warp has read S_j
+      if (j + 2 < n_kv) {
+        if (!mbar_wait_warp(s_free0 + 8 * (j & 1), static_cast<uint32_t>((j >> 1) & 1),
+                            abort_flag, p.err, kSiteAttnMma) ||
+            !issue_s(j + 2)) {
+          ok = false;
+          break;
+        }
+      }
     }
     commit(acc_done);
     commit(drain);
@@ -543,8 +603,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const float2 nd2 = make_float2(rt[128 + qr], rt[128 + qr]);  // -D
     bool ok = true;
     for (int j = 0; j < n_kv && ok; ++j) {
-      if (!mbar_wait_warp(s_full, static_cast<uint32_t>(j & 1), abort_flag, p.err,
-                          kSiteAttnSoftmax)) {
+      if (!mbar_wait_warp(s_full0 + 8 * (j & 1), static_cast<uint32_t>((j >> 1) & 1), abort_flag,
+                          p.err, kSiteAttnSoftmax)) {
         ok = false;
         break;
       }
@@ -552,14 +612,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool diag = p.causal && j == ib;
       const int klim = p.N - j * 128;  // keys >= klim are past the sequence
       const bool masked = diag || klim < 128;
-#pragma unroll 1
+      const uint32_t tS = t_lane + C::TQ_S + 128u * static_cast<uint32_t>(j & 1);
+      uint32_t pp[64];  // P of this query row, fp16 pairs, kept for the dS phase
+      // ---- phase 1: P = 2^(S c + a') from S alone
+#pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
-        uint32_t sr[32], dr[32];
-        tmem_ld_32x32b_x32(t_lane + C::TM_S + cc * 32, sr);
-        tmem_ld_32x32b_x32(t_lane + C::TM_DP + cc * 32, dr);
+        uint32_t sr[32];
+        tmem_ld_32x32b_x32(tS + cc * 32, sr);
         tmem_ld_wait();
-        uint32_t ds16[16];
-        // dS = P (dP - D), P = 2^(S c - (m + ln l) log2 e), two keys at a time
+        if (cc == 3) {
+          // every score of buffer j % 2 is in registers: S_j+2 may go there
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_free0 + 8 * (j & 1));
+        }
         auto tile = [&](auto mask) {
 #pragma unroll
           for (int k = 0; k < 32; k += 2) {
@@ -571,21 +637,39 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               if (kc >= klim || (diag && kc > qr)) pr.x = 0.f;
               if (kc + 1 >= klim || (diag && kc + 1 > qr)) pr.y = 0.f;
             }
-            const float2 ds = __fmul2_rn(
-                pr, __fadd2_rn(make_float2(__uint_as_float(dr[k]), __uint_as_float(dr[k + 1])),
-                               nd2));
-            ds16[k >> 1] = pack_f16x2(ds.x, ds.y);
+            pp[cc * 16 + (k >> 1)] = pack_f16x2(pr.x, pr.y);
           }
         };
         if (masked)
           tile(std::true_type{});
         else
           tile(std::false_type{});
-        tmem_st16(t_lane + C::TM_S + packed_col(cc), ds16);
+      }
+      // ---- phase 2: dS = P (dP - D)
+      if (!mbar_wait_warp(dp_full, static_cast<uint32_t>(j & 1), abort_flag, p.err,
+                          kSiteAttnSoftmax)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t dr[32], ds16[16];
+        tmem_ld_32x32b_x32(t_lane + C::TQ_DP + cc * 32, dr);
+        tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < 32; k += 2) {
+          const float2 pr =
+              __half22float2(*reinterpret_cast<const __half2*>(&pp[cc * 16 + (k >> 1)]));
+          const float2 v = __fmul2_rn(
+              pr, __fadd2_rn(make_float2(__uint_as_float(dr[k]), __uint_as_float(dr[k + 1])), nd2));
+          ds16[k >> 1] = pack_f16x2(v.x, v.y);
+        }
+        tmem_st16(t_lane + C::TQ_DP + packed_col(cc), ds16);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_chunk0 + 8 * cc);
+        if (lane == 0) mbar_arrive(ds_chunk0 + 8 * cc);
       }
     }
     if (ok && mbar_wait_warp(acc_done, 0, abort_flag, p.err, kSiteAttnSoftmax)) {
@@ -594,7 +678,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t v[32];
-        tmem_ld_32x32b_x32(t_lane + C::TM_A0 + cc * 32, v);
+        tmem_ld_32x32b_x32(t_lane + C::TQ_A + cc * 32, v);
         tmem_ld_wait();
         if (q_ok) {
 #pragma unroll
