@@ -75,8 +75,8 @@ __global__ void pack3_f32_to_f16_kernel(const float* __restrict__ a, const float
 //   dx_ln = LN'(X[g]) applied to DY[r] (gamma from `gamma`)
 //   OUT[g] = (accumulate ? OUT[g] : RES[g]) + dx_ln;  OUT16[r] = fp16(OUT[g]) if OUT16
 //   rowstat[r] = (mean, rstd) of X[g]
-template <typename TX>
-__global__ void ln_backward_kernel(const TX* __restrict__ X, const __nv_bfloat16* __restrict__ gamma,
+template <typename TX, typename TG = __nv_bfloat16>
+__global__ void ln_backward_kernel(const TX* __restrict__ X, const TG* __restrict__ gamma,
                                    const float* __restrict__ DY, const float* __restrict__ RES,
                                    float* __restrict__ OUT, __half* __restrict__ OUT16,
                                    float2* __restrict__ rowstat, long long rows, int d,
@@ -104,7 +104,7 @@ __global__ void ln_backward_kernel(const TX* __restrict__ X, const __nv_bfloat16
   const float rstd = rsqrtf(warp_sum(v) / d + 1e-5f);
   float a = 0.f, b = 0.f;  // sum dxh, sum dxh * xh
   for (int c = lane; c < d; c += 32) {
-    const float dxh = dy[c] * __bfloat162float(gamma[c]);
+    const float dxh = dy[c] * ld_as_float(gamma + c);
     a += dxh;
     b += dxh * (ld_as_float(x + c) - mu) * rstd;
   }
@@ -114,7 +114,7 @@ __global__ void ln_backward_kernel(const TX* __restrict__ X, const __nv_bfloat16
   const float* res = accumulate ? out : RES + g * d;
   for (int c = lane; c < d; c += 32) {
     const float xh = (ld_as_float(x + c) - mu) * rstd;
-    const float dxh = dy[c] * __bfloat162float(gamma[c]);
+    const float dxh = dy[c] * ld_as_float(gamma + c);
     const float val = res[c] + rstd * (dxh - a - xh * b);
     out[c] = val;
     if (OUT16) OUT16[r * d + c] = __float2half(val);

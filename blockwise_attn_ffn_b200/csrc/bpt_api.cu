@@ -33,6 +33,7 @@
 #include "gemm_tc.cuh"
 #include "rows.cuh"
 #include "simt_f32.cuh"
+#include "backward_f32.cuh"
 
 namespace {
 
@@ -712,6 +713,185 @@ cudaError_t launch_colsum(const TA* A, int a_global, const TX* X, const float2* 
   return cudaGetLastError();
 }
 
+// Workspace of the fp32 backward (after the forward plan's regions; fp32
+// throughout): FFN pre-activation and its gradient, wave copies of dZ, dY
+// and dO, dVn, the attention row terms, LN row statistics, y, LN1(x), dQ,
+// dK, dV, dU and the column-sum partials.
+struct BwdLayoutF32 {
+  size_t off_hpre, off_dh, off_dzw, off_dvn, off_dyw, off_dow, off_rt, off_rowstat, off_y, off_u,
+      off_dq, off_dk, off_dv, off_du, off_part, total;
+  int64_t part_cols;
+};
+
+BwdLayoutF32 make_bwd_layout_f32(const Plan& P) {
+  BwdLayoutF32 L{};
+  const size_t R = size_t(P.P * P.blk), M = size_t(P.B * P.N), d = size_t(P.d),
+               dff = size_t(P.d_ff), h = size_t(P.h);
+  size_t off = align_up(P.total, 1024);
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 1024);
+    return o;
+  };
+  L.off_hpre = take(R * dff * 4);
+  L.off_dh = take(R * dff * 4);
+  L.off_dzw = take(R * d * 4);
+  L.off_dvn = take(R * d * 4);
+  L.off_dyw = take(R * d * 4);
+  L.off_dow = take(R * d * 4);
+  L.off_rt = take(R * h * 8);
+  L.off_rowstat = take(std::max(R, M) * 8);
+  L.off_y = take(M * d * 4);
+  L.off_u = take(M * d * 4);
+  L.off_dq = take(M * d * 4);
+  L.off_dk = take(M * d * 4);
+  L.off_dv = take(M * d * 4);
+  L.off_du = take(M * d * 4);
+  L.part_cols = int64_t(std::max(d, dff));
+  L.off_part = take(2 * size_t(kColChunks) * size_t(L.part_cols) * 4);
+  L.total = off;
+  return L;
+}
+
+// fp32 backward on the CUDA cores: the bf16 schedule (waves recomputed from
+// x and (m, l), gradients accumulated wave by wave, no atomics), fp32 SIMT
+// kernels (backward_f32.cuh) for the products.
+bpt_status backward_f32(const Plan& P, const BwdLayoutF32& L, const float* x, const float* ln1,
+                        const float* W_Q, const float* W_K, const float* W_V, const float* W_O,
+                        const float* ln2, const float* W_1, const float* b_1, const float* W_2,
+                        const float* stats, const float* dZ, float* dx, float* d_ln1,
+                        float* dW_Q, float* dW_K, float* dW_V, float* dW_O, float* d_ln2,
+                        float* dW_1, float* db_1, float* dW_2, float* db_2, uint8_t* ws,
+                        cudaStream_t s) {
+  const int64_t M = P.B * P.N, d = P.d, d_ff = P.d_ff, h = P.h;
+  uint32_t* err = reinterpret_cast<uint32_t*>(ws);
+  float* qkv = reinterpret_cast<float*>(ws + P.off_qkv);
+  float* so = reinterpret_cast<float*>(ws + P.off_o);
+  float* sv = reinterpret_cast<float*>(ws + P.off_v);
+  float* sh = reinterpret_cast<float*>(ws + P.off_h);
+  float* hpre = reinterpret_cast<float*>(ws + L.off_hpre);
+  float* dh = reinterpret_cast<float*>(ws + L.off_dh);
+  float* dzw = reinterpret_cast<float*>(ws + L.off_dzw);
+  float* dvn = reinterpret_cast<float*>(ws + L.off_dvn);
+  float* dyw = reinterpret_cast<float*>(ws + L.off_dyw);
+  float* dow = reinterpret_cast<float*>(ws + L.off_dow);
+  float2* rt = reinterpret_cast<float2*>(ws + L.off_rt);
+  float2* rowstat = reinterpret_cast<float2*>(ws + L.off_rowstat);
+  float* y = reinterpret_cast<float*>(ws + L.off_y);
+  float* u = reinterpret_cast<float*>(ws + L.off_u);
+  float* dq = reinterpret_cast<float*>(ws + L.off_dq);
+  float* dk = reinterpret_cast<float*>(ws + L.off_dk);
+  float* dv = reinterpret_cast<float*>(ws + L.off_dv);
+  float* du = reinterpret_cast<float*>(ws + L.off_du);
+  float* part_a = reinterpret_cast<float*>(ws + L.off_part);
+  float* part_b = part_a + size_t(kColChunks) * size_t(L.part_cols);
+  const float* gamma1 = ln1;
+  const float* gamma2 = ln2;
+
+  const std::pair<float*, size_t> zero[] = {
+      {dW_Q, size_t(d * d)}, {dW_K, size_t(d * d)}, {dW_V, size_t(d * d)}, {dW_O, size_t(d * d)},
+      {dW_1, size_t(d * d_ff)}, {db_1, size_t(d_ff)}, {dW_2, size_t(d_ff * d)}, {db_2, size_t(d)},
+      {d_ln1, size_t(2 * d)}, {d_ln2, size_t(2 * d)}, {dk, size_t(M * d)}, {dv, size_t(M * d)}};
+  for (const auto& z : zero)
+    if (cudaMemsetAsync(z.first, 0, z.second * sizeof(float), s) != cudaSuccess)
+      return BPT_ERR_CUDA;
+  // C (+)= op(A) op(B) on the CUDA cores
+  auto gemm = [&](int64_t m, int64_t n, int64_t k, const float* A, int64_t lda, int a_t,
+                  const float* B, int64_t ldb, int b_t, float* C, int64_t ldc, int acc) {
+    bpt::GemmGenF32 g{int(m), int(n), int(k), A, lda, a_t, B, ldb, b_t, C, ldc, acc};
+    const dim3 grid(unsigned((n + 63) / 64), unsigned((m + 63) / 64));
+    bpt::gemm_f32_gen_kernel<<<grid, 256, 0, s>>>(g);
+    return cudaGetLastError() == cudaSuccess;
+  };
+  auto blocks = [](int64_t n) { return unsigned(std::min<int64_t>((n + 255) / 256, 4096)); };
+  RowMap ident{0, 1, 1, 1, 1};
+  if (launch_ln<float, float, float>(x, ln1, u, M, d, ident, err, s) != cudaSuccess)
+    return BPT_ERR_CUDA;
+  const float* wqkv[3] = {W_Q, W_K, W_V};
+  for (int i = 0; i < 3; ++i)
+    if (!gemm(M, d, d, u, d, 0, wqkv[i], d, 0, qkv + i * d, 3 * d, 0)) return BPT_ERR_CUDA;
+  const float scale = float(1.0 / std::sqrt(double(P.dk)));
+  for (int64_t w = 0; w < P.n_waves; ++w) {
+    const Wave wv = P.wave(w);
+    const int64_t rows = wv.count * P.blk;
+    RowMap map{int(wv.item0), int(P.nb), int(P.N), int(P.blk), 0};
+    // forward recomputation of this wave: o, y, LN2(y), FFN pre-activation and hidden
+    {
+      bpt::AttnF32Params ap{};
+      ap.qkv = qkv; ap.o = so; ap.N = int(P.N); ap.nb = int(P.nb); ap.h = int(h);
+      ap.d = int(d); ap.causal = P.causal; ap.item0 = int(wv.item0); ap.blk = int(P.blk);
+      ap.scale = scale;
+      ap.stats = nullptr;
+      const size_t smem = size_t(3 * 64 * P.dk + 64 * 65) * 4;
+      bpt::attn_f32_kernel<<<unsigned(wv.count * h), 256, smem, s>>>(ap);
+      if (cudaGetLastError() != cudaSuccess) return BPT_ERR_CUDA;
+    }
+    {
+      bpt::GemmF32Params g{};
+      g.M = int(rows); g.N = int(d); g.K = int(d); g.n_sub = int(d);
+      g.A = so; g.B[0] = g.B[1] = g.B[2] = W_O;
+      g.epi = bpt::kEpiResidX; g.out = y; g.ld_out = d; g.resid = x; g.ld_resid = d;
+      g.bias = nullptr; g.map = map;
+      const dim3 grid(unsigned((d + bpt::kF32Tile - 1) / bpt::kF32Tile),
+                      unsigned((rows + bpt::kF32Tile - 1) / bpt::kF32Tile));
+      bpt::gemm_f32_kernel<<<grid, 256, 0, s>>>(g);
+      if (cudaGetLastError() != cudaSuccess) return BPT_ERR_CUDA;
+    }
+    if (launch_ln<float, float, float>(y, ln2, sv, rows, d, map, err, s) != cudaSuccess)
+      return BPT_ERR_CUDA;
+    if (!gemm(rows, d_ff, d, sv, d, 0, W_1, d_ff, 0, hpre, d_ff, 0)) return BPT_ERR_CUDA;
+    bpt::bias_gelu_keep_f32_kernel<<<blocks(rows * d_ff), 256, 0, s>>>(hpre, b_1, sh, rows,
+                                                                        int(d_ff));
+    // FFN backward
+    bpt::gather_rows_f32_kernel<<<blocks(rows * d), 256, 0, s>>>(dZ, dzw, rows, int(d), map);
+    if (!gemm(d_ff, d, rows, sh, d_ff, 1, dzw, d, 0, dW_2, d, 1) ||
+        !gemm(rows, d_ff, d, dzw, d, 0, W_2, d, 1, dh, d_ff, 0))
+      return BPT_ERR_CUDA;
+    bpt::gelu_grad_mul_f32_kernel<<<blocks(rows * d_ff), 256, 0, s>>>(dh, hpre, rows * d_ff);
+    if (!gemm(d, d_ff, rows, sv, d, 1, dh, d_ff, 0, dW_1, d_ff, 1)) return BPT_ERR_CUDA;
+    if (launch_colsum<float, float>(dh, 0, nullptr, nullptr, rows, d_ff, map, part_a, part_b,
+                                    db_1, nullptr, s) != cudaSuccess ||
+        launch_colsum<float, float>(dZ, 1, nullptr, nullptr, rows, d, map, part_a, part_b, db_2,
+                                    nullptr, s) != cudaSuccess)
+      return BPT_ERR_CUDA;
+    if (!gemm(rows, d, d_ff, dh, d_ff, 0, W_1, d_ff, 1, dvn, d, 0)) return BPT_ERR_CUDA;
+    // LN2 backward: dY = dZ + LN2'(dVn) -> dx (global rows), then its wave copy
+    bpt::ln_backward_kernel<float, float><<<unsigned((rows * 32 + 255) / 256), 256, 0, s>>>(
+        y, gamma2, dvn, dZ, dx, nullptr, rowstat, rows, int(d), map, 0);
+    if (launch_colsum<float, float>(dvn, 0, y, rowstat, rows, d, map, part_a, part_b, d_ln2 + d,
+                                    d_ln2, s) != cudaSuccess)
+      return BPT_ERR_CUDA;
+    bpt::gather_rows_f32_kernel<<<blocks(rows * d), 256, 0, s>>>(dx, dyw, rows, int(d), map);
+    // W_O backward
+    if (!gemm(d, d, rows, so, d, 1, dyw, d, 0, dW_O, d, 1) ||
+        !gemm(rows, d, d, dyw, d, 0, W_O, d, 1, dow, d, 0))
+      return BPT_ERR_CUDA;
+    // attention backward of this wave's query rows
+    bpt::attn_row_terms_f32_kernel<<<unsigned((rows * 32 + 255) / 256), 256, 0, s>>>(
+        dow, so, reinterpret_cast<const float2*>(stats), rt, rows, int(d), int(h), map);
+    bpt::AttnBwdF32Params ab{};
+    ab.qkv = qkv; ab.dO = dow; ab.rt = rt; ab.dq = dq; ab.dk = dk; ab.dv = dv;
+    ab.rows = rows; ab.N = int(P.N); ab.d = int(d); ab.h = int(h); ab.causal = P.causal;
+    ab.scale = scale; ab.map = map;
+    bpt::attn_bwd_dq_f32_kernel<<<unsigned((rows * h * 32 + 255) / 256), 256, 0, s>>>(ab);
+    bpt::attn_bwd_dkv_f32_kernel<<<unsigned((M * h * 32 + 255) / 256), 256, 0, s>>>(ab, M);
+    if (cudaGetLastError() != cudaSuccess) return BPT_ERR_CUDA;
+  }
+  // QKV projection and LN1 backward over all rows
+  const float* dqkv[3] = {dq, dk, dv};
+  float* dWqkv[3] = {dW_Q, dW_K, dW_V};
+  for (int i = 0; i < 3; ++i)
+    if (!gemm(d, d, M, u, d, 1, dqkv[i], d, 0, dWqkv[i], d, 1) ||
+        !gemm(M, d, d, dqkv[i], d, 0, wqkv[i], d, 1, du, d, i > 0 ? 1 : 0))
+      return BPT_ERR_CUDA;
+  bpt::ln_backward_kernel<float, float><<<unsigned((M * 32 + 255) / 256), 256, 0, s>>>(
+      x, gamma1, du, nullptr, dx, nullptr, rowstat, M, int(d), ident, 1);
+  if (launch_colsum<float, float>(du, 0, x, rowstat, M, d, ident, part_a, part_b, d_ln1 + d,
+                                  d_ln1, s) != cudaSuccess)
+    return BPT_ERR_CUDA;
+  return BPT_OK;
+}
+
 bpt_status backward_bf16(const Plan& P, const BwdLayout& L, const void* x, const void* ln1,
                          const void* W_Q, const void* W_K, const void* W_V, const void* W_O,
                          const void* ln2, const void* W_1, const void* b_1, const void* W_2,
@@ -1069,9 +1249,8 @@ bpt_status bpt_layer_backward_workspace_size(int64_t B, int64_t N, int64_t d, in
   if (bytes == nullptr) return BPT_ERR_INVALID_ARG;
   const bpt_status st = check_shape(B, N, d, h, d_ff, causal, dtype);
   if (st != BPT_OK) return st;
-  if (dtype != BPT_BF16) return BPT_ERR_UNSUPPORTED;
   const Plan P = make_plan(B, N, d, h, d_ff, causal, dtype);
-  *bytes = make_bwd_layout(P).total;
+  *bytes = dtype == BPT_BF16 ? make_bwd_layout(P).total : make_bwd_layout_f32(P).total;
   return BPT_OK;
 }
 
@@ -1087,7 +1266,6 @@ bpt_status bpt_layer_backward(const void* x, const void* ln1, const void* W_Q, c
   (void)b_2;  // the output's bias does not enter any gradient but its own
   bpt_status st = check_shape(B, N, d, h, d_ff, causal, dtype);
   if (st != BPT_OK) return st;
-  if (dtype != BPT_BF16) return BPT_ERR_UNSUPPORTED;
   if (B == 0 || N == 0) return BPT_OK;
   const void* ins[] = {x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, stats, dZ, workspace};
   for (const void* p : ins)
@@ -1098,16 +1276,17 @@ bpt_status bpt_layer_backward(const void* x, const void* ln1, const void* W_Q, c
                               size_t(2 * d) * 4, size_t(d * d_ff) * 4, size_t(d_ff) * 4,
                               size_t(d_ff * d) * 4, size_t(d) * 4};
   const Plan P = make_plan(B, N, d, h, d_ff, causal, dtype);
-  const BwdLayout L = make_bwd_layout(P);
-  if (workspace_bytes < L.total) return BPT_ERR_WORKSPACE;
+  const size_t ws_need =
+      dtype == BPT_BF16 ? make_bwd_layout(P).total : make_bwd_layout_f32(P).total;
+  if (workspace_bytes < ws_need) return BPT_ERR_WORKSPACE;
   // Outputs must be aligned and must not overlap each other, the workspace,
   // or the inputs they are written after being read from (x, stats, dZ).
   const uintptr_t wsb = reinterpret_cast<uintptr_t>(workspace);
   const std::pair<uintptr_t, size_t> reads[] = {
-      {reinterpret_cast<uintptr_t>(x), size_t(B * N * d) * 2},
+      {reinterpret_cast<uintptr_t>(x), size_t(B * N * d) * P.esize},
       {reinterpret_cast<uintptr_t>(stats), size_t(B * h * N) * 8},
       {reinterpret_cast<uintptr_t>(dZ), size_t(B * N * d) * 4},
-      {wsb, L.total}};
+      {wsb, ws_need}};
   for (int i = 0; i < 11; ++i) {
     if (outs[i] == nullptr || misaligned(outs[i])) return BPT_ERR_INVALID_ARG;
     const uintptr_t a = reinterpret_cast<uintptr_t>(outs[i]);
@@ -1121,11 +1300,18 @@ bpt_status bpt_layer_backward(const void* x, const void* ln1, const void* W_Q, c
   int sms = 0;
   st = device_info(&sms);
   if (st != BPT_OK) return st;
-  st = get_encoder();
-  if (st != BPT_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   if (cudaMemsetAsync(ws, 0, kHeaderBytes, s) != cudaSuccess) return BPT_ERR_CUDA;
+  if (dtype == BPT_F32) {
+    auto f = [](const void* q) { return static_cast<const float*>(q); };
+    return backward_f32(P, make_bwd_layout_f32(P), f(x), f(ln1), f(W_Q), f(W_K), f(W_V), f(W_O),
+                        f(ln2), f(W_1), f(b_1), f(W_2), stats, dZ, dx, d_ln1, dW_Q, dW_K, dW_V,
+                        dW_O, d_ln2, dW_1, db_1, dW_2, db_2, ws, s);
+  }
+  st = get_encoder();
+  if (st != BPT_OK) return st;
+  const BwdLayout L = make_bwd_layout(P);
   return backward_bf16(P, L, x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, stats, dZ, dx, d_ln1,
                        dW_Q, dW_K, dW_V, dW_O, d_ln2, dW_1, db_1, dW_2, db_2, ws, s, sms);
 }

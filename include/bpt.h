@@ -198,9 +198,8 @@ bpt_status bpt_layer_forward_bsfa(const void* x, const void* ln1, const void* W_
 
 /*
  * bpt_layer_backward_workspace_size -- device workspace bytes
- * bpt_layer_backward needs (pure host arithmetic).  BPT_BF16 layers only
- * (BPT_ERR_UNSUPPORTED for BPT_F32); otherwise the shape rules of
- * bpt_layer_workspace_size.
+ * bpt_layer_backward needs (pure host arithmetic) for a layer of the given
+ * dtype; the shape rules of bpt_layer_workspace_size.
  */
 bpt_status bpt_layer_backward_workspace_size(int64_t B, int64_t N, int64_t d, int64_t h,
                                              int64_t d_ff, int causal, bpt_dtype dtype,
@@ -215,7 +214,7 @@ bpt_status bpt_layer_backward_workspace_size(int64_t B, int64_t N, int64_t d, in
  * [N, N] or [N, d_ff] tensor is formed (the FFN hidden exists for one wave of
  * query blocks at a time, as in the forward).
  *
- *   x, ln1, W_Q .. b_2   the forward's inputs (bf16, as bpt_layer_forward)
+ *   x, ln1, W_Q .. b_2   the forward's inputs (dtype, as bpt_layer_forward)
  *   stats [B, h, N, 2] fp32   the (m, l) bpt_layer_forward_train wrote
  *   dZ    [B, N, d] fp32      upstream gradient of the layer output
  * Outputs, fp32, overwritten (not accumulated):
@@ -226,15 +225,17 @@ bpt_status bpt_layer_backward_workspace_size(int64_t B, int64_t N, int64_t d, in
  * overlap each other, the workspace, x, stats or dZ.  Workspace: >=
  * bpt_layer_backward_workspace_size bytes, caller-owned.
  *
- * Arithmetic: the GEMMs run on the tensor cores with fp16 operands (the
- * activations, upstream gradient and intermediate gradients rounded to fp16
- * as in the forward) and fp32 accumulation; weight gradients accumulate in
- * fp32 across waves; LayerNorm, GELU' and the bias / gamma / beta sums are
+ * Arithmetic, BPT_BF16: the GEMMs run on the tensor cores with fp16 operands
+ * (the activations, upstream gradient and intermediate gradients rounded to
+ * fp16 as in the forward) and fp32 accumulation; weight gradients accumulate
+ * in fp32 across waves; LayerNorm, GELU' and the bias / gamma / beta sums are
  * fp32 (the sums in a fixed order: results are deterministic).  The
  * attention gradients recompute P = exp(s - m) / l on the tensor cores (fp16
  * Q, K, V, dO, P and dS, fp32 accumulation), dK and dV by key block and dQ
- * by query block, without atomics.
- * Returns BPT_ERR_UNSUPPORTED for BPT_F32; BPT_ERR_INVALID_ARG for a null,
+ * by query block, without atomics.  BPT_F32: the same schedule with every
+ * product and sum in fp32 on the CUDA cores (meant for small layers: the
+ * attention gradients take one warp per row and head).
+ * Returns BPT_ERR_INVALID_ARG for a null,
  * misaligned or overlapping pointer; BPT_ERR_WORKSPACE if the workspace is
  * too small; otherwise as bpt_layer_forward (device errors via
  * bpt_read_device_error).

@@ -5,7 +5,7 @@ of query blocks from x and the saved (m, l) (bpt_layer_forward_train) and
 accumulates the gradients; the oracle is the chain rule through the unfused
 layer (``oracle.layer_backward``, pinned against torch autograd).
 
-Tolerance.  Every GEMM operand on the backward path is rounded to fp16
+Tolerance (bf16 layers).  Every GEMM operand on the backward path is rounded to fp16
 (relative 2^-11 ~ 4.9e-4) and the longest chain (dZ -> dH -> dHpre -> dVn ->
 dY -> dO -> dS -> dQ, dK, dV -> dU -> dx) passes about ten such roundings,
 each product accumulated in fp32: per-element relative error of order 5e-3.
@@ -108,3 +108,52 @@ def test_backward_is_deterministic():
     b = run_backward(cfg, inp, dZ)
     for k in a:
         np.testing.assert_array_equal(a[k], b[k], err_msg=k)
+
+
+# fp32 layers: the same schedule on the CUDA cores, every product in fp32.
+# Errors are fp32 rounding along the same chain (unit roundoff 6e-8, sums of
+# a few hundred terms): held to relative L2 1e-4 and elementwise 1e-3 of the
+# tensor's largest magnitude.
+F32_CASES = [
+    small("bwd_f32_causal_ragged", 2, 150, 64, 2, 192, True, dtype="f32", seed=31, bias=0.5),
+    small("bwd_f32_noncausal", 1, 100, 96, 3, 160, False, dtype="f32", seed=32),
+    small("bwd_f32_dk128_multiblock", 1, 200, 256, 2, 256, True, dtype="f32", seed=33),
+]
+
+
+def check_f32(name, got, want):
+    assert np.all(np.isfinite(got)), f"{name}: non-finite gradient"
+    scale = np.abs(want).max()
+    rel_l2 = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
+    mx = np.abs(got - want).max()
+    print(f"  {name:12s} rel L2 {rel_l2:.2e}  max {mx / max(scale, 1e-30):.2e} of scale")
+    assert rel_l2 <= 1e-4, f"{name}: relative L2 error {rel_l2:.3e}"
+    assert mx <= 1e-3 * scale, f"{name}: max abs error {mx:.3e} vs scale {scale:.3e}"
+
+
+@pytest.mark.parametrize("cfg", F32_CASES, ids=lambda c: c.name)
+def test_f32_backward_matches_oracle(cfg):
+    inp = make_inputs(cfg)
+    dZ = upstream(cfg)
+    got = run_backward(cfg, inp, dZ)
+    want = oracle.layer_backward(inp, cfg.h, cfg.causal, dZ.astype(np.float64))
+    for k in NAMES:
+        check_f32(k, got[k], want[k])
+    for k, (g, b) in {"ln1": ("gamma1", "beta1"), "ln2": ("gamma2", "beta2")}.items():
+        check_f32(k + ".gamma", got[k][0], want[g])
+        check_f32(k + ".beta", got[k][1], want[b])
+
+
+def test_f32_backward_multi_wave():
+    cfg = small("bwd_f32_split", 1, 300, 64, 2, 192, True, dtype="f32", seed=34)
+    assert bpt.bpt_debug_set_max_wave(2) == bpt.BPT_OK
+    try:
+        inp = make_inputs(cfg)
+        dZ = upstream(cfg)
+        got = run_backward(cfg, inp, dZ)
+    finally:
+        bpt.bpt_debug_set_max_wave(0)
+    want = oracle.layer_backward(inp, cfg.h, cfg.causal, dZ.astype(np.float64))
+    for k in NAMES:
+        check_f32(k, got[k], want[k])
+
