@@ -370,6 +370,11 @@ __global__ void __launch_bounds__(384, 1)
         // PV_X(j) 32 keys at a time, each chunk as soon as its P is stored
         bool kept = true;
         for (int c = 0; c < 4; ++c) {
+          // A pruned block hands all four chunks over at once, after S_X(j)
+          // was read in full: its first hand-over is all the UMMA warp needs.
+          // (The skipped phases complete regardless; the next block's waits,
+          // one phase later, are unaffected.)
+          if (GATE && c > 0 && !kept) continue;
           if (!mbar_wait_warp(p_chunk0 + 8 * (4 * x + c), pph[x], abort_flag, p.err,
                               kSiteAttnMma)) {
             ok = false;
