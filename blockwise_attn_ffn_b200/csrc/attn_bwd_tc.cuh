@@ -86,6 +86,15 @@ struct AttnBwdCfg {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kBwdThreads = 256;
+#ifndef BPT_BWD_HANDOVERS
+#define BPT_BWD_HANDOVERS 2
+#endif
+// Hand-overs per 128-column tile from the elementwise warps to the UMMA warp
+// (4: every 32 columns; 2: every 64).  Each costs the UMMA warp a barrier
+// wait (~100 clocks even when complete), and that warp is the critical path.
+constexpr int kBwdHandovers = BPT_BWD_HANDOVERS;
+static_assert(kBwdHandovers == 2 || kBwdHandovers == 4, "2 or 4 hand-overs per tile");
+constexpr int kBwdChunksPerHand = 4 / kBwdHandovers;
 
 // Issue a 128 x 128 x d_k SS product: D[tmem] = A[a_lo] B[b_lo]^T, both
 // K-major tiles (the k-step walks 32 B inside a 64-column chunk, then the
@@ -269,12 +278,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // one gradient product, 32 query columns at a time as the elementwise
     // warps hand them over on chunk barriers cb[0..3]
     auto issue_grad = [&](int t, uint32_t cb, uint32_t acc, uint32_t a_tm, uint32_t b_lo) {
-      for (int cc = 0; cc < 4; ++cc) {
-        if (!mbar_wait_warp(cb + 8 * cc, static_cast<uint32_t>(t & 1), abort_flag, p.err,
+      for (int hh = 0; hh < kBwdHandovers; ++hh) {
+        if (!mbar_wait_warp(cb + 8 * hh, static_cast<uint32_t>(t & 1), abort_flag, p.err,
                             kSiteAttnMma))
           return false;
         tc_fence_after();
-        if (leader) bwd_issue_ts_chunk<D>(acc, a_tm, b_lo, idesc_o, cc, t == 0);
+        if (leader)
+          for (int q = 0; q < kBwdChunksPerHand; ++q)
+            bwd_issue_ts_chunk<D>(acc, a_tm, b_lo, idesc_o, hh * kBwdChunksPerHand + q, t == 0);
         __syncwarp();
       }
       return true;
@@ -358,7 +369,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_chunk0 + 8 * cc);
+        if (lane == 0 && (cc + 1) % kBwdChunksPerHand == 0)
+          mbar_arrive(p_chunk0 + 8 * (cc / kBwdChunksPerHand));
       }
       // ---- phase 2: dS^T = P^T (dP^T - D)
       if (!mbar_wait_warp(dp_full, static_cast<uint32_t>(t & 1), abort_flag, p.err,
@@ -384,7 +396,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(ds_chunk0 + 8 * cc);
+        if (lane == 0 && (cc + 1) % kBwdChunksPerHand == 0)
+          mbar_arrive(ds_chunk0 + 8 * (cc / kBwdChunksPerHand));
       }
     }
     if (ok && mbar_wait_warp(acc_done, 0, abort_flag, p.err, kSiteAttnSoftmax)) {
@@ -560,16 +573,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               issue_dp(0) && (n_kv < 2 || issue_s(1));
     for (int j = 0; j < n_kv && ok; ++j) {
       // dQ += dS_j K_j, 32 key columns at a time as they are handed over
-      for (int cc = 0; cc < 4; ++cc) {
-        if (!mbar_wait_warp(ds_chunk0 + 8 * cc, static_cast<uint32_t>(j & 1), abort_flag, p.err,
+      for (int hh = 0; hh < kBwdHandovers; ++hh) {
+        if (!mbar_wait_warp(ds_chunk0 + 8 * hh, static_cast<uint32_t>(j & 1), abort_flag, p.err,
                             kSiteAttnMma)) {
           ok = false;
           break;
         }
         tc_fence_after();
         if (leader)
-          bwd_issue_ts_chunk<D>(tmem + C::TQ_A, tmem + C::TQ_DP, sdesc_lo(k_slot(j), C::CHUNK),
-                                idesc_o, cc, j == 0);
+          for (int q = 0; q < kBwdChunksPerHand; ++q)
+            bwd_issue_ts_chunk<D>(tmem + C::TQ_A, tmem + C::TQ_DP, sdesc_lo(k_slot(j), C::CHUNK),
+                                  idesc_o, hh * kBwdChunksPerHand + q, j == 0);
         __syncwarp();
       }
       if (!ok) break;
@@ -669,7 +683,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(ds_chunk0 + 8 * cc);
+        if (lane == 0 && (cc + 1) % kBwdChunksPerHand == 0)
+          mbar_arrive(ds_chunk0 + 8 * (cc / kBwdChunksPerHand));
       }
     }
     if (ok && mbar_wait_warp(acc_done, 0, abort_flag, p.err, kSiteAttnSoftmax)) {
