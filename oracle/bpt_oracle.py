@@ -34,7 +34,7 @@ value up to rounding order):
 6. H = GELU(Vn W_1 + b_1), GELU(z) = z/2 (1 + erf(z / sqrt 2))
 7. Z = Y + H W_2 + b_2
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 LayerNorm epsilon 1e-5 inside the square root, biased variance; exact erf
 GELU; heads are contiguous column slices concatenated in head order; the
 causal mask keeps the diagonal (j <= i); Q/K/V/O carry no bias.

@@ -21,7 +21,7 @@ What is computed, per batch element and head t, with blocks of b rows
   row p's attention = softmax over the allowed keys of the kept blocks only,
                 times their values.
 
-Readings (listed in the design doc): a pruned block is left out of the softmax
+Readings where the page is silent: a pruned block is left out of the softmax
 as well as the value product (the page skips the block after the gate, so it
 enters neither the normaliser nor the output); the diagonal block is never
 gated (the page gates off-diagonal blocks); without a causal mask every
