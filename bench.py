@@ -45,8 +45,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # digest covers the attention kernel, the shared device helpers and the host
 # launch code; after any change the bench reports null until it is retaken.
 ATTN_TRAFFIC = {
-    # 12 launches (6 forwards x 2 waves): waves of 406 + 114 and 1295 + 128 MB
-    "long_n64k": {"digest": "a046c820ae04ea4f", "bytes_per_launch": 971326165},
+    # 12 launches (6 forwards x 2 waves): waves of 405 + 114 and 1286 + 127 MB
+    "long_n64k": {"digest": "959c59fdb1694afd", "bytes_per_launch": 966207189},
 }
 TRAFFIC_SOURCES = ("blockwise_attn_ffn_b200/csrc/attn_pair_tc.cuh",
                    "blockwise_attn_ffn_b200/csrc/common.cuh",

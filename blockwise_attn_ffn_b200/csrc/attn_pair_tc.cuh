@@ -74,6 +74,23 @@ struct AttnPairParams {
 };
 
 
+#ifndef BPT_FWD_HANDOVERS_DK128
+#define BPT_FWD_HANDOVERS_DK128 2
+#endif
+#ifndef BPT_FWD_HANDOVERS_DK64
+#define BPT_FWD_HANDOVERS_DK64 4
+#endif
+// P hand-overs per 128-key tile from a softmax warpgroup to the UMMA warp
+// (4: every 32 keys; 2: every 64).  Measured: every 64 keys is faster at
+// d_k = 128 (each wait costs the UMMA warp ~100 clocks), every 32 at d_k =
+// 64 (shorter PV products, earlier overlap matters more).
+template <int D>
+constexpr int fwd_handovers() {
+  return D == 128 ? BPT_FWD_HANDOVERS_DK128 : BPT_FWD_HANDOVERS_DK64;
+}
+static_assert(BPT_FWD_HANDOVERS_DK128 == 2 || BPT_FWD_HANDOVERS_DK128 == 4, "2 or 4");
+static_assert(BPT_FWD_HANDOVERS_DK64 == 2 || BPT_FWD_HANDOVERS_DK64 == 4, "2 or 4");
+
 template <int D, int EMU>
 struct AttnPairCfg {
   static constexpr int BQ = 128;
@@ -181,6 +198,8 @@ template <int D, int EMU, bool GATE = false>
 __global__ void __launch_bounds__(384, 1)
     attn_pair_tc_kernel(const __grid_constant__ CUtensorMap mapQKV, const AttnPairParams p) {
   using C = AttnPairCfg<D, EMU>;
+  constexpr int kFwdHandovers = fwd_handovers<D>();
+  constexpr int kFwdChunksPerHand = 4 / kFwdHandovers;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -367,23 +386,25 @@ __global__ void __launch_bounds__(384, 1)
         if (j >= nX) continue;
         const uint32_t tS = tmem + (x == 0 ? 0u : C::TM_S_B);
         const uint32_t tO = tmem + (x == 0 ? C::TM_O_A : C::TM_O_B);
-        // PV_X(j) 32 keys at a time, each chunk as soon as its P is stored
+        // PV_X(j) as the P hand-overs come (each 128 / kFwdHandovers keys)
         bool kept = true;
-        for (int c = 0; c < 4; ++c) {
-          // A pruned block hands all four chunks over at once, after S_X(j)
-          // was read in full: its first hand-over is all the UMMA warp needs.
+        for (int hh = 0; hh < kFwdHandovers; ++hh) {
+          // A pruned block hands everything over at once, after S_X(j) was
+          // read in full: its first hand-over is all the UMMA warp needs.
           // (The skipped phases complete regardless; the next block's waits,
           // one phase later, are unaffected.)
-          if (GATE && c > 0 && !kept) continue;
-          if (!mbar_wait_warp(p_chunk0 + 8 * (4 * x + c), pph[x], abort_flag, p.err,
+          if (GATE && hh > 0 && !kept) continue;
+          if (!mbar_wait_warp(p_chunk0 + 8 * (4 * x + hh), pph[x], abort_flag, p.err,
                               kSiteAttnMma)) {
             ok = false;
             break;
           }
           tc_fence_after();
           // (the tile's decision was written before its first P hand-over)
-          if (c == 0) kept = !GATE || *reinterpret_cast<volatile int*>(&gate_keep[x]) != 0;
-          if (kept) issue_pv_chunk(tS, v_lo, tO, c, !o_started[x]);
+          if (hh == 0) kept = !GATE || *reinterpret_cast<volatile int*>(&gate_keep[x]) != 0;
+          if (kept)
+            for (int q = 0; q < kFwdChunksPerHand; ++q)
+              issue_pv_chunk(tS, v_lo, tO, hh * kFwdChunksPerHand + q, !o_started[x]);
         }
         if (!ok) break;
         pph[x] ^= 1u;
@@ -570,7 +591,8 @@ __global__ void __launch_bounds__(384, 1)
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_chunk + 8 * cc);
+            if (lane == 0 && (cc + 1) % kFwdChunksPerHand == 0)
+              mbar_arrive(p_chunk + 8 * (cc / kFwdChunksPerHand));
           }
         };
         if (masked || emu_group_mask(EMU) == 0u)
@@ -587,7 +609,7 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0)
-          for (int cc = 0; cc < 4; ++cc) mbar_arrive(p_chunk + 8 * cc);
+          for (int hh = 0; hh < kFwdHandovers; ++hh) mbar_arrive(p_chunk + 8 * hh);
       }  // keep_blk
     }
     if (ok && mbar_wait_fast(o_done, 0, abort_flag, p.err, kSiteAttnSoftmax)) {
