@@ -178,3 +178,51 @@ def test_bsfa_rejects_bad_gate_buffers():
 def test_bsfa_empty_is_a_no_op():
     assert fwd_bsfa([None] * 13, B=0) == bpt.BPT_OK
     assert fwd_bsfa([None] * 13, N=0) == bpt.BPT_OK
+
+
+# ------------------------------------------------------------- backward ABI
+def bwd(ins, outs, ws_bytes=1 << 31, B=1, N=256, d=64, h=1, d_ff=256, causal=1, dtype=F32):
+    """ins: 14 fake pointers (x, ln1, W_Q..b_2, stats, dZ, workspace); outs: 11."""
+    return bpt.bpt_layer_backward(*ins[:13], B, N, d, h, d_ff, causal, dtype, *outs, ins[13],
+                                  ws_bytes, None)
+
+
+BWD_IN = [0x10000000 + i * 0x1000000 for i in range(13)] + [0x80000000]
+BWD_OUT = [0x30000000 + i * 0x1000000 for i in range(11)]
+
+
+@pytest.mark.parametrize("dtype", [BF, F32])
+def test_backward_workspace_size_for_both_dtypes(dtype):
+    st, small_ws = bpt.bpt_layer_backward_workspace_size(1, 256, 256, 2, 512, 1, dtype)
+    assert st == bpt.BPT_OK and small_ws > 0
+    st, big_ws = bpt.bpt_layer_backward_workspace_size(1, 4096, 256, 2, 512, 1, dtype)
+    assert st == bpt.BPT_OK and big_ws > small_ws
+    assert bpt.bpt_layer_backward_workspace_size(1, 256, 100, 3, 512, 1, dtype)[0] == \
+        bpt.BPT_ERR_INVALID_ARG
+
+
+def test_backward_rejects_bad_pointers_and_small_workspace():
+    for i in range(14):
+        ins = list(BWD_IN)
+        ins[i] = None
+        assert bwd(ins, BWD_OUT) == bpt.BPT_ERR_INVALID_ARG, i
+    for i in range(11):
+        outs = list(BWD_OUT)
+        outs[i] = None
+        assert bwd(BWD_IN, outs) == bpt.BPT_ERR_INVALID_ARG, i
+        outs = list(BWD_OUT)
+        outs[i] += 8
+        assert bwd(BWD_IN, outs) == bpt.BPT_ERR_INVALID_ARG, i
+    outs = list(BWD_OUT)
+    outs[1] = outs[0]  # two outputs overlap
+    assert bwd(BWD_IN, outs) == bpt.BPT_ERR_INVALID_ARG
+    outs = list(BWD_OUT)
+    outs[0] = BWD_IN[12]  # dx over dZ
+    assert bwd(BWD_IN, outs) == bpt.BPT_ERR_INVALID_ARG
+    for dtype in (BF, F32):
+        st, need = bpt.bpt_layer_backward_workspace_size(1, 256, 64, 1, 256, 1, dtype)
+        assert bwd(BWD_IN, BWD_OUT, ws_bytes=need - 1, dtype=dtype) == bpt.BPT_ERR_WORKSPACE
+
+
+def test_backward_empty_is_a_no_op():
+    assert bwd([None] * 14, [None] * 11, B=0) == bpt.BPT_OK
