@@ -173,7 +173,7 @@ def layer_backward(x: torch.Tensor, p: Dict[str, torch.Tensor], h: int, causal: 
                    stream: Optional[torch.cuda.Stream] = None):
     """Gradients via ``bpt_layer_backward``; returns (grads, workspace) with
     grads[name] fp32 for name in GRAD_SHAPES (ln1 / ln2 as [2, d]: d gamma;
-    d beta).  x and p as for ``layer_forward`` (bf16); stats from
+    d beta).  x and p as for ``layer_forward`` (bf16 or fp32); stats from
     ``layer_forward_train``; dZ [B, N, d] fp32."""
     if x.dim() != 3:
         raise ValueError("x must be [B, N, d]")
