@@ -18,7 +18,7 @@
 //       being computed, then dS^T once dP^T is done; P^T stays in registers
 //       (fp16 pairs) in between.  The UMMA warp issues
 //         S_0, dP_0, then per block t: dV_t, S_t+1, dK_t, dP_t+1,
-//       each gradient product 32 query columns at a time as they are handed
+//       each gradient product 64 query columns at a time as they are handed
 //       over, and S_t+1 as soon as S_t has been read.  At the end dK, dV are
 //       added into the fp32 gradients (waves run in stream order, so each
 //       key row is updated by one CTA at a time).
@@ -171,8 +171,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t ring_empty0 = smem_u32(bars + 1 + C::NSLOT);
   const uint32_t s_full = smem_u32(bars + 1 + 2 * C::NSLOT);
   const uint32_t dp_full = smem_u32(bars + 2 + 2 * C::NSLOT);
-  const uint32_t p_chunk0 = smem_u32(bars + 3 + 2 * C::NSLOT);   // [4]: P^T columns 32c..
-  const uint32_t ds_chunk0 = smem_u32(bars + 7 + 2 * C::NSLOT);  // [4]: dS^T columns 32c..
+  const uint32_t p_chunk0 = smem_u32(bars + 3 + 2 * C::NSLOT);   // [kBwdHandovers]: P^T
+  const uint32_t ds_chunk0 = smem_u32(bars + 7 + 2 * C::NSLOT);  // [kBwdHandovers]: dS^T
   const uint32_t acc_done = smem_u32(bars + 11 + 2 * C::NSLOT);
   const uint32_t drain = smem_u32(bars + 12 + 2 * C::NSLOT);
   __shared__ uint32_t tmem_base_sh;
@@ -275,8 +275,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       __syncwarp();
       commit(dp_full);
     };
-    // one gradient product, 32 query columns at a time as the elementwise
-    // warps hand them over on chunk barriers cb[0..3]
+    // one gradient product, 128 / kBwdHandovers query columns at a time as
+    // the elementwise warps hand them over on barriers cb[0 .. kBwdHandovers)
     auto issue_grad = [&](int t, uint32_t cb, uint32_t acc, uint32_t a_tm, uint32_t b_lo) {
       for (int hh = 0; hh < kBwdHandovers; ++hh) {
         if (!mbar_wait_warp(cb + 8 * hh, static_cast<uint32_t>(t & 1), abort_flag, p.err,
@@ -451,7 +451,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t s_full0 = smem_u32(bars + 11);  // [2]: S_j landed in buffer j % 2
   const uint32_t s_free0 = smem_u32(bars + 13);  // [2]: buffer j % 2 read by every warp
   const uint32_t dp_full = smem_u32(bars + 15);
-  const uint32_t ds_chunk0 = smem_u32(bars + 16);  // [4]: dS columns 32c.. handed over
+  const uint32_t ds_chunk0 = smem_u32(bars + 16);  // [kBwdHandovers]: dS column groups
   const uint32_t acc_done = smem_u32(bars + 20);
   const uint32_t drain = smem_u32(bars + 21);
   __shared__ uint32_t tmem_base_sh;
@@ -572,7 +572,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool ok = mbar_wait_warp(q_full, 0, abort_flag, p.err, kSiteAttnMma) && issue_s(0) &&
               issue_dp(0) && (n_kv < 2 || issue_s(1));
     for (int j = 0; j < n_kv && ok; ++j) {
-      // dQ += dS_j K_j, 32 key columns at a time as they are handed over
+      // dQ += dS_j K_j, 128 / kBwdHandovers key columns at a time as handed over
       for (int hh = 0; hh < kBwdHandovers; ++hh) {
         if (!mbar_wait_warp(ds_chunk0 + 8 * hh, static_cast<uint32_t>(j & 1), abort_flag, p.err,
                             kSiteAttnMma)) {
