@@ -293,6 +293,57 @@ def test_single_token_attention_is_V():
     np.testing.assert_allclose(it["O"], it["V"], rtol=1e-15, atol=0)
 
 
+# ------------------------------------------------- every intermediate ----
+def torch_intermediates(inp, h, causal, b):
+    """Steps 1-7 of batch element b, each formed from torch float64 library
+    routines (layer_norm, matmul, scaled_dot_product_attention, gelu)."""
+    T = lambda k: torch.from_numpy(np.asarray(inp[k], np.float64))
+    X = T("x")[b]
+    N, d = X.shape
+    d_k = d // h
+    U = F.layer_norm(X, (d,), T("gamma1"), T("beta1"), eps=1e-5)
+    Q, K, V = U @ T("W_Q"), U @ T("W_K"), U @ T("W_V")
+    heads = lambda A: A.reshape(N, h, d_k).transpose(0, 1)
+    O = F.scaled_dot_product_attention(heads(Q), heads(K), heads(V), is_causal=causal)
+    O = O.transpose(0, 1).reshape(N, d)
+    Y = X + O @ T("W_O")
+    Vn = F.layer_norm(Y, (d,), T("gamma2"), T("beta2"), eps=1e-5)
+    Hpre = Vn @ T("W_1") + T("b_1")
+    H = F.gelu(Hpre)
+    Z = Y + H @ T("W_2") + T("b_2")
+    return {k: v.numpy() for k, v in dict(U=U, Q=Q, K=K, V=V, O=O, Y=Y, Vn=Vn, Hpre=Hpre,
+                                          H=H, Z=Z).items()}
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("b", [0, 1])
+def test_layer_intermediates_vs_torch_library(causal, b):
+    """Every intermediate (the oracle the GPU's Q/K/V are compared with) equals
+    the torch float64 library composition, with non-zero biases and LN
+    parameters away from (1, 0), so a swapped weight, a swapped LN parameter
+    or a dropped bias changes some key by far more than the tolerance."""
+    cfg, inp = tiny(N=37, d=32, h=4, d_ff=96, causal=causal, bias=0.5, ln=0.4)
+    got = oracle.layer_intermediates(inp, cfg.h, causal, b=b)
+    want = torch_intermediates(inp, cfg.h, causal, b)
+    assert sorted(got) == sorted(want)
+    for k in want:
+        np.testing.assert_allclose(got[k], want[k], rtol=1e-11, atol=1e-11, err_msg=k)
+    # and the last step is the oracle's plain definition of the layer
+    np.testing.assert_allclose(got["Z"], oracle.layer_unfused(inp, cfg.h, causal)[b],
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_layer_intermediates_distinguish_the_projections():
+    """Guards the comparison above against a fixture in which the three
+    projections (or the two LayerNorms) would coincide."""
+    cfg, inp = tiny(N=9, d=16, h=2, d_ff=32, bias=0.5, ln=0.4)
+    it = oracle.layer_intermediates(inp, cfg.h, True)
+    for a, c in (("Q", "K"), ("K", "V"), ("Q", "V")):
+        assert np.abs(it[a] - it[c]).max() > 0.1
+    assert np.abs(inp["gamma1"] - inp["gamma2"]).max() > 0.1
+    assert np.abs(inp["b_1"]).max() > 0.1
+
+
 # -------------------------------------------------------- sampled rows ----
 @pytest.mark.parametrize("causal", [False, True])
 def test_layer_rows_equals_full_layer_small(causal):
