@@ -333,6 +333,129 @@ def run_reference(args, cfg, rank, world):
 
 
 # ------------------------------------------------------------------ main --
+# ----------------------------------------------------------- forward timing --
+def time_forward(bpt, cfg, x, p, opts, steps, warmup, stream, dev, dist, world, out=None,
+                 ws=None, profile=True, per_step_events=True):
+    """Times `steps` forwards (after `warmup`) with CUDA events on the
+    launching stream, max over ranks.  Returns a dict with the step time, the
+    per-step times, the per-kernel CUDA-event times and the buffers used."""
+    import torch
+    from blockwise_attn_ffn_b200 import dist as bdist
+    out, ws = bpt.layer_forward(x, p, cfg.h, cfg.causal, out=out, workspace=ws, opts=opts)
+    torch.cuda.synchronize(dev)
+    st, site = bpt.bpt_read_device_error(ws.data_ptr(), stream.cuda_stream)
+    if st != bpt.BPT_OK:
+        raise SystemExit(f"device error {bpt.status_string(st)} site {site}")
+    for _ in range(warmup):
+        bpt.layer_forward(x, p, cfg.h, cfg.causal, out=out, workspace=ws, opts=opts)
+    torch.cuda.synchronize(dev)
+    bpt.bpt_profile_read()  # clear
+    bpt.bpt_profile_enable(profile)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1 if per_step_events else 2)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    ev[0].record(stream)
+    for i in range(steps):
+        bpt.layer_forward(x, p, cfg.h, cfg.causal, out=out, workspace=ws, opts=opts)
+        if per_step_events:
+            ev[i + 1].record(stream)
+    if not per_step_events:
+        ev[1].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    bpt.bpt_profile_enable(False)
+    _, kind_ms, kind_n = bpt.bpt_profile_read()
+    st, site = bpt.bpt_read_device_error(ws.data_ptr(), stream.cuda_stream)
+    if st != bpt.BPT_OK:
+        raise SystemExit(f"device error {bpt.status_string(st)} site {site}")
+    ms_total = bdist.max_over_ranks(ev[0].elapsed_time(ev[-1]), dist, dev)
+    per_step = ([ev[i].elapsed_time(ev[i + 1]) for i in range(steps)] if per_step_events
+                else [ms_total / steps])
+    return {"ms_step": ms_total / steps, "per_step": per_step, "kind_ms": kind_ms,
+            "kind_n": kind_n, "out": out, "ws": ws}
+
+
+def kernel_table(kind_ms, kind_n, steps, flops):
+    """Per-kernel CUDA-event time per step, share and TFLOP/s."""
+    total = sum(kind_ms.values())
+    flop_kind = {"qkv": flops["qkv"], "attn": flops["attention"], "wo": flops["wo"],
+                 "w1": flops["ffn"] / 2, "w2": flops["ffn"] / 2,
+                 "tail": flops["wo"] + flops["ffn"]}
+    table = {}
+    for k, ms in kind_ms.items():
+        if kind_n.get(k, 0) == 0:
+            continue
+        e = {"ms_per_step": ms / steps, "launches_per_step": kind_n[k] / steps,
+             "share": ms / total if total else None}
+        if k in flop_kind and ms > 0:
+            e["tflops"] = flop_kind[k] / (ms / steps / 1e3) / 1e12
+        table[k] = e
+    return table
+
+
+def peak_bytes_above(dev, fn):
+    """Peak device bytes allocated by fn() above what is allocated before it."""
+    import torch
+    torch.cuda.synchronize(dev)
+    base = torch.cuda.memory_allocated(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+    keep = fn()
+    torch.cuda.synchronize(dev)
+    peak = torch.cuda.max_memory_allocated(dev) - base
+    del keep
+    return int(peak)
+
+
+def other_workloads(bpt, args, names, stream, dev, peaks):
+    """Each named workload timed on this GPU (fused schedule; waves as well
+    for bf16 layers): tokens/s, TFLOP/s and the fraction of the burst peak."""
+    import torch
+    res = {}
+    for name in names:
+        cfg = WORKLOADS[name]
+        inp = make_inputs(cfg)
+        p = bpt.to_device(inp, cfg.dtype, dev)
+        del inp
+        flops = accounting.layer_flops(cfg.B, cfg.N, cfg.d, cfg.h, cfg.d_ff, cfg.causal)
+        steps = max(3, min(args.steps, int(2000.0 / max(1.0, flops["total"] / 1e12 * 1.2))))
+        entry = {"B": cfg.B, "N": cfg.N, "d": cfg.d, "h": cfg.h, "d_ff": cfg.d_ff,
+                 "dtype": cfg.dtype, "steps": steps, "flops_per_step": flops["total"]}
+        schedules = ["fused", "waves"] if cfg.dtype == "bf16" else ["waves"]
+        for sched in schedules:
+            opts = bpt.make_options(schedule=sched)
+            r = time_forward(bpt, cfg, p["x"], p, opts, steps, 3, stream, dev, None, 1,
+                             profile=True, per_step_events=False)
+            tf = flops["total"] / (r["ms_step"] / 1e3) / 1e12
+            entry[sched] = {"ms_per_step": r["ms_step"],
+                            "tokens_per_s": cfg.B * cfg.N / (r["ms_step"] / 1e3),
+                            "tflops": tf, "pct_bf16_peak": tf / peaks["bf16_tflops"],
+                            "kernels": kernel_table(r["kind_ms"], r["kind_n"], steps, flops)}
+            del r
+        if cfg.dtype == "f32":
+            entry["note"] = "fp32 layer on the CUDA cores (FFMA); % of the bf16 tensor peak " \
+                            "for reference only"
+        res[name] = entry
+        del p
+        torch.cuda.empty_cache()
+    return res
+
+
+def relaunch_under_torchrun(args) -> int:
+    """`bench.py --gpus N` started as a plain process: start the N ranks
+    ourselves (one process per GPU) with the same arguments."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={args.gpus}", "--master-addr=127.0.0.1",
+           f"--master-port={port}", os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
+# ------------------------------------------------------------------ main --
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -355,14 +478,23 @@ def main():
                     help="skip the gated-attention (BSFA) forward measurement")
     ap.add_argument("--bsfa-k", type=int, default=32,
                     help="off-diagonal key blocks kept per query block by the BSFA thresholds")
+    ap.add_argument("--schedule", default="fused", choices=["fused", "waves"],
+                    help="layer body after attention: one persistent per-block kernel "
+                         "(fused) or wave-level kernels (waves)")
     ap.add_argument("--attn-qpc", type=int, default=2, choices=[1, 2],
                     help="query blocks per attention CTA (2: paired, 256 query rows per "
                          "K/V tile; 1: one 128-row block)")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip timing the other four workloads")
+    ap.add_argument("--no-alt-schedule", action="store_true",
+                    help="skip timing the other schedule on the bench workload")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
 
     from blockwise_attn_ffn_b200 import dist as bdist
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return relaunch_under_torchrun(args)
     rank, local_rank, world = bdist.env_rank()
     cfg = WORKLOADS[args.workload]
     if args.seq_len:
@@ -381,65 +513,62 @@ def main():
     dev = torch.device("cuda", local_rank)
     if world > 1:
         bdist.init_process_group("nccl", device=dev)
+    stream = torch.cuda.current_stream(dev)
 
     # Inputs: the workload's weights on every rank, a rank-seeded x each.
     inp = bdist.rank_inputs(cfg, rank)
-    torch.cuda.reset_peak_memory_stats(dev)
-    base_mem = torch.cuda.memory_allocated(dev)
     p = bpt.to_device(inp, cfg.dtype, dev)
     x_host = None
     if not args.no_e2e:
         x_host = bpt.to_device(inp, cfg.dtype, dev, pin_x=True)["x"]
     del inp
     x = p["x"]
-    if bpt.bpt_debug_set_attn_qpc(args.attn_qpc) != bpt.BPT_OK:
-        raise SystemExit("bpt_debug_set_attn_qpc failed")
-    out, ws = bpt.layer_forward(x, p, cfg.h, cfg.causal)
-    torch.cuda.synchronize(dev)
-    stream = torch.cuda.current_stream(dev)
-    st, site = bpt.bpt_read_device_error(ws.data_ptr(), stream.cuda_stream)
-    if st != bpt.BPT_OK:
-        raise SystemExit(f"device error {bpt.status_string(st)} site {site}")
-    peak_fused = torch.cuda.max_memory_allocated(dev) - base_mem
+    opts = bpt.make_options(schedule=args.schedule, attn_qpc=args.attn_qpc)
+    alt_sched = "waves" if args.schedule == "fused" else "fused"
+    alt_opts = bpt.make_options(schedule=alt_sched, attn_qpc=args.attn_qpc)
 
-    for _ in range(args.warmup):
-        bpt.layer_forward(x, p, cfg.h, cfg.causal, out=out, workspace=ws)
-    torch.cuda.synchronize(dev)
+    # Peak device bytes above the resident inputs (x and the parameters), for
+    # each schedule: out + workspace of one forward.
+    inputs_bytes = int(torch.cuda.memory_allocated(dev))
+
+    def one_forward(o):
+        def run():
+            r = bpt.layer_forward(x, p, cfg.h, cfg.causal, opts=o)
+            torch.cuda.synchronize(dev)
+            return r
+        return run
+    peak_main = peak_bytes_above(dev, one_forward(opts))
+    peak_alt = peak_bytes_above(dev, one_forward(alt_opts)) if cfg.dtype == "bf16" else None
+    torch.cuda.empty_cache()
 
     flops = accounting.layer_flops(cfg.B, cfg.N, cfg.d, cfg.h, cfg.d_ff, cfg.causal)
-    _, launches_per_step = bpt.bpt_layer_launch_count(cfg.B, cfg.N, cfg.d, cfg.h, cfg.d_ff,
-                                                      cfg.causal, bpt.BPT_BF16 if cfg.dtype == "bf16" else bpt.BPT_F32)
+    code = bpt.BPT_BF16 if cfg.dtype == "bf16" else bpt.BPT_F32
+    _, launches_per_step = bpt.bpt_layer_launch_count_opt(cfg.B, cfg.N, cfg.d, cfg.h, cfg.d_ff,
+                                                          cfg.causal, code, opts)
 
     # -------- timed region (device time, CUDA events on the launching stream)
-    bpt.bpt_profile_read()  # clear
-    bpt.bpt_profile_enable(True)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clk:
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize(dev)
-        step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps - 1)]
-        ev0.record(stream)
-        for i in range(args.steps):
-            bpt.layer_forward(x, p, cfg.h, cfg.causal, out=out, workspace=ws)
-            if i + 1 < args.steps:
-                step_ev[i].record(stream)
-        ev1.record(stream)
-        torch.cuda.synchronize(dev)
-        if world > 1:
-            dist.barrier()
-    bpt.bpt_profile_enable(False)
-    ms_total = ev0.elapsed_time(ev1)
-    marks = [ev0] + step_ev + [ev1]
-    per_step = [marks[i].elapsed_time(marks[i + 1]) for i in range(args.steps)]
-    _, kind_ms, kind_n = bpt.bpt_profile_read()
-    st, site = bpt.bpt_read_device_error(ws.data_ptr(), stream.cuda_stream)
-    if st != bpt.BPT_OK:
-        raise SystemExit(f"device error {bpt.status_string(st)} site {site}")
-    ms_total = bdist.max_over_ranks(ms_total, dist, dev)
-    ms_step = ms_total / args.steps
+        main_r = time_forward(bpt, cfg, x, p, opts, args.steps, args.warmup, stream, dev, dist,
+                              world)
+    out, ws = main_r["out"], main_r["ws"]
+    ms_step = main_r["ms_step"]
+    per_step = main_r["per_step"]
+    kind_ms, kind_n = main_r["kind_ms"], main_r["kind_n"]
     tokens_step = cfg.B * cfg.N * world
     value = bdist.weak_scaling_tokens_per_s(cfg, world, ms_step)
+
+    # -------- the other schedule, same workload (no clock record: context)
+    alt = None
+    if not args.no_alt_schedule and cfg.dtype == "bf16":
+        r = time_forward(bpt, cfg, x, p, alt_opts, max(3, args.steps // 2), args.warmup, stream,
+                         dev, dist, world)
+        alt = {"schedule": alt_sched, "ms_per_step": r["ms_step"],
+               "tokens_per_s": bdist.weak_scaling_tokens_per_s(cfg, world, r["ms_step"]),
+               "tflops": flops["total"] * world / (r["ms_step"] / 1e3) / 1e12,
+               "kernels": kernel_table(r["kind_ms"], r["kind_n"], max(3, args.steps // 2), flops),
+               "peak_bytes_above_inputs": peak_alt}
+        del r
+        torch.cuda.empty_cache()
 
     # -------- end to end: pinned x -> device, forward, out -> pinned host,
     # every step.  The copies run on their own streams with double-buffered
@@ -469,7 +598,7 @@ def main():
                 if out_free[b] is not None:
                     stream.wait_event(out_free[b])
                 bpt.layer_forward(xs[b], p, cfg.h, cfg.causal, out=outs[b], workspace=ws,
-                                  stream=stream)
+                                  stream=stream, opts=opts)
                 done = torch.cuda.Event()
                 done.record(stream)
                 in_free[b] = done
@@ -509,16 +638,9 @@ def main():
     attn_flops_launch = flops["attention"] * args.steps / n_attn
     achieved = attn_flops_launch / (attn_ms_launch / 1e3) / 1e12
     attn_bytes_launch = accounting.attention_bytes(cfg.B, cfg.N, cfg.d, cfg.h) * args.steps / n_attn
+    peak_burst = peaks["bf16_tflops"]
     peak_sus = peaks["bf16_tflops_sustained"]
-    total_kernel_ms = sum(kind_ms.values())
-    kernels = {k: {"ms_per_step": kind_ms[k] / args.steps, "launches_per_step": kind_n[k] / args.steps,
-                   "share": kind_ms[k] / total_kernel_ms if total_kernel_ms else None}
-               for k in kind_ms}
-    flop_kind = {"qkv": flops["qkv"], "attn": flops["attention"], "wo": flops["wo"],
-                 "w1": flops["ffn"] / 2, "w2": flops["ffn"] / 2}
-    for k, f in flop_kind.items():
-        ms = kind_ms[k] / args.steps
-        kernels[k]["tflops"] = f / (ms / 1e3) / 1e12 if ms > 0 else None
+    kernels = kernel_table(kind_ms, kind_n, args.steps, flops)
     tflops = flops["total"] * world / (ms_step / 1e3) / 1e12
     # Step a1+a2 (LN1 + QKV projection): x, W_Q|W_K|W_V and QKV touched once.
     esz_in = 2 if cfg.dtype == "bf16" else 4
@@ -537,9 +659,10 @@ def main():
                        "exactly each call), fp32 accumulation, fp32 residual stream and output")
         if cfg.dtype == "bf16" else "fp32 throughout (CUDA cores)",
         "data": "synthetic: seeded N(0,1) x, N(0,1/fan_in) weights, LN gamma~1+0.1N, beta~0.1N",
-        "config": dict(workload_config(cfg, world), attn_query_blocks_per_cta=args.attn_qpc),
+        "config": dict(workload_config(cfg, world), attn_query_blocks_per_cta=args.attn_qpc,
+                       schedule=args.schedule),
         "tflops": tflops,
-        "pct_bf16_peak": tflops / world / peaks["bf16_tflops"],
+        "pct_bf16_peak": tflops / world / peak_burst,
         "pct_bf16_peak_sustained": tflops / world / peak_sus,
         "pct_nominal_2250": tflops / world / 2250.0,
         "ms_per_step_median": float(np.median(per_step)),
@@ -550,28 +673,43 @@ def main():
                     "note": "LN1 + QKV projection kernels: x + W_QKV + QKV once / their time"},
         "peak_src": peak_src,
         "roofline": {"bound": "tensor", "kernel": "attn_pair_tc_kernel", "achieved": achieved,
-                     "peak": peak_sus, "unit": "TFLOP/s", "frac": achieved / peak_sus,
-                     "peak_kind": f"bf16_tflops_sustained ({peak_src})",
-                     "frac_of_burst": achieved / peaks["bf16_tflops"],
+                     "peak": peak_burst, "unit": "TFLOP/s", "frac": achieved / peak_burst,
+                     "peak_kind": f"bf16_tflops burst ({peak_src}); fp16 operands, same "
+                                  "dense rate",
+                     "frac_of_sustained": achieved / peak_sus,
                      "traffic": attn_traffic(cfg.name),
                      "traffic_unit": "bytes per launch (ncu dram read + write)",
                      "algorithmic_bytes_per_launch": attn_bytes_launch},
         "kernels": kernels,
-        "peak_bytes": {"fused_device_total": int(peak_fused),
-                       "unfused_activations_analytic": int(cfg.B * unfused["total"] * esz),
-                       "unfused_ffn_hidden_analytic": int(cfg.B * unfused["ffn_hidden"] * esz)},
+        "alt_schedule": alt,
+        "peak_bytes": {
+            "base": "bytes allocated above the resident inputs (x and the parameters) during "
+                    "one forward: out + workspace for the library; every activation for the "
+                    "unfused torch schedule",
+            "inputs_resident": inputs_bytes,
+            args.schedule: int(peak_main),
+            alt_sched: peak_alt,
+            "unfused_activations_analytic": int(cfg.B * unfused["total"] * esz),
+            "unfused_ffn_hidden_analytic": int(cfg.B * unfused["ffn_hidden"] * esz)},
         "gpu_launches": int(launches_per_step * args.steps),
         "e2e": e2e,
     }
-    with_clk = clk.summary()
-    line["clocks"] = with_clk
+    line["clocks"] = clk.summary()
     if not args.no_backward and cfg.dtype == "bf16":
         line["backward"] = measure_backward(bpt, cfg, x, p, stream, dev, args, flops, world,
                                             peaks, dist)
     if not args.no_bsfa and cfg.dtype == "bf16":
         line["bsfa"] = measure_bsfa(bpt, cfg, x, p, out, ms_step, stream, dev, args, world, dist)
     if not args.no_unfused_peak and cfg.dtype == "bf16":
+        del out, ws, main_r
+        torch.cuda.empty_cache()
         line["peak_bytes"]["unfused_torch_measured"] = unfused_torch_peak_bytes(cfg, p, dev)
+    if not args.no_other_workloads and world == 1 and args.seq_len is None:
+        del p, x
+        torch.cuda.empty_cache()
+        names = [n for n in ("tiny_f32", "gpt2s_n2k", "mid_n16k", "long_n64k", "wide_n128k")
+                 if n != cfg.name]
+        line["other_workloads"] = other_workloads(bpt, args, names, stream, dev, peaks)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_rate(cfg, args.cpu_rows)

@@ -7,9 +7,15 @@ call, the seeded input generator and the FLOP/byte accountant.
 """
 from ._lib import (  # noqa: F401
     BPT_BF16, BPT_ERR_CUDA, BPT_ERR_INVALID_ARG, BPT_ERR_RANGE, BPT_ERR_TIMEOUT, BPT_ERR_UNSUPPORTED,
-    BPT_ERR_WORKSPACE, BPT_F32, BPT_OK, BPT_STATIC_WORKSPACE_BYTES, BPT_WAVE_BLOCKS, EXPORTED, KINDS, LIB_PATH, BptError,
-    bpt_debug_inject_fault, bpt_debug_set_attn_qpc, bpt_debug_set_max_wave, bpt_layer_forward, bpt_layer_forward_bsfa, bpt_layer_forward_static, bpt_layer_forward_train, bpt_layer_backward, bpt_layer_backward_workspace_size, bpt_layer_launch_count, bpt_layer_workspace_size, bpt_profile_enable,
-    bpt_profile_read, bpt_read_device_error, bpt_status_string, load, status_string,
+    BPT_ERR_WORKSPACE, BPT_F32, BPT_OK, BPT_SCHEDULE_FUSED, BPT_SCHEDULE_WAVES,
+    BPT_STATIC_WORKSPACE_BYTES, BPT_TAIL_MAX_PAIRS, BPT_WAVE_BLOCKS, EXPORTED, KINDS, LIB_PATH,
+    BptError, Options, bpt_layer_backward, bpt_layer_backward_opt,
+    bpt_layer_backward_workspace_size, bpt_layer_backward_workspace_size_opt,
+    bpt_layer_forward, bpt_layer_forward_bsfa, bpt_layer_forward_bsfa_opt, bpt_layer_forward_opt,
+    bpt_layer_forward_static, bpt_layer_forward_train, bpt_layer_launch_count,
+    bpt_layer_launch_count_opt, bpt_layer_workspace_size, bpt_layer_workspace_size_opt,
+    bpt_profile_enable, bpt_profile_read, bpt_read_device_error, bpt_status_string, load,
+    make_options, status_string,
 )
 from .layer import (  # noqa: F401
     GRAD_SHAPES, PARAM_NAMES, layer_backward, layer_forward, layer_forward_bsfa,

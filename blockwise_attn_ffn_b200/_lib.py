@@ -18,19 +18,48 @@ LIB_PATH = os.path.join(HERE, "libbpt.so")
 BPT_OK, BPT_ERR_INVALID_ARG, BPT_ERR_UNSUPPORTED, BPT_ERR_WORKSPACE, BPT_ERR_CUDA, \
     BPT_ERR_TIMEOUT, BPT_ERR_RANGE = range(7)
 BPT_F32, BPT_BF16 = 0, 1
-KINDS = ["ln1", "qkv", "attn", "wo", "ln2", "w1", "w2", "cvt"]
+KINDS = ["ln1", "qkv", "attn", "wo", "ln2", "w1", "w2", "cvt", "tail"]
 BPT_WAVE_BLOCKS = 256
+BPT_TAIL_MAX_PAIRS = 74
+BPT_SCHEDULE_FUSED, BPT_SCHEDULE_WAVES = 0, 1
 BPT_STATIC_WORKSPACE_BYTES = 64 * 1024 * 1024
 
 EXPORTED = [
     "bpt_layer_workspace_size", "bpt_layer_forward", "bpt_read_device_error",
     "bpt_status_string", "bpt_profile_enable", "bpt_profile_read",
-    "bpt_layer_launch_count", "bpt_layer_forward_static", "bpt_debug_inject_fault",
+    "bpt_layer_launch_count", "bpt_layer_forward_static",
     "bpt_layer_forward_train", "bpt_layer_forward_bsfa", "bpt_layer_backward_workspace_size",
     "bpt_layer_backward",
-    "bpt_debug_set_max_wave",
-    "bpt_debug_set_attn_qpc",
+    "bpt_layer_workspace_size_opt", "bpt_layer_forward_opt", "bpt_layer_forward_bsfa_opt",
+    "bpt_layer_backward_workspace_size_opt", "bpt_layer_backward_opt",
+    "bpt_layer_launch_count_opt",
 ]
+
+
+class Options(ctypes.Structure):
+    """``bpt_options`` (include/bpt.h): per-call choices of the *_opt calls."""
+    _fields_ = [("schedule", ctypes.c_int32), ("attn_qpc", ctypes.c_int32),
+                ("max_wave", ctypes.c_int64), ("fault", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+def make_options(schedule=None, attn_qpc=0, max_wave=0, fault=0, reserved=0) -> Options:
+    """An ``Options`` value; ``schedule`` may be "fused", "waves" or the code."""
+    if schedule is None or schedule == "fused":
+        schedule = BPT_SCHEDULE_FUSED
+    elif schedule == "waves":
+        schedule = BPT_SCHEDULE_WAVES
+    return Options(int(schedule), int(attn_qpc), int(max_wave), int(fault), int(reserved))
+
+
+def _opts_ref(opts):
+    """None, an ``Options`` or a dict of its fields -> argument for a const
+    bpt_options* parameter."""
+    if opts is None:
+        return None
+    if isinstance(opts, dict):
+        opts = make_options(**opts)
+    return ctypes.byref(opts)
 
 _lib: Optional[ctypes.CDLL] = None
 
@@ -68,10 +97,26 @@ def load() -> ctypes.CDLL:
     lib.bpt_layer_backward.argtypes = ([vp] * 13 + [i64] * 5 + [i32, i32] + [vp] * 12 +
                                        [ctypes.c_size_t, vp])
     lib.bpt_layer_backward.restype = i32
-    lib.bpt_debug_set_max_wave.argtypes = [i64]
-    lib.bpt_debug_set_max_wave.restype = i32
-    lib.bpt_debug_set_attn_qpc.argtypes = [i32]
-    lib.bpt_debug_set_attn_qpc.restype = i32
+    op = ctypes.POINTER(Options)
+    lib.bpt_layer_workspace_size_opt.argtypes = [i64, i64, i64, i64, i64, i32, i32, op,
+                                                 ctypes.POINTER(ctypes.c_size_t)]
+    lib.bpt_layer_workspace_size_opt.restype = i32
+    lib.bpt_layer_forward_opt.argtypes = ([vp] * 11 + [i64] * 5 +
+                                          [i32, i32, vp, vp, vp, ctypes.c_size_t, op, vp])
+    lib.bpt_layer_forward_opt.restype = i32
+    lib.bpt_layer_forward_bsfa_opt.argtypes = ([vp] * 11 + [i64] * 5 +
+                                               [i32, i32, vp, vp, vp, vp, vp, ctypes.c_size_t,
+                                                op, vp])
+    lib.bpt_layer_forward_bsfa_opt.restype = i32
+    lib.bpt_layer_backward_workspace_size_opt.argtypes = [i64, i64, i64, i64, i64, i32, i32, op,
+                                                          ctypes.POINTER(ctypes.c_size_t)]
+    lib.bpt_layer_backward_workspace_size_opt.restype = i32
+    lib.bpt_layer_backward_opt.argtypes = ([vp] * 13 + [i64] * 5 + [i32, i32] + [vp] * 12 +
+                                           [ctypes.c_size_t, op, vp])
+    lib.bpt_layer_backward_opt.restype = i32
+    lib.bpt_layer_launch_count_opt.argtypes = [i64, i64, i64, i64, i64, i32, i32, op,
+                                               ctypes.POINTER(ctypes.c_int64)]
+    lib.bpt_layer_launch_count_opt.restype = i32
     lib.bpt_read_device_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     lib.bpt_read_device_error.restype = i32
     lib.bpt_status_string.argtypes = [i32]
@@ -86,8 +131,6 @@ def load() -> ctypes.CDLL:
     lib.bpt_layer_launch_count.restype = i32
     lib.bpt_layer_forward_static.argtypes = [vp] * 11 + [i64] * 5 + [i32, i32, vp, vp]
     lib.bpt_layer_forward_static.restype = i32
-    lib.bpt_debug_inject_fault.argtypes = [i32]
-    lib.bpt_debug_inject_fault.restype = i32
     _lib = lib
     return lib
 
@@ -102,6 +145,58 @@ def bpt_layer_workspace_size(B, N, d, h, d_ff, causal, dtype) -> Tuple[int, int]
     out = ctypes.c_size_t(0)
     st = load().bpt_layer_workspace_size(B, N, d, h, d_ff, int(bool(causal)), dtype,
                                          ctypes.byref(out))
+    return st, out.value
+
+
+def bpt_layer_workspace_size_opt(B, N, d, h, d_ff, causal, dtype, opts) -> Tuple[int, int]:
+    """Returns (status, bytes) for the given options (None, Options or dict)."""
+    out = ctypes.c_size_t(0)
+    st = load().bpt_layer_workspace_size_opt(B, N, d, h, d_ff, int(bool(causal)), dtype,
+                                             _opts_ref(opts), ctypes.byref(out))
+    return st, out.value
+
+
+def bpt_layer_forward_opt(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
+                          B, N, d, h, d_ff, causal, dtype, out, stats, workspace,
+                          workspace_bytes, opts, stream) -> int:
+    """Pointer-level call with options (stats may be None); returns the status."""
+    return load().bpt_layer_forward_opt(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
+                                        B, N, d, h, d_ff, int(bool(causal)), dtype, out, stats,
+                                        workspace, workspace_bytes, _opts_ref(opts), stream)
+
+
+def bpt_layer_forward_bsfa_opt(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
+                               B, N, d, h, d_ff, causal, dtype, thresholds, block_max, kept,
+                               out, workspace, workspace_bytes, opts, stream) -> int:
+    return load().bpt_layer_forward_bsfa_opt(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2,
+                                             b_2, B, N, d, h, d_ff, int(bool(causal)), dtype,
+                                             thresholds, block_max, kept, out, workspace,
+                                             workspace_bytes, _opts_ref(opts), stream)
+
+
+def bpt_layer_backward_workspace_size_opt(B, N, d, h, d_ff, causal, dtype,
+                                          opts) -> Tuple[int, int]:
+    out = ctypes.c_size_t(0)
+    st = load().bpt_layer_backward_workspace_size_opt(B, N, d, h, d_ff, int(bool(causal)),
+                                                      dtype, _opts_ref(opts), ctypes.byref(out))
+    return st, out.value
+
+
+def bpt_layer_backward_opt(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, stats, dZ,
+                           B, N, d, h, d_ff, causal, dtype, dx, d_ln1, dW_Q, dW_K, dW_V, dW_O,
+                           d_ln2, dW_1, db_1, dW_2, db_2, workspace, workspace_bytes, opts,
+                           stream) -> int:
+    return load().bpt_layer_backward_opt(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
+                                         stats, dZ, B, N, d, h, d_ff, int(bool(causal)), dtype,
+                                         dx, d_ln1, dW_Q, dW_K, dW_V, dW_O, d_ln2, dW_1, db_1,
+                                         dW_2, db_2, workspace, workspace_bytes,
+                                         _opts_ref(opts), stream)
+
+
+def bpt_layer_launch_count_opt(B, N, d, h, d_ff, causal, dtype, opts) -> Tuple[int, int]:
+    out = ctypes.c_int64(0)
+    st = load().bpt_layer_launch_count_opt(B, N, d, h, d_ff, int(bool(causal)), dtype,
+                                           _opts_ref(opts), ctypes.byref(out))
     return st, out.value
 
 
@@ -150,16 +245,9 @@ def bpt_layer_backward(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, stat
                                      workspace, workspace_bytes, stream)
 
 
-def bpt_debug_set_max_wave(blocks: int) -> int:
-    return load().bpt_debug_set_max_wave(blocks)
-
-
-def bpt_debug_set_attn_qpc(qpc: int) -> int:
-    return load().bpt_debug_set_attn_qpc(qpc)
-
-
 def bpt_read_device_error(workspace, stream) -> Tuple[int, int]:
-    """Returns (status, site)."""
+    """Returns (status, site); workspace None reads the header of the array
+    bpt_layer_forward_static uses."""
     site = ctypes.c_uint32(0)
     st = load().bpt_read_device_error(workspace, stream, ctypes.byref(site))
     return st, site.value
@@ -192,12 +280,6 @@ def bpt_layer_forward_static(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2
     return load().bpt_layer_forward_static(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
                                            B, N, d, h, d_ff, int(bool(causal)), dtype, out,
                                            stream)
-
-
-def bpt_debug_inject_fault(code: int) -> int:
-    """Test hook: the next bf16 forward loses one TMA load (1: QKV GEMM,
-    2: attention) so a bounded wait runs out and reports BPT_ERR_TIMEOUT."""
-    return load().bpt_debug_inject_fault(int(code))
 
 
 def bpt_layer_launch_count(B, N, d, h, d_ff, causal, dtype) -> Tuple[int, int]:

@@ -60,7 +60,13 @@ struct AttnPairParams {
   int seqs;    // >0: the wave is `seqs` whole sequences; 0: part of one sequence
   int hg;      // heads per group (divides h): CTAs run group by group, so the
                // K/V that concurrent CTAs sweep is that of hg heads only
-  __half* o;         // [count * 128, d] block scratch (fp16)
+  __half* o;         // output, fp16: o_tok = 0: [count * 128, o_ld] block
+                     // scratch in wave order; o_tok = 1: [B*N, o_ld] token
+                     // rows (the Q columns of the QKV buffer: each block's
+                     // output replaces its own queries; rows past N are not
+                     // written)
+  long long o_ld;    // row stride of o (elements)
+  int o_tok;
   float scale_log2;  // log2(e) / sqrt(d_k)
   float2* stats;     // nullable: per-row softmax statistics [B][h][N] (m, l)
   uint32_t* err;
@@ -626,13 +632,22 @@ __global__ void __launch_bounds__(384, 1)
           p.stats[(static_cast<long long>(bidx) * p.h + head) * p.N + pos] = make_float2(m_s, l_s);
         }
       }
-      const long long srow = static_cast<long long>(itemA + x - p.item0) * C::BQ + r;
-      __half* dst = p.o + srow * p.d + head * D;
+      long long orow;
+      bool store = true;
+      if (p.o_tok) {
+        const int pos = iX * C::BQ + r;
+        store = pos < p.N;
+        orow = static_cast<long long>(bidx) * p.N + pos;
+      } else {
+        orow = static_cast<long long>(itemA + x - p.item0) * C::BQ + r;
+      }
+      __half* dst = p.o + orow * p.o_ld + head * D;
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tO + cc * 32, v);
         tmem_ld_wait();
+        if (!store) continue;
         uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {

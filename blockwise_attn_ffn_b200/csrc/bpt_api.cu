@@ -4,15 +4,20 @@
 // Schedule ("Blockwise Parallel Transformer — BPT", sections "The fused
 // blockwise algorithm" and "Why parallel is in the name"): the outer loop over
 // query blocks is embarrassingly parallel, and P concurrent blocks cost
-// P x O(b d) of transient memory.  On this GPU one wave holds up to
-// BPT_WAVE_BLOCKS query blocks; per wave the loop body runs as five
-// stream-ordered kernels whose intermediates are wave-shaped:
-//   attention (online softmax over K/V blocks)  -> o      [P b, d]
+// P x O(b d) of transient memory.  Before the loop: the bf16 -> fp16 weight
+// copy, LN1 (into out, reused as scratch) and the QKV GEMM.  Then, for bf16
+// layers (the fused schedule, default):
+//   attention (online softmax over K/V blocks) -> o over each block's Q rows
+//   tail kernel: per query block, W_O + x, LN2, W_1 + b_1 + GELU chunk by
+//   chunk, W_2 + b_2 + y  (tail_tc.cuh; scratch per CTA pair)
+// or (the waves schedule, and fp32 layers) waves of up to BPT_WAVE_BLOCKS
+// query blocks, each running five stream-ordered kernels whose
+// intermediates are wave-shaped:
+//   attention                                   -> o      [P b, d]
 //   W_O GEMM, epilogue + x                      -> y      (into out rows)
 //   LN2                                         -> v      [P b, d]
 //   W_1 GEMM, epilogue + b_1, GELU              -> H      [P b, d_ff]
 //   W_2 GEMM, epilogue + b_2 + y                -> Z      (into out rows)
-// Before the waves: LN1 (into out, reused as scratch) and the QKV GEMM.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -33,6 +38,7 @@
 #include "gemm_tc.cuh"
 #include "rows.cuh"
 #include "simt_f32.cuh"
+#include "tail_tc.cuh"
 #include "backward_f32.cuh"
 
 namespace {
@@ -40,10 +46,31 @@ namespace {
 using bpt::RowMap;
 
 constexpr int64_t kMaxWave = BPT_WAVE_BLOCKS;
-// Query blocks per wave (test hook bpt_debug_set_max_wave lowers it).
-std::atomic<int64_t> g_max_wave{kMaxWave};
-// Query blocks per attention CTA: 2 (paired) unless bpt_debug_set_attn_qpc.
-std::atomic<int> g_attn_qpc{2};
+static_assert(BPT_TAIL_MAX_PAIRS == bpt::kTailMaxPairs, "tail pairs");
+
+// Per-call options (bpt_options), validated, defaults filled in.
+struct Opts {
+  int fused = 1;             // bf16 forward: fused tail (1) or waves (0)
+  int qpc = 2;               // query blocks per attention CTA
+  int64_t max_wave = kMaxWave;
+  int fault = 0;             // test hook
+};
+
+bpt_status read_opts(const bpt_options* o, Opts* r) {
+  *r = Opts{};
+  if (o == nullptr) return BPT_OK;
+  if (o->reserved != 0) return BPT_ERR_INVALID_ARG;
+  if (o->schedule != BPT_SCHEDULE_FUSED && o->schedule != BPT_SCHEDULE_WAVES)
+    return BPT_ERR_INVALID_ARG;
+  if (o->attn_qpc != 0 && o->attn_qpc != 1 && o->attn_qpc != 2) return BPT_ERR_INVALID_ARG;
+  if (o->max_wave < 0 || o->max_wave > kMaxWave) return BPT_ERR_INVALID_ARG;
+  if (o->fault < 0 || o->fault > 3) return BPT_ERR_INVALID_ARG;
+  r->fused = o->schedule == BPT_SCHEDULE_FUSED ? 1 : 0;
+  r->qpc = o->attn_qpc == 0 ? 2 : o->attn_qpc;
+  r->max_wave = o->max_wave == 0 ? kMaxWave : o->max_wave;
+  r->fault = o->fault;
+  return BPT_OK;
+}
 // 16-column groups (of eight per 128-key row) whose exp2 runs on the FMA
 // pipe instead of MUFU (compile-time tuning knobs; 2 of 8 measured fastest).
 #ifndef BPT_EMU_DK128
@@ -77,7 +104,10 @@ struct Plan {
   int64_t G;     // >0: each wave holds G whole sequences
   int64_t n_waves, P;
   size_t esize;
-  size_t off_w16, off_qkv, off_o, off_v, off_h, total;
+  Opts opt;
+  bool fused;          // bf16 layer on the fused schedule
+  int64_t tail_pairs;  // fused: CTA pairs the scratch is sized for
+  size_t off_w16, off_qkv, off_o, off_v, off_h, off_tv, off_th, total;
 
   Wave wave(int64_t w) const {
     Wave r;
@@ -121,9 +151,12 @@ bpt_status check_shape(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff,
   return BPT_OK;
 }
 
+// The waves layout (wave scratch o / v / H) serves the waves schedule, the
+// fp32 path and the backward; the fused schedule uses tail scratch instead.
 Plan make_plan(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff, int causal,
-               bpt_dtype dtype) {
+               bpt_dtype dtype, const Opts& opt = Opts{}, bool forward = true) {
   Plan p{};
+  p.opt = opt;
   p.B = B; p.N = N; p.d = d; p.h = h; p.d_ff = d_ff; p.dk = d / h;
   p.causal = causal ? 1 : 0;
   p.dtype = dtype;
@@ -134,31 +167,44 @@ Plan make_plan(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff, int cau
   if (p.items == 0) {
     p.n_waves = 0;
     p.P = 0;
-  } else if (p.nb > g_max_wave.load()) {
-    const int64_t mw = g_max_wave.load();
+  } else if (p.nb > opt.max_wave) {
+    const int64_t mw = opt.max_wave;
     p.cps = (p.nb + mw - 1) / mw;
     p.G = 0;
     p.n_waves = B * p.cps;
     p.P = (p.nb + p.cps - 1) / p.cps;
   } else {
     p.cps = 0;
-    p.G = std::max<int64_t>(1, std::min<int64_t>(B, g_max_wave.load() / p.nb));
+    p.G = std::max<int64_t>(1, std::min<int64_t>(B, opt.max_wave / p.nb));
     p.n_waves = (B + p.G - 1) / p.G;
     p.P = p.G * p.nb;
   }
+  p.fused = forward && dtype == BPT_BF16 && opt.fused != 0 && p.items > 0;
+  p.tail_pairs = p.fused ? std::min<int64_t>(bpt::kTailMaxPairs, (p.items + 1) / 2) : 0;
   size_t off = align_up(kHeaderBytes, 1024);
   p.off_w16 = off;
   if (dtype == BPT_BF16)  // fp16 copies of W_Q, W_K, W_V, W_O, W_1, W_2
     off = align_up(off + (size_t(4 * d * d) + size_t(2 * d * d_ff)) * 2, 1024);
   p.off_qkv = off;
   off = align_up(off + size_t(B * N) * size_t(3 * d) * p.esize, 1024);
-  const size_t rows = size_t(p.P * p.blk);
-  p.off_o = off;
-  off = align_up(off + rows * size_t(d) * p.esize, 1024);
-  p.off_v = off;
-  off = align_up(off + rows * size_t(d) * p.esize, 1024);
-  p.off_h = off;
-  off = align_up(off + rows * size_t(d_ff) * p.esize, 1024);
+  if (p.fused) {
+    // per CTA pair: LN2(y) [256, d] and the FFN hidden [256, d_ff], fp16
+    const size_t rows = size_t(p.tail_pairs) * 256;
+    p.off_o = p.off_v = p.off_h = 0;
+    p.off_tv = off;
+    off = align_up(off + rows * size_t(d) * 2, 1024);
+    p.off_th = off;
+    off = align_up(off + rows * size_t(d_ff) * 2, 1024);
+  } else {
+    const size_t rows = size_t(p.P * p.blk);
+    p.off_tv = p.off_th = 0;
+    p.off_o = off;
+    off = align_up(off + rows * size_t(d) * p.esize, 1024);
+    p.off_v = off;
+    off = align_up(off + rows * size_t(d) * p.esize, 1024);
+    p.off_h = off;
+    off = align_up(off + rows * size_t(d_ff) * p.esize, 1024);
+  }
   p.total = off;
   return p;
 }
@@ -213,6 +259,7 @@ bpt_status device_info(int* sms, int* pair_clusters = nullptr) {
           set_smem(bpt::attn_bwd_dkv_tc_kernel<128>, bpt::AttnBwdCfg<128>::KV_SMEM) ||
           set_smem(bpt::attn_bwd_dq_tc_kernel<64>, bpt::AttnBwdCfg<64>::Q_SMEM) ||
           set_smem(bpt::attn_bwd_dkv_tc_kernel<64>, bpt::AttnBwdCfg<64>::KV_SMEM) ||
+          set_smem(bpt::tail_pair_kernel, bpt::kPairSmem) ||
           cudaFuncSetAttribute(bpt::attn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (3 * 64 * 128 + 64 * 65) * 4) != cudaSuccess)
         return BPT_ERR_CUDA;
@@ -311,7 +358,6 @@ struct ProfRec {
   cudaEvent_t a, b;
 };
 bool g_prof_on = false;
-int g_fault = 0;  // test hook, consumed by the next bf16 forward
 std::vector<ProfRec> g_prof;
 std::vector<cudaEvent_t> g_event_pool;
 
@@ -413,13 +459,17 @@ struct AttnGate {
 
 // One wave of the tensor-core attention: o (fp16 block rows) and, if stats is
 // non-null, the per-row (m, l); gated when gate is non-null.
+// o_tok: o is the Q columns of the QKV buffer, token rows (fused schedule);
+// otherwise wave scratch rows [count * 128, d].
 cudaError_t launch_attn(const Plan& P, const Wave& wv_, const CUtensorMap& mQKV, __half* so,
                         float* stats, uint32_t* err, int fault, cudaStream_t s,
-                        const AttnGate* gate = nullptr) {
+                        const AttnGate* gate = nullptr, bool o_tok = false) {
   bpt::AttnPairParams ap{};
   ap.N = int(P.N); ap.nb = int(P.nb); ap.h = int(P.h); ap.d = int(P.d);
   ap.causal = P.causal; ap.item0 = int(wv_.item0); ap.count = int(wv_.count);
   ap.seqs = int(wv_.seqs); ap.o = so; ap.err = err;
+  ap.o_tok = o_tok ? 1 : 0;
+  ap.o_ld = o_tok ? 3 * P.d : P.d;
   ap.scale_log2 = float(1.4426950408889634 / std::sqrt(double(P.dk)));
   ap.stats = reinterpret_cast<float2*>(stats);
   const int64_t kv_head = (wv_.seqs > 0 ? wv_.seqs : 1) * P.N * P.dk * 2 * 2;
@@ -430,7 +480,7 @@ cudaError_t launch_attn(const Plan& P, const Wave& wv_, const CUtensorMap& mQKV,
       break;
     }
   ap.fault = fault;
-  ap.qpc = g_attn_qpc.load();
+  ap.qpc = P.opt.qpc;
   const int64_t units = wv_.seqs == 0 ? (wv_.count + ap.qpc - 1) / ap.qpc
                                       : wv_.seqs * ((P.nb + ap.qpc - 1) / ap.qpc);
   const unsigned grid = unsigned(units * P.h);
@@ -462,12 +512,7 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
   using bf = __nv_bfloat16;
   using hf = __half;
   const int64_t M = P.B * P.N, d = P.d, d_ff = P.d_ff;
-  int fault = 0;
-  {
-    std::lock_guard<std::mutex> lk(g_mu);
-    fault = g_fault;
-    g_fault = 0;
-  }
+  const int fault = P.opt.fault;
   uint32_t* err = reinterpret_cast<uint32_t*>(ws);
   // Tensor-core operands are fp16: the bf16 weights are copied to fp16 once
   // per call (exact in the fp16 normal range), activations are stored fp16.
@@ -491,9 +536,17 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
   const int qkv_chunks = (d % 128 == 0) ? 2 : 1;
   bool ok = map_a(&mXn, xn, M, d) && map_b(&mWq, wq, d, d, qkv_chunks) &&
             map_b(&mWk, wk, d, d, qkv_chunks) && map_b(&mWv, wv, d, d, qkv_chunks) &&
-            map_qkv(&mQKV, qkv, P.B, P.N, d, P.dk) && map_a(&mO, so, R, d) &&
-            map_b(&mWo, wo, d, d, 2) && map_a(&mV, sv, R, d) && map_b(&mW1, w1, d, d_ff, 2) &&
-            map_a(&mH, sh, R, d_ff) && map_b(&mW2, w2, d_ff, d, 2);
+            map_qkv(&mQKV, qkv, P.B, P.N, d, P.dk) && map_b(&mWo, wo, d, d, 2) &&
+            map_b(&mW1, w1, d, d_ff, 2) && map_b(&mW2, w2, d_ff, d, 2);
+  if (P.fused) {
+    // tail A operands: o = the Q columns of QKV (token rows, row stride 3d),
+    // and the per-pair scratch rows of LN2(y) and the hidden
+    const int64_t trows = P.tail_pairs * 256;
+    ok = ok && map_a(&mO, qkv, M, d, 3 * d) &&
+         map_a(&mV, ws + P.off_tv, trows, d) && map_a(&mH, ws + P.off_th, trows, d_ff);
+  } else {
+    ok = ok && map_a(&mO, so, R, d) && map_a(&mV, sv, R, d) && map_a(&mH, sh, R, d_ff);
+  }
   if (!ok) return BPT_ERR_CUDA;
 
   {
@@ -532,6 +585,40 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
     g.fault = fault == 1 ? 1 : 0;
     LaunchScope ls(BPT_KIND_QKV, s);
     if (launch_gemm(mXn, mWq, mWk, mWv, g, sms, s) != cudaSuccess) return BPT_ERR_CUDA;
+  }
+  if (P.fused) {
+    // attention over every query block, o over each block's Q rows
+    const Wave all{0, P.items, P.B};
+    {
+      LaunchScope ls(BPT_KIND_ATTN, s);
+      if (launch_attn(P, all, mQKV, qkv, stats, err, fault == 2 ? 2 : 0, s, gate, true) !=
+          cudaSuccess)
+        return BPT_ERR_CUDA;
+    }
+    int dummy = 0, pairs_max = 0;
+    if (device_info(&dummy, &pairs_max) != BPT_OK) return BPT_ERR_CUDA;
+    bpt::TailParams tp{};
+    tp.blocks = int(P.items);
+    tp.items = int((P.items + 1) / 2);
+    tp.nb = int(P.nb);
+    tp.N = int(P.N);
+    tp.d = int(d);
+    tp.d_ff = int(d_ff);
+    tp.out = out;
+    tp.x = static_cast<const bf*>(x);
+    tp.ln2 = static_cast<const bf*>(ln2);
+    tp.b1 = static_cast<const bf*>(b_1);
+    tp.b2 = static_cast<const bf*>(b_2);
+    tp.v_scr = reinterpret_cast<hf*>(ws + P.off_tv);
+    tp.h_scr = reinterpret_cast<hf*>(ws + P.off_th);
+    tp.err = err;
+    tp.fault = fault == 3 ? 3 : 0;
+    const int64_t pairs = std::max<int64_t>(1, std::min<int64_t>(P.tail_pairs, pairs_max));
+    LaunchScope ls(BPT_KIND_TAIL, s);
+    bpt::tail_pair_kernel<<<unsigned(2 * pairs), bpt::kTailThreads, bpt::kPairSmem, s>>>(
+        mO, mWo, mV, mW1, mH, mW2, tp);
+    if (cudaGetLastError() != cudaSuccess) return BPT_ERR_CUDA;
+    return BPT_OK;
   }
   for (int64_t w = 0; w < P.n_waves; ++w) {
     const Wave wv_ = P.wave(w);
@@ -1102,38 +1189,64 @@ bpt_status backward_bf16(const Plan& P, const BwdLayout& L, const void* x, const
   return BPT_OK;
 }
 
-// Shared body of bpt_layer_forward and bpt_layer_forward_train (stats may be
-// null: no statistics are written).
+// Byte range of a buffer, for overlap checks.
+struct Span {
+  uintptr_t a, b;
+  Span(const void* p, size_t n)
+      : a(reinterpret_cast<uintptr_t>(p)), b(reinterpret_cast<uintptr_t>(p) + n) {}
+  bool overlaps(const Span& o) const { return a < o.b && o.a < b; }
+};
+
+// The forward's input spans (x and every parameter).
+std::vector<Span> forward_inputs(const void* x, const void* ln1, const void* W_Q, const void* W_K,
+                                 const void* W_V, const void* W_O, const void* ln2,
+                                 const void* W_1, const void* b_1, const void* W_2,
+                                 const void* b_2, int64_t B, int64_t N, int64_t d, int64_t d_ff,
+                                 size_t esize) {
+  return {Span(x, size_t(B * N * d) * esize), Span(ln1, size_t(2 * d) * esize),
+          Span(W_Q, size_t(d * d) * esize),   Span(W_K, size_t(d * d) * esize),
+          Span(W_V, size_t(d * d) * esize),   Span(W_O, size_t(d * d) * esize),
+          Span(ln2, size_t(2 * d) * esize),   Span(W_1, size_t(d * d_ff) * esize),
+          Span(b_1, size_t(d_ff) * esize),    Span(W_2, size_t(d_ff * d) * esize),
+          Span(b_2, size_t(d) * esize)};
+}
+
+// Shared body of the forward entry points (stats may be null: no statistics
+// are written; gate non-null: gated attention).
 bpt_status layer_forward_impl(const void* x, const void* ln1, const void* W_Q, const void* W_K,
                               const void* W_V, const void* W_O, const void* ln2, const void* W_1,
                               const void* b_1, const void* W_2, const void* b_2, int64_t B,
                               int64_t N, int64_t d, int64_t h, int64_t d_ff, int causal,
                               bpt_dtype dtype, float* out, float* stats, void* workspace,
-                              size_t workspace_bytes, bpt_stream_t stream,
-                              const AttnGate* gate = nullptr) {
+                              size_t workspace_bytes, const bpt_options* opts,
+                              bpt_stream_t stream, const AttnGate* gate = nullptr) {
   bpt_status st = check_shape(B, N, d, h, d_ff, causal, dtype);
+  if (st != BPT_OK) return st;
+  Opts opt;
+  st = read_opts(opts, &opt);
   if (st != BPT_OK) return st;
   if (gate != nullptr && dtype != BPT_BF16) return BPT_ERR_UNSUPPORTED;
   if (B == 0 || N == 0) return BPT_OK;
   const void* ptrs[] = {x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, out, workspace};
   for (const void* p : ptrs)
     if (p == nullptr || misaligned(p)) return BPT_ERR_INVALID_ARG;
-  const Plan P = make_plan(B, N, d, h, d_ff, causal, dtype);
+  const Plan P = make_plan(B, N, d, h, d_ff, causal, dtype, opt);
   if (workspace_bytes < P.total) return BPT_ERR_WORKSPACE;
-  // out must not overlap x (it is written before x is last read)
-  const uintptr_t xo = reinterpret_cast<uintptr_t>(x), oo = reinterpret_cast<uintptr_t>(out);
-  const size_t xbytes = size_t(B * N * d) * P.esize, obytes = size_t(B * N * d) * 4;
-  if (xo < oo + obytes && oo < xo + xbytes) return BPT_ERR_INVALID_ARG;
-  const uintptr_t wo = reinterpret_cast<uintptr_t>(workspace);
-  if (wo < oo + obytes && oo < wo + P.total) return BPT_ERR_INVALID_ARG;
+  // out and the workspace are written while the inputs are still read: they
+  // must overlap no input and not each other; stats likewise.
+  const std::vector<Span> ins =
+      forward_inputs(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, B, N, d, d_ff, P.esize);
+  const Span so(out, size_t(B * N * d) * 4), sw(workspace, P.total);
+  if (so.overlaps(sw)) return BPT_ERR_INVALID_ARG;
+  for (const Span& in : ins)
+    if (so.overlaps(in) || sw.overlaps(in)) return BPT_ERR_INVALID_ARG;
   if (stats != nullptr) {
-    // stats must not overlap out, x or the workspace (all written or read here)
-    const uintptr_t so = reinterpret_cast<uintptr_t>(stats);
-    const size_t sbytes = size_t(B * h * N) * 2 * sizeof(float);
-    if (misaligned(stats) || (so < oo + obytes && oo < so + sbytes) ||
-        (so < xo + xbytes && xo < so + sbytes) || (so < wo + P.total && wo < so + sbytes))
-      return BPT_ERR_INVALID_ARG;
+    const Span ss(stats, size_t(B * h * N) * 2 * sizeof(float));
+    if (misaligned(stats) || ss.overlaps(so) || ss.overlaps(sw)) return BPT_ERR_INVALID_ARG;
+    for (const Span& in : ins)
+      if (ss.overlaps(in)) return BPT_ERR_INVALID_ARG;
   }
+  if (opt.fault != 0 && dtype != BPT_BF16) return BPT_ERR_INVALID_ARG;
 
   int sms = 0;
   st = device_info(&sms);
@@ -1155,59 +1268,13 @@ bpt_status layer_forward_impl(const void* x, const void* ln1, const void* W_Q, c
                      static_cast<const float*>(b_2), out, stats, ws, s);
 }
 
-
-extern "C" {
-
-bpt_status bpt_layer_workspace_size(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff,
-                                    int causal, bpt_dtype dtype, size_t* bytes) {
-  if (!bytes) return BPT_ERR_INVALID_ARG;
-  const bpt_status st = check_shape(B, N, d, h, d_ff, causal, dtype);
-  if (st != BPT_OK) return st;
-  *bytes = make_plan(B, N, d, h, d_ff, causal, dtype).total;
-  return BPT_OK;
-}
-
-bpt_status bpt_layer_launch_count(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff,
-                                  int causal, bpt_dtype dtype, int64_t* launches) {
-  if (!launches) return BPT_ERR_INVALID_ARG;
-  const bpt_status st = check_shape(B, N, d, h, d_ff, causal, dtype);
-  if (st != BPT_OK) return st;
-  const Plan P = make_plan(B, N, d, h, d_ff, causal, dtype);
-  *launches = P.items == 0 ? 0 : (dtype == BPT_BF16 ? 3 : 2) + 5 * P.n_waves;
-  return BPT_OK;
-}
-
-bpt_status bpt_layer_forward(const void* x, const void* ln1, const void* W_Q, const void* W_K,
-                             const void* W_V, const void* W_O, const void* ln2, const void* W_1,
-                             const void* b_1, const void* W_2, const void* b_2, int64_t B,
-                             int64_t N, int64_t d, int64_t h, int64_t d_ff, int causal,
-                             bpt_dtype dtype, float* out, void* workspace, size_t workspace_bytes,
-                             bpt_stream_t stream) {
-  return layer_forward_impl(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, B, N, d, h, d_ff,
-                            causal, dtype, out, nullptr, workspace, workspace_bytes, stream);
-}
-
-bpt_status bpt_layer_forward_train(const void* x, const void* ln1, const void* W_Q,
-                                   const void* W_K, const void* W_V, const void* W_O,
-                                   const void* ln2, const void* W_1, const void* b_1,
-                                   const void* W_2, const void* b_2, int64_t B, int64_t N,
-                                   int64_t d, int64_t h, int64_t d_ff, int causal,
-                                   bpt_dtype dtype, float* out, float* stats, void* workspace,
-                                   size_t workspace_bytes, bpt_stream_t stream) {
-  if (stats == nullptr) return BPT_ERR_INVALID_ARG;
-  return layer_forward_impl(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, B, N, d, h, d_ff,
-                            causal, dtype, out, stats, workspace, workspace_bytes, stream);
-}
-
-
-bpt_status bpt_layer_forward_bsfa(const void* x, const void* ln1, const void* W_Q,
-                                  const void* W_K, const void* W_V, const void* W_O,
-                                  const void* ln2, const void* W_1, const void* b_1,
-                                  const void* W_2, const void* b_2, int64_t B, int64_t N,
-                                  int64_t d, int64_t h, int64_t d_ff, int causal,
-                                  bpt_dtype dtype, const float* thresholds, float* block_max,
-                                  uint8_t* kept, float* out, void* workspace,
-                                  size_t workspace_bytes, bpt_stream_t stream) {
+bpt_status bsfa_impl(const void* x, const void* ln1, const void* W_Q, const void* W_K,
+                     const void* W_V, const void* W_O, const void* ln2, const void* W_1,
+                     const void* b_1, const void* W_2, const void* b_2, int64_t B, int64_t N,
+                     int64_t d, int64_t h, int64_t d_ff, int causal, bpt_dtype dtype,
+                     const float* thresholds, float* block_max, uint8_t* kept, float* out,
+                     void* workspace, size_t workspace_bytes, const bpt_options* opts,
+                     bpt_stream_t stream) {
   bpt_status st = check_shape(B, N, d, h, d_ff, causal, dtype);
   if (st != BPT_OK) return st;
   if (dtype != BPT_BF16) return BPT_ERR_UNSUPPORTED;
@@ -1215,57 +1282,49 @@ bpt_status bpt_layer_forward_bsfa(const void* x, const void* ln1, const void* W_
   if (B == 0 || N == 0) return BPT_OK;
   const size_t nb = size_t((N + 127) / 128);
   const size_t tbytes = size_t(h) * nb * 4, pairs = size_t(B) * size_t(h) * nb * nb;
-  auto span = [](const void* p, size_t n) {
-    return std::make_pair(reinterpret_cast<uintptr_t>(p), reinterpret_cast<uintptr_t>(p) + n);
-  };
-  auto overlap = [](std::pair<uintptr_t, uintptr_t> a, std::pair<uintptr_t, uintptr_t> b) {
-    return a.first < b.second && b.first < a.second;
-  };
-  const auto o = span(out, size_t(B * N * d) * 4), w = span(workspace, workspace_bytes),
-             t = span(thresholds, tbytes), xs = span(x, size_t(B * N * d) * 2);
-  if ((reinterpret_cast<uintptr_t>(thresholds) & 3u) || overlap(t, o) || overlap(t, w))
+  const Span o(out, size_t(B * N * d) * 4), w(workspace, workspace_bytes),
+      t(thresholds, tbytes);
+  const std::vector<Span> ins =
+      forward_inputs(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, B, N, d, d_ff, 2);
+  if ((reinterpret_cast<uintptr_t>(thresholds) & 3u) || t.overlaps(o) || t.overlaps(w))
     return BPT_ERR_INVALID_ARG;
   if (block_max != nullptr) {
-    const auto m = span(block_max, pairs * 4);
-    if ((reinterpret_cast<uintptr_t>(block_max) & 3u) || overlap(m, o) || overlap(m, w) ||
-        overlap(m, t) || overlap(m, xs))
+    const Span m(block_max, pairs * 4);
+    if ((reinterpret_cast<uintptr_t>(block_max) & 3u) || m.overlaps(o) || m.overlaps(w) ||
+        m.overlaps(t))
       return BPT_ERR_INVALID_ARG;
+    for (const Span& in : ins)
+      if (m.overlaps(in)) return BPT_ERR_INVALID_ARG;
   }
   if (kept != nullptr) {
-    const auto k = span(kept, pairs);
-    if (overlap(k, o) || overlap(k, w) || overlap(k, t) || overlap(k, xs) ||
-        (block_max != nullptr && overlap(k, span(block_max, pairs * 4))))
+    const Span k(kept, pairs);
+    if (k.overlaps(o) || k.overlaps(w) || k.overlaps(t) ||
+        (block_max != nullptr && k.overlaps(Span(block_max, pairs * 4))))
       return BPT_ERR_INVALID_ARG;
+    for (const Span& in : ins)
+      if (k.overlaps(in)) return BPT_ERR_INVALID_ARG;
   }
   const AttnGate gate{thresholds, block_max, kept};
   return layer_forward_impl(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, B, N, d, h, d_ff,
-                            causal, dtype, out, nullptr, workspace, workspace_bytes, stream,
+                            causal, dtype, out, nullptr, workspace, workspace_bytes, opts, stream,
                             &gate);
 }
 
-bpt_status bpt_layer_backward_workspace_size(int64_t B, int64_t N, int64_t d, int64_t h,
-                                             int64_t d_ff, int causal, bpt_dtype dtype,
-                                             size_t* bytes) {
-  if (bytes == nullptr) return BPT_ERR_INVALID_ARG;
-  const bpt_status st = check_shape(B, N, d, h, d_ff, causal, dtype);
-  if (st != BPT_OK) return st;
-  const Plan P = make_plan(B, N, d, h, d_ff, causal, dtype);
-  *bytes = dtype == BPT_BF16 ? make_bwd_layout(P).total : make_bwd_layout_f32(P).total;
-  return BPT_OK;
-}
-
-bpt_status bpt_layer_backward(const void* x, const void* ln1, const void* W_Q, const void* W_K,
-                              const void* W_V, const void* W_O, const void* ln2, const void* W_1,
-                              const void* b_1, const void* W_2, const void* b_2,
-                              const float* stats, const float* dZ, int64_t B, int64_t N,
-                              int64_t d, int64_t h, int64_t d_ff, int causal, bpt_dtype dtype,
-                              float* dx, float* d_ln1, float* dW_Q, float* dW_K, float* dW_V,
-                              float* dW_O, float* d_ln2, float* dW_1, float* db_1, float* dW_2,
-                              float* db_2, void* workspace, size_t workspace_bytes,
-                              bpt_stream_t stream) {
+bpt_status backward_impl(const void* x, const void* ln1, const void* W_Q, const void* W_K,
+                         const void* W_V, const void* W_O, const void* ln2, const void* W_1,
+                         const void* b_1, const void* W_2, const void* b_2, const float* stats,
+                         const float* dZ, int64_t B, int64_t N, int64_t d, int64_t h,
+                         int64_t d_ff, int causal, bpt_dtype dtype, float* dx, float* d_ln1,
+                         float* dW_Q, float* dW_K, float* dW_V, float* dW_O, float* d_ln2,
+                         float* dW_1, float* db_1, float* dW_2, float* db_2, void* workspace,
+                         size_t workspace_bytes, const bpt_options* opts, bpt_stream_t stream) {
   (void)b_2;  // the output's bias does not enter any gradient but its own
   bpt_status st = check_shape(B, N, d, h, d_ff, causal, dtype);
   if (st != BPT_OK) return st;
+  Opts opt;
+  st = read_opts(opts, &opt);
+  if (st != BPT_OK) return st;
+  if (opt.fault != 0) return BPT_ERR_INVALID_ARG;
   if (B == 0 || N == 0) return BPT_OK;
   const void* ins[] = {x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, stats, dZ, workspace};
   for (const void* p : ins)
@@ -1275,27 +1334,27 @@ bpt_status bpt_layer_backward(const void* x, const void* ln1, const void* W_Q, c
                               size_t(d * d) * 4, size_t(d * d) * 4, size_t(d * d) * 4,
                               size_t(2 * d) * 4, size_t(d * d_ff) * 4, size_t(d_ff) * 4,
                               size_t(d_ff * d) * 4, size_t(d) * 4};
-  const Plan P = make_plan(B, N, d, h, d_ff, causal, dtype);
+  const Plan P = make_plan(B, N, d, h, d_ff, causal, dtype, opt, false);
   const size_t ws_need =
       dtype == BPT_BF16 ? make_bwd_layout(P).total : make_bwd_layout_f32(P).total;
   if (workspace_bytes < ws_need) return BPT_ERR_WORKSPACE;
   // Outputs must be aligned and must not overlap each other, the workspace,
-  // or the inputs they are written after being read from (x, stats, dZ).
-  const uintptr_t wsb = reinterpret_cast<uintptr_t>(workspace);
-  const std::pair<uintptr_t, size_t> reads[] = {
-      {reinterpret_cast<uintptr_t>(x), size_t(B * N * d) * P.esize},
-      {reinterpret_cast<uintptr_t>(stats), size_t(B * h * N) * 8},
-      {reinterpret_cast<uintptr_t>(dZ), size_t(B * N * d) * 4},
-      {wsb, ws_need}};
+  // or any input (every input is read after some output is first written).
+  std::vector<Span> reads =
+      forward_inputs(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, B, N, d, d_ff, P.esize);
+  reads.push_back(Span(stats, size_t(B * h * N) * 8));
+  reads.push_back(Span(dZ, size_t(B * N * d) * 4));
+  const Span sw(workspace, ws_need);
+  for (const Span& r : reads)
+    if (sw.overlaps(r)) return BPT_ERR_INVALID_ARG;
+  reads.push_back(sw);
   for (int i = 0; i < 11; ++i) {
     if (outs[i] == nullptr || misaligned(outs[i])) return BPT_ERR_INVALID_ARG;
-    const uintptr_t a = reinterpret_cast<uintptr_t>(outs[i]);
-    for (const auto& r : reads)
-      if (a < r.first + r.second && r.first < a + out_bytes[i]) return BPT_ERR_INVALID_ARG;
-    for (int j = 0; j < i; ++j) {
-      const uintptr_t b = reinterpret_cast<uintptr_t>(outs[j]);
-      if (a < b + out_bytes[j] && b < a + out_bytes[i]) return BPT_ERR_INVALID_ARG;
-    }
+    const Span a(outs[i], out_bytes[i]);
+    for (const Span& r : reads)
+      if (a.overlaps(r)) return BPT_ERR_INVALID_ARG;
+    for (int j = 0; j < i; ++j)
+      if (a.overlaps(Span(outs[j], out_bytes[j]))) return BPT_ERR_INVALID_ARG;
   }
   int sms = 0;
   st = device_info(&sms);
@@ -1316,8 +1375,174 @@ bpt_status bpt_layer_backward(const void* x, const void* ln1, const void* W_Q, c
                        dW_Q, dW_K, dW_V, dW_O, d_ln2, dW_1, db_1, dW_2, db_2, ws, s, sms);
 }
 
+bpt_status plan_for(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff, int causal,
+                    bpt_dtype dtype, const bpt_options* opts, bool forward, Plan* P) {
+  bpt_status st = check_shape(B, N, d, h, d_ff, causal, dtype);
+  if (st != BPT_OK) return st;
+  Opts opt;
+  st = read_opts(opts, &opt);
+  if (st != BPT_OK) return st;
+  *P = make_plan(B, N, d, h, d_ff, causal, dtype, opt, forward);
+  return BPT_OK;
+}
+
+// Device address of the allocation-free entry point's array (defined below).
+bpt_status static_ws_address(void** ptr);
+
+extern "C" {
+
+bpt_status bpt_layer_workspace_size_opt(int64_t B, int64_t N, int64_t d, int64_t h,
+                                        int64_t d_ff, int causal, bpt_dtype dtype,
+                                        const bpt_options* opts, size_t* bytes) {
+  if (!bytes) return BPT_ERR_INVALID_ARG;
+  Plan P;
+  const bpt_status st = plan_for(B, N, d, h, d_ff, causal, dtype, opts, true, &P);
+  if (st != BPT_OK) return st;
+  *bytes = P.total;
+  return BPT_OK;
+}
+
+bpt_status bpt_layer_workspace_size(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff,
+                                    int causal, bpt_dtype dtype, size_t* bytes) {
+  return bpt_layer_workspace_size_opt(B, N, d, h, d_ff, causal, dtype, nullptr, bytes);
+}
+
+bpt_status bpt_layer_launch_count_opt(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff,
+                                      int causal, bpt_dtype dtype, const bpt_options* opts,
+                                      int64_t* launches) {
+  if (!launches) return BPT_ERR_INVALID_ARG;
+  Plan P;
+  const bpt_status st = plan_for(B, N, d, h, d_ff, causal, dtype, opts, true, &P);
+  if (st != BPT_OK) return st;
+  if (P.items == 0)
+    *launches = 0;
+  else if (P.fused)
+    *launches = 5;  // weight copy, LN1, QKV GEMM, attention, tail
+  else
+    *launches = (dtype == BPT_BF16 ? 3 : 2) + 5 * P.n_waves;
+  return BPT_OK;
+}
+
+bpt_status bpt_layer_launch_count(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff,
+                                  int causal, bpt_dtype dtype, int64_t* launches) {
+  return bpt_layer_launch_count_opt(B, N, d, h, d_ff, causal, dtype, nullptr, launches);
+}
+
+bpt_status bpt_layer_forward(const void* x, const void* ln1, const void* W_Q, const void* W_K,
+                             const void* W_V, const void* W_O, const void* ln2, const void* W_1,
+                             const void* b_1, const void* W_2, const void* b_2, int64_t B,
+                             int64_t N, int64_t d, int64_t h, int64_t d_ff, int causal,
+                             bpt_dtype dtype, float* out, void* workspace, size_t workspace_bytes,
+                             bpt_stream_t stream) {
+  return layer_forward_impl(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, B, N, d, h, d_ff,
+                            causal, dtype, out, nullptr, workspace, workspace_bytes, nullptr,
+                            stream);
+}
+
+bpt_status bpt_layer_forward_opt(const void* x, const void* ln1, const void* W_Q,
+                                 const void* W_K, const void* W_V, const void* W_O,
+                                 const void* ln2, const void* W_1, const void* b_1,
+                                 const void* W_2, const void* b_2, int64_t B, int64_t N,
+                                 int64_t d, int64_t h, int64_t d_ff, int causal, bpt_dtype dtype,
+                                 float* out, float* stats, void* workspace,
+                                 size_t workspace_bytes, const bpt_options* opts,
+                                 bpt_stream_t stream) {
+  return layer_forward_impl(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, B, N, d, h, d_ff,
+                            causal, dtype, out, stats, workspace, workspace_bytes, opts, stream);
+}
+
+bpt_status bpt_layer_forward_train(const void* x, const void* ln1, const void* W_Q,
+                                   const void* W_K, const void* W_V, const void* W_O,
+                                   const void* ln2, const void* W_1, const void* b_1,
+                                   const void* W_2, const void* b_2, int64_t B, int64_t N,
+                                   int64_t d, int64_t h, int64_t d_ff, int causal,
+                                   bpt_dtype dtype, float* out, float* stats, void* workspace,
+                                   size_t workspace_bytes, bpt_stream_t stream) {
+  if (stats == nullptr) return BPT_ERR_INVALID_ARG;
+  return layer_forward_impl(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, B, N, d, h, d_ff,
+                            causal, dtype, out, stats, workspace, workspace_bytes, nullptr,
+                            stream);
+}
+
+bpt_status bpt_layer_forward_bsfa(const void* x, const void* ln1, const void* W_Q,
+                                  const void* W_K, const void* W_V, const void* W_O,
+                                  const void* ln2, const void* W_1, const void* b_1,
+                                  const void* W_2, const void* b_2, int64_t B, int64_t N,
+                                  int64_t d, int64_t h, int64_t d_ff, int causal,
+                                  bpt_dtype dtype, const float* thresholds, float* block_max,
+                                  uint8_t* kept, float* out, void* workspace,
+                                  size_t workspace_bytes, bpt_stream_t stream) {
+  return bsfa_impl(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, B, N, d, h, d_ff, causal,
+                   dtype, thresholds, block_max, kept, out, workspace, workspace_bytes, nullptr,
+                   stream);
+}
+
+bpt_status bpt_layer_forward_bsfa_opt(const void* x, const void* ln1, const void* W_Q,
+                                      const void* W_K, const void* W_V, const void* W_O,
+                                      const void* ln2, const void* W_1, const void* b_1,
+                                      const void* W_2, const void* b_2, int64_t B, int64_t N,
+                                      int64_t d, int64_t h, int64_t d_ff, int causal,
+                                      bpt_dtype dtype, const float* thresholds, float* block_max,
+                                      uint8_t* kept, float* out, void* workspace,
+                                      size_t workspace_bytes, const bpt_options* opts,
+                                      bpt_stream_t stream) {
+  return bsfa_impl(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, B, N, d, h, d_ff, causal,
+                   dtype, thresholds, block_max, kept, out, workspace, workspace_bytes, opts,
+                   stream);
+}
+
+bpt_status bpt_layer_backward_workspace_size_opt(int64_t B, int64_t N, int64_t d, int64_t h,
+                                                 int64_t d_ff, int causal, bpt_dtype dtype,
+                                                 const bpt_options* opts, size_t* bytes) {
+  if (bytes == nullptr) return BPT_ERR_INVALID_ARG;
+  Plan P;
+  const bpt_status st = plan_for(B, N, d, h, d_ff, causal, dtype, opts, false, &P);
+  if (st != BPT_OK) return st;
+  *bytes = dtype == BPT_BF16 ? make_bwd_layout(P).total : make_bwd_layout_f32(P).total;
+  return BPT_OK;
+}
+
+bpt_status bpt_layer_backward_workspace_size(int64_t B, int64_t N, int64_t d, int64_t h,
+                                             int64_t d_ff, int causal, bpt_dtype dtype,
+                                             size_t* bytes) {
+  return bpt_layer_backward_workspace_size_opt(B, N, d, h, d_ff, causal, dtype, nullptr, bytes);
+}
+
+bpt_status bpt_layer_backward(const void* x, const void* ln1, const void* W_Q, const void* W_K,
+                              const void* W_V, const void* W_O, const void* ln2, const void* W_1,
+                              const void* b_1, const void* W_2, const void* b_2,
+                              const float* stats, const float* dZ, int64_t B, int64_t N,
+                              int64_t d, int64_t h, int64_t d_ff, int causal, bpt_dtype dtype,
+                              float* dx, float* d_ln1, float* dW_Q, float* dW_K, float* dW_V,
+                              float* dW_O, float* d_ln2, float* dW_1, float* db_1, float* dW_2,
+                              float* db_2, void* workspace, size_t workspace_bytes,
+                              bpt_stream_t stream) {
+  return backward_impl(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, stats, dZ, B, N, d, h,
+                       d_ff, causal, dtype, dx, d_ln1, dW_Q, dW_K, dW_V, dW_O, d_ln2, dW_1, db_1,
+                       dW_2, db_2, workspace, workspace_bytes, nullptr, stream);
+}
+
+bpt_status bpt_layer_backward_opt(const void* x, const void* ln1, const void* W_Q,
+                                  const void* W_K, const void* W_V, const void* W_O,
+                                  const void* ln2, const void* W_1, const void* b_1,
+                                  const void* W_2, const void* b_2, const float* stats,
+                                  const float* dZ, int64_t B, int64_t N, int64_t d, int64_t h,
+                                  int64_t d_ff, int causal, bpt_dtype dtype, float* dx,
+                                  float* d_ln1, float* dW_Q, float* dW_K, float* dW_V,
+                                  float* dW_O, float* d_ln2, float* dW_1, float* db_1,
+                                  float* dW_2, float* db_2, void* workspace,
+                                  size_t workspace_bytes, const bpt_options* opts,
+                                  bpt_stream_t stream) {
+  return backward_impl(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, stats, dZ, B, N, d, h,
+                       d_ff, causal, dtype, dx, d_ln1, dW_Q, dW_K, dW_V, dW_O, d_ln2, dW_1, db_1,
+                       dW_2, db_2, workspace, workspace_bytes, opts, stream);
+}
+
 bpt_status bpt_read_device_error(void* workspace, bpt_stream_t stream, uint32_t* site) {
-  if (!workspace) return BPT_ERR_INVALID_ARG;
+  if (!workspace) {
+    const bpt_status st = static_ws_address(&workspace);
+    if (st != BPT_OK) return st;
+  }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return BPT_ERR_CUDA;
   uint32_t word = 0;
@@ -1342,25 +1567,6 @@ const char* bpt_status_string(bpt_status status) {
     case BPT_ERR_RANGE: return "BPT_ERR_RANGE: a tensor-core operand exceeded the fp16 range";
   }
   return "BPT_UNKNOWN_STATUS";
-}
-
-bpt_status bpt_debug_set_max_wave(int64_t blocks) {
-  if (blocks < 0 || blocks > kMaxWave) return BPT_ERR_INVALID_ARG;
-  g_max_wave.store(blocks == 0 ? kMaxWave : blocks);
-  return BPT_OK;
-}
-
-bpt_status bpt_debug_set_attn_qpc(int qpc) {
-  if (qpc != 1 && qpc != 2) return BPT_ERR_INVALID_ARG;
-  g_attn_qpc.store(qpc);
-  return BPT_OK;
-}
-
-bpt_status bpt_debug_inject_fault(int code) {
-  if (code < 0 || code > 2) return BPT_ERR_INVALID_ARG;
-  std::lock_guard<std::mutex> lk(g_mu);
-  g_fault = code;
-  return BPT_OK;
 }
 
 bpt_status bpt_profile_enable(int enable) {
@@ -1393,26 +1599,49 @@ bpt_status bpt_profile_read(double* ms, int64_t* launches, int n) {
 // Workspace of bpt_layer_forward_static: a file-scope device array, so that
 // callers that may not allocate still get the full layer.  In host code the
 // symbol is only a stand-in; its device address comes from
-// cudaGetSymbolAddress, looked up once per device with that device current.
+// cudaGetSymbolAddress, looked up with the device current and cached per
+// (device, CUDA context): a caller that switches contexts, or a context
+// created after a device reset, gets a fresh lookup.
 static __device__ __align__(256) uint8_t g_bpt_static_ws[BPT_STATIC_WORKSPACE_BYTES];
 
 namespace {
-void* g_static_ws_ptr[64] = {};
+struct StaticWs {
+  void* ctx = nullptr;
+  void* ptr = nullptr;
+};
+StaticWs g_static_ws[64];
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+}  // namespace
 
 bpt_status static_ws_address(void** ptr) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BPT_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_mu);
-  if (g_static_ws_ptr[dev] == nullptr) {
+  if (g_ctx_get_current == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return BPT_ERR_CUDA;
+    g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+  }
+  CUcontext ctx = nullptr;
+  if (g_ctx_get_current(&ctx) != CUDA_SUCCESS) return BPT_ERR_CUDA;
+  StaticWs& e = g_static_ws[dev];
+  if (ctx == nullptr || e.ptr == nullptr || e.ctx != static_cast<void*>(ctx)) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_bpt_static_ws) != cudaSuccess || p == nullptr)
       return BPT_ERR_CUDA;
-    g_static_ws_ptr[dev] = p;
+    // the lookup made the runtime's context current if none was
+    if (ctx == nullptr && (g_ctx_get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr))
+      return BPT_ERR_CUDA;
+    e.ctx = static_cast<void*>(ctx);
+    e.ptr = p;
   }
-  *ptr = g_static_ws_ptr[dev];
+  *ptr = e.ptr;
   return BPT_OK;
 }
-}  // namespace
 
 extern "C" bpt_status bpt_layer_forward_static(const void* x, const void* ln1, const void* W_Q,
                                                const void* W_K, const void* W_V, const void* W_O,

@@ -49,10 +49,11 @@ def to_device(inp: Dict[str, np.ndarray], dtype: str, device="cuda",
 
 
 def workspace_for(B: int, N: int, d: int, h: int, d_ff: int, causal: bool,
-                  dtype: torch.dtype, device="cuda") -> torch.Tensor:
-    """Allocates (through torch) a workspace of the size the library asks for."""
+                  dtype: torch.dtype, device="cuda", opts=None) -> torch.Tensor:
+    """Allocates (through torch) a workspace of the size the library asks for
+    (``opts``: None, an ``Options`` or a dict of its fields)."""
     code = _lib.BPT_BF16 if dtype == torch.bfloat16 else _lib.BPT_F32
-    st, nbytes = _lib.bpt_layer_workspace_size(B, N, d, h, d_ff, causal, code)
+    st, nbytes = _lib.bpt_layer_workspace_size_opt(B, N, d, h, d_ff, causal, code, opts)
     if st != _lib.BPT_OK:
         raise _lib.BptError(st, "bpt_layer_workspace_size")
     return torch.empty(nbytes, dtype=torch.uint8, device=device)
@@ -61,11 +62,13 @@ def workspace_for(B: int, N: int, d: int, h: int, d_ff: int, causal: bool,
 def layer_forward(x: torch.Tensor, p: Dict[str, torch.Tensor], h: int, causal: bool,
                   out: Optional[torch.Tensor] = None,
                   workspace: Optional[torch.Tensor] = None,
-                  stream: Optional[torch.cuda.Stream] = None):
-    """Z = BPT layer(x) via ``bpt_layer_forward``; returns (out, workspace).
+                  stream: Optional[torch.cuda.Stream] = None, opts=None):
+    """Z = BPT layer(x) via ``bpt_layer_forward`` (``bpt_layer_forward_opt``
+    when ``opts`` is given); returns (out, workspace).
 
     x: [B, N, d] bf16 or fp32 on the GPU; p: ``PARAM_NAMES`` tensors of the
-    same dtype (ln1/ln2 as [2, d]); out: [B, N, d] fp32.
+    same dtype (ln1/ln2 as [2, d]); out: [B, N, d] fp32; opts: None, an
+    ``Options`` or a dict of its fields (schedule, attn_qpc, max_wave, fault).
     """
     if x.dim() != 3:
         raise ValueError("x must be [B, N, d]")
@@ -79,11 +82,17 @@ def layer_forward(x: torch.Tensor, p: Dict[str, torch.Tensor], h: int, causal: b
     if out is None:
         out = torch.empty((B, N, d), dtype=torch.float32, device=x.device)
     if workspace is None:
-        workspace = workspace_for(B, N, d, h, d_ff, causal, x.dtype, x.device)
+        workspace = workspace_for(B, N, d, h, d_ff, causal, x.dtype, x.device, opts)
     s = stream if stream is not None else torch.cuda.current_stream(x.device)
-    st = _lib.bpt_layer_forward(*[t.data_ptr() for t in tensors], B, N, d, h, d_ff, causal,
-                                code, out.data_ptr(), workspace.data_ptr(), workspace.numel(),
-                                s.cuda_stream)
+    if opts is None:
+        st = _lib.bpt_layer_forward(*[t.data_ptr() for t in tensors], B, N, d, h, d_ff, causal,
+                                    code, out.data_ptr(), workspace.data_ptr(),
+                                    workspace.numel(), s.cuda_stream)
+    else:
+        st = _lib.bpt_layer_forward_opt(*[t.data_ptr() for t in tensors], B, N, d, h, d_ff,
+                                        causal, code, out.data_ptr(), None,
+                                        workspace.data_ptr(), workspace.numel(), opts,
+                                        s.cuda_stream)
     if st != _lib.BPT_OK:
         raise _lib.BptError(st, "bpt_layer_forward")
     return out, workspace
@@ -93,7 +102,7 @@ def layer_forward_train(x: torch.Tensor, p: Dict[str, torch.Tensor], h: int, cau
                         out: Optional[torch.Tensor] = None,
                         stats: Optional[torch.Tensor] = None,
                         workspace: Optional[torch.Tensor] = None,
-                        stream: Optional[torch.cuda.Stream] = None):
+                        stream: Optional[torch.cuda.Stream] = None, opts=None):
     """``layer_forward`` that also returns the per-row softmax statistics via
     ``bpt_layer_forward_train``: (out, stats, workspace), stats [B, h, N, 2]
     fp32 holding (m, l) per (batch, head, query row)."""
@@ -111,11 +120,17 @@ def layer_forward_train(x: torch.Tensor, p: Dict[str, torch.Tensor], h: int, cau
     if stats is None:
         stats = torch.empty((B, h, N, 2), dtype=torch.float32, device=x.device)
     if workspace is None:
-        workspace = workspace_for(B, N, d, h, d_ff, causal, x.dtype, x.device)
+        workspace = workspace_for(B, N, d, h, d_ff, causal, x.dtype, x.device, opts)
     s = stream if stream is not None else torch.cuda.current_stream(x.device)
-    st = _lib.bpt_layer_forward_train(*[t.data_ptr() for t in tensors], B, N, d, h, d_ff, causal,
-                                      code, out.data_ptr(), stats.data_ptr(),
-                                      workspace.data_ptr(), workspace.numel(), s.cuda_stream)
+    if opts is None:
+        st = _lib.bpt_layer_forward_train(*[t.data_ptr() for t in tensors], B, N, d, h, d_ff,
+                                          causal, code, out.data_ptr(), stats.data_ptr(),
+                                          workspace.data_ptr(), workspace.numel(), s.cuda_stream)
+    else:
+        st = _lib.bpt_layer_forward_opt(*[t.data_ptr() for t in tensors], B, N, d, h, d_ff,
+                                        causal, code, out.data_ptr(), stats.data_ptr(),
+                                        workspace.data_ptr(), workspace.numel(), opts,
+                                        s.cuda_stream)
     if st != _lib.BPT_OK:
         raise _lib.BptError(st, "bpt_layer_forward_train")
     return out, stats, workspace
@@ -125,7 +140,7 @@ def layer_forward_bsfa(x: torch.Tensor, p: Dict[str, torch.Tensor], h: int, caus
                        thresholds: torch.Tensor, block_max: bool = False, kept: bool = False,
                        out: Optional[torch.Tensor] = None,
                        workspace: Optional[torch.Tensor] = None,
-                       stream: Optional[torch.cuda.Stream] = None):
+                       stream: Optional[torch.cuda.Stream] = None, opts=None):
     """``layer_forward`` with block-gated attention via ``bpt_layer_forward_bsfa``.
 
     thresholds: fp32 CUDA tensor [h, nb], nb = ceil(N / 128).  Returns
@@ -151,14 +166,14 @@ def layer_forward_bsfa(x: torch.Tensor, p: Dict[str, torch.Tensor], h: int, caus
     if out is None:
         out = torch.empty((B, N, d), dtype=torch.float32, device=x.device)
     if workspace is None:
-        workspace = workspace_for(B, N, d, h, d_ff, causal, x.dtype, x.device)
+        workspace = workspace_for(B, N, d, h, d_ff, causal, x.dtype, x.device, opts)
     s = stream if stream is not None else torch.cuda.current_stream(x.device)
-    st = _lib.bpt_layer_forward_bsfa(*[t.data_ptr() for t in tensors], B, N, d, h, d_ff, causal,
-                                     code, thresholds.data_ptr(),
-                                     bm.data_ptr() if bm is not None else None,
-                                     kp.data_ptr() if kp is not None else None,
-                                     out.data_ptr(), workspace.data_ptr(), workspace.numel(),
-                                     s.cuda_stream)
+    st = _lib.bpt_layer_forward_bsfa_opt(*[t.data_ptr() for t in tensors], B, N, d, h, d_ff,
+                                         causal, code, thresholds.data_ptr(),
+                                         bm.data_ptr() if bm is not None else None,
+                                         kp.data_ptr() if kp is not None else None,
+                                         out.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                         opts, s.cuda_stream)
     if st != _lib.BPT_OK:
         raise _lib.BptError(st, "bpt_layer_forward_bsfa")
     return out, bm, kp, workspace
@@ -170,7 +185,7 @@ GRAD_SHAPES = ["x", "ln1", "W_Q", "W_K", "W_V", "W_O", "ln2", "W_1", "b_1", "W_2
 def layer_backward(x: torch.Tensor, p: Dict[str, torch.Tensor], h: int, causal: bool,
                    stats: torch.Tensor, dZ: torch.Tensor,
                    workspace: Optional[torch.Tensor] = None,
-                   stream: Optional[torch.cuda.Stream] = None):
+                   stream: Optional[torch.cuda.Stream] = None, opts=None):
     """Gradients via ``bpt_layer_backward``; returns (grads, workspace) with
     grads[name] fp32 for name in GRAD_SHAPES (ln1 / ln2 as [2, d]: d gamma;
     d beta).  x and p as for ``layer_forward`` (bf16 or fp32); stats from
@@ -187,7 +202,8 @@ def layer_backward(x: torch.Tensor, p: Dict[str, torch.Tensor], h: int, causal: 
     if stats.dtype != torch.float32 or dZ.dtype != torch.float32 or not dZ.is_contiguous():
         raise ValueError("stats and dZ must be contiguous fp32 CUDA tensors")
     if workspace is None:
-        st, nbytes = _lib.bpt_layer_backward_workspace_size(B, N, d, h, d_ff, causal, code)
+        st, nbytes = _lib.bpt_layer_backward_workspace_size_opt(B, N, d, h, d_ff, causal, code,
+                                                                opts)
         if st != _lib.BPT_OK:
             raise _lib.BptError(st, "bpt_layer_backward_workspace_size")
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
@@ -195,10 +211,11 @@ def layer_backward(x: torch.Tensor, p: Dict[str, torch.Tensor], h: int, causal: 
                             device=x.device) for k in GRAD_SHAPES}
     s = stream if stream is not None else torch.cuda.current_stream(x.device)
     order = ["x", "ln1", "W_Q", "W_K", "W_V", "W_O", "ln2", "W_1", "b_1", "W_2", "b_2"]
-    st = _lib.bpt_layer_backward(*[t.data_ptr() for t in tensors], stats.data_ptr(),
-                                 dZ.data_ptr(), B, N, d, h, d_ff, causal, code,
-                                 *[grads[k].data_ptr() for k in order],
-                                 workspace.data_ptr(), workspace.numel(), s.cuda_stream)
+    st = _lib.bpt_layer_backward_opt(*[t.data_ptr() for t in tensors], stats.data_ptr(),
+                                     dZ.data_ptr(), B, N, d, h, d_ff, causal, code,
+                                     *[grads[k].data_ptr() for k in order],
+                                     workspace.data_ptr(), workspace.numel(), opts,
+                                     s.cuda_stream)
     if st != _lib.BPT_OK:
         raise _lib.BptError(st, "bpt_layer_backward")
     return grads, workspace

@@ -17,13 +17,25 @@
  * W_O carry no bias.
  *
  * How it is computed: blockwise, as the pages' two-level loop.  The outer loop
- * over query blocks of b rows (b = 128 for bf16, 64 for fp32) runs in waves of
- * at most BPT_WAVE_BLOCKS concurrent blocks; for each wave the kernels run
- * exact blockwise attention with an online softmax (causal blocks j > i are
- * skipped), then W_O + residual, LN2, W_1 + b_1 + GELU and W_2 + b_2 +
- * residual for the wave's rows only.  Neither the [N, N] scores nor the
- * [N, d_ff] FFN hidden state ever exists; the only sequence-shaped buffers are
- * x, out and the Q/K/V projection in the workspace.
+ * runs over query blocks of b rows (b = 128 for bf16, 64 for fp32).  For
+ * BPT_BF16 layers (default schedule, BPT_SCHEDULE_FUSED): after LN1 and the
+ * Q/K/V projection, one kernel runs exact blockwise attention with an online
+ * softmax (causal blocks j > i are skipped) for every query block and writes
+ * each block's output over that block's own queries; then one persistent
+ * kernel takes the query blocks two at a time and, per block, forms
+ * y = x + o W_O, LN2(y), the FFN hidden chunk by chunk (256 columns of d_ff
+ * at a time) and Z = y + FFN + b_2, with the hidden of the blocks in flight
+ * in a per-SM-pair scratch.  What exists at once:
+ *   - never: the [N, N] scores;
+ *   - sequence-shaped: x, out and the Q/K/V projection (workspace);
+ *   - block-shaped: LN2(y) and the FFN hidden of at most
+ *     2 * BPT_TAIL_MAX_PAIRS query blocks (the blocks in flight), so the
+ *     [N, d_ff] hidden exists only when the whole layer has that few blocks
+ *     (B * ceil(N / 128) <= 148).
+ * BPT_SCHEDULE_WAVES (and every BPT_F32 layer) runs the body instead in
+ * waves of at most BPT_WAVE_BLOCKS query blocks, five stream-ordered kernels
+ * per wave, with the wave's o, LN2(y) and hidden in the workspace: the
+ * [N, d_ff] hidden exists at once whenever B * ceil(N / b) <= BPT_WAVE_BLOCKS.
  *
  * Conventions shared by every entry point:
  *   - All pointers except `bytes` and the profile arrays are DEVICE pointers
@@ -65,8 +77,57 @@ typedef enum {
 /* Same object as cudaStream_t; 0 is the legacy default stream. */
 typedef struct CUstream_st* bpt_stream_t;
 
-/* Maximum query blocks processed concurrently (one wave of the outer loop). */
+/* Maximum query blocks processed concurrently by one wave of the waves
+ * schedule (BPT_SCHEDULE_WAVES, and every BPT_F32 layer). */
 #define BPT_WAVE_BLOCKS 256
+/* CTA pairs (two SMs each) of the fused schedule's layer-body kernel; each
+ * pair has two 128-row query blocks in flight. */
+#define BPT_TAIL_MAX_PAIRS 74
+
+/* Schedules of the layer body after attention (bpt_options.schedule). */
+enum {
+  BPT_SCHEDULE_FUSED = 0, /* default: one persistent kernel, block-shaped scratch */
+  BPT_SCHEDULE_WAVES = 1  /* waves of query blocks, one kernel per step per wave */
+};
+
+/*
+ * bpt_options -- per-call choices of the *_opt entry points.  A NULL pointer,
+ * or a zero-initialised struct, means the defaults.  Every choice gives the
+ * same result up to the order of fp32 sums; the ones marked "bitwise" give
+ * bitwise the same output.
+ *   schedule  BPT_SCHEDULE_FUSED or BPT_SCHEDULE_WAVES (bitwise: both run
+ *             the same per-element arithmetic).  BPT_F32 layers always use
+ *             waves.  The backward pass always uses waves.
+ *   attn_qpc  query blocks per attention CTA: 0 = default (2), 1 or 2
+ *             (bitwise).  2 pairs two 128-row query blocks in one CTA, so
+ *             each K/V tile brought in serves 256 query rows ("Blockwise
+ *             Parallel Transformer — BPT", section "Choosing the block size:
+ *             arithmetic intensity": FLOPs per byte re-read equal the rows
+ *             sharing it); 1 gives every query block its own CTA.
+ *   max_wave  waves schedule only: query blocks per wave, 0 = default
+ *             (BPT_WAVE_BLOCKS), else 1..BPT_WAVE_BLOCKS; small values make
+ *             small layers run the multi-wave paths (a sequence split over
+ *             several waves).  Workspace sizes depend on it: query them with
+ *             the same options.
+ *   fault     TEST HOOK for the failure-detection path (BPT_BF16 forward
+ *             only), 0 = none.  1: the QKV GEMM's CTA 0 never loads its first
+ *             stage; 2: the attention's CTA 0 never loads V_0; 3 (fused
+ *             schedule): the layer-body kernel's CTA 0 never loads its first
+ *             A tile.  The wait for
+ *             the missing load runs out (about 2 s), the kernel records
+ *             BPT_ERR_TIMEOUT in the device error word, drains what it issued,
+ *             frees its tensor memory and exits; `out` is garbage for that
+ *             call and the context stays usable.
+ *   reserved  must be 0.
+ * Returns BPT_ERR_INVALID_ARG for any other value.
+ */
+typedef struct {
+  int32_t schedule;
+  int32_t attn_qpc;
+  int64_t max_wave;
+  int32_t fault;
+  int32_t reserved;
+} bpt_options;
 
 /*
  * bpt_layer_workspace_size -- device workspace bytes bpt_layer_forward needs.
@@ -76,16 +137,24 @@ typedef struct CUstream_st* bpt_stream_t;
  *   weights        BPT_BF16 only: fp16 copies of W_Q, W_K, W_V, W_O ([d, d]
  *                  each), W_1 [d, d_ff], W_2 [d_ff, d], in that order
  *   QKV            [B*N, 3d] (Q | K | V per row); fp16 for BPT_BF16, fp32
- *                  for BPT_F32 (the "operand type" below)
- *   block scratch  P*b rows of o [d], LN2(y) [d] and FFN hidden [d_ff], in
- *                  the operand type, P = blocks in the largest wave
- *                  (<= BPT_WAVE_BLOCKS)
- * The scratch term does not grow with N once B*ceil(N/b) >= BPT_WAVE_BLOCKS.
+ *                  for BPT_F32 (the "operand type" below).  The fused
+ *                  schedule writes each row's attention output over its Q.
+ *   block scratch  fused schedule: 256*P rows of LN2(y) [d] and FFN hidden
+ *                  [d_ff] (fp16), P = min(BPT_TAIL_MAX_PAIRS, ceil(B*nb/2)),
+ *                  nb = ceil(N / 128): at most 148*128*(2d + 2 d_ff) bytes,
+ *                  for every N.  Waves schedule: P*b rows of o [d], LN2(y)
+ *                  [d] and FFN hidden [d_ff] in the operand type, P = blocks
+ *                  in the largest wave (<= BPT_WAVE_BLOCKS).
  * Returns BPT_ERR_INVALID_ARG for bytes == NULL or negative / inconsistent
  * sizes, BPT_ERR_UNSUPPORTED for shapes bpt_layer_forward rejects.
+ * bpt_layer_workspace_size_opt: the same for the given options (NULL: the
+ * defaults, as bpt_layer_workspace_size).
  */
 bpt_status bpt_layer_workspace_size(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff,
                                     int causal, bpt_dtype dtype, size_t* bytes);
+bpt_status bpt_layer_workspace_size_opt(int64_t B, int64_t N, int64_t d, int64_t h,
+                                        int64_t d_ff, int causal, bpt_dtype dtype,
+                                        const bpt_options* opts, size_t* bytes);
 
 /*
  * bpt_layer_forward -- Z = layer(x), written to `out`.
@@ -125,6 +194,22 @@ bpt_status bpt_layer_forward(const void* x, const void* ln1, const void* W_Q, co
                              int64_t N, int64_t d, int64_t h, int64_t d_ff, int causal,
                              bpt_dtype dtype, float* out, void* workspace, size_t workspace_bytes,
                              bpt_stream_t stream);
+
+/*
+ * bpt_layer_forward_opt -- bpt_layer_forward with per-call options (see
+ * bpt_options; NULL = the defaults) and optional statistics: `stats` NULL is
+ * bpt_layer_forward, non-NULL is bpt_layer_forward_train (same layout and
+ * rules).  The workspace must be at least bpt_layer_workspace_size_opt with
+ * the same options.
+ */
+bpt_status bpt_layer_forward_opt(const void* x, const void* ln1, const void* W_Q,
+                                 const void* W_K, const void* W_V, const void* W_O,
+                                 const void* ln2, const void* W_1, const void* b_1,
+                                 const void* W_2, const void* b_2, int64_t B, int64_t N,
+                                 int64_t d, int64_t h, int64_t d_ff, int causal, bpt_dtype dtype,
+                                 float* out, float* stats, void* workspace,
+                                 size_t workspace_bytes, const bpt_options* opts,
+                                 bpt_stream_t stream);
 
 /*
  * bpt_layer_forward_train -- bpt_layer_forward that also writes the per-row
@@ -195,6 +280,16 @@ bpt_status bpt_layer_forward_bsfa(const void* x, const void* ln1, const void* W_
                                   bpt_dtype dtype, const float* thresholds, float* block_max,
                                   uint8_t* kept, float* out, void* workspace,
                                   size_t workspace_bytes, bpt_stream_t stream);
+/* bpt_layer_forward_bsfa with per-call options (bpt_options; NULL = defaults). */
+bpt_status bpt_layer_forward_bsfa_opt(const void* x, const void* ln1, const void* W_Q,
+                                      const void* W_K, const void* W_V, const void* W_O,
+                                      const void* ln2, const void* W_1, const void* b_1,
+                                      const void* W_2, const void* b_2, int64_t B, int64_t N,
+                                      int64_t d, int64_t h, int64_t d_ff, int causal,
+                                      bpt_dtype dtype, const float* thresholds, float* block_max,
+                                      uint8_t* kept, float* out, void* workspace,
+                                      size_t workspace_bytes, const bpt_options* opts,
+                                      bpt_stream_t stream);
 
 /*
  * bpt_layer_backward_workspace_size -- device workspace bytes
@@ -204,6 +299,9 @@ bpt_status bpt_layer_forward_bsfa(const void* x, const void* ln1, const void* W_
 bpt_status bpt_layer_backward_workspace_size(int64_t B, int64_t N, int64_t d, int64_t h,
                                              int64_t d_ff, int causal, bpt_dtype dtype,
                                              size_t* bytes);
+bpt_status bpt_layer_backward_workspace_size_opt(int64_t B, int64_t N, int64_t d, int64_t h,
+                                                 int64_t d_ff, int causal, bpt_dtype dtype,
+                                                 const bpt_options* opts, size_t* bytes);
 
 /*
  * bpt_layer_backward -- gradients of sum(Z * dZ) with respect to x and every
@@ -249,14 +347,29 @@ bpt_status bpt_layer_backward(const void* x, const void* ln1, const void* W_Q, c
                               float* dW_O, float* d_ln2, float* dW_1, float* db_1, float* dW_2,
                               float* db_2, void* workspace, size_t workspace_bytes,
                               bpt_stream_t stream);
+/* bpt_layer_backward with per-call options (attn_qpc and max_wave apply; the
+ * backward always runs the waves schedule; fault must be 0). */
+bpt_status bpt_layer_backward_opt(const void* x, const void* ln1, const void* W_Q,
+                                  const void* W_K, const void* W_V, const void* W_O,
+                                  const void* ln2, const void* W_1, const void* b_1,
+                                  const void* W_2, const void* b_2, const float* stats,
+                                  const float* dZ, int64_t B, int64_t N, int64_t d, int64_t h,
+                                  int64_t d_ff, int causal, bpt_dtype dtype, float* dx,
+                                  float* d_ln1, float* dW_Q, float* dW_K, float* dW_V,
+                                  float* dW_O, float* d_ln2, float* dW_1, float* db_1,
+                                  float* dW_2, float* db_2, void* workspace,
+                                  size_t workspace_bytes, const bpt_options* opts,
+                                  bpt_stream_t stream);
 
 /*
  * bpt_read_device_error -- synchronises `stream`, reads and clears the error
- * word in the workspace header (written by the latest bpt_layer_forward on
- * this workspace).  Returns BPT_OK if nothing was recorded, BPT_ERR_TIMEOUT if
- * a kernel gave up waiting, BPT_ERR_RANGE if an fp16 operand overflowed
- * (*site, if non-NULL, receives the code of the place that recorded it), or
- * BPT_ERR_CUDA if synchronisation failed.
+ * word in the workspace header (written by the latest call on this
+ * workspace).  workspace == NULL reads the header of the array that
+ * bpt_layer_forward_static uses as its workspace, on the current device.
+ * Returns BPT_OK if nothing was recorded, BPT_ERR_TIMEOUT if a kernel gave up
+ * waiting, BPT_ERR_RANGE if an fp16 operand overflowed (*site, if non-NULL,
+ * receives the code of the place that recorded it), or BPT_ERR_CUDA if
+ * synchronisation failed.
  */
 bpt_status bpt_read_device_error(void* workspace, bpt_stream_t stream, uint32_t* site);
 
@@ -279,69 +392,36 @@ enum {
   BPT_KIND_LN2 = 4,
   BPT_KIND_W1 = 5,
   BPT_KIND_W2 = 6,
-  BPT_KIND_CVT = 7, /* bf16 -> fp16 weight copy */
-  BPT_KIND_COUNT = 8
+  BPT_KIND_CVT = 7,  /* bf16 -> fp16 weight copy */
+  BPT_KIND_TAIL = 8, /* fused schedule: W_O, LN2, W_1, W_2 in one kernel */
+  BPT_KIND_COUNT = 9
 };
 bpt_status bpt_profile_enable(int enable);
 bpt_status bpt_profile_read(double* ms, int64_t* launches, int n);
 
-/*
- * bpt_debug_set_max_wave -- TEST HOOK: caps the query blocks of a wave at
- * `blocks` (1..BPT_WAVE_BLOCKS; 0 restores BPT_WAVE_BLOCKS) for the calls
- * that follow, so that small layers exercise the multi-wave paths (a
- * sequence split over several waves, or one sequence per wave).  Results
- * are the same up to the order of fp32 sums; workspace sizes must be queried
- * after the call.  Returns BPT_ERR_INVALID_ARG outside that range.
- */
-bpt_status bpt_debug_set_max_wave(int64_t blocks);
-
-/*
- * bpt_debug_set_attn_qpc -- TUNING HOOK: query blocks per attention CTA for
- * the calls that follow.  2 (the default) pairs two 128-row query blocks in
- * one CTA, so each K/V tile brought in from L2 serves 256 query rows; 1
- * gives every query block its own CTA.  ("Blockwise Parallel Transformer —
- * BPT", section "Choosing the block size: arithmetic intensity": the FLOPs
- * done per byte re-read equal the rows a block shares them over; the pages
- * state it for the FFN weights, and the same ratio holds for the K/V tiles
- * each query block re-reads, 4 b d_k FLOPs per 4 d_k bytes of K and V per
- * key.)  Outputs are bitwise the same either way: a query block's
- * arithmetic does not depend on its partner.  Returns BPT_ERR_INVALID_ARG
- * for any other value.
- */
-bpt_status bpt_debug_set_attn_qpc(int qpc);
-
-/*
- * bpt_debug_inject_fault -- TEST HOOK for the failure-detection path.  The
- * next BPT_BF16 bpt_layer_forward makes one CTA skip one TMA load, so that
- * the wait for it runs out (after about 2 s) instead of completing:
- *   code 1: the QKV GEMM's CTA 0 never loads its first stage;
- *   code 2: the first attention wave's CTA 0 never loads V_0.
- * The kernel then records BPT_ERR_TIMEOUT in the device error word, drains
- * the loads and tensor-core work it did issue, frees its tensor memory and
- * exits; the layer's output is garbage for that call and the context stays
- * usable.  code 0 cancels.  The hook is consumed by one forward call.
- * Returns BPT_ERR_INVALID_ARG for other codes.
- */
-bpt_status bpt_debug_inject_fault(int code);
-
-/* Kernel launches one bpt_layer_forward call makes for these sizes. */
+/* Kernel launches one bpt_layer_forward call makes for these sizes (_opt:
+ * with those options). */
 bpt_status bpt_layer_launch_count(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff,
                                   int causal, bpt_dtype dtype, int64_t* launches);
+bpt_status bpt_layer_launch_count_opt(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff,
+                                      int causal, bpt_dtype dtype, const bpt_options* opts,
+                                      int64_t* launches);
 
 /*
  * bpt_layer_forward_static -- bpt_layer_forward for callers that cannot
  * allocate device memory.  The paper has no counterpart: this is a deployment
  * convenience of this library, not part of the method.
  *
- * Some callers are not allowed to allocate: code that runs while its stream is
- * being captured into a CUDA graph (an allocation may synchronise the device
- * and break the capture), plug-ins whose host framework owns all device memory,
- * and latency-critical loops that cannot pay for an allocation.  This entry
- * point takes the same arguments as bpt_layer_forward minus the workspace and
- * uses instead a workspace of BPT_STATIC_WORKSPACE_BYTES that lives in a
- * file-scope __device__ array of the library.  The caller still provides x,
- * the parameters and out.  It calls no cudaMalloc, cudaFree or other
- * allocating routine.
+ * Some callers are not allowed to allocate device memory: plug-ins and
+ * extensions whose host framework owns all device memory and hands out only
+ * the tensors of a call, embedded or real-time deployments that reserve
+ * memory once at start-up and forbid later allocation, and latency-critical
+ * loops that cannot pay for an allocation (it may synchronise the device).
+ * This entry point takes the same arguments as bpt_layer_forward minus the
+ * workspace and uses instead a workspace of BPT_STATIC_WORKSPACE_BYTES that
+ * lives in a file-scope __device__ array of the library.  The caller still
+ * provides x, the parameters and out.  It calls no cudaMalloc, cudaFree or
+ * other allocating routine.
  *
  *   - Size limit: layers whose bpt_layer_workspace_size exceeds
  *     BPT_STATIC_WORKSPACE_BYTES are rejected with BPT_ERR_WORKSPACE before
@@ -350,8 +430,8 @@ bpt_status bpt_layer_launch_count(int64_t B, int64_t N, int64_t d, int64_t h, in
  *   - Memory: every GPU that loads the library holds the array until the
  *     process exits, whether or not this entry point is used.
  *   - First call on a device: it looks up the array's device address (once
- *     per device, with that device current).  Make that first call before any
- *     stream capture begins.
+ *     per device and CUDA context, with that device current).  Make that
+ *     first call before any stream capture begins.
  *   - Sharing: all calls on a device use the same array, and it keeps the
  *     last call's contents (each call clears the header it needs).  Calls
  *     whose work overlaps on the GPU (different streams, no ordering) race on
@@ -359,8 +439,12 @@ bpt_status bpt_layer_launch_count(int64_t B, int64_t N, int64_t d, int64_t h, in
  *     events.
  *   - Profiling: returns BPT_ERR_INVALID_ARG while bpt_profile_enable is on
  *     (profiling creates event objects).
- *   - A kernel that gives up waiting records it in the array's header, which
- *     the caller cannot read; as with any timeout, `out` is then undefined.
+ *   - Device errors (a wait that ran out, BPT_ERR_TIMEOUT; an fp16 operand
+ *     beyond +-65504, BPT_ERR_RANGE, which large bf16 inputs or weights can
+ *     cause) are recorded in the array's header: read them with
+ *     bpt_read_device_error(NULL, stream, &site).  `out` is undefined after
+ *     either.
+ * The result is bitwise that of bpt_layer_forward with default options.
  */
 #define BPT_STATIC_WORKSPACE_BYTES (64u * 1024u * 1024u)
 bpt_status bpt_layer_forward_static(const void* x, const void* ln1, const void* W_Q,

@@ -20,13 +20,14 @@ def tol_for(cfg: LayerShape):
     return TOL_F32 if cfg.dtype == "f32" else TOL_BF16
 
 
-def run_cuda(cfg: LayerShape, inp=None, B=None):
-    """One forward through bpt_layer_forward; returns (Z float32 numpy, dev, ws)."""
+def run_cuda(cfg: LayerShape, inp=None, B=None, opts=None):
+    """One forward through bpt_layer_forward (bpt_layer_forward_opt with
+    ``opts``); returns (Z float32 numpy, dev, ws)."""
     if inp is None:
         inp = make_inputs(cfg, B=B)
     dev = bpt.to_device(inp, cfg.dtype)
     x = dev["x"]
-    out, ws = bpt.layer_forward(x, dev, cfg.h, cfg.causal)
+    out, ws = bpt.layer_forward(x, dev, cfg.h, cfg.causal, opts=opts)
     st, site = bpt.bpt_read_device_error(ws.data_ptr(), torch.cuda.current_stream().cuda_stream)
     assert st == bpt.BPT_OK, f"device error {bpt.status_string(st)} at site {site}"
     return out.float().cpu().numpy(), dev, ws

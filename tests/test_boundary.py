@@ -71,13 +71,36 @@ def test_workspace_null_out_pointer(lib):
 
 
 def test_workspace_is_block_shaped():
-    """Beyond the QKV projection (3 B N d elements) the workspace does not grow
-    with N once a wave is full, and never exceeds that bound."""
+    """Fused schedule: beyond the fp16 weights and the QKV projection (3 B N d
+    elements) the workspace is at most 148 query blocks x b x (2d + 2 d_ff)
+    bytes (LN2(y) and the FFN hidden of the blocks in flight) for EVERY N,
+    and constant once the layer has that many blocks."""
+    d, h, d_ff = 2048, 16, 8192
+    weights = (4 * d * d + 2 * d * d_ff) * 2
+    bound = 2 * bpt.BPT_TAIL_MAX_PAIRS * 128 * (2 * d + 2 * d_ff)
+    extra = {}
+    for B, N in ((1, 128), (1, 1000), (1, 8192), (1, 16384), (1, 32768), (1, 65536),
+                 (1, 131072), (4, 65536), (64, 2048)):
+        st, nbytes = bpt.bpt_layer_workspace_size(B, N, d, h, d_ff, 1, BF)
+        assert st == bpt.BPT_OK
+        e = nbytes - 3 * B * N * d * 2 - weights
+        assert 0 < e <= bound + 4096, (B, N, e)
+        blocks = B * ((N + 127) // 128)
+        # never more than the blocks the layer has (2 per CTA pair, rounded up)
+        assert e <= ((blocks + 1) // 2) * 256 * (2 * d + 2 * d_ff) + 4096, (B, N, e)
+        extra[(B, N)] = e
+    full = [e for (B, N), e in extra.items() if B * N >= 128 * 148]
+    assert max(full) - min(full) <= 4096           # alignment slack only
+
+
+def test_waves_workspace_is_wave_shaped():
+    """Waves schedule: the scratch stops growing with N once a wave is full."""
     d, h, d_ff = 2048, 16, 8192
     weights = (4 * d * d + 2 * d * d_ff) * 2
     extra = []
     for N in (8192, 16384, 32768, 65536, 131072):
-        st, nbytes = bpt.bpt_layer_workspace_size(1, N, d, h, d_ff, 1, BF)
+        st, nbytes = bpt.bpt_layer_workspace_size_opt(1, N, d, h, d_ff, 1, BF,
+                                                      {"schedule": "waves"})
         assert st == bpt.BPT_OK
         extra.append(nbytes - 3 * N * d * 2 - weights)
     full = extra[2:]
@@ -87,10 +110,32 @@ def test_workspace_is_block_shaped():
     assert max(full) <= bound + 8192
 
 
+def test_options_validation():
+    ok = bpt.bpt_layer_workspace_size_opt
+    args = (1, 1024, 256, 2, 512, 1, BF)
+    assert ok(*args, None)[0] == bpt.BPT_OK
+    assert ok(*args, None) == bpt.bpt_layer_workspace_size(*args)
+    assert ok(*args, {})[1] == ok(*args, None)[1]            # zeroed struct = defaults
+    for bad in ({"schedule": 2}, {"schedule": -1}, {"attn_qpc": 3}, {"max_wave": -1},
+                {"max_wave": bpt.BPT_WAVE_BLOCKS + 1}, {"fault": 4}, {"reserved": 1}):
+        assert ok(*args, bad)[0] == bpt.BPT_ERR_INVALID_ARG, bad
+    # the wave size only shapes the waves schedule's scratch
+    assert ok(*args, {"max_wave": 2})[1] == ok(*args, None)[1]
+    assert (ok(*args, {"schedule": "waves", "max_wave": 2})[1]
+            < ok(*args, {"schedule": "waves"})[1])
+    # fp32 layers ignore the schedule
+    f = (1, 256, 64, 1, 256, 0, F32)
+    assert ok(*f, {"schedule": "waves"}) == ok(*f, None)
+
+
 def test_launch_count():
+    # fused: weight copy, LN1, QKV, attention, layer body
     st, n = bpt.bpt_layer_launch_count(1, 65536, 2048, 16, 8192, 1, BF)
+    assert st == bpt.BPT_OK and n == 5
+    waves = {"schedule": "waves"}
+    st, n = bpt.bpt_layer_launch_count_opt(1, 65536, 2048, 16, 8192, 1, BF, waves)
     assert st == bpt.BPT_OK and n == 3 + 5 * 2   # weight copy, LN1, QKV; two waves
-    st, n = bpt.bpt_layer_launch_count(8, 2048, 768, 12, 3072, 1, BF)
+    st, n = bpt.bpt_layer_launch_count_opt(8, 2048, 768, 12, 3072, 1, BF, waves)
     assert st == bpt.BPT_OK and n == 3 + 5      # one wave of 8 sequences
     st, n = bpt.bpt_layer_launch_count(1, 256, 64, 1, 256, 0, F32)
     assert st == bpt.BPT_OK and n == 2 + 5      # fp32: no weight copy
@@ -132,6 +177,26 @@ def test_forward_rejects_aliasing_out_and_x():
     assert fwd(p) == bpt.BPT_ERR_INVALID_ARG
 
 
+@pytest.mark.parametrize("i", range(1, 11))
+def test_forward_rejects_out_or_workspace_over_any_parameter(i):
+    """out and the workspace are written while every parameter is still read."""
+    p = list(GOOD)
+    p[11] = p[i] + 16          # out starting inside parameter i
+    assert fwd(p) == bpt.BPT_ERR_INVALID_ARG
+    p = list(GOOD)
+    p[i] = p[12] + 4096        # parameter i inside the workspace
+    assert fwd(p) == bpt.BPT_ERR_INVALID_ARG
+
+
+def test_forward_rejects_workspace_over_x_or_out():
+    p = list(GOOD)
+    p[12] = p[0] + 1024        # workspace starting inside x
+    assert fwd(p) == bpt.BPT_ERR_INVALID_ARG
+    p = list(GOOD)
+    p[12] = p[11] + 1024       # workspace starting inside out
+    assert fwd(p) == bpt.BPT_ERR_INVALID_ARG
+
+
 def test_forward_rejects_unsupported_shapes():
     assert fwd(GOOD, d=96, h=3) == bpt.BPT_ERR_UNSUPPORTED
     assert fwd(GOOD, d=100, h=3) == bpt.BPT_ERR_INVALID_ARG
@@ -142,9 +207,14 @@ def test_forward_empty_is_a_no_op():
     assert fwd([None] * 13, N=0) == bpt.BPT_OK
 
 
-def test_read_error_rejects_null():
+def test_read_error_null_means_the_static_array():
+    """NULL selects the allocation-free entry point's array; with no GPU its
+    address cannot be looked up, which is reported, not dereferenced."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("covered by the GPU test of the allocation-free entry point")
     st, _ = bpt.bpt_read_device_error(None, None)
-    assert st == bpt.BPT_ERR_INVALID_ARG
+    assert st == bpt.BPT_ERR_CUDA
 
 
 def test_library_has_no_host_fallback_symbols(lib):

@@ -38,12 +38,14 @@ def upstream(cfg, seed=77):
     return np.random.default_rng(seed).standard_normal((cfg.B, cfg.N, cfg.d)).astype(np.float32)
 
 
-def run_backward(cfg, inp, dZ):
+def run_backward(cfg, inp, dZ, max_wave=0):
     dev = bpt.to_device(inp, cfg.dtype)
     x = dev["x"]
-    _, stats, ws = bpt.layer_forward_train(x, dev, cfg.h, cfg.causal)
+    fwd_opts = {"schedule": "waves", "max_wave": max_wave} if max_wave else None
+    _, stats, ws = bpt.layer_forward_train(x, dev, cfg.h, cfg.causal, opts=fwd_opts)
     grads, bws = bpt.layer_backward(x, dev, cfg.h, cfg.causal, stats,
-                                    torch.from_numpy(dZ).cuda())
+                                    torch.from_numpy(dZ).cuda(),
+                                    opts={"max_wave": max_wave} if max_wave else None)
     for w in (ws, bws):
         st, site = bpt.bpt_read_device_error(w.data_ptr(), torch.cuda.current_stream().cuda_stream)
         assert st == bpt.BPT_OK, f"device error {bpt.status_string(st)} at site {site}"
@@ -74,7 +76,7 @@ def test_backward_matches_oracle(cfg):
         check(k + ".beta", got[k][1], want[b])
 
 
-# Multi-wave schedules on small layers (bpt_debug_set_max_wave): a sequence
+# Multi-wave schedules on small layers (bpt_options.max_wave): a sequence
 # split over three waves, and one whole sequence per wave.
 WAVE_CASES = [
     (small("bwd_split_sequence", 1, 700, 256, 2, 512, True, seed=25), 2),
@@ -85,13 +87,9 @@ WAVE_CASES = [
 
 @pytest.mark.parametrize("cfg,blocks", WAVE_CASES, ids=lambda c: getattr(c, "name", str(c)))
 def test_backward_multi_wave(cfg, blocks):
-    assert bpt.bpt_debug_set_max_wave(blocks) == bpt.BPT_OK
-    try:
-        inp = make_inputs(cfg)
-        dZ = upstream(cfg)
-        got = run_backward(cfg, inp, dZ)
-    finally:
-        bpt.bpt_debug_set_max_wave(0)
+    inp = make_inputs(cfg)
+    dZ = upstream(cfg)
+    got = run_backward(cfg, inp, dZ, max_wave=blocks)
     want = oracle.layer_backward(inp, cfg.h, cfg.causal, dZ.astype(np.float64))
     for k in NAMES:
         check(k, got[k], want[k])
@@ -146,13 +144,9 @@ def test_f32_backward_matches_oracle(cfg):
 
 def test_f32_backward_multi_wave():
     cfg = small("bwd_f32_split", 1, 300, 64, 2, 192, True, dtype="f32", seed=34)
-    assert bpt.bpt_debug_set_max_wave(2) == bpt.BPT_OK
-    try:
-        inp = make_inputs(cfg)
-        dZ = upstream(cfg)
-        got = run_backward(cfg, inp, dZ)
-    finally:
-        bpt.bpt_debug_set_max_wave(0)
+    inp = make_inputs(cfg)
+    dZ = upstream(cfg)
+    got = run_backward(cfg, inp, dZ, max_wave=2)
     want = oracle.layer_backward(inp, cfg.h, cfg.causal, dZ.astype(np.float64))
     for k in NAMES:
         check_f32(k, got[k], want[k])

@@ -52,10 +52,10 @@ def gap_thresholds(bmax, causal, rng):
     return T
 
 
-def run_bsfa(cfg, dev, T):
+def run_bsfa(cfg, dev, T, opts=None):
     out, bm, kp, ws = bpt.layer_forward_bsfa(dev["x"], dev, cfg.h, cfg.causal,
                                              torch.from_numpy(T.astype(np.float32)).cuda(),
-                                             block_max=True, kept=True)
+                                             block_max=True, kept=True, opts=opts)
     st, site = bpt.bpt_read_device_error(ws.data_ptr(), torch.cuda.current_stream().cuda_stream)
     assert st == bpt.BPT_OK, f"device error {bpt.status_string(st)} at site {site}"
     return out.cpu().numpy(), bm.cpu().numpy(), kp.cpu().numpy().astype(bool)
@@ -119,15 +119,8 @@ def test_gate_is_independent_of_pairing_and_waves():
     rng = np.random.default_rng(7)
     T = gap_thresholds(oracle.layer_block_max(inp, cfg.h, cfg.causal), cfg.causal, rng)
     base, _, kp0 = run_bsfa(cfg, dev, T)
-    try:
-        assert bpt.bpt_debug_set_attn_qpc(1) == bpt.BPT_OK
-        one, _, kp1 = run_bsfa(cfg, dev, T)
-        assert bpt.bpt_debug_set_attn_qpc(2) == bpt.BPT_OK
-        assert bpt.bpt_debug_set_max_wave(3) == bpt.BPT_OK
-        waves, _, kp2 = run_bsfa(cfg, dev, T)
-    finally:
-        bpt.bpt_debug_set_attn_qpc(2)
-        bpt.bpt_debug_set_max_wave(0)
+    one, _, kp1 = run_bsfa(cfg, dev, T, opts={"attn_qpc": 1})
+    waves, _, kp2 = run_bsfa(cfg, dev, T, opts={"schedule": "waves", "max_wave": 3})
     np.testing.assert_array_equal(one, base)
     np.testing.assert_array_equal(kp1, kp0)
     np.testing.assert_array_equal(kp2, kp0)

@@ -51,12 +51,19 @@ def test_pairing_is_bitwise_neutral_at_full_size(dev):
     x = dev["x"]
     out2, ws = bpt.layer_forward(x, dev, CFG.h, CFG.causal)
     out2 = out2.clone()
-    try:
-        assert bpt.bpt_debug_set_attn_qpc(1) == bpt.BPT_OK
-        out1, _ = bpt.layer_forward(x, dev, CFG.h, CFG.causal, workspace=ws)
-    finally:
-        bpt.bpt_debug_set_attn_qpc(2)
+    out1, _ = bpt.layer_forward(x, dev, CFG.h, CFG.causal, workspace=ws, opts={"attn_qpc": 1})
     assert torch.equal(out1, out2)
+
+
+def test_fused_schedule_is_bitwise_the_waves_schedule_at_full_size(dev):
+    """The persistent per-block tail and the wave-level kernels run the same
+    per-element arithmetic: bitwise equal layer outputs on the workload."""
+    x = dev["x"]
+    fused, _ = bpt.layer_forward(x, dev, CFG.h, CFG.causal)
+    fused = fused.clone()
+    waves, _ = bpt.layer_forward(x, dev, CFG.h, CFG.causal, opts={"schedule": "waves"})
+    assert torch.isfinite(fused).all()
+    assert torch.equal(fused, waves)
 
 
 def test_gating_without_thresholds_is_the_dense_forward_at_full_size(dev):

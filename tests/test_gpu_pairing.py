@@ -1,5 +1,5 @@
 """Query blocks per attention CTA: paired (256 query rows share each K/V tile,
-the default) against one block per CTA (bpt_debug_set_attn_qpc).
+the default) against one block per CTA (bpt_options.attn_qpc).
 
 "Blockwise Parallel Transformer — BPT", section "Choosing the block size:
 arithmetic intensity": the work done per byte re-read grows with the rows
@@ -28,30 +28,27 @@ CASES = [
 ]
 
 
-def forward_train(cfg, dev):
-    out, stats, ws = bpt.layer_forward_train(dev["x"], dev, cfg.h, cfg.causal)
+def forward_train(cfg, dev, opts):
+    out, stats, ws = bpt.layer_forward_train(dev["x"], dev, cfg.h, cfg.causal, opts=opts)
     st, site = bpt.bpt_read_device_error(ws.data_ptr(), torch.cuda.current_stream().cuda_stream)
     assert st == bpt.BPT_OK, f"device error {bpt.status_string(st)} at site {site}"
     return out.cpu().numpy(), stats.cpu().numpy()
 
 
+@pytest.mark.parametrize("schedule", ["fused", "waves"])
 @pytest.mark.parametrize("cfg,wave", CASES, ids=lambda c: getattr(c, "name", str(c)))
-def test_single_block_ctas_match_pairs_bitwise(cfg, wave):
+def test_single_block_ctas_match_pairs_bitwise(cfg, wave, schedule):
     dev = bpt.to_device(make_inputs(cfg), cfg.dtype)
-    assert bpt.bpt_debug_set_max_wave(wave) == bpt.BPT_OK
-    try:
-        assert bpt.bpt_debug_set_attn_qpc(2) == bpt.BPT_OK
-        out2, st2 = forward_train(cfg, dev)
-        assert bpt.bpt_debug_set_attn_qpc(1) == bpt.BPT_OK
-        out1, st1 = forward_train(cfg, dev)
-    finally:
-        bpt.bpt_debug_set_attn_qpc(2)
-        bpt.bpt_debug_set_max_wave(0)
+    base = {"schedule": schedule, "max_wave": wave if schedule == "waves" else 0}
+    out2, st2 = forward_train(cfg, dev, dict(base, attn_qpc=2))
+    out1, st1 = forward_train(cfg, dev, dict(base, attn_qpc=1))
     assert np.all(np.isfinite(out2))
     np.testing.assert_array_equal(out1, out2)
     np.testing.assert_array_equal(st1, st2)
 
 
 def test_qpc_rejects_other_values():
-    for bad in (0, 3, -1):
-        assert bpt.bpt_debug_set_attn_qpc(bad) == bpt.BPT_ERR_INVALID_ARG
+    for bad in (3, -1):
+        st, _ = bpt.bpt_layer_workspace_size_opt(1, 256, 256, 2, 512, True, bpt.BPT_BF16,
+                                                 {"attn_qpc": bad})
+        assert st == bpt.BPT_ERR_INVALID_ARG

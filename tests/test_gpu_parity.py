@@ -41,12 +41,45 @@ SMALL = [
 ]
 
 
+@pytest.mark.parametrize("schedule", ["fused", "waves"])
 @pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
-def test_small_layers_elementwise(cfg):
+def test_small_layers_elementwise(cfg, schedule):
+    if cfg.dtype == "f32" and schedule == "fused":
+        pytest.skip("fp32 layers always run the waves schedule")
     inp = make_inputs(cfg)
-    got, _, _ = run_cuda(cfg, inp)
+    got, _, _ = run_cuda(cfg, inp, opts={"schedule": schedule})
     want = oracle.layer_unfused(inp, cfg.h, cfg.causal)
     compare(got, want, tol_for(cfg))
+
+
+# The fused layer body (one persistent kernel, two query blocks per CTA pair)
+# against the wave kernels: the same per-element arithmetic, so bitwise equal.
+# Cases: an odd block count (a pair item with one block), ragged sequences in a
+# batch (an item whose two blocks belong to different sequences), d and d_ff
+# = 64 (mod 128), and more items than CTA pairs (each pair runs several items,
+# so every hand-off barrier goes through both phases).
+FUSED_CASES = [
+    small("fz_odd_blocks", 1, 640, 256, 2, 512, True, seed=51),
+    small("fz_ragged_batch", 3, 300, 256, 4, 512, False, seed=52, bias=0.5),
+    small("fz_straddle", 1, 260, 192, 3, 448, True, seed=53),
+    small("fz_many_items", 1, 128 * 301, 128, 2, 256, True, seed=54),
+    small("fz_many_items_batch", 7, 128 * 45 - 3, 256, 2, 320, True, seed=55),
+]
+
+
+@pytest.mark.parametrize("cfg", FUSED_CASES, ids=lambda c: c.name)
+def test_fused_schedule_is_bitwise_the_waves_schedule(cfg):
+    inp = make_inputs(cfg)
+    fused, _, _ = run_cuda(cfg, inp)
+    waves, _, _ = run_cuda(cfg, inp, opts={"schedule": "waves"})
+    assert np.all(np.isfinite(fused))
+    np.testing.assert_array_equal(fused, waves)
+    if cfg.B * cfg.N <= 4096:
+        compare(fused, oracle.layer_unfused(inp, cfg.h, cfg.causal), tol_for(cfg))
+    else:
+        rows = sample_rows(cfg, 64)
+        compare(fused[rows[:, 0], rows[:, 1]], oracle.layer_rows(inp, cfg.h, cfg.causal, rows),
+                tol_for(cfg))
 
 
 def test_tiny_f32_workload():
@@ -58,9 +91,10 @@ def test_tiny_f32_workload():
 
 @pytest.mark.parametrize("cfg", [SMALL[0], SMALL[2], SMALL[7], SMALL[8]], ids=lambda c: c.name)
 def test_qkv_projection_in_workspace(cfg):
-    """Step a2 alone: the Q/K/V rows the prologue GEMM wrote."""
+    """Step a2 alone: the Q/K/V rows the prologue GEMM wrote (waves schedule,
+    which keeps Q)."""
     inp = make_inputs(cfg)
-    _, _, ws = run_cuda(cfg, inp)
+    _, _, ws = run_cuda(cfg, inp, opts={"schedule": "waves"})
     qkv = workspace_qkv(ws, cfg, cfg.B)
     for b in range(cfg.B):
         it = oracle.layer_intermediates(inp, cfg.h, cfg.causal, b=b)
@@ -69,28 +103,45 @@ def test_qkv_projection_in_workspace(cfg):
         compare(qkv[b], want, tol)
 
 
-def test_deterministic():
+@pytest.mark.parametrize("cfg", [SMALL[0], SMALL[2], SMALL[7]], ids=lambda c: c.name)
+def test_attention_output_over_queries(cfg):
+    """Steps a3-a5 alone, fused schedule: each row's attention output o (heads
+    concatenated) stands where its Q was; K and V are untouched."""
+    inp = make_inputs(cfg)
+    _, _, ws = run_cuda(cfg, inp)
+    qkv = workspace_qkv(ws, cfg, cfg.B)
+    for b in range(cfg.B):
+        it = oracle.layer_intermediates(inp, cfg.h, cfg.causal, b=b)
+        compare(qkv[b, :, :cfg.d], it["O"], (2e-2, 2e-3))
+        compare(qkv[b, :, cfg.d:], np.concatenate([it["K"], it["V"]], axis=1), (2e-2, 2e-3))
+
+
+@pytest.mark.parametrize("schedule", ["fused", "waves"])
+def test_deterministic(schedule):
     cfg = SMALL[0]
     inp = make_inputs(cfg)
-    a, _, _ = run_cuda(cfg, inp)
-    b, _, _ = run_cuda(cfg, inp)
+    a, _, _ = run_cuda(cfg, inp, opts={"schedule": schedule})
+    b, _, _ = run_cuda(cfg, inp, opts={"schedule": schedule})
     np.testing.assert_array_equal(a, b)
 
 
-def test_several_waves_in_one_sequence():
-    """nb > BPT_WAVE_BLOCKS: the sequence is processed in several waves."""
+@pytest.mark.parametrize("schedule", ["fused", "waves"])
+def test_several_waves_in_one_sequence(schedule):
+    """nb > BPT_WAVE_BLOCKS: the sequence is processed in several waves (or,
+    fused, several items per CTA pair)."""
     cfg = small("waves", 1, 128 * 300, 128, 2, 256, True, seed=5)
     inp = make_inputs(cfg)
-    got, _, _ = run_cuda(cfg, inp)
+    got, _, _ = run_cuda(cfg, inp, opts={"schedule": schedule})
     rows = sample_rows(cfg, 96)
     want = oracle.layer_rows(inp, cfg.h, cfg.causal, rows)
     compare(got[rows[:, 0], rows[:, 1]], want, tol_for(cfg))
 
 
-def test_several_waves_of_whole_sequences():
+@pytest.mark.parametrize("schedule", ["fused", "waves"])
+def test_several_waves_of_whole_sequences(schedule):
     cfg = small("seqwaves", 5, 128 * 100, 128, 2, 256, True, seed=6)
     inp = make_inputs(cfg)
-    got, _, _ = run_cuda(cfg, inp)
+    got, _, _ = run_cuda(cfg, inp, opts={"schedule": schedule})
     rows = sample_rows(cfg, 96)
     want = oracle.layer_rows(inp, cfg.h, cfg.causal, rows)
     compare(got[rows[:, 0], rows[:, 1]], want, tol_for(cfg))

@@ -22,13 +22,16 @@ CFG = LayerShape("watchdog", B=1, N=512, d=256, h=2, d_ff=512, causal=True, dtyp
                  block=128, seed=41, ln_scale=0.1)
 
 
-@pytest.mark.parametrize("code", [1, 2], ids=["gemm_lost_stage", "attention_lost_v"])
-def test_lost_arrive_reports_timeout_and_context_survives(code):
+@pytest.mark.parametrize("code,schedule", [(1, "fused"), (2, "fused"), (3, "fused"),
+                                           (2, "waves")],
+                         ids=["gemm_lost_stage", "attention_lost_v", "tail_lost_stage",
+                              "waves_attention_lost_v"])
+def test_lost_arrive_reports_timeout_and_context_survives(code, schedule):
     inp = make_inputs(CFG)
     dev = bpt.to_device(inp, CFG.dtype)
     stream = torch.cuda.current_stream().cuda_stream
-    assert bpt.bpt_debug_inject_fault(code) == bpt.BPT_OK
-    out, ws = bpt.layer_forward(dev["x"], dev, CFG.h, CFG.causal)
+    opts = {"schedule": schedule, "fault": code}
+    out, ws = bpt.layer_forward(dev["x"], dev, CFG.h, CFG.causal, opts=opts)
     st, site = bpt.bpt_read_device_error(ws.data_ptr(), stream)
     assert st == bpt.BPT_ERR_TIMEOUT, bpt.status_string(st)
     assert site != 0
@@ -38,5 +41,7 @@ def test_lost_arrive_reports_timeout_and_context_survives(code):
 
 
 def test_fault_hook_rejects_unknown_codes():
-    assert bpt.bpt_debug_inject_fault(7) == bpt.BPT_ERR_INVALID_ARG
-    assert bpt.bpt_debug_inject_fault(0) == bpt.BPT_OK
+    for bad in (7, -1):
+        st, _ = bpt.bpt_layer_workspace_size_opt(1, 512, 256, 2, 512, True, bpt.BPT_BF16,
+                                                 {"fault": bad})
+        assert st == bpt.BPT_ERR_INVALID_ARG
