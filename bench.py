@@ -105,7 +105,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -245,7 +245,22 @@ def measure_bsfa(bpt, cfg, x, p, out_dense, ms_dense, stream, dev, args, world, 
                                            workspace=ws)
     vis = np.tril(np.ones((nb, nb), bool)) if cfg.causal else np.ones((nb, nb), bool)
     off = vis & ~np.eye(nb, dtype=bool)
-    kept_frac = float(kept.cpu().numpy()[:, :, off].mean()) if off.any() else 1.0
+    kp = kept.cpu().numpy().astype(bool)
+    kept_frac = float(kp[:, :, off].mean()) if off.any() else 1.0
+    # V tiles the gated kernel loads: a CTA's two query blocks (2q, 2q+1) share
+    # each V_j, loaded when either block that visits j keeps it
+    v_loaded = v_total = 0
+    for q0 in range(0, nb, 2):
+        rows = [i for i in (q0, q0 + 1) if i < nb]
+        for j in range(nb):
+            vis_rows = [i for i in rows if vis[i, j]]
+            if not vis_rows:
+                continue
+            any_keep = np.zeros(kp.shape[:2], bool)
+            for i in vis_rows:
+                any_keep |= kp[:, :, i, j]
+            v_loaded += int(any_keep.sum())
+            v_total += any_keep.size
     for _ in range(args.warmup):
         bpt.layer_forward_bsfa(x, p, cfg.h, cfg.causal, T, out=o2, workspace=ws)
     torch.cuda.synchronize(dev)
@@ -262,7 +277,10 @@ def measure_bsfa(bpt, cfg, x, p, out_dense, ms_dense, stream, dev, args, world, 
         raise SystemExit(f"device error in bsfa {bpt.status_string(st)} site {site}")
     ms = bdist.max_over_ranks(e0.elapsed_time(e1), dist, dev) / args.steps
     dev_max = float((o2 - out_dense).abs().max())
-    return {"k": args.bsfa_k, "kept_offdiag_frac": kept_frac, "ms_per_step": ms,
+    return {"k": args.bsfa_k, "kept_offdiag_frac": kept_frac,
+            "v_tiles_loaded_frac": v_loaded / max(1, v_total),
+            "v_bytes_skipped_per_forward": int((v_total - v_loaded) * 128 * cfg.d_k * 2),
+            "ms_per_step": ms,
             "tokens_per_s": cfg.B * cfg.N * world / (ms / 1e3),
             "speedup_vs_dense": ms_dense / ms, "max_abs_dev_vs_dense": dev_max,
             "max_abs_dense": float(out_dense.abs().max()), "steps": args.steps,
@@ -270,7 +288,8 @@ def measure_bsfa(bpt, cfg, x, p, out_dense, ms_dense, stream, dev, args, world, 
                            "of one other seeded synthetic x (same weights)",
             "note": "approximate attention (the pages' method): synthetic inputs have no "
                     "learned attention sparsity, so the deviation says nothing about model "
-                    "quality; V tiles of pruned blocks are still loaded"}
+                    "quality; a V tile is loaded only when a query block that visits it "
+                    "keeps the block"}
 
 
 # ------------------------------------------------- unfused peak bytes --
@@ -442,6 +461,72 @@ def other_workloads(bpt, args, names, stream, dev, peaks):
     return res
 
 
+def run_sequence_parallel(args, cfg, rank, world, dev, dist):
+    """One sequence split over the ranks (zig-zag chunks; per step: shard
+    projection, one NCCL all-gather of K | V into each GPU's own buffer,
+    shard attention + layer body).  Strong scaling: the whole job is one
+    pass over the workload's batch; value = its tokens / max-over-ranks time."""
+    import torch
+    import blockwise_attn_ffn_b200 as bpt
+    from blockwise_attn_ffn_b200 import dist as bdist
+    from blockwise_attn_ffn_b200 import shard
+    stream = torch.cuda.current_stream(dev)
+    inp = make_inputs(cfg)
+    p = bpt.to_device(inp, cfg.dtype, dev)
+    del inp
+    rows = torch.from_numpy(shard.token_rows(cfg.N, world, rank)).to(dev)
+    x_loc = p["x"][:, rows].contiguous()
+    x_host = x_loc.cpu().pin_memory()
+    del p["x"]
+    out, bufs = shard.sequence_parallel_forward(x_loc, p, cfg.h, cfg.causal, cfg.N, dist)
+    for _ in range(args.warmup):
+        shard.sequence_parallel_forward(x_loc, p, cfg.h, cfg.causal, cfg.N, dist, bufs=bufs)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            shard.sequence_parallel_forward(x_loc, p, cfg.h, cfg.causal, cfg.N, dist, bufs=bufs)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+    st, site = bpt.bpt_read_device_error(bufs["ws"].data_ptr(), stream.cuda_stream)
+    if st != bpt.BPT_OK:
+        raise SystemExit(f"device error {bpt.status_string(st)} site {site}")
+    ms = bdist.max_over_ranks(e0.elapsed_time(e1), dist, dev) / args.steps
+    # end to end: the rank's rows up from pinned host memory, its output down
+    host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    dist.barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        x_loc.copy_(x_host, non_blocking=True)
+        shard.sequence_parallel_forward(x_loc, p, cfg.h, cfg.causal, cfg.N, dist, bufs=bufs)
+        host_out.copy_(bufs["out"], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_e2e = bdist.max_over_ranks(e0.elapsed_time(e1), dist, dev) / args.steps
+    flops = accounting.layer_flops(cfg.B, cfg.N, cfg.d, cfg.h, cfg.d_ff, cfg.causal)
+    peaks, peak_src = load_peaks()
+    tokens = cfg.B * cfg.N
+    tf = flops["total"] / (ms / 1e3) / 1e12
+    kv_bytes = int(bufs["kv_loc"].numel() * 2)
+    return {
+        "metric": METRIC, "value": tokens / (ms / 1e3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic: seeded N(0,1) x, N(0,1/fan_in) weights, LN gamma~1+0.1N, beta~0.1N",
+        "config": dict(workload_config(cfg, 1), parallelism=f"sequence{world}",
+                       shard="zig-zag chunks r and 2G-1-r; one NCCL all-gather of K|V per step"),
+        "tflops": tf, "pct_bf16_peak": tf / world / peaks["bf16_tflops"], "peak_src": peak_src,
+        "allgather_bytes_per_rank": kv_bytes * (world - 1),
+        "gpu_launches": 5 * args.steps,
+        "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": int(x_loc.numel() * 2) * world,
+                "d2h_bytes_per_step": int(out.numel() * 4) * world, "ms_per_step": ms_e2e},
+        "clocks": clk.summary()}
+
+
 def relaunch_under_torchrun(args) -> int:
     """`bench.py --gpus N` started as a plain process: start the N ranks
     ourselves (one process per GPU) with the same arguments."""
@@ -488,6 +573,9 @@ def main():
                     help="skip timing the other four workloads")
     ap.add_argument("--no-alt-schedule", action="store_true",
                     help="skip timing the other schedule on the bench workload")
+    ap.add_argument("--parallel", default="data", choices=["data", "sequence"],
+                    help="several GPUs: each runs its own batch (data, weak scaling) or one "
+                         "sequence is split over them (sequence, strong scaling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -514,6 +602,13 @@ def main():
     if world > 1:
         bdist.init_process_group("nccl", device=dev)
     stream = torch.cuda.current_stream(dev)
+    if args.parallel == "sequence" and world > 1:
+        line = run_sequence_parallel(args, cfg, rank, world, dev, dist)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        dist.barrier()
+        dist.destroy_process_group()
+        return 0
 
     # Inputs: the workload's weights on every rank, a rank-seeded x each.
     inp = bdist.rank_inputs(cfg, rank)

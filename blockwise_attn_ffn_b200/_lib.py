@@ -33,6 +33,7 @@ EXPORTED = [
     "bpt_layer_workspace_size_opt", "bpt_layer_forward_opt", "bpt_layer_forward_bsfa_opt",
     "bpt_layer_backward_workspace_size_opt", "bpt_layer_backward_opt",
     "bpt_layer_launch_count_opt",
+    "bpt_layer_shard_workspace_size", "bpt_layer_shard_project", "bpt_layer_shard_forward",
 ]
 
 
@@ -117,6 +118,12 @@ def load() -> ctypes.CDLL:
     lib.bpt_layer_launch_count_opt.argtypes = [i64, i64, i64, i64, i64, i32, i32, op,
                                                ctypes.POINTER(ctypes.c_int64)]
     lib.bpt_layer_launch_count_opt.restype = i32
+    lib.bpt_layer_shard_workspace_size.argtypes = [i64] * 6 + [i32, i32,
+                                                               ctypes.POINTER(ctypes.c_size_t)]
+    lib.bpt_layer_shard_workspace_size.restype = i32
+    for fn in (lib.bpt_layer_shard_project, lib.bpt_layer_shard_forward):
+        fn.argtypes = [vp] * 11 + [i64] * 7 + [i32, i32, vp, vp, vp, ctypes.c_size_t, vp]
+        fn.restype = i32
     lib.bpt_read_device_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     lib.bpt_read_device_error.restype = i32
     lib.bpt_status_string.argtypes = [i32]
@@ -191,6 +198,29 @@ def bpt_layer_backward_opt(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, 
                                          dx, d_ln1, dW_Q, dW_K, dW_V, dW_O, d_ln2, dW_1, db_1,
                                          dW_2, db_2, workspace, workspace_bytes,
                                          _opts_ref(opts), stream)
+
+
+def bpt_layer_shard_workspace_size(B, N, G, d, h, d_ff, causal, dtype) -> Tuple[int, int]:
+    out = ctypes.c_size_t(0)
+    st = load().bpt_layer_shard_workspace_size(B, N, G, d, h, d_ff, int(bool(causal)), dtype,
+                                               ctypes.byref(out))
+    return st, out.value
+
+
+def bpt_layer_shard_project(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, B, N, G, rank,
+                            d, h, d_ff, causal, dtype, kv_loc, out, workspace, workspace_bytes,
+                            stream) -> int:
+    return load().bpt_layer_shard_project(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
+                                          B, N, G, rank, d, h, d_ff, int(bool(causal)), dtype,
+                                          kv_loc, out, workspace, workspace_bytes, stream)
+
+
+def bpt_layer_shard_forward(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, B, N, G, rank,
+                            d, h, d_ff, causal, dtype, kv_all, out, workspace, workspace_bytes,
+                            stream) -> int:
+    return load().bpt_layer_shard_forward(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
+                                          B, N, G, rank, d, h, d_ff, int(bool(causal)), dtype,
+                                          kv_all, out, workspace, workspace_bytes, stream)
 
 
 def bpt_layer_launch_count_opt(B, N, d, h, d_ff, causal, dtype, opts) -> Tuple[int, int]:

@@ -73,6 +73,13 @@ struct AttnPairParams {
   int fault;         // test hook: 2 = CTA 0 never loads V_0 (a lost arrive)
   int qpc;           // query blocks per CTA: 2 (a pair, 256 query rows sharing
                      // each K/V tile) or 1 (one 128-row block)
+  // Sequence shard (kernel instantiated with SHARD only).  The sequence of
+  // N_kv tokens is cut into 2G chunks of kv_cb query/key blocks; this rank
+  // owns chunks q_c0 and q_c1 (its local blocks 0..kv_cb-1 and kv_cb..2kv_cb-1).
+  // Q, o and the block indices above are local; keys come from the all-gathered
+  // K | V of every rank, [G][B][N / G][2d], where chunk c is held by rank
+  // c < G ? c : 2G-1-c as its local chunk c < G ? 0 : 1.
+  int kv_cb, q_c0, q_c1, kv_G, N_kv;
   // Block gating (kernel instantiated with GATE only):
   const float* gate_t;  // [h][nb] thresholds T in units of s = q.k / sqrt(d_k)
   float* gate_bmax;     // nullable [B][h][nb][nb]: s_max of each visited pair
@@ -192,17 +199,27 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
+// Global block of local query block i on a sequence shard.
+__device__ __forceinline__ int shard_global_block(const AttnPairParams& p, int i) {
+  return (i < p.kv_cb ? p.q_c0 : p.q_c1) * p.kv_cb + (i % p.kv_cb);
+}
+
 // GATE: block-sparse gating ("Block Sparse Flash Attention", sections
 // "Methodology and Mechanism" and "Gating Mechanism and Threshold
 // Calibration").  After S_X(j) the tile's four softmax warps reduce their
 // row maxima (valid query rows only) to the block maximum s_max; an
 // off-diagonal block with s_max < T[head, i] is pruned: no exponentials, no
 // change to (m, l), no PV product (the UMMA warp reads the tile's decision
-// after the P hand-over).  The K/V ring still loads V_j: it is fetched
-// before S_j exists, and with head-grouped CTAs it comes from L2.
-template <int D, int EMU, bool GATE = false>
+// after the P hand-over).  The ring then carries K one block ahead of V
+// (K_0 K_1 V_0 K_2 V_1 ...): the producer issues V_j only once the tiles that
+// visit block j have decided, at once if tile A keeps it, and completes the
+// slot without a load when every visiting tile prunes it, so pruned blocks
+// cost no V traffic ("Block Sparse Flash Attention", "Methodology and
+// Mechanism": a pruned block's values are neither loaded nor multiplied).
+template <int D, int EMU, bool GATE = false, bool SHARD = false>
 __global__ void __launch_bounds__(384, 1)
-    attn_pair_tc_kernel(const __grid_constant__ CUtensorMap mapQKV, const AttnPairParams p) {
+    attn_pair_tc_kernel(const __grid_constant__ CUtensorMap mapQKV,
+                        const __grid_constant__ CUtensorMap mapKV, const AttnPairParams p) {
   using C = AttnPairCfg<D, EMU>;
   constexpr int kFwdHandovers = fwd_handovers<D>();
   constexpr int kFwdChunksPerHand = 4 / kFwdHandovers;
@@ -224,6 +241,9 @@ __global__ void __launch_bounds__(384, 1)
   // in one 64-bit word, so a reader sees a value together with its block
   __shared__ unsigned long long gate_slot[2][4];
   __shared__ int gate_keep[2];      // per tile: the current block's decision
+  // per tile, the decisions of the last four blocks as ((j + 1) << 1) | keep,
+  // at [j & 3]: the producer issues V_j only once they are known
+  __shared__ int gate_dec[2][4];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // blockIdx -> (head group, work rank, head): within a group, consecutive
@@ -239,8 +259,13 @@ __global__ void __launch_bounds__(384, 1)
   const int bidx = itemA / p.nb;
   const int iA = itemA - bidx * p.nb;
   const int iB = iA + 1;
-  const int nA = p.causal ? iA + 1 : p.nb;
-  const int nB = has_b ? (p.causal ? iB + 1 : p.nb) : 0;
+  // global block positions (for the causal range and the diagonal) and the
+  // key blocks of the whole sequence
+  const int gA = SHARD ? shard_global_block(p, iA) : iA;
+  const int gB = SHARD ? shard_global_block(p, iB) : iB;
+  const int nb_kv = SHARD ? p.N_kv / C::BKV : p.nb;
+  const int nA = p.causal ? gA + 1 : nb_kv;
+  const int nB = has_b ? (p.causal ? gB + 1 : nb_kv) : 0;
   const int n_kv = nA > nB ? nA : nB;
 
   if (threadIdx.x == 0) {
@@ -255,8 +280,10 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(o_done0 + 8 * x, 1);
     }
     mbar_init(drain, 1);
-    if constexpr (GATE)
+    if constexpr (GATE) {
       for (int i = 0; i < 8; ++i) (&gate_slot[0][0])[i] = 0ull;
+      for (int i = 0; i < 8; ++i) (&gate_dec[0][0])[i] = 0;
+    }
     abort_sh = 0;
     fence_mbar_init();
   }
@@ -276,7 +303,10 @@ __global__ void __launch_bounds__(384, 1)
     // The whole warp runs the role (warp-uniform coordinates); the elected
     // lane issues the TMA loads.
     const bool leader = elect_one();
-    if (leader) tma_prefetch_desc(&mapQKV);
+    if (leader) {
+      tma_prefetch_desc(&mapQKV);
+      if constexpr (SHARD) tma_prefetch_desc(&mapKV);
+    }
     int armed[C::NSLOT];
     for (int s = 0; s < C::NSLOT; ++s) armed[s] = -1;
     if (leader) {
@@ -288,24 +318,112 @@ __global__ void __launch_bounds__(384, 1)
     int slot = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int j = 0; j < n_kv && ok; ++j) {
-      for (int w = 0; w < 2; ++w) {
+    if constexpr (!GATE) {
+      // ring order K_0 V_0 K_1 V_1 ...
+      for (int j = 0; j < n_kv && ok; ++j) {
+        for (int w = 0; w < 2; ++w) {
+          if (!mbar_wait_warp(ring_empty0 + 8 * slot, phase ^ 1u, abort_flag, p.err,
+                              kSiteAttnProducer)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = ring_full0 + 8 * slot;
+          const bool lost = p.fault == 2 && blockIdx.x == 0 && j == 0 && w == 1;
+          if (!lost) {
+            armed[slot] = static_cast<int>(phase);
+            if (leader) {
+              mbar_arrive_expect_tx(fb, C::TILE);
+              if constexpr (SHARD) {
+                // key block j of the sequence: its owner rank and local block
+                const int c = j / p.kv_cb;
+                const int owner = c < p.kv_G ? c : 2 * p.kv_G - 1 - c;
+                const int lb = (c < p.kv_G ? 0 : p.kv_cb) + (j - c * p.kv_cb);
+                const int col = w == 0 ? head * D : p.d + head * D;  // in K | V
+                tma_load_5d(smem_u32(smem + C::OFF_RING + slot * C::TILE), &mapKV, fb, 0,
+                            lb * C::BKV, col / 64, bidx, owner);
+              } else {
+                const int col = w == 0 ? colK : colV;
+                tma_load_4d(smem_u32(smem + C::OFF_RING + slot * C::TILE), &mapQKV, fb, 0,
+                            j * C::BKV, col / 64, bidx);
+              }
+            }
+          }
+          if (++slot == C::NSLOT) {
+            slot = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    } else {
+      // Gated ring order: K_0 K_1 V_0 K_2 V_1 ... V_n-1, so
+      // K runs one block ahead of V and V_j waits for the gate decisions of
+      // block j (issued at once when tile A keeps it; skipped when every tile
+      // that visits block j prunes it).
+      for (int t = 0; t < 2 * n_kv && ok; ++t) {
+        int j, w;  // key block, 0 = K / 1 = V
+        if (t == 0) {
+          j = 0;
+          w = 0;
+        } else if ((t & 1) && (t + 1) / 2 < n_kv) {
+          j = (t + 1) / 2;
+          w = 0;
+        } else {
+          j = (t & 1) ? n_kv - 1 : t / 2 - 1;
+          w = 1;
+        }
         if (!mbar_wait_warp(ring_empty0 + 8 * slot, phase ^ 1u, abort_flag, p.err,
                             kSiteAttnProducer)) {
           ok = false;
           break;
         }
-        const uint32_t fb = ring_full0 + 8 * slot;
-        const bool lost = p.fault == 2 && blockIdx.x == 0 && j == 0 && w == 1;
-        if (!lost) {
-          armed[slot] = static_cast<int>(phase);
-          const int col = w == 0 ? colK : colV;
-          if (leader) {
-            mbar_arrive_expect_tx(fb, C::TILE);
-            tma_load_4d(smem_u32(smem + C::OFF_RING + slot * C::TILE), &mapQKV, fb, 0,
-                        j * C::BKV, col / 64, bidx);
+        bool load = true;
+        if (GATE && w == 1) {
+          // wait (bounded) for the decisions of the tiles that visit block j
+          const bool needA = j < nA, needB = j < nB;
+          const int tag = (j + 1) << 1;
+          bool seen = false;
+          const uint64_t g0 = global_ns();
+          for (uint32_t it = 0;; ++it) {
+            const int da = *reinterpret_cast<volatile int*>(&gate_dec[0][j & 3]);
+            const int db = *reinterpret_cast<volatile int*>(&gate_dec[1][j & 3]);
+            const bool haveA = !needA || (da & ~1) == tag;
+            const bool haveB = !needB || (db & ~1) == tag;
+            const bool keepA = needA && da == (tag | 1);
+            const bool keepB = needB && db == (tag | 1);
+            if (keepA || (haveA && haveB)) {
+              load = keepA || keepB;
+              seen = true;
+              break;
+            }
+            if ((it & 63u) == 63u) {
+              if (*abort_flag) break;
+              if (global_ns() - g0 > BPT_WAIT_LIMIT_NS) {
+                record_error(p.err, kErrTimeout, kSiteAttnProducer);
+                *abort_flag = 1;
+                break;
+              }
+            }
+          }
+          if (!__all_sync(0xffffffffu, seen)) {
+            ok = false;
+            break;
           }
         }
+        const uint32_t fb = ring_full0 + 8 * slot;
+        {
+          armed[slot] = static_cast<int>(phase);
+          if (leader) {
+            if (!load) {
+              mbar_arrive_expect_tx(fb, 0);  // V_j not needed: the slot completes empty
+            } else {
+              mbar_arrive_expect_tx(fb, C::TILE);
+              const int col = w == 0 ? colK : colV;
+              tma_load_4d(smem_u32(smem + C::OFF_RING + slot * C::TILE), &mapQKV, fb, 0,
+                          j * C::BKV, col / 64, bidx);
+            }
+          }
+        }
+        __syncwarp();
         if (++slot == C::NSLOT) {
           slot = 0;
           phase ^= 1u;
@@ -380,11 +498,28 @@ __global__ void __launch_bounds__(384, 1)
       commit(ring_empty0 + 8 * slot_of(0));
     }
     for (int j = 0; j < n_kv && ok; ++j) {
-      const int tk = 2 * (j + 1), tv = 2 * j + 1;
+      // ring positions of K_j+1 and V_j (see the producer's order)
+      const int tk = GATE ? 2 * j + 1 : 2 * (j + 1);
+      const int tv = GATE ? (j < n_kv - 1 ? 2 * j + 2 : 2 * n_kv - 1) : 2 * j + 1;
       bool k_ready = false;
-      if (!mbar_wait_warp(ring_full0 + 8 * slot_of(tv), phase_of(tv), abort_flag, p.err,
-                          kSiteAttnMma))
-        break;
+      // V_j is waited for before its first PV chunk, or (every visiting tile
+      // pruned block j: the producer completes the slot without loading) at
+      // the end of the block, before the slot is released
+      bool v_ready = false;
+      if constexpr (!GATE) {  // dense: V_j is always loaded; wait at once
+        if (!mbar_wait_warp(ring_full0 + 8 * slot_of(tv), phase_of(tv), abort_flag, p.err,
+                            kSiteAttnMma))
+          break;
+        v_ready = true;
+      }
+      auto wait_v = [&]() {
+        if (!v_ready) {
+          ok = mbar_wait_warp(ring_full0 + 8 * slot_of(tv), phase_of(tv), abort_flag, p.err,
+                              kSiteAttnMma);
+          v_ready = true;
+        }
+        return ok;
+      };
       const uint32_t v_lo = sdesc_lo(ring + slot_of(tv) * C::TILE, C::CHUNK);
       const uint32_t k_lo = sdesc_lo(ring + slot_of(tk) * C::TILE, 16);
       for (int x = 0; x < 2 && ok; ++x) {
@@ -408,6 +543,7 @@ __global__ void __launch_bounds__(384, 1)
           tc_fence_after();
           // (the tile's decision was written before its first P hand-over)
           if (hh == 0) kept = !GATE || *reinterpret_cast<volatile int*>(&gate_keep[x]) != 0;
+          if (kept && !wait_v()) break;
           if (kept)
             for (int q = 0; q < kFwdChunksPerHand; ++q)
               issue_pv_chunk(tS, v_lo, tO, hh * kFwdChunksPerHand + q, !o_started[x]);
@@ -431,7 +567,7 @@ __global__ void __launch_bounds__(384, 1)
           commit(o_done0 + 8 * x);
         }
       }
-      if (!ok) break;
+      if (!ok || !wait_v()) break;
       commit(ring_empty0 + 8 * slot_of(tv));
       if (k_ready) commit(ring_empty0 + 8 * slot_of(tk));
     }
@@ -444,13 +580,14 @@ __global__ void __launch_bounds__(384, 1)
     const int r = e * 32 + lane;    // query row within the tile
     const int nX = x == 0 ? nA : nB;
     const int iX = x == 0 ? iA : iB;
+    const int gX = x == 0 ? gA : gB;  // global block (the diagonal)
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(e * 32) << 16);
     const uint32_t tS = t_lane + (x == 0 ? 0u : C::TM_S_B);
     const uint32_t tO = t_lane + (x == 0 ? C::TM_O_A : C::TM_O_B);
     const uint32_t s_full = s_full0 + 8 * x, o_done = o_done0 + 8 * x;
     const uint32_t p_chunk = p_chunk0 + 8 * (4 * x);  // [4]
     const float c = p.scale_log2;
-    const bool ragged = (p.N % C::BKV) != 0;
+    const bool ragged = !SHARD && (p.N % C::BKV) != 0;
     float m_run = -INFINITY;  // reference maximum (moves only by > 2^8 in exp2 units)
     float m_true = -INFINITY;  // exact running row maximum, for the statistics
     float l = 0.f;
@@ -471,7 +608,7 @@ __global__ void __launch_bounds__(384, 1)
       for (int cc = 0; cc < C::BKV / 32; ++cc)
         tmem_ld_32x32b_x32(tS + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[cc * 32]));
       tmem_ld_wait();
-      const bool masked = p.causal ? (j == iX) : (ragged && j == p.nb - 1);
+      const bool masked = p.causal ? (j == gX) : (ragged && j == p.nb - 1);
       if (masked) {
         const int lim = p.causal ? r + 1 : p.N - j * C::BKV;
 #pragma unroll
@@ -534,9 +671,11 @@ __global__ void __launch_bounds__(384, 1)
           break;
         }
         const float smax = bmax * (p.scale_log2 * 0.69314718055994531f);
-        keep_blk = (j == iX) || (smax >= t_thr);
+        keep_blk = (j == gX) || (smax >= t_thr);
         if (e == 0 && lane == 0) {
           gate_keep[x] = keep_blk ? 1 : 0;
+          *reinterpret_cast<volatile int*>(&gate_dec[x][j & 3]) =
+              ((j + 1) << 1) | (keep_blk ? 1 : 0);
           const long long o = ((static_cast<long long>(bidx) * p.h + head) * p.nb + iX) * p.nb + j;
           if (p.gate_bmax != nullptr) p.gate_bmax[o] = smax;
           if (p.gate_kept != nullptr) p.gate_kept[o] = keep_blk ? 1 : 0;

@@ -248,6 +248,10 @@ bpt_status device_info(int* sms, int* pair_clusters = nullptr) {
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                bpt::AttnPairCfg<128, kEmu128>::SMEM) != cudaSuccess ||
           set_smem(bpt::attn_pair_tc_kernel<64, kEmu64, true>, bpt::AttnPairCfg<64, kEmu64>::SMEM) ||
+          set_smem(bpt::attn_pair_tc_kernel<64, kEmu64, false, true>,
+                   bpt::AttnPairCfg<64, kEmu64>::SMEM) ||
+          set_smem(bpt::attn_pair_tc_kernel<128, kEmu128, false, true>,
+                   bpt::AttnPairCfg<128, kEmu128>::SMEM) ||
           set_smem(bpt::attn_pair_tc_kernel<128, kEmu128, true>,
                    bpt::AttnPairCfg<128, kEmu128>::SMEM) ||
           set_smem(bpt::gemm_f16_pair_kernel<4, bpt::kLayAkBn>, bpt::kPairSmem) ||
@@ -306,8 +310,8 @@ bpt_status get_encoder() {
 // fp16 tiles with the 128-byte swizzle; dims/strides innermost first.
 bool encode_f16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
                 const uint64_t* strides_bytes, const uint32_t* box) {
-  cuuint64_t gd[4], gs[3];
-  cuuint32_t bx[4], es[4] = {1, 1, 1, 1};
+  cuuint64_t gd[5], gs[4];
+  cuuint32_t bx[5], es[5] = {1, 1, 1, 1, 1};
   for (int i = 0; i < rank; ++i) {
     gd[i] = dims[i];
     bx[i] = box[i];
@@ -336,10 +340,10 @@ bool map_a(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int64_t ld
 // 64-column chunks.  The B operand of the forward (weights), and the A
 // operand [K, M] of the weight-gradient GEMMs.
 bool map_b(CUtensorMap* m, const void* base, int64_t K, int64_t cols, int chunks,
-           int64_t ld = 0) {
+           int64_t ld = 0, int box_rows = 128) {
   const uint64_t dims[3] = {64, uint64_t(K), uint64_t(cols / 64)};
   const uint64_t st[2] = {uint64_t(ld > 0 ? ld : cols) * 2, 128};
-  const uint32_t box[3] = {64, 128, uint32_t(chunks)};
+  const uint32_t box[3] = {64, uint32_t(box_rows), uint32_t(chunks)};
   return encode_f16(m, base, 3, dims, st, box);
 }
 // QKV [B][N][3d] viewed as [B][3d/64][N][64]: a box is 128 tokens x the
@@ -350,6 +354,18 @@ bool map_qkv(CUtensorMap* m, const void* base, int64_t B, int64_t N, int64_t d, 
   const uint64_t st[3] = {uint64_t(3 * d) * 2, 128, uint64_t(N) * uint64_t(3 * d) * 2};
   const uint32_t box[4] = {64, 128, uint32_t(dk / 64), 1};
   return encode_f16(m, base, 4, dims, st, box);
+}
+
+// All-gathered K | V of a sequence shard, [G][B][n_loc][2d], viewed as
+// [G][B][2d/64][n_loc][64]: a box is 128 tokens x the d_k/64 chunks of one
+// head's K or V of one rank's batch element.
+bool map_kv_shards(CUtensorMap* m, const void* base, int64_t G, int64_t B, int64_t n_loc,
+                   int64_t d, int64_t dk) {
+  const uint64_t row = uint64_t(2 * d) * 2;
+  const uint64_t dims[5] = {64, uint64_t(n_loc), uint64_t(2 * d / 64), uint64_t(B), uint64_t(G)};
+  const uint64_t st[4] = {row, 128, uint64_t(n_loc) * row, uint64_t(B * n_loc) * row};
+  const uint32_t box[5] = {64, 128, uint32_t(dk / 64), 1, 1};
+  return encode_f16(m, base, 5, dims, st, box);
 }
 
 // -------------------------------------------------------------- profiling --
@@ -457,13 +473,23 @@ struct AttnGate {
   uint8_t* kept;    // nullable [B][h][nb][nb]
 };
 
+// Sequence shard of the attention: keys and values of the whole sequence in
+// the all-gathered buffer (5-D tensor map), zig-zag chunk ownership.
+struct AttnShard {
+  const CUtensorMap* mKV;  // [G][B][N / G][2d] viewed as [G][B][2d/64][N/G][64]
+  int cb, c0, c1, G;       // blocks per chunk, this rank's chunks, ranks
+  int64_t N_kv;            // tokens of the whole sequence
+};
+
 // One wave of the tensor-core attention: o (fp16 block rows) and, if stats is
 // non-null, the per-row (m, l); gated when gate is non-null.
 // o_tok: o is the Q columns of the QKV buffer, token rows (fused schedule);
-// otherwise wave scratch rows [count * 128, d].
+// otherwise wave scratch rows [count * 128, d].  shard: o_tok over the
+// shard's own Q buffer [rows, d] (mQKV maps it), keys from shard->mKV.
 cudaError_t launch_attn(const Plan& P, const Wave& wv_, const CUtensorMap& mQKV, __half* so,
                         float* stats, uint32_t* err, int fault, cudaStream_t s,
-                        const AttnGate* gate = nullptr, bool o_tok = false) {
+                        const AttnGate* gate = nullptr, bool o_tok = false,
+                        const AttnShard* shard = nullptr) {
   bpt::AttnPairParams ap{};
   ap.N = int(P.N); ap.nb = int(P.nb); ap.h = int(P.h); ap.d = int(P.d);
   ap.causal = P.causal; ap.item0 = int(wv_.item0); ap.count = int(wv_.count);
@@ -472,7 +498,15 @@ cudaError_t launch_attn(const Plan& P, const Wave& wv_, const CUtensorMap& mQKV,
   ap.o_ld = o_tok ? 3 * P.d : P.d;
   ap.scale_log2 = float(1.4426950408889634 / std::sqrt(double(P.dk)));
   ap.stats = reinterpret_cast<float2*>(stats);
-  const int64_t kv_head = (wv_.seqs > 0 ? wv_.seqs : 1) * P.N * P.dk * 2 * 2;
+  if (shard) {
+    ap.kv_cb = shard->cb;
+    ap.q_c0 = shard->c0;
+    ap.q_c1 = shard->c1;
+    ap.kv_G = shard->G;
+    ap.N_kv = int(shard->N_kv);
+  }
+  const int64_t kv_head =
+      (wv_.seqs > 0 ? wv_.seqs : 1) * (shard ? shard->N_kv : P.N) * P.dk * 2 * 2;
   ap.hg = 1;
   for (int g = int(P.h); g > 1; --g)
     if (P.h % g == 0 && g * kv_head <= (int64_t(BPT_ATTN_KV_BUDGET_MB) << 20)) {
@@ -484,31 +518,50 @@ cudaError_t launch_attn(const Plan& P, const Wave& wv_, const CUtensorMap& mQKV,
   const int64_t units = wv_.seqs == 0 ? (wv_.count + ap.qpc - 1) / ap.qpc
                                       : wv_.seqs * ((P.nb + ap.qpc - 1) / ap.qpc);
   const unsigned grid = unsigned(units * P.h);
+  const CUtensorMap& mKV = shard ? *shard->mKV : mQKV;
   if (gate != nullptr) {
     ap.gate_t = gate->t;
     ap.gate_bmax = gate->bmax;
     ap.gate_kept = gate->kept;
     if (P.dk == 128)
       bpt::attn_pair_tc_kernel<128, kEmu128, true>
-          <<<grid, 384, bpt::AttnPairCfg<128, kEmu128>::SMEM, s>>>(mQKV, ap);
+          <<<grid, 384, bpt::AttnPairCfg<128, kEmu128>::SMEM, s>>>(mQKV, mKV, ap);
     else
       bpt::attn_pair_tc_kernel<64, kEmu64, true>
-          <<<grid, 384, bpt::AttnPairCfg<64, kEmu64>::SMEM, s>>>(mQKV, ap);
+          <<<grid, 384, bpt::AttnPairCfg<64, kEmu64>::SMEM, s>>>(mQKV, mKV, ap);
+  } else if (shard != nullptr) {
+    if (P.dk == 128)
+      bpt::attn_pair_tc_kernel<128, kEmu128, false, true>
+          <<<grid, 384, bpt::AttnPairCfg<128, kEmu128>::SMEM, s>>>(mQKV, mKV, ap);
+    else
+      bpt::attn_pair_tc_kernel<64, kEmu64, false, true>
+          <<<grid, 384, bpt::AttnPairCfg<64, kEmu64>::SMEM, s>>>(mQKV, mKV, ap);
   } else if (P.dk == 128) {
     bpt::attn_pair_tc_kernel<128, kEmu128>
-        <<<grid, 384, bpt::AttnPairCfg<128, kEmu128>::SMEM, s>>>(mQKV, ap);
+        <<<grid, 384, bpt::AttnPairCfg<128, kEmu128>::SMEM, s>>>(mQKV, mKV, ap);
   } else {
     bpt::attn_pair_tc_kernel<64, kEmu64>
-        <<<grid, 384, bpt::AttnPairCfg<64, kEmu64>::SMEM, s>>>(mQKV, ap);
+        <<<grid, 384, bpt::AttnPairCfg<64, kEmu64>::SMEM, s>>>(mQKV, mKV, ap);
   }
   return cudaGetLastError();
 }
+
+// One rank's part of a sequence-sharded forward (bpt_layer_shard_*): the
+// plan is that of the rank's own n_loc = N / G rows; phase 1 writes its K | V
+// to kv_loc, phase 2 attends against every rank's K | V in kv_all.
+struct ShardSpec {
+  int phase;          // 1: projection, 2: attention + layer body
+  int G, rank;
+  int64_t N;          // tokens of the whole sequence
+  __half* kv_loc;     // phase 1: [B, n_loc, 2d]
+  const void* kv_all; // phase 2: [G, B, n_loc, 2d]
+};
 
 bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const void* W_Q,
                         const void* W_K, const void* W_V, const void* W_O, const void* ln2,
                         const void* W_1, const void* b_1, const void* W_2, const void* b_2,
                         float* out, float* stats, uint8_t* ws, cudaStream_t s, int sms,
-                        const AttnGate* gate) {
+                        const AttnGate* gate, const ShardSpec* shard = nullptr) {
   using bf = __nv_bfloat16;
   using hf = __half;
   const int64_t M = P.B * P.N, d = P.d, d_ff = P.d_ff;
@@ -530,7 +583,7 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
   hf* sh = reinterpret_cast<hf*>(ws + P.off_h);
   const int64_t R = P.P * P.blk;  // scratch rows
 
-  CUtensorMap mXn, mWq, mWk, mWv, mQKV, mO, mWo, mV, mW1, mH, mW2;
+  CUtensorMap mXn, mWq, mWk, mWv, mQKV, mO, mWo, mV, mW1, mH, mW2, mH1, mW2e;
   // A CTA's 128 B columns stay inside one of W_Q | W_K | W_V when d is a
   // multiple of 128 (one two-chunk box); otherwise it loads one chunk per box.
   const int qkv_chunks = (d % 128 == 0) ? 2 : 1;
@@ -543,12 +596,20 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
     // and the per-pair scratch rows of LN2(y) and the hidden
     const int64_t trows = P.tail_pairs * 256;
     ok = ok && map_a(&mO, qkv, M, d, 3 * d) &&
-         map_a(&mV, ws + P.off_tv, trows, d) && map_a(&mH, ws + P.off_th, trows, d_ff);
+         map_a(&mV, ws + P.off_tv, trows, d) && map_a(&mH, ws + P.off_th, trows, d_ff) &&
+         // 512-column W_2 tiles: H in 64-deep single-chunk boxes, W_2 as
+         // 64 K rows x four 64-column chunks
+         map_a(&mH1, ws + P.off_th, trows, d_ff, 0, 1) && map_b(&mW2e, w2, d_ff, d, 4, 0, 64);
   } else {
     ok = ok && map_a(&mO, so, R, d) && map_a(&mV, sv, R, d) && map_a(&mH, sh, R, d_ff);
   }
+  CUtensorMap mKV;
+  if (shard != nullptr && shard->phase == 2)
+    ok = ok && map_kv_shards(&mKV, shard->kv_all, shard->G, P.B, P.N, d, P.dk);
   if (!ok) return BPT_ERR_CUDA;
 
+  RowMap ident{0, 1, 1, 1, 1};
+  if (shard == nullptr || shard->phase == 1) {
   {
     bpt::CvtSegments cs{};
     const void* src[6] = {W_Q, W_K, W_V, W_O, W_1, W_2};
@@ -567,7 +628,6 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
     bpt::cvt_bf16_to_f16_kernel<<<grid, 256, 0, s>>>(cs, err);
     if (cudaGetLastError() != cudaSuccess) return BPT_ERR_CUDA;
   }
-  RowMap ident{0, 1, 1, 1, 1};
   {
     LaunchScope ls(BPT_KIND_LN1, s);
     if (launch_ln<bf, hf, bf>(static_cast<const bf*>(x), static_cast<const bf*>(ln1), xn, M, d,
@@ -580,19 +640,35 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
     g.n_sub = int(d); g.n_maps = 3; g.b_chunks = qkv_chunks;
     g.epi = bpt::kEpiStoreF16;
     g.out_h = qkv; g.ld_out = 3 * d;
+    if (shard != nullptr) {  // K | V of the shard's rows go to kv_loc
+      g.split_col = int(d);
+      g.out_h2 = shard->kv_loc;
+      g.ld_out2 = 2 * d;
+    }
     g.map = ident;
     g.err = err;
     g.fault = fault == 1 ? 1 : 0;
     LaunchScope ls(BPT_KIND_QKV, s);
     if (launch_gemm(mXn, mWq, mWk, mWv, g, sms, s) != cudaSuccess) return BPT_ERR_CUDA;
   }
+  }  // projection
+  if (shard != nullptr && shard->phase == 1) return BPT_OK;
   if (P.fused) {
     // attention over every query block, o over each block's Q rows
     const Wave all{0, P.items, P.B};
+    AttnShard as{};
+    if (shard != nullptr) {
+      as.mKV = &mKV;
+      as.G = shard->G;
+      as.cb = int(P.N / 2 / 128);
+      as.c0 = shard->rank;
+      as.c1 = 2 * shard->G - 1 - shard->rank;
+      as.N_kv = shard->N;
+    }
     {
       LaunchScope ls(BPT_KIND_ATTN, s);
-      if (launch_attn(P, all, mQKV, qkv, stats, err, fault == 2 ? 2 : 0, s, gate, true) !=
-          cudaSuccess)
+      if (launch_attn(P, all, mQKV, qkv, stats, err, fault == 2 ? 2 : 0, s, gate, true,
+                      shard != nullptr ? &as : nullptr) != cudaSuccess)
         return BPT_ERR_CUDA;
     }
     int dummy = 0, pairs_max = 0;
@@ -616,7 +692,7 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
     const int64_t pairs = std::max<int64_t>(1, std::min<int64_t>(P.tail_pairs, pairs_max));
     LaunchScope ls(BPT_KIND_TAIL, s);
     bpt::tail_pair_kernel<<<unsigned(2 * pairs), bpt::kTailThreads, bpt::kPairSmem, s>>>(
-        mO, mWo, mV, mW1, mH, mW2, tp);
+        mO, mWo, mV, mW1, mH, mW2, mH1, mW2e, tp);
     if (cudaGetLastError() != cudaSuccess) return BPT_ERR_CUDA;
     return BPT_OK;
   }
@@ -1375,6 +1451,53 @@ bpt_status backward_impl(const void* x, const void* ln1, const void* W_Q, const 
                        dW_Q, dW_K, dW_V, dW_O, d_ln2, dW_1, db_1, dW_2, db_2, ws, s, sms);
 }
 
+// Shared body of the sequence-shard entry points (phase 1: projection into
+// kv_loc; phase 2: attention against kv_all + layer body).
+bpt_status shard_impl(int phase, const void* x, const void* ln1, const void* W_Q,
+                      const void* W_K, const void* W_V, const void* W_O, const void* ln2,
+                      const void* W_1, const void* b_1, const void* W_2, const void* b_2,
+                      int64_t B, int64_t N, int64_t G, int64_t rank, int64_t d, int64_t h,
+                      int64_t d_ff, int causal, bpt_dtype dtype, void* kv, float* out,
+                      void* workspace, size_t workspace_bytes, bpt_stream_t stream) {
+  if (G < 1 || rank < 0 || rank >= G || N <= 0 || B <= 0) return BPT_ERR_INVALID_ARG;
+  if (dtype != BPT_BF16) return BPT_ERR_UNSUPPORTED;
+  if (N % (256 * G) != 0) return BPT_ERR_UNSUPPORTED;  // 2G chunks of whole blocks
+  const int64_t n_loc = N / G;
+  bpt_status st = check_shape(B, n_loc, d, h, d_ff, causal, dtype);
+  if (st != BPT_OK) return st;
+  if (B * N > (int64_t(1) << 30)) return BPT_ERR_UNSUPPORTED;
+  const void* ptrs[] = {x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, out, workspace, kv};
+  for (const void* p : ptrs)
+    if (p == nullptr || misaligned(p)) return BPT_ERR_INVALID_ARG;
+  const Plan P = make_plan(B, n_loc, d, h, d_ff, causal, dtype);
+  if (workspace_bytes < P.total) return BPT_ERR_WORKSPACE;
+  const std::vector<Span> ins =
+      forward_inputs(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, B, n_loc, d, d_ff, 2);
+  const Span so(out, size_t(B * n_loc * d) * 4), sw(workspace, P.total);
+  const Span sk(kv, size_t(phase == 1 ? 1 : G) * size_t(B * n_loc * 2 * d) * 2);
+  if (so.overlaps(sw) || sk.overlaps(so) || sk.overlaps(sw)) return BPT_ERR_INVALID_ARG;
+  for (const Span& in : ins)
+    if (so.overlaps(in) || sw.overlaps(in) || (phase == 1 && sk.overlaps(in)))
+      return BPT_ERR_INVALID_ARG;
+  int sms = 0;
+  st = device_info(&sms);
+  if (st != BPT_OK) return st;
+  st = get_encoder();
+  if (st != BPT_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (phase == 1 && cudaMemsetAsync(ws, 0, kHeaderBytes, s) != cudaSuccess) return BPT_ERR_CUDA;
+  ShardSpec sh{};
+  sh.phase = phase;
+  sh.G = int(G);
+  sh.rank = int(rank);
+  sh.N = N;
+  sh.kv_loc = phase == 1 ? static_cast<__half*>(kv) : nullptr;
+  sh.kv_all = phase == 2 ? kv : nullptr;
+  return forward_bf16(P, x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, out, nullptr, ws, s,
+                      sms, nullptr, &sh);
+}
+
 bpt_status plan_for(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff, int causal,
                     bpt_dtype dtype, const bpt_options* opts, bool forward, Plan* P) {
   bpt_status st = check_shape(B, N, d, h, d_ff, causal, dtype);
@@ -1536,6 +1659,40 @@ bpt_status bpt_layer_backward_opt(const void* x, const void* ln1, const void* W_
   return backward_impl(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, stats, dZ, B, N, d, h,
                        d_ff, causal, dtype, dx, d_ln1, dW_Q, dW_K, dW_V, dW_O, d_ln2, dW_1, db_1,
                        dW_2, db_2, workspace, workspace_bytes, opts, stream);
+}
+
+bpt_status bpt_layer_shard_workspace_size(int64_t B, int64_t N, int64_t G, int64_t d,
+                                          int64_t h, int64_t d_ff, int causal, bpt_dtype dtype,
+                                          size_t* bytes) {
+  if (bytes == nullptr || G < 1 || N <= 0 || B <= 0) return BPT_ERR_INVALID_ARG;
+  if (dtype != BPT_BF16) return BPT_ERR_UNSUPPORTED;
+  if (N % (256 * G) != 0) return BPT_ERR_UNSUPPORTED;
+  return bpt_layer_workspace_size(B, N / G, d, h, d_ff, causal, dtype, bytes);
+}
+
+bpt_status bpt_layer_shard_project(const void* x, const void* ln1, const void* W_Q,
+                                   const void* W_K, const void* W_V, const void* W_O,
+                                   const void* ln2, const void* W_1, const void* b_1,
+                                   const void* W_2, const void* b_2, int64_t B, int64_t N,
+                                   int64_t G, int64_t rank, int64_t d, int64_t h, int64_t d_ff,
+                                   int causal, bpt_dtype dtype, void* kv_loc, float* out,
+                                   void* workspace, size_t workspace_bytes,
+                                   bpt_stream_t stream) {
+  return shard_impl(1, x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, B, N, G, rank, d, h,
+                    d_ff, causal, dtype, kv_loc, out, workspace, workspace_bytes, stream);
+}
+
+bpt_status bpt_layer_shard_forward(const void* x, const void* ln1, const void* W_Q,
+                                   const void* W_K, const void* W_V, const void* W_O,
+                                   const void* ln2, const void* W_1, const void* b_1,
+                                   const void* W_2, const void* b_2, int64_t B, int64_t N,
+                                   int64_t G, int64_t rank, int64_t d, int64_t h, int64_t d_ff,
+                                   int causal, bpt_dtype dtype, const void* kv_all, float* out,
+                                   void* workspace, size_t workspace_bytes,
+                                   bpt_stream_t stream) {
+  return shard_impl(2, x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, B, N, G, rank, d, h,
+                    d_ff, causal, dtype, const_cast<void*>(kv_all), out, workspace,
+                    workspace_bytes, stream);
 }
 
 bpt_status bpt_read_device_error(void* workspace, bpt_stream_t stream, uint32_t* site) {

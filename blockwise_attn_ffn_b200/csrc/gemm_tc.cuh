@@ -27,7 +27,9 @@
 // leave the TMA and UMMA warps more issue slots.
 //
 // Epilogues (all in fp32 before the final rounding):
-//   kEpiStoreF16    out_h[row, col]  = acc                       (QKV, fp16)
+//   kEpiStoreF16    out_h[row, col]  = acc                       (QKV, fp16; with
+//                   split_col > 0 columns >= split_col go to out_h2, which is
+//                   how a sequence shard stores Q apart from its K | V)
 //   kEpiResidX      out_f32[g, col]  = x[g, col] + acc           (y = x + o W_O)
 //   kEpiGeluBias    out_h[row, col]  = GELU(acc + bias[col])     (FFN hidden, fp16)
 //   kEpiBiasAccum   out_f32[g, col] += acc + bias[col]           (Z = y + h W_2 + b_2)
@@ -64,8 +66,11 @@ struct GemmParams {
   int b_chunks;    // 64-column chunks per B box: 2, or 1 if n_sub % 128 != 0
   int epi;
   __half* out_h;
-  __half* out_h2;  // kEpiGeluBiasKeep: pre-activation copy (same ld as out_h)
+  __half* out_h2;  // kEpiGeluBiasKeep: pre-activation copy (same ld as out_h);
+                   // kEpiStoreF16 with split_col > 0: columns >= split_col
   long long ld_out;
+  int split_col;       // kEpiStoreF16: 0, or the first column stored to out_h2
+  long long ld_out2;   // row stride of out_h2 for the split store
   float* out_f32;
   long long ld_f32;
   const __nv_bfloat16* resid;
@@ -165,6 +170,8 @@ __device__ __forceinline__ void gemm_epilogue_row(const GemmParams& p, uint32_t 
         }
       }
       uint4* dst = reinterpret_cast<uint4*>(p.out_h + row * p.ld_out + col0);
+      if (p.epi == kEpiStoreF16 && p.split_col > 0 && col0 >= p.split_col)
+        dst = reinterpret_cast<uint4*>(p.out_h2 + row * p.ld_out2 + (col0 - p.split_col));
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint4 w;

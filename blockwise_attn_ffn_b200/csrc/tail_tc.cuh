@@ -16,7 +16,8 @@
 //   C  v   = LN2(y)           the epilogue warps, one warp per row -> v scratch
 //   D  H_c = GELU(v W_1[:, c] + b_1[c])   c = 256-column chunks of d_ff
 //                                                        K = d     -> H scratch
-//   E  Z   = y + H W_2 + b_2  N-tiles of 256 over d,    K = d_ff  -> out (fp32)
+//   E  Z   = y + H W_2 + b_2  N-tiles of 512 (256 if d % 512 != 0) over d,
+//                                                        K = d_ff  -> out (fp32)
 //
 // o is read from the Q columns of the QKV buffer (the attention kernel wrote
 // each block's output over the block's own queries).  v [256, d] and
@@ -74,11 +75,14 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 
 // LN2 of the CTA's 128 rows of an item, one warp per row (rows w, w + 8, ..),
 // reading y from `out` three times (sum, squared deviations, normalise) in
-// the summation order of ln_rows_kernel.  Rows without a token (ragged last
-// block, absent second block) get zeros.
+// the summation order of ln_rows_kernel (lane l sums its 8-element chunks
+// (l + 32 q) * 8 in q order, then a warp sum).  Rows without a token (ragged
+// last block, absent second block) get zeros.  It runs while the tensor
+// cores work on the previous item's W_2 tiles (see the item order below).
 __device__ __forceinline__ void tail_ln2(const TailParams& p, const RowMap& map, int m_valid,
                                          int s_base, long long v_row0, int w, int lane) {
   const int d = p.d;
+#pragma unroll 1
   for (int q = w; q < 128; q += kTailEpi) {
     const int s = s_base + q;
     const long long g = s < m_valid ? map.map(s) : -1;
@@ -95,7 +99,7 @@ __device__ __forceinline__ void tail_ln2(const TailParams& p, const RowMap& map,
       float v[8];
       load8(yrow + c, v);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) sum += v[k];
+      for (int e = 0; e < 8; ++e) sum += v[e];
     }
     const float mean = warp_sum(sum) / static_cast<float>(d);
     float sq = 0.f;
@@ -103,8 +107,8 @@ __device__ __forceinline__ void tail_ln2(const TailParams& p, const RowMap& map,
       float v[8];
       load8(yrow + c, v);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const float t = v[k] - mean;
+      for (int e = 0; e < 8; ++e) {
+        const float t = v[e] - mean;
         sq += t * t;
       }
     }
@@ -116,32 +120,49 @@ __device__ __forceinline__ void tail_ln2(const TailParams& p, const RowMap& map,
       load8(p.ln2 + c, gm);
       load8(p.ln2 + d + c, bt);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) o[k] = (v[k] - mean) * rstd * gm[k] + bt[k];
+      for (int e = 0; e < 8; ++e) o[e] = (v[e] - mean) * rstd * gm[e] + bt[e];
       store8(vrow + c, o, bad);
     }
     if (bad) record_error(p.err, kErrRange, kSiteRangeLN);
   }
 }
 
-// Phase of tile t of an item (0: y tiles, 1: H chunks, 2: Z tiles) and its
-// N-tile index within the phase.
+// The tiles of one item.  y tiles and H chunks are 256 columns wide (K = d,
+// 128-deep stages); Z tiles are 512 columns wide when e512 (d % 512 == 0; K =
+// d_ff in 64-deep stages; the two 256-column halves share every H load, which
+// halves the re-reads of the hidden), else 256.  The epilogue sees a
+// 512-column tile as two consecutive 256-column accumulator slots.
 struct TailShape {
-  int nB, nD, kbD, kbF;  // y / Z tiles per item, H chunks, K blocks over d and d_ff
-  __device__ __forceinline__ int tiles() const { return 2 * nB + nD; }
-  __device__ __forceinline__ void at(int t, int& phase, int& n) const {
-    if (t < nB) {
-      phase = 0;
-      n = t;
-    } else if (t < nB + nD) {
-      phase = 1;
-      n = t - nB;
-    } else {
-      phase = 2;
-      n = t - nB - nD;
-    }
+  int nB, nD, nE, kbD, kbF, kbF64;  // tiles per phase; K blocks over d, d_ff (128 / 64 deep)
+  bool e512;
+  __device__ __forceinline__ int kblocks(int phase) const {
+    return phase == 2 ? (e512 ? kbF64 : kbF) : kbD;
   }
-  __device__ __forceinline__ int kblocks(int phase) const { return phase == 2 ? kbF : kbD; }
 };
+
+// Segment order of a pair's J items (B = y tiles, D = H chunks, E = Z tiles):
+//   B0 D0 | B1 E0 D1 | B2 E1 D2 | ... | B(J-1) E(J-2) D(J-1) | E(J-1)
+// Item j's LN2 runs in the epilogue between B(j) and E(j-1), so the tensor
+// cores compute E(j-1) meanwhile; and E(j) waits for the whole hidden of item
+// j behind B(j+1).  One H buffer suffices: UMMA work issued by one thread
+// completes in order, so every load of E(j) has landed before any D(j+1)
+// epilogue store.
+__device__ __forceinline__ void tail_segment(int s, int J, int& phase, int& j) {
+  if (s < 2) {
+    phase = s == 0 ? 0 : 1;
+    j = 0;
+    return;
+  }
+  const int t = s - 2;
+  if (t == 3 * (J - 1)) {
+    phase = 2;
+    j = J - 1;
+    return;
+  }
+  const int q = t / 3 + 1, r = t % 3;
+  phase = r == 0 ? 0 : (r == 1 ? 2 : 1);
+  j = r == 1 ? q - 1 : q;
+}
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTailThreads, 1)
     tail_pair_kernel(const __grid_constant__ CUtensorMap mapO,
@@ -149,7 +170,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTailThreads, 1)
                      const __grid_constant__ CUtensorMap mapV,
                      const __grid_constant__ CUtensorMap mapW1,
                      const __grid_constant__ CUtensorMap mapH,
-                     const __grid_constant__ CUtensorMap mapW2, const TailParams p) {
+                     const __grid_constant__ CUtensorMap mapW2,
+                     const __grid_constant__ CUtensorMap mapH1,
+                     const __grid_constant__ CUtensorMap mapW2e, const TailParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -171,12 +194,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTailThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const int pair = static_cast<int>(cluster_id_x());
   const int npairs = static_cast<int>(nclusters_x());
+  // this pair's items: pair, pair + npairs, ...
+  const int J = pair < p.items ? (p.items - pair + npairs - 1) / npairs : 0;
+  const int n_seg = 3 * J;
   TailShape sh;
+  sh.e512 = p.d % 512 == 0;
   sh.nB = (p.d + kGemmBN - 1) / kGemmBN;
   sh.nD = (p.d_ff + kGemmBN - 1) / kGemmBN;
+  sh.nE = sh.e512 ? p.d / 512 : sh.nB;
   sh.kbD = (p.d + kGemmBK - 1) / kGemmBK;
   sh.kbF = (p.d_ff + kGemmBK - 1) / kGemmBK;
-  const int tiles = sh.tiles();
+  sh.kbF64 = (p.d_ff + 63) / 64;
 
   if (threadIdx.x == 0) {
     for (int s2 = 0; s2 < kPairStages; ++s2) {
@@ -214,28 +242,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTailThreads, 1)
       tma_prefetch_desc(&mapW1);
       tma_prefetch_desc(&mapH);
       tma_prefetch_desc(&mapW2);
+      tma_prefetch_desc(&mapH1);
+      tma_prefetch_desc(&mapW2e);
     }
     int armed[kPairStages];
     for (int s2 = 0; s2 < kPairStages; ++s2) armed[s2] = -1;
     int stage = 0;
     uint32_t phase_bit = 0;
     bool ok = true;
-    uint32_t it_par = 0;  // parity of this pair's item count (hand-off phases)
     const int scr_row = pair * 256 + static_cast<int>(rank) * 128;
-    for (int item = pair; item < p.items && ok; item += npairs, it_par ^= 1u) {
+    for (int sg = 0; sg < n_seg && ok; ++sg) {
+      int ph, j;
+      tail_segment(sg, J, ph, j);
+      const int item = pair + j * npairs;
       // token row of this CTA's block (an absent second block reads block 0's
       // rows: its results are never stored)
       int blk = 2 * item + static_cast<int>(rank);
       if (blk >= p.blocks) blk = 0;
       const int bseq = blk / p.nb;
       const int tok_row = bseq * p.N + (blk - bseq * p.nb) * 128;
-      for (int t = 0; t < tiles && ok; ++t) {
-        int ph, n;
-        sh.at(t, ph, n);
-        const CUtensorMap* ma = ph == 0 ? &mapO : (ph == 1 ? &mapV : &mapH);
-        const CUtensorMap* mb = ph == 0 ? &mapWo : (ph == 1 ? &mapW1 : &mapW2);
-        const int a_row = ph == 0 ? tok_row : scr_row;
-        const int kbs = sh.kblocks(ph);
+      // a 512-column Z tile: A in 64-deep single-chunk boxes (mapH1), B as
+      // this CTA's contiguous 256-column slab, 64 K rows (mapW2e)
+      const bool wide = ph == 2 && sh.e512;
+      const CUtensorMap* ma = ph == 0 ? &mapO : (ph == 1 ? &mapV : (wide ? &mapH1 : &mapH));
+      const CUtensorMap* mb = ph == 0 ? &mapWo : (ph == 1 ? &mapW1 : (wide ? &mapW2e : &mapW2));
+      const int a_row = ph == 0 ? tok_row : scr_row;
+      const int kbs = sh.kblocks(ph);
+      const int tiles = ph == 0 ? sh.nB : (ph == 1 ? sh.nD : sh.nE);
+      const uint32_t stage_bytes =
+          wide ? 2u * (kPairABytes / 2 + kPairBBytes) : 2u * kPairStageBytes;
+      for (int n = 0; n < tiles && ok; ++n) {
         for (int kb = 0; kb < kbs; ++kb) {
           if (!mbar_wait_warp(empty0 + 8 * stage, phase_bit ^ 1u, abort_flag, p.err,
                               kSiteGemmProducer)) {
@@ -245,23 +281,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTailThreads, 1)
           const uint32_t fb_leader = map_to_rank(full0 + 8 * stage, 0);
           if (rank == 0) armed[stage] = static_cast<int>(phase_bit);
           if (leader) {
-            if (rank == 0) mbar_arrive_expect_tx(full0 + 8 * stage, 2 * kPairStageBytes);
-            tma_load_3d_pair(smem_u32(sB + stage * kPairBBytes), mb, fb_leader, 0,
-                             kb * kGemmBK, n * 4 + static_cast<int>(rank) * 2);
+            if (rank == 0) mbar_arrive_expect_tx(full0 + 8 * stage, stage_bytes);
+            if (wide)
+              tma_load_3d_pair(smem_u32(sB + stage * kPairBBytes), mb, fb_leader, 0, kb * 64,
+                               n * 8 + static_cast<int>(rank) * 4);
+            else
+              tma_load_3d_pair(smem_u32(sB + stage * kPairBBytes), mb, fb_leader, 0,
+                               kb * kGemmBK, n * 4 + static_cast<int>(rank) * 2);
           }
           __syncwarp();
-          // A of the first H chunk / Z tile waits for LN2 / the whole hidden
+          // A of item j's first H chunk / Z tile waits for its LN2 / whole hidden
           if (kb == 0 && n == 0 && ph > 0) {
-            if (!mbar_wait_warp(ph == 1 ? v_ready : h_ready, it_par, abort_flag, p.err,
-                                kSiteGemmProducer)) {
+            if (!mbar_wait_warp(ph == 1 ? v_ready : h_ready, static_cast<uint32_t>(j & 1),
+                                abort_flag, p.err, kSiteGemmProducer)) {
               ok = false;
               break;
             }
           }
-          const bool lost = p.fault == 3 && pair == 0 && rank == 0 && item == pair && t == 0 &&
+          const bool lost = p.fault == 3 && pair == 0 && rank == 0 && sg == 0 && n == 0 &&
                             kb == 0;
           if (leader && !lost)
-            tma_load_3d_pair(smem_u32(sA + stage * kPairABytes), ma, fb_leader, 0, a_row, kb * 2);
+            tma_load_3d_pair(smem_u32(sA + stage * kPairABytes), ma, fb_leader, 0, a_row,
+                             wide ? kb : kb * 2);
           __syncwarp();
           if (++stage == kPairStages) {
             stage = 0;
@@ -292,30 +333,61 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTailThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int item = pair; item < p.items && ok; item += npairs) {
-      for (int t = 0; t < tiles && ok; ++t) {
-        int ph, n;
-        sh.at(t, ph, n);
-        const int kbs = sh.kblocks(ph);
-        if (!mbar_wait_warp(acce0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.err, kSiteGemmMma)) {
+    auto next_slot = [&]() {
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    };
+    for (int sg = 0; sg < n_seg && ok; ++sg) {
+      int ph, j;
+      tail_segment(sg, J, ph, j);
+      const bool wide = ph == 2 && sh.e512;
+      const int kbs = sh.kblocks(ph);
+      const int tiles = ph == 0 ? sh.nB : (ph == 1 ? sh.nD : sh.nE);
+      for (int n = 0; n < tiles && ok; ++n) {
+        // accumulator slots: one, or two consecutive for a 512-column tile
+        const int s0 = acc;
+        const uint32_t p0 = acc_phase;
+        next_slot();
+        const int s1 = acc;
+        const uint32_t p1 = acc_phase;
+        if (wide) next_slot();
+        if (!mbar_wait_warp(acce0 + 8 * s0, p0 ^ 1u, abort_flag, p.err, kSiteGemmMma) ||
+            (wide && !mbar_wait_warp(acce0 + 8 * s1, p1 ^ 1u, abort_flag, p.err, kSiteGemmMma))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * kGemmBN);
+        const uint32_t d0 = tmem + static_cast<uint32_t>(s0 * kGemmBN);
+        const uint32_t d1 = tmem + static_cast<uint32_t>(s1 * kGemmBN);
         for (int kb = 0; kb < kbs; ++kb) {
           if (!mbar_wait_warp(full0 + 8 * stage, phase_bit, abort_flag, p.err, kSiteGemmMma)) {
             ok = false;
             break;
           }
           const uint32_t a_lo = sdesc_lo(smem_u32(sA + stage * kPairABytes), 16);
-          const uint32_t b_lo = sdesc_lo(smem_u32(sB + stage * kPairBBytes), kPairBBytes / 2);
           constexpr uint32_t hi = sdesc_hi(1024);
           if (leader) {
+            if (wide) {
+              // A: one 64-column chunk (four 16-deep k-steps of 32 bytes); B:
+              // [4 chunks][64 K rows][64], instruction i on chunks 2i, 2i+1
+              const uint32_t b0 = sdesc_lo(smem_u32(sB + stage * kPairBBytes), 8192);
+              const uint32_t b1 = sdesc_lo(smem_u32(sB + stage * kPairBBytes + 16384), 8192);
 #pragma unroll
-            for (int k = 0; k < kGemmBK / 16; ++k)
-              umma_ss_pair(d_tmem, a_lo + (k >> 2) * ((kPairABytes / 2) >> 4) + 2u * (k & 3), hi,
-                           b_lo + 128u * k, hi, idesc, (kb | k) != 0 ? 1u : 0u);
+              for (int k = 0; k < 4; ++k) {
+                const uint32_t accum = (kb | k) != 0 ? 1u : 0u;
+                umma_ss_pair(d0, a_lo + 2u * k, hi, b0 + 128u * k, hi, idesc, accum);
+                umma_ss_pair(d1, a_lo + 2u * k, hi, b1 + 128u * k, hi, idesc, accum);
+              }
+            } else {
+              const uint32_t b_lo =
+                  sdesc_lo(smem_u32(sB + stage * kPairBBytes), kPairBBytes / 2);
+#pragma unroll
+              for (int k = 0; k < kGemmBK / 16; ++k)
+                umma_ss_pair(d0, a_lo + (k >> 2) * ((kPairABytes / 2) >> 4) + 2u * (k & 3), hi,
+                             b_lo + 128u * k, hi, idesc, (kb | k) != 0 ? 1u : 0u);
+            }
             umma_commit_pair_mc(empty0 + 8 * stage, 0x3);
           }
           __syncwarp();
@@ -325,12 +397,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTailThreads, 1)
           }
         }
         if (!ok) break;
-        if (leader) umma_commit_pair_mc(accf0 + 8 * acc, 0x3);
-        __syncwarp();
-        if (++acc == 2) {
-          acc = 0;
-          acc_phase ^= 1u;
+        if (leader) {
+          umma_commit_pair_mc(accf0 + 8 * s0, 0x3);
+          if (wide) umma_commit_pair_mc(accf0 + 8 * s1, 0x3);
         }
+        __syncwarp();
       }
     }
     if (leader) umma_commit_pair(drain);
@@ -344,46 +415,56 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTailThreads, 1)
     const int part = ew >> 2;
     int acc = 0;
     uint32_t acc_phase = 0;
-    uint32_t it_par = 0;
     const int s_base = static_cast<int>(rank) * 128;
     const long long v_row0 = static_cast<long long>(pair) * 256 + s_base;
     bool ok = true;
-    for (int item = pair; item < p.items && ok; item += npairs, it_par ^= 1u) {
+    for (int sg = 0; sg < n_seg && ok; ++sg) {
+      int ph, j;
+      tail_segment(sg, J, ph, j);
+      const int item = pair + j * npairs;
       const int m_valid = 2 * item + 1 < p.blocks ? 256 : 128;
       const RowMap map{2 * item, p.nb, p.N, 128, 0};
       GemmParams gp{};
       gp.err = p.err;
-      for (int t = 0; t < tiles && ok; ++t) {
-        int ph, n;
-        sh.at(t, ph, n);
+      if (ph == 1) {
+        gp.epi = kEpiGeluBias;
+        gp.M = 0x7fffffff;
+        gp.N = p.d_ff;
+        gp.out_h = p.h_scr;
+        gp.ld_out = p.d_ff;
+        gp.bias = p.b1;
+      } else {
+        gp.epi = ph == 0 ? kEpiResidX : kEpiBiasAccum;
+        gp.M = m_valid;
+        gp.N = p.d;
+        gp.out_f32 = p.out;
+        gp.ld_f32 = p.d;
+        gp.resid = p.x;
+        gp.ld_resid = p.d;
+        gp.bias = p.b2;
+        gp.map = map;
+      }
+      // logical 256-column tiles of the segment
+      const int tiles = ph == 0 ? sh.nB : (ph == 1 ? sh.nD : (sh.e512 ? 2 * sh.nE : sh.nE));
+      for (int n = 0; n < tiles && ok; ++n) {
+        int col;
+        if (ph == 2 && sh.e512)
+          // Z tile T = n / 2: CTA r loaded columns 512T + 256r .. +255 as B, and
+          // instruction i = n % 2 took 128 of them from each CTA (TMEM columns
+          // 0..127 from CTA 0, 128..255 from CTA 1): part j holds 512T + 256j + 128i
+          col = (n >> 1) * 512 + part * 256 + (n & 1) * 128;
+        else
+          col = n * kGemmBN + part * kCols;
         if (!mbar_wait_fast(accf0 + 8 * acc, acc_phase, abort_flag, p.err, kSiteGemmEpilogue)) {
           ok = false;
           break;
         }
         tc_fence_after();
         long long row = s_base + e * 32 + lane;  // item-local row (mapped), or scratch row
-        if (ph == 1) {
-          gp.epi = kEpiGeluBias;
-          gp.M = 0x7fffffff;
-          gp.N = p.d_ff;
-          gp.out_h = p.h_scr;
-          gp.ld_out = p.d_ff;
-          gp.bias = p.b1;
-          row += static_cast<long long>(pair) * 256;
-        } else {
-          gp.epi = ph == 0 ? kEpiResidX : kEpiBiasAccum;
-          gp.M = m_valid;
-          gp.N = p.d;
-          gp.out_f32 = p.out;
-          gp.ld_f32 = p.d;
-          gp.resid = p.x;
-          gp.ld_resid = p.d;
-          gp.bias = p.b2;
-          gp.map = map;
-        }
+        if (ph == 1) row += static_cast<long long>(pair) * 256;
         const uint32_t t_row = tmem + (static_cast<uint32_t>(e * 32) << 16) +
                                static_cast<uint32_t>(acc * kGemmBN + part * kCols);
-        gemm_epilogue_row(gp, t_row, row, n * kGemmBN + part * kCols, kCols);
+        gemm_epilogue_row(gp, t_row, row, col, kCols);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(map_to_rank(acce0 + 8 * acc, 0));
@@ -391,23 +472,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTailThreads, 1)
           acc = 0;
           acc_phase ^= 1u;
         }
-        if (ph == 0 && n == sh.nB - 1) {
-          // every y tile of the item is stored: LN2 of the CTA's rows
-          if (lane == 0) mbar_arrive(ep_sync);
-          if (!mbar_wait_fast(ep_sync, it_par, abort_flag, p.err, kSiteGemmEpilogue)) {
-            ok = false;
-            break;
-          }
-          tail_ln2(p, map, m_valid, s_base, v_row0, ew, lane);
-          fence_proxy_async_global();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(v_ready);
-        } else if (ph == 1 && n == sh.nD - 1) {
-          // every H chunk of the item is stored
-          fence_proxy_async_global();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(h_ready);
+      }
+      if (!ok) break;
+      if (ph == 0) {
+        // every y tile of item j is stored: LN2 of the CTA's rows
+        if (lane == 0) mbar_arrive(ep_sync);
+        if (!mbar_wait_fast(ep_sync, static_cast<uint32_t>(j & 1), abort_flag, p.err,
+                            kSiteGemmEpilogue)) {
+          ok = false;
+          break;
         }
+        tail_ln2(p, map, m_valid, s_base, v_row0, ew, lane);
+        fence_proxy_async_global();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(v_ready);
+      } else if (ph == 1) {
+        // every H chunk of item j is stored
+        fence_proxy_async_global();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(h_ready);
       }
     }
   }

@@ -267,8 +267,9 @@ bpt_status bpt_layer_forward_train(const void* x, const void* ln1, const void* W
  *              0 where pruned; unvisited pairs untouched.
  * block_max and kept must not overlap x, out, the workspace, thresholds or
  * each other.  Every other argument, the supported shapes and the workspace
- * are those of bpt_layer_forward.  V tiles are still loaded for pruned
- * blocks (the K/V ring fetches them before the scores exist).
+ * are those of bpt_layer_forward.  The value tile of a block is loaded only
+ * when a query block that visits it keeps it (the kernel fetches V after the
+ * gate decisions; the two query blocks of an attention CTA share each tile).
  * Returns BPT_ERR_UNSUPPORTED for dtype BPT_F32, BPT_ERR_INVALID_ARG for a
  * NULL, misaligned or overlapping buffer; otherwise as bpt_layer_forward.
  */
@@ -360,6 +361,57 @@ bpt_status bpt_layer_backward_opt(const void* x, const void* ln1, const void* W_
                                   float* dW_2, float* db_2, void* workspace,
                                   size_t workspace_bytes, const bpt_options* opts,
                                   bpt_stream_t stream);
+
+/*
+ * Sequence sharding over G GPUs ("Blockwise Parallel Transformer — BPT",
+ * section "BPT and Ring Attention": BPT is the per-device kernel and the
+ * sequence is split across devices, each device's queries needing the keys
+ * and values of the others; section "Why parallel is in the name": query
+ * blocks are independent).  Zig-zag ownership balances the causal work: the
+ * sequence of N tokens is cut into 2G chunks of N / (2G) tokens and rank r
+ * owns chunks r and 2G-1-r; its n_loc = N / G local rows are chunk r
+ * followed by chunk 2G-1-r, in token order within each.  Per forward, each
+ * rank calls
+ *   1. bpt_layer_shard_project: LN1 and the Q/K/V projection of its own
+ *      rows; writes K | V of those rows to kv_loc [B, n_loc, 2d] fp16 and
+ *      keeps Q (and the fp16 weights) in its workspace;
+ *   2. an all-gather of kv_loc over the G ranks into kv_all
+ *      [G, B, n_loc, 2d] fp16 in this GPU's memory, rank-major (one NCCL
+ *      all_gather_into_tensor; the library does no communication);
+ *   3. bpt_layer_shard_forward: attention of its rows against every rank's
+ *      K | V (read from kv_all through the chunk ownership, no reordering
+ *      copy), then the fused layer body; writes Z of its rows to out
+ *      [B, n_loc, d] fp32.
+ * Step 3 must get the workspace step 1 used, unchanged, and the parameters
+ * of step 1.  The output rows equal bitwise those of bpt_layer_forward on
+ * the whole sequence (same per-element arithmetic).
+ * Supported: BPT_BF16 only; N % (256 G) == 0 (whole 128-token blocks per
+ * chunk); G >= 1; 0 <= rank < G; the shapes of bpt_layer_forward for
+ * n_loc tokens.  x is the rank's local rows [B, n_loc, d].  kv_loc / kv_all
+ * must not overlap out, the workspace or the inputs.  The workspace size is
+ * bpt_layer_shard_workspace_size (that of bpt_layer_workspace_size for
+ * n_loc tokens).  Returns BPT_ERR_UNSUPPORTED for other dtypes or N, and as
+ * bpt_layer_forward otherwise.
+ */
+bpt_status bpt_layer_shard_workspace_size(int64_t B, int64_t N, int64_t G, int64_t d,
+                                          int64_t h, int64_t d_ff, int causal, bpt_dtype dtype,
+                                          size_t* bytes);
+bpt_status bpt_layer_shard_project(const void* x, const void* ln1, const void* W_Q,
+                                   const void* W_K, const void* W_V, const void* W_O,
+                                   const void* ln2, const void* W_1, const void* b_1,
+                                   const void* W_2, const void* b_2, int64_t B, int64_t N,
+                                   int64_t G, int64_t rank, int64_t d, int64_t h, int64_t d_ff,
+                                   int causal, bpt_dtype dtype, void* kv_loc, float* out,
+                                   void* workspace, size_t workspace_bytes,
+                                   bpt_stream_t stream);
+bpt_status bpt_layer_shard_forward(const void* x, const void* ln1, const void* W_Q,
+                                   const void* W_K, const void* W_V, const void* W_O,
+                                   const void* ln2, const void* W_1, const void* b_1,
+                                   const void* W_2, const void* b_2, int64_t B, int64_t N,
+                                   int64_t G, int64_t rank, int64_t d, int64_t h, int64_t d_ff,
+                                   int causal, bpt_dtype dtype, const void* kv_all, float* out,
+                                   void* workspace, size_t workspace_bytes,
+                                   bpt_stream_t stream);
 
 /*
  * bpt_read_device_error -- synchronises `stream`, reads and clears the error

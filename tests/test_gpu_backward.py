@@ -6,11 +6,13 @@ accumulates the gradients; the oracle is the chain rule through the unfused
 layer (``oracle.layer_backward``, pinned against torch autograd).
 
 Tolerance (bf16 layers).  Every GEMM operand on the backward path is rounded to fp16
-(relative 2^-11 ~ 4.9e-4) and the longest chain (dZ -> dH -> dHpre -> dVn ->
-dY -> dO -> dS -> dQ, dK, dV -> dU -> dx) passes about ten such roundings,
-each product accumulated in fp32: per-element relative error of order 5e-3.
-Each gradient tensor is held to a relative L2 error of 1e-2 and a largest
-elementwise error of 5 % of the tensor's largest magnitude.
+(relative error <= 2^-11 ~ 4.9e-4, ~2.8e-4 rms for a uniformly distributed
+rounding error) and the longest chain (dZ -> dH -> dHpre -> dVn -> dY -> dO
+-> dS -> dQ, dK, dV -> dU -> dx) passes about ten such roundings, each
+product accumulated in fp32: independent roundings give a relative rms error
+near sqrt(10) x 2.8e-4 ~ 9e-4.  Each gradient tensor is held to a relative L2
+error of 3e-3 (3x that) and a largest elementwise error of 1 % of the
+tensor's largest magnitude (a few rms).  Measured: <= 7.7e-4 and <= 1.2e-3.
 """
 import numpy as np
 import pytest
@@ -18,7 +20,7 @@ import torch
 
 import blockwise_attn_ffn_b200 as bpt
 import oracle
-from blockwise_attn_ffn_b200.inputs import LayerShape, make_inputs
+from blockwise_attn_ffn_b200.inputs import WORKLOADS, LayerShape, make_inputs
 from test_gpu_parity import small
 
 pytestmark = pytest.mark.gpu
@@ -58,8 +60,8 @@ def check(name, got, want):
     rel_l2 = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
     mx = np.abs(got - want).max()
     print(f"  {name:12s} rel L2 {rel_l2:.2e}  max {mx / max(scale, 1e-30):.2e} of scale")
-    assert rel_l2 <= 1e-2, f"{name}: relative L2 error {rel_l2:.3e}"
-    assert mx <= 5e-2 * scale, f"{name}: max abs error {mx:.3e} vs scale {scale:.3e}"
+    assert rel_l2 <= 3e-3, f"{name}: relative L2 error {rel_l2:.3e}"
+    assert mx <= 1e-2 * scale, f"{name}: max abs error {mx:.3e} vs scale {scale:.3e}"
     return rel_l2
 
 
@@ -151,3 +153,20 @@ def test_f32_backward_multi_wave():
     for k in NAMES:
         check_f32(k, got[k], want[k])
 
+
+
+def test_backward_full_gpt2_small_workload():
+    """Every gradient of the whole GPT-2-small-shaped workload (B 8, N 2048,
+    d 768, 12 heads, d_ff 3072, causal) against the fp64 backward oracle:
+    the full-size check of the block recomputation at the shape it runs in
+    production, every element compared."""
+    cfg = WORKLOADS["gpt2s_n2k"]
+    inp = make_inputs(cfg)
+    dZ = upstream(cfg)
+    got = run_backward(cfg, inp, dZ)
+    want = oracle.layer_backward(inp, cfg.h, cfg.causal, dZ.astype(np.float64))
+    for k in NAMES:
+        check(k, got[k], want[k])
+    for k, (g, b) in {"ln1": ("gamma1", "beta1"), "ln2": ("gamma2", "beta2")}.items():
+        check(k + ".gamma", got[k][0], want[g])
+        check(k + ".beta", got[k][1], want[b])
