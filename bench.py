@@ -39,14 +39,14 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per attention
-# launch, the mean over one step's launches, from one ncu capture of the
-# default bench command.  Valid only for the sources it was taken on: the
-# digest covers the attention kernel, the shared device helpers and the host
-# launch code; after any change the bench reports null until it is retaken.
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
+# launch of the default bench command, from a one-kernel, one-launch ncu
+# capture with those two metrics only (one pass: nothing saved or replayed;
+# profiles/attn_pair_tc_long_n64k_dram.md).  Valid only for the sources it was
+# taken on: the digest covers the attention kernel, the shared device helpers
+# and the host launch code; after a change the bench reports null until the
+# one-launch capture is taken again.
 ATTN_TRAFFIC = {
-    # 12 launches (6 forwards x 2 waves): waves of 405 + 114 and 1286 + 127 MB
-    "long_n64k": {"digest": "959c59fdb1694afd", "bytes_per_launch": 966207189},
 }
 TRAFFIC_SOURCES = ("blockwise_attn_ffn_b200/csrc/attn_pair_tc.cuh",
                    "blockwise_attn_ffn_b200/csrc/common.cuh",
@@ -566,9 +566,10 @@ def main():
     ap.add_argument("--schedule", default="fused", choices=["fused", "waves"],
                     help="layer body after attention: one persistent per-block kernel "
                          "(fused) or wave-level kernels (waves)")
-    ap.add_argument("--attn-qpc", type=int, default=2, choices=[1, 2],
-                    help="query blocks per attention CTA (2: paired, 256 query rows per "
-                         "K/V tile; 1: one 128-row block)")
+    ap.add_argument("--attn-qpc", type=int, default=2, choices=[1, 2, 4],
+                    help="query rows per K/V tile in 128-row blocks (2: two blocks per CTA, "
+                         "256 rows; 1: one block, 128 rows; 4: a cluster of two CTAs sharing "
+                         "each tile over DSMEM, 512 rows)")
     ap.add_argument("--no-other-workloads", action="store_true",
                     help="skip timing the other four workloads")
     ap.add_argument("--no-alt-schedule", action="store_true",

@@ -149,6 +149,30 @@ __device__ __forceinline__ void attn_pair_decode(const AttnPairParams& p, int ra
   }
 }
 
+// XP: work rank -> the first block item of the cluster's four query blocks
+// and how many of them exist (1..4).  Longest first, as attn_pair_decode.
+__device__ __forceinline__ void attn_quad_decode(const AttnPairParams& p, int rank, int& item0q,
+                                                 int& nq) {
+  if (p.seqs == 0) {
+    const int nunits = (p.count + 3) / 4;
+    const int q = p.causal ? (nunits - 1 - rank) : rank;
+    item0q = p.item0 + 4 * q;
+    nq = min(4, p.count - 4 * q);
+  } else {
+    const int pp = (p.nb + 3) / 4;  // units per sequence
+    int s, q;
+    if (p.causal) {
+      q = pp - 1 - rank / p.seqs;
+      s = rank % p.seqs;
+    } else {
+      s = rank / pp;
+      q = rank % pp;
+    }
+    item0q = p.item0 + s * p.nb + 4 * q;
+    nq = min(4, p.nb - 4 * q);
+  }
+}
+
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -216,10 +240,21 @@ __device__ __forceinline__ int shard_global_block(const AttnPairParams& p, int i
 // slot without a load when every visiting tile prunes it, so pruned blocks
 // cost no V traffic ("Block Sparse Flash Attention", "Methodology and
 // Mechanism": a pruned block's values are neither loaded nor multiplied).
-template <int D, int EMU, bool GATE = false, bool SHARD = false>
+// XP: b = 512.  A cluster of two CTAs takes four consecutive query blocks
+// (two per CTA) and shares every K/V tile: each CTA TMA-loads one 64-key half
+// of each tile from L2 (mapKV: 64-row boxes of QKV) and copies it into the
+// partner's ring slot over DSMEM (a shared-to-shared bulk copy; no multicast
+// load), so each K/V byte fetched from L2 serves 512 query rows.  The
+// products stay per CTA (same arithmetic as b = 256).  Ring barriers then
+// count both CTAs: a slot is full when the own half has landed (the copier
+// warp's arrive) and the partner's copy has (its bytes), and empty when both
+// CTAs' UMMA warps have released it (multicast commit).  Both CTAs walk the
+// key blocks of all four query blocks.
+template <int D, int EMU, bool GATE = false, bool SHARD = false, bool XP = false>
 __global__ void __launch_bounds__(384, 1)
     attn_pair_tc_kernel(const __grid_constant__ CUtensorMap mapQKV,
                         const __grid_constant__ CUtensorMap mapKV, const AttnPairParams p) {
+  static_assert(!(XP && (GATE || SHARD)), "the b = 512 pair is dense and unsharded");
   using C = AttnPairCfg<D, EMU>;
   constexpr int kFwdHandovers = fwd_handovers<D>();
   constexpr int kFwdChunksPerHand = 4 / kFwdHandovers;
@@ -235,6 +270,7 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t p_chunk0 = smem_u32(bars + 3 + 2 * C::NSLOT);
   const uint32_t o_done0 = smem_u32(bars + 11 + 2 * C::NSLOT);  // [A, B]
   const uint32_t drain = smem_u32(bars + 13 + 2 * C::NSLOT);
+  const uint32_t half0 = smem_u32(bars + 14 + 2 * C::NSLOT);  // XP: own half landed
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   // per tile, per softmax warp: {max of its rows (float bits), block count}
@@ -247,15 +283,35 @@ __global__ void __launch_bounds__(384, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // blockIdx -> (head group, work rank, head): within a group, consecutive
-  // CTAs take the group's heads for one rank, longest ranks first.
-  const int per_group = int(gridDim.x / p.h) * p.hg;
-  const int grp = blockIdx.x / per_group;
-  const int in_grp = blockIdx.x - grp * per_group;
-  const int rank = in_grp / p.hg;
-  const int head = grp * p.hg + (in_grp - rank * p.hg);
-  int itemA;
+  // CTAs (XP: clusters) take the group's heads for one rank, longest ranks
+  // first.
+  int itemA, head;
   bool has_b;
-  attn_pair_decode(p, rank, itemA, has_b);
+  int xr = 0;         // XP: rank in the cluster
+  bool has_a = true;  // XP: the CTA has query blocks
+  int last_item = 0;  // XP: the last block item of the cluster's four
+  if constexpr (XP) {
+    xr = int(blockIdx.x & 1);
+    const int cl = int(blockIdx.x >> 1);
+    const int per_group = int(gridDim.x / 2 / p.h) * p.hg;
+    const int grp = cl / per_group;
+    const int in_grp = cl - grp * per_group;
+    const int rank = in_grp / p.hg;
+    head = grp * p.hg + (in_grp - rank * p.hg);
+    int item0q, nq;
+    attn_quad_decode(p, rank, item0q, nq);
+    has_a = 2 * xr < nq;
+    has_b = 2 * xr + 1 < nq;
+    itemA = has_a ? item0q + 2 * xr : item0q;
+    last_item = item0q + nq - 1;
+  } else {
+    const int per_group = int(gridDim.x / p.h) * p.hg;
+    const int grp = blockIdx.x / per_group;
+    const int in_grp = blockIdx.x - grp * per_group;
+    const int rank = in_grp / p.hg;
+    head = grp * p.hg + (in_grp - rank * p.hg);
+    attn_pair_decode(p, rank, itemA, has_b);
+  }
   const int bidx = itemA / p.nb;
   const int iA = itemA - bidx * p.nb;
   const int iB = iA + 1;
@@ -264,15 +320,18 @@ __global__ void __launch_bounds__(384, 1)
   const int gA = SHARD ? shard_global_block(p, iA) : iA;
   const int gB = SHARD ? shard_global_block(p, iB) : iB;
   const int nb_kv = SHARD ? p.N_kv / C::BKV : p.nb;
-  const int nA = p.causal ? gA + 1 : nb_kv;
+  const int nA = XP && !has_a ? 0 : (p.causal ? gA + 1 : nb_kv);
   const int nB = has_b ? (p.causal ? gB + 1 : nb_kv) : 0;
-  const int n_kv = nA > nB ? nA : nB;
+  // key blocks the ring carries: this CTA's, or (XP) the cluster's
+  int n_kv = nA > nB ? nA : nB;
+  if constexpr (XP) n_kv = p.causal ? last_item - bidx * p.nb + 1 : nb_kv;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < C::NSLOT; ++s) {
-      mbar_init(ring_full0 + 8 * s, 1);
-      mbar_init(ring_empty0 + 8 * s, 1);
+      mbar_init(ring_full0 + 8 * s, XP ? 2 : 1);
+      mbar_init(ring_empty0 + 8 * s, XP ? 2 : 1);
+      if constexpr (XP) mbar_init(half0 + 8 * s, 1);
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(s_full0 + 8 * x, 1);
@@ -293,6 +352,7 @@ __global__ void __launch_bounds__(384, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (XP) cluster_sync();  // the partner's barriers exist before any copy
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
   volatile int* abort_flag = &abort_sh;
@@ -310,15 +370,53 @@ __global__ void __launch_bounds__(384, 1)
     int armed[C::NSLOT];
     for (int s = 0; s < C::NSLOT; ++s) armed[s] = -1;
     if (leader) {
-      mbar_arrive_expect_tx(q_full, C::TILE * (has_b ? 2 : 1));
-      tma_load_4d(smem_u32(smem + C::OFF_QA), &mapQKV, q_full, 0, iA * C::BQ, colQ / 64, bidx);
+      if constexpr (XP) {
+        mbar_arrive_expect_tx(q_full, C::TILE * ((has_a ? 1 : 0) + (has_b ? 1 : 0)));
+        if (has_a)
+          tma_load_4d(smem_u32(smem + C::OFF_QA), &mapQKV, q_full, 0, iA * C::BQ, colQ / 64,
+                      bidx);
+      } else {
+        mbar_arrive_expect_tx(q_full, C::TILE * (has_b ? 2 : 1));
+        tma_load_4d(smem_u32(smem + C::OFF_QA), &mapQKV, q_full, 0, iA * C::BQ, colQ / 64, bidx);
+      }
       if (has_b)
         tma_load_4d(smem_u32(smem + C::OFF_QB), &mapQKV, q_full, 0, iB * C::BQ, colQ / 64, bidx);
     }
     int slot = 0;
     uint32_t phase = 0;
     bool ok = true;
-    if constexpr (!GATE) {
+    if constexpr (XP) {
+      // this CTA's 64-key half of every K/V tile: one 8 KB box per 64-column
+      // chunk (rows 64 xr .. of the chunk); the partner's half arrives by copy
+      int armed_h[C::NSLOT];
+      for (int s = 0; s < C::NSLOT; ++s) armed_h[s] = -1;
+      for (int t = 0; t < 2 * n_kv && ok; ++t) {
+        const int j = t >> 1, w = t & 1;
+        if (!mbar_wait_warp(ring_empty0 + 8 * slot, phase ^ 1u, abort_flag, p.err,
+                            kSiteAttnProducer)) {
+          ok = false;
+          break;
+        }
+        armed[slot] = static_cast<int>(phase);
+        armed_h[slot] = static_cast<int>(phase);
+        if (leader) {
+          mbar_arrive_expect_tx(ring_full0 + 8 * slot, C::TILE / 2);  // the partner's half
+          mbar_arrive_expect_tx(half0 + 8 * slot, C::TILE / 2);
+          const int col = w == 0 ? colK : colV;
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_4d(smem_u32(smem + C::OFF_RING + slot * C::TILE + c * C::CHUNK + xr * 8192),
+                        &mapKV, half0 + 8 * slot, 0, j * C::BKV + xr * 64, col / 64 + c, bidx);
+        }
+        __syncwarp();
+        if (++slot == C::NSLOT) {
+          slot = 0;
+          phase ^= 1u;
+        }
+      }
+      for (int s = 0; s < C::NSLOT; ++s)
+        if (armed_h[s] >= 0) mbar_wait_drain(half0 + 8 * s, static_cast<uint32_t>(armed_h[s]), p.err);
+    } else if constexpr (!GATE) {
       // ring order K_0 V_0 K_1 V_1 ...
       for (int j = 0; j < n_kv && ok; ++j) {
         for (int w = 0; w < 2; ++w) {
@@ -433,6 +531,29 @@ __global__ void __launch_bounds__(384, 1)
     mbar_wait_drain(q_full, 0, p.err);
     for (int s = 0; s < C::NSLOT; ++s)
       if (armed[s] >= 0) mbar_wait_drain(ring_full0 + 8 * s, static_cast<uint32_t>(armed[s]), p.err);
+  } else if (XP && warp == 3) {
+    // ------------------------------------------- XP: copy own halves across
+    const bool leader = elect_one();
+    const uint32_t peer = static_cast<uint32_t>(xr ^ 1);
+    int slot = 0;
+    uint32_t phase = 0;
+    for (int t = 0; t < 2 * n_kv; ++t) {
+      if (!mbar_wait_warp(half0 + 8 * slot, phase, abort_flag, p.err, kSiteAttnProducer)) break;
+      if (leader) {
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          const uint32_t off = C::OFF_RING + slot * C::TILE + c * C::CHUNK + xr * 8192;
+          bulk_copy_to_peer(map_to_rank(smem_u32(smem + off), peer), smem_u32(smem + off), 8192,
+                            map_to_rank(ring_full0 + 8 * slot, peer));
+        }
+        mbar_arrive(ring_full0 + 8 * slot);  // own half landed
+      }
+      __syncwarp();
+      if (++slot == C::NSLOT) {
+        slot = 0;
+        phase ^= 1u;
+      }
+    }
   } else if (warp == 1) {
     // ----------------------------------------------------------- UMMA issue
     // The whole warp runs the role so that descriptors stay warp-uniform; the
@@ -478,6 +599,16 @@ __global__ void __launch_bounds__(384, 1)
       if (leader) umma_commit(bar);
       __syncwarp();
     };
+    // a ring slot is released to both CTAs of an XP cluster
+    auto release = [&](uint32_t bar) {
+      if (leader) {
+        if constexpr (XP)
+          umma_commit_mc(bar, 0x3);
+        else
+          umma_commit(bar);
+      }
+      __syncwarp();
+    };
     uint32_t pph[2] = {0, 0};
     bool o_started[2] = {false, false};  // first PV of a tile overwrites O
     bool ok = mbar_wait_warp(q_full, 0, abort_flag, p.err, kSiteAttnMma);
@@ -495,7 +626,7 @@ __global__ void __launch_bounds__(384, 1)
         issue_s(qb_lo, k0_lo, tmem + C::TM_S_B);
         commit(s_full0 + 8);
       }
-      commit(ring_empty0 + 8 * slot_of(0));
+      release(ring_empty0 + 8 * slot_of(0));
     }
     for (int j = 0; j < n_kv && ok; ++j) {
       // ring positions of K_j+1 and V_j (see the producer's order)
@@ -568,8 +699,15 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       if (!ok || !wait_v()) break;
-      commit(ring_empty0 + 8 * slot_of(tv));
-      if (k_ready) commit(ring_empty0 + 8 * slot_of(tk));
+      if (XP && !k_ready && j + 1 < n_kv) {
+        // the cluster's ring goes on past this CTA's blocks: consume K_j+1
+        if (!mbar_wait_warp(ring_full0 + 8 * slot_of(tk), phase_of(tk), abort_flag, p.err,
+                            kSiteAttnMma))
+          break;
+        k_ready = true;
+      }
+      release(ring_empty0 + 8 * slot_of(tv));
+      if (k_ready) release(ring_empty0 + 8 * slot_of(tk));
     }
     commit(drain);
     mbar_wait_drain(drain, 0, p.err);
@@ -803,6 +941,7 @@ __global__ void __launch_bounds__(384, 1)
 
   tc_fence_before();
   __syncthreads();
+  if constexpr (XP) cluster_sync();  // no copy into a CTA that has left
   tc_fence_after();
   if (warp == 2) tmem_dealloc(tmem, C::TMEM_COLS);
 }

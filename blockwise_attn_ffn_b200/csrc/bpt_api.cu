@@ -62,7 +62,8 @@ bpt_status read_opts(const bpt_options* o, Opts* r) {
   if (o->reserved != 0) return BPT_ERR_INVALID_ARG;
   if (o->schedule != BPT_SCHEDULE_FUSED && o->schedule != BPT_SCHEDULE_WAVES)
     return BPT_ERR_INVALID_ARG;
-  if (o->attn_qpc != 0 && o->attn_qpc != 1 && o->attn_qpc != 2) return BPT_ERR_INVALID_ARG;
+  if (o->attn_qpc != 0 && o->attn_qpc != 1 && o->attn_qpc != 2 && o->attn_qpc != 4)
+    return BPT_ERR_INVALID_ARG;
   if (o->max_wave < 0 || o->max_wave > kMaxWave) return BPT_ERR_INVALID_ARG;
   if (o->fault < 0 || o->fault > 3) return BPT_ERR_INVALID_ARG;
   r->fused = o->schedule == BPT_SCHEDULE_FUSED ? 1 : 0;
@@ -248,6 +249,10 @@ bpt_status device_info(int* sms, int* pair_clusters = nullptr) {
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                bpt::AttnPairCfg<128, kEmu128>::SMEM) != cudaSuccess ||
           set_smem(bpt::attn_pair_tc_kernel<64, kEmu64, true>, bpt::AttnPairCfg<64, kEmu64>::SMEM) ||
+          set_smem(bpt::attn_pair_tc_kernel<64, kEmu64, false, false, true>,
+                   bpt::AttnPairCfg<64, kEmu64>::SMEM) ||
+          set_smem(bpt::attn_pair_tc_kernel<128, kEmu128, false, false, true>,
+                   bpt::AttnPairCfg<128, kEmu128>::SMEM) ||
           set_smem(bpt::attn_pair_tc_kernel<64, kEmu64, false, true>,
                    bpt::AttnPairCfg<64, kEmu64>::SMEM) ||
           set_smem(bpt::attn_pair_tc_kernel<128, kEmu128, false, true>,
@@ -353,6 +358,15 @@ bool map_qkv(CUtensorMap* m, const void* base, int64_t B, int64_t N, int64_t d, 
   const uint64_t dims[4] = {64, uint64_t(N), uint64_t(3 * d / 64), uint64_t(B)};
   const uint64_t st[3] = {uint64_t(3 * d) * 2, 128, uint64_t(N) * uint64_t(3 * d) * 2};
   const uint32_t box[4] = {64, 128, uint32_t(dk / 64), 1};
+  return encode_f16(m, base, 4, dims, st, box);
+}
+
+// QKV viewed as map_qkv, 64-token boxes of one 64-column chunk (8 KB): the
+// half tiles a b = 512 attention cluster loads, one per CTA.
+bool map_qkv_half(CUtensorMap* m, const void* base, int64_t B, int64_t N, int64_t d) {
+  const uint64_t dims[4] = {64, uint64_t(N), uint64_t(3 * d / 64), uint64_t(B)};
+  const uint64_t st[3] = {uint64_t(3 * d) * 2, 128, uint64_t(N) * uint64_t(3 * d) * 2};
+  const uint32_t box[4] = {64, 64, 1, 1};
   return encode_f16(m, base, 4, dims, st, box);
 }
 
@@ -489,7 +503,7 @@ struct AttnShard {
 cudaError_t launch_attn(const Plan& P, const Wave& wv_, const CUtensorMap& mQKV, __half* so,
                         float* stats, uint32_t* err, int fault, cudaStream_t s,
                         const AttnGate* gate = nullptr, bool o_tok = false,
-                        const AttnShard* shard = nullptr) {
+                        const AttnShard* shard = nullptr, const CUtensorMap* xp_map = nullptr) {
   bpt::AttnPairParams ap{};
   ap.N = int(P.N); ap.nb = int(P.nb); ap.h = int(P.h); ap.d = int(P.d);
   ap.causal = P.causal; ap.item0 = int(wv_.item0); ap.count = int(wv_.count);
@@ -519,6 +533,29 @@ cudaError_t launch_attn(const Plan& P, const Wave& wv_, const CUtensorMap& mQKV,
                                       : wv_.seqs * ((P.nb + ap.qpc - 1) / ap.qpc);
   const unsigned grid = unsigned(units * P.h);
   const CUtensorMap& mKV = shard ? *shard->mKV : mQKV;
+  if (ap.qpc == 4) {
+    // b = 512: clusters of two CTAs, each with two query blocks, sharing K/V
+    if (gate != nullptr || shard != nullptr || xp_map == nullptr) return cudaErrorInvalidValue;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * grid);
+    cfg.blockDim = dim3(384);
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (P.dk == 128) {
+      cfg.dynamicSmemBytes = bpt::AttnPairCfg<128, kEmu128>::SMEM;
+      return cudaLaunchKernelEx(&cfg, bpt::attn_pair_tc_kernel<128, kEmu128, false, false, true>,
+                                mQKV, *xp_map, ap);
+    }
+    cfg.dynamicSmemBytes = bpt::AttnPairCfg<64, kEmu64>::SMEM;
+    return cudaLaunchKernelEx(&cfg, bpt::attn_pair_tc_kernel<64, kEmu64, false, false, true>,
+                              mQKV, *xp_map, ap);
+  }
   if (gate != nullptr) {
     ap.gate_t = gate->t;
     ap.gate_bmax = gate->bmax;
@@ -603,9 +640,10 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
   } else {
     ok = ok && map_a(&mO, so, R, d) && map_a(&mV, sv, R, d) && map_a(&mH, sh, R, d_ff);
   }
-  CUtensorMap mKV;
+  CUtensorMap mKV, mQKVh;
   if (shard != nullptr && shard->phase == 2)
     ok = ok && map_kv_shards(&mKV, shard->kv_all, shard->G, P.B, P.N, d, P.dk);
+  if (P.opt.qpc == 4) ok = ok && map_qkv_half(&mQKVh, qkv, P.B, P.N, d);
   if (!ok) return BPT_ERR_CUDA;
 
   RowMap ident{0, 1, 1, 1, 1};
@@ -668,7 +706,7 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
     {
       LaunchScope ls(BPT_KIND_ATTN, s);
       if (launch_attn(P, all, mQKV, qkv, stats, err, fault == 2 ? 2 : 0, s, gate, true,
-                      shard != nullptr ? &as : nullptr) != cudaSuccess)
+                      shard != nullptr ? &as : nullptr, &mQKVh) != cudaSuccess)
         return BPT_ERR_CUDA;
     }
     int dummy = 0, pairs_max = 0;
@@ -702,7 +740,8 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
     RowMap map{int(wv_.item0), int(P.nb), int(P.N), int(P.blk), 0};
     {
       LaunchScope ls(BPT_KIND_ATTN, s);
-      if (launch_attn(P, wv_, mQKV, so, stats, err, (fault == 2 && w == 0) ? 2 : 0, s, gate) !=
+      if (launch_attn(P, wv_, mQKV, so, stats, err, (fault == 2 && w == 0) ? 2 : 0, s, gate,
+                      false, nullptr, &mQKVh) !=
           cudaSuccess)
         return BPT_ERR_CUDA;
     }
@@ -1114,6 +1153,8 @@ bpt_status backward_bf16(const Plan& P, const BwdLayout& L, const void* x, const
             map_b(&mOt, so, R, d, 2) && map_b(&mDyB, dy16, R, d, 2) &&
             map_a(&mDyA, dy16, R, d) && map_a(&mWok, wo, d, d) && map_b(&mUt, u16, M, d, 2) &&
             map_a(&mDO, do16, R, d, 0, int(P.dk / 64));
+  CUtensorMap mQKVh;
+  if (P.opt.qpc == 4) ok = ok && map_qkv_half(&mQKVh, qkv, P.B, P.N, d);
   const hf* wqkv[3] = {wq, wk, wv};
   for (int i = 0; i < 3 && ok; ++i)
     ok = map_b(&mDqB[i], dqkv16 + i * d, M, d, 2, 3 * d) &&
@@ -1171,7 +1212,9 @@ bpt_status backward_bf16(const Plan& P, const BwdLayout& L, const void* x, const
     const int64_t rows = wv_.count * P.blk;
     RowMap map{int(wv_.item0), int(P.nb), int(P.N), int(P.blk), 0};
     // forward recomputation of this wave: o, y, LN2(y), FFN pre-activation and hidden
-    if (launch_attn(P, wv_, mQKV, so, nullptr, err, 0, s) != cudaSuccess) return BPT_ERR_CUDA;
+    if (launch_attn(P, wv_, mQKV, so, nullptr, err, 0, s, nullptr, false, nullptr, &mQKVh) !=
+        cudaSuccess)
+      return BPT_ERR_CUDA;
     if (!gemm(mO, mWo, rows, d, d, bpt::kEpiResidX, bpt::kLayAkBn, map, [&](bpt::GemmParams& g) {
           g.out_f32 = y; g.ld_f32 = d; g.resid = static_cast<const bf*>(x); g.ld_resid = d;
         }))
@@ -1302,6 +1345,7 @@ bpt_status layer_forward_impl(const void* x, const void* ln1, const void* W_Q, c
   st = read_opts(opts, &opt);
   if (st != BPT_OK) return st;
   if (gate != nullptr && dtype != BPT_BF16) return BPT_ERR_UNSUPPORTED;
+  if (gate != nullptr && opt.qpc == 4) return BPT_ERR_UNSUPPORTED;  // the b = 512 pair is dense
   if (B == 0 || N == 0) return BPT_OK;
   const void* ptrs[] = {x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, out, workspace};
   for (const void* p : ptrs)

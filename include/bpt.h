@@ -98,12 +98,16 @@ enum {
  *   schedule  BPT_SCHEDULE_FUSED or BPT_SCHEDULE_WAVES (bitwise: both run
  *             the same per-element arithmetic).  BPT_F32 layers always use
  *             waves.  The backward pass always uses waves.
- *   attn_qpc  query blocks per attention CTA: 0 = default (2), 1 or 2
- *             (bitwise).  2 pairs two 128-row query blocks in one CTA, so
- *             each K/V tile brought in serves 256 query rows ("Blockwise
- *             Parallel Transformer — BPT", section "Choosing the block size:
- *             arithmetic intensity": FLOPs per byte re-read equal the rows
- *             sharing it); 1 gives every query block its own CTA.
+ *   attn_qpc  query rows sharing each K/V tile, in 128-row blocks: 0 =
+ *             default (2), 1, 2 or 4 (bitwise).  2 pairs two query blocks in
+ *             one CTA, so each K/V tile brought in serves 256 query rows
+ *             ("Blockwise Parallel Transformer — BPT", section "Choosing the
+ *             block size: arithmetic intensity": FLOPs per byte re-read equal
+ *             the rows sharing it); 1 gives every query block its own CTA; 4
+ *             runs clusters of two such CTAs that each load half of every K/V
+ *             tile and copy it to the other over distributed shared memory
+ *             (512 rows per tile fetched; dense attention only: the gated
+ *             entry points return BPT_ERR_UNSUPPORTED with 4).
  *   max_wave  waves schedule only: query blocks per wave, 0 = default
  *             (BPT_WAVE_BLOCKS), else 1..BPT_WAVE_BLOCKS; small values make
  *             small layers run the multi-wave paths (a sequence split over

@@ -1,5 +1,6 @@
-"""Query blocks per attention CTA: paired (256 query rows share each K/V tile,
-the default) against one block per CTA (bpt_options.attn_qpc).
+"""Query rows sharing each K/V tile: one 128-row block per CTA (b = 128), two
+blocks per CTA (b = 256, the default) and a cluster of two such CTAs that
+exchange K/V halves over DSMEM (b = 512) (bpt_options.attn_qpc = 1, 2, 4).
 
 "Blockwise Parallel Transformer — BPT", section "Choosing the block size:
 arithmetic intensity": the work done per byte re-read grows with the rows
@@ -37,18 +38,49 @@ def forward_train(cfg, dev, opts):
 
 @pytest.mark.parametrize("schedule", ["fused", "waves"])
 @pytest.mark.parametrize("cfg,wave", CASES, ids=lambda c: getattr(c, "name", str(c)))
-def test_single_block_ctas_match_pairs_bitwise(cfg, wave, schedule):
+def test_block_sharing_is_bitwise_neutral(cfg, wave, schedule):
+    """One 128-row block per CTA (b = 128), two (b = 256, default) and a
+    cluster of two CTAs sharing each K/V tile over DSMEM (b = 512): the same
+    layer output and statistics, bit for bit."""
     dev = bpt.to_device(make_inputs(cfg), cfg.dtype)
     base = {"schedule": schedule, "max_wave": wave if schedule == "waves" else 0}
     out2, st2 = forward_train(cfg, dev, dict(base, attn_qpc=2))
     out1, st1 = forward_train(cfg, dev, dict(base, attn_qpc=1))
+    out4, st4 = forward_train(cfg, dev, dict(base, attn_qpc=4))
     assert np.all(np.isfinite(out2))
     np.testing.assert_array_equal(out1, out2)
     np.testing.assert_array_equal(st1, st2)
+    np.testing.assert_array_equal(out4, out2)
+    np.testing.assert_array_equal(st4, st2)
+
+
+def test_b512_backward_recomputation_matches():
+    """The backward's forward recomputation through the b = 512 attention
+    gives the same gradients as through the default one."""
+    cfg = CASES[0][0]
+    inp = make_inputs(cfg)
+    dev = bpt.to_device(inp, cfg.dtype)
+    _, stats, _ = bpt.layer_forward_train(dev["x"], dev, cfg.h, cfg.causal)
+    dZ = torch.from_numpy(np.random.default_rng(3).standard_normal(
+        (cfg.B, cfg.N, cfg.d)).astype(np.float32)).cuda()
+    g2, _ = bpt.layer_backward(dev["x"], dev, cfg.h, cfg.causal, stats, dZ)
+    g4, _ = bpt.layer_backward(dev["x"], dev, cfg.h, cfg.causal, stats, dZ,
+                               opts={"attn_qpc": 4})
+    for k in g2:
+        assert torch.equal(g2[k], g4[k]), k
+
+
+def test_b512_rejects_gating():
+    cfg = CASES[0][0]
+    dev = bpt.to_device(make_inputs(cfg), cfg.dtype)
+    nb = (cfg.N + 127) // 128
+    T = torch.full((cfg.h, nb), float("-inf"), dtype=torch.float32, device="cuda")
+    with pytest.raises(bpt.BptError):
+        bpt.layer_forward_bsfa(dev["x"], dev, cfg.h, cfg.causal, T, opts={"attn_qpc": 4})
 
 
 def test_qpc_rejects_other_values():
-    for bad in (3, -1):
+    for bad in (3, 5, -1):
         st, _ = bpt.bpt_layer_workspace_size_opt(1, 256, 256, 2, 512, True, bpt.BPT_BF16,
                                                  {"attn_qpc": bad})
         assert st == bpt.BPT_ERR_INVALID_ARG
