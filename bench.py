@@ -566,10 +566,10 @@ def main():
     ap.add_argument("--schedule", default="fused", choices=["fused", "waves"],
                     help="layer body after attention: one persistent per-block kernel "
                          "(fused) or wave-level kernels (waves)")
-    ap.add_argument("--attn-qpc", type=int, default=2, choices=[1, 2, 4],
-                    help="query rows per K/V tile in 128-row blocks (2: two blocks per CTA, "
-                         "256 rows; 1: one block, 128 rows; 4: a cluster of two CTAs sharing "
-                         "each tile over DSMEM, 512 rows)")
+    ap.add_argument("--attn-block", type=int, default=256, choices=[64, 128, 256, 512],
+                    help="b, the query rows sharing each K/V tile (256: two 128-row blocks "
+                         "per CTA; 128: one block per CTA; 64: one 64-row block per CTA, two "
+                         "CTAs per SM; 512: a cluster of two CTAs sharing each tile over DSMEM)")
     ap.add_argument("--no-other-workloads", action="store_true",
                     help="skip timing the other four workloads")
     ap.add_argument("--no-alt-schedule", action="store_true",
@@ -619,9 +619,9 @@ def main():
         x_host = bpt.to_device(inp, cfg.dtype, dev, pin_x=True)["x"]
     del inp
     x = p["x"]
-    opts = bpt.make_options(schedule=args.schedule, attn_qpc=args.attn_qpc)
+    opts = bpt.make_options(schedule=args.schedule, attn_block=args.attn_block)
     alt_sched = "waves" if args.schedule == "fused" else "fused"
-    alt_opts = bpt.make_options(schedule=alt_sched, attn_qpc=args.attn_qpc)
+    alt_opts = bpt.make_options(schedule=alt_sched, attn_block=args.attn_block)
 
     # Peak device bytes above the resident inputs (x and the parameters), for
     # each schedule: out + workspace of one forward.
@@ -755,7 +755,7 @@ def main():
                        "exactly each call), fp32 accumulation, fp32 residual stream and output")
         if cfg.dtype == "bf16" else "fp32 throughout (CUDA cores)",
         "data": "synthetic: seeded N(0,1) x, N(0,1/fan_in) weights, LN gamma~1+0.1N, beta~0.1N",
-        "config": dict(workload_config(cfg, world), attn_query_blocks_per_cta=args.attn_qpc,
+        "config": dict(workload_config(cfg, world), attn_block=args.attn_block,
                        schedule=args.schedule),
         "tflops": tflops,
         "pct_bf16_peak": tflops / world / peak_burst,

@@ -39,18 +39,18 @@ EXPORTED = [
 
 class Options(ctypes.Structure):
     """``bpt_options`` (include/bpt.h): per-call choices of the *_opt calls."""
-    _fields_ = [("schedule", ctypes.c_int32), ("attn_qpc", ctypes.c_int32),
+    _fields_ = [("schedule", ctypes.c_int32), ("attn_block", ctypes.c_int32),
                 ("max_wave", ctypes.c_int64), ("fault", ctypes.c_int32),
                 ("reserved", ctypes.c_int32)]
 
 
-def make_options(schedule=None, attn_qpc=0, max_wave=0, fault=0, reserved=0) -> Options:
+def make_options(schedule=None, attn_block=0, max_wave=0, fault=0, reserved=0) -> Options:
     """An ``Options`` value; ``schedule`` may be "fused", "waves" or the code."""
     if schedule is None or schedule == "fused":
         schedule = BPT_SCHEDULE_FUSED
     elif schedule == "waves":
         schedule = BPT_SCHEDULE_WAVES
-    return Options(int(schedule), int(attn_qpc), int(max_wave), int(fault), int(reserved))
+    return Options(int(schedule), int(attn_block), int(max_wave), int(fault), int(reserved))
 
 
 def _opts_ref(opts):

@@ -754,12 +754,12 @@ __global__ void __launch_bounds__(384, 1)
           if (k >= lim) sr[k] = __float_as_uint(-INFINITY);
       }
       // Row max as eight independent partial maxima (short dependency chains),
-      // three-input max.
+      // three-input max over columns k + q and k + 8 + q.
       float mxp[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mxp[k] = __uint_as_float(sr[k]);
+      for (int k = 0; k < 8; ++k) mxp[k] = -INFINITY;
 #pragma unroll
-      for (int k = 8; k < C::BKV; k += 16)
+      for (int k = 0; k < C::BKV; k += 16)
 #pragma unroll
         for (int q = 0; q < 8; ++q)
           mxp[q] = max3f(mxp[q], __uint_as_float(sr[k + q]), __uint_as_float(sr[k + 8 + q]));

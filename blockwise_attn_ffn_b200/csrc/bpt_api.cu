@@ -33,6 +33,7 @@
 #include "bpt.h"
 #include "attn_bwd_tc.cuh"
 #include "attn_pair_tc.cuh"
+#include "attn_b64_tc.cuh"
 #include "backward.cuh"
 #include "common.cuh"
 #include "gemm_tc.cuh"
@@ -51,7 +52,8 @@ static_assert(BPT_TAIL_MAX_PAIRS == bpt::kTailMaxPairs, "tail pairs");
 // Per-call options (bpt_options), validated, defaults filled in.
 struct Opts {
   int fused = 1;             // bf16 forward: fused tail (1) or waves (0)
-  int qpc = 2;               // query blocks per attention CTA
+  int qpc = 2;               // 128-row query blocks per attention CTA (b / 128)
+  int b64 = 0;               // b = 64: one 64-row query block per CTA
   int64_t max_wave = kMaxWave;
   int fault = 0;             // test hook
 };
@@ -62,12 +64,15 @@ bpt_status read_opts(const bpt_options* o, Opts* r) {
   if (o->reserved != 0) return BPT_ERR_INVALID_ARG;
   if (o->schedule != BPT_SCHEDULE_FUSED && o->schedule != BPT_SCHEDULE_WAVES)
     return BPT_ERR_INVALID_ARG;
-  if (o->attn_qpc != 0 && o->attn_qpc != 1 && o->attn_qpc != 2 && o->attn_qpc != 4)
+  if (o->attn_block != 0 && o->attn_block != 64 && o->attn_block != 128 &&
+      o->attn_block != 256 && o->attn_block != 512)
     return BPT_ERR_INVALID_ARG;
   if (o->max_wave < 0 || o->max_wave > kMaxWave) return BPT_ERR_INVALID_ARG;
   if (o->fault < 0 || o->fault > 3) return BPT_ERR_INVALID_ARG;
   r->fused = o->schedule == BPT_SCHEDULE_FUSED ? 1 : 0;
-  r->qpc = o->attn_qpc == 0 ? 2 : o->attn_qpc;
+  const int b = o->attn_block == 0 ? 256 : o->attn_block;
+  r->b64 = b == 64 ? 1 : 0;
+  r->qpc = b == 64 ? 1 : b / 128;
   r->max_wave = o->max_wave == 0 ? kMaxWave : o->max_wave;
   r->fault = o->fault;
   return BPT_OK;
@@ -242,12 +247,8 @@ bpt_status device_info(int* sms, int* pair_clusters = nullptr) {
     di.ok = (major == 10 && minor == 0);
     di.sms = n;
     if (di.ok) {
-      if (cudaFuncSetAttribute(bpt::attn_pair_tc_kernel<64, kEmu64>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               bpt::AttnPairCfg<64, kEmu64>::SMEM) != cudaSuccess ||
-          cudaFuncSetAttribute(bpt::attn_pair_tc_kernel<128, kEmu128>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               bpt::AttnPairCfg<128, kEmu128>::SMEM) != cudaSuccess ||
+      if (set_smem(bpt::attn_pair_tc_kernel<64, kEmu64>, bpt::AttnPairCfg<64, kEmu64>::SMEM) ||
+          set_smem(bpt::attn_pair_tc_kernel<128, kEmu128>, bpt::AttnPairCfg<128, kEmu128>::SMEM) ||
           set_smem(bpt::attn_pair_tc_kernel<64, kEmu64, true>, bpt::AttnPairCfg<64, kEmu64>::SMEM) ||
           set_smem(bpt::attn_pair_tc_kernel<64, kEmu64, false, false, true>,
                    bpt::AttnPairCfg<64, kEmu64>::SMEM) ||
@@ -269,6 +270,8 @@ bpt_status device_info(int* sms, int* pair_clusters = nullptr) {
           set_smem(bpt::attn_bwd_dq_tc_kernel<64>, bpt::AttnBwdCfg<64>::Q_SMEM) ||
           set_smem(bpt::attn_bwd_dkv_tc_kernel<64>, bpt::AttnBwdCfg<64>::KV_SMEM) ||
           set_smem(bpt::tail_pair_kernel, bpt::kPairSmem) ||
+          set_smem(bpt::attn_b64_tc_kernel<128, kEmu128>, bpt::AttnB64Cfg<128>::SMEM) ||
+          set_smem(bpt::attn_b64_tc_kernel<64, kEmu64>, bpt::AttnB64Cfg<64>::SMEM) ||
           cudaFuncSetAttribute(bpt::attn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (3 * 64 * 128 + 64 * 65) * 4) != cudaSuccess)
         return BPT_ERR_CUDA;
@@ -367,6 +370,15 @@ bool map_qkv_half(CUtensorMap* m, const void* base, int64_t B, int64_t N, int64_
   const uint64_t dims[4] = {64, uint64_t(N), uint64_t(3 * d / 64), uint64_t(B)};
   const uint64_t st[3] = {uint64_t(3 * d) * 2, 128, uint64_t(N) * uint64_t(3 * d) * 2};
   const uint32_t box[4] = {64, 64, 1, 1};
+  return encode_f16(m, base, 4, dims, st, box);
+}
+
+// QKV viewed as map_qkv, 64-token boxes of one head's d_k / 64 chunks: the
+// Q tile of a b = 64 attention CTA.
+bool map_q64(CUtensorMap* m, const void* base, int64_t B, int64_t N, int64_t d, int64_t dk) {
+  const uint64_t dims[4] = {64, uint64_t(N), uint64_t(3 * d / 64), uint64_t(B)};
+  const uint64_t st[3] = {uint64_t(3 * d) * 2, 128, uint64_t(N) * uint64_t(3 * d) * 2};
+  const uint32_t box[4] = {64, 64, uint32_t(dk / 64), 1};
   return encode_f16(m, base, 4, dims, st, box);
 }
 
@@ -529,6 +541,19 @@ cudaError_t launch_attn(const Plan& P, const Wave& wv_, const CUtensorMap& mQKV,
     }
   ap.fault = fault;
   ap.qpc = P.opt.qpc;
+  if (P.opt.b64) {
+    // b = 64: one CTA per 64-row query block and head, two CTAs per SM
+    if (gate != nullptr || shard != nullptr || xp_map == nullptr) return cudaErrorInvalidValue;
+    const int64_t units64 = 2 * (wv_.seqs == 0 ? wv_.count : wv_.seqs * P.nb);
+    const unsigned grid64 = unsigned(units64 * P.h);
+    if (P.dk == 128)
+      bpt::attn_b64_tc_kernel<128, kEmu128>
+          <<<grid64, 256, bpt::AttnB64Cfg<128>::SMEM, s>>>(*xp_map, mQKV, ap);
+    else
+      bpt::attn_b64_tc_kernel<64, kEmu64>
+          <<<grid64, 256, bpt::AttnB64Cfg<64>::SMEM, s>>>(*xp_map, mQKV, ap);
+    return cudaGetLastError();
+  }
   const int64_t units = wv_.seqs == 0 ? (wv_.count + ap.qpc - 1) / ap.qpc
                                       : wv_.seqs * ((P.nb + ap.qpc - 1) / ap.qpc);
   const unsigned grid = unsigned(units * P.h);
@@ -644,6 +669,7 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
   if (shard != nullptr && shard->phase == 2)
     ok = ok && map_kv_shards(&mKV, shard->kv_all, shard->G, P.B, P.N, d, P.dk);
   if (P.opt.qpc == 4) ok = ok && map_qkv_half(&mQKVh, qkv, P.B, P.N, d);
+  if (P.opt.b64) ok = ok && map_q64(&mQKVh, qkv, P.B, P.N, d, P.dk);
   if (!ok) return BPT_ERR_CUDA;
 
   RowMap ident{0, 1, 1, 1, 1};
@@ -1155,6 +1181,7 @@ bpt_status backward_bf16(const Plan& P, const BwdLayout& L, const void* x, const
             map_a(&mDO, do16, R, d, 0, int(P.dk / 64));
   CUtensorMap mQKVh;
   if (P.opt.qpc == 4) ok = ok && map_qkv_half(&mQKVh, qkv, P.B, P.N, d);
+  if (P.opt.b64) ok = ok && map_q64(&mQKVh, qkv, P.B, P.N, d, P.dk);
   const hf* wqkv[3] = {wq, wk, wv};
   for (int i = 0; i < 3 && ok; ++i)
     ok = map_b(&mDqB[i], dqkv16 + i * d, M, d, 2, 3 * d) &&
@@ -1345,7 +1372,8 @@ bpt_status layer_forward_impl(const void* x, const void* ln1, const void* W_Q, c
   st = read_opts(opts, &opt);
   if (st != BPT_OK) return st;
   if (gate != nullptr && dtype != BPT_BF16) return BPT_ERR_UNSUPPORTED;
-  if (gate != nullptr && opt.qpc == 4) return BPT_ERR_UNSUPPORTED;  // the b = 512 pair is dense
+  // the b = 512 cluster and the b = 64 kernel are dense
+  if (gate != nullptr && (opt.qpc == 4 || opt.b64)) return BPT_ERR_UNSUPPORTED;
   if (B == 0 || N == 0) return BPT_OK;
   const void* ptrs[] = {x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, out, workspace};
   for (const void* p : ptrs)

@@ -68,7 +68,7 @@ def layer_forward(x: torch.Tensor, p: Dict[str, torch.Tensor], h: int, causal: b
 
     x: [B, N, d] bf16 or fp32 on the GPU; p: ``PARAM_NAMES`` tensors of the
     same dtype (ln1/ln2 as [2, d]); out: [B, N, d] fp32; opts: None, an
-    ``Options`` or a dict of its fields (schedule, attn_qpc, max_wave, fault).
+    ``Options`` or a dict of its fields (schedule, attn_block, max_wave, fault).
     """
     if x.dim() != 3:
         raise ValueError("x must be [B, N, d]")

@@ -98,16 +98,19 @@ enum {
  *   schedule  BPT_SCHEDULE_FUSED or BPT_SCHEDULE_WAVES (bitwise: both run
  *             the same per-element arithmetic).  BPT_F32 layers always use
  *             waves.  The backward pass always uses waves.
- *   attn_qpc  query rows sharing each K/V tile, in 128-row blocks: 0 =
- *             default (2), 1, 2 or 4 (bitwise).  2 pairs two query blocks in
- *             one CTA, so each K/V tile brought in serves 256 query rows
- *             ("Blockwise Parallel Transformer — BPT", section "Choosing the
- *             block size: arithmetic intensity": FLOPs per byte re-read equal
- *             the rows sharing it); 1 gives every query block its own CTA; 4
- *             runs clusters of two such CTAs that each load half of every K/V
- *             tile and copy it to the other over distributed shared memory
- *             (512 rows per tile fetched; dense attention only: the gated
- *             entry points return BPT_ERR_UNSUPPORTED with 4).
+ *   attn_block  b, the query rows sharing each K/V tile: 0 = default
+ *             (256), 64, 128, 256 or 512 (bitwise: the softmax arithmetic of a
+ *             query row does not depend on b).  Each K/V tile brought into
+ *             shared memory serves b query rows ("Blockwise Parallel
+ *             Transformer — BPT", section "Choosing the block size:
+ *             arithmetic intensity": FLOPs per byte re-read equal the rows
+ *             sharing it).  256 pairs two 128-row query blocks in one CTA;
+ *             128 gives every query block its own CTA; 64 runs one 64-row
+ *             block per CTA, two CTAs per SM; 512 runs clusters of two
+ *             256-row CTAs that each load half of every K/V tile and copy it
+ *             to the other over distributed shared memory.  64 and 512 are
+ *             dense attention only: the gated entry points return
+ *             BPT_ERR_UNSUPPORTED with them.
  *   max_wave  waves schedule only: query blocks per wave, 0 = default
  *             (BPT_WAVE_BLOCKS), else 1..BPT_WAVE_BLOCKS; small values make
  *             small layers run the multi-wave paths (a sequence split over
@@ -127,7 +130,7 @@ enum {
  */
 typedef struct {
   int32_t schedule;
-  int32_t attn_qpc;
+  int32_t attn_block;
   int64_t max_wave;
   int32_t fault;
   int32_t reserved;
@@ -352,7 +355,7 @@ bpt_status bpt_layer_backward(const void* x, const void* ln1, const void* W_Q, c
                               float* dW_O, float* d_ln2, float* dW_1, float* db_1, float* dW_2,
                               float* db_2, void* workspace, size_t workspace_bytes,
                               bpt_stream_t stream);
-/* bpt_layer_backward with per-call options (attn_qpc and max_wave apply; the
+/* bpt_layer_backward with per-call options (attn_block and max_wave apply; the
  * backward always runs the waves schedule; fault must be 0). */
 bpt_status bpt_layer_backward_opt(const void* x, const void* ln1, const void* W_Q,
                                   const void* W_K, const void* W_V, const void* W_O,

@@ -116,7 +116,7 @@ def test_options_validation():
     assert ok(*args, None)[0] == bpt.BPT_OK
     assert ok(*args, None) == bpt.bpt_layer_workspace_size(*args)
     assert ok(*args, {})[1] == ok(*args, None)[1]            # zeroed struct = defaults
-    for bad in ({"schedule": 2}, {"schedule": -1}, {"attn_qpc": 3}, {"max_wave": -1},
+    for bad in ({"schedule": 2}, {"schedule": -1}, {"attn_block": 3}, {"max_wave": -1},
                 {"max_wave": bpt.BPT_WAVE_BLOCKS + 1}, {"fault": 4}, {"reserved": 1}):
         assert ok(*args, bad)[0] == bpt.BPT_ERR_INVALID_ARG, bad
     # the wave size only shapes the waves schedule's scratch

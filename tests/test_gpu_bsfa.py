@@ -119,7 +119,7 @@ def test_gate_is_independent_of_pairing_and_waves():
     rng = np.random.default_rng(7)
     T = gap_thresholds(oracle.layer_block_max(inp, cfg.h, cfg.causal), cfg.causal, rng)
     base, _, kp0 = run_bsfa(cfg, dev, T)
-    one, _, kp1 = run_bsfa(cfg, dev, T, opts={"attn_qpc": 1})
+    one, _, kp1 = run_bsfa(cfg, dev, T, opts={"attn_block": 128})
     waves, _, kp2 = run_bsfa(cfg, dev, T, opts={"schedule": "waves", "max_wave": 3})
     np.testing.assert_array_equal(one, base)
     np.testing.assert_array_equal(kp1, kp0)

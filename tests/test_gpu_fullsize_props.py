@@ -51,7 +51,7 @@ def test_pairing_is_bitwise_neutral_at_full_size(dev):
     x = dev["x"]
     out2, ws = bpt.layer_forward(x, dev, CFG.h, CFG.causal)
     out2 = out2.clone()
-    out1, _ = bpt.layer_forward(x, dev, CFG.h, CFG.causal, workspace=ws, opts={"attn_qpc": 1})
+    out1, _ = bpt.layer_forward(x, dev, CFG.h, CFG.causal, workspace=ws, opts={"attn_block": 128})
     assert torch.equal(out1, out2)
 
 

@@ -1,6 +1,7 @@
-"""Query rows sharing each K/V tile: one 128-row block per CTA (b = 128), two
-blocks per CTA (b = 256, the default) and a cluster of two such CTAs that
-exchange K/V halves over DSMEM (b = 512) (bpt_options.attn_qpc = 1, 2, 4).
+"""Query rows sharing each K/V tile (bpt_options.attn_block = b): one 64-row
+block per CTA, two CTAs per SM (b = 64), one 128-row block per CTA
+(b = 128), two blocks per CTA (b = 256, the default) and a cluster of two
+such CTAs that exchange K/V halves over DSMEM (b = 512).
 
 "Blockwise Parallel Transformer — BPT", section "Choosing the block size:
 arithmetic intensity": the work done per byte re-read grows with the rows
@@ -26,6 +27,8 @@ CASES = [
     (small("qpc_dk64_noncausal_ragged", 2, 300, 256, 4, 512, False, seed=42), 0),
     (small("qpc_dk128_split_sequence", 1, 900, 256, 2, 512, True, seed=43), 3),
     (small("qpc_dk64_whole_sequences", 3, 256, 256, 4, 512, True, seed=44), 2),
+    (small("qpc_dk64_causal_ragged_half", 2, 700, 256, 4, 512, True, seed=45), 0),
+    (small("qpc_dk128_noncausal_short", 2, 60, 256, 2, 512, False, seed=46), 0),
 ]
 
 
@@ -39,48 +42,47 @@ def forward_train(cfg, dev, opts):
 @pytest.mark.parametrize("schedule", ["fused", "waves"])
 @pytest.mark.parametrize("cfg,wave", CASES, ids=lambda c: getattr(c, "name", str(c)))
 def test_block_sharing_is_bitwise_neutral(cfg, wave, schedule):
-    """One 128-row block per CTA (b = 128), two (b = 256, default) and a
-    cluster of two CTAs sharing each K/V tile over DSMEM (b = 512): the same
-    layer output and statistics, bit for bit."""
+    """b = 64, 128, 256 (default) and 512: the same layer output and softmax
+    statistics, bit for bit."""
     dev = bpt.to_device(make_inputs(cfg), cfg.dtype)
     base = {"schedule": schedule, "max_wave": wave if schedule == "waves" else 0}
-    out2, st2 = forward_train(cfg, dev, dict(base, attn_qpc=2))
-    out1, st1 = forward_train(cfg, dev, dict(base, attn_qpc=1))
-    out4, st4 = forward_train(cfg, dev, dict(base, attn_qpc=4))
-    assert np.all(np.isfinite(out2))
-    np.testing.assert_array_equal(out1, out2)
-    np.testing.assert_array_equal(st1, st2)
-    np.testing.assert_array_equal(out4, out2)
-    np.testing.assert_array_equal(st4, st2)
+    out_ref, st_ref = forward_train(cfg, dev, dict(base, attn_block=256))
+    assert np.all(np.isfinite(out_ref))
+    for b in (64, 128, 512):
+        out, st = forward_train(cfg, dev, dict(base, attn_block=b))
+        np.testing.assert_array_equal(out, out_ref, err_msg=f"b = {b}")
+        np.testing.assert_array_equal(st, st_ref, err_msg=f"b = {b}")
 
 
-def test_b512_backward_recomputation_matches():
-    """The backward's forward recomputation through the b = 512 attention
-    gives the same gradients as through the default one."""
+@pytest.mark.parametrize("b", [64, 512])
+def test_backward_recomputation_matches(b):
+    """The backward's forward recomputation through the b = 64 and b = 512
+    attention kernels gives the same gradients as through the default one."""
     cfg = CASES[0][0]
     inp = make_inputs(cfg)
     dev = bpt.to_device(inp, cfg.dtype)
     _, stats, _ = bpt.layer_forward_train(dev["x"], dev, cfg.h, cfg.causal)
     dZ = torch.from_numpy(np.random.default_rng(3).standard_normal(
         (cfg.B, cfg.N, cfg.d)).astype(np.float32)).cuda()
-    g2, _ = bpt.layer_backward(dev["x"], dev, cfg.h, cfg.causal, stats, dZ)
-    g4, _ = bpt.layer_backward(dev["x"], dev, cfg.h, cfg.causal, stats, dZ,
-                               opts={"attn_qpc": 4})
-    for k in g2:
-        assert torch.equal(g2[k], g4[k]), k
+    g_ref, _ = bpt.layer_backward(dev["x"], dev, cfg.h, cfg.causal, stats, dZ)
+    g, _ = bpt.layer_backward(dev["x"], dev, cfg.h, cfg.causal, stats, dZ,
+                              opts={"attn_block": b})
+    for k in g_ref:
+        assert torch.equal(g_ref[k], g[k]), k
 
 
-def test_b512_rejects_gating():
+@pytest.mark.parametrize("b", [64, 512])
+def test_dense_only_block_sizes_reject_gating(b):
     cfg = CASES[0][0]
     dev = bpt.to_device(make_inputs(cfg), cfg.dtype)
     nb = (cfg.N + 127) // 128
     T = torch.full((cfg.h, nb), float("-inf"), dtype=torch.float32, device="cuda")
     with pytest.raises(bpt.BptError):
-        bpt.layer_forward_bsfa(dev["x"], dev, cfg.h, cfg.causal, T, opts={"attn_qpc": 4})
+        bpt.layer_forward_bsfa(dev["x"], dev, cfg.h, cfg.causal, T, opts={"attn_block": b})
 
 
-def test_qpc_rejects_other_values():
-    for bad in (3, 5, -1):
+def test_attn_block_rejects_other_values():
+    for bad in (1, 2, 4, 32, 192, 1024, -1):
         st, _ = bpt.bpt_layer_workspace_size_opt(1, 256, 256, 2, 512, True, bpt.BPT_BF16,
-                                                 {"attn_qpc": bad})
+                                                 {"attn_block": bad})
         assert st == bpt.BPT_ERR_INVALID_ARG
