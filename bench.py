@@ -200,21 +200,49 @@ def measure_backward(bpt, cfg, x, p, stream, dev, args, flops, world, peaks, dis
         bpt.layer_forward_train(x, p, cfg.h, cfg.causal, out=out, stats=stats, workspace=ws)
         bpt.layer_backward(x, p, cfg.h, cfg.causal, stats, dZ, workspace=bws)
     e2.record(stream)
+    # the same with the attention output kept by the forward (no attention
+    # recomputation in the backward; +2 B N d bytes of fp16 activation)
+    o = torch.empty(x.shape, dtype=torch.float16, device=dev)
+    bpt.layer_forward_train(x, p, cfg.h, cfg.causal, out=out, stats=stats, workspace=ws,
+                            keep_o=o)
+    bpt.layer_backward(x, p, cfg.h, cfg.causal, stats, dZ, workspace=bws, o=o)
+    e3, e4 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
+    if world > 1:
+        dist.barrier()
+    e2b = torch.cuda.Event(enable_timing=True)
+    e2b.record(stream)
+    for _ in range(k):
+        bpt.layer_backward(x, p, cfg.h, cfg.causal, stats, dZ, workspace=bws, o=o)
+    e3.record(stream)
+    for _ in range(k):
+        bpt.layer_forward_train(x, p, cfg.h, cfg.causal, out=out, stats=stats, workspace=ws,
+                                keep_o=o)
+        bpt.layer_backward(x, p, cfg.h, cfg.causal, stats, dZ, workspace=bws, o=o)
+    e4.record(stream)
     torch.cuda.synchronize(dev)
     st, site = bpt.bpt_read_device_error(bws.data_ptr(), stream.cuda_stream)
     if st != bpt.BPT_OK:
         raise SystemExit(f"device error in backward {bpt.status_string(st)} site {site}")
     bwd_ms = bdist.max_over_ranks(e0.elapsed_time(e1), dist, dev) / k
     step_ms = bdist.max_over_ranks(e1.elapsed_time(e2), dist, dev) / k
+    bwd_o_ms = bdist.max_over_ranks(e2b.elapsed_time(e3), dist, dev) / k
+    step_o_ms = bdist.max_over_ranks(e3.elapsed_time(e4), dist, dev) / k
     grad_tf = 2 * flops["total"] * world / (bwd_ms / 1e3) / 1e12
     tokens = cfg.B * cfg.N * world
     return {"ms_per_step": bwd_ms, "tokens_per_s": tokens / (bwd_ms / 1e3),
             "grad_tflops": grad_tf, "pct_bf16_peak": grad_tf / world / peaks["bf16_tflops"],
             "train_step_ms": step_ms, "train_step_tokens_per_s": tokens / (step_ms / 1e3),
             "train_step_tflops": 3 * flops["total"] * world / (step_ms / 1e3) / 1e12,
+            "keep_o": {"ms_per_step": bwd_o_ms,
+                       "grad_tflops": 2 * flops["total"] * world / (bwd_o_ms / 1e3) / 1e12,
+                       "train_step_ms": step_o_ms,
+                       "train_step_tokens_per_s": tokens / (step_o_ms / 1e3),
+                       "kept_bytes": int(o.numel() * 2)},
             "steps": k, "workspace_bytes": int(bws.numel()),
             "note": "grad FLOPs = 2 x forward algorithmic FLOPs; train step = forward_train + "
-                    "backward (3 x forward FLOPs counted; recomputation not counted)"}
+                    "backward (3 x forward FLOPs counted; recomputation not counted); keep_o: "
+                    "the forward keeps the attention output and the backward reads it instead "
+                    "of recomputing the attention"}
 
 
 # ---------------------------------------------- gated attention (BSFA) --

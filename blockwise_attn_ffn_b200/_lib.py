@@ -34,6 +34,7 @@ EXPORTED = [
     "bpt_layer_backward_workspace_size_opt", "bpt_layer_backward_opt",
     "bpt_layer_launch_count_opt",
     "bpt_layer_shard_workspace_size", "bpt_layer_shard_project", "bpt_layer_shard_forward",
+    "bpt_layer_forward_train_keep_o", "bpt_layer_backward_keep_o",
 ]
 
 
@@ -115,6 +116,13 @@ def load() -> ctypes.CDLL:
     lib.bpt_layer_backward_opt.argtypes = ([vp] * 13 + [i64] * 5 + [i32, i32] + [vp] * 12 +
                                            [ctypes.c_size_t, op, vp])
     lib.bpt_layer_backward_opt.restype = i32
+    lib.bpt_layer_forward_train_keep_o.argtypes = ([vp] * 11 + [i64] * 5 +
+                                                   [i32, i32, vp, vp, vp, vp, ctypes.c_size_t,
+                                                    op, vp])
+    lib.bpt_layer_forward_train_keep_o.restype = i32
+    lib.bpt_layer_backward_keep_o.argtypes = ([vp] * 14 + [i64] * 5 + [i32, i32] + [vp] * 12 +
+                                              [ctypes.c_size_t, op, vp])
+    lib.bpt_layer_backward_keep_o.restype = i32
     lib.bpt_layer_launch_count_opt.argtypes = [i64, i64, i64, i64, i64, i32, i32, op,
                                                ctypes.POINTER(ctypes.c_int64)]
     lib.bpt_layer_launch_count_opt.restype = i32
@@ -198,6 +206,26 @@ def bpt_layer_backward_opt(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, 
                                          dx, d_ln1, dW_Q, dW_K, dW_V, dW_O, d_ln2, dW_1, db_1,
                                          dW_2, db_2, workspace, workspace_bytes,
                                          _opts_ref(opts), stream)
+
+
+def bpt_layer_forward_train_keep_o(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
+                                   B, N, d, h, d_ff, causal, dtype, out, stats, o, workspace,
+                                   workspace_bytes, opts, stream) -> int:
+    return load().bpt_layer_forward_train_keep_o(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2,
+                                                 b_2, B, N, d, h, d_ff, int(bool(causal)),
+                                                 dtype, out, stats, o, workspace,
+                                                 workspace_bytes, _opts_ref(opts), stream)
+
+
+def bpt_layer_backward_keep_o(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, stats, o,
+                              dZ, B, N, d, h, d_ff, causal, dtype, dx, d_ln1, dW_Q, dW_K, dW_V,
+                              dW_O, d_ln2, dW_1, db_1, dW_2, db_2, workspace, workspace_bytes,
+                              opts, stream) -> int:
+    return load().bpt_layer_backward_keep_o(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2,
+                                            stats, o, dZ, B, N, d, h, d_ff, int(bool(causal)),
+                                            dtype, dx, d_ln1, dW_Q, dW_K, dW_V, dW_O, d_ln2,
+                                            dW_1, db_1, dW_2, db_2, workspace, workspace_bytes,
+                                            _opts_ref(opts), stream)
 
 
 def bpt_layer_shard_workspace_size(B, N, G, d, h, d_ff, causal, dtype) -> Tuple[int, int]:

@@ -24,6 +24,31 @@ __device__ __forceinline__ float ld_as_float(const float* p) { return *p; }
 __device__ __forceinline__ float ld_as_float(const __half* p) { return __half2float(*p); }
 __device__ __forceinline__ float ld_as_float(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
+// Row copies of fp16 [., d] tensors between wave block rows and token rows
+// (d % 8 == 0; row strides in elements, multiples of 8):
+//   scatter = 0: out[r, :] = in[map(r), :], zeros where map(r) < 0;
+//   scatter = 1: out[map(r), :] = in[r, :] where map(r) >= 0.
+__global__ void rows_copy_f16_kernel(const __half* __restrict__ in, long long ld_in,
+                                     __half* __restrict__ out, long long ld_out, long long rows,
+                                     int d, RowMap map, int scatter) {
+  const long long per_row = d / 8;
+  const long long total = rows * per_row;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long r = i / per_row;
+    const int c = static_cast<int>(i - r * per_row) * 8;
+    const long long g = map.map(r);
+    if (scatter) {
+      if (g >= 0)
+        *reinterpret_cast<uint4*>(out + g * ld_out + c) =
+            *reinterpret_cast<const uint4*>(in + r * ld_in + c);
+    } else {
+      *reinterpret_cast<uint4*>(out + r * ld_out + c) =
+          g >= 0 ? *reinterpret_cast<const uint4*>(in + g * ld_in + c) : make_uint4(0, 0, 0, 0);
+    }
+  }
+}
+
 // out[r, :] = fp16(in[map(r), :]) for r < rows; d % 8 == 0.
 __global__ void rows_f32_to_f16_kernel(const float* __restrict__ in, __half* __restrict__ out,
                                        long long rows, int d, RowMap map) {

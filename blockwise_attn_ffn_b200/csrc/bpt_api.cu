@@ -515,13 +515,14 @@ struct AttnShard {
 cudaError_t launch_attn(const Plan& P, const Wave& wv_, const CUtensorMap& mQKV, __half* so,
                         float* stats, uint32_t* err, int fault, cudaStream_t s,
                         const AttnGate* gate = nullptr, bool o_tok = false,
-                        const AttnShard* shard = nullptr, const CUtensorMap* xp_map = nullptr) {
+                        const AttnShard* shard = nullptr, const CUtensorMap* xp_map = nullptr,
+                        int64_t o_ld = 0) {
   bpt::AttnPairParams ap{};
   ap.N = int(P.N); ap.nb = int(P.nb); ap.h = int(P.h); ap.d = int(P.d);
   ap.causal = P.causal; ap.item0 = int(wv_.item0); ap.count = int(wv_.count);
   ap.seqs = int(wv_.seqs); ap.o = so; ap.err = err;
   ap.o_tok = o_tok ? 1 : 0;
-  ap.o_ld = o_tok ? 3 * P.d : P.d;
+  ap.o_ld = o_ld != 0 ? o_ld : (o_tok ? 3 * P.d : P.d);
   ap.scale_log2 = float(1.4426950408889634 / std::sqrt(double(P.dk)));
   ap.stats = reinterpret_cast<float2*>(stats);
   if (shard) {
@@ -623,7 +624,8 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
                         const void* W_K, const void* W_V, const void* W_O, const void* ln2,
                         const void* W_1, const void* b_1, const void* W_2, const void* b_2,
                         float* out, float* stats, uint8_t* ws, cudaStream_t s, int sms,
-                        const AttnGate* gate, const ShardSpec* shard = nullptr) {
+                        const AttnGate* gate, const ShardSpec* shard = nullptr,
+                        __half* o_keep = nullptr) {
   using bf = __nv_bfloat16;
   using hf = __half;
   const int64_t M = P.B * P.N, d = P.d, d_ff = P.d_ff;
@@ -657,7 +659,8 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
     // tail A operands: o = the Q columns of QKV (token rows, row stride 3d),
     // and the per-pair scratch rows of LN2(y) and the hidden
     const int64_t trows = P.tail_pairs * 256;
-    ok = ok && map_a(&mO, qkv, M, d, 3 * d) &&
+    // (o_keep: the attention writes o there instead, [B*N, d])
+    ok = ok && (o_keep != nullptr ? map_a(&mO, o_keep, M, d) : map_a(&mO, qkv, M, d, 3 * d)) &&
          map_a(&mV, ws + P.off_tv, trows, d) && map_a(&mH, ws + P.off_th, trows, d_ff) &&
          // 512-column W_2 tiles: H in 64-deep single-chunk boxes, W_2 as
          // 64 K rows x four 64-column chunks
@@ -731,8 +734,9 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
     }
     {
       LaunchScope ls(BPT_KIND_ATTN, s);
-      if (launch_attn(P, all, mQKV, qkv, stats, err, fault == 2 ? 2 : 0, s, gate, true,
-                      shard != nullptr ? &as : nullptr, &mQKVh) != cudaSuccess)
+      if (launch_attn(P, all, mQKV, o_keep != nullptr ? o_keep : qkv, stats, err,
+                      fault == 2 ? 2 : 0, s, gate, true, shard != nullptr ? &as : nullptr, &mQKVh,
+                      o_keep != nullptr ? d : 0) != cudaSuccess)
         return BPT_ERR_CUDA;
     }
     int dummy = 0, pairs_max = 0;
@@ -770,6 +774,12 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
                       false, nullptr, &mQKVh) !=
           cudaSuccess)
         return BPT_ERR_CUDA;
+      if (o_keep != nullptr) {  // the wave's o rows to their token rows
+        bpt::rows_copy_f16_kernel<<<unsigned(std::min<int64_t>((rows * d / 8 + 255) / 256,
+                                                               int64_t(sms) * 16)),
+                                    256, 0, s>>>(so, d, o_keep, d, rows, int(d), map, 1);
+        if (cudaGetLastError() != cudaSuccess) return BPT_ERR_CUDA;
+      }
     }
     {
       bpt::GemmParams g{};
@@ -1126,7 +1136,7 @@ bpt_status backward_bf16(const Plan& P, const BwdLayout& L, const void* x, const
                          const float* stats, const float* dZ, float* dx, float* d_ln1,
                          float* dW_Q, float* dW_K, float* dW_V, float* dW_O, float* d_ln2,
                          float* dW_1, float* db_1, float* dW_2, float* db_2, uint8_t* ws,
-                         cudaStream_t s, int sms) {
+                         cudaStream_t s, int sms, const __half* o_keep) {
   using bf = __nv_bfloat16;
   using hf = __half;
   const int64_t M = P.B * P.N, d = P.d, d_ff = P.d_ff, h = P.h;
@@ -1238,10 +1248,16 @@ bpt_status backward_bf16(const Plan& P, const BwdLayout& L, const void* x, const
     const Wave wv_ = P.wave(w);
     const int64_t rows = wv_.count * P.blk;
     RowMap map{int(wv_.item0), int(P.nb), int(P.N), int(P.blk), 0};
-    // forward recomputation of this wave: o, y, LN2(y), FFN pre-activation and hidden
-    if (launch_attn(P, wv_, mQKV, so, nullptr, err, 0, s, nullptr, false, nullptr, &mQKVh) !=
-        cudaSuccess)
+    // forward recomputation of this wave: o (or the forward's, kept), y, LN2(y),
+    // FFN pre-activation and hidden
+    if (o_keep != nullptr) {
+      bpt::rows_copy_f16_kernel<<<unsigned(std::min<int64_t>((rows * d / 8 + 255) / 256,
+                                                             int64_t(sms) * 16)),
+                                  256, 0, s>>>(o_keep, d, so, d, rows, int(d), map, 0);
+    } else if (launch_attn(P, wv_, mQKV, so, nullptr, err, 0, s, nullptr, false, nullptr,
+                           &mQKVh) != cudaSuccess) {
       return BPT_ERR_CUDA;
+    }
     if (!gemm(mO, mWo, rows, d, d, bpt::kEpiResidX, bpt::kLayAkBn, map, [&](bpt::GemmParams& g) {
           g.out_f32 = y; g.ld_f32 = d; g.resid = static_cast<const bf*>(x); g.ld_resid = d;
         }))
@@ -1365,13 +1381,15 @@ bpt_status layer_forward_impl(const void* x, const void* ln1, const void* W_Q, c
                               int64_t N, int64_t d, int64_t h, int64_t d_ff, int causal,
                               bpt_dtype dtype, float* out, float* stats, void* workspace,
                               size_t workspace_bytes, const bpt_options* opts,
-                              bpt_stream_t stream, const AttnGate* gate = nullptr) {
+                              bpt_stream_t stream, const AttnGate* gate = nullptr,
+                              void* o_keep = nullptr) {
   bpt_status st = check_shape(B, N, d, h, d_ff, causal, dtype);
   if (st != BPT_OK) return st;
   Opts opt;
   st = read_opts(opts, &opt);
   if (st != BPT_OK) return st;
   if (gate != nullptr && dtype != BPT_BF16) return BPT_ERR_UNSUPPORTED;
+  if (o_keep != nullptr && dtype != BPT_BF16) return BPT_ERR_UNSUPPORTED;
   // the b = 512 cluster and the b = 64 kernel are dense
   if (gate != nullptr && (opt.qpc == 4 || opt.b64)) return BPT_ERR_UNSUPPORTED;
   if (B == 0 || N == 0) return BPT_OK;
@@ -1394,6 +1412,14 @@ bpt_status layer_forward_impl(const void* x, const void* ln1, const void* W_Q, c
     for (const Span& in : ins)
       if (ss.overlaps(in)) return BPT_ERR_INVALID_ARG;
   }
+  if (o_keep != nullptr) {
+    const Span sk(o_keep, size_t(B * N * d) * 2);
+    if (misaligned(o_keep) || sk.overlaps(so) || sk.overlaps(sw)) return BPT_ERR_INVALID_ARG;
+    if (stats != nullptr && sk.overlaps(Span(stats, size_t(B * h * N) * 2 * sizeof(float))))
+      return BPT_ERR_INVALID_ARG;
+    for (const Span& in : ins)
+      if (sk.overlaps(in)) return BPT_ERR_INVALID_ARG;
+  }
   if (opt.fault != 0 && dtype != BPT_BF16) return BPT_ERR_INVALID_ARG;
 
   int sms = 0;
@@ -1406,7 +1432,7 @@ bpt_status layer_forward_impl(const void* x, const void* ln1, const void* W_Q, c
     st = get_encoder();
     if (st != BPT_OK) return st;
     return forward_bf16(P, x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, out, stats, ws, s,
-                        sms, gate);
+                        sms, gate, nullptr, static_cast<__half*>(o_keep));
   }
   return forward_f32(P, static_cast<const float*>(x), static_cast<const float*>(ln1),
                      static_cast<const float*>(W_Q), static_cast<const float*>(W_K),
@@ -1465,10 +1491,12 @@ bpt_status backward_impl(const void* x, const void* ln1, const void* W_Q, const 
                          int64_t d_ff, int causal, bpt_dtype dtype, float* dx, float* d_ln1,
                          float* dW_Q, float* dW_K, float* dW_V, float* dW_O, float* d_ln2,
                          float* dW_1, float* db_1, float* dW_2, float* db_2, void* workspace,
-                         size_t workspace_bytes, const bpt_options* opts, bpt_stream_t stream) {
+                         size_t workspace_bytes, const bpt_options* opts, bpt_stream_t stream,
+                         const void* o_keep = nullptr) {
   (void)b_2;  // the output's bias does not enter any gradient but its own
   bpt_status st = check_shape(B, N, d, h, d_ff, causal, dtype);
   if (st != BPT_OK) return st;
+  if (o_keep != nullptr && dtype != BPT_BF16) return BPT_ERR_UNSUPPORTED;
   Opts opt;
   st = read_opts(opts, &opt);
   if (st != BPT_OK) return st;
@@ -1492,6 +1520,10 @@ bpt_status backward_impl(const void* x, const void* ln1, const void* W_Q, const 
       forward_inputs(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, B, N, d, d_ff, P.esize);
   reads.push_back(Span(stats, size_t(B * h * N) * 8));
   reads.push_back(Span(dZ, size_t(B * N * d) * 4));
+  if (o_keep != nullptr) {
+    if (misaligned(o_keep)) return BPT_ERR_INVALID_ARG;
+    reads.push_back(Span(o_keep, size_t(B * N * d) * 2));
+  }
   const Span sw(workspace, ws_need);
   for (const Span& r : reads)
     if (sw.overlaps(r)) return BPT_ERR_INVALID_ARG;
@@ -1520,7 +1552,8 @@ bpt_status backward_impl(const void* x, const void* ln1, const void* W_Q, const 
   if (st != BPT_OK) return st;
   const BwdLayout L = make_bwd_layout(P);
   return backward_bf16(P, L, x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, stats, dZ, dx, d_ln1,
-                       dW_Q, dW_K, dW_V, dW_O, d_ln2, dW_1, db_1, dW_2, db_2, ws, s, sms);
+                       dW_Q, dW_K, dW_V, dW_O, d_ln2, dW_1, db_1, dW_2, db_2, ws, s, sms,
+                       static_cast<const __half*>(o_keep));
 }
 
 // Shared body of the sequence-shard entry points (phase 1: projection into
@@ -1659,6 +1692,20 @@ bpt_status bpt_layer_forward_train(const void* x, const void* ln1, const void* W
                             stream);
 }
 
+bpt_status bpt_layer_forward_train_keep_o(const void* x, const void* ln1, const void* W_Q,
+                                          const void* W_K, const void* W_V, const void* W_O,
+                                          const void* ln2, const void* W_1, const void* b_1,
+                                          const void* W_2, const void* b_2, int64_t B,
+                                          int64_t N, int64_t d, int64_t h, int64_t d_ff,
+                                          int causal, bpt_dtype dtype, float* out, float* stats,
+                                          void* o, void* workspace, size_t workspace_bytes,
+                                          const bpt_options* opts, bpt_stream_t stream) {
+  if (stats == nullptr || o == nullptr) return BPT_ERR_INVALID_ARG;
+  return layer_forward_impl(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, B, N, d, h, d_ff,
+                            causal, dtype, out, stats, workspace, workspace_bytes, opts, stream,
+                            nullptr, o);
+}
+
 bpt_status bpt_layer_forward_bsfa(const void* x, const void* ln1, const void* W_Q,
                                   const void* W_K, const void* W_V, const void* W_O,
                                   const void* ln2, const void* W_1, const void* b_1,
@@ -1731,6 +1778,23 @@ bpt_status bpt_layer_backward_opt(const void* x, const void* ln1, const void* W_
   return backward_impl(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, stats, dZ, B, N, d, h,
                        d_ff, causal, dtype, dx, d_ln1, dW_Q, dW_K, dW_V, dW_O, d_ln2, dW_1, db_1,
                        dW_2, db_2, workspace, workspace_bytes, opts, stream);
+}
+
+bpt_status bpt_layer_backward_keep_o(const void* x, const void* ln1, const void* W_Q,
+                                     const void* W_K, const void* W_V, const void* W_O,
+                                     const void* ln2, const void* W_1, const void* b_1,
+                                     const void* W_2, const void* b_2, const float* stats,
+                                     const void* o, const float* dZ, int64_t B, int64_t N,
+                                     int64_t d, int64_t h, int64_t d_ff, int causal,
+                                     bpt_dtype dtype, float* dx, float* d_ln1, float* dW_Q,
+                                     float* dW_K, float* dW_V, float* dW_O, float* d_ln2,
+                                     float* dW_1, float* db_1, float* dW_2, float* db_2,
+                                     void* workspace, size_t workspace_bytes,
+                                     const bpt_options* opts, bpt_stream_t stream) {
+  if (o == nullptr) return BPT_ERR_INVALID_ARG;
+  return backward_impl(x, ln1, W_Q, W_K, W_V, W_O, ln2, W_1, b_1, W_2, b_2, stats, dZ, B, N, d, h,
+                       d_ff, causal, dtype, dx, d_ln1, dW_Q, dW_K, dW_V, dW_O, d_ln2, dW_1, db_1,
+                       dW_2, db_2, workspace, workspace_bytes, opts, stream, o);
 }
 
 bpt_status bpt_layer_shard_workspace_size(int64_t B, int64_t N, int64_t G, int64_t d,

@@ -102,10 +102,13 @@ def layer_forward_train(x: torch.Tensor, p: Dict[str, torch.Tensor], h: int, cau
                         out: Optional[torch.Tensor] = None,
                         stats: Optional[torch.Tensor] = None,
                         workspace: Optional[torch.Tensor] = None,
-                        stream: Optional[torch.cuda.Stream] = None, opts=None):
+                        stream: Optional[torch.cuda.Stream] = None, opts=None,
+                        keep_o: Optional[torch.Tensor] = None):
     """``layer_forward`` that also returns the per-row softmax statistics via
     ``bpt_layer_forward_train``: (out, stats, workspace), stats [B, h, N, 2]
-    fp32 holding (m, l) per (batch, head, query row)."""
+    fp32 holding (m, l) per (batch, head, query row).  With ``keep_o`` (an
+    fp16 [B, N, d] tensor, bf16 layers) the attention output is kept there
+    too (``bpt_layer_forward_train_keep_o``), for ``layer_backward(o=...)``."""
     if x.dim() != 3:
         raise ValueError("x must be [B, N, d]")
     B, N, d = x.shape
@@ -122,7 +125,16 @@ def layer_forward_train(x: torch.Tensor, p: Dict[str, torch.Tensor], h: int, cau
     if workspace is None:
         workspace = workspace_for(B, N, d, h, d_ff, causal, x.dtype, x.device, opts)
     s = stream if stream is not None else torch.cuda.current_stream(x.device)
-    if opts is None:
+    if keep_o is not None:
+        if (keep_o.dtype != torch.float16 or tuple(keep_o.shape) != (B, N, d)
+                or not keep_o.is_contiguous()):
+            raise ValueError(f"keep_o must be a contiguous fp16 [{B}, {N}, {d}] tensor")
+        st = _lib.bpt_layer_forward_train_keep_o(*[t.data_ptr() for t in tensors], B, N, d, h,
+                                                 d_ff, causal, code, out.data_ptr(),
+                                                 stats.data_ptr(), keep_o.data_ptr(),
+                                                 workspace.data_ptr(), workspace.numel(), opts,
+                                                 s.cuda_stream)
+    elif opts is None:
         st = _lib.bpt_layer_forward_train(*[t.data_ptr() for t in tensors], B, N, d, h, d_ff,
                                           causal, code, out.data_ptr(), stats.data_ptr(),
                                           workspace.data_ptr(), workspace.numel(), s.cuda_stream)
@@ -185,11 +197,14 @@ GRAD_SHAPES = ["x", "ln1", "W_Q", "W_K", "W_V", "W_O", "ln2", "W_1", "b_1", "W_2
 def layer_backward(x: torch.Tensor, p: Dict[str, torch.Tensor], h: int, causal: bool,
                    stats: torch.Tensor, dZ: torch.Tensor,
                    workspace: Optional[torch.Tensor] = None,
-                   stream: Optional[torch.cuda.Stream] = None, opts=None):
+                   stream: Optional[torch.cuda.Stream] = None, opts=None,
+                   o: Optional[torch.Tensor] = None):
     """Gradients via ``bpt_layer_backward``; returns (grads, workspace) with
     grads[name] fp32 for name in GRAD_SHAPES (ln1 / ln2 as [2, d]: d gamma;
     d beta).  x and p as for ``layer_forward`` (bf16 or fp32); stats from
-    ``layer_forward_train``; dZ [B, N, d] fp32."""
+    ``layer_forward_train``; dZ [B, N, d] fp32.  ``o``: the attention output
+    ``layer_forward_train(keep_o=...)`` kept (``bpt_layer_backward_keep_o``:
+    no attention recomputation, same gradients)."""
     if x.dim() != 3:
         raise ValueError("x must be [B, N, d]")
     B, N, d = x.shape
@@ -211,11 +226,20 @@ def layer_backward(x: torch.Tensor, p: Dict[str, torch.Tensor], h: int, causal: 
                             device=x.device) for k in GRAD_SHAPES}
     s = stream if stream is not None else torch.cuda.current_stream(x.device)
     order = ["x", "ln1", "W_Q", "W_K", "W_V", "W_O", "ln2", "W_1", "b_1", "W_2", "b_2"]
-    st = _lib.bpt_layer_backward_opt(*[t.data_ptr() for t in tensors], stats.data_ptr(),
-                                     dZ.data_ptr(), B, N, d, h, d_ff, causal, code,
-                                     *[grads[k].data_ptr() for k in order],
-                                     workspace.data_ptr(), workspace.numel(), opts,
-                                     s.cuda_stream)
+    if o is not None:
+        if o.dtype != torch.float16 or tuple(o.shape) != (B, N, d) or not o.is_contiguous():
+            raise ValueError(f"o must be a contiguous fp16 [{B}, {N}, {d}] tensor")
+        st = _lib.bpt_layer_backward_keep_o(*[t.data_ptr() for t in tensors], stats.data_ptr(),
+                                            o.data_ptr(), dZ.data_ptr(), B, N, d, h, d_ff,
+                                            causal, code, *[grads[k].data_ptr() for k in order],
+                                            workspace.data_ptr(), workspace.numel(), opts,
+                                            s.cuda_stream)
+    else:
+        st = _lib.bpt_layer_backward_opt(*[t.data_ptr() for t in tensors], stats.data_ptr(),
+                                         dZ.data_ptr(), B, N, d, h, d_ff, causal, code,
+                                         *[grads[k].data_ptr() for k in order],
+                                         workspace.data_ptr(), workspace.numel(), opts,
+                                         s.cuda_stream)
     if st != _lib.BPT_OK:
         raise _lib.BptError(st, "bpt_layer_backward")
     return grads, workspace

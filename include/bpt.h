@@ -246,6 +246,32 @@ bpt_status bpt_layer_forward_train(const void* x, const void* ln1, const void* W
                                    size_t workspace_bytes, bpt_stream_t stream);
 
 /*
+ * bpt_layer_forward_train_keep_o -- bpt_layer_forward_train that also keeps
+ * the attention output, so that bpt_layer_backward_keep_o need not recompute
+ * it.  The pages' backward ("The backward pass") recomputes each block's
+ * attention from (m, l); keeping o trades 2 B N d bytes of activation memory
+ * for that recomputation (a full causal attention forward).  BPT_BF16 only.
+ *
+ *   o   [B, N, d] fp16, device, caller-owned, 16-byte aligned; must not
+ *       overlap x, any parameter, out, stats or the workspace.  Row (b, i)
+ *       holds the attention output of token i of sequence b, heads
+ *       concatenated: softmax(q k^T / sqrt(d_k)) v per head, before W_O,
+ *       exactly the fp16 values the layer body multiplied by W_O.
+ *   opts  NULL or per-call options (as bpt_layer_forward_opt).
+ * Everything else as bpt_layer_forward_train.  Returns BPT_ERR_UNSUPPORTED
+ * for BPT_F32, BPT_ERR_INVALID_ARG for stats == NULL, o == NULL, misaligned
+ * or overlapping buffers.
+ */
+bpt_status bpt_layer_forward_train_keep_o(const void* x, const void* ln1, const void* W_Q,
+                                          const void* W_K, const void* W_V, const void* W_O,
+                                          const void* ln2, const void* W_1, const void* b_1,
+                                          const void* W_2, const void* b_2, int64_t B,
+                                          int64_t N, int64_t d, int64_t h, int64_t d_ff,
+                                          int causal, bpt_dtype dtype, float* out, float* stats,
+                                          void* o, void* workspace, size_t workspace_bytes,
+                                          const bpt_options* opts, bpt_stream_t stream);
+
+/*
  * bpt_layer_forward_bsfa -- bpt_layer_forward with block-sparse gating of the
  * attention ("Block Sparse Flash Attention", sections "Methodology and
  * Mechanism" and "Gating Mechanism and Threshold Calibration": exact scores
@@ -368,6 +394,28 @@ bpt_status bpt_layer_backward_opt(const void* x, const void* ln1, const void* W_
                                   float* dW_2, float* db_2, void* workspace,
                                   size_t workspace_bytes, const bpt_options* opts,
                                   bpt_stream_t stream);
+
+/*
+ * bpt_layer_backward_keep_o -- bpt_layer_backward with the attention output
+ * `o` that bpt_layer_forward_train_keep_o wrote for the same inputs (fp16
+ * [B, N, d], 16-byte aligned, read only; must not overlap any output or the
+ * workspace).  Each wave takes its o rows from `o` instead of recomputing
+ * the attention forward; the gradients are bitwise those of
+ * bpt_layer_backward (the recomputation reproduces o exactly).  BPT_BF16
+ * only (BPT_ERR_UNSUPPORTED otherwise); workspace size as
+ * bpt_layer_backward_workspace_size_opt with the same options.
+ */
+bpt_status bpt_layer_backward_keep_o(const void* x, const void* ln1, const void* W_Q,
+                                     const void* W_K, const void* W_V, const void* W_O,
+                                     const void* ln2, const void* W_1, const void* b_1,
+                                     const void* W_2, const void* b_2, const float* stats,
+                                     const void* o, const float* dZ, int64_t B, int64_t N,
+                                     int64_t d, int64_t h, int64_t d_ff, int causal,
+                                     bpt_dtype dtype, float* dx, float* d_ln1, float* dW_Q,
+                                     float* dW_K, float* dW_V, float* dW_O, float* d_ln2,
+                                     float* dW_1, float* db_1, float* dW_2, float* db_2,
+                                     void* workspace, size_t workspace_bytes,
+                                     const bpt_options* opts, bpt_stream_t stream);
 
 /*
  * Sequence sharding over G GPUs ("Blockwise Parallel Transformer — BPT",

@@ -296,3 +296,40 @@ def test_backward_rejects_bad_pointers_and_small_workspace():
 
 def test_backward_empty_is_a_no_op():
     assert bwd([None] * 14, [None] * 11, B=0) == bpt.BPT_OK
+
+
+# ---------------------------------------------- kept attention output (keep_o)
+def fwd_keep_o(p, o, stats, dtype=BF, ws_bytes=1 << 31, B=1, N=256, d=256, h=2, d_ff=512):
+    return bpt.bpt_layer_forward_train_keep_o(*p[:11], B, N, d, h, d_ff, 1, dtype, p[11], stats,
+                                              o, p[12], ws_bytes, None, None)
+
+
+def test_forward_keep_o_argument_checks():
+    """Checked on the host before anything is enqueued (no GPU needed)."""
+    stats, o = 0xA0000000, 0xB0000000
+    assert fwd_keep_o(GOOD, None, stats) == bpt.BPT_ERR_INVALID_ARG
+    assert fwd_keep_o(GOOD, o, None) == bpt.BPT_ERR_INVALID_ARG
+    assert fwd_keep_o(GOOD, o + 8, stats) == bpt.BPT_ERR_INVALID_ARG       # misaligned
+    assert fwd_keep_o(GOOD, GOOD[0], stats) == bpt.BPT_ERR_INVALID_ARG     # o over x
+    assert fwd_keep_o(GOOD, GOOD[11], stats) == bpt.BPT_ERR_INVALID_ARG    # o over out
+    assert fwd_keep_o(GOOD, GOOD[12] + 4096, stats) == bpt.BPT_ERR_INVALID_ARG  # in workspace
+    assert fwd_keep_o(GOOD, stats + 64, stats) == bpt.BPT_ERR_INVALID_ARG  # o over stats
+    for i in range(1, 11):
+        assert fwd_keep_o(GOOD, GOOD[i], stats) == bpt.BPT_ERR_INVALID_ARG, i
+    assert fwd_keep_o(GOOD, o, stats, dtype=F32) == bpt.BPT_ERR_UNSUPPORTED
+
+
+def bwd_keep_o(ins, o, outs, ws_bytes=1 << 31, dtype=BF, B=1, N=256, d=64, h=1, d_ff=256):
+    return bpt.bpt_layer_backward_keep_o(*ins[:12], o, ins[12], B, N, d, h, d_ff, 1, dtype,
+                                         *outs, ins[13], ws_bytes, None, None)
+
+
+def test_backward_keep_o_argument_checks():
+    o = 0xC0000000
+    assert bwd_keep_o(BWD_IN, None, BWD_OUT) == bpt.BPT_ERR_INVALID_ARG
+    assert bwd_keep_o(BWD_IN, o + 8, BWD_OUT) == bpt.BPT_ERR_INVALID_ARG   # misaligned
+    outs = list(BWD_OUT)
+    outs[0] = o                                                             # dx over o
+    assert bwd_keep_o(BWD_IN, o, outs) == bpt.BPT_ERR_INVALID_ARG
+    assert bwd_keep_o(BWD_IN, BWD_IN[13] + 4096, BWD_OUT) == bpt.BPT_ERR_INVALID_ARG  # in ws
+    assert bwd_keep_o(BWD_IN, o, BWD_OUT, dtype=F32) == bpt.BPT_ERR_UNSUPPORTED

@@ -170,3 +170,46 @@ def test_backward_full_gpt2_small_workload():
     for k, (g, b) in {"ln1": ("gamma1", "beta1"), "ln2": ("gamma2", "beta2")}.items():
         check(k + ".gamma", got[k][0], want[g])
         check(k + ".beta", got[k][1], want[b])
+
+
+KEEP_O_CASES = [
+    (CASES[0], "fused", 0),                 # two sequences, one wave
+    (CASES[2], "fused", 0),                 # ragged N (padded rows in the last block)
+    (CASES[1], "waves", 1),                 # waves forward, one block per wave
+    (small("keep_o_dk128_split", 1, 900, 256, 2, 512, True, seed=25), "waves", 3),
+]
+
+
+@pytest.mark.parametrize("cfg,schedule,wave", KEEP_O_CASES,
+                         ids=lambda c: getattr(c, "name", str(c)))
+def test_backward_with_kept_attention_output(cfg, schedule, wave):
+    """bpt_layer_forward_train_keep_o writes the attention output it fed to
+    W_O (checked against the oracle's O), with out and stats bitwise those
+    of bpt_layer_forward_train; bpt_layer_backward_keep_o, which reads it
+    instead of recomputing the attention, gives bitwise the gradients of
+    bpt_layer_backward."""
+    inp = make_inputs(cfg)
+    dev = bpt.to_device(inp, cfg.dtype)
+    x = dev["x"]
+    opts = {"schedule": schedule, "max_wave": wave}
+    out0, stats0, _ = bpt.layer_forward_train(x, dev, cfg.h, cfg.causal, opts=opts)
+    o = torch.full((cfg.B, cfg.N, cfg.d), float("nan"), dtype=torch.float16, device="cuda")
+    out1, stats1, ws = bpt.layer_forward_train(x, dev, cfg.h, cfg.causal, opts=opts, keep_o=o)
+    st, site = bpt.bpt_read_device_error(ws.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    assert st == bpt.BPT_OK, f"device error {bpt.status_string(st)} at site {site}"
+    assert torch.equal(out0, out1) and torch.equal(stats0, stats1)
+    got_o = o.float().cpu().numpy()
+    assert np.all(np.isfinite(got_o))
+    for b in range(cfg.B):
+        want_o = oracle.layer_intermediates(inp, cfg.h, cfg.causal, b)["O"]
+        err = np.abs(got_o[b] - want_o)
+        # fp16 scores / P / V and an fp16 output: a few fp16 roundings of values <= ~3
+        assert err.max() < 2e-2 and err.mean() < 2e-3, (b, err.max(), err.mean())
+    dZ = torch.from_numpy(upstream(cfg)).cuda()
+    bopts = {"max_wave": wave} if wave else None
+    g_rec, _ = bpt.layer_backward(x, dev, cfg.h, cfg.causal, stats1, dZ, opts=bopts)
+    g_kept, bws = bpt.layer_backward(x, dev, cfg.h, cfg.causal, stats1, dZ, opts=bopts, o=o)
+    st, site = bpt.bpt_read_device_error(bws.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    assert st == bpt.BPT_OK, f"device error {bpt.status_string(st)} at site {site}"
+    for k in g_rec:
+        assert torch.equal(g_rec[k], g_kept[k]), k
