@@ -42,23 +42,33 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
 # launch of the default bench command, from a one-kernel, one-launch ncu
 # capture with those two metrics only (one pass: nothing saved or replayed;
-# profiles/attn_pair_tc_long_n64k_dram.md).  Valid only for the sources it was
-# taken on: the digest covers the attention kernel, the shared device helpers
-# and the host launch code; after a change the bench reports null until the
-# one-launch capture is taken again.
+# profiles/attn_pair_tc_long_n64k_dram.md).  Valid only for the code it was
+# taken on: the digest covers the attention kernel, the shared device helpers,
+# the host function that configures its launch (grid, head groups, the K/V
+# budget) and the fused schedule's call of it; after a change there the bench
+# reports null until the one-launch capture is taken again.
 ATTN_TRAFFIC = {
+    "long_n64k": {"bytes_per_launch": 1446684672, "digest": "c86a6a3184ec91f3"},
 }
-TRAFFIC_SOURCES = ("blockwise_attn_ffn_b200/csrc/attn_pair_tc.cuh",
-                   "blockwise_attn_ffn_b200/csrc/common.cuh",
-                   "blockwise_attn_ffn_b200/csrc/bpt_api.cu")
+TRAFFIC_FILES = ("blockwise_attn_ffn_b200/csrc/attn_pair_tc.cuh",
+                 "blockwise_attn_ffn_b200/csrc/common.cuh")
+TRAFFIC_API = "blockwise_attn_ffn_b200/csrc/bpt_api.cu"
 
 
 def sources_digest() -> str:
     import hashlib
+    import re
     h = hashlib.sha256()
-    for rel in TRAFFIC_SOURCES:
+    for rel in TRAFFIC_FILES:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
+    with open(os.path.join(ROOT, TRAFFIC_API)) as f:
+        api = f.read()
+    a = api.index("cudaError_t launch_attn(")
+    h.update(api[a:api.index("\n}\n", a)].encode())
+    a = api.index("// attention over every query block")
+    h.update(api[a:api.index("LaunchScope ls(BPT_KIND_TAIL", a)].encode())
+    h.update(re.search(r"#define BPT_ATTN_KV_BUDGET_MB \d+", api).group(0).encode())
     return h.hexdigest()[:16]
 
 
