@@ -86,3 +86,24 @@ def test_attn_block_rejects_other_values():
         st, _ = bpt.bpt_layer_workspace_size_opt(1, 256, 256, 2, 512, True, bpt.BPT_BF16,
                                                  {"attn_block": bad})
         assert st == bpt.BPT_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("cfg,wave", [CASES[0], CASES[1], CASES[3]],
+                         ids=lambda c: getattr(c, "name", str(c)))
+def test_kept_attention_output_is_block_size_neutral(cfg, wave):
+    """bpt_layer_forward_train_keep_o with every block size: the same output,
+    statistics and kept attention output, bit for bit (each kernel writes o
+    to the caller's buffer through the same row-stride override)."""
+    dev = bpt.to_device(make_inputs(cfg), cfg.dtype)
+    got = {}
+    for b in (256, 64, 128, 512):
+        o = torch.full((cfg.B, cfg.N, cfg.d), float("nan"), dtype=torch.float16, device="cuda")
+        out, stats, ws = bpt.layer_forward_train(dev["x"], dev, cfg.h, cfg.causal,
+                                                 opts={"attn_block": b}, keep_o=o)
+        st, site = bpt.bpt_read_device_error(ws.data_ptr(), torch.cuda.current_stream().cuda_stream)
+        assert st == bpt.BPT_OK, f"b = {b}: {bpt.status_string(st)} at site {site}"
+        got[b] = (out.cpu().numpy(), stats.cpu().numpy(), o.float().cpu().numpy())
+    assert np.all(np.isfinite(got[256][2]))
+    for b in (64, 128, 512):
+        for k, name in enumerate(("out", "stats", "o")):
+            np.testing.assert_array_equal(got[b][k], got[256][k], err_msg=f"b = {b}: {name}")
