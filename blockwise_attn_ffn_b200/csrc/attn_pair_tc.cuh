@@ -80,7 +80,7 @@ struct AttnPairParams {
   // K | V of every rank, [G][B][N / G][2d], where chunk c is held by rank
   // c < G ? c : 2G-1-c as its local chunk c < G ? 0 : 1.
   int kv_cb, q_c0, q_c1, kv_G, N_kv;
-  // Block gating (kernel instantiated with GATE only):
+  // Block gating (attn_gate_tc_kernel only):
   const float* gate_t;  // [h][nb] thresholds T in units of s = q.k / sqrt(d_k)
   float* gate_bmax;     // nullable [B][h][nb][nb]: s_max of each visited pair
   uint8_t* gate_kept;   // nullable [B][h][nb][nb]: 1 processed, 0 pruned
@@ -228,18 +228,6 @@ __device__ __forceinline__ int shard_global_block(const AttnPairParams& p, int i
   return (i < p.kv_cb ? p.q_c0 : p.q_c1) * p.kv_cb + (i % p.kv_cb);
 }
 
-// GATE: block-sparse gating ("Block Sparse Flash Attention", sections
-// "Methodology and Mechanism" and "Gating Mechanism and Threshold
-// Calibration").  After S_X(j) the tile's four softmax warps reduce their
-// row maxima (valid query rows only) to the block maximum s_max; an
-// off-diagonal block with s_max < T[head, i] is pruned: no exponentials, no
-// change to (m, l), no PV product (the UMMA warp reads the tile's decision
-// after the P hand-over).  The ring then carries K one block ahead of V
-// (K_0 K_1 V_0 K_2 V_1 ...): the producer issues V_j only once the tiles that
-// visit block j have decided, at once if tile A keeps it, and completes the
-// slot without a load when every visiting tile prunes it, so pruned blocks
-// cost no V traffic ("Block Sparse Flash Attention", "Methodology and
-// Mechanism": a pruned block's values are neither loaded nor multiplied).
 // XP: b = 512.  A cluster of two CTAs takes four consecutive query blocks
 // (two per CTA) and shares every K/V tile: each CTA TMA-loads one 64-key half
 // of each tile from L2 (mapKV: 64-row boxes of QKV) and copies it into the
@@ -250,11 +238,11 @@ __device__ __forceinline__ int shard_global_block(const AttnPairParams& p, int i
 // warp's arrive) and the partner's copy has (its bytes), and empty when both
 // CTAs' UMMA warps have released it (multicast commit).  Both CTAs walk the
 // key blocks of all four query blocks.
-template <int D, int EMU, bool GATE = false, bool SHARD = false, bool XP = false>
+template <int D, int EMU, bool SHARD = false, bool XP = false>
 __global__ void __launch_bounds__(384, 1)
     attn_pair_tc_kernel(const __grid_constant__ CUtensorMap mapQKV,
                         const __grid_constant__ CUtensorMap mapKV, const AttnPairParams p) {
-  static_assert(!(XP && (GATE || SHARD)), "the b = 512 pair is dense and unsharded");
+  static_assert(!(XP && SHARD), "the b = 512 pair is unsharded");
   using C = AttnPairCfg<D, EMU>;
   constexpr int kFwdHandovers = fwd_handovers<D>();
   constexpr int kFwdChunksPerHand = 4 / kFwdHandovers;
@@ -273,13 +261,6 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t half0 = smem_u32(bars + 14 + 2 * C::NSLOT);  // XP: own half landed
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
-  // per tile, per softmax warp: {max of its rows (float bits), block count}
-  // in one 64-bit word, so a reader sees a value together with its block
-  __shared__ unsigned long long gate_slot[2][4];
-  __shared__ int gate_keep[2];      // per tile: the current block's decision
-  // per tile, the decisions of the last four blocks as ((j + 1) << 1) | keep,
-  // at [j & 3]: the producer issues V_j only once they are known
-  __shared__ int gate_dec[2][4];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // blockIdx -> (head group, work rank, head): within a group, consecutive
@@ -339,10 +320,6 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(o_done0 + 8 * x, 1);
     }
     mbar_init(drain, 1);
-    if constexpr (GATE) {
-      for (int i = 0; i < 8; ++i) (&gate_slot[0][0])[i] = 0ull;
-      for (int i = 0; i < 8; ++i) (&gate_dec[0][0])[i] = 0;
-    }
     abort_sh = 0;
     fence_mbar_init();
   }
@@ -416,7 +393,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       for (int s = 0; s < C::NSLOT; ++s)
         if (armed_h[s] >= 0) mbar_wait_drain(half0 + 8 * s, static_cast<uint32_t>(armed_h[s]), p.err);
-    } else if constexpr (!GATE) {
+    } else {
       // ring order K_0 V_0 K_1 V_1 ...
       for (int j = 0; j < n_kv && ok; ++j) {
         for (int w = 0; w < 2; ++w) {
@@ -450,81 +427,6 @@ __global__ void __launch_bounds__(384, 1)
             slot = 0;
             phase ^= 1u;
           }
-        }
-      }
-    } else {
-      // Gated ring order: K_0 K_1 V_0 K_2 V_1 ... V_n-1, so
-      // K runs one block ahead of V and V_j waits for the gate decisions of
-      // block j (issued at once when tile A keeps it; skipped when every tile
-      // that visits block j prunes it).
-      for (int t = 0; t < 2 * n_kv && ok; ++t) {
-        int j, w;  // key block, 0 = K / 1 = V
-        if (t == 0) {
-          j = 0;
-          w = 0;
-        } else if ((t & 1) && (t + 1) / 2 < n_kv) {
-          j = (t + 1) / 2;
-          w = 0;
-        } else {
-          j = (t & 1) ? n_kv - 1 : t / 2 - 1;
-          w = 1;
-        }
-        if (!mbar_wait_warp(ring_empty0 + 8 * slot, phase ^ 1u, abort_flag, p.err,
-                            kSiteAttnProducer)) {
-          ok = false;
-          break;
-        }
-        bool load = true;
-        if (GATE && w == 1) {
-          // wait (bounded) for the decisions of the tiles that visit block j
-          const bool needA = j < nA, needB = j < nB;
-          const int tag = (j + 1) << 1;
-          bool seen = false;
-          const uint64_t g0 = global_ns();
-          for (uint32_t it = 0;; ++it) {
-            const int da = *reinterpret_cast<volatile int*>(&gate_dec[0][j & 3]);
-            const int db = *reinterpret_cast<volatile int*>(&gate_dec[1][j & 3]);
-            const bool haveA = !needA || (da & ~1) == tag;
-            const bool haveB = !needB || (db & ~1) == tag;
-            const bool keepA = needA && da == (tag | 1);
-            const bool keepB = needB && db == (tag | 1);
-            if (keepA || (haveA && haveB)) {
-              load = keepA || keepB;
-              seen = true;
-              break;
-            }
-            if ((it & 63u) == 63u) {
-              if (*abort_flag) break;
-              if (global_ns() - g0 > BPT_WAIT_LIMIT_NS) {
-                record_error(p.err, kErrTimeout, kSiteAttnProducer);
-                *abort_flag = 1;
-                break;
-              }
-            }
-          }
-          if (!__all_sync(0xffffffffu, seen)) {
-            ok = false;
-            break;
-          }
-        }
-        const uint32_t fb = ring_full0 + 8 * slot;
-        {
-          armed[slot] = static_cast<int>(phase);
-          if (leader) {
-            if (!load) {
-              mbar_arrive_expect_tx(fb, 0);  // V_j not needed: the slot completes empty
-            } else {
-              mbar_arrive_expect_tx(fb, C::TILE);
-              const int col = w == 0 ? colK : colV;
-              tma_load_4d(smem_u32(smem + C::OFF_RING + slot * C::TILE), &mapQKV, fb, 0,
-                          j * C::BKV, col / 64, bidx);
-            }
-          }
-        }
-        __syncwarp();
-        if (++slot == C::NSLOT) {
-          slot = 0;
-          phase ^= 1u;
         }
       }
     }
@@ -630,27 +532,12 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int j = 0; j < n_kv && ok; ++j) {
       // ring positions of K_j+1 and V_j (see the producer's order)
-      const int tk = GATE ? 2 * j + 1 : 2 * (j + 1);
-      const int tv = GATE ? (j < n_kv - 1 ? 2 * j + 2 : 2 * n_kv - 1) : 2 * j + 1;
+      const int tk = 2 * (j + 1);
+      const int tv = 2 * j + 1;
       bool k_ready = false;
-      // V_j is waited for before its first PV chunk, or (every visiting tile
-      // pruned block j: the producer completes the slot without loading) at
-      // the end of the block, before the slot is released
-      bool v_ready = false;
-      if constexpr (!GATE) {  // dense: V_j is always loaded; wait at once
-        if (!mbar_wait_warp(ring_full0 + 8 * slot_of(tv), phase_of(tv), abort_flag, p.err,
-                            kSiteAttnMma))
-          break;
-        v_ready = true;
-      }
-      auto wait_v = [&]() {
-        if (!v_ready) {
-          ok = mbar_wait_warp(ring_full0 + 8 * slot_of(tv), phase_of(tv), abort_flag, p.err,
-                              kSiteAttnMma);
-          v_ready = true;
-        }
-        return ok;
-      };
+      if (!mbar_wait_warp(ring_full0 + 8 * slot_of(tv), phase_of(tv), abort_flag, p.err,
+                          kSiteAttnMma))
+        break;
       const uint32_t v_lo = sdesc_lo(ring + slot_of(tv) * C::TILE, C::CHUNK);
       const uint32_t k_lo = sdesc_lo(ring + slot_of(tk) * C::TILE, 16);
       for (int x = 0; x < 2 && ok; ++x) {
@@ -659,29 +546,19 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t tS = tmem + (x == 0 ? 0u : C::TM_S_B);
         const uint32_t tO = tmem + (x == 0 ? C::TM_O_A : C::TM_O_B);
         // PV_X(j) as the P hand-overs come (each 128 / kFwdHandovers keys)
-        bool kept = true;
         for (int hh = 0; hh < kFwdHandovers; ++hh) {
-          // A pruned block hands everything over at once, after S_X(j) was
-          // read in full: its first hand-over is all the UMMA warp needs.
-          // (The skipped phases complete regardless; the next block's waits,
-          // one phase later, are unaffected.)
-          if (GATE && hh > 0 && !kept) continue;
           if (!mbar_wait_warp(p_chunk0 + 8 * (4 * x + hh), pph[x], abort_flag, p.err,
                               kSiteAttnMma)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          // (the tile's decision was written before its first P hand-over)
-          if (hh == 0) kept = !GATE || *reinterpret_cast<volatile int*>(&gate_keep[x]) != 0;
-          if (kept && !wait_v()) break;
-          if (kept)
-            for (int q = 0; q < kFwdChunksPerHand; ++q)
-              issue_pv_chunk(tS, v_lo, tO, hh * kFwdChunksPerHand + q, !o_started[x]);
+          for (int q = 0; q < kFwdChunksPerHand; ++q)
+            issue_pv_chunk(tS, v_lo, tO, hh * kFwdChunksPerHand + q, !o_started[x]);
         }
         if (!ok) break;
         pph[x] ^= 1u;
-        if (kept) o_started[x] = true;
+        o_started[x] = true;
         if (j + 1 < nX) {
           if (!k_ready) {
             if (!mbar_wait_warp(ring_full0 + 8 * slot_of(tk), phase_of(tk), abort_flag, p.err,
@@ -698,7 +575,7 @@ __global__ void __launch_bounds__(384, 1)
           commit(o_done0 + 8 * x);
         }
       }
-      if (!ok || !wait_v()) break;
+      if (!ok) break;
       if (XP && !k_ready && j + 1 < n_kv) {
         // the cluster's ring goes on past this CTA's blocks: consume K_j+1
         if (!mbar_wait_warp(ring_full0 + 8 * slot_of(tk), phase_of(tk), abort_flag, p.err,
@@ -729,11 +606,7 @@ __global__ void __launch_bounds__(384, 1)
     float m_run = -INFINITY;  // reference maximum (moves only by > 2^8 in exp2 units)
     float m_true = -INFINITY;  // exact running row maximum, for the statistics
     float l = 0.f;
-    bool o_live = false;       // O holds a PV product (a block has been kept)
-    // the tile's threshold (loaded once: the loop below stores to global
-    // memory, so the compiler would not hoist it)
-    float t_thr = 0.f;
-    if constexpr (GATE) t_thr = nX > 0 ? p.gate_t[head * p.nb + iX] : 0.f;
+    bool o_live = false;       // O holds a PV product
     bool ok = nX > 0;
     for (int j = 0; j < nX && ok; ++j) {
       if (!mbar_wait_fast(s_full, j & 1, abort_flag, p.err, kSiteAttnSoftmax)) {
@@ -766,134 +639,72 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int k = 0; k < 4; ++k) mxp[k] = fmaxf(mxp[k], mxp[k + 4]);
       const float mx = fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3]));
-      bool keep_blk = true;
-      if constexpr (GATE) {
-        // block maximum over the tile's valid query rows, in units of s
-        float wm = (iX * C::BQ + r < p.N) ? mx : -INFINITY;
+      m_true = fmaxf(m_true, mx);
+      float m_new = m_run;
+      bool need = false;
+      if (mx > m_run) {
+        need = (m_run == -INFINITY) || ((mx - m_run) * c > 8.0f);
+        if (need) m_new = mx;
+      }
+      const bool warp_need = __any_sync(0xffffffffu, need) && o_live;
+      const float alpha =
+          need ? (m_run == -INFINITY ? 0.f : ex2_approx((m_run - m_new) * c)) : 1.f;
+      // Rescale O first: the PV of this block starts with its first P
+      // chunk (PV_X(j-1) is complete: S_X(j), issued after it, has landed).
+      if (warp_need) {
+#pragma unroll 1
+        for (int cc = 0; cc < D / 8; ++cc) {
+          uint32_t v[8];
+          tmem_ld_32x32b_x8(tO + cc * 8, v);
+          tmem_ld_wait();
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, o));
-        // exchange through shared memory: write {max, j + 1}, then poll the
-        // tile's four slots until each carries block j (a warp cannot reach
-        // block j + 1 before all four have read block j: S_j+1 waits for
-        // their P hand-over).  The poll is bounded like every other wait.
-        const uint32_t tag = static_cast<uint32_t>(j + 1);
-        if (lane == 0)
-          *reinterpret_cast<volatile unsigned long long*>(&gate_slot[x][e]) =
-              (static_cast<unsigned long long>(tag) << 32) | __float_as_uint(wm);
-        float bmax = -INFINITY;
-        bool seen = false;
-        const uint64_t g0 = global_ns();
-        for (uint32_t it = 0;; ++it) {
-          const volatile unsigned long long* sl = &gate_slot[x][0];
-          const unsigned long long v0 = sl[0], v1 = sl[1], v2 = sl[2], v3 = sl[3];
-          if (static_cast<uint32_t>(v0 >> 32) == tag && static_cast<uint32_t>(v1 >> 32) == tag &&
-              static_cast<uint32_t>(v2 >> 32) == tag && static_cast<uint32_t>(v3 >> 32) == tag) {
-            bmax = fmaxf(fmaxf(__uint_as_float(static_cast<uint32_t>(v0)),
-                               __uint_as_float(static_cast<uint32_t>(v1))),
-                         fmaxf(__uint_as_float(static_cast<uint32_t>(v2)),
-                               __uint_as_float(static_cast<uint32_t>(v3))));
-            seen = true;
-            break;
-          }
-          if ((it & 63u) == 63u) {
-            if (*abort_flag) break;
-            if (global_ns() - g0 > BPT_WAIT_LIMIT_NS) {
-              record_error(p.err, kErrTimeout, kSiteAttnSoftmax);
-              *abort_flag = 1;
-              break;
-            }
-          }
-        }
-        if (!__all_sync(0xffffffffu, seen)) {
-          ok = false;
-          break;
-        }
-        const float smax = bmax * (p.scale_log2 * 0.69314718055994531f);
-        keep_blk = (j == gX) || (smax >= t_thr);
-        if (e == 0 && lane == 0) {
-          gate_keep[x] = keep_blk ? 1 : 0;
-          *reinterpret_cast<volatile int*>(&gate_dec[x][j & 3]) =
-              ((j + 1) << 1) | (keep_blk ? 1 : 0);
-          const long long o = ((static_cast<long long>(bidx) * p.h + head) * p.nb + iX) * p.nb + j;
-          if (p.gate_bmax != nullptr) p.gate_bmax[o] = smax;
-          if (p.gate_kept != nullptr) p.gate_kept[o] = keep_blk ? 1 : 0;
+          for (int k = 0; k < 8; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * alpha);
+          tmem_st_32x32b_x8(tO + cc * 8, v);
         }
       }
-      if (keep_blk) {
-        m_true = fmaxf(m_true, mx);
-        float m_new = m_run;
-        bool need = false;
-        if (mx > m_run) {
-          need = (m_run == -INFINITY) || ((mx - m_run) * c > 8.0f);
-          if (need) m_new = mx;
-        }
-        const bool warp_need = __any_sync(0xffffffffu, need) && o_live;
-        const float alpha =
-            need ? (m_run == -INFINITY ? 0.f : ex2_approx((m_run - m_new) * c)) : 1.f;
-        // Rescale O first: the PV of this block starts with its first P
-        // chunk (PV_X(j-1) is complete: S_X(j), issued after it, has landed).
-        if (warp_need) {
-#pragma unroll 1
-          for (int cc = 0; cc < D / 8; ++cc) {
-            uint32_t v[8];
-            tmem_ld_32x32b_x8(tO + cc * 8, v);
-            tmem_ld_wait();
+      const float2 cc2 = make_float2(c, c);
+      const float2 mref2 = make_float2(-m_new * c, -m_new * c);
+      float2 sum2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
+      // One unrolled loop per tile kind, so the MUFU / FMA choice of each
+      // 16-column group is fixed at compile time (no per-element branch).
+      // Each 32-key chunk of P is handed over as soon as it is stored.
+      auto exp_row = [&](auto emu_mask) {
+        constexpr uint32_t kMask = decltype(emu_mask)::value;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * alpha);
-            tmem_st_32x32b_x8(tO + cc * 8, v);
-          }
-        }
-        const float2 cc2 = make_float2(c, c);
-        const float2 mref2 = make_float2(-m_new * c, -m_new * c);
-        float2 sum2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                          make_float2(0.f, 0.f)};
-        // One unrolled loop per tile kind, so the MUFU / FMA choice of each
-        // 16-column group is fixed at compile time (no per-element branch).
-        // Each 32-key chunk of P is handed over as soon as it is stored.
-        auto exp_row = [&](auto emu_mask) {
-          constexpr uint32_t kMask = decltype(emu_mask)::value;
+        for (int cc = 0; cc < C::BKV / 32; ++cc) {
+          uint32_t pk[16];
 #pragma unroll
-          for (int cc = 0; cc < C::BKV / 32; ++cc) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int k = 0; k < 32; k += 2) {
-              const int col = cc * 32 + k;
-              float2 a = __ffma2_rn(
-                  make_float2(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])), cc2, mref2);
-              float2 e2;
-              if ((kMask >> (col >> 4)) & 1u) {
-                e2 = exp2_poly2(a);
-              } else {
-                e2.x = ex2_approx(a.x);
-                e2.y = ex2_approx(a.y);
-              }
-              sum2[(k >> 1) & 3] = __fadd2_rn(sum2[(k >> 1) & 3], e2);
-              pk[k >> 1] = pack_f16x2(e2.x, e2.y);
+          for (int k = 0; k < 32; k += 2) {
+            const int col = cc * 32 + k;
+            float2 a = __ffma2_rn(
+                make_float2(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])), cc2, mref2);
+            float2 e2;
+            if ((kMask >> (col >> 4)) & 1u) {
+              e2 = exp2_poly2(a);
+            } else {
+              e2.x = ex2_approx(a.x);
+              e2.y = ex2_approx(a.y);
             }
-            tmem_st_32x32b_x16(tS + cc * 16, pk);
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0 && (cc + 1) % kFwdChunksPerHand == 0)
-              mbar_arrive(p_chunk + 8 * (cc / kFwdChunksPerHand));
+            sum2[(k >> 1) & 3] = __fadd2_rn(sum2[(k >> 1) & 3], e2);
+            pk[k >> 1] = pack_f16x2(e2.x, e2.y);
           }
-        };
-        if (masked || emu_group_mask(EMU) == 0u)
-          exp_row(std::integral_constant<uint32_t, 0u>{});
-        else
-          exp_row(std::integral_constant<uint32_t, emu_group_mask(EMU)>{});
-        sum2[0] = __fadd2_rn(__fadd2_rn(sum2[0], sum2[1]), __fadd2_rn(sum2[2], sum2[3]));
-        l = alpha * l + (sum2[0].x + sum2[0].y);
-        m_run = m_new;
-        o_live = true;
-      } else {
-        // pruned: no P; the hand-overs still tell the UMMA warp that S_X(j)
-        // has been read and carry the decision
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0)
-          for (int hh = 0; hh < kFwdHandovers; ++hh) mbar_arrive(p_chunk + 8 * hh);
-      }  // keep_blk
+          tmem_st_32x32b_x16(tS + cc * 16, pk);
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0 && (cc + 1) % kFwdChunksPerHand == 0)
+            mbar_arrive(p_chunk + 8 * (cc / kFwdChunksPerHand));
+        }
+      };
+      if (masked || emu_group_mask(EMU) == 0u)
+        exp_row(std::integral_constant<uint32_t, 0u>{});
+      else
+        exp_row(std::integral_constant<uint32_t, emu_group_mask(EMU)>{});
+      sum2[0] = __fadd2_rn(__fadd2_rn(sum2[0], sum2[1]), __fadd2_rn(sum2[2], sum2[3]));
+      l = alpha * l + (sum2[0].x + sum2[0].y);
+      m_run = m_new;
+      o_live = true;
     }
     if (ok && mbar_wait_fast(o_done, 0, abort_flag, p.err, kSiteAttnSoftmax)) {
       tc_fence_after();

@@ -34,6 +34,7 @@
 #include "attn_bwd_tc.cuh"
 #include "attn_pair_tc.cuh"
 #include "attn_b64_tc.cuh"
+#include "attn_gate_tc.cuh"
 #include "backward.cuh"
 #include "common.cuh"
 #include "gemm_tc.cuh"
@@ -249,15 +250,15 @@ bpt_status device_info(int* sms, int* pair_clusters = nullptr) {
     if (di.ok) {
       if (set_smem(bpt::attn_pair_tc_kernel<64, kEmu64>, bpt::AttnPairCfg<64, kEmu64>::SMEM) ||
           set_smem(bpt::attn_pair_tc_kernel<128, kEmu128>, bpt::AttnPairCfg<128, kEmu128>::SMEM) ||
-          set_smem(bpt::attn_pair_tc_kernel<64, kEmu64, true>, bpt::AttnPairCfg<64, kEmu64>::SMEM) ||
-          set_smem(bpt::attn_pair_tc_kernel<64, kEmu64, false, false, true>,
-                   bpt::AttnPairCfg<64, kEmu64>::SMEM) ||
-          set_smem(bpt::attn_pair_tc_kernel<128, kEmu128, false, false, true>,
-                   bpt::AttnPairCfg<128, kEmu128>::SMEM) ||
+          set_smem(bpt::attn_gate_tc_kernel<64, kEmu64>, bpt::AttnGateCfg<64>::SMEM) ||
+          set_smem(bpt::attn_gate_tc_kernel<128, kEmu128>, bpt::AttnGateCfg<128>::SMEM) ||
+          // b = 512 cluster pair (SHARD = false, XP = true) and sequence shard
           set_smem(bpt::attn_pair_tc_kernel<64, kEmu64, false, true>,
                    bpt::AttnPairCfg<64, kEmu64>::SMEM) ||
           set_smem(bpt::attn_pair_tc_kernel<128, kEmu128, false, true>,
                    bpt::AttnPairCfg<128, kEmu128>::SMEM) ||
+          set_smem(bpt::attn_pair_tc_kernel<64, kEmu64, true>,
+                   bpt::AttnPairCfg<64, kEmu64>::SMEM) ||
           set_smem(bpt::attn_pair_tc_kernel<128, kEmu128, true>,
                    bpt::AttnPairCfg<128, kEmu128>::SMEM) ||
           set_smem(bpt::gemm_f16_pair_kernel<4, bpt::kLayAkBn>, bpt::kPairSmem) ||
@@ -575,11 +576,11 @@ cudaError_t launch_attn(const Plan& P, const Wave& wv_, const CUtensorMap& mQKV,
     cfg.numAttrs = 1;
     if (P.dk == 128) {
       cfg.dynamicSmemBytes = bpt::AttnPairCfg<128, kEmu128>::SMEM;
-      return cudaLaunchKernelEx(&cfg, bpt::attn_pair_tc_kernel<128, kEmu128, false, false, true>,
+      return cudaLaunchKernelEx(&cfg, bpt::attn_pair_tc_kernel<128, kEmu128, false, true>,
                                 mQKV, *xp_map, ap);
     }
     cfg.dynamicSmemBytes = bpt::AttnPairCfg<64, kEmu64>::SMEM;
-    return cudaLaunchKernelEx(&cfg, bpt::attn_pair_tc_kernel<64, kEmu64, false, false, true>,
+    return cudaLaunchKernelEx(&cfg, bpt::attn_pair_tc_kernel<64, kEmu64, false, true>,
                               mQKV, *xp_map, ap);
   }
   if (gate != nullptr) {
@@ -587,17 +588,16 @@ cudaError_t launch_attn(const Plan& P, const Wave& wv_, const CUtensorMap& mQKV,
     ap.gate_bmax = gate->bmax;
     ap.gate_kept = gate->kept;
     if (P.dk == 128)
+      bpt::attn_gate_tc_kernel<128, kEmu128>
+          <<<grid, 384, bpt::AttnGateCfg<128>::SMEM, s>>>(mQKV, ap);
+    else
+      bpt::attn_gate_tc_kernel<64, kEmu64><<<grid, 384, bpt::AttnGateCfg<64>::SMEM, s>>>(mQKV, ap);
+  } else if (shard != nullptr) {
+    if (P.dk == 128)
       bpt::attn_pair_tc_kernel<128, kEmu128, true>
           <<<grid, 384, bpt::AttnPairCfg<128, kEmu128>::SMEM, s>>>(mQKV, mKV, ap);
     else
       bpt::attn_pair_tc_kernel<64, kEmu64, true>
-          <<<grid, 384, bpt::AttnPairCfg<64, kEmu64>::SMEM, s>>>(mQKV, mKV, ap);
-  } else if (shard != nullptr) {
-    if (P.dk == 128)
-      bpt::attn_pair_tc_kernel<128, kEmu128, false, true>
-          <<<grid, 384, bpt::AttnPairCfg<128, kEmu128>::SMEM, s>>>(mQKV, mKV, ap);
-    else
-      bpt::attn_pair_tc_kernel<64, kEmu64, false, true>
           <<<grid, 384, bpt::AttnPairCfg<64, kEmu64>::SMEM, s>>>(mQKV, mKV, ap);
   } else if (P.dk == 128) {
     bpt::attn_pair_tc_kernel<128, kEmu128>

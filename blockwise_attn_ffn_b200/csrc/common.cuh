@@ -97,6 +97,26 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile i
   }
 }
 
+// mbar_wait inlined whole: for waits placed where many registers are live
+// (a call there makes the caller spill them).
+__device__ __forceinline__ bool mbar_wait_inline(uint32_t bar, uint32_t parity,
+                                                 volatile int* abort_flag, uint32_t* err,
+                                                 uint32_t site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0u) {
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > BPT_WAIT_LIMIT_NS) {
+        record_error(err, kErrTimeout, site);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
 // Same as mbar_wait, with the already-complete case inlined (no call).
 __device__ __forceinline__ bool mbar_wait_fast(uint32_t bar, uint32_t parity,
                                                volatile int* abort_flag, uint32_t* err,
@@ -189,6 +209,14 @@ __device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map
 // proxy (tensor core operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 16-byte store to a shared-memory address (32-bit shared window).
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
 }
 
 // --------------------------------------------------------------- tcgen05 --
