@@ -147,33 +147,71 @@ __global__ void ln_backward_kernel(const TX* __restrict__ X, const TG* __restric
   if (rowstat && lane == 0) rowstat[r] = make_float2(mu, rstd);
 }
 
+// Four consecutive elements as fp32 (p 4-element aligned).
+__device__ __forceinline__ float4 ld4_as_float(const float* p) {
+  return *reinterpret_cast<const float4*>(p);
+}
+__device__ __forceinline__ float4 ld4_as_float(const __half* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+  const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+__device__ __forceinline__ float4 ld4_as_float(const __nv_bfloat16* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+
 // Column sums over `rows` rows split into row chunks, one partial per chunk:
 //   part_a[chunk, c] = sum_r A[row(r), c]
 //   part_b[chunk, c] = sum_r A[row(r), c] * (X[g(r), c] - mean_r) * rstd_r   (if X)
 // A is indexed by the local row (a_global = 0) or by g = map(r) (a_global = 1).
+// With a wave map a chunk is one query block (rows_per_chunk = map.blk), whose
+// valid rows map to consecutive token rows; with the identity map, any run of
+// rows.  Each thread sums four adjacent columns (d % 4 == 0) over its chunk's
+// rows in order.
 template <typename TA, typename TX>
 __global__ void colsum_partial_kernel(const TA* __restrict__ A, int a_global,
                                       const TX* __restrict__ X, const float2* __restrict__ rowstat,
                                       float* __restrict__ part_a, float* __restrict__ part_b,
                                       long long rows, int d, int rows_per_chunk, RowMap map) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  const int c = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
   const int chunk = blockIdx.y;
   if (c >= d) return;
   const long long r0 = static_cast<long long>(chunk) * rows_per_chunk;
-  const long long r1 = min(rows, r0 + rows_per_chunk);
-  float sa = 0.f, sb = 0.f;
-  for (long long r = r0; r < r1; ++r) {
-    const long long g = map.map(r);
-    if (g < 0) continue;
-    const float a = ld_as_float(A + (a_global ? g : r) * d + c);
-    sa += a;
+  long long g0;  // token row of the chunk's first row
+  int nv;        // rows of the chunk that exist
+  if (map.identity) {
+    g0 = r0;
+    nv = static_cast<int>(min(static_cast<long long>(rows_per_chunk), rows - r0));
+  } else {
+    const long long item = map.item0 + r0 / map.blk;
+    const long long b = item / map.nb;
+    const long long pos0 = (item - b * map.nb) * map.blk;
+    g0 = b * map.N + pos0;
+    nv = static_cast<int>(min(static_cast<long long>(map.blk), map.N - pos0));
+  }
+  float4 sa = make_float4(0.f, 0.f, 0.f, 0.f), sb = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+  for (int i = 0; i < nv; ++i) {
+    const float4 a = ld4_as_float(A + (a_global ? g0 + i : r0 + i) * d + c);
+    sa.x += a.x;
+    sa.y += a.y;
+    sa.z += a.z;
+    sa.w += a.w;
     if (X) {
-      const float2 st = rowstat[r];
-      sb += a * (ld_as_float(X + g * d + c) - st.x) * st.y;
+      const float2 st = rowstat[r0 + i];
+      const float4 x = ld4_as_float(X + (g0 + i) * d + c);
+      sb.x += a.x * (x.x - st.x) * st.y;
+      sb.y += a.y * (x.y - st.x) * st.y;
+      sb.z += a.z * (x.z - st.x) * st.y;
+      sb.w += a.w * (x.w - st.x) * st.y;
     }
   }
-  part_a[static_cast<long long>(chunk) * d + c] = sa;
-  if (X) part_b[static_cast<long long>(chunk) * d + c] = sb;
+  *reinterpret_cast<float4*>(part_a + static_cast<long long>(chunk) * d + c) = sa;
+  if (X) *reinterpret_cast<float4*>(part_b + static_cast<long long>(chunk) * d + c) = sb;
 }
 
 // out[c] += sum over chunks of part[chunk, c], chunks in order (deterministic).

@@ -939,11 +939,14 @@ template <typename TA, typename TX>
 cudaError_t launch_colsum(const TA* A, int a_global, const TX* X, const float2* rowstat,
                           int64_t rows, int64_t d, RowMap map, float* part_a, float* part_b,
                           float* out_a, float* out_b, cudaStream_t s) {
-  const int rpc = int((rows + kColChunks - 1) / kColChunks);
+  // a wave map: one chunk per query block (at most BPT_WAVE_BLOCKS of them);
+  // the identity map: kColChunks runs of rows
+  const int rpc = map.identity ? int((rows + kColChunks - 1) / kColChunks) : map.blk;
   const int chunks = int((rows + rpc - 1) / rpc);
-  bpt::colsum_partial_kernel<TA, TX><<<dim3(unsigned((d + 255) / 256), unsigned(chunks)), 256, 0,
-                                        s>>>(A, a_global, X, rowstat, part_a, part_b, rows, int(d),
-                                             rpc, map);
+  if (chunks > kColChunks || d % 4 != 0) return cudaErrorInvalidValue;
+  bpt::colsum_partial_kernel<TA, TX><<<dim3(unsigned((d / 4 + 255) / 256), unsigned(chunks)), 256,
+                                        0, s>>>(A, a_global, X, rowstat, part_a, part_b, rows,
+                                                int(d), rpc, map);
   bpt::colsum_reduce_kernel<<<unsigned((d + 255) / 256), 256, 0, s>>>(part_a, chunks, int(d),
                                                                      out_a);
   if (X) bpt::colsum_reduce_kernel<<<unsigned((d + 255) / 256), 256, 0, s>>>(part_b, chunks,
