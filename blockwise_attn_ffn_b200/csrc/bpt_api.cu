@@ -94,7 +94,12 @@ bpt_status read_opts(const bpt_options* o, Opts* r) {
 #endif
 constexpr int kEmu128 = BPT_EMU_DK128;
 constexpr int kEmu64 = BPT_EMU_DK64;
-constexpr size_t kHeaderBytes = 256;
+// Workspace header: the device error word at offset 0; from kTailFlagOffset
+// the fused layer body's hand-over counters for shared items ([2][pairs][2]
+// uint32, zeroed before each launch that shares items).
+constexpr size_t kTailFlagOffset = 256;
+constexpr size_t kTailFlagBytes = size_t(2 * bpt::kTailMaxPairs * 2) * sizeof(uint32_t);
+constexpr size_t kHeaderBytes = kTailFlagOffset + kTailFlagBytes;
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -758,7 +763,35 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
     tp.err = err;
     tp.fault = fault == 3 ? 3 : 0;
     const int64_t pairs = std::max<int64_t>(1, std::min<int64_t>(P.tail_pairs, pairs_max));
+    // Share the items left over after the whole rounds between two pairs
+    // each when at most half of the pairs would otherwise work in the last
+    // round and every half is a whole number of tiles (y tiles and H chunks
+    // of 256 columns, Z tiles of 512).
+    const int64_t left = tp.items % pairs;
+    tp.split = (left > 0 && 2 * left <= pairs && d % 1024 == 0 && d_ff % 512 == 0) ? 1 : 0;
+    tp.flags = reinterpret_cast<uint32_t*>(ws + kTailFlagOffset);
     LaunchScope ls(BPT_KIND_TAIL, s);
+    if (tp.split) {
+      // A pair waits for its partner's hand-overs, so all pairs must be
+      // resident at once: a cooperative launch guarantees it (or fails, and
+      // the layer body runs without sharing).
+      if (cudaMemsetAsync(tp.flags, 0, kTailFlagBytes, s) != cudaSuccess) return BPT_ERR_CUDA;
+      cudaLaunchConfig_t cfg{};
+      cfg.gridDim = dim3(unsigned(2 * pairs));
+      cfg.blockDim = dim3(bpt::kTailThreads);
+      cfg.dynamicSmemBytes = bpt::kPairSmem;
+      cfg.stream = s;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeCooperative;
+      attr[0].val.cooperative = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if (cudaLaunchKernelEx(&cfg, bpt::tail_pair_kernel, mO, mWo, mV, mW1, mH, mW2, mH1, mW2e,
+                             tp) == cudaSuccess)
+        return BPT_OK;
+      (void)cudaGetLastError();
+      tp.split = 0;
+    }
     bpt::tail_pair_kernel<<<unsigned(2 * pairs), bpt::kTailThreads, bpt::kPairSmem, s>>>(
         mO, mWo, mV, mW1, mH, mW2, mH1, mW2e, tp);
     if (cudaGetLastError() != cudaSuccess) return BPT_ERR_CUDA;

@@ -26,6 +26,7 @@ enum : uint32_t {
   kSiteAttnProducer = 4, kSiteAttnMma = 5, kSiteAttnSoftmax = 6,
   kSiteDrain = 7,
   kSiteRangeWeights = 8, kSiteRangeQKV = 9, kSiteRangeHidden = 10, kSiteRangeLN = 11,
+  kSiteTailPartner = 12,
 };
 
 // Largest finite fp16 value; operands beyond it (or NaN) are reported.
@@ -154,6 +155,45 @@ __device__ __noinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint
       record_error(err, kErrTimeout, kSiteDrain);
       return false;
     }
+  }
+}
+
+// ------------------------------------------------- counters across CTAs --
+// A hand-over between CTAs on different SMs: the writers make their global
+// stores visible at GPU scope and add to a counter with release semantics;
+// the reader polls it with acquire loads.
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* a) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_gpu_add(uint32_t* a, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(a), "r"(v) : "memory");
+}
+
+// Whole-warp bounded wait until *a >= target.  Every lane polls (so each
+// lane's later loads are ordered after its own acquire); lane 0 decides when
+// to give up, as mbar_wait does, and the warp follows it.
+__device__ __noinline__ bool flag_wait_warp(const uint32_t* a, uint32_t target,
+                                            volatile int* abort_flag, uint32_t* err,
+                                            uint32_t site) {
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (__all_sync(0xffffffffu, ld_acquire_gpu(a) >= target)) return true;
+    if ((it & 15u) == 15u) {
+      int give_up = 0;
+      if ((threadIdx.x & 31) == 0) {
+        if (*abort_flag) {
+          give_up = 1;
+        } else if (global_ns() - t0 > BPT_WAIT_LIMIT_NS) {
+          record_error(err, kErrTimeout, site);
+          *abort_flag = 1;
+          give_up = 1;
+        }
+      }
+      if (__shfl_sync(0xffffffffu, give_up, 0)) return false;
+    }
+    __nanosleep(100);
   }
 }
 

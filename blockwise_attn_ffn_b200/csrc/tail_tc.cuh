@@ -37,6 +37,17 @@
 // The producer issues each stage's B (weight) load before it waits for a
 // hand-off, so the weights stream in while the epilogue finishes.
 //
+// Items are dealt round-robin over the pairs.  When R whole rounds leave L
+// items over (0 < L <= pairs / 2), the last round would keep L pairs busy for
+// a whole item while the others idle; instead each left-over item is shared
+// by two pairs (q and q + L), each computing half of its y tiles, all of its
+// LN2, half of its H chunks and half of its Z tiles (by columns).  LN2 needs
+// the other pair's y columns, and a Z tile (K = d_ff) needs the other pair's
+// H columns, read from that pair's scratch; two counters per CTA in global
+// memory (written with release, polled with acquire, bounded) carry these
+// two hand-overs.  Every output element still comes from the same products
+// in the same K order, so sharing changes no bit of the result.
+//
 // Arithmetic per element is that of the wave path (same UMMA shapes and
 // K order, same epilogues, LN2 with the summation order of ln_rows_kernel),
 // so the two schedules give bitwise the same output.
@@ -61,6 +72,8 @@ struct TailParams {
   __half* v_scr;                   // [pairs*256, d]
   __half* h_scr;                   // [pairs*256, d_ff]
   uint32_t* err;
+  uint32_t* flags;  // shared items: [2][kTailMaxPairs][2] arrival counters, zero at launch
+  int split;        // share the left-over items (needs d % 1024 == 0, d_ff % 512 == 0)
   int fault;  // test hook: 3 = pair 0's leader never loads its first A tile
 };
 
@@ -71,6 +84,56 @@ constexpr int kTailMaxPairs = 74;
 
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Counter of a CTA's hand-over to the partner pair: kind 0 = its y columns
+// of the shared item are stored, 1 = its H columns are.  Each of the CTA's
+// epilogue warps adds one.
+__device__ __forceinline__ int tail_flag(int kind, int pair, uint32_t rank) {
+  return (kind * kTailMaxPairs + pair) * 2 + static_cast<int>(rank);
+}
+
+// A pair's items: j = 0 .. J-1, whole items pair + j * npairs, then (when
+// half >= 0) its half of the shared item hitem, computed with `partner`.
+struct TailPlan {
+  int J, Jfull, hitem, half, partner;
+  int first, stride;
+  __device__ __forceinline__ int item(int j) const { return j < Jfull ? first + j * stride : hitem; }
+  __device__ __forceinline__ int half_of(int j) const { return j < Jfull ? -1 : half; }
+};
+
+__device__ __forceinline__ TailPlan tail_plan(const TailParams& p, int pair, int npairs) {
+  TailPlan pl{};
+  pl.first = pair;
+  pl.stride = npairs;
+  pl.half = -1;
+  pl.hitem = 0;
+  pl.partner = pair;
+  const int R = p.items / npairs, L = p.items - R * npairs;
+  if (p.split && L > 0 && 2 * L <= npairs) {
+    pl.Jfull = R;
+    pl.J = R;
+    if (pair < 2 * L) {
+      pl.half = pair >= L ? 1 : 0;
+      pl.hitem = R * npairs + pair - pl.half * L;
+      pl.partner = pl.half ? pair - L : pair + L;
+      pl.J = R + 1;
+    }
+  } else {
+    pl.Jfull = pl.J = pair < p.items ? (p.items - pair + npairs - 1) / npairs : 0;
+  }
+  return pl;
+}
+
+// Tiles [n0, n1) of a segment of `tiles` tiles: all of them, or half h.
+__device__ __forceinline__ void tail_range(int tiles, int h, int& n0, int& n1) {
+  if (h < 0) {
+    n0 = 0;
+    n1 = tiles;
+  } else {
+    n0 = h * (tiles / 2);
+    n1 = n0 + tiles / 2;
+  }
 }
 
 // LN2 of the CTA's 128 rows of an item, one warp per row (rows w, w + 8, ..),
@@ -194,8 +257,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTailThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const int pair = static_cast<int>(cluster_id_x());
   const int npairs = static_cast<int>(nclusters_x());
-  // this pair's items: pair, pair + npairs, ...
-  const int J = pair < p.items ? (p.items - pair + npairs - 1) / npairs : 0;
+  const TailPlan pl = tail_plan(p, pair, npairs);
+  const int J = pl.J;
   const int n_seg = 3 * J;
   TailShape sh;
   sh.e512 = p.d % 512 == 0;
@@ -251,10 +314,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTailThreads, 1)
     uint32_t phase_bit = 0;
     bool ok = true;
     const int scr_row = pair * 256 + static_cast<int>(rank) * 128;
+    const int scr_row_partner = pl.partner * 256 + static_cast<int>(rank) * 128;
     for (int sg = 0; sg < n_seg && ok; ++sg) {
       int ph, j;
       tail_segment(sg, J, ph, j);
-      const int item = pair + j * npairs;
+      const int item = pl.item(j);
+      const int hf = pl.half_of(j);
       // token row of this CTA's block (an absent second block reads block 0's
       // rows: its results are never stored)
       int blk = 2 * item + static_cast<int>(rank);
@@ -271,7 +336,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTailThreads, 1)
       const int tiles = ph == 0 ? sh.nB : (ph == 1 ? sh.nD : sh.nE);
       const uint32_t stage_bytes =
           wide ? 2u * (kPairABytes / 2 + kPairBBytes) : 2u * kPairStageBytes;
-      for (int n = 0; n < tiles && ok; ++n) {
+      int n0, n1;
+      tail_range(tiles, hf, n0, n1);
+      for (int n = n0; n < n1 && ok; ++n) {
         for (int kb = 0; kb < kbs; ++kb) {
           if (!mbar_wait_warp(empty0 + 8 * stage, phase_bit ^ 1u, abort_flag, p.err,
                               kSiteGemmProducer)) {
@@ -290,19 +357,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTailThreads, 1)
                                kb * kGemmBK, n * 4 + static_cast<int>(rank) * 2);
           }
           __syncwarp();
-          // A of item j's first H chunk / Z tile waits for its LN2 / whole hidden
-          if (kb == 0 && n == 0 && ph > 0) {
+          // A of item j's first H chunk / Z tile waits for its LN2 / whole
+          // hidden (of a shared item: also the partner's half of the hidden)
+          if (kb == 0 && n == n0 && ph > 0) {
             if (!mbar_wait_warp(ph == 1 ? v_ready : h_ready, static_cast<uint32_t>(j & 1),
                                 abort_flag, p.err, kSiteGemmProducer)) {
               ok = false;
               break;
             }
+            if (ph == 2 && hf >= 0) {
+              if (!flag_wait_warp(p.flags + tail_flag(1, pl.partner, rank), kTailEpi,
+                                  abort_flag, p.err, kSiteTailPartner)) {
+                ok = false;
+                break;
+              }
+              fence_proxy_async_global();
+            }
           }
+          // K blocks of a shared item's Z tile in the partner's half of d_ff
+          // read the partner's hidden rows
+          const bool theirs = ph == 2 && hf >= 0 && (kb >= kbs / 2 ? 1 : 0) != hf;
           const bool lost = p.fault == 3 && pair == 0 && rank == 0 && sg == 0 && n == 0 &&
                             kb == 0;
           if (leader && !lost)
-            tma_load_3d_pair(smem_u32(sA + stage * kPairABytes), ma, fb_leader, 0, a_row,
-                             wide ? kb : kb * 2);
+            tma_load_3d_pair(smem_u32(sA + stage * kPairABytes), ma, fb_leader, 0,
+                             theirs ? scr_row_partner : a_row, wide ? kb : kb * 2);
           __syncwarp();
           if (++stage == kPairStages) {
             stage = 0;
@@ -345,7 +424,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTailThreads, 1)
       const bool wide = ph == 2 && sh.e512;
       const int kbs = sh.kblocks(ph);
       const int tiles = ph == 0 ? sh.nB : (ph == 1 ? sh.nD : sh.nE);
-      for (int n = 0; n < tiles && ok; ++n) {
+      int n0, n1;
+      tail_range(tiles, pl.half_of(j), n0, n1);
+      for (int n = n0; n < n1 && ok; ++n) {
         // accumulator slots: one, or two consecutive for a 512-column tile
         const int s0 = acc;
         const uint32_t p0 = acc_phase;
@@ -421,7 +502,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTailThreads, 1)
     for (int sg = 0; sg < n_seg && ok; ++sg) {
       int ph, j;
       tail_segment(sg, J, ph, j);
-      const int item = pair + j * npairs;
+      const int item = pl.item(j);
+      const int hf = pl.half_of(j);
       const int m_valid = 2 * item + 1 < p.blocks ? 256 : 128;
       const RowMap map{2 * item, p.nb, p.N, 128, 0};
       GemmParams gp{};
@@ -446,7 +528,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTailThreads, 1)
       }
       // logical 256-column tiles of the segment
       const int tiles = ph == 0 ? sh.nB : (ph == 1 ? sh.nD : (sh.e512 ? 2 * sh.nE : sh.nE));
-      for (int n = 0; n < tiles && ok; ++n) {
+      int n0, n1;
+      tail_range(tiles, hf, n0, n1);
+      for (int n = n0; n < n1 && ok; ++n) {
         int col;
         if (ph == 2 && sh.e512)
           // Z tile T = n / 2: CTA r loaded columns 512T + 256r .. +255 as B, and
@@ -475,10 +559,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTailThreads, 1)
       }
       if (!ok) break;
       if (ph == 0) {
-        // every y tile of item j is stored: LN2 of the CTA's rows
+        // every y tile of item j is stored: LN2 of the CTA's rows (of a
+        // shared item, once the partner's y columns are stored too)
+        if (hf >= 0) {
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) red_release_gpu_add(p.flags + tail_flag(0, pair, rank), 1u);
+        }
         if (lane == 0) mbar_arrive(ep_sync);
         if (!mbar_wait_fast(ep_sync, static_cast<uint32_t>(j & 1), abort_flag, p.err,
                             kSiteGemmEpilogue)) {
+          ok = false;
+          break;
+        }
+        if (hf >= 0 && !flag_wait_warp(p.flags + tail_flag(0, pl.partner, rank), kTailEpi,
+                                       abort_flag, p.err, kSiteTailPartner)) {
           ok = false;
           break;
         }
@@ -487,10 +582,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTailThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(v_ready);
       } else if (ph == 1) {
-        // every H chunk of item j is stored
+        // every H chunk of item j is stored (of a shared item: also for the
+        // partner, whose Z tiles read this half of the hidden)
         fence_proxy_async_global();
+        if (hf >= 0) __threadfence();
         __syncwarp();
-        if (lane == 0) mbar_arrive(h_ready);
+        if (lane == 0) {
+          mbar_arrive(h_ready);
+          if (hf >= 0) red_release_gpu_add(p.flags + tail_flag(1, pair, rank), 1u);
+        }
       }
     }
   }

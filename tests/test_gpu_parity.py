@@ -82,6 +82,52 @@ def test_fused_schedule_is_bitwise_the_waves_schedule(cfg):
                 tol_for(cfg))
 
 
+# Items left over after the whole rounds of CTA pairs are shared by two pairs
+# when at most half of the pairs would work in the last round (d % 1024 == 0,
+# d_ff % 512 == 0): each pair computes half of the item's columns and reads
+# the other pair's y and FFN hidden through global memory.  168 blocks = 84
+# items on 74 pairs: 10 shared, the last block ragged; 149 blocks: one shared
+# item holding a single block; 6 ragged sequences of 37 blocks: 37 shared
+# items (the most: every pair works in the last round), one of them (blocks
+# 184, 185) across two sequences, d_k = 64.  Bitwise equal to the waves schedule, and held to the oracle on rows of
+# the shared items.
+SHARED_CASES = [
+    small("fz_shared_ragged", 1, 128 * 167 + 78, 1024, 8, 1024, True, seed=56),
+    small("fz_shared_one_block", 1, 128 * 149, 1024, 8, 1536, True, seed=57),
+    small("fz_shared_most", 6, 128 * 37 - 5, 1024, 16, 1536, False, seed=58, bias=0.5),
+]
+
+
+def shared_item_rows(cfg, pairs=74):
+    """(batch, row) pairs in the items past the last whole round of `pairs`
+    CTA pairs: the first, a middle and the last row of each of their blocks."""
+    nb = (cfg.N + 127) // 128
+    blocks = cfg.B * nb
+    items = (blocks + 1) // 2
+    rows = set()
+    for it in range(items // pairs * pairs, items):
+        for blk in (2 * it, 2 * it + 1):
+            if blk >= blocks:
+                continue
+            b, pos = divmod(blk, nb)
+            lo, hi = pos * 128, min(cfg.N, pos * 128 + 128) - 1
+            rows.update((b, r) for r in (lo, (lo + hi) // 2, hi))
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+@pytest.mark.parametrize("cfg", SHARED_CASES, ids=lambda c: c.name)
+def test_shared_items_are_bitwise_the_waves_schedule(cfg):
+    inp = make_inputs(cfg)
+    fused, _, _ = run_cuda(cfg, inp)
+    waves, _, _ = run_cuda(cfg, inp, opts={"schedule": "waves"})
+    assert np.all(np.isfinite(fused))
+    np.testing.assert_array_equal(fused, waves)
+    rows = np.unique(np.concatenate([shared_item_rows(cfg), sample_rows(cfg, 16)]), axis=0)
+    assert len(rows) > 16
+    compare(fused[rows[:, 0], rows[:, 1]], oracle.layer_rows(inp, cfg.h, cfg.causal, rows),
+            tol_for(cfg))
+
+
 def test_tiny_f32_workload():
     cfg = WORKLOADS["tiny_f32"]
     inp = make_inputs(cfg)
