@@ -140,7 +140,9 @@ typedef struct {
  * bpt_layer_workspace_size -- device workspace bytes bpt_layer_forward needs.
  *
  * Pure host arithmetic.  Layout (each region 1024-byte aligned):
- *   [0, 256)       header; uint32 at offset 0 = device error word
+ *   [0, 2048)      header: uint32 at offset 0 = device error word; bytes
+ *                  [256, 1440) = counters the fused schedule's layer body
+ *                  uses to hand work between CTA pairs
  *   weights        BPT_BF16 only: fp16 copies of W_Q, W_K, W_V, W_O ([d, d]
  *                  each), W_1 [d, d_ff], W_2 [d_ff, d], in that order
  *   QKV            [B*N, 3d] (Q | K | V per row); fp16 for BPT_BF16, fp32

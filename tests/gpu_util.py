@@ -53,10 +53,11 @@ def compare(got: np.ndarray, want: np.ndarray, tol):
 def workspace_qkv(ws: torch.Tensor, cfg: LayerShape, B: int) -> np.ndarray:
     """The QKV projection the library leaves in its workspace ([B*N, 3d]).
 
-    Layout (include/bpt.h): 1024-byte header region, then for bf16 layers the
-    fp16 weight copies, then QKV in the operand type (fp16 / fp32).
+    Layout (include/bpt.h): a 2048-byte header region (error word, hand-over
+    counters), then for bf16 layers the fp16 weight copies, then QKV in the
+    operand type (fp16 / fp32).
     """
-    off = 1024
+    off = 2048
     n = B * cfg.N * 3 * cfg.d
     if cfg.dtype == "bf16":
         w16 = (4 * cfg.d * cfg.d + 2 * cfg.d * cfg.d_ff) * 2
