@@ -128,6 +128,26 @@ def test_shared_items_are_bitwise_the_waves_schedule(cfg):
             tol_for(cfg))
 
 
+@pytest.mark.parametrize("cfg,shared", [(SHARED_CASES[0], 10), (SHARED_CASES[2], 37),
+                                        (FUSED_CASES[3], 0)],
+                         ids=["10_shared", "37_shared", "none_shared"])
+def test_shared_items_hand_over_through_the_header(cfg, shared):
+    """The hand-over counters (workspace header bytes [256, 1440), include/bpt.h:
+    [kind][pair][CTA rank] uint32, kinds y and H) after a forward: each CTA of
+    the 2 * shared pairs that share an item counted its eight epilogue warps
+    for both hand-overs, every other entry stayed zero.  So the shared order
+    really ran (a refused cooperative launch would leave all zeros)."""
+    dev = bpt.to_device(make_inputs(cfg), cfg.dtype)
+    _, ws = bpt.layer_forward(dev["x"], dev, cfg.h, cfg.causal)
+    st, site = bpt.bpt_read_device_error(ws.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    assert st == bpt.BPT_OK, f"device error {bpt.status_string(st)} at site {site}"
+    pairs = bpt.BPT_TAIL_MAX_PAIRS
+    flags = ws[256:256 + 2 * pairs * 2 * 4].view(torch.int32).cpu().numpy().reshape(2, pairs, 2)
+    want = np.zeros_like(flags)
+    want[:, :2 * shared, :] = 8
+    np.testing.assert_array_equal(flags, want)
+
+
 def test_tiny_f32_workload():
     cfg = WORKLOADS["tiny_f32"]
     inp = make_inputs(cfg)
