@@ -92,6 +92,11 @@ bpt_status read_opts(const bpt_options* o, Opts* r) {
 #ifndef BPT_ATTN_KV_BUDGET_MB
 #define BPT_ATTN_KV_BUDGET_MB 64
 #endif
+// 1: the fused layer body shares the items left over after its last whole
+// round between two CTA pairs (tail_tc.cuh); 0: one pair per item.
+#ifndef BPT_TAIL_SHARE_ITEMS
+#define BPT_TAIL_SHARE_ITEMS 1
+#endif
 constexpr int kEmu128 = BPT_EMU_DK128;
 constexpr int kEmu64 = BPT_EMU_DK64;
 // Workspace header: the device error word at offset 0; from kTailFlagOffset
@@ -768,7 +773,8 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
     // round and every half is a whole number of tiles (y tiles and H chunks
     // of 256 columns, Z tiles of 512).
     const int64_t left = tp.items % pairs;
-    tp.split = (left > 0 && 2 * left <= pairs && d % 1024 == 0 && d_ff % 512 == 0) ? 1 : 0;
+    tp.split = (BPT_TAIL_SHARE_ITEMS && left > 0 && 2 * left <= pairs && d % 1024 == 0 &&
+                d_ff % 512 == 0) ? 1 : 0;
     tp.flags = reinterpret_cast<uint32_t*>(ws + kTailFlagOffset);
     LaunchScope ls(BPT_KIND_TAIL, s);
     if (tp.split) {

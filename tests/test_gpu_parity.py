@@ -10,6 +10,7 @@ import numpy as np
 import pytest
 import torch
 
+import blockwise_attn_ffn_b200 as bpt
 import oracle
 from blockwise_attn_ffn_b200.inputs import LayerShape, WORKLOADS, make_inputs, sample_rows
 
