@@ -776,6 +776,13 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
     tp.split = (BPT_TAIL_SHARE_ITEMS && left > 0 && 2 * left <= pairs && d % 1024 == 0 &&
                 d_ff % 512 == 0) ? 1 : 0;
     tp.flags = reinterpret_cast<uint32_t*>(ws + kTailFlagOffset);
+    if (tp.split) {
+      // Under stream capture (a CUDA graph being recorded) the body runs
+      // unshared with a plain launch, which graphs always accept.
+      cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+      if (cudaStreamIsCapturing(s, &cap) != cudaSuccess) return BPT_ERR_CUDA;
+      if (cap != cudaStreamCaptureStatusNone) tp.split = 0;
+    }
     LaunchScope ls(BPT_KIND_TAIL, s);
     if (tp.split) {
       // A pair waits for its partner's hand-overs, so all pairs must be

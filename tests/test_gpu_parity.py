@@ -149,6 +149,34 @@ def test_shared_items_hand_over_through_the_header(cfg, shared):
     np.testing.assert_array_equal(flags, want)
 
 
+def test_fused_forward_replays_from_a_cuda_graph():
+    """A whole forward recorded by stream capture into a CUDA graph (its
+    memsets and every launch) replays bitwise equal to the eager call, twice.
+    The shape shares left-over items when run eagerly; under capture the layer
+    body runs unshared (a plain launch), which gives the same bits."""
+    cfg = SHARED_CASES[0]
+    dev = bpt.to_device(make_inputs(cfg), cfg.dtype)
+    want, ws = bpt.layer_forward(dev["x"], dev, cfg.h, cfg.causal)
+    want = want.clone()
+    out = torch.empty_like(want)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):  # first call on this stream outside the capture
+        bpt.layer_forward(dev["x"], dev, cfg.h, cfg.causal, out=out, workspace=ws)
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        bpt.layer_forward(dev["x"], dev, cfg.h, cfg.causal, out=out, workspace=ws)
+    for _ in range(2):
+        out.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        st, site = bpt.bpt_read_device_error(ws.data_ptr(), torch.cuda.current_stream().cuda_stream)
+        assert st == bpt.BPT_OK, f"device error {bpt.status_string(st)} at site {site}"
+        assert torch.equal(out, want)
+    del graph
+
+
 def test_tiny_f32_workload():
     cfg = WORKLOADS["tiny_f32"]
     inp = make_inputs(cfg)
