@@ -15,7 +15,8 @@ from ._lib import (  # noqa: F401
     bpt_layer_forward_static, bpt_layer_forward_train, bpt_layer_forward_train_keep_o,
     bpt_layer_launch_count,
     bpt_layer_launch_count_opt, bpt_layer_shard_forward, bpt_layer_shard_project,
-    bpt_layer_shard_workspace_size, bpt_layer_workspace_size, bpt_layer_workspace_size_opt,
+    bpt_layer_shard_workspace_size, bpt_layer_tail_plan, bpt_layer_workspace_size,
+    bpt_layer_workspace_size_opt,
     bpt_profile_enable, bpt_profile_read, bpt_read_device_error, bpt_status_string, load,
     make_options, status_string,
 )

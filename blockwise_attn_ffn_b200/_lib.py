@@ -35,6 +35,7 @@ EXPORTED = [
     "bpt_layer_launch_count_opt",
     "bpt_layer_shard_workspace_size", "bpt_layer_shard_project", "bpt_layer_shard_forward",
     "bpt_layer_forward_train_keep_o", "bpt_layer_backward_keep_o",
+    "bpt_layer_tail_plan",
 ]
 
 
@@ -144,6 +145,9 @@ def load() -> ctypes.CDLL:
     lib.bpt_layer_launch_count.argtypes = [i64, i64, i64, i64, i64, i32, i32,
                                            ctypes.POINTER(ctypes.c_int64)]
     lib.bpt_layer_launch_count.restype = i32
+    p32 = ctypes.POINTER(ctypes.c_int32)
+    lib.bpt_layer_tail_plan.argtypes = [i64, i64, i64, i64, i64, i32, i32, p32, p32, p32, i32]
+    lib.bpt_layer_tail_plan.restype = i32
     lib.bpt_layer_forward_static.argtypes = [vp] * 11 + [i64] * 5 + [i32, i32, vp, vp]
     lib.bpt_layer_forward_static.restype = i32
     _lib = lib
@@ -345,3 +349,20 @@ def bpt_layer_launch_count(B, N, d, h, d_ff, causal, dtype) -> Tuple[int, int]:
     st = load().bpt_layer_launch_count(B, N, d, h, d_ff, int(bool(causal)), dtype,
                                        ctypes.byref(out))
     return st, out.value
+
+
+def bpt_layer_tail_plan(B, N, d, h, d_ff, causal, resident_pairs, rows=None):
+    """Returns (status, pairs, shared, plan): plan is a list of
+    (whole items, whole items before the shared one, shared item or -1,
+    half or -1, partner or -1) per CTA pair, for the first `rows` pairs
+    (default: BPT_TAIL_MAX_PAIRS)."""
+    rows = BPT_TAIL_MAX_PAIRS if rows is None else rows
+    pairs = ctypes.c_int32(0)
+    shared = ctypes.c_int32(0)
+    buf = (ctypes.c_int32 * (5 * max(rows, 1)))()
+    st = load().bpt_layer_tail_plan(B, N, d, h, d_ff, int(bool(causal)), resident_pairs,
+                                    ctypes.byref(pairs), ctypes.byref(shared),
+                                    buf if rows > 0 else None, rows)
+    n = min(pairs.value, rows) if st == BPT_OK else 0
+    plan = [tuple(buf[5 * q:5 * q + 5]) for q in range(n)]
+    return st, pairs.value, shared.value, plan

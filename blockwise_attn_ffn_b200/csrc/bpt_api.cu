@@ -772,9 +772,8 @@ bpt_status forward_bf16(const Plan& P, const void* x, const void* ln1, const voi
     // each when at most half of the pairs would otherwise work in the last
     // round and every half is a whole number of tiles (y tiles and H chunks
     // of 256 columns, Z tiles of 512).
-    const int64_t left = tp.items % pairs;
-    tp.split = (BPT_TAIL_SHARE_ITEMS && left > 0 && 2 * left <= pairs && d % 1024 == 0 &&
-                d_ff % 512 == 0) ? 1 : 0;
+    tp.split = (BPT_TAIL_SHARE_ITEMS && bpt::tail_shares(tp.items, int(pairs), int(d), int(d_ff)))
+                   ? 1 : 0;
     tp.flags = reinterpret_cast<uint32_t*>(ws + kTailFlagOffset);
     if (tp.split) {
       // Under stream capture (a CUDA graph being recorded) the body runs
@@ -1703,6 +1702,38 @@ bpt_status bpt_layer_launch_count_opt(int64_t B, int64_t N, int64_t d, int64_t h
 bpt_status bpt_layer_launch_count(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff,
                                   int causal, bpt_dtype dtype, int64_t* launches) {
   return bpt_layer_launch_count_opt(B, N, d, h, d_ff, causal, dtype, nullptr, launches);
+}
+
+bpt_status bpt_layer_tail_plan(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff,
+                               int causal, int32_t resident_pairs, int32_t* pairs,
+                               int32_t* shared, int32_t* plan, int32_t plan_rows) {
+  if (!pairs || !shared || resident_pairs < 1 || resident_pairs > BPT_TAIL_MAX_PAIRS ||
+      plan_rows < 0 || (plan == nullptr && plan_rows > 0))
+    return BPT_ERR_INVALID_ARG;
+  Plan P;
+  const bpt_status st = plan_for(B, N, d, h, d_ff, causal, BPT_BF16, nullptr, true, &P);
+  if (st != BPT_OK) return st;
+  *pairs = 0;
+  *shared = 0;
+  if (P.items == 0) return BPT_OK;
+  // as the fused forward launches the layer body
+  bpt::TailParams tp{};
+  tp.blocks = int(P.items);
+  tp.items = int((P.items + 1) / 2);
+  const int np = int(std::max<int64_t>(1, std::min<int64_t>(P.tail_pairs, resident_pairs)));
+  tp.split = (BPT_TAIL_SHARE_ITEMS && bpt::tail_shares(tp.items, np, int(d), int(d_ff))) ? 1 : 0;
+  *pairs = np;
+  *shared = tp.split ? tp.items % np : 0;
+  for (int q = 0; q < std::min(np, int(plan_rows)); ++q) {
+    const bpt::TailPlan pl = bpt::tail_plan(tp, q, np);
+    int32_t* r = plan + 5 * q;
+    r[0] = pl.J;
+    r[1] = pl.Jfull;
+    r[2] = pl.half >= 0 ? pl.hitem : -1;
+    r[3] = pl.half;
+    r[4] = pl.half >= 0 ? pl.partner : -1;
+  }
+  return BPT_OK;
 }
 
 bpt_status bpt_layer_forward(const void* x, const void* ln1, const void* W_Q, const void* W_K,

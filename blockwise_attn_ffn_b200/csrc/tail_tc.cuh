@@ -98,11 +98,22 @@ __device__ __forceinline__ int tail_flag(int kind, int pair, uint32_t rank) {
 struct TailPlan {
   int J, Jfull, hitem, half, partner;
   int first, stride;
-  __device__ __forceinline__ int item(int j) const { return j < Jfull ? first + j * stride : hitem; }
-  __device__ __forceinline__ int half_of(int j) const { return j < Jfull ? -1 : half; }
+  __host__ __device__ __forceinline__ int item(int j) const {
+    return j < Jfull ? first + j * stride : hitem;
+  }
+  __host__ __device__ __forceinline__ int half_of(int j) const { return j < Jfull ? -1 : half; }
 };
 
-__device__ __forceinline__ TailPlan tail_plan(const TailParams& p, int pair, int npairs) {
+// Whether the launch shares the left-over items: L = items mod pairs with
+// 0 < L <= pairs / 2, and every half a whole number of tiles (y tiles and H
+// chunks of 256 columns, Z tiles of 512).
+__host__ __device__ __forceinline__ bool tail_shares(int items, int pairs, int d, int d_ff) {
+  const int left = items % pairs;
+  return left > 0 && 2 * left <= pairs && d % 1024 == 0 && d_ff % 512 == 0;
+}
+
+// Also compiled for the host, where bpt_layer_tail_plan reports it.
+__host__ __device__ __forceinline__ TailPlan tail_plan(const TailParams& p, int pair, int npairs) {
   TailPlan pl{};
   pl.first = pair;
   pl.stride = npairs;

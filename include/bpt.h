@@ -512,6 +512,33 @@ bpt_status bpt_profile_read(double* ms, int64_t* launches, int n);
  * with those options). */
 bpt_status bpt_layer_launch_count(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff,
                                   int causal, bpt_dtype dtype, int64_t* launches);
+
+/*
+ * bpt_layer_tail_plan -- the work list of the fused schedule's layer body
+ * (y = x + o W_O, LN2, the FFN, per two-block item; "Blockwise Parallel
+ * Transformer — BPT", section "The fused blockwise algorithm") for a bf16
+ * layer of these sizes, when `resident_pairs` CTA pairs (1 ..
+ * BPT_TAIL_MAX_PAIRS; 74 on a B200) can run at once.  Pure host arithmetic,
+ * computed by the code the kernel runs.
+ *
+ * Items are two consecutive query blocks (items = ceil(B*nb / 2), nb =
+ * ceil(N / 128)), on P = min(resident_pairs, items) pairs (*pairs = P): pair
+ * q takes whole items q, q + P, ...  When R whole rounds leave L = items - R*P
+ * items with 0 < L <= P / 2, d % 1024 == 0 and d_ff % 512 == 0, those are
+ * shared: pair q and pair q + L (q < L) each compute half of item R*P + q by
+ * columns (*shared = L; otherwise 0).  A launch that cannot be cooperative,
+ * or that is recorded by stream capture, runs unshared.
+ * plan: for pairs q < min(P, plan_rows), five int32 per pair: whole items,
+ * whole items before the shared one (equal), the shared item or -1, this
+ * pair's half of it (0 / 1) or -1, the partner pair or -1.  NULL with
+ * plan_rows = 0 asks for *pairs and *shared only.
+ * Returns BPT_ERR_INVALID_ARG for NULL pairs / shared, resident_pairs out of
+ * range, plan_rows < 0 or plan == NULL with plan_rows > 0, and the statuses of
+ * bpt_layer_workspace_size for the sizes (as a bf16 layer).
+ */
+bpt_status bpt_layer_tail_plan(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff,
+                               int causal, int32_t resident_pairs, int32_t* pairs,
+                               int32_t* shared, int32_t* plan, int32_t plan_rows);
 bpt_status bpt_layer_launch_count_opt(int64_t B, int64_t N, int64_t d, int64_t h, int64_t d_ff,
                                       int causal, bpt_dtype dtype, const bpt_options* opts,
                                       int64_t* launches);
